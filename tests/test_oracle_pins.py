@@ -1,0 +1,327 @@
+"""Pins of the fp64 oracle to facts other than itself (CPU only).
+
+The pages print no worked numbers for the mixer, so each part of the oracle is
+tied to a closed form, a brute-force restatement, an invariant or a textbook
+identity, each chosen so that a plausible mistake (a dropped term, a wrong
+sign, an off-by-one in time, B and C swapped, the conv taps reversed, eps
+outside the root) fails at least one test.  The tests call only ``oracle``
+and the seeded input generator.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from mamba_selective_scan_jamba_b200 import synth
+
+RNG = np.random.default_rng(20240328)
+
+
+def rand_scan_inputs(L, d, N, with_h0=True, seed=0):
+    r = np.random.default_rng(seed)
+    delta = np.exp(r.uniform(np.log(1e-3), np.log(0.5), size=(L, d)))
+    A = -np.exp(r.uniform(np.log(0.25), np.log(8.0), size=(d, N)))
+    Bm = r.normal(size=(L, N))
+    Cm = r.normal(size=(L, N))
+    u = r.normal(size=(L, d))
+    D = r.normal(size=d)
+    h0 = r.normal(size=(d, N)) if with_h0 else None
+    return delta, A, Bm, Cm, u, D, h0
+
+
+# ------------------------------------------------------------------ scan core
+def test_scan_L1_closed_form():
+    """L = 1 from h0 = 0: h = delta*B*u and y = C.(delta*B*u) + D*u."""
+    delta, A, Bm, Cm, u, D, _ = rand_scan_inputs(1, 5, 16, seed=1)
+    y, hT = oracle.scan(delta, A, Bm, Cm, u, D, None)
+    h = delta[0][:, None] * Bm[0][None, :] * u[0][:, None]
+    np.testing.assert_allclose(hT, h, rtol=1e-14, atol=0)
+    np.testing.assert_allclose(y[0], h @ Cm[0] + D * u[0], rtol=1e-14, atol=1e-15)
+
+
+def test_scan_geometric_series():
+    """Constant delta, A, B, C, u: h_t = a^t h0 + b (1 - a^t) / (1 - a), a = exp(delta A),
+    b = delta B u, with t counting updates (h_1 is the state after the first token)."""
+    L, d, N = 37, 3, 16
+    r = np.random.default_rng(2)
+    dl = np.array([0.01, 0.3, 2.0])
+    A = -np.exp(r.uniform(-1, 2, size=(d, N)))
+    B1, C1 = r.normal(size=N), r.normal(size=N)
+    u1 = np.array([0.7, -1.3, 0.2])
+    D = r.normal(size=d)
+    h0 = r.normal(size=(d, N))
+    delta = np.tile(dl, (L, 1))
+    y, hT = oracle.scan(delta, A, np.tile(B1, (L, 1)), np.tile(C1, (L, 1)), np.tile(u1, (L, 1)),
+                        D, h0)
+    a = np.exp(dl[:, None] * A)
+    b = dl[:, None] * B1[None, :] * u1[:, None]
+    for t in (1, 2, 10, L):
+        ht = a ** t * h0 + b * (1 - a ** t) / (1 - a)
+        np.testing.assert_allclose(y[t - 1], ht @ C1 + D * u1, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(hT, a ** L * h0 + b * (1 - a ** L) / (1 - a), rtol=1e-12, atol=1e-14)
+
+
+def hidden_attention(delta, A, Bm, Cm, u, D, h0):
+    """Materialised form (Ali, Zimerman & Wolf, "The hidden attention of Mamba
+    models", cited by the Jamba paper): y_t = sum_{s<=t} sum_n C_t,n
+    (prod_{r=s+1..t} e^{delta_r A_n}) delta_s B_s,n u_s + C_t.(prod_{r<=t} e^{delta_r A}) h0
+    + D u_t, one term at a time."""
+    L, d = delta.shape
+    N = A.shape[1]
+    y = np.zeros((L, d))
+    for c in range(d):
+        for t in range(L):
+            acc = 0.0
+            for n in range(N):
+                for s in range(t + 1):
+                    decay = 1.0
+                    for rr in range(s + 1, t + 1):
+                        decay *= math.exp(delta[rr, c] * A[c, n])
+                    acc += Cm[t, n] * decay * delta[s, c] * Bm[s, n] * u[s, c]
+                if h0 is not None:
+                    decay = 1.0
+                    for rr in range(0, t + 1):
+                        decay *= math.exp(delta[rr, c] * A[c, n])
+                    acc += Cm[t, n] * decay * h0[c, n]
+            y[t, c] = acc + D[c] * u[t, c]
+    return y
+
+
+@pytest.mark.parametrize("L,d,N,with_h0", [(1, 2, 3, False), (7, 3, 4, True), (13, 2, 16, True)])
+def test_scan_hidden_attention_bruteforce(L, d, N, with_h0):
+    delta, A, Bm, Cm, u, D, h0 = rand_scan_inputs(L, d, N, with_h0, seed=L * 31 + d)
+    y, _ = oracle.scan(delta, A, Bm, Cm, u, D, h0)
+    np.testing.assert_allclose(y, hidden_attention(delta, A, Bm, Cm, u, D, h0), rtol=1e-12,
+                               atol=1e-13)
+
+
+def test_scan_matches_guide_toy_loop():
+    """The aifetchly guide's toy SSM (``SimpleMambaSSM.forward``) discretises with
+    exp(delta A) and delta B, zero initial state, no D: vectorised over channels
+    here, one time step per iteration."""
+    L, d, N = 9, 4, 16
+    delta, A, Bm, Cm, u, _, _ = rand_scan_inputs(L, d, N, seed=5)
+    dA = np.exp(delta[:, :, None] * A[None, :, :])           # [L, d, N]
+    dB = delta[:, :, None] * Bm[:, None, :]                   # [L, d, N]
+    h = np.zeros((d, N))
+    ys = []
+    for t in range(L):
+        h = dA[t] * h + dB[t] * u[t][:, None]
+        ys.append((h * Cm[t][None, :]).sum(-1))
+    y, _ = oracle.scan(delta, A, Bm, Cm, u, np.zeros(d), None)
+    np.testing.assert_allclose(y, np.stack(ys), rtol=1e-13, atol=1e-14)
+
+
+def test_scan_limits_and_linearity():
+    L, d, N = 11, 3, 16
+    delta, A, Bm, Cm, u, D, h0 = rand_scan_inputs(L, d, N, seed=6)
+    # delta -> 0: the state never moves; y = C_t.h0 + D u_t
+    y, hT = oracle.scan(np.zeros_like(delta), A, Bm, Cm, u, D, h0)
+    np.testing.assert_allclose(hT, h0, rtol=0, atol=0)
+    np.testing.assert_allclose(y, Cm @ h0.T + D * u, rtol=1e-13, atol=1e-14)
+    # very fast decay: the state forgets everything but the current token
+    big = np.full_like(delta, 1.0)
+    Abig = np.full_like(A, -1e4)
+    y, hT = oracle.scan(big, Abig, Bm, Cm, u, D, h0)
+    np.testing.assert_allclose(hT, (Bm[-1][None, :] * u[-1][:, None]), rtol=1e-12)
+    # linearity in (u, h0) for fixed delta, A, B, C, D
+    u2 = np.random.default_rng(7).normal(size=u.shape)
+    h02 = np.random.default_rng(8).normal(size=h0.shape)
+    ya, ha = oracle.scan(delta, A, Bm, Cm, u, D, h0)
+    yb, hb = oracle.scan(delta, A, Bm, Cm, u2, D, h02)
+    yc, hc = oracle.scan(delta, A, Bm, Cm, 2 * u - 3 * u2, D, 2 * h0 - 3 * h02)
+    np.testing.assert_allclose(yc, 2 * ya - 3 * yb, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(hc, 2 * ha - 3 * hb, rtol=1e-11, atol=1e-12)
+
+
+# --------------------------------------------------------- front-end pieces
+def test_conv_impulse_response_and_history():
+    """A unit impulse at t = 0 returns the taps reversed in time: the last tap
+    multiplies the current token.  With x = 0, only the cached history acts."""
+    L, d, K = 6, 3, 4
+    r = np.random.default_rng(9)
+    w = r.normal(size=(d, K))
+    b = r.normal(size=d)
+    x = np.zeros((L, d))
+    x[0, :] = 1.0
+    xc = oracle.conv(x, w, b)
+    for t in range(L):
+        want = b + (w[:, K - 1 - t] if t < K else 0.0)
+        np.testing.assert_array_equal(xc[t], want)
+    hist = r.normal(size=(d, K - 1))   # oldest first
+    xc = oracle.conv(np.zeros((L, d)), w, np.zeros(d), hist)
+    np.testing.assert_allclose(xc[0], (w[:, :K - 1] * hist).sum(1), rtol=1e-15)
+    np.testing.assert_allclose(xc[1], (w[:, :K - 2] * hist[:, 1:]).sum(1), rtol=1e-15)
+    np.testing.assert_allclose(xc[2], w[:, 0] * hist[:, 2], rtol=1e-15)
+    np.testing.assert_array_equal(xc[3:], 0.0)
+
+
+def test_silu_identities():
+    v = np.linspace(-30, 30, 1201)
+    s = oracle.silu(v)
+    np.testing.assert_allclose(s - oracle.silu(-v), v, rtol=1e-14, atol=1e-14)  # x(s(x)+s(-x)) = x
+    assert oracle.silu(np.array([0.0]))[0] == 0.0
+    np.testing.assert_allclose(oracle.silu(np.array([40.0])), [40.0], rtol=1e-15)
+
+
+def test_rmsnorm_identities():
+    r = np.random.default_rng(10)
+    v = r.normal(size=(5, 256)) * 3.0
+    out = oracle.rmsnorm(v, np.ones(256), 0.0)
+    np.testing.assert_allclose(np.sqrt((out ** 2).mean(-1)), 1.0, rtol=1e-14)
+    np.testing.assert_allclose(oracle.rmsnorm(7.5 * v, np.ones(256), 0.0), out, rtol=1e-14)
+    # eps sits inside the root: a constant vector a*1 maps to a / sqrt(a^2 + eps)
+    a, eps = 0.01, 1e-6
+    np.testing.assert_allclose(oracle.rmsnorm(np.full((1, 16), a), np.ones(16), eps),
+                               np.full((1, 16), a / math.sqrt(a * a + eps)), rtol=1e-15)
+    w = r.normal(size=16)
+    np.testing.assert_allclose(oracle.rmsnorm(v[:, :16], w, 0.0),
+                               oracle.rmsnorm(v[:, :16], np.ones(16), 0.0) * w, rtol=1e-15)
+
+
+def test_softplus_identities():
+    dt = np.exp(np.linspace(np.log(1e-6), np.log(50.0), 500))
+    inv = np.log(np.expm1(dt))   # softplus^-1
+    np.testing.assert_allclose(oracle.softplus(inv), dt, rtol=1e-13)
+    assert abs(oracle.softplus1(0.0) - math.log(2.0)) < 1e-16
+    assert abs(oracle.softplus1(-40.0) - math.exp(-40.0)) < 1e-30
+    assert oracle.softplus1(800.0) == 800.0
+
+
+def test_round_bf16():
+    assert oracle.round_bf16(1.0) == 1.0
+    assert oracle.round_bf16(1.0 + 2 ** -8) == 1.0            # tie -> even
+    assert oracle.round_bf16(1.0 + 3 * 2 ** -8) == 1.0 + 2 ** -6  # tie -> even (up)
+    assert oracle.round_bf16(1.0 + 2 ** -8 + 2 ** -20) == 1.0 + 2 ** -7
+
+
+# ------------------------------------------------------------- whole mixer
+def tiny(extra=True, io="f32", L=24, d=40, R=8, B=2, seed=11):
+    return synth.Workload("pin", B, L, d, R, io, seed=seed, extra=extra)
+
+
+def test_mixer_split_invariant():
+    """Running [0, L1) and then [L1, L) from the carried conv and SSM states
+    reproduces the full run, including cuts inside the conv window."""
+    w = tiny()
+    W = synth.make_weights(w)
+    A = synth.make_activations(w)
+    m = oracle.dims_of(w)
+    y, fs, fc = oracle.mixer_fwd(m, A["x"], A["z"], W, A["init_conv_state"], A["init_ssm_state"])
+    for L1 in (1, 2, 3, 17):
+        m1 = oracle.dims_of(w, seqlen=L1)
+        m2 = oracle.dims_of(w, seqlen=w.seqlen - L1)
+        y1, s1, c1 = oracle.mixer_fwd(m1, A["x"][:, :L1], A["z"][:, :L1], W, A["init_conv_state"],
+                                      A["init_ssm_state"])
+        y2, s2, c2 = oracle.mixer_fwd(m2, A["x"][:, L1:], A["z"][:, L1:], W, c1, s1)
+        np.testing.assert_allclose(np.concatenate([y1, y2], 1), y, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(s2, fs, rtol=1e-12, atol=1e-13)
+        np.testing.assert_array_equal(c2, fc)
+
+
+def test_mixer_step_equals_forward():
+    w = tiny(L=9)
+    W = synth.make_weights(w)
+    A = synth.make_activations(w)
+    m = oracle.dims_of(w)
+    y, fs, fc = oracle.mixer_fwd(m, A["x"], A["z"], W, A["init_conv_state"], A["init_ssm_state"])
+    cs, ss = A["init_conv_state"], A["init_ssm_state"]
+    ms = oracle.dims_of(w, seqlen=1)
+    for t in range(w.seqlen):
+        yt, cs, ss = oracle.mixer_step(ms, A["x"][:, t], A["z"][:, t], cs, ss, W)
+        np.testing.assert_allclose(yt, y[:, t], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(ss, fs, rtol=1e-12, atol=1e-13)
+    np.testing.assert_array_equal(cs, fc)
+
+
+def test_mixer_channel_permutation_and_batch_independence():
+    w = tiny(B=3)
+    W = synth.make_weights(w)
+    A = synth.make_activations(w)
+    m = oracle.dims_of(w)
+    y, fs, fc = oracle.mixer_fwd(m, A["x"], A["z"], W, A["init_conv_state"], A["init_ssm_state"])
+    perm = np.random.default_rng(12).permutation(w.d_inner)
+    Wp = dict(W)
+    for k in ("conv_w", "conv_b", "dtproj_w", "dt_bias", "A_log", "D"):
+        Wp[k] = W[k][perm]
+    Wp["xproj_w"] = W["xproj_w"][:, perm]
+    yp, fsp, fcp = oracle.mixer_fwd(m, A["x"][:, :, perm], A["z"][:, :, perm], Wp,
+                                    A["init_conv_state"][:, perm], A["init_ssm_state"][:, perm])
+    np.testing.assert_allclose(yp, y[:, :, perm], rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(fsp, fs[:, perm], rtol=1e-13, atol=1e-14)
+    m1 = oracle.dims_of(w, batch=1)
+    for b in range(w.batch):
+        yb, fsb, _ = oracle.mixer_fwd(m1, A["x"][b:b + 1], A["z"][b:b + 1], W,
+                                      A["init_conv_state"][b:b + 1], A["init_ssm_state"][b:b + 1])
+        np.testing.assert_array_equal(yb[0], y[b])
+        np.testing.assert_array_equal(fsb[0], fs[b])
+
+
+def test_mixer_gate_skip_and_split_order():
+    """x_proj rows are [dt | B | C].  With the C rows zeroed the output is the
+    skip path alone, y = D u SiLU(z); with the B rows zeroed and h0 = 0 the
+    state never leaves zero; with the dt rows zeroed, delta = softplus(dt_bias)."""
+    w = tiny(extra=True, B=1)
+    W = synth.make_weights(w)
+    A = synth.make_activations(w)
+    R, N = w.dt_rank, w.d_state
+    m = oracle.dims_of(w)
+    x = A["x"][0].astype(np.float64)
+    u = oracle.silu(oracle.conv(x, W["conv_w"], W["conv_b"], A["init_conv_state"][0]))
+    gate = oracle.silu(A["z"][0])
+    # C rows zero
+    Wc = dict(W)
+    Wc["xproj_w"] = W["xproj_w"].copy()
+    Wc["xproj_w"][R + N:] = 0
+    y, fs, _ = oracle.mixer_fwd(m, A["x"], A["z"], Wc, A["init_conv_state"], None)
+    np.testing.assert_allclose(y[0], W["D"] * u * gate, rtol=1e-13, atol=1e-14)
+    assert np.abs(fs).max() > 0
+    # B rows zero, h0 = 0: state stays 0, y = D u SiLU(z)
+    Wb = dict(W)
+    Wb["xproj_w"] = W["xproj_w"].copy()
+    Wb["xproj_w"][R:R + N] = 0
+    y, fs, _ = oracle.mixer_fwd(m, A["x"], A["z"], Wb, A["init_conv_state"], None)
+    np.testing.assert_array_equal(fs, 0.0)
+    np.testing.assert_allclose(y[0], W["D"] * u * gate, rtol=1e-13, atol=1e-14)
+    # dt rows zero: delta = softplus(dt_bias) for every token
+    Wd = dict(W)
+    Wd["xproj_w"] = W["xproj_w"].copy()
+    Wd["xproj_w"][:R] = 0
+    y, fs, _ = oracle.mixer_fwd(m, A["x"], A["z"], Wd, A["init_conv_state"], A["init_ssm_state"])
+    p = u @ W["xproj_w"].astype(np.float64).T
+    Bn = oracle.rmsnorm(p[:, R:R + N], W["b_norm_w"], w.eps)
+    Cn = oracle.rmsnorm(p[:, R + N:], W["c_norm_w"], w.eps)
+    delta = np.tile(np.log1p(np.exp(W["dt_bias"].astype(np.float64))), (w.seqlen, 1))
+    ys, hT = oracle.scan(delta, -np.exp(W["A_log"].astype(np.float64)), Bn, Cn, u, W["D"],
+                         A["init_ssm_state"][0])
+    np.testing.assert_allclose(y[0], ys * gate, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(fs[0], hT, rtol=1e-11, atol=1e-13)
+
+
+def test_mirror_rounding_is_small():
+    """Mirror mode rounds u and dt_n to bf16; on bf16 inputs it must stay within a
+    few bf16 ulps of the exact run, and equal it when the rounding is a no-op."""
+    w = tiny(io="bf16")
+    W = synth.make_weights(w)
+    A = synth.make_activations(w)
+    y, fs, _ = oracle.mixer_fwd(oracle.dims_of(w), A["x"], A["z"], W, A["init_conv_state"],
+                                A["init_ssm_state"])
+    ym, fsm, _ = oracle.mixer_fwd(oracle.dims_of(w, mirror=True), A["x"], A["z"], W,
+                                  A["init_conv_state"], A["init_ssm_state"])
+    assert np.abs(ym - y).max() < 2e-2 * max(1.0, np.abs(y).max())
+    assert 0 < np.abs(fsm - fs).max() < 1e-2
+
+
+def test_sampled_channels_match_full():
+    w = tiny()
+    W = synth.make_weights(w)
+    A = synth.make_activations(w)
+    m = oracle.dims_of(w)
+    y, fs, fc = oracle.mixer_fwd(m, A["x"], A["z"], W, A["init_conv_state"], A["init_ssm_state"])
+    ch = [0, 7, 39]
+    ys, fss, fcs = oracle.mixer_fwd(m, A["x"], A["z"], W, A["init_conv_state"],
+                                    A["init_ssm_state"], channels=ch)
+    np.testing.assert_array_equal(ys, y[:, :, ch])
+    np.testing.assert_array_equal(fss, fs[:, ch])
+    np.testing.assert_array_equal(fcs, fc[:, ch])
