@@ -1,0 +1,381 @@
+"""Benchmark of the Jamba Mamba-1 mixer core (libjmix) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl jmix|reference]
+                    [--workload jamba_b8_l4096] [--no-cpu-baseline] [--no-e2e]
+
+One step = one jm_mixer_fwd over the workload's whole batch (conv + SiLU,
+x_proj, RMSNorms, dt_proj + softplus, selective scan, D skip, SiLU(z) gate,
+final states), inputs already in HBM.  Under torchrun each rank runs its own
+batch (independent sequences, no collective on the data path: weak scaling);
+time is the max over ranks of the CUDA-event time on the launching stream.
+Rank 0 prints one JSON line.
+
+--impl reference times the fp64 CPU oracle (the only reference that exists for
+this path) on the host cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "Mamba-mixer tokens/sec at Jamba shapes (d_inner 8192, N 16) and % of roofline"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="jmix", choices=["jmix", "reference"])
+    ap.add_argument("--workload", default="jamba_b8_l4096")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            m = json.load(f)
+        return dict(hbm=m["hbm_gbs"], bf16=m["bf16_tflops"],
+                    bf16_sust=m["bf16_tflops_sustained"], sm_max=m.get("sm_max_mhz", 1965.0),
+                    src="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, sm_max=1965.0, src="fallback")
+
+
+# ----------------------------------------------------------------- per-unit work
+def work_per_token(w):
+    """Algorithmic work per token (a token = one position across all d_inner channels)."""
+    d, R, N = w.d_inner, w.dt_rank, w.d_state
+    es = 2 if w.io == "bf16" else 4
+    return dict(bytes=3 * d * es,                       # x, z in; y out
+                tc_flop=2 * d * (R + 2 * N) + 2 * R * d,  # x_proj + dt_proj
+                exp=d * N)                              # scan decays
+
+
+def kernel_units(name, w, tokens):
+    """(bound, algorithmic amount, unit) of one launch of a kernel over `tokens` tokens."""
+    d, R, N = w.d_inner, w.dt_rank, w.d_state
+    es = 2 if w.io == "bf16" else 4
+    if "scan" in name:
+        return "alu", tokens * d * N, "Gexp/s"
+    if "x_proj" in name or "xproj" in name:
+        return "tensor", tokens * 2 * d * (R + 2 * N), "TFLOP/s"
+    if "dt_proj" in name:
+        return "tensor", tokens * 2 * R * d, "TFLOP/s"
+    if "conv" in name:
+        return "hbm", tokens * d * es * 2, "GB/s"     # x in, u out
+    return "hbm", tokens * (R + 2 * N) * 4 * 2, "GB/s"
+
+
+# ------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.proc = None
+        self.lines = []
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", gpu_id], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self, t0: float, t1: float):
+        import datetime
+        rows = []
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 10:
+                continue
+            try:
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(f[2]), float(f[3]), f[4], f[5:]))
+            except Exception:
+                continue
+        inside = [r for r in rows if t0 - 0.05 <= r[0] <= t1 + 0.05] or rows
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        reasons = set()
+        for r in inside:
+            for n, v in zip(names[1:], r[4][1:]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(r[1] for r in inside),
+                "sm_max_mhz": max(r[2] for r in inside), "reasons": sorted(reasons),
+                "samples": len(inside)}
+
+
+# ------------------------------------------------------------- cpu baseline
+def oracle_rate(w, target_s: float, threads: int = 0):
+    """Time the fp64 oracle on sequence 0 of the workload, with a sample length
+    chosen so that the run takes about target_s seconds.  Returns
+    (tokens/s, cores, sample description)."""
+    import oracle
+    from mamba_selective_scan_jamba_b200 import synth
+    cores = threads or os.cpu_count() or 1
+    W = synth.make_weights(w)
+    L0 = min(w.seqlen, 64)
+    A = synth.make_activations(w.with_(batch=1, seqlen=L0))
+    t = time.perf_counter()
+    oracle.mixer_fwd(oracle.dims_of(w, batch=1, seqlen=L0, threads=cores), A["x"], A["z"], W)
+    dt0 = time.perf_counter() - t
+    L = int(max(16, min(w.seqlen, L0 * target_s / max(dt0, 1e-3))))
+    A = synth.make_activations(w.with_(batch=1, seqlen=L))
+    t = time.perf_counter()
+    oracle.mixer_fwd(oracle.dims_of(w, batch=1, seqlen=L, threads=cores), A["x"], A["z"], W)
+    dt = time.perf_counter() - t
+    return L / dt, cores, (f"sequence 0 of {w.name}, first {L} tokens (B=1, L={L}, "
+                           f"d_inner={w.d_inner}, dt_rank={w.dt_rank}), fp64 oracle, "
+                           f"{cores} threads, {dt:.1f} s")
+
+
+def reference_arm(args, w, rank, world):
+    if rank != 0:
+        return
+    import oracle
+    from mamba_selective_scan_jamba_b200 import synth
+    cores = os.cpu_count() or 1
+    W = synth.make_weights(w)
+    # calibrate a per-step sample of about 2 s
+    rate, _, _ = oracle_rate(w, 1.0, cores)
+    L = int(max(16, min(w.seqlen, rate * 2.0)))
+    A = synth.make_activations(w.with_(batch=1, seqlen=L))
+    m = oracle.dims_of(w, batch=1, seqlen=L, threads=cores)
+    for _ in range(args.warmup):
+        oracle.mixer_fwd(m, A["x"], A["z"], W)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.mixer_fwd(m, A["x"], A["z"], W)
+    dt = (time.perf_counter() - t) / max(1, args.steps)
+    value = L / dt
+    sample = (f"per step: sequence 0 of {w.name}, first {L} tokens (B=1, L={L}), fp64 oracle "
+              f"on {cores} host threads")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen,
+                       "d_inner": w.d_inner, "d_state": w.d_state, "dt_rank": w.dt_rank},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------- main
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from mamba_selective_scan_jamba_b200 import synth
+    base = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        reference_arm(args, base, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from mamba_selective_scan_jamba_b200 import devio, jmix
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    P = peaks()
+    # weak scaling: rank r owns sequences r*B .. r*B+B-1 of a world*B batch
+    w = base
+    wall = base.with_(batch=base.batch * world)
+    W = synth.make_weights(w)
+    A = synth.make_activations(wall, rank * w.batch, (rank + 1) * w.batch)
+    dev = torch.device("cuda", local)
+    Wd = devio.weights_to_device(W, dev)
+    x = devio.to_device(A["x"], dev)
+    z = devio.to_device(A["z"], dev)
+    y = torch.empty_like(x)
+    fs = torch.empty((w.batch, w.d_inner, w.d_state), dtype=torch.float32, device=dev)
+    d = devio.dims_of(w)
+    nbytes = jmix.jm_mixer_fwd_workspace_size(d)
+    ws = devio.workspace(nbytes, dev)
+    stream = torch.cuda.Stream(device=dev)
+    in_bytes = x.numel() * x.element_size() * 2
+
+    def step():
+        jmix.jm_mixer_fwd(d, x, z, Wd, y, fs, ws, nbytes, stream=stream)
+
+    with torch.cuda.stream(stream):
+        step()
+    stream.synchronize()
+    nk = jmix.jm_last_launch_count()
+    names = [jmix.jm_last_kernel_name(i) for i in range(nk)]
+    assert jmix.jm_poll_error(ws, stream) == jmix.JM_OK, jmix.jm_last_error()
+
+    # per-kernel events for every timed step (recorded on the launching stream)
+    K, Wm = args.steps, args.warmup
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(K)]
+    with torch.cuda.stream(stream):
+        for row in evs:           # materialise the events so their handles exist
+            for e in row:
+                e.record(stream)
+    stream.synchronize()
+    handles = [[e.cuda_event for e in row] for row in evs]
+
+    with torch.cuda.stream(stream):
+        for _ in range(Wm):
+            step()
+    stream.synchronize()
+    props = torch.cuda.get_device_properties(dev)
+    uuid = str(getattr(props, "uuid", ""))
+    gpu_id = (uuid if uuid.startswith("GPU-") else "GPU-" + uuid) if uuid else str(local)
+    sampler = ClockSampler(gpu_id)
+    time.sleep(0.6)   # let the sampler start
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    launches = 0
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for i in range(K):
+            jmix.jm_set_kernel_events(handles[i])
+            step()
+            launches += jmix.jm_last_launch_count()
+        end.record(stream)
+    jmix.jm_set_kernel_events(None)
+    stream.synchronize()
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    if world > 1:
+        dist.barrier()
+    time.sleep(0.3)
+    sampler.stop()
+    clocks = sampler.summary(t_wall0, t_wall1)
+    assert jmix.jm_poll_error(ws, stream) == jmix.JM_OK, jmix.jm_last_error()
+    ms = start.elapsed_time(end) / K
+    per_kernel = [sum(evs[i][k].elapsed_time(evs[i][k + 1]) for i in range(K)) / K
+                  for k in range(nk)]
+    if world > 1:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    tokens_rank = w.batch * w.seqlen
+    value = tokens_rank * world / (ms / 1e3)
+
+    # roofline of the dominant kernel
+    kd = max(range(nk), key=lambda k: per_kernel[k])
+    bound, amount, unit = kernel_units(names[kd], w, tokens_rank)
+    t_k = per_kernel[kd] / 1e3
+    if bound == "alu":
+        clk = P["sm_max"] * 1e6
+        peak = 16 * 148 * clk / 1e9        # MUFU ex2: 16 per clock per SM, 148 SMs
+        achieved = amount / t_k / 1e9
+    elif bound == "tensor":
+        peak = P["bf16_sust"]
+        achieved = amount / t_k / 1e12
+    else:
+        peak = P["hbm"]
+        achieved = amount / t_k / 1e9
+    wt = work_per_token(w)
+    t_ns = max(wt["tc_flop"] / (P["bf16_sust"] * 1e12), wt["bytes"] / (P["hbm"] * 1e9))
+    roof_tok_s = 1.0 / t_ns
+    roofline = {"kernel": names[kd], "bound": bound, "achieved": achieved, "peak": peak,
+                "unit": unit, "frac": achieved / peak, "traffic": None,
+                "peak_source": (f"MUFU 16/clk/SM x 148 SMs x {P['sm_max']:.0f} MHz (derived)"
+                                if bound == "alu" else f"{P['src']} MEASURED_PEAKS.json"),
+                "kernel_ms": per_kernel[kd],
+                "kernels_ms": {names[k]: round(per_kernel[k], 4) for k in range(nk)},
+                "north_star": {"roofline_tokens_per_s": roof_tok_s,
+                               "frac": value / world / roof_tok_s,
+                               "definition": "max(tc_flop/bf16 sustained peak, bytes/HBM) "
+                                             "per token, bytes = x,z in + y out"}}
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+            "warmup": Wm, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if w.io == "bf16" else "f32",
+            "data": "synthetic",
+            "config": {"workload": w.name, "batch_per_gpu": w.batch, "seqlen": w.seqlen,
+                       "d_inner": w.d_inner, "d_state": w.d_state, "dt_rank": w.dt_rank,
+                       "parallelism": f"replicas x{world} (independent sequences)",
+                       "l2": f"no flush: x+z = {in_bytes / 1e9:.2f} GB per step > 126 MB L2"},
+            "roofline": roofline, "gpu_launches": launches, "clocks": clocks}
+
+    # end to end through the host-buffer entry point
+    if not args.no_e2e:
+        xh, zh = devio.to_pinned(A["x"]), devio.to_pinned(A["z"])
+        yh = torch.empty(x.shape, dtype=x.dtype).pin_memory()
+        fsh = torch.empty(fs.shape, dtype=torch.float32).pin_memory()
+        Ke = max(1, min(K, 10))
+
+        def e2e_step():
+            jmix.jm_mixer_fwd_host(d, xh, zh, yh, fsh, x, z, y, fs, Wd, ws, nbytes,
+                                   stream=stream)
+
+        with torch.cuda.stream(stream):
+            e2e_step()
+        stream.synchronize()
+        if world > 1:
+            dist.barrier()
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            s2.record(stream)
+            for _ in range(Ke):
+                e2e_step()
+            e2.record(stream)
+        stream.synchronize()
+        ems = s2.elapsed_time(e2) / Ke
+        if world > 1:
+            t = torch.tensor([ems], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        line["e2e"] = {"value": tokens_rank * world / (ems / 1e3), "unit": "tokens/s",
+                       "h2d_bytes_per_step": in_bytes,
+                       "d2h_bytes_per_step": y.numel() * y.element_size() + fs.numel() * 4,
+                       "ms_per_step": ems, "steps": Ke,
+                       "api": "jm_mixer_fwd_host (pinned host x, z -> y, final_state)"}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, cores, sample = oracle_rate(w, 12.0)
+        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores,
+                                "kind": "oracle", "sample": sample}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,164 @@
+/* libjmix -- the Mamba-1 mixer core of Jamba v0.1 on B200 (sm_100a).
+ *
+ * The mixer core runs from the in_proj output (x, z) to the gated output y
+ * (TransformerLens "Jamba" adapter page: the Jamba Mamba mixer is Mamba-1 with
+ * in_proj / conv1d / x_proj / dt_proj / out_proj plus Jamba's own
+ * dt_layernorm / b_layernorm / c_layernorm on the selective parameters):
+ *
+ *   u      = SiLU(causal depthwise conv1d(x) + conv_b)         width d_conv
+ *   [dt|B|C] = u . xproj_w^T                                   x_proj, d_inner -> R + 2N
+ *   dt_n, B_n, C_n = RMSNorm(dt) w_dt, RMSNorm(B) w_B, RMSNorm(C) w_C
+ *   delta  = softplus(dt_n . dtproj_w^T + dt_bias)              dt_proj, R -> d_inner
+ *   h_t    = exp(delta_t A) * h_{t-1} + delta_t B_t u_t,  A = -exp(A_log)
+ *   y_t    = (C_t . h_t + D u_t) * SiLU(z_t)
+ *
+ * (discretisation exp(delta A), B-bar ~ delta B and the recurrence: aifetchly
+ * "Jamba Guide", section "Inside the Mamba State-Space Layers"; A_log and
+ * softplus(dt_proj(.)): the same guide, "Hands-On Implementation"; sizes
+ * d_inner 8192, d_state 16, d_conv 4, dt_rank 256: llm-architectures-explained
+ * "Jamba v0.1", "Every architecture field"; the cached conv and recurrent
+ * states that decoding threads through: TransformerLens "Jamba" adapter page.)
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ * Layouts are row-major, last index contiguous:
+ *   x, z, y          [batch, seqlen, d_inner]          io dtype
+ *   conv_w           [d_inner, d_conv]                 io dtype; tap d_conv-1 multiplies the current token
+ *   conv_b           [d_inner]                         io dtype
+ *   xproj_w          [dt_rank + 2*d_state, d_inner]    io dtype; rows are dt, then B, then C
+ *   dt_norm_w        [dt_rank]; b_norm_w, c_norm_w [d_state]   io dtype
+ *   dtproj_w         [d_inner, dt_rank]                io dtype
+ *   dt_bias, D       [d_inner]                         float32
+ *   A_log            [d_inner, d_state]                float32
+ *   conv states      [batch, d_inner, d_conv-1]        io dtype, oldest tap first
+ *   SSM states       [batch, d_inner, d_state]         float32
+ * All pointers given to the compute entry points are DEVICE pointers (the
+ * _host variant below is the one exception), owned by the caller.  libjmix
+ * never allocates, frees or synchronises, except jm_poll_error (which
+ * synchronises the given stream).  Calls are asynchronous on `stream`.
+ *
+ * Errors: host-side validation runs before any launch and returns
+ * JM_ERR_INVALID_ARG (NULL required pointer, negative size, pointer not
+ * 16-byte aligned, d_inner or dt_rank not a multiple of 8, y overlapping x or
+ * z, workspace too small -> JM_ERR_WORKSPACE) or JM_ERR_UNSUPPORTED
+ * (d_state != 16, d_conv != 4, dt_rank > 256).  A failed launch returns
+ * JM_ERR_CUDA.  Nothing is launched when validation fails.  There is no
+ * fallback path.  jm_last_error() gives a message for the calling thread.
+ */
+#ifndef JMIX_H
+#define JMIX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* jm_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  JM_OK = 0,
+  JM_ERR_INVALID_ARG = 1,
+  JM_ERR_UNSUPPORTED = 2,
+  JM_ERR_CUDA = 3,
+  JM_ERR_TIMEOUT = 4,  /* a bounded device-side wait ran out (reported by jm_poll_error) */
+  JM_ERR_WORKSPACE = 5
+} jm_status;
+
+typedef enum { JM_F32 = 0, JM_BF16 = 1 } jm_dtype;
+
+typedef struct {
+  int64_t batch;    /* sequences, >= 0 */
+  int64_t seqlen;   /* tokens per sequence, >= 0 (jm_mixer_step: must be 1) */
+  int64_t d_inner;  /* channels, > 0, multiple of 8 */
+  int64_t d_state;  /* N, must be 16 */
+  int64_t d_conv;   /* conv width, must be 4 */
+  int64_t dt_rank;  /* R, 8..256, multiple of 8 */
+  float eps;        /* RMSNorm epsilon, inside the square root, >= 0 */
+  jm_dtype io;      /* dtype of x, z, y, conv states and the io-dtype weights */
+} jm_dims;
+
+/* Bytes of device workspace jm_mixer_fwd needs for these dims (0 if the dims
+ * are invalid; see jm_last_error).  The workspace must be 256-byte aligned.
+ * Its first 256 bytes hold device-side error flags that jm_poll_error reads. */
+size_t jm_mixer_fwd_workspace_size(const jm_dims* dims);
+
+/* Same for jm_mixer_step (dims->seqlen must be 1). */
+size_t jm_mixer_step_workspace_size(const jm_dims* dims);
+
+/* Mixer forward over whole sequences: the formulas above for t = 0..seqlen-1.
+ *   x, z            in:  [B, L, d]
+ *   y               out: [B, L, d]; must not overlap x or z
+ *   final_state     out: [B, d, N] float32, h after the last token (required)
+ *   init_conv_state in:  [B, d, d_conv-1] conv history before token 0, or NULL = zeros
+ *   init_ssm_state  in:  [B, d, N] h before token 0, or NULL = zeros
+ *   final_conv_state out: [B, d, d_conv-1] the last d_conv-1 conv inputs, or NULL = skip;
+ *                   may equal init_conv_state (updated in place)
+ *   workspace       scratch of at least jm_mixer_fwd_workspace_size(dims) bytes
+ * With seqlen == 0 the final states are the initial ones (or zeros). */
+jm_status jm_mixer_fwd(const jm_dims* dims, const void* x, const void* z, const void* conv_w,
+                       const void* conv_b, const void* xproj_w, const void* dt_norm_w,
+                       const void* b_norm_w, const void* c_norm_w, const void* dtproj_w,
+                       const float* dt_bias, const float* A_log, const float* D, void* y,
+                       float* final_state, const void* init_conv_state,
+                       const float* init_ssm_state, void* final_conv_state, void* workspace,
+                       size_t ws_bytes, jm_stream_t stream);
+
+/* One decode step for every sequence (dims->seqlen must be 1): the forward
+ * with the cached states as history, then, in place,
+ *   conv_state[b, c, :] <- [conv_state[b, c, 1:], x_t[b, c]]  and  ssm_state <- h.
+ *   x_t, z_t   in:  [B, d];   y_t out: [B, d] (must not overlap x_t, z_t)
+ *   conv_state in/out [B, d, d_conv-1];  ssm_state in/out [B, d, N] float32 */
+jm_status jm_mixer_step(const jm_dims* dims, const void* x_t, const void* z_t, void* conv_state,
+                        float* ssm_state, const void* conv_w, const void* conv_b,
+                        const void* xproj_w, const void* dt_norm_w, const void* b_norm_w,
+                        const void* c_norm_w, const void* dtproj_w, const float* dt_bias,
+                        const float* A_log, const float* D, void* y_t, void* workspace,
+                        size_t ws_bytes, jm_stream_t stream);
+
+/* End-to-end forward from HOST buffers: copies x_host and z_host (pinned host
+ * memory, [B, L, d] io dtype) into the caller's device buffers x_dev / z_dev,
+ * runs jm_mixer_fwd, and copies y and the final SSM state back into y_host
+ * and final_state_host.  All copies are cudaMemcpyAsync on `stream`; the call
+ * returns without waiting (synchronise the stream before reading y_host).
+ * Weights and the optional states are device pointers as in jm_mixer_fwd. */
+jm_status jm_mixer_fwd_host(const jm_dims* dims, const void* x_host, const void* z_host,
+                            void* y_host, float* final_state_host, void* x_dev, void* z_dev,
+                            void* y_dev, float* final_state_dev, const void* conv_w,
+                            const void* conv_b, const void* xproj_w, const void* dt_norm_w,
+                            const void* b_norm_w, const void* c_norm_w, const void* dtproj_w,
+                            const float* dt_bias, const float* A_log, const float* D,
+                            void* workspace, size_t ws_bytes, jm_stream_t stream);
+
+/* Synchronises `stream`, then reads the error flags in `workspace`'s first
+ * 256 bytes: JM_ERR_TIMEOUT if a bounded device-side wait ran out since the
+ * last call that cleared them (every jm_mixer_fwd / jm_mixer_step clears
+ * them), JM_ERR_CUDA if the stream reports an error, JM_OK otherwise. */
+jm_status jm_poll_error(void* workspace, jm_stream_t stream);
+
+/* Message of the last failed call on this thread ("" if none). */
+const char* jm_last_error(void);
+
+/* Number of kernel launches the last successful jm_mixer_fwd / jm_mixer_step /
+ * jm_mixer_fwd_host on this thread issued (for launch accounting). */
+int jm_last_launch_count(void);
+
+/* Name of the index-th kernel the last successful compute call on this thread
+ * launched ("" when out of range).  The string is static. */
+const char* jm_last_kernel_name(int index);
+
+/* Per-kernel timing hook for benchmarks.  `events` is an array of n_events
+ * cudaEvent_t handles created by the caller.  While set (for calls on this
+ * thread), each compute call records events[0] on its stream before its
+ * first kernel and events[i] right after its i-th kernel, for i < n_events;
+ * the caller reads the kernel durations with cudaEventElapsedTime.  Pass
+ * (NULL, 0) to stop.  Returns JM_ERR_INVALID_ARG for a NULL array with
+ * n_events > 0. */
+jm_status jm_set_kernel_events(void* const* events, int n_events);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* JMIX_H */

@@ -1,0 +1,379 @@
+// The libjmix C ABI: host-side validation, workspace sizing and dispatch.
+// Every check runs before any launch; no entry point allocates device memory.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "jmix_internal.cuh"
+
+#define JM_API extern "C" __attribute__((visibility("default")))
+
+namespace jmix {
+
+static thread_local char g_msg[512];
+static thread_local int g_launches = 0;
+static thread_local void* const* g_events = nullptr;
+static thread_local int g_n_events = 0;
+
+void launches_begin(Problem& p) {
+  if (p.events && p.n_events > 0) cudaEventRecord((cudaEvent_t)p.events[0], p.stream);
+}
+
+static thread_local const char* g_names[kMaxLaunches];
+
+void launched(Problem& p, const char* name) {
+  if (p.launches < kMaxLaunches) p.names[p.launches] = name;
+  p.launches++;
+  if (p.events && p.launches < p.n_events)
+    cudaEventRecord((cudaEvent_t)p.events[p.launches], p.stream);
+}
+
+void set_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+}
+
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return na && nb && x < y + nb && y < x + na;
+}
+
+jm_status check_dims(const jm_dims* dm, bool step) {
+  if (!dm) {
+    set_error("dims is NULL");
+    return JM_ERR_INVALID_ARG;
+  }
+  if (dm->batch < 0 || dm->seqlen < 0 || dm->d_inner <= 0 || dm->dt_rank <= 0 ||
+      dm->d_state <= 0 || dm->d_conv <= 0) {
+    set_error("sizes must be positive (batch, seqlen >= 0)");
+    return JM_ERR_INVALID_ARG;
+  }
+  if (step && dm->seqlen != 1) {
+    set_error("jm_mixer_step needs seqlen == 1 (got %lld)", (long long)dm->seqlen);
+    return JM_ERR_INVALID_ARG;
+  }
+  if (dm->io != JM_F32 && dm->io != JM_BF16) {
+    set_error("io dtype must be JM_F32 or JM_BF16");
+    return JM_ERR_INVALID_ARG;
+  }
+  if (!(dm->eps >= 0.0f) || dm->eps != dm->eps || dm->eps > 1e30f) {
+    set_error("eps must be finite and >= 0");
+    return JM_ERR_INVALID_ARG;
+  }
+  if (dm->d_state != kN || dm->d_conv != kConv) {
+    set_error("only d_state == 16 and d_conv == 4 are built (got %lld, %lld)",
+              (long long)dm->d_state, (long long)dm->d_conv);
+    return JM_ERR_UNSUPPORTED;
+  }
+  if (dm->d_inner % 8 || dm->dt_rank % 8) {
+    set_error("d_inner and dt_rank must be multiples of 8 (got %lld, %lld)",
+              (long long)dm->d_inner, (long long)dm->dt_rank);
+    return JM_ERR_INVALID_ARG;
+  }
+  if (dm->dt_rank > kMaxRank) {
+    set_error("dt_rank > %d is not built (got %lld)", kMaxRank, (long long)dm->dt_rank);
+    return JM_ERR_UNSUPPORTED;
+  }
+  // element counts must stay far inside int64
+  const double tok = (double)dm->batch * (double)dm->seqlen;
+  if (tok * (double)dm->d_inner > 4.0e15) {
+    set_error("problem too large");
+    return JM_ERR_INVALID_ARG;
+  }
+  return JM_OK;
+}
+
+void fill_problem(Problem& p, const jm_dims* dm) {
+  memset(&p, 0, sizeof(p));
+  p.B = dm->batch;
+  p.L = dm->seqlen;
+  p.d = dm->d_inner;
+  p.R = dm->dt_rank;
+  p.P = dm->dt_rank + 2 * kN;
+  p.T = dm->batch * dm->seqlen;
+  p.eps = dm->eps;
+  p.io = dm->io;
+}
+
+size_t ws_bytes_for(const Problem& p) {
+  return p.io == JM_BF16 ? fast_ws_bytes(p) : simple_ws_bytes(p);
+}
+
+cudaError_t dispatch(Problem& p) {
+  return p.io == JM_BF16 ? run_fast(p) : run_simple(p);
+}
+
+size_t esize(jm_dtype io) { return io == JM_BF16 ? 2 : 4; }
+
+// Pointer checks common to fwd and step.  io-dtype tensors used as TMA or
+// 128-bit vector operands must be 16-byte aligned; float32 ones 16 bytes too.
+jm_status check_common(const Problem& p, const char* const names[], const void* const ptrs[],
+                       int n) {
+  for (int i = 0; i < n; ++i) {
+    if (!ptrs[i]) {
+      set_error("%s is NULL", names[i]);
+      return JM_ERR_INVALID_ARG;
+    }
+    if (!aligned(ptrs[i], 16)) {
+      set_error("%s is not 16-byte aligned", names[i]);
+      return JM_ERR_INVALID_ARG;
+    }
+  }
+  return JM_OK;
+}
+
+jm_status check_ws(const Problem& p, void* ws, size_t ws_bytes) {
+  size_t need = ws_bytes_for(p);
+  if (!ws) {
+    set_error("workspace is NULL");
+    return JM_ERR_WORKSPACE;
+  }
+  if (!aligned(ws, 256)) {
+    set_error("workspace must be 256-byte aligned");
+    return JM_ERR_WORKSPACE;
+  }
+  if (ws_bytes < need) {
+    set_error("workspace too small: %zu bytes given, %zu needed", ws_bytes, need);
+    return JM_ERR_WORKSPACE;
+  }
+  return JM_OK;
+}
+
+jm_status finish(Problem& p, cudaError_t e) {
+  if (e != cudaSuccess) {
+    set_error("CUDA error: %s", cudaGetErrorString(e));
+    return JM_ERR_CUDA;
+  }
+  g_launches = p.launches;
+  for (int i = 0; i < kMaxLaunches; ++i) g_names[i] = i < p.launches ? p.names[i] : nullptr;
+  g_msg[0] = 0;
+  return JM_OK;
+}
+
+}  // namespace
+}  // namespace jmix
+
+using namespace jmix;
+
+JM_API size_t jm_mixer_fwd_workspace_size(const jm_dims* dims) {
+  if (check_dims(dims, false) != JM_OK) return 0;
+  Problem p;
+  fill_problem(p, dims);
+  return ws_bytes_for(p);
+}
+
+JM_API size_t jm_mixer_step_workspace_size(const jm_dims* dims) {
+  if (check_dims(dims, true) != JM_OK) return 0;
+  Problem p;
+  fill_problem(p, dims);
+  p.decode = true;
+  return ws_bytes_for(p);
+}
+
+static jm_status fwd_impl(const jm_dims* dims, const void* x, const void* z, const void* conv_w,
+                          const void* conv_b, const void* xproj_w, const void* dt_norm_w,
+                          const void* b_norm_w, const void* c_norm_w, const void* dtproj_w,
+                          const float* dt_bias, const float* A_log, const float* D, void* y,
+                          float* final_state, const void* init_conv_state,
+                          const float* init_ssm_state, void* final_conv_state, void* workspace,
+                          size_t ws_bytes, jm_stream_t stream, bool step, Problem& p) {
+  jm_status st = check_dims(dims, step);
+  if (st != JM_OK) return st;
+  fill_problem(p, dims);
+  p.decode = step;
+  const char* const wn[] = {"conv_w", "conv_b", "xproj_w", "dt_norm_w", "b_norm_w", "c_norm_w",
+                            "dtproj_w", "dt_bias", "A_log", "D", "final_state"};
+  const void* const wp[] = {conv_w, conv_b, xproj_w, dt_norm_w, b_norm_w, c_norm_w,
+                            dtproj_w, dt_bias, A_log, D, final_state};
+  if ((st = check_common(p, wn, wp, 11)) != JM_OK) return st;
+  const size_t es = esize(p.io);
+  const size_t act = (size_t)p.T * (size_t)p.d * es;
+  if (p.T > 0) {
+    const char* const an[] = {"x", "z", "y"};
+    const void* const ap[] = {x, z, y};
+    if ((st = check_common(p, an, ap, 3)) != JM_OK) return st;
+    if (overlap(y, act, x, act) || overlap(y, act, z, act)) {
+      set_error("y overlaps x or z");
+      return JM_ERR_INVALID_ARG;
+    }
+  }
+  const char* const on[] = {"init_conv_state", "init_ssm_state", "final_conv_state"};
+  const void* const op[] = {init_conv_state, init_ssm_state, final_conv_state};
+  for (int i = 0; i < 3; ++i)
+    if (op[i] && !aligned(op[i], 16)) {
+      set_error("%s is not 16-byte aligned", on[i]);
+      return JM_ERR_INVALID_ARG;
+    }
+  if ((st = check_ws(p, workspace, ws_bytes)) != JM_OK) return st;
+  p.x = x;
+  p.z = z;
+  p.conv_w = conv_w;
+  p.conv_b = conv_b;
+  p.xproj_w = xproj_w;
+  p.dtn_w = dt_norm_w;
+  p.bn_w = b_norm_w;
+  p.cn_w = c_norm_w;
+  p.dtproj_w = dtproj_w;
+  p.dt_bias = dt_bias;
+  p.A_log = A_log;
+  p.D = D;
+  p.y = y;
+  p.final_state = final_state;
+  p.init_conv = init_conv_state;
+  p.init_ssm = init_ssm_state;
+  p.final_conv = final_conv_state;
+  p.ws = static_cast<char*>(workspace);
+  p.ws_bytes = ws_bytes;
+  p.stream = reinterpret_cast<cudaStream_t>(stream);
+  p.launches = 0;
+  p.events = g_events;
+  p.n_events = g_n_events;
+  if (p.B == 0) return finish(p, cudaSuccess);
+  if (p.L == 0) {
+    // nothing to scan: the final states are the initial ones
+    const size_t ssz = (size_t)p.B * p.d * kN * 4, csz = (size_t)p.B * p.d * (kConv - 1) * es;
+    cudaError_t e = init_ssm_state
+                        ? cudaMemcpyAsync(final_state, init_ssm_state, ssz,
+                                          cudaMemcpyDeviceToDevice, p.stream)
+                        : cudaMemsetAsync(final_state, 0, ssz, p.stream);
+    if (e == cudaSuccess && final_conv_state && final_conv_state != init_conv_state)
+      e = init_conv_state ? cudaMemcpyAsync(final_conv_state, init_conv_state, csz,
+                                            cudaMemcpyDeviceToDevice, p.stream)
+                          : cudaMemsetAsync(final_conv_state, 0, csz, p.stream);
+    return finish(p, e);
+  }
+  return finish(p, dispatch(p));
+}
+
+JM_API jm_status jm_mixer_fwd(const jm_dims* dims, const void* x, const void* z,
+                              const void* conv_w, const void* conv_b, const void* xproj_w,
+                              const void* dt_norm_w, const void* b_norm_w, const void* c_norm_w,
+                              const void* dtproj_w, const float* dt_bias, const float* A_log,
+                              const float* D, void* y, float* final_state,
+                              const void* init_conv_state, const float* init_ssm_state,
+                              void* final_conv_state, void* workspace, size_t ws_bytes,
+                              jm_stream_t stream) {
+  Problem p;
+  return fwd_impl(dims, x, z, conv_w, conv_b, xproj_w, dt_norm_w, b_norm_w, c_norm_w, dtproj_w,
+                  dt_bias, A_log, D, y, final_state, init_conv_state, init_ssm_state,
+                  final_conv_state, workspace, ws_bytes, stream, false, p);
+}
+
+JM_API jm_status jm_mixer_step(const jm_dims* dims, const void* x_t, const void* z_t,
+                               void* conv_state, float* ssm_state, const void* conv_w,
+                               const void* conv_b, const void* xproj_w, const void* dt_norm_w,
+                               const void* b_norm_w, const void* c_norm_w, const void* dtproj_w,
+                               const float* dt_bias, const float* A_log, const float* D,
+                               void* y_t, void* workspace, size_t ws_bytes, jm_stream_t stream) {
+  if (!conv_state || !ssm_state) {
+    set_error("conv_state and ssm_state are required");
+    return JM_ERR_INVALID_ARG;
+  }
+  Problem p;
+  return fwd_impl(dims, x_t, z_t, conv_w, conv_b, xproj_w, dt_norm_w, b_norm_w, c_norm_w,
+                  dtproj_w, dt_bias, A_log, D, y_t, ssm_state, conv_state, ssm_state, conv_state,
+                  workspace, ws_bytes, stream, true, p);
+}
+
+JM_API jm_status jm_mixer_fwd_host(const jm_dims* dims, const void* x_host, const void* z_host,
+                                   void* y_host, float* final_state_host, void* x_dev,
+                                   void* z_dev, void* y_dev, float* final_state_dev,
+                                   const void* conv_w, const void* conv_b, const void* xproj_w,
+                                   const void* dt_norm_w, const void* b_norm_w,
+                                   const void* c_norm_w, const void* dtproj_w,
+                                   const float* dt_bias, const float* A_log, const float* D,
+                                   void* workspace, size_t ws_bytes, jm_stream_t stream) {
+  jm_status st = check_dims(dims, false);
+  if (st != JM_OK) return st;
+  const size_t act = (size_t)dims->batch * dims->seqlen * dims->d_inner * esize(dims->io);
+  const size_t sst = (size_t)dims->batch * dims->d_inner * kN * 4;
+  if (act && (!x_host || !z_host || !y_host)) {
+    set_error("host buffers are required");
+    return JM_ERR_INVALID_ARG;
+  }
+  if (!final_state_host) {
+    set_error("final_state_host is NULL");
+    return JM_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // validate everything before the first copy is queued
+  Problem probe;
+  fill_problem(probe, dims);
+  if ((st = check_ws(probe, workspace, ws_bytes)) != JM_OK) return st;
+  if (act && (!x_dev || !z_dev || !y_dev)) {
+    set_error("device staging buffers are required");
+    return JM_ERR_INVALID_ARG;
+  }
+  cudaError_t e = cudaSuccess;
+  if (act) {
+    e = cudaMemcpyAsync(x_dev, x_host, act, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(z_dev, z_host, act, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) {
+      set_error("CUDA error: %s", cudaGetErrorString(e));
+      return JM_ERR_CUDA;
+    }
+  }
+  Problem p;
+  st = fwd_impl(dims, x_dev, z_dev, conv_w, conv_b, xproj_w, dt_norm_w, b_norm_w, c_norm_w,
+                dtproj_w, dt_bias, A_log, D, y_dev, final_state_dev, nullptr, nullptr, nullptr,
+                workspace, ws_bytes, stream, false, p);
+  if (st != JM_OK) return st;
+  if (act) e = cudaMemcpyAsync(y_host, y_dev, act, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(final_state_host, final_state_dev, sst, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) {
+    set_error("CUDA error: %s", cudaGetErrorString(e));
+    return JM_ERR_CUDA;
+  }
+  return JM_OK;
+}
+
+JM_API jm_status jm_poll_error(void* workspace, jm_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    set_error("CUDA error: %s", cudaGetErrorString(e));
+    return JM_ERR_CUDA;
+  }
+  if (!workspace) {
+    set_error("workspace is NULL");
+    return JM_ERR_INVALID_ARG;
+  }
+  ErrFlags f;
+  e = cudaMemcpyAsync(&f, workspace, sizeof(f), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    set_error("CUDA error: %s", cudaGetErrorString(e));
+    return JM_ERR_CUDA;
+  }
+  if (f.timeout) {
+    set_error("a bounded device-side wait ran out (site %u)", f.where);
+    return JM_ERR_TIMEOUT;
+  }
+  return JM_OK;
+}
+
+JM_API const char* jm_last_error(void) { return g_msg; }
+
+JM_API int jm_last_launch_count(void) { return g_launches; }
+
+JM_API const char* jm_last_kernel_name(int index) {
+  if (index < 0 || index >= kMaxLaunches || index >= g_launches || !g_names[index]) return "";
+  return g_names[index];
+}
+
+JM_API jm_status jm_set_kernel_events(void* const* events, int n_events) {
+  if (n_events < 0 || (n_events > 0 && !events)) {
+    set_error("events must be NULL with n_events == 0, or an array of n_events events");
+    return JM_ERR_INVALID_ARG;
+  }
+  g_events = n_events ? events : nullptr;
+  g_n_events = n_events;
+  return JM_OK;
+}

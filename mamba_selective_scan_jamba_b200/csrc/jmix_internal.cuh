@@ -1,0 +1,77 @@
+// Internal declarations shared by the libjmix translation units.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "jmix.h"
+
+namespace jmix {
+
+constexpr int kN = 16;       // d_state (compile time)
+constexpr int kConv = 4;     // d_conv (compile time)
+constexpr int kMaxRank = 256;
+
+// The first 256 bytes of every workspace.
+struct ErrFlags {
+  unsigned int timeout;   // a bounded wait ran out
+  unsigned int where;     // kernel-specific code of the first wait that ran out
+  unsigned int pad[62];
+};
+static_assert(sizeof(ErrFlags) == 256, "error header is 256 bytes");
+
+// One mixer call (forward or decode step) after host validation.
+struct Problem {
+  int64_t B, L, d, R, P, T;
+  float eps;
+  jm_dtype io;
+  const void* x;
+  const void* z;
+  const void* conv_w;
+  const void* conv_b;
+  const void* xproj_w;
+  const void* dtn_w;
+  const void* bn_w;
+  const void* cn_w;
+  const void* dtproj_w;
+  const float* dt_bias;
+  const float* A_log;
+  const float* D;
+  void* y;
+  float* final_state;
+  const void* init_conv;   // may be null
+  const float* init_ssm;   // may be null
+  void* final_conv;        // may be null; may equal init_conv
+  char* ws;
+  size_t ws_bytes;
+  cudaStream_t stream;
+  bool decode;             // jm_mixer_step
+  int launches;            // kernels launched so far by this call
+  void* const* events;     // optional per-kernel timing events (jm_set_kernel_events)
+  int n_events;
+  const char* names[16];   // kernel names in launch order
+};
+
+// Records events[0] (if timing events are set) before the first kernel.
+void launches_begin(Problem& p);
+// Counts one kernel launch (named `name` for jm_last_kernel_name) and
+// records events[launches] after it.
+void launched(Problem& p, const char* name);
+
+constexpr int kMaxLaunches = 16;
+
+inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// The portable SIMT path (any io dtype; the only path for float32 io).
+size_t simple_ws_bytes(const Problem& p);
+cudaError_t run_simple(Problem& p);
+
+// The bf16 path on tcgen05 tensor cores.
+size_t fast_ws_bytes(const Problem& p);
+cudaError_t run_fast(Problem& p);
+
+// Per-thread message for jm_last_error.
+void set_error(const char* fmt, ...);
+
+}  // namespace jmix

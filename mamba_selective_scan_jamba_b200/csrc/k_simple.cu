@@ -1,0 +1,257 @@
+// The portable SIMT path of the mixer core: one kernel per step, float32
+// arithmetic throughout, intermediates in the workspace as float32.
+//
+// It is the only path for float32 io (TF32 tensor cores cannot meet a 1e-4
+// tolerance) and serves any io dtype.  In bf16 mode it rounds at the same two
+// points as the tensor-core path: u after the SiLU and dt_n before dt_proj.
+//
+// Steps (TransformerLens "Jamba" adapter page for the pipeline; aifetchly
+// "Jamba Guide", "Inside the Mamba State-Space Layers", for the scan):
+//   k_conv_silu     u = SiLU(conv1d(x) + conv_b)
+//   k_gemm_nt       p = u . xproj_w^T                 (x_proj)
+//   k_norms         dt_n, B_n, C_n = RMSNorm(.) w
+//   k_gemm_nt       delta = softplus(dt_n . dtproj_w^T + dt_bias)   (dt_proj)
+//   k_scan_simple   h, y (one thread per (sequence, channel), 16 states)
+//   k_final_conv    final conv state
+#include "jmix_internal.cuh"
+
+namespace jmix {
+namespace {
+
+__device__ __forceinline__ float ld(const float* p) { return *p; }
+__device__ __forceinline__ float ld(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+__device__ __forceinline__ void st(float* p, float v) { *p = v; }
+__device__ __forceinline__ void st(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+__device__ __forceinline__ float to_bf16_value(float v) {
+  return __bfloat162float(__float2bfloat16_rn(v));
+}
+
+__device__ __forceinline__ float silu_precise(float v) { return v / (1.0f + expf(-v)); }
+
+__device__ __forceinline__ float softplus_precise(float v) {
+  return fmaxf(v, 0.0f) + log1pf(expf(-fabsf(v)));
+}
+
+template <typename T>
+__global__ void k_conv_silu(const T* __restrict__ x, const T* __restrict__ conv_w,
+                            const T* __restrict__ conv_b, const T* __restrict__ hist, int64_t L,
+                            int64_t d, int64_t total, int round_u, float* __restrict__ u) {
+  int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= total) return;
+  int64_t c = i % d, g = i / d;
+  int64_t b = g / L, t = g % L;
+  float acc = ld(conv_b + c);
+#pragma unroll
+  for (int k = 0; k < kConv; ++k) {
+    int64_t tau = t - (kConv - 1) + k;
+    float xv = 0.0f;
+    if (tau >= 0)
+      xv = ld(x + (b * L + tau) * d + c);
+    else if (hist)
+      xv = ld(hist + (b * d + c) * (kConv - 1) + (kConv - 1) + tau);
+    acc = fmaf(ld(conv_w + c * kConv + k), xv, acc);
+  }
+  float v = silu_precise(acc);
+  u[i] = round_u ? to_bf16_value(v) : v;
+}
+
+// out[m, n] = sum_k A[m, k] * W[n, k]   (A float32 [M, K], W io dtype [N, K])
+// EPI 0: plain store.  EPI 1: out = softplus(acc + bias[n]).
+// Tile 32 (m) x 32 (n), k-step 32, 256 threads, 4 outputs per thread.
+template <typename T, int EPI>
+__global__ void k_gemm_nt(const float* __restrict__ A, const T* __restrict__ W, int64_t M,
+                          int64_t N, int64_t K, const float* __restrict__ bias,
+                          float* __restrict__ out) {
+  __shared__ float As[32][33];
+  __shared__ float Ws[32][33];
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int64_t m0 = (int64_t)blockIdx.y * 32, n0 = (int64_t)blockIdx.x * 32;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int64_t k0 = 0; k0 < K; k0 += 32) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      int r = ty + 8 * i;
+      int64_t m = m0 + r, n = n0 + r, k = k0 + tx;
+      As[r][tx] = (m < M && k < K) ? A[m * K + k] : 0.0f;
+      Ws[r][tx] = (n < N && k < K) ? ld(W + n * K + k) : 0.0f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < 32; ++kk) {
+      float w = Ws[tx][kk];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[i] = fmaf(As[ty + 8 * i][kk], w, acc[i]);
+    }
+    __syncthreads();
+  }
+  const int64_t n = n0 + tx;
+  if (n >= N) return;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    int64_t m = m0 + ty + 8 * i;
+    if (m >= M) continue;
+    float v = acc[i];
+    if (EPI == 1) v = softplus_precise(v + bias[n]);
+    out[m * N + n] = v;
+  }
+}
+
+// One warp per token: RMSNorm of the dt (R), B (16) and C (16) slices of p.
+template <typename T>
+__global__ void k_norms(const float* __restrict__ p, const T* __restrict__ wdt,
+                        const T* __restrict__ wb, const T* __restrict__ wc, int64_t Tn, int R,
+                        float eps, int round_dt, float* __restrict__ dtn, float* __restrict__ Bn,
+                        float* __restrict__ Cn) {
+  const int lane = threadIdx.x & 31;
+  const int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (g >= Tn) return;
+  const int P = R + 2 * kN;
+  const float* row = p + g * P;
+  float ss = 0.f;
+  for (int j = lane; j < R; j += 32) ss = fmaf(row[j], row[j], ss);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float inv_dt = 1.0f / sqrtf(ss / (float)R + eps);
+  for (int j = lane; j < R; j += 32) {
+    float v = row[j] * inv_dt * ld(wdt + j);
+    dtn[g * R + j] = round_dt ? to_bf16_value(v) : v;
+  }
+  // lanes 0..15 -> B, 16..31 -> C
+  const int n = lane & 15;
+  const float v = row[R + lane];
+  float s2 = v * v;
+#pragma unroll
+  for (int o = 8; o; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+  const float inv = 1.0f / sqrtf(s2 / (float)kN + eps);
+  if (lane < 16)
+    Bn[g * kN + n] = v * inv * ld(wb + n);
+  else
+    Cn[g * kN + n] = v * inv * ld(wc + n);
+}
+
+// One thread per (sequence, channel): the recurrence over all tokens, the D
+// skip, the SiLU(z) gate and the final state.
+template <typename T>
+__global__ void k_scan_simple(const float* __restrict__ delta, const float* __restrict__ u,
+                              const float* __restrict__ Bn, const float* __restrict__ Cn,
+                              const T* __restrict__ z, const float* __restrict__ A_log,
+                              const float* __restrict__ Dv, const float* h0, float* hT, T* y,
+                              int64_t L, int64_t d) {
+  const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t b = blockIdx.y;
+  if (c >= d) return;
+  float h[kN], A[kN];
+#pragma unroll
+  for (int n = 0; n < kN; ++n) {
+    A[n] = -expf(A_log[c * kN + n]);
+    h[n] = h0 ? h0[(b * d + c) * kN + n] : 0.0f;
+  }
+  const float Dc = Dv[c];
+  for (int64_t t = 0; t < L; ++t) {
+    const int64_t g = b * L + t;
+    const float dl = delta[g * d + c], uv = u[g * d + c];
+    const float du = dl * uv;
+    float acc = 0.f;
+#pragma unroll
+    for (int n = 0; n < kN; ++n) {
+      h[n] = fmaf(expf(dl * A[n]), h[n], du * __ldg(Bn + g * kN + n));
+      acc = fmaf(__ldg(Cn + g * kN + n), h[n], acc);
+    }
+    const float ys = fmaf(Dc, uv, acc);
+    st(y + g * d + c, ys * silu_precise(ld(z + g * d + c)));
+  }
+#pragma unroll
+  for (int n = 0; n < kN; ++n) hT[(b * d + c) * kN + n] = h[n];
+}
+
+// final_conv[b, c, k] = X(L - (K-1) + k, c); reads before writes, so
+// final_conv may equal hist.
+template <typename T>
+__global__ void k_final_conv(const T* __restrict__ x, const T* hist, T* final_conv, int64_t L,
+                             int64_t d, int64_t total) {
+  int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= total) return;
+  int64_t c = i % d, b = i / d;
+  T v[kConv - 1];
+#pragma unroll
+  for (int k = 0; k < kConv - 1; ++k) {
+    int64_t tau = L - (kConv - 1) + k;
+    if (tau >= 0)
+      v[k] = x[(b * L + tau) * d + c];
+    else if (hist)
+      v[k] = hist[(b * d + c) * (kConv - 1) + (kConv - 1) + tau];
+    else
+      v[k] = T(0.0f);
+  }
+#pragma unroll
+  for (int k = 0; k < kConv - 1; ++k) final_conv[(b * d + c) * (kConv - 1) + k] = v[k];
+}
+
+struct SimpleWs {
+  float *u, *delta, *p, *dtn, *Bn, *Cn;
+  size_t bytes;
+};
+
+SimpleWs simple_layout(const Problem& p, char* base) {
+  SimpleWs w{};
+  size_t off = sizeof(ErrFlags);
+  auto take = [&](size_t n) {
+    size_t o = off;
+    off = align256(off + n);
+    return base ? reinterpret_cast<float*>(base + o) : nullptr;
+  };
+  const size_t T = (size_t)p.T, d = (size_t)p.d;
+  w.u = take(T * d * 4);
+  w.delta = take(T * d * 4);
+  w.p = take(T * (size_t)p.P * 4);
+  w.dtn = take(T * (size_t)p.R * 4);
+  w.Bn = take(T * kN * 4);
+  w.Cn = take(T * kN * 4);
+  w.bytes = off;
+  return w;
+}
+
+template <typename T>
+cudaError_t run_simple_t(Problem& p) {
+  SimpleWs w = simple_layout(p, p.ws);
+  cudaStream_t s = p.stream;
+  const int round = p.io == JM_BF16 ? 1 : 0;
+  const int64_t td = p.T * p.d;
+  cudaMemsetAsync(p.ws, 0, sizeof(ErrFlags), s);
+  launches_begin(p);
+  k_conv_silu<T><<<(unsigned)((td + 255) / 256), 256, 0, s>>>(
+      (const T*)p.x, (const T*)p.conv_w, (const T*)p.conv_b, (const T*)p.init_conv, p.L, p.d, td,
+      round, w.u);
+  launched(p, "k_conv_silu");
+  k_gemm_nt<T, 0><<<dim3((unsigned)((p.P + 31) / 32), (unsigned)((p.T + 31) / 32)), 256, 0, s>>>(
+      w.u, (const T*)p.xproj_w, p.T, p.P, p.d, nullptr, w.p);
+  launched(p, "k_gemm_nt(x_proj)");
+  k_norms<T><<<(unsigned)((p.T + 7) / 8), 256, 0, s>>>(w.p, (const T*)p.dtn_w, (const T*)p.bn_w,
+                                                        (const T*)p.cn_w, p.T, (int)p.R, p.eps,
+                                                        round, w.dtn, w.Bn, w.Cn);
+  launched(p, "k_norms");
+  k_gemm_nt<T, 1><<<dim3((unsigned)((p.d + 31) / 32), (unsigned)((p.T + 31) / 32)), 256, 0, s>>>(
+      w.dtn, (const T*)p.dtproj_w, p.T, p.d, p.R, p.dt_bias, w.delta);
+  launched(p, "k_gemm_nt(dt_proj)");
+  k_scan_simple<T><<<dim3((unsigned)((p.d + 127) / 128), (unsigned)p.B), 128, 0, s>>>(
+      w.delta, w.u, w.Bn, w.Cn, (const T*)p.z, p.A_log, p.D, p.init_ssm, p.final_state, (T*)p.y,
+      p.L, p.d);
+  launched(p, "k_scan_simple");
+  if (p.final_conv) {
+    const int64_t bd = p.B * p.d;
+    k_final_conv<T><<<(unsigned)((bd + 255) / 256), 256, 0, s>>>(
+        (const T*)p.x, (const T*)p.init_conv, (T*)p.final_conv, p.L, p.d, bd);
+    launched(p, "k_final_conv");
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t simple_ws_bytes(const Problem& p) { return simple_layout(p, nullptr).bytes; }
+
+cudaError_t run_simple(Problem& p) {
+  return p.io == JM_BF16 ? run_simple_t<__nv_bfloat16>(p) : run_simple_t<float>(p);
+}
+
+}  // namespace jmix

@@ -1,0 +1,181 @@
+"""Python binding of libjmix (ctypes; argument marshalling only).
+
+Every name mirrors the C ABI in ``include/jmix.h``.  Tensors may be torch
+tensors (their ``data_ptr()`` is passed) or raw integer addresses.  Every
+computation runs in libjmix's CUDA kernels; if the library is missing this
+module raises instead of falling back to anything else.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Mapping, Optional
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "_build", "libjmix.so")
+
+JM_OK, JM_ERR_INVALID_ARG, JM_ERR_UNSUPPORTED, JM_ERR_CUDA, JM_ERR_TIMEOUT, JM_ERR_WORKSPACE = range(6)
+JM_F32, JM_BF16 = 0, 1
+STATUS_NAMES = {0: "JM_OK", 1: "JM_ERR_INVALID_ARG", 2: "JM_ERR_UNSUPPORTED", 3: "JM_ERR_CUDA",
+                4: "JM_ERR_TIMEOUT", 5: "JM_ERR_WORKSPACE"}
+
+WEIGHT_NAMES = ("conv_w", "conv_b", "xproj_w", "dt_norm_w", "b_norm_w", "c_norm_w", "dtproj_w",
+                "dt_bias", "A_log", "D")
+
+EXPORTED = ("jm_mixer_fwd_workspace_size", "jm_mixer_step_workspace_size", "jm_mixer_fwd",
+            "jm_mixer_step", "jm_mixer_fwd_host", "jm_poll_error", "jm_last_error",
+            "jm_last_launch_count", "jm_last_kernel_name", "jm_set_kernel_events")
+
+
+class jm_dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64),
+                ("d_inner", ctypes.c_int64), ("d_state", ctypes.c_int64),
+                ("d_conv", ctypes.c_int64), ("dt_rank", ctypes.c_int64),
+                ("eps", ctypes.c_float), ("io", ctypes.c_int)]
+
+
+class JmixError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+_lib = None
+_vp = ctypes.c_void_p
+
+
+def load(path: Optional[str] = None) -> ctypes.CDLL:
+    """Load libjmix.so (built by ``build.build_libjmix``); raises if it is absent."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise FileNotFoundError(f"libjmix is not built ({p}); run __graft_entry__.build()")
+    lib = ctypes.CDLL(p)
+    lib.jm_mixer_fwd_workspace_size.restype = ctypes.c_size_t
+    lib.jm_mixer_fwd_workspace_size.argtypes = [ctypes.POINTER(jm_dims)]
+    lib.jm_mixer_step_workspace_size.restype = ctypes.c_size_t
+    lib.jm_mixer_step_workspace_size.argtypes = [ctypes.POINTER(jm_dims)]
+    lib.jm_mixer_fwd.restype = ctypes.c_int
+    lib.jm_mixer_fwd.argtypes = [ctypes.POINTER(jm_dims)] + [_vp] * 18 + [ctypes.c_size_t, _vp]
+    lib.jm_mixer_step.restype = ctypes.c_int
+    lib.jm_mixer_step.argtypes = [ctypes.POINTER(jm_dims)] + [_vp] * 16 + [ctypes.c_size_t, _vp]
+    lib.jm_mixer_fwd_host.restype = ctypes.c_int
+    lib.jm_mixer_fwd_host.argtypes = [ctypes.POINTER(jm_dims)] + [_vp] * 19 + [ctypes.c_size_t, _vp]
+    lib.jm_poll_error.restype = ctypes.c_int
+    lib.jm_poll_error.argtypes = [_vp, _vp]
+    lib.jm_last_error.restype = ctypes.c_char_p
+    lib.jm_last_error.argtypes = []
+    lib.jm_last_launch_count.restype = ctypes.c_int
+    lib.jm_last_launch_count.argtypes = []
+    lib.jm_last_kernel_name.restype = ctypes.c_char_p
+    lib.jm_last_kernel_name.argtypes = [ctypes.c_int]
+    lib.jm_set_kernel_events.restype = ctypes.c_int
+    lib.jm_set_kernel_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int]
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def dims(batch: int, seqlen: int, d_inner: int, dt_rank: int, io: int = JM_BF16,
+         eps: float = 1e-6, d_state: int = 16, d_conv: int = 4) -> jm_dims:
+    return jm_dims(batch, seqlen, d_inner, d_state, d_conv, dt_rank, eps, io)
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int) -> None:
+    if status != JM_OK:
+        raise JmixError(status, load().jm_last_error().decode())
+
+
+def jm_mixer_fwd_workspace_size(d: jm_dims) -> int:
+    return load().jm_mixer_fwd_workspace_size(ctypes.byref(d))
+
+
+def jm_mixer_step_workspace_size(d: jm_dims) -> int:
+    return load().jm_mixer_step_workspace_size(ctypes.byref(d))
+
+
+def _weights(w: Mapping):
+    return [_ptr(w[k]) for k in WEIGHT_NAMES]
+
+
+def jm_mixer_fwd(d: jm_dims, x, z, w: Mapping, y, final_state, workspace, ws_bytes: int,
+                 init_conv_state=None, init_ssm_state=None, final_conv_state=None,
+                 stream=None, check: bool = True) -> int:
+    st = load().jm_mixer_fwd(ctypes.byref(d), _ptr(x), _ptr(z), *_weights(w), _ptr(y),
+                             _ptr(final_state), _ptr(init_conv_state), _ptr(init_ssm_state),
+                             _ptr(final_conv_state), _ptr(workspace), ws_bytes, _stream(stream))
+    if check:
+        _check(st)
+    return st
+
+
+def jm_mixer_step(d: jm_dims, x_t, z_t, conv_state, ssm_state, w: Mapping, y_t, workspace,
+                  ws_bytes: int, stream=None, check: bool = True) -> int:
+    st = load().jm_mixer_step(ctypes.byref(d), _ptr(x_t), _ptr(z_t), _ptr(conv_state),
+                              _ptr(ssm_state), *_weights(w), _ptr(y_t), _ptr(workspace), ws_bytes,
+                              _stream(stream))
+    if check:
+        _check(st)
+    return st
+
+
+def jm_mixer_fwd_host(d: jm_dims, x_host, z_host, y_host, final_state_host, x_dev, z_dev, y_dev,
+                      final_state_dev, w: Mapping, workspace, ws_bytes: int, stream=None,
+                      check: bool = True) -> int:
+    st = load().jm_mixer_fwd_host(ctypes.byref(d), _ptr(x_host), _ptr(z_host), _ptr(y_host),
+                                  _ptr(final_state_host), _ptr(x_dev), _ptr(z_dev), _ptr(y_dev),
+                                  _ptr(final_state_dev), *_weights(w), _ptr(workspace), ws_bytes,
+                                  _stream(stream))
+    if check:
+        _check(st)
+    return st
+
+
+def jm_poll_error(workspace, stream=None) -> int:
+    return load().jm_poll_error(_ptr(workspace), _stream(stream))
+
+
+def jm_last_error() -> str:
+    return load().jm_last_error().decode()
+
+
+def jm_last_launch_count() -> int:
+    return load().jm_last_launch_count()
+
+
+def jm_last_kernel_name(index: int) -> str:
+    return load().jm_last_kernel_name(index).decode()
+
+
+_event_arr = None
+
+
+def jm_set_kernel_events(handles) -> None:
+    """Set (a sequence of raw cudaEvent_t handles) or clear (None) the per-kernel
+    timing events."""
+    global _event_arr
+    if not handles:
+        _event_arr = None
+        _check(load().jm_set_kernel_events(None, 0))
+        return
+    _event_arr = (ctypes.c_void_p * len(handles))(*handles)
+    _check(load().jm_set_kernel_events(_event_arr, len(handles)))

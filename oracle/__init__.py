@@ -154,13 +154,15 @@ def scan(delta, A, Bm, Cm, u, D, h0=None):
 def mixer_fwd(m: OrcDims, x, z, weights: Dict[str, np.ndarray], init_conv_state=None,
               init_ssm_state=None, channels: Optional[Sequence[int]] = None):
     """Mixer forward.  Returns (y [B,L,d or nch], final_state [B,d or nch,N],
-    final_conv [B,d or nch,K-1]) in float64."""
+    final_conv [B,d or nch,K-1]) in float64.  With ``channels``, the front end
+    still runs over every channel but only the chosen channels are scanned, and
+    x is read in its stored form (no float64 copy of a full-size x)."""
     B, L, d, N, K = m.batch, m.seqlen, m.d_inner, m.d_state, m.d_conv
-    W = [_f64(weights[k]) for k in _WNAMES]
-    x, z = _f64(x), _f64(z)
     assert x.shape == (B, L, d) and z.shape == (B, L, d)
+    W = [_f64(weights[k]) for k in _WNAMES]
     ic, iss = _f64(init_conv_state), _f64(init_ssm_state)
     if channels is None:
+        x, z = _f64(x), _f64(z)
         y = np.empty((B, L, d))
         fs = np.empty((B, d, N))
         fc = np.empty((B, d, K - 1))
@@ -169,10 +171,16 @@ def mixer_fwd(m: OrcDims, x, z, weights: Dict[str, np.ndarray], init_conv_state=
         return y, fs, fc
     ch = np.ascontiguousarray(channels, dtype=np.int64)
     nch = ch.size
+    xs = np.ascontiguousarray(x)
+    xkind = {np.dtype(np.uint16): 1, np.dtype(np.float32): 2}.get(xs.dtype, 0)
+    if xkind == 0:
+        xs = np.ascontiguousarray(xs, dtype=np.float64)
+    zsel = _f64(np.asarray(z)[:, :, ch])
     y = np.empty((B, L, nch))
     fs = np.empty((B, nch, N))
     fc = np.empty((B, nch, K - 1))
-    _L().orc_mixer_fwd_channels(ctypes.byref(m), _p(x), _p(z), *[_p(a) for a in W], _p(ic),
+    _L().orc_mixer_fwd_channels(ctypes.byref(m), xs.ctypes.data_as(ctypes.c_void_p),
+                                ctypes.c_int32(xkind), _p(zsel), *[_p(a) for a in W], _p(ic),
                                 _p(iss), ctypes.c_int64(nch),
                                 ch.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), _p(y), _p(fs),
                                 _p(fc))

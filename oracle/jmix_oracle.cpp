@@ -81,6 +81,23 @@ double round_bf16(double v) {
 
 double silu(double v) { return v / (1.0 + std::exp(-v)); }
 
+// Exact value of element i of a stored input: kind 0 = double, 1 = bf16 bit
+// pattern (uint16), 2 = float32.  (Input marshalling only.)
+struct Stored {
+  const void* p;
+  int32_t kind;
+  double operator[](int64_t i) const {
+    if (kind == 1) {
+      uint32_t u = (uint32_t)((const uint16_t*)p)[i] << 16;
+      float f;
+      std::memcpy(&f, &u, 4);
+      return (double)f;
+    }
+    if (kind == 2) return (double)((const float*)p)[i];
+    return ((const double*)p)[i];
+  }
+};
+
 double softplus(double v) { return std::max(v, 0.0) + std::log1p(std::exp(-std::fabs(v))); }
 
 }  // namespace
@@ -162,7 +179,7 @@ void orc_scan(int64_t L, int64_t d, int64_t N, const double* delta, const double
 
 // Front end of one sequence for tokens [t0, t1): u (optionally mirror-rounded),
 // p rows, normalised dt_n / Bn / Cn rows.
-static void front_end_rows(const orc_dims* m, const double* x, const double* conv_w,
+static void front_end_rows(const orc_dims* m, Stored x, const double* conv_w,
                            const double* conv_b, const double* xproj_wT /*[d,P]*/,
                            const double* dtn_w, const double* bn_w, const double* cn_w,
                            const double* hist, int64_t t0, int64_t t1, double* u_rows /*[t1-t0,d]*/,
@@ -221,9 +238,11 @@ static void dt_proj_channels(const orc_dims* m, const double* dtn, const double*
 // The whole mixer forward for the channels ch[0..nch) of every sequence.  The
 // front end (conv, x_proj, norms) runs over all channels, since B, C and dt
 // depend on all of them; dt_proj, the scan and the gate run only for ch.
-// y: [B, L, nch]; final_state: [B, nch, N] (or null); final_conv: [B, nch, K-1]
-// (or null).
-void orc_mixer_fwd_channels(const orc_dims* m, const double* x, const double* z,
+// x: [B, L, d] stored as x_kind (see Stored); z_sel: [B, L, nch], the z values
+// of the chosen channels.  y: [B, L, nch]; final_state: [B, nch, N] (or null);
+// final_conv: [B, nch, K-1] (or null).
+void orc_mixer_fwd_channels(const orc_dims* m, const void* x_data, int32_t x_kind,
+                            const double* z_sel,
                             const double* conv_w, const double* conv_b, const double* xproj_w,
                             const double* dtn_w, const double* bn_w, const double* cn_w,
                             const double* dtproj_w, const double* dt_bias, const double* A_log,
@@ -239,7 +258,10 @@ void orc_mixer_fwd_channels(const orc_dims* m, const double* x, const double* z,
   const int64_t blk = 64;
   const int64_t nblk = (L + blk - 1) / blk;
   for (int64_t b = 0; b < Bt; ++b) {
-    const double* xb = x + b * L * d;
+    const Stored xb{x_kind == 1   ? (const void*)((const uint16_t*)x_data + b * L * d)
+                    : x_kind == 2 ? (const void*)((const float*)x_data + b * L * d)
+                                  : (const void*)((const double*)x_data + b * L * d),
+                    x_kind};
     const double* hist = init_conv ? init_conv + b * d * (K - 1) : nullptr;
     parallel_for(nblk, threads, [&](int64_t ib) {
       int64_t t0 = ib * blk, t1 = std::min(L, t0 + blk);
@@ -265,7 +287,7 @@ void orc_mixer_fwd_channels(const orc_dims* m, const double* x, const double* z,
           acc += Cn[t * N + n] * h[n];
         }
         double ys = acc + D[c] * uv;
-        y[(b * L + t) * nch + i] = ys * silu(z[(b * L + t) * d + c]);
+        y[(b * L + t) * nch + i] = ys * silu(z_sel[(b * L + t) * nch + i]);
       }
       if (final_state)
         for (int64_t n = 0; n < N; ++n) final_state[(b * nch + i) * N + n] = h[n];
@@ -289,9 +311,9 @@ void orc_mixer_fwd(const orc_dims* m, const double* x, const double* z, const do
                    double* final_state, double* final_conv) {
   std::vector<int64_t> ch(m->d_inner);
   for (int64_t c = 0; c < m->d_inner; ++c) ch[c] = c;
-  orc_mixer_fwd_channels(m, x, z, conv_w, conv_b, xproj_w, dtn_w, bn_w, cn_w, dtproj_w, dt_bias,
-                         A_log, D, init_conv, init_ssm, m->d_inner, ch.data(), y, final_state,
-                         final_conv);
+  orc_mixer_fwd_channels(m, x, 0, z, conv_w, conv_b, xproj_w, dtn_w, bn_w, cn_w, dtproj_w,
+                         dt_bias, A_log, D, init_conv, init_ssm, m->d_inner, ch.data(), y,
+                         final_state, final_conv);
 }
 
 // One decode step for every sequence: the forward with L = 1 and the cached

@@ -1,0 +1,118 @@
+"""CPU checks of the C ABI: the library loads, exports every declared entry
+point, and rejects bad arguments on the host before any launch (none of the
+calls below reaches a CUDA call, so no GPU is needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from mamba_selective_scan_jamba_b200 import build, jmix
+
+HEADER = os.path.join(build.INCLUDE, "jmix.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build_libjmix()
+    return jmix.load()
+
+
+def declared_entry_points():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(jm_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_entry_points()
+    assert "jm_mixer_fwd" in names and "jm_mixer_step" in names
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(jmix.EXPORTED) == names
+
+
+def test_no_other_symbols_exported():
+    out = os.popen(f"nm -D --defined-only {jmix.LIB_PATH}").read()
+    syms = [l.split()[-1] for l in out.splitlines() if " T " in l]
+    assert sorted(syms) == sorted(jmix.EXPORTED)
+
+
+def test_built_for_sm100a_only():
+    flags = " ".join(build.NVCC_FLAGS)
+    assert "arch=compute_100a,code=sm_100a" in flags
+    assert flags.count("-gencode") == 1
+
+
+FAKE = 1 << 40   # an aligned, never-dereferenced address
+
+
+def fwd(d, ws_bytes=1 << 30, **over):
+    args = dict(x=FAKE, z=FAKE + (1 << 36), y=FAKE + (2 << 36), final_state=FAKE,
+                workspace=FAKE, init_conv_state=None, init_ssm_state=None, final_conv_state=None)
+    args.update(over)
+    W = {k: FAKE for k in jmix.WEIGHT_NAMES}
+    return jmix.jm_mixer_fwd(d, args["x"], args["z"], W, args["y"], args["final_state"],
+                             args["workspace"], ws_bytes, args["init_conv_state"],
+                             args["init_ssm_state"], args["final_conv_state"], stream=0,
+                             check=False)
+
+
+def test_workspace_size_rules(lib):
+    d = jmix.dims(8, 4096, 8192, 256)
+    n = jmix.jm_mixer_fwd_workspace_size(d)
+    assert n >= 256 + 8 * 4096 * 288 * 4
+    assert jmix.jm_mixer_fwd_workspace_size(jmix.dims(1, 4096, 8192, 256, d_state=8)) == 0
+    assert "d_state" in jmix.jm_last_error()
+    assert jmix.jm_mixer_step_workspace_size(jmix.dims(256, 2, 8192, 256)) == 0
+    assert jmix.jm_mixer_step_workspace_size(jmix.dims(256, 1, 8192, 256)) > 0
+
+
+@pytest.mark.parametrize("bad,code,msg", [
+    (dict(d_state=8), jmix.JM_ERR_UNSUPPORTED, "d_state"),
+    (dict(d_conv=3), jmix.JM_ERR_UNSUPPORTED, "d_conv"),
+    (dict(dt_rank=264), jmix.JM_ERR_UNSUPPORTED, "dt_rank"),
+    (dict(d_inner=100), jmix.JM_ERR_INVALID_ARG, "multiples of 8"),
+    (dict(dt_rank=12), jmix.JM_ERR_INVALID_ARG, "multiples of 8"),
+    (dict(batch=-1), jmix.JM_ERR_INVALID_ARG, "positive"),
+    (dict(eps=-1.0), jmix.JM_ERR_INVALID_ARG, "eps"),
+    (dict(io=7), jmix.JM_ERR_INVALID_ARG, "io dtype"),
+])
+def test_rejects_bad_dims(lib, bad, code, msg):
+    kw = dict(batch=2, seqlen=16, d_inner=256, dt_rank=16)
+    kw.update(bad)
+    d = jmix.dims(**kw)
+    assert fwd(d) == code
+    assert msg in jmix.jm_last_error()
+
+
+def test_rejects_bad_pointers(lib):
+    d = jmix.dims(2, 16, 256, 16)
+    assert fwd(d, x=None) == jmix.JM_ERR_INVALID_ARG and "x is NULL" in jmix.jm_last_error()
+    assert fwd(d, x=FAKE + 2) == jmix.JM_ERR_INVALID_ARG and "aligned" in jmix.jm_last_error()
+    assert fwd(d, y=FAKE) == jmix.JM_ERR_INVALID_ARG and "overlaps" in jmix.jm_last_error()
+    assert fwd(d, final_state=None) == jmix.JM_ERR_INVALID_ARG
+    assert fwd(d, init_ssm_state=FAKE + 4) == jmix.JM_ERR_INVALID_ARG
+    assert fwd(d, ws_bytes=100) == jmix.JM_ERR_WORKSPACE and "too small" in jmix.jm_last_error()
+    assert fwd(d, workspace=FAKE + 16) == jmix.JM_ERR_WORKSPACE
+    assert fwd(d, workspace=None) == jmix.JM_ERR_WORKSPACE
+
+
+def test_step_rejects_seqlen_and_missing_state(lib):
+    W = {k: FAKE for k in jmix.WEIGHT_NAMES}
+    d = jmix.dims(4, 2, 256, 16)
+    st = jmix.jm_mixer_step(d, FAKE, FAKE, FAKE, FAKE, W, FAKE + (1 << 36), FAKE, 1 << 30,
+                            stream=0, check=False)
+    assert st == jmix.JM_ERR_INVALID_ARG and "seqlen" in jmix.jm_last_error()
+    d = jmix.dims(4, 1, 256, 16)
+    st = jmix.jm_mixer_step(d, FAKE, FAKE, None, FAKE, W, FAKE + (1 << 36), FAKE, 1 << 30,
+                            stream=0, check=False)
+    assert st == jmix.JM_ERR_INVALID_ARG
+
+
+def test_binding_raises_on_error(lib):
+    with pytest.raises(jmix.JmixError) as e:
+        W = {k: FAKE for k in jmix.WEIGHT_NAMES}
+        jmix.jm_mixer_fwd(jmix.dims(1, 4, 256, 16, d_conv=2), FAKE, FAKE, W, FAKE, FAKE, FAKE,
+                          1 << 30, stream=0)
+    assert e.value.status == jmix.JM_ERR_UNSUPPORTED

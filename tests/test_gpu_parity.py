@@ -1,0 +1,216 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle, on cuda:0.
+
+Small cases span several channel tiles, token tiles and ragged tails and use
+random conv_b / norm weights / D / A_log and nonzero initial states, so every
+term of the mixer is exercised.  The full-size workloads are checked on sampled
+channels, which the oracle can compute exactly (the front end still runs over
+every channel, since dt, B and C depend on all of them).
+"""
+import numpy as np
+import pytest
+
+import oracle
+from mamba_selective_scan_jamba_b200 import synth
+from tests.helpers import TOL, check_fwd, f64, gpu_fwd, max_scaled_err
+
+pytestmark = pytest.mark.gpu
+
+
+def small(B, L, d, R, io="bf16", extra=True, seed=101):
+    return synth.Workload(f"small_{B}x{L}x{d}x{R}_{io}", B, L, d, R, io, seed=seed, extra=extra)
+
+
+def test_tiny_fp32_workload():
+    check_fwd(synth.WORKLOADS["tiny_fp32"])
+
+
+@pytest.mark.parametrize("B,L,d,R", [(1, 77, 128, 8), (2, 131, 200, 40), (3, 5, 64, 16)])
+def test_fp32_extra_terms_and_ragged(B, L, d, R):
+    check_fwd(small(B, L, d, R, io="f32"))
+
+
+@pytest.mark.parametrize("B,L,d,R,extra", [
+    (2, 300, 384, 64, True),      # 3 channel tiles, ragged token tail
+    (1, 77, 200, 40, True),       # channel tail (200 = 128 + 72), odd rank
+    (3, 1, 256, 16, True),        # L = 1: history only from the initial conv state
+    (2, 2, 256, 16, True),
+    (2, 3, 256, 16, True),
+    (2, 515, 1024, 256, True),    # Jamba rank, ragged L
+    (1, 130, 8192, 256, False),   # Jamba shapes, short sequence, the workloads' constants
+])
+def test_bf16_cases(B, L, d, R, extra):
+    check_fwd(small(B, L, d, R, extra=extra))
+
+
+def test_bf16_without_initial_states():
+    check_fwd(small(2, 150, 256, 32), use_init=False)
+
+
+def test_seqlen_zero_and_batch_zero():
+    import torch
+    from mamba_selective_scan_jamba_b200 import devio, jmix
+    w = small(2, 0, 128, 16)
+    W = devio.weights_to_device(synth.make_weights(w))
+    A = synth.make_activations(w.with_(seqlen=4))
+    ic = devio.to_device(A["init_conv_state"])
+    iss = devio.to_device(A["init_ssm_state"])
+    fs = torch.full((2, 128, 16), 7.0, device="cuda")
+    fc = torch.empty_like(ic)
+    d = devio.dims_of(w)
+    n = jmix.jm_mixer_fwd_workspace_size(d)
+    ws = devio.workspace(n)
+    x = torch.empty(16, dtype=torch.bfloat16, device="cuda")   # never read
+    y = torch.empty(16, dtype=torch.bfloat16, device="cuda")
+    jmix.jm_mixer_fwd(d, x, x, W, y, fs, ws, n, ic, iss, fc)
+    torch.cuda.synchronize()
+    assert torch.equal(fs, iss) and torch.equal(fc, ic)
+    jmix.jm_mixer_fwd(d, x, x, W, y, fs, ws, n, None, None, fc)
+    torch.cuda.synchronize()
+    assert (fs == 0).all() and (fc.float() == 0).all()
+    d0 = devio.dims_of(w.with_(batch=0, seqlen=5))
+    jmix.jm_mixer_fwd(d0, x, x, W, y, fs, ws, n)
+
+
+def test_gpu_split_invariance():
+    """Running the first L1 tokens, then the rest from the returned states, gives
+    the same y and final state as one call (conv history spans the cut)."""
+    import torch
+    from mamba_selective_scan_jamba_b200 import devio
+    w = small(2, 260, 256, 32)
+    W = synth.make_weights(w)
+    A = synth.make_activations(w)
+    y, fs, fc = gpu_fwd(w, W, A)
+    L1 = 131
+    w1, w2 = w.with_(seqlen=L1), w.with_(seqlen=w.seqlen - L1)
+    A1 = dict(A, x=A["x"][:, :L1].copy(), z=A["z"][:, :L1].copy())
+    y1, fs1, fc1 = gpu_fwd(w1, W, A1)
+    A2 = dict(x=A["x"][:, L1:].copy(), z=A["z"][:, L1:].copy(), init_conv_state=fc1,
+              init_ssm_state=fs1)
+    y2, fs2, fc2 = gpu_fwd(w2, W, A2)
+    assert max_scaled_err(f64(np.concatenate([y1, y2], 1)), f64(y)) <= 1e-2
+    assert max_scaled_err(fs2, fs) <= 1e-5
+    np.testing.assert_array_equal(fc2, fc)
+
+
+def test_host_entry_point_matches_device_call():
+    import torch
+    from mamba_selective_scan_jamba_b200 import devio, jmix
+    w = small(2, 96, 256, 32, extra=False)
+    W = synth.make_weights(w)
+    A = synth.make_activations(w)
+    y_ref, fs_ref, _ = gpu_fwd(w, W, A, use_init=False, want_conv=False)
+    Wd = devio.weights_to_device(W)
+    xh, zh = devio.to_pinned(A["x"]), devio.to_pinned(A["z"])
+    yh = torch.empty_like(xh).pin_memory()
+    fsh = torch.empty((2, 256, 16), dtype=torch.float32).pin_memory()
+    xd, zd = torch.empty_like(xh, device="cuda"), torch.empty_like(zh, device="cuda")
+    yd = torch.empty_like(xd)
+    fsd = torch.empty((2, 256, 16), dtype=torch.float32, device="cuda")
+    d = devio.dims_of(w)
+    n = jmix.jm_mixer_fwd_workspace_size(d)
+    ws = devio.workspace(n)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        jmix.jm_mixer_fwd_host(d, xh, zh, yh, fsh, xd, zd, yd, fsd, Wd, ws, n, stream=s)
+    s.synchronize()
+    np.testing.assert_array_equal(devio.to_host(yh), y_ref)
+    np.testing.assert_array_equal(fsh.numpy(), fs_ref)
+
+
+def run_decode(w: synth.Workload, steps: int, channels=None, threads=0):
+    """GPU decode steps vs the oracle; returns errors."""
+    import torch
+    from mamba_selective_scan_jamba_b200 import devio, jmix
+    W = synth.make_weights(w)
+    S = synth.make_decode_state(w)
+    Wd = devio.weights_to_device(W)
+    cs = devio.to_device(S["conv_state"])
+    ss = devio.to_device(S["ssm_state"])
+    d = devio.dims_of(w)
+    n = jmix.jm_mixer_step_workspace_size(d)
+    ws = devio.workspace(n)
+    ch = np.arange(w.d_inner) if channels is None else np.asarray(channels)
+    m_exact = oracle.dims_of(w, seqlen=1, threads=threads)
+    m_mirror = oracle.dims_of(w, seqlen=1, mirror=(w.io == "bf16"), threads=threads)
+    cs_ref = f64(S["conv_state"])                 # exact: conv states are copies of inputs
+    ss_ex = f64(S["ssm_state"])
+    ss_mi = ss_ex.copy()
+    worst = {"y": 0.0, "state": 0.0}
+    tol = TOL[w.io]
+    for t in range(steps):
+        tok = synth.make_decode_token(w, t)
+        xt, zt = devio.to_device(tok["x_t"]), devio.to_device(tok["z_t"])
+        yt = torch.empty_like(xt)
+        jmix.jm_mixer_step(d, xt, zt, cs, ss, Wd, yt, ws, n)
+        y_gpu = f64(devio.to_host(yt))[:, ch]
+        x3, z3 = tok["x_t"][:, None, :], tok["z_t"][:, None, :]
+        y_ex, fs_ex, _ = oracle.mixer_fwd(m_exact, x3, z3, W, cs_ref, ss_ex, channels=ch)
+        if w.io == "bf16":
+            _, fs_mi, _ = oracle.mixer_fwd(m_mirror, x3, z3, W, cs_ref, ss_mi, channels=ch)
+            ss_mi[:, ch] = fs_mi
+        else:
+            ss_mi[:, ch] = fs_ex
+        ss_ex[:, ch] = fs_ex
+        cs_ref = np.concatenate([cs_ref[:, :, 1:], f64(tok["x_t"])[:, :, None]], axis=2)
+        worst["y"] = max(worst["y"], max_scaled_err(y_gpu, y_ex[:, 0]))
+    assert jmix.jm_poll_error(ws) == jmix.JM_OK
+    torch.cuda.synchronize()
+    worst["state"] = max_scaled_err(devio.to_host(ss)[:, ch], ss_mi[:, ch])
+    np.testing.assert_array_equal(f64(devio.to_host(cs)), cs_ref)
+    assert worst["y"] <= tol["y"], worst
+    assert worst["state"] <= tol["state"], worst
+    return worst
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_decode_small(io):
+    w = synth.Workload("dec", 5, 1, 256, 16, io, seed=9, extra=True, steps=8)
+    run_decode(w, 8)
+
+
+def test_decode_step_matches_forward():
+    """Steps from zero states equal one forward call (same kernels' contract)."""
+    import torch
+    from mamba_selective_scan_jamba_b200 import devio, jmix
+    w = small(3, 6, 256, 32, extra=True)
+    W = synth.make_weights(w)
+    A = synth.make_activations(w)
+    y, fs, fc = gpu_fwd(w, W, A)
+    Wd = devio.weights_to_device(W)
+    cs = devio.to_device(A["init_conv_state"])
+    ss = devio.to_device(A["init_ssm_state"])
+    d = devio.dims_of(w, seqlen=1)
+    n = jmix.jm_mixer_step_workspace_size(d)
+    ws = devio.workspace(n)
+    for t in range(w.seqlen):
+        xt = devio.to_device(np.ascontiguousarray(A["x"][:, t]))
+        zt = devio.to_device(np.ascontiguousarray(A["z"][:, t]))
+        yt = torch.empty_like(xt)
+        jmix.jm_mixer_step(d, xt, zt, cs, ss, Wd, yt, ws, n)
+        assert max_scaled_err(f64(devio.to_host(yt)), f64(y[:, t])) <= 1e-2
+    assert max_scaled_err(devio.to_host(ss), fs) <= 1e-5
+    np.testing.assert_array_equal(devio.to_host(cs), fc)
+
+
+# ------------------------------------------------------------- full sizes
+FULL_CH = [0, 1, 127, 128, 1000, 4095, 4096, 5555, 8064, 8191]
+
+
+@pytest.mark.slow
+def test_full_jamba_b1_l4096():
+    check_fwd(synth.WORKLOADS["jamba_b1_l4096"], channels=FULL_CH)
+
+
+@pytest.mark.slow
+def test_full_jamba_b8_l4096():
+    check_fwd(synth.WORKLOADS["jamba_b8_l4096"], channels=FULL_CH[::3])
+
+
+@pytest.mark.slow
+def test_full_jamba_b1_l262144():
+    check_fwd(synth.WORKLOADS["jamba_b1_l262144"], channels=[0, 3333, 8191])
+
+
+@pytest.mark.slow
+def test_full_decode_b256_64_steps():
+    run_decode(synth.WORKLOADS["jamba_decode_b256"], 64, channels=FULL_CH)
