@@ -166,9 +166,10 @@ def reference_arm(args, w, rank, world):
     from mamba_selective_scan_jamba_b200 import synth
     cores = os.cpu_count() or 1
     W = synth.make_weights(w)
-    # calibrate a per-step sample of about 2 s
+    # per-step sample sized so that warm-up + timed steps take about two minutes
+    per_step_s = min(2.0, 120.0 / max(1, args.steps + args.warmup))
     rate, _, _ = oracle_rate(w, 1.0, cores)
-    L = int(max(16, min(w.seqlen, rate * 2.0)))
+    L = int(max(8, min(w.seqlen, rate * per_step_s)))
     A = synth.make_activations(w.with_(batch=1, seqlen=L))
     m = oracle.dims_of(w, batch=1, seqlen=L, threads=cores)
     for _ in range(args.warmup):

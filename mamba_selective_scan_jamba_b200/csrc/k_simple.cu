@@ -3,7 +3,8 @@
 //
 // It is the only path for float32 io (TF32 tensor cores cannot meet a 1e-4
 // tolerance) and serves any io dtype.  In bf16 mode it rounds at the same two
-// points as the tensor-core path: u after the SiLU and dt_n before dt_proj.
+// points as the tensor-core path, which stores them as fp16: u after the SiLU
+// and dt_n before dt_proj.
 //
 // Steps (TransformerLens "Jamba" adapter page for the pipeline; aifetchly
 // "Jamba Guide", "Inside the Mamba State-Space Layers", for the scan):
@@ -13,6 +14,8 @@
 //   k_gemm_nt       delta = softplus(dt_n . dtproj_w^T + dt_bias)   (dt_proj)
 //   k_scan_simple   h, y (one thread per (sequence, channel), 16 states)
 //   k_final_conv    final conv state
+#include <cuda_fp16.h>
+
 #include "jmix_internal.cuh"
 
 namespace jmix {
@@ -22,9 +25,7 @@ __device__ __forceinline__ float ld(const float* p) { return *p; }
 __device__ __forceinline__ float ld(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 __device__ __forceinline__ void st(float* p, float v) { *p = v; }
 __device__ __forceinline__ void st(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
-__device__ __forceinline__ float to_bf16_value(float v) {
-  return __bfloat162float(__float2bfloat16_rn(v));
-}
+__device__ __forceinline__ float to_fp16_value(float v) { return __half2float(__float2half_rn(v)); }
 
 __device__ __forceinline__ float silu_precise(float v) { return v / (1.0f + expf(-v)); }
 
@@ -52,7 +53,7 @@ __global__ void k_conv_silu(const T* __restrict__ x, const T* __restrict__ conv_
     acc = fmaf(ld(conv_w + c * kConv + k), xv, acc);
   }
   float v = silu_precise(acc);
-  u[i] = round_u ? to_bf16_value(v) : v;
+  u[i] = round_u ? to_fp16_value(v) : v;
 }
 
 // out[m, n] = sum_k A[m, k] * W[n, k]   (A float32 [M, K], W io dtype [N, K])
@@ -114,7 +115,7 @@ __global__ void k_norms(const float* __restrict__ p, const T* __restrict__ wdt,
   const float inv_dt = 1.0f / sqrtf(ss / (float)R + eps);
   for (int j = lane; j < R; j += 32) {
     float v = row[j] * inv_dt * ld(wdt + j);
-    dtn[g * R + j] = round_dt ? to_bf16_value(v) : v;
+    dtn[g * R + j] = round_dt ? to_fp16_value(v) : v;
   }
   // lanes 0..15 -> B, 16..31 -> C
   const int n = lane & 15;

@@ -60,6 +60,8 @@ def _L():
         lib = ctypes.CDLL(LIB)
         lib.orc_round_bf16.restype = ctypes.c_double
         lib.orc_round_bf16.argtypes = [ctypes.c_double]
+        lib.orc_round_fp16.restype = ctypes.c_double
+        lib.orc_round_fp16.argtypes = [ctypes.c_double]
         lib.orc_softplus1.restype = ctypes.c_double
         lib.orc_softplus1.argtypes = [ctypes.c_double]
         _lib = lib
@@ -97,6 +99,10 @@ _WNAMES = ("conv_w", "conv_b", "xproj_w", "dt_norm_w", "b_norm_w", "c_norm_w", "
 
 def round_bf16(v: float) -> float:
     return _L().orc_round_bf16(float(v))
+
+
+def round_fp16(v: float) -> float:
+    return _L().orc_round_fp16(float(v))
 
 
 def softplus1(v: float) -> float:

@@ -30,11 +30,12 @@
 //   6. gate: y = ys * z / (1 + exp(-z)).  Final SSM state = h after the last
 //      token; final conv state = the last K-1 conv inputs, oldest first.
 //
-// Mirror mode (mirror_bf16 = 1) rounds at the two points where the bf16 CUDA
-// path stores a value in bf16: u after the SiLU (it feeds both x_proj and the
-// scan) and dt_n (the dt_proj operand).  The rounding is taken in the kernel's
-// precision: to float32 (nearest even), then to bf16 (nearest even).
-// Nothing else is rounded.
+// Mirror mode (mirror_bf16 = 1) rounds at the two points where the bf16-io
+// CUDA path stores an intermediate: u after the SiLU (it feeds both x_proj and
+// the scan) and dt_n (the dt_proj operand).  Both are stored as IEEE fp16, the
+// tensor-core operand type of that path.  The rounding is taken in the kernel's
+// precision: to float32 (nearest even), then to fp16 (nearest even).  Nothing
+// else is rounded.
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
@@ -79,6 +80,13 @@ double round_bf16(double v) {
   return (double)f;
 }
 
+// float32 (nearest even), then IEEE binary16 (nearest even, subnormals kept).
+double round_fp16(double v) {
+  float f = (float)v;
+  _Float16 h = (_Float16)f;
+  return (double)(float)h;
+}
+
 double silu(double v) { return v / (1.0 + std::exp(-v)); }
 
 // Exact value of element i of a stored input: kind 0 = double, 1 = bf16 bit
@@ -112,6 +120,7 @@ typedef struct {
 } orc_dims;
 
 double orc_round_bf16(double v) { return round_bf16(v); }
+double orc_round_fp16(double v) { return round_fp16(v); }
 double orc_softplus1(double v) { return softplus(v); }
 
 // Step 1 for one sequence: xc [L,d] (pre-activation) from x [L,d].
@@ -196,7 +205,7 @@ static void front_end_rows(const orc_dims* m, Stored x, const double* conv_w,
         acc += conv_w[c * K + k] * xv;
       }
       double uv = silu(acc);
-      ur[c] = m->mirror_bf16 ? round_bf16(uv) : uv;
+      ur[c] = m->mirror_bf16 ? round_fp16(uv) : uv;
     }
     // p[j] = sum_c W_x[j,c] u[c], summed in ascending c for every j
     std::fill(p.begin(), p.end(), 0.0);
@@ -209,7 +218,7 @@ static void front_end_rows(const orc_dims* m, Stored x, const double* conv_w,
     orc_rmsnorm(1, N, N, p.data() + R, bn_w, m->eps, Bn + t * N);
     orc_rmsnorm(1, N, N, p.data() + R + N, cn_w, m->eps, Cn + t * N);
     if (m->mirror_bf16)
-      for (int64_t r = 0; r < R; ++r) dtn[t * R + r] = round_bf16(dtn[t * R + r]);
+      for (int64_t r = 0; r < R; ++r) dtn[t * R + r] = round_fp16(dtn[t * R + r]);
   }
 }
 

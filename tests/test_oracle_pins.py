@@ -189,6 +189,15 @@ def test_softplus_identities():
     assert oracle.softplus1(800.0) == 800.0
 
 
+def test_round_fp16():
+    assert oracle.round_fp16(1.0) == 1.0
+    assert oracle.round_fp16(1.0 + 2 ** -11) == 1.0                   # tie -> even
+    assert oracle.round_fp16(1.0 + 3 * 2 ** -11) == 1.0 + 2 ** -9     # tie -> even (up)
+    assert oracle.round_fp16(2 ** -24) == 2 ** -24                    # smallest subnormal kept
+    assert oracle.round_fp16(65504.0) == 65504.0
+    np.testing.assert_equal(np.float16(0.1).astype(np.float64), oracle.round_fp16(0.1))
+
+
 def test_round_bf16():
     assert oracle.round_bf16(1.0) == 1.0
     assert oracle.round_bf16(1.0 + 2 ** -8) == 1.0            # tie -> even
@@ -300,8 +309,8 @@ def test_mixer_gate_skip_and_split_order():
 
 
 def test_mirror_rounding_is_small():
-    """Mirror mode rounds u and dt_n to bf16; on bf16 inputs it must stay within a
-    few bf16 ulps of the exact run, and equal it when the rounding is a no-op."""
+    """Mirror mode rounds u and dt_n to fp16; on bf16 inputs it must stay well
+    inside the bf16-io output tolerance of the exact run."""
     w = tiny(io="bf16")
     W = synth.make_weights(w)
     A = synth.make_activations(w)
@@ -309,8 +318,8 @@ def test_mirror_rounding_is_small():
                                 A["init_ssm_state"])
     ym, fsm, _ = oracle.mixer_fwd(oracle.dims_of(w, mirror=True), A["x"], A["z"], W,
                                   A["init_conv_state"], A["init_ssm_state"])
-    assert np.abs(ym - y).max() < 2e-2 * max(1.0, np.abs(y).max())
-    assert 0 < np.abs(fsm - fs).max() < 1e-2
+    assert (np.abs(ym - y) / np.maximum(1.0, np.abs(y))).max() < 5e-3
+    assert 0 < np.abs(fsm - fs).max() < 2e-3
 
 
 def test_sampled_channels_match_full():
