@@ -1,8 +1,701 @@
-// bf16 path: placeholder that routes to the SIMT kernels until the
-// tensor-core kernels land.
+// The bf16-io path of the mixer core on sm_100a.
+//
+//   k_conv_silu16   u = SiLU(conv1d(x) + conv_b), stored as fp16; the same launch
+//                   converts xproj_w and dtproj_w from bf16 to fp16 (exact for
+//                   |w| >= 2^-14; fp16 subnormals below) for the tensor cores.
+//   k_xproj         p = u . xproj_w^T on tcgen05 (TMA -> SMEM -> MMA -> TMEM),
+//                   split over d_inner; partial tiles added into p (fp32).
+//   k_norms16       dt_n (fp16) and B_n, C_n (fp32) = RMSNorm(.) w.
+//   k_scan_fused    per (sequence, 128 channels): dt_proj on tcgen05 into TMEM,
+//                   softplus, the selective scan with fp32 state in registers,
+//                   the D skip, the SiLU(z) gate, the final SSM and conv states.
+//
+// Why fp16 operands: u and dt_n feed the two contractions; with 10 mantissa
+// bits their rounding moves y by <= ~3e-3 of max(1,|y|), against ~2e-2 for
+// bf16 operands, at the same tensor-core rate.
+//
+// Formulas: TransformerLens "Jamba" adapter page (mixer pipeline with the
+// dt/B/C RMSNorms); aifetchly "Jamba Guide", "Inside the Mamba State-Space
+// Layers" (exp(delta A) discretisation, delta B, h_t = Abar h_{t-1} + Bbar x_t,
+// y_t = C_t h_t) and "Hands-On Implementation" (A = -exp(A_log),
+// delta = softplus(dt_proj(.))).
+#include <cuda.h>
+#include <cuda_fp16.h>
+
 #include "jmix_internal.cuh"
+#include "sm100.cuh"
 
 namespace jmix {
-size_t fast_ws_bytes(const Problem& p) { return simple_ws_bytes(p); }
-cudaError_t run_fast(Problem& p) { return run_simple(p); }
+namespace {
+
+using namespace sm100;
+typedef __nv_bfloat16 bf16;
+
+constexpr int kConvG = 16;        // tokens per thread in k_conv_silu16
+constexpr int kXM = 128;          // x_proj tile: tokens
+constexpr int kXK = 64;           // x_proj tile: channels per k-chunk (one 128-B swizzle atom)
+constexpr int kXStages = 4;
+constexpr int kSQ = 16;           // scan: tokens per chunk
+constexpr int kSC = 128;          // scan: channels per CTA
+constexpr int kMaxSlabs = kMaxRank / 64;
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ float bf(bf16 v) { return __bfloat162float(v); }
+
+__device__ __forceinline__ void unpack8_bf16(const uint4& q, float (&o)[8]) {
+  const bf16* h = reinterpret_cast<const bf16*>(&q);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) o[i] = __bfloat162float(h[i]);
+}
+
+__device__ __forceinline__ float silu_acc(float v) {
+  // v * sigmoid(v) with an IEEE reciprocal: sigmoid -> 0 cleanly for v << 0
+  return v * __frcp_rn(1.0f + expf(-v));
+}
+
+__device__ __forceinline__ __half to_half_sat(float v) {
+  return __float2half_rn(fminf(fmaxf(v, -65504.0f), 65504.0f));
+}
+
+// ------------------------------------------------------------------ conv + SiLU
+// Thread = 8 consecutive channels x kConvG consecutive tokens of one sequence
+// (a sliding window of the last 3 inputs in registers).  Threads past the conv
+// range convert 8 weights each.
+__global__ void __launch_bounds__(256) k_conv_silu16(
+    const bf16* __restrict__ x, const bf16* __restrict__ conv_w, const bf16* __restrict__ conv_b,
+    const bf16* __restrict__ hist, int64_t B, int64_t L, int64_t d, __half* __restrict__ u,
+    int64_t n_conv, const bf16* __restrict__ wx, int64_t n_wx8, __half* __restrict__ wx16,
+    const bf16* __restrict__ wdt, int64_t n_wdt8, __half* __restrict__ wdt16) {
+  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (tid < n_conv) {
+    const int64_t ncg = d >> 3;
+    const int64_t cg = tid % ncg;
+    const int64_t rest = tid / ncg;
+    const int64_t nck = (L + kConvG - 1) / kConvG;
+    const int64_t ck = rest % nck, b = rest / nck;
+    const int64_t c0 = cg * 8, t0 = ck * kConvG;
+    float w[8][kConv], bias[8];
+    {
+      const uint4* wp = reinterpret_cast<const uint4*>(conv_w + c0 * kConv);
+      float tmp[32];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float o[8];
+        unpack8_bf16(__ldg(wp + q), o);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) tmp[q * 8 + i] = o[i];
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+#pragma unroll
+        for (int k = 0; k < kConv; ++k) w[j][k] = tmp[j * kConv + k];
+      unpack8_bf16(__ldg(reinterpret_cast<const uint4*>(conv_b + c0)), bias);
+    }
+    float win[kConv - 1][8];
+#pragma unroll
+    for (int k = 0; k < kConv - 1; ++k) {
+      const int64_t tau = t0 - (kConv - 1) + k;
+      if (tau >= 0) {
+        unpack8_bf16(__ldg(reinterpret_cast<const uint4*>(x + (b * L + tau) * d + c0)), win[k]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          win[k][j] = hist ? bf(hist[(b * d + c0 + j) * (kConv - 1) + (kConv - 1) + tau]) : 0.0f;
+      }
+    }
+    const int64_t t1 = t0 + kConvG < L ? t0 + kConvG : L;
+    for (int64_t t = t0; t < t1; ++t) {
+      float xt[8];
+      unpack8_bf16(__ldg(reinterpret_cast<const uint4*>(x + (b * L + t) * d + c0)), xt);
+      __align__(16) __half out[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float acc = bias[j];
+#pragma unroll
+        for (int k = 0; k < kConv - 1; ++k) acc = fmaf(w[j][k], win[k][j], acc);
+        acc = fmaf(w[j][kConv - 1], xt[j], acc);
+        out[j] = to_half_sat(silu_acc(acc));
+      }
+      *reinterpret_cast<uint4*>(u + (b * L + t) * d + c0) = *reinterpret_cast<uint4*>(out);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+#pragma unroll
+        for (int k = 0; k < kConv - 2; ++k) win[k][j] = win[k + 1][j];
+        win[kConv - 2][j] = xt[j];
+      }
+    }
+    return;
+  }
+  int64_t i = tid - n_conv;
+  const bf16* src;
+  __half* dst;
+  if (i < n_wx8) {
+    src = wx;
+    dst = wx16;
+  } else if ((i -= n_wx8) < n_wdt8) {
+    src = wdt;
+    dst = wdt16;
+  } else {
+    return;
+  }
+  float o[8];
+  unpack8_bf16(__ldg(reinterpret_cast<const uint4*>(src) + i), o);
+  __align__(16) __half h[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) h[j] = __float2half_rn(o[j]);
+  reinterpret_cast<uint4*>(dst)[i] = *reinterpret_cast<uint4*>(h);
+}
+
+// ------------------------------------------------------------------- x_proj
+struct XprojArgs {
+  int64_t T;
+  int P, Ntot, N1, N2;
+  int kchunks, ksplit;
+  uint32_t tmem_cols;
+  float* p;
+  ErrFlags* err;
+};
+
+constexpr int kXThreads = 192;  // warp 0 TMA, warp 1 MMA + TMEM, warps 2..5 epilogue
+
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
+  return (1u << 4)                                  // D format: f32
+         | (0u << 7) | (0u << 10)                   // A, B format: f16
+         | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__global__ void __launch_bounds__(kXThreads, 1)
+    k_xproj(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_w,
+            const XprojArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const int a_bytes = kXM * 128;
+  const int b_bytes = a.Ntot * 128;
+  const int stage_bytes = a_bytes + b_bytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kXStages * stage_bytes);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kXStages;
+  uint64_t* acc_full = bars + 2 * kXStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kXStages + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m_tile = blockIdx.x, split = blockIdx.y;
+  const int k_begin = (int)((int64_t)split * a.kchunks / a.ksplit);
+  const int k_end = (int)((int64_t)(split + 1) * a.kchunks / a.ksplit);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kXStages; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    mbar_init(smem_u32(acc_full), 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), a.tmem_cols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_u);
+    prefetch_tmap(&tm_w);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int kc = k_begin, i = 0; kc < k_end; ++kc, ++i) {
+        const int s = i % kXStages;
+        const uint32_t ph = (uint32_t)(i / kXStages) & 1u;
+        if (i >= kXStages && !mbar_wait(smem_u32(&empty[s]), ph ^ 1u, a.err, 11)) break;
+        uint8_t* As = smem + s * stage_bytes;
+        uint8_t* Bs = As + a_bytes;
+        const uint32_t fb = smem_u32(&full[s]);
+        mbar_arrive_expect_tx(fb, (uint32_t)stage_bytes);
+        tma_load_2d(smem_u32(As), &tm_u, fb, kc * kXK, m_tile * kXM);
+        tma_load_2d(smem_u32(Bs), &tm_w, fb, kc * kXK, 0);
+        if (a.N2) tma_load_2d(smem_u32(Bs + a.N1 * 128), &tm_w, fb, kc * kXK, a.N1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id1 = idesc_f16_f32(kXM, a.N1);
+      const uint32_t id2 = idesc_f16_f32(kXM, a.N2 ? a.N2 : 16);
+      for (int kc = k_begin, i = 0; kc < k_end; ++kc, ++i) {
+        const int s = i % kXStages;
+        const uint32_t ph = (uint32_t)(i / kXStages) & 1u;
+        if (!mbar_wait(smem_u32(&full[s]), ph, a.err, 12)) break;
+        tc_fence_after();
+        const uint32_t ab = smem_u32(smem + s * stage_bytes);
+        const uint32_t bb = ab + a_bytes;
+#pragma unroll
+        for (int kk = 0; kk < kXK / 16; ++kk) {
+          const uint64_t ad = sw128_kmajor_desc(ab + kk * 32);
+          const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+          umma_f16(tmem, ad, sw128_kmajor_desc(bb + kk * 32), id1, acc);
+          if (a.N2)
+            umma_f16(tmem + a.N1, ad, sw128_kmajor_desc(bb + a.N1 * 128 + kk * 32), id2, acc);
+        }
+        umma_commit(smem_u32(&empty[s]));
+      }
+      umma_commit(smem_u32(acc_full));
+    }
+  } else {
+    // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 = tile rows
+    const bool ok = mbar_wait(smem_u32(acc_full), 0, a.err, 13);
+    tc_fence_after();
+    const int lg = warp & 3;
+    const int64_t g = (int64_t)m_tile * kXM + lg * 32 + lane;
+    const bool row_ok = ok && g < a.T && k_end > k_begin;
+    for (int c0 = 0; c0 < a.Ntot; c0 += 16) {
+      uint32_t r[16];
+      tmem_ld16(tmem + ((uint32_t)(lg * 32) << 16) + (uint32_t)c0, r);
+      tmem_ld_wait();
+      if (row_ok) {
+#pragma unroll
+        for (int j = 0; j < 16; j += 4) {
+          const int col = c0 + j;
+          if (col < a.P)
+            atomicAdd(reinterpret_cast<float4*>(a.p + g * a.P + col),
+                      make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
+                                  __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3])));
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, a.tmem_cols);
+  }
+}
+
+// -------------------------------------------------------------------- norms
+template <typename W>
+__global__ void __launch_bounds__(256) k_norms16(const float* __restrict__ p,
+                                                const W* __restrict__ wdt,
+                                                const W* __restrict__ wb, const W* __restrict__ wc,
+                                                int64_t Tn, int R, float eps,
+                                                __half* __restrict__ dtn, float* __restrict__ bc) {
+  const int lane = threadIdx.x & 31;
+  const int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (g >= Tn) return;
+  const int P = R + 2 * kN;
+  const float* row = p + g * P;
+  float ss = 0.f;
+  for (int j = lane; j < R; j += 32) ss = fmaf(row[j], row[j], ss);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float inv = 1.0f / sqrtf(ss / (float)R + eps);
+  for (int j = lane; j < R; j += 32)
+    dtn[g * R + j] = __float2half_rn(row[j] * inv * (float)wdt[j]);
+  const float v = row[R + lane];
+  float s2 = v * v;
+#pragma unroll
+  for (int o = 8; o; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+  const float inv2 = 1.0f / sqrtf(s2 / (float)kN + eps);
+  const float wv = lane < 16 ? (float)wb[lane] : (float)wc[lane - 16];
+  bc[g * 2 * kN + lane] = v * inv2 * wv;
+}
+
+// ------------------------------------------------------- fused dt_proj + scan
+struct ScanArgs {
+  int64_t L, d, T;
+  int R, nslab;
+  const float* dt_bias;
+  const float* A_log;
+  const float* D;
+  const float* h0;
+  float* hT;
+  bf16* y;
+  const bf16* x;
+  const bf16* hist;
+  bf16* final_conv;
+  ErrFlags* err;
+};
+
+constexpr int kScanThreads = 160;  // warps 0..3: one channel per thread; warp 4: TMA + MMA
+constexpr int kWdtBytes = kMaxSlabs * kSC * 128;                  // 64 KB
+constexpr int kDtnStage = kMaxSlabs * kSQ * 128;                  // 8 KB
+constexpr int kUStage = kSQ * kSC * 2;                            // 4 KB
+constexpr int kBCStage = kSQ * 2 * kN * 4;                        // 2 KB
+constexpr int kStageBytes = kDtnStage + 2 * kUStage + kBCStage;   // 18 KB
+constexpr int kScanSmem = 1024 + kWdtBytes + 2 * kStageBytes + 256;
+
+__device__ __forceinline__ float softplus_acc(float v) {
+  return fmaxf(v, 0.0f) + log1pf(expf(-fabsf(v)));
+}
+
+__global__ void __launch_bounds__(kScanThreads, 2)
+    k_scan_fused(const __grid_constant__ CUtensorMap tm_wdt,
+                 const __grid_constant__ CUtensorMap tm_dtn,
+                 const __grid_constant__ CUtensorMap tm_bc, const __grid_constant__ CUtensorMap tm_u,
+                 const __grid_constant__ CUtensorMap tm_z, const ScanArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* wdt_s = smem;
+  uint8_t* stage0 = smem + kWdtBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stage0 + 2 * kStageBytes);
+  uint64_t* full = bars;          // [2] TMA landed
+  uint64_t* mma_done = bars + 2;  // [2] dt_proj accumulator ready
+  uint64_t* empty = bars + 4;     // [2] compute warps done with the stage
+  uint64_t* wfull = bars + 6;     // W_dt tile landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 7);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t c0 = (int64_t)blockIdx.x * kSC;
+  const int64_t b = blockIdx.y;
+  const int64_t g0 = b * a.L;
+  const int nch = (int)((a.L + kSQ - 1) / kSQ);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&mma_done[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 4);
+    }
+    mbar_init(smem_u32(wfull), 1);
+    fence_mbar_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(smem_u32(tmem_slot), 2 * kSQ);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto stage_ptr = [&](int s) { return stage0 + s * kStageBytes; };
+
+  if (warp == 4) {
+    if (lane == 0) {
+      prefetch_tmap(&tm_wdt);
+      prefetch_tmap(&tm_dtn);
+      prefetch_tmap(&tm_bc);
+      prefetch_tmap(&tm_u);
+      prefetch_tmap(&tm_z);
+      const uint32_t wb = smem_u32(wfull);
+      mbar_arrive_expect_tx(wb, (uint32_t)(a.nslab * kSC * 128));
+      for (int j = 0; j < a.nslab; ++j)
+        tma_load_2d(smem_u32(wdt_s + j * kSC * 128), &tm_wdt, wb, j * 64, (int32_t)c0);
+      const uint32_t stage_tx = (uint32_t)(a.nslab * kSQ * 128 + 2 * kUStage + kBCStage);
+      auto issue_tma = [&](int k) {
+        const int s = k & 1;
+        uint8_t* st = stage_ptr(s);
+        const uint32_t fb = smem_u32(&full[s]);
+        const int32_t row = (int32_t)(g0 + (int64_t)k * kSQ);
+        mbar_arrive_expect_tx(fb, stage_tx);
+        for (int j = 0; j < a.nslab; ++j)
+          tma_load_2d(smem_u32(st + j * kSQ * 128), &tm_dtn, fb, j * 64, row);
+        tma_load_2d(smem_u32(st + kDtnStage), &tm_u, fb, (int32_t)c0, row);
+        tma_load_2d(smem_u32(st + kDtnStage + kUStage), &tm_z, fb, (int32_t)c0, row);
+        tma_load_2d(smem_u32(st + kDtnStage + 2 * kUStage), &tm_bc, fb, 0, row);
+      };
+      const uint32_t idesc = idesc_f16_f32(kSC, kSQ);
+      bool ok = mbar_wait(wb, 0, a.err, 21);
+      auto issue_mma = [&](int k) -> bool {
+        const int s = k & 1;
+        if (!mbar_wait(smem_u32(&full[s]), (uint32_t)(k >> 1) & 1u, a.err, 22)) return false;
+        tc_fence_after();
+        const uint32_t wbase = smem_u32(wdt_s), dbase = smem_u32(stage_ptr(s));
+        for (int j = 0; j < a.nslab; ++j)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_f16(tmem + (uint32_t)(s * kSQ), sw128_kmajor_desc(wbase + j * kSC * 128 + kk * 32),
+                      sw128_kmajor_desc(dbase + j * kSQ * 128 + kk * 32), idesc,
+                      (j > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(smem_u32(&mma_done[s]));
+        return true;
+      };
+      if (ok) {
+        issue_tma(0);
+        if (nch > 1) issue_tma(1);
+        ok = issue_mma(0);
+      }
+      for (int k = 0; ok && k < nch; ++k) {
+        if (k + 1 < nch) {
+          if (k >= 1 && !mbar_wait(smem_u32(&empty[(k + 1) & 1]), (uint32_t)((k - 1) >> 1) & 1u,
+                                   a.err, 23))
+            break;
+          if (!issue_mma(k + 1)) break;
+        }
+        if (k + 2 < nch) {
+          if (!mbar_wait(smem_u32(&empty[k & 1]), (uint32_t)(k >> 1) & 1u, a.err, 24)) break;
+          issue_tma(k + 2);
+        }
+      }
+    }
+  } else {
+    // compute warps: thread = channel c0 + 32*warp + lane = TMEM lane
+    const int cl = warp * 32 + lane;
+    const int64_t c = c0 + cl;
+    const bool cok = c < a.d;
+    float A2[kN], h[kN];
+#pragma unroll
+    for (int n = 0; n < kN; ++n) {
+      A2[n] = cok ? -expf(a.A_log[c * kN + n]) * kLog2e : 0.0f;
+      h[n] = (cok && a.h0) ? a.h0[(b * a.d + c) * kN + n] : 0.0f;
+    }
+    const float bias = cok ? a.dt_bias[c] : 0.0f;
+    const float Dc = cok ? a.D[c] : 0.0f;
+    bf16* yrow = a.y + g0 * a.d + c;
+    for (int k = 0; k < nch; ++k) {
+      const int s = k & 1;
+      const uint32_t ph = (uint32_t)(k >> 1) & 1u;
+      if (!mbar_wait(smem_u32(&mma_done[s]), ph, a.err, 25)) break;
+      if (!mbar_wait(smem_u32(&full[s]), ph, a.err, 26)) break;
+      tc_fence_after();
+      uint32_t r[16];
+      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(s * kSQ), r);
+      tmem_ld_wait();
+      const uint8_t* st = stage_ptr(s);
+      const __half* us = reinterpret_cast<const __half*>(st + kDtnStage);
+      const bf16* zs = reinterpret_cast<const bf16*>(st + kDtnStage + kUStage);
+      const float4* bcs = reinterpret_cast<const float4*>(st + kDtnStage + 2 * kUStage);
+      const int64_t tbase = (int64_t)k * kSQ;
+      const int nt = (int)((a.L - tbase) < kSQ ? (a.L - tbase) : kSQ);
+#pragma unroll
+      for (int t = 0; t < kSQ; ++t) {
+        if (t >= nt) break;
+        const float dl = softplus_acc(__uint_as_float(r[t]) + bias);
+        const float uv = __half2float(us[t * kSC + cl]);
+        const float zv = bf(zs[t * kSC + cl]);
+        const float du = dl * uv;
+        float acc = 0.0f;
+#pragma unroll
+        for (int q = 0; q < kN / 4; ++q) {
+          const float4 Bq = bcs[t * 8 + q];
+          const float4 Cq = bcs[t * 8 + 4 + q];
+          const float bq[4] = {Bq.x, Bq.y, Bq.z, Bq.w};
+          const float cq[4] = {Cq.x, Cq.y, Cq.z, Cq.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int n = q * 4 + i;
+            const float da = ex2_approx(dl * A2[n]);
+            h[n] = fmaf(da, h[n], du * bq[i]);
+            acc = fmaf(cq[i], h[n], acc);
+          }
+        }
+        const float ys = fmaf(Dc, uv, acc);
+        if (cok) yrow[(tbase + t) * a.d] = __float2bfloat16_rn(ys * silu_acc(zv));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
+    }
+    if (cok) {
+#pragma unroll
+      for (int n = 0; n < kN; ++n) a.hT[(b * a.d + c) * kN + n] = h[n];
+      if (a.final_conv) {
+        bf16 v[kConv - 1];
+#pragma unroll
+        for (int k = 0; k < kConv - 1; ++k) {
+          const int64_t tau = a.L - (kConv - 1) + k;
+          if (tau >= 0)
+            v[k] = a.x[(g0 + tau) * a.d + c];
+          else
+            v[k] = a.hist ? a.hist[(b * a.d + c) * (kConv - 1) + (kConv - 1) + tau]
+                          : __float2bfloat16_rn(0.0f);
+        }
+#pragma unroll
+        for (int k = 0; k < kConv - 1; ++k) a.final_conv[(b * a.d + c) * (kConv - 1) + k] = v[k];
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 2 * kSQ);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D tensor map of a row-major [rows, cols] matrix, box [box_rows, box_cols].
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, size_t esize, const void* base,
+              uint64_t rows, uint64_t cols, uint32_t box_cols, uint32_t box_rows, bool swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * esize};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE,
+            swz ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct FastWs {
+  char* hdr;
+  float* p;
+  __half* u;
+  __half* dtn;
+  float* bc;
+  __half* wx;
+  __half* wdt;
+  size_t bytes;
+  size_t zero_bytes;  // header + p, cleared each call
+};
+
+FastWs fast_layout(const Problem& pr, char* base) {
+  FastWs w{};
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    size_t o = off;
+    off = align256(off + n);
+    return base ? base + o : nullptr;
+  };
+  const size_t T = (size_t)pr.T, d = (size_t)pr.d, P = (size_t)pr.P, R = (size_t)pr.R;
+  w.hdr = take(sizeof(ErrFlags));
+  w.p = reinterpret_cast<float*>(take(T * P * 4));
+  w.zero_bytes = off;
+  w.u = reinterpret_cast<__half*>(take(T * d * 2));
+  w.dtn = reinterpret_cast<__half*>(take(T * R * 2));
+  w.bc = reinterpret_cast<float*>(take(T * 2 * kN * 4));
+  w.wx = reinterpret_cast<__half*>(take(P * d * 2));
+  w.wdt = reinterpret_cast<__half*>(take(d * R * 2));
+  w.bytes = off;
+  return w;
+}
+
+int g_num_sms = 0;
+
+int num_sms() {
+  if (!g_num_sms) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (g_num_sms <= 0) g_num_sms = 148;
+  }
+  return g_num_sms;
+}
+
+cudaError_t run_fast_fwd(Problem& p) {
+  FastWs w = fast_layout(p, p.ws);
+  cudaStream_t s = p.stream;
+  ErrFlags* err = reinterpret_cast<ErrFlags*>(w.hdr);
+  cudaError_t e = cudaMemsetAsync(p.ws, 0, w.zero_bytes, s);
+  if (e != cudaSuccess) return e;
+  launches_begin(p);
+
+  // 1. conv + SiLU -> u (fp16); weights -> fp16
+  {
+    const int64_t n_conv = (p.d / 8) * ((p.L + kConvG - 1) / kConvG) * p.B;
+    const int64_t n_wx8 = (int64_t)p.P * p.d / 8, n_wdt8 = p.d * p.R / 8;
+    const int64_t total = n_conv + n_wx8 + n_wdt8;
+    k_conv_silu16<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
+        (const bf16*)p.x, (const bf16*)p.conv_w, (const bf16*)p.conv_b, (const bf16*)p.init_conv,
+        p.B, p.L, p.d, w.u, n_conv, (const bf16*)p.xproj_w, n_wx8, w.wx,
+        (const bf16*)p.dtproj_w, n_wdt8, w.wdt);
+    launched(p, "k_conv_silu16");
+  }
+  // 2. x_proj on tcgen05
+  {
+    CUtensorMap tu, tw;
+    XprojArgs xa;
+    xa.T = p.T;
+    xa.P = (int)p.P;
+    // one MMA of N <= 256, or two equal halves (the second W box then has the
+    // same row count as the first, so both fill exactly their part of the stage)
+    if (p.P <= 256) {
+      xa.N1 = (int)((p.P + 15) / 16 * 16);
+      xa.N2 = 0;
+    } else {
+      xa.N1 = (int)(((p.P + 1) / 2 + 15) / 16 * 16);
+      xa.N2 = xa.N1;
+    }
+    xa.Ntot = xa.N1 + xa.N2;
+    xa.kchunks = (int)((p.d + kXK - 1) / kXK);
+    const int64_t mtiles = (p.T + kXM - 1) / kXM;
+    int64_t ks = (2 * num_sms() + mtiles - 1) / mtiles;
+    if (ks < 1) ks = 1;
+    if (ks > xa.kchunks) ks = xa.kchunks;
+    xa.ksplit = (int)ks;
+    xa.tmem_cols = xa.Ntot <= 32 ? 32 : xa.Ntot <= 64 ? 64 : xa.Ntot <= 128 ? 128
+                   : xa.Ntot <= 256 ? 256 : 512;
+    xa.p = w.p;
+    xa.err = err;
+    if (!make_map(&tu, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w.u, p.T, p.d, kXK, kXM, true) ||
+        !make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w.wx, p.P, p.d, kXK, xa.N1, true))
+      return cudaErrorInvalidValue;
+    const int smem = 1024 + kXStages * (kXM * 128 + xa.Ntot * 128) + 256;
+    cudaFuncSetAttribute(k_xproj, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    k_xproj<<<dim3((unsigned)mtiles, (unsigned)xa.ksplit), kXThreads, smem, s>>>(tu, tw, xa);
+    launched(p, "k_xproj");
+  }
+  // 3. RMSNorms
+  k_norms16<bf16><<<(unsigned)((p.T + 7) / 8), 256, 0, s>>>(
+      w.p, (const bf16*)p.dtn_w, (const bf16*)p.bn_w, (const bf16*)p.cn_w, p.T, (int)p.R, p.eps,
+      w.dtn, w.bc);
+  launched(p, "k_norms16");
+  // 4. dt_proj + scan + gate
+  {
+    CUtensorMap twdt, tdtn, tbc, tuu, tz;
+    if (!make_map(&twdt, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w.wdt, p.d, p.R, 64, kSC, true) ||
+        !make_map(&tdtn, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w.dtn, p.T, p.R, 64, kSQ, true) ||
+        !make_map(&tbc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, w.bc, p.T, 2 * kN, 2 * kN, kSQ,
+                  false) ||
+        !make_map(&tuu, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w.u, p.T, p.d, kSC, kSQ, false) ||
+        !make_map(&tz, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.z, p.T, p.d, kSC, kSQ, false))
+      return cudaErrorInvalidValue;
+    ScanArgs sa;
+    sa.L = p.L;
+    sa.d = p.d;
+    sa.T = p.T;
+    sa.R = (int)p.R;
+    sa.nslab = (int)((p.R + 63) / 64);
+    sa.dt_bias = p.dt_bias;
+    sa.A_log = p.A_log;
+    sa.D = p.D;
+    sa.h0 = p.init_ssm;
+    sa.hT = p.final_state;
+    sa.y = (bf16*)p.y;
+    sa.x = (const bf16*)p.x;
+    sa.hist = (const bf16*)p.init_conv;
+    sa.final_conv = (bf16*)p.final_conv;
+    sa.err = err;
+    cudaFuncSetAttribute(k_scan_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, kScanSmem);
+    k_scan_fused<<<dim3((unsigned)((p.d + kSC - 1) / kSC), (unsigned)p.B), kScanThreads, kScanSmem,
+                   s>>>(twdt, tdtn, tbc, tuu, tz, sa);
+    launched(p, "k_scan_fused");
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t fast_ws_bytes(const Problem& p) {
+  return p.decode ? simple_ws_bytes(p) : fast_layout(p, nullptr).bytes;
+}
+
+cudaError_t run_fast(Problem& p) {
+  if (p.decode) return run_simple(p);
+  return run_fast_fwd(p);
+}
+
 }  // namespace jmix

@@ -109,8 +109,9 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem, M x K, K-major] * B[smem, N x K, K-major]^T, bf16 in, fp32 acc.
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+// D[tmem] (+)= A[smem, M x K, K-major] * B[smem, N x K, K-major]^T with 16-bit
+// inputs (kind::f16: fp16 or bf16, as the instruction descriptor says), fp32 acc.
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                           uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
