@@ -117,6 +117,34 @@ jm_status jm_mixer_step(const jm_dims* dims, const void* x_t, const void* z_t, v
                         const float* A_log, const float* D, void* y_t, void* workspace,
                         size_t ws_bytes, jm_stream_t stream);
 
+/* jm_mixer_step without a caller workspace, for callers that cannot allocate
+ * device memory: code inside CUDA stream capture (where cudaMalloc is not
+ * allowed), serving engines that hand all device memory to their own caches
+ * and give plug-ins no allocator, or host code that must stay off the
+ * allocator.  The paper has no counterpart to this entry point.
+ *
+ * Arguments and results are those of jm_mixer_step without workspace and
+ * ws_bytes.  The scratch is a static 32 MiB device array inside libjmix, held
+ * by every GPU that loads the library until the process exits; a step at
+ * Jamba v0.1 mixer shapes (d_inner 8192, dt_rank 256) needs about 17 MiB for
+ * 256 sequences.  A step that needs more returns JM_ERR_UNSUPPORTED with a
+ * message and launches nothing.  The function itself allocates nothing.
+ *
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  All calls share the one array, and each call clears what it needs
+ * cleared, so the previous call's contents never leak into a result; but two
+ * calls whose kernels overlap on the GPU (different streams, or different
+ * host threads on one device) race on the array and must be serialised by the
+ * caller.  jm_poll_error does not apply (there is no caller workspace); launch
+ * errors are returned as JM_ERR_CUDA. */
+jm_status jm_mixer_step_noalloc(const jm_dims* dims, const void* x_t, const void* z_t,
+                                void* conv_state, float* ssm_state, const void* conv_w,
+                                const void* conv_b, const void* xproj_w, const void* dt_norm_w,
+                                const void* b_norm_w, const void* c_norm_w,
+                                const void* dtproj_w, const float* dt_bias, const float* A_log,
+                                const float* D, void* y_t, jm_stream_t stream);
+
 /* End-to-end forward from HOST buffers: copies x_host and z_host (pinned host
  * memory, [B, L, d] io dtype) into the caller's device buffers x_dev / z_dev,
  * runs jm_mixer_fwd, and copies y and the final SSM state back into y_host

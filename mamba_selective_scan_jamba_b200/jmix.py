@@ -24,7 +24,8 @@ WEIGHT_NAMES = ("conv_w", "conv_b", "xproj_w", "dt_norm_w", "b_norm_w", "c_norm_
 
 EXPORTED = ("jm_mixer_fwd_workspace_size", "jm_mixer_step_workspace_size", "jm_mixer_fwd",
             "jm_mixer_step", "jm_mixer_fwd_host", "jm_poll_error", "jm_last_error",
-            "jm_last_launch_count", "jm_last_kernel_name", "jm_set_kernel_events")
+            "jm_last_launch_count", "jm_last_kernel_name", "jm_set_kernel_events",
+            "jm_mixer_step_noalloc")
 
 
 class jm_dims(ctypes.Structure):
@@ -61,6 +62,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.jm_mixer_fwd.argtypes = [ctypes.POINTER(jm_dims)] + [_vp] * 18 + [ctypes.c_size_t, _vp]
     lib.jm_mixer_step.restype = ctypes.c_int
     lib.jm_mixer_step.argtypes = [ctypes.POINTER(jm_dims)] + [_vp] * 16 + [ctypes.c_size_t, _vp]
+    lib.jm_mixer_step_noalloc.restype = ctypes.c_int
+    lib.jm_mixer_step_noalloc.argtypes = [ctypes.POINTER(jm_dims)] + [_vp] * 15 + [_vp]
     lib.jm_mixer_fwd_host.restype = ctypes.c_int
     lib.jm_mixer_fwd_host.argtypes = [ctypes.POINTER(jm_dims)] + [_vp] * 19 + [ctypes.c_size_t, _vp]
     lib.jm_poll_error.restype = ctypes.c_int
@@ -133,6 +136,16 @@ def jm_mixer_step(d: jm_dims, x_t, z_t, conv_state, ssm_state, w: Mapping, y_t, 
     st = load().jm_mixer_step(ctypes.byref(d), _ptr(x_t), _ptr(z_t), _ptr(conv_state),
                               _ptr(ssm_state), *_weights(w), _ptr(y_t), _ptr(workspace), ws_bytes,
                               _stream(stream))
+    if check:
+        _check(st)
+    return st
+
+
+def jm_mixer_step_noalloc(d: jm_dims, x_t, z_t, conv_state, ssm_state, w: Mapping, y_t,
+                          stream=None, check: bool = True) -> int:
+    """jm_mixer_step with libjmix's static scratch instead of a caller workspace."""
+    st = load().jm_mixer_step_noalloc(ctypes.byref(d), _ptr(x_t), _ptr(z_t), _ptr(conv_state),
+                                      _ptr(ssm_state), *_weights(w), _ptr(y_t), _stream(stream))
     if check:
         _check(st)
     return st
