@@ -41,6 +41,8 @@ def parse():
     ap.add_argument("--workload", default="jamba_b8_l4096")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--seqlen", type=int, default=0,
+                    help="override the workload's sequence length (profiling captures)")
     return ap.parse_args()
 
 
@@ -202,6 +204,8 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     from mamba_selective_scan_jamba_b200 import synth
     base = synth.WORKLOADS[args.workload]
+    if args.seqlen:
+        base = base.with_(seqlen=args.seqlen, name=f"{base.name}_L{args.seqlen}")
     if args.impl == "reference":
         reference_arm(args, base, rank, world)
         return

@@ -1,18 +1,21 @@
 // The bf16-io path of the mixer core on sm_100a.
 //
-//   k_conv_silu16   u = SiLU(conv1d(x) + conv_b), stored as fp16; the same launch
-//                   converts xproj_w and dtproj_w from bf16 to fp16 (exact for
-//                   |w| >= 2^-14; fp16 subnormals below) for the tensor cores.
+//   k_conv_silu16   u = SiLU(conv1d(x) + conv_b) rounded to fp16, the x_proj
+//                   operand; the same launch converts xproj_w and dtproj_w from
+//                   bf16 to fp16 (exact for |w| >= 2^-14; fp16 subnormals below).
 //   k_xproj         p = u . xproj_w^T on tcgen05 (TMA -> SMEM -> MMA -> TMEM),
 //                   split over d_inner; partial tiles added into p (fp32).
-//   k_norms16       dt_n (fp16) and B_n, C_n (fp32) = RMSNorm(.) w.
+//   k_norms16       dt_n (fp16, the dt_proj operand), B_n and C_n (fp32) = RMSNorm(.) w.
 //   k_scan_fused    per (sequence, 128 channels): dt_proj on tcgen05 into TMEM,
-//                   softplus, the selective scan with fp32 state in registers,
-//                   the D skip, the SiLU(z) gate, the final SSM and conv states.
+//                   softplus, the conv + SiLU recomputed in fp32 from x, the
+//                   selective scan with fp32 state in registers, the D skip, the
+//                   SiLU(z) gate, the final SSM and conv states.
 //
-// Why fp16 operands: u and dt_n feed the two contractions; with 10 mantissa
-// bits their rounding moves y by <= ~3e-3 of max(1,|y|), against ~2e-2 for
-// bf16 operands, at the same tensor-core rate.
+// Precision: the quantised intermediates are the two tensor-core operands, u
+// for x_proj and dt_n for dt_proj, in fp16 (10 mantissa bits; their rounding
+// moves y by <= ~3e-3 of max(1,|y|), against ~2e-2 for bf16 at the same
+// tensor-core rate).  The scan's own u is float32, so no per-channel rounding
+// decision reaches the state directly.
 //
 // Formulas: TransformerLens "Jamba" adapter page (mixer pipeline with the
 // dt/B/C RMSNorms); aifetchly "Jamba Guide", "Inside the Mamba State-Space
@@ -23,6 +26,7 @@
 #include <cuda_fp16.h>
 
 #include "jmix_internal.cuh"
+#include "poly_consts.cuh"
 #include "sm100.cuh"
 
 namespace jmix {
@@ -31,7 +35,7 @@ namespace {
 using namespace sm100;
 typedef __nv_bfloat16 bf16;
 
-constexpr int kConvG = 16;        // tokens per thread in k_conv_silu16
+constexpr int kConvG = 4;         // tokens per thread in k_conv_silu16
 constexpr int kXM = 128;          // x_proj tile: tokens
 constexpr int kXK = 64;           // x_proj tile: channels per k-chunk (one 128-B swizzle atom)
 constexpr int kXStages = 4;
@@ -48,20 +52,24 @@ __device__ __forceinline__ void unpack8_bf16(const uint4& q, float (&o)[8]) {
   for (int i = 0; i < 8; ++i) o[i] = __bfloat162float(h[i]);
 }
 
-__device__ __forceinline__ float silu_acc(float v) {
-  // v * sigmoid(v) with an IEEE reciprocal: sigmoid -> 0 cleanly for v << 0
-  return v * __frcp_rn(1.0f + expf(-v));
-}
-
 __device__ __forceinline__ __half to_half_sat(float v) {
   return __float2half_rn(fminf(fmaxf(v, -65504.0f), 65504.0f));
 }
 
 // ------------------------------------------------------------------ conv + SiLU
-// Thread = 8 consecutive channels x kConvG consecutive tokens of one sequence
-// (a sliding window of the last 3 inputs in registers).  Threads past the conv
-// range convert 8 weights each.
-__global__ void __launch_bounds__(256) k_conv_silu16(
+// Thread = 8 consecutive channels x kConvG consecutive tokens of one sequence.
+// All of its x rows (the 3-token history and its tokens) are loaded before any
+// arithmetic, so each thread keeps ~11 16-byte loads in flight.  Threads past
+// the conv range convert 8 weights each.
+__device__ __forceinline__ float silu_u(float v) {
+  // v * sigmoid(v); relative error ~1e-6, far below the fp16 rounding of u
+  float e, r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-v * kLog2e));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.0f + e));
+  return v * r;
+}
+
+__global__ void __launch_bounds__(256, 2) k_conv_silu16(
     const bf16* __restrict__ x, const bf16* __restrict__ conv_w, const bf16* __restrict__ conv_b,
     const bf16* __restrict__ hist, int64_t B, int64_t L, int64_t d, __half* __restrict__ u,
     int64_t n_conv, const bf16* __restrict__ wx, int64_t n_wx8, __half* __restrict__ wx16,
@@ -74,54 +82,62 @@ __global__ void __launch_bounds__(256) k_conv_silu16(
     const int64_t nck = (L + kConvG - 1) / kConvG;
     const int64_t ck = rest % nck, b = rest / nck;
     const int64_t c0 = cg * 8, t0 = ck * kConvG;
+    const int nt = (int)((L - t0) < kConvG ? (L - t0) : kConvG);
+    constexpr int kW = kConv - 1;
+    // rows[0..2] = tokens t0-3..t0-1, rows[3..] = tokens t0..t0+nt-1
+    uint4 rows[kW + kConvG];
+#pragma unroll
+    for (int i = 0; i < kW + kConvG; ++i) {
+      const int64_t tau = t0 - kW + i;
+      if (tau >= 0 && i < kW + nt)
+        rows[i] = __ldg(reinterpret_cast<const uint4*>(x + (b * L + tau) * d + c0));
+      else
+        rows[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
     float w[8][kConv], bias[8];
     {
       const uint4* wp = reinterpret_cast<const uint4*>(conv_w + c0 * kConv);
-      float tmp[32];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         float o[8];
         unpack8_bf16(__ldg(wp + q), o);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) tmp[q * 8 + i] = o[i];
+        for (int i = 0; i < 8; ++i) w[(q * 8 + i) / kConv][(q * 8 + i) % kConv] = o[i];
       }
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-#pragma unroll
-        for (int k = 0; k < kConv; ++k) w[j][k] = tmp[j * kConv + k];
       unpack8_bf16(__ldg(reinterpret_cast<const uint4*>(conv_b + c0)), bias);
     }
-    float win[kConv - 1][8];
+    float win[kW][8];
 #pragma unroll
-    for (int k = 0; k < kConv - 1; ++k) {
-      const int64_t tau = t0 - (kConv - 1) + k;
+    for (int k = 0; k < kW; ++k) {
+      const int64_t tau = t0 - kW + k;
       if (tau >= 0) {
-        unpack8_bf16(__ldg(reinterpret_cast<const uint4*>(x + (b * L + tau) * d + c0)), win[k]);
+        unpack8_bf16(rows[k], win[k]);
       } else {
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-          win[k][j] = hist ? bf(hist[(b * d + c0 + j) * (kConv - 1) + (kConv - 1) + tau]) : 0.0f;
+          win[k][j] = hist ? bf(hist[(b * d + c0 + j) * kW + kW + tau]) : 0.0f;
       }
     }
-    const int64_t t1 = t0 + kConvG < L ? t0 + kConvG : L;
-    for (int64_t t = t0; t < t1; ++t) {
+#pragma unroll
+    for (int i = 0; i < kConvG; ++i) {
+      if (i >= nt) break;
       float xt[8];
-      unpack8_bf16(__ldg(reinterpret_cast<const uint4*>(x + (b * L + t) * d + c0)), xt);
+      unpack8_bf16(rows[kW + i], xt);
       __align__(16) __half out[8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         float acc = bias[j];
 #pragma unroll
-        for (int k = 0; k < kConv - 1; ++k) acc = fmaf(w[j][k], win[k][j], acc);
-        acc = fmaf(w[j][kConv - 1], xt[j], acc);
-        out[j] = to_half_sat(silu_acc(acc));
+        for (int k = 0; k < kW; ++k) acc = fmaf(w[j][k], win[k][j], acc);
+        acc = fmaf(w[j][kW], xt[j], acc);
+        out[j] = to_half_sat(silu_u(acc));
       }
-      *reinterpret_cast<uint4*>(u + (b * L + t) * d + c0) = *reinterpret_cast<uint4*>(out);
+      *reinterpret_cast<uint4*>(u + (b * L + t0 + i) * d + c0) = *reinterpret_cast<uint4*>(out);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
 #pragma unroll
-        for (int k = 0; k < kConv - 2; ++k) win[k][j] = win[k + 1][j];
-        win[kConv - 2][j] = xt[j];
+        for (int k = 0; k < kW - 1; ++k) win[k][j] = win[k + 1][j];
+        win[kW - 1][j] = xt[j];
       }
     }
     return;
@@ -275,12 +291,14 @@ __global__ void __launch_bounds__(kXThreads, 1)
 }
 
 // -------------------------------------------------------------------- norms
+// dt_n is written in fp16, the dt_proj operand type.
 template <typename W>
 __global__ void __launch_bounds__(256) k_norms16(const float* __restrict__ p,
                                                 const W* __restrict__ wdt,
                                                 const W* __restrict__ wb, const W* __restrict__ wc,
                                                 int64_t Tn, int R, float eps,
-                                                __half* __restrict__ dtn, float* __restrict__ bc) {
+                                                __half* __restrict__ dtn,
+                                                float* __restrict__ bc) {
   const int lane = threadIdx.x & 31;
   const int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (g >= Tn) return;
@@ -291,8 +309,7 @@ __global__ void __launch_bounds__(256) k_norms16(const float* __restrict__ p,
 #pragma unroll
   for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   const float inv = 1.0f / sqrtf(ss / (float)R + eps);
-  for (int j = lane; j < R; j += 32)
-    dtn[g * R + j] = __float2half_rn(row[j] * inv * (float)wdt[j]);
+  for (int j = lane; j < R; j += 32) dtn[g * R + j] = __float2half_rn(row[j] * inv * (float)wdt[j]);
   const float v = row[R + lane];
   float s2 = v * v;
 #pragma unroll
@@ -306,13 +323,16 @@ __global__ void __launch_bounds__(256) k_norms16(const float* __restrict__ p,
 struct ScanArgs {
   int64_t L, d, T;
   int R, nslab;
+  const bf16* x;
+  const bf16* z;
+  const bf16* conv_w;
+  const bf16* conv_b;
   const float* dt_bias;
   const float* A_log;
   const float* D;
   const float* h0;
   float* hT;
   bf16* y;
-  const bf16* x;
   const bf16* hist;
   bf16* final_conv;
   ErrFlags* err;
@@ -320,30 +340,90 @@ struct ScanArgs {
 
 constexpr int kScanThreads = 160;  // warps 0..3: one channel per thread; warp 4: TMA + MMA
 constexpr int kWdtBytes = kMaxSlabs * kSC * 128;                  // 64 KB
-constexpr int kDtnStage = kMaxSlabs * kSQ * 128;                  // 8 KB
-constexpr int kUStage = kSQ * kSC * 2;                            // 4 KB
+constexpr int kDtnStage = kMaxSlabs * kSQ * 128;                  // 8 KB (SW128 slabs)
+constexpr int kXStage = kSQ * kSC * 2;                            // 4 KB (x or z tile)
 constexpr int kBCStage = kSQ * 2 * kN * 4;                        // 2 KB
-constexpr int kStageBytes = kDtnStage + 2 * kUStage + kBCStage;   // 18 KB
+constexpr int kStageBytes = kDtnStage + 2 * kXStage + kBCStage;   // 18 KB
 constexpr int kScanSmem = 1024 + kWdtBytes + 2 * kStageBytes + 256;
 
-__device__ __forceinline__ float softplus_acc(float v) {
-  return fmaxf(v, 0.0f) + log1pf(expf(-fabsf(v)));
+// softplus(v) = max(v, 0) + log1p(exp(-|v|)): one MUFU ex2, log1p by a
+// degree-8 minimax polynomial on the FMA pipe (relative error < 3e-7).
+__device__ __forceinline__ float softplus_fast(float v) {
+  const float w = ex2_approx(-fabsf(v) * kLog2e);
+  float q = poly::L8;
+  q = fmaf(q, w, poly::L7);
+  q = fmaf(q, w, poly::L6);
+  q = fmaf(q, w, poly::L5);
+  q = fmaf(q, w, poly::L4);
+  q = fmaf(q, w, poly::L3);
+  q = fmaf(q, w, poly::L2);
+  q = fmaf(q, w, poly::L1);
+  q = fmaf(q, w, poly::L0);
+  return fmaf(w, q, fmaxf(v, 0.0f));
+}
+
+
+
+// 2^x for a pair of x <= 0 on the FMA pipe: exact base-2 range reduction
+// x = j + f (j = round(x), |f| <= 1/2, via the 1.5*2^23 rounding constant),
+// 2^f by the degree-6 minimax polynomial, and 2^j added into the exponent
+// field.  x is clamped at -126 (results below 2^-126 are flushed anyway).
+__device__ __forceinline__ float2 exp2_pair_fma(float2 x) {
+  const float kRound = 12582912.0f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -126.0f);
+  x.y = fmaxf(x.y, -126.0f);
+  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
+  const float2 j = __fadd2_rn(t, make_float2(-kRound, -kRound));
+  const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), x);
+  float2 p = make_float2(poly::E6, poly::E6);
+  p = __ffma2_rn(p, f, make_float2(poly::E5, poly::E5));
+  p = __ffma2_rn(p, f, make_float2(poly::E4, poly::E4));
+  p = __ffma2_rn(p, f, make_float2(poly::E3, poly::E3));
+  p = __ffma2_rn(p, f, make_float2(poly::E2, poly::E2));
+  p = __ffma2_rn(p, f, make_float2(poly::E1, poly::E1));
+  p = __ffma2_rn(p, f, make_float2(poly::E0, poly::E0));
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
+#ifndef JMIX_SW_PAIRS
+#define JMIX_SW_PAIRS 0
+#endif
+// State pairs (of 8) whose decay is computed on the FMA pipe instead of MUFU;
+// balances the two pipes (16 MUFU ex2 / clk / SM against 128 FMA / clk / SM).
+constexpr int kSwPairs = JMIX_SW_PAIRS;
+#ifndef JMIX_SCAN_G
+#define JMIX_SCAN_G 8
+#endif
+constexpr int kG = JMIX_SCAN_G;  // tokens per TMEM load / unrolled group in the scan loop
+
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// z * sigmoid(z) for the bf16 output gate, sigmoid(z) = (1 + tanh(z/2)) / 2:
+// one MUFU op, absolute error of sigmoid ~3e-4, far inside the output's tolerance.
+__device__ __forceinline__ float silu_gate(float z) {
+  const float hz = 0.5f * z;
+  return fmaf(hz, tanh_approx(hz), hz);
 }
 
 __global__ void __launch_bounds__(kScanThreads, 2)
     k_scan_fused(const __grid_constant__ CUtensorMap tm_wdt,
                  const __grid_constant__ CUtensorMap tm_dtn,
-                 const __grid_constant__ CUtensorMap tm_bc, const __grid_constant__ CUtensorMap tm_u,
+                 const __grid_constant__ CUtensorMap tm_bc, const __grid_constant__ CUtensorMap tm_x,
                  const __grid_constant__ CUtensorMap tm_z, const ScanArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* wdt_s = smem;
-  uint8_t* stage0 = smem + kWdtBytes;
+  uint8_t* wdt_s = smem;              // W_dt tile: nslab x [128 ch x 64] (SW128)
+  uint8_t* stage0 = smem + kWdtBytes;  // 2 x {dt_n (SW128), x tile, z tile, B/C rows}
   uint64_t* bars = reinterpret_cast<uint64_t*>(stage0 + 2 * kStageBytes);
-  uint64_t* full = bars;          // [2] TMA landed
+  uint64_t* full = bars;          // [2] stage landed
   uint64_t* mma_done = bars + 2;  // [2] dt_proj accumulator ready
-  uint64_t* empty = bars + 4;     // [2] compute warps done with the stage
+  uint64_t* empty = bars + 4;     // [2] compute warps done with the stage / accumulator
   uint64_t* wfull = bars + 6;     // W_dt tile landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 7);
 
@@ -378,14 +458,14 @@ __global__ void __launch_bounds__(kScanThreads, 2)
       prefetch_tmap(&tm_wdt);
       prefetch_tmap(&tm_dtn);
       prefetch_tmap(&tm_bc);
-      prefetch_tmap(&tm_u);
+      prefetch_tmap(&tm_x);
       prefetch_tmap(&tm_z);
       const uint32_t wb = smem_u32(wfull);
       mbar_arrive_expect_tx(wb, (uint32_t)(a.nslab * kSC * 128));
       for (int j = 0; j < a.nslab; ++j)
         tma_load_2d(smem_u32(wdt_s + j * kSC * 128), &tm_wdt, wb, j * 64, (int32_t)c0);
-      const uint32_t stage_tx = (uint32_t)(a.nslab * kSQ * 128 + 2 * kUStage + kBCStage);
-      auto issue_tma = [&](int k) {
+      const uint32_t stage_tx = (uint32_t)(a.nslab * kSQ * 128 + 2 * kXStage + kBCStage);
+      auto issue_stage = [&](int k) {
         const int s = k & 1;
         uint8_t* st = stage_ptr(s);
         const uint32_t fb = smem_u32(&full[s]);
@@ -393,57 +473,71 @@ __global__ void __launch_bounds__(kScanThreads, 2)
         mbar_arrive_expect_tx(fb, stage_tx);
         for (int j = 0; j < a.nslab; ++j)
           tma_load_2d(smem_u32(st + j * kSQ * 128), &tm_dtn, fb, j * 64, row);
-        tma_load_2d(smem_u32(st + kDtnStage), &tm_u, fb, (int32_t)c0, row);
-        tma_load_2d(smem_u32(st + kDtnStage + kUStage), &tm_z, fb, (int32_t)c0, row);
-        tma_load_2d(smem_u32(st + kDtnStage + 2 * kUStage), &tm_bc, fb, 0, row);
+        tma_load_2d(smem_u32(st + kDtnStage), &tm_x, fb, (int32_t)c0, row);
+        tma_load_2d(smem_u32(st + kDtnStage + kXStage), &tm_z, fb, (int32_t)c0, row);
+        tma_load_2d(smem_u32(st + kDtnStage + 2 * kXStage), &tm_bc, fb, 0, row);
       };
       const uint32_t idesc = idesc_f16_f32(kSC, kSQ);
-      bool ok = mbar_wait(wb, 0, a.err, 21);
       auto issue_mma = [&](int k) -> bool {
         const int s = k & 1;
         if (!mbar_wait(smem_u32(&full[s]), (uint32_t)(k >> 1) & 1u, a.err, 22)) return false;
         tc_fence_after();
-        const uint32_t wbase = smem_u32(wdt_s), dbase = smem_u32(stage_ptr(s));
+        const uint32_t wbase = smem_u32(wdt_s), db = smem_u32(stage_ptr(s));
+        const uint32_t d_tmem = tmem + (uint32_t)(s * kSQ);
         for (int j = 0; j < a.nslab; ++j)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            umma_f16(tmem + (uint32_t)(s * kSQ), sw128_kmajor_desc(wbase + j * kSC * 128 + kk * 32),
-                      sw128_kmajor_desc(dbase + j * kSQ * 128 + kk * 32), idesc,
-                      (j > 0 || kk > 0) ? 1u : 0u);
+            umma_f16(d_tmem, sw128_kmajor_desc(wbase + j * kSC * 128 + kk * 32),
+                     sw128_kmajor_desc(db + j * kSQ * 128 + kk * 32), idesc,
+                     (j > 0 || kk > 0) ? 1u : 0u);
         umma_commit(smem_u32(&mma_done[s]));
         return true;
       };
+      bool ok = mbar_wait(wb, 0, a.err, 21);
       if (ok) {
-        issue_tma(0);
-        if (nch > 1) issue_tma(1);
+        issue_stage(0);
+        if (nch > 1) issue_stage(1);
         ok = issue_mma(0);
       }
       for (int k = 0; ok && k < nch; ++k) {
         if (k + 1 < nch) {
+          // accumulator (k+1)&1 was last read by the compute warps for chunk k-1
           if (k >= 1 && !mbar_wait(smem_u32(&empty[(k + 1) & 1]), (uint32_t)((k - 1) >> 1) & 1u,
                                    a.err, 23))
             break;
           if (!issue_mma(k + 1)) break;
         }
         if (k + 2 < nch) {
+          // stage k&1 (dt_n read by MMA k, B/C read by chunk k) is free after chunk k
           if (!mbar_wait(smem_u32(&empty[k & 1]), (uint32_t)(k >> 1) & 1u, a.err, 24)) break;
-          issue_tma(k + 2);
+          issue_stage(k + 2);
         }
       }
     }
   } else {
-    // compute warps: thread = channel c0 + 32*warp + lane = TMEM lane
+    // compute warps: thread = channel c0 + 32*warp + lane = TMEM lane; its 16
+    // states live in registers as 8 float2 pairs, and so does the conv window.
+    // x and z are read straight from global memory one token group ahead.
     const int cl = warp * 32 + lane;
     const int64_t c = c0 + cl;
     const bool cok = c < a.d;
-    float A2[kN], h[kN];
+    float2 A2[kN / 2], h[kN / 2];
 #pragma unroll
-    for (int n = 0; n < kN; ++n) {
-      A2[n] = cok ? -expf(a.A_log[c * kN + n]) * kLog2e : 0.0f;
-      h[n] = (cok && a.h0) ? a.h0[(b * a.d + c) * kN + n] : 0.0f;
+    for (int q = 0; q < kN / 2; ++q) {
+      A2[q].x = cok ? -expf(a.A_log[c * kN + 2 * q]) * kLog2e : 0.0f;
+      A2[q].y = cok ? -expf(a.A_log[c * kN + 2 * q + 1]) * kLog2e : 0.0f;
+      h[q].x = (cok && a.h0) ? a.h0[(b * a.d + c) * kN + 2 * q] : 0.0f;
+      h[q].y = (cok && a.h0) ? a.h0[(b * a.d + c) * kN + 2 * q + 1] : 0.0f;
     }
     const float bias = cok ? a.dt_bias[c] : 0.0f;
     const float Dc = cok ? a.D[c] : 0.0f;
+    float cw[kConv], xw[kConv - 1];
+#pragma unroll
+    for (int k = 0; k < kConv; ++k) cw[k] = cok ? bf(a.conv_w[c * kConv + k]) : 0.0f;
+    const float cb = cok ? bf(a.conv_b[c]) : 0.0f;
+#pragma unroll
+    for (int k = 0; k < kConv - 1; ++k)
+      xw[k] = (cok && a.hist) ? bf(a.hist[(b * a.d + c) * (kConv - 1) + k]) : 0.0f;
     bf16* yrow = a.y + g0 * a.d + c;
     for (int k = 0; k < nch; ++k) {
       const int s = k & 1;
@@ -451,39 +545,73 @@ __global__ void __launch_bounds__(kScanThreads, 2)
       if (!mbar_wait(smem_u32(&mma_done[s]), ph, a.err, 25)) break;
       if (!mbar_wait(smem_u32(&full[s]), ph, a.err, 26)) break;
       tc_fence_after();
-      uint32_t r[16];
-      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(s * kSQ), r);
-      tmem_ld_wait();
       const uint8_t* st = stage_ptr(s);
-      const __half* us = reinterpret_cast<const __half*>(st + kDtnStage);
-      const bf16* zs = reinterpret_cast<const bf16*>(st + kDtnStage + kUStage);
-      const float4* bcs = reinterpret_cast<const float4*>(st + kDtnStage + 2 * kUStage);
+      const bf16* xs = reinterpret_cast<const bf16*>(st + kDtnStage);
+      const bf16* zs = reinterpret_cast<const bf16*>(st + kDtnStage + kXStage);
+      const float4* bcs = reinterpret_cast<const float4*>(st + kDtnStage + 2 * kXStage);
       const int64_t tbase = (int64_t)k * kSQ;
       const int nt = (int)((a.L - tbase) < kSQ ? (a.L - tbase) : kSQ);
+      const uint32_t tacc = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(s * kSQ);
+#pragma unroll 1
+      for (int g0t = 0; g0t < nt; g0t += kG) {
+        uint32_t r[kG];
+        tmem_ld_cols<kG>(tacc + (uint32_t)g0t, r);
+        tmem_ld_wait();
+        // per-token terms: u = SiLU(conv) in float32, delta, delta*u, D*u, SiLU(z)
+        float dl[kG], du[kG], dsk[kG], gz[kG];
 #pragma unroll
-      for (int t = 0; t < kSQ; ++t) {
-        if (t >= nt) break;
-        const float dl = softplus_acc(__uint_as_float(r[t]) + bias);
-        const float uv = __half2float(us[t * kSC + cl]);
-        const float zv = bf(zs[t * kSC + cl]);
-        const float du = dl * uv;
-        float acc = 0.0f;
-#pragma unroll
-        for (int q = 0; q < kN / 4; ++q) {
-          const float4 Bq = bcs[t * 8 + q];
-          const float4 Cq = bcs[t * 8 + 4 + q];
-          const float bq[4] = {Bq.x, Bq.y, Bq.z, Bq.w};
-          const float cq[4] = {Cq.x, Cq.y, Cq.z, Cq.w};
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int n = q * 4 + i;
-            const float da = ex2_approx(dl * A2[n]);
-            h[n] = fmaf(da, h[n], du * bq[i]);
-            acc = fmaf(cq[i], h[n], acc);
+        for (int i = 0; i < kG; ++i) {
+          const float xt = bf(xs[(g0t + i) * kSC + cl]);
+          float xc = fmaf(cw[0], xw[0], cb);
+          xc = fmaf(cw[1], xw[1], xc);
+          xc = fmaf(cw[2], xw[2], xc);
+          xc = fmaf(cw[3], xt, xc);
+          const float uv = silu_u(xc);
+          if (g0t + i < nt) {
+            xw[0] = xw[1];
+            xw[1] = xw[2];
+            xw[2] = xt;
           }
+          dl[i] = softplus_fast(__uint_as_float(r[i]) + bias);
+          du[i] = dl[i] * uv;
+          dsk[i] = Dc * uv;
+          gz[i] = silu_gate(bf(zs[(g0t + i) * kSC + cl]));
         }
-        const float ys = fmaf(Dc, uv, acc);
-        if (cok) yrow[(tbase + t) * a.d] = __float2bfloat16_rn(ys * silu_acc(zv));
+#pragma unroll
+        for (int i = 0; i < kG; ++i) {
+          const int t = g0t + i;
+          if (t >= nt) break;
+          const float2 dl2 = make_float2(dl[i], dl[i]);
+          const float2 du2 = make_float2(du[i], du[i]);
+          float2 acc[4];
+#pragma unroll
+          for (int q4 = 0; q4 < kN / 4; ++q4) {
+            const float4 Bq = bcs[t * 8 + q4];
+            const float4 Cq = bcs[t * 8 + 4 + q4];
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              const int q = q4 * 2 + half;
+              const float2 Bp = half ? make_float2(Bq.z, Bq.w) : make_float2(Bq.x, Bq.y);
+              const float2 Cp = half ? make_float2(Cq.z, Cq.w) : make_float2(Cq.x, Cq.y);
+              const float2 x = __fmul2_rn(dl2, A2[q]);
+              float2 da;
+              if (q >= kN / 2 - kSwPairs) {
+                da = exp2_pair_fma(x);
+              } else {
+                da.x = ex2_approx(x.x);
+                da.y = ex2_approx(x.y);
+              }
+              h[q] = __ffma2_rn(da, h[q], __fmul2_rn(du2, Bp));
+              // four independent partial sums of C.h (short dependency chains)
+              acc[q4] = half ? __ffma2_rn(Cp, h[q], acc[q4]) : __fmul2_rn(Cp, h[q]);
+            }
+          }
+          const float2 s01 = __fadd2_rn(acc[0], acc[1]);
+          const float2 s23 = __fadd2_rn(acc[2], acc[3]);
+          const float2 sa = __fadd2_rn(s01, s23);
+          const float ys = (sa.x + sa.y) + dsk[i];
+          if (cok) yrow[(tbase + t) * a.d] = __float2bfloat16_rn(ys * gz[i]);
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -491,20 +619,15 @@ __global__ void __launch_bounds__(kScanThreads, 2)
     }
     if (cok) {
 #pragma unroll
-      for (int n = 0; n < kN; ++n) a.hT[(b * a.d + c) * kN + n] = h[n];
+      for (int q = 0; q < kN / 2; ++q) {
+        a.hT[(b * a.d + c) * kN + 2 * q] = h[q].x;
+        a.hT[(b * a.d + c) * kN + 2 * q + 1] = h[q].y;
+      }
+      // the conv window now holds the last d_conv-1 inputs (exact bf16 values)
       if (a.final_conv) {
-        bf16 v[kConv - 1];
 #pragma unroll
-        for (int k = 0; k < kConv - 1; ++k) {
-          const int64_t tau = a.L - (kConv - 1) + k;
-          if (tau >= 0)
-            v[k] = a.x[(g0 + tau) * a.d + c];
-          else
-            v[k] = a.hist ? a.hist[(b * a.d + c) * (kConv - 1) + (kConv - 1) + tau]
-                          : __float2bfloat16_rn(0.0f);
-        }
-#pragma unroll
-        for (int k = 0; k < kConv - 1; ++k) a.final_conv[(b * a.d + c) * (kConv - 1) + k] = v[k];
+        for (int k = 0; k < kConv - 1; ++k)
+          a.final_conv[(b * a.d + c) * (kConv - 1) + k] = __float2bfloat16_rn(xw[k]);
       }
     }
   }
@@ -655,12 +778,12 @@ cudaError_t run_fast_fwd(Problem& p) {
   launched(p, "k_norms16");
   // 4. dt_proj + scan + gate
   {
-    CUtensorMap twdt, tdtn, tbc, tuu, tz;
+    CUtensorMap twdt, tdtn, tbc, tx, tz;
     if (!make_map(&twdt, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w.wdt, p.d, p.R, 64, kSC, true) ||
         !make_map(&tdtn, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w.dtn, p.T, p.R, 64, kSQ, true) ||
         !make_map(&tbc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, w.bc, p.T, 2 * kN, 2 * kN, kSQ,
                   false) ||
-        !make_map(&tuu, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w.u, p.T, p.d, kSC, kSQ, false) ||
+        !make_map(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.x, p.T, p.d, kSC, kSQ, false) ||
         !make_map(&tz, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.z, p.T, p.d, kSC, kSQ, false))
       return cudaErrorInvalidValue;
     ScanArgs sa;
@@ -669,19 +792,22 @@ cudaError_t run_fast_fwd(Problem& p) {
     sa.T = p.T;
     sa.R = (int)p.R;
     sa.nslab = (int)((p.R + 63) / 64);
+    sa.x = (const bf16*)p.x;
+    sa.z = (const bf16*)p.z;
+    sa.conv_w = (const bf16*)p.conv_w;
+    sa.conv_b = (const bf16*)p.conv_b;
     sa.dt_bias = p.dt_bias;
     sa.A_log = p.A_log;
     sa.D = p.D;
     sa.h0 = p.init_ssm;
     sa.hT = p.final_state;
     sa.y = (bf16*)p.y;
-    sa.x = (const bf16*)p.x;
     sa.hist = (const bf16*)p.init_conv;
     sa.final_conv = (bf16*)p.final_conv;
     sa.err = err;
     cudaFuncSetAttribute(k_scan_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, kScanSmem);
     k_scan_fused<<<dim3((unsigned)((p.d + kSC - 1) / kSC), (unsigned)p.B), kScanThreads, kScanSmem,
-                   s>>>(twdt, tdtn, tbc, tuu, tz, sa);
+                   s>>>(twdt, tdtn, tbc, tx, tz, sa);
     launched(p, "k_scan_fused");
   }
   return cudaGetLastError();

@@ -2,9 +2,9 @@
 // arithmetic throughout, intermediates in the workspace as float32.
 //
 // It is the only path for float32 io (TF32 tensor cores cannot meet a 1e-4
-// tolerance) and serves any io dtype.  In bf16 mode it rounds at the same two
-// points as the tensor-core path, which stores them as fp16: u after the SiLU
-// and dt_n before dt_proj.
+// tolerance) and serves any io dtype.  In bf16 mode it rounds where the
+// tensor-core path quantises: u to fp16 as the x_proj operand and dt_n to fp16
+// as the dt_proj operand (the scan keeps the float32 u).
 //
 // Steps (TransformerLens "Jamba" adapter page for the pipeline; aifetchly
 // "Jamba Guide", "Inside the Mamba State-Space Layers", for the scan):
@@ -36,7 +36,7 @@ __device__ __forceinline__ float softplus_precise(float v) {
 template <typename T>
 __global__ void k_conv_silu(const T* __restrict__ x, const T* __restrict__ conv_w,
                             const T* __restrict__ conv_b, const T* __restrict__ hist, int64_t L,
-                            int64_t d, int64_t total, int round_u, float* __restrict__ u) {
+                            int64_t d, int64_t total, float* __restrict__ u) {
   int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= total) return;
   int64_t c = i % d, g = i / d;
@@ -52,8 +52,7 @@ __global__ void k_conv_silu(const T* __restrict__ x, const T* __restrict__ conv_
       xv = ld(hist + (b * d + c) * (kConv - 1) + (kConv - 1) + tau);
     acc = fmaf(ld(conv_w + c * kConv + k), xv, acc);
   }
-  float v = silu_precise(acc);
-  u[i] = round_u ? to_fp16_value(v) : v;
+  u[i] = silu_precise(acc);
 }
 
 // out[m, n] = sum_k A[m, k] * W[n, k]   (A float32 [M, K], W io dtype [N, K])
@@ -61,7 +60,7 @@ __global__ void k_conv_silu(const T* __restrict__ x, const T* __restrict__ conv_
 // Tile 32 (m) x 32 (n), k-step 32, 256 threads, 4 outputs per thread.
 template <typename T, int EPI>
 __global__ void k_gemm_nt(const float* __restrict__ A, const T* __restrict__ W, int64_t M,
-                          int64_t N, int64_t K, const float* __restrict__ bias,
+                          int64_t N, int64_t K, const float* __restrict__ bias, int round_a,
                           float* __restrict__ out) {
   __shared__ float As[32][33];
   __shared__ float Ws[32][33];
@@ -73,7 +72,8 @@ __global__ void k_gemm_nt(const float* __restrict__ A, const T* __restrict__ W, 
     for (int i = 0; i < 4; ++i) {
       int r = ty + 8 * i;
       int64_t m = m0 + r, n = n0 + r, k = k0 + tx;
-      As[r][tx] = (m < M && k < K) ? A[m * K + k] : 0.0f;
+      const float av = (m < M && k < K) ? A[m * K + k] : 0.0f;
+      As[r][tx] = round_a ? to_fp16_value(av) : av;
       Ws[r][tx] = (n < N && k < K) ? ld(W + n * K + k) : 0.0f;
     }
     __syncthreads();
@@ -101,7 +101,7 @@ __global__ void k_gemm_nt(const float* __restrict__ A, const T* __restrict__ W, 
 template <typename T>
 __global__ void k_norms(const float* __restrict__ p, const T* __restrict__ wdt,
                         const T* __restrict__ wb, const T* __restrict__ wc, int64_t Tn, int R,
-                        float eps, int round_dt, float* __restrict__ dtn, float* __restrict__ Bn,
+                        float eps, float* __restrict__ dtn, float* __restrict__ Bn,
                         float* __restrict__ Cn) {
   const int lane = threadIdx.x & 31;
   const int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -114,8 +114,7 @@ __global__ void k_norms(const float* __restrict__ p, const T* __restrict__ wdt,
   for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   const float inv_dt = 1.0f / sqrtf(ss / (float)R + eps);
   for (int j = lane; j < R; j += 32) {
-    float v = row[j] * inv_dt * ld(wdt + j);
-    dtn[g * R + j] = round_dt ? to_fp16_value(v) : v;
+    dtn[g * R + j] = row[j] * inv_dt * ld(wdt + j);
   }
   // lanes 0..15 -> B, 16..31 -> C
   const int n = lane & 15;
@@ -222,17 +221,17 @@ cudaError_t run_simple_t(Problem& p) {
   launches_begin(p);
   k_conv_silu<T><<<(unsigned)((td + 255) / 256), 256, 0, s>>>(
       (const T*)p.x, (const T*)p.conv_w, (const T*)p.conv_b, (const T*)p.init_conv, p.L, p.d, td,
-      round, w.u);
+      w.u);
   launched(p, "k_conv_silu");
   k_gemm_nt<T, 0><<<dim3((unsigned)((p.P + 31) / 32), (unsigned)((p.T + 31) / 32)), 256, 0, s>>>(
-      w.u, (const T*)p.xproj_w, p.T, p.P, p.d, nullptr, w.p);
+      w.u, (const T*)p.xproj_w, p.T, p.P, p.d, nullptr, round, w.p);
   launched(p, "k_gemm_nt(x_proj)");
   k_norms<T><<<(unsigned)((p.T + 7) / 8), 256, 0, s>>>(w.p, (const T*)p.dtn_w, (const T*)p.bn_w,
                                                         (const T*)p.cn_w, p.T, (int)p.R, p.eps,
-                                                        round, w.dtn, w.Bn, w.Cn);
+                                                        w.dtn, w.Bn, w.Cn);
   launched(p, "k_norms");
   k_gemm_nt<T, 1><<<dim3((unsigned)((p.d + 31) / 32), (unsigned)((p.T + 31) / 32)), 256, 0, s>>>(
-      w.dtn, (const T*)p.dtproj_w, p.T, p.d, p.R, p.dt_bias, w.delta);
+      w.dtn, (const T*)p.dtproj_w, p.T, p.d, p.R, p.dt_bias, round, w.delta);
   launched(p, "k_gemm_nt(dt_proj)");
   k_scan_simple<T><<<dim3((unsigned)((p.d + 127) / 128), (unsigned)p.B), 128, 0, s>>>(
       w.delta, w.u, w.Bn, w.Cn, (const T*)p.z, p.A_log, p.D, p.init_ssm, p.final_state, (T*)p.y,

@@ -30,12 +30,11 @@
 //   6. gate: y = ys * z / (1 + exp(-z)).  Final SSM state = h after the last
 //      token; final conv state = the last K-1 conv inputs, oldest first.
 //
-// Mirror mode (mirror_bf16 = 1) rounds at the two points where the bf16-io
-// CUDA path stores an intermediate: u after the SiLU (it feeds both x_proj and
-// the scan) and dt_n (the dt_proj operand).  Both are stored as IEEE fp16, the
-// tensor-core operand type of that path.  The rounding is taken in the kernel's
-// precision: to float32 (nearest even), then to fp16 (nearest even).  Nothing
-// else is rounded.
+// Mirror mode (mirror_bf16 = 1) rounds where the bf16-io CUDA path quantises
+// an intermediate: the two tensor-core operands, u as the x_proj operand and
+// dt_n as the dt_proj operand, both stored as IEEE fp16.  The rounding is taken
+// in the kernel's precision: to float32 (nearest even), then to fp16 (nearest
+// even).  The scan uses the unrounded u.  Nothing else is rounded.
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
@@ -186,8 +185,8 @@ void orc_scan(int64_t L, int64_t d, int64_t N, const double* delta, const double
   orc_scan_range(L, d, N, delta, A, Bm, Cm, u, D, h0, y, hT, 0, d);
 }
 
-// Front end of one sequence for tokens [t0, t1): u (optionally mirror-rounded),
-// p rows, normalised dt_n / Bn / Cn rows.
+// Front end of one sequence for tokens [t0, t1): u, p rows (from the
+// mirror-rounded u in mirror mode), normalised dt_n (mirror-rounded) / Bn / Cn.
 static void front_end_rows(const orc_dims* m, Stored x, const double* conv_w,
                            const double* conv_b, const double* xproj_wT /*[d,P]*/,
                            const double* dtn_w, const double* bn_w, const double* cn_w,
@@ -204,13 +203,12 @@ static void front_end_rows(const orc_dims* m, Stored x, const double* conv_w,
         double xv = tau >= 0 ? x[tau * d + c] : (hist ? hist[c * (K - 1) + (K - 1) + tau] : 0.0);
         acc += conv_w[c * K + k] * xv;
       }
-      double uv = silu(acc);
-      ur[c] = m->mirror_bf16 ? round_fp16(uv) : uv;
+      ur[c] = silu(acc);
     }
     // p[j] = sum_c W_x[j,c] u[c], summed in ascending c for every j
     std::fill(p.begin(), p.end(), 0.0);
     for (int64_t c = 0; c < d; ++c) {
-      const double uc = ur[c];
+      const double uc = m->mirror_bf16 ? round_fp16(ur[c]) : ur[c];
       const double* wr = xproj_wT + c * P;
       for (int64_t j = 0; j < P; ++j) p[j] += wr[j] * uc;
     }
