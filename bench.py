@@ -41,6 +41,7 @@ def parse():
     ap.add_argument("--workload", default="jamba_b8_l4096")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--seqlen", type=int, default=0,
                     help="override the workload's sequence length (profiling captures)")
     return ap.parse_args()
@@ -135,6 +136,59 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(r[1] for r in inside),
                 "sm_max_mhz": max(r[2] for r in inside), "reasons": sorted(reasons),
                 "samples": len(inside)}
+
+
+# ------------------------------------------------------------------ decode
+def decode_bench(dev, stream, steps: int = 64, warmup: int = 5):
+    """64 consecutive jm_mixer_step calls on the decode workload (B=256 sequences at
+    Jamba shapes, states updated in place); returns a dict for the JSON line."""
+    import torch
+    from mamba_selective_scan_jamba_b200 import devio, jmix, synth
+    w = synth.WORKLOADS["jamba_decode_b256"]
+    W = synth.make_weights(w)
+    S = synth.make_decode_state(w)
+    Wd = devio.weights_to_device(W, dev)
+    cs = devio.to_device(S["conv_state"], dev)
+    ss = devio.to_device(S["ssm_state"], dev)
+    toks = [synth.make_decode_token(w, t) for t in range(4)]
+    xs = [devio.to_device(t["x_t"], dev) for t in toks]
+    zs = [devio.to_device(t["z_t"], dev) for t in toks]
+    y = torch.empty_like(xs[0])
+    d = devio.dims_of(w)
+    n = jmix.jm_mixer_step_workspace_size(d)
+    ws = devio.workspace(n, dev)
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
+            jmix.jm_mixer_step(d, xs[i % 4], zs[i % 4], cs, ss, Wd, y, ws, n, stream=stream)
+    stream.synchronize()
+    nk = jmix.jm_last_launch_count()
+    names = [jmix.jm_last_kernel_name(i) for i in range(nk)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for row in evs:
+            for e in row:
+                e.record(stream)
+    stream.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        for i in range(steps):
+            jmix.jm_set_kernel_events([e.cuda_event for e in evs[i]])
+            jmix.jm_mixer_step(d, xs[i % 4], zs[i % 4], cs, ss, Wd, y, ws, n, stream=stream)
+        b.record(stream)
+    jmix.jm_set_kernel_events(None)
+    stream.synchronize()
+    assert jmix.jm_poll_error(ws, stream) == jmix.JM_OK, jmix.jm_last_error()
+    ms = a.elapsed_time(b) / steps
+    per = {names[k]: round(sum(evs[i][k].elapsed_time(evs[i][k + 1]) for i in range(steps))
+                           / steps * 1e3, 2) for k in range(nk)}
+    # algorithmic bytes per step: ssm state r+w, conv state r+w, x_t, z_t, y_t
+    B, dd, N = w.batch, w.d_inner, w.d_state
+    nbytes = B * dd * (N * 4 * 2 + 3 * 2 * 2 + 2 * 3)
+    return {"workload": w.name, "batch": B, "steps": steps, "us_per_step": ms * 1e3,
+            "tokens_per_s": B / (ms / 1e3), "algorithmic_bytes_per_step": nbytes,
+            "achieved_GBps": nbytes / (ms / 1e3) / 1e9, "kernels_us": per,
+            "launches_per_step": nk}
 
 
 # ------------------------------------------------------------- cpu baseline
@@ -371,6 +425,10 @@ def main():
                        "ms_per_step": ems, "steps": Ke,
                        "api": "jm_mixer_fwd_host (pinned host x, z -> y, final_state)"}
 
+    if not args.no_decode:
+        dec = decode_bench(dev, stream)
+        dec["hbm_frac"] = dec["achieved_GBps"] / P["hbm"]
+        line["decode"] = dec
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, cores, sample = oracle_rate(w, 12.0)
         line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores,

@@ -126,7 +126,7 @@ jm_status jm_mixer_step(const jm_dims* dims, const void* x_t, const void* z_t, v
  * Arguments and results are those of jm_mixer_step without workspace and
  * ws_bytes.  The scratch is a static 32 MiB device array inside libjmix, held
  * by every GPU that loads the library until the process exits; a step at
- * Jamba v0.1 mixer shapes (d_inner 8192, dt_rank 256) needs about 17 MiB for
+ * Jamba v0.1 mixer shapes (d_inner 8192, dt_rank 256) needs about 14 MiB for
  * 256 sequences.  A step that needs more returns JM_ERR_UNSUPPORTED with a
  * message and launches nothing.  The function itself allocates nothing.
  *

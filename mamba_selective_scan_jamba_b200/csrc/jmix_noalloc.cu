@@ -18,7 +18,7 @@ namespace jmix {
 namespace {
 
 // 32 MiB: enough for a decode step of 256 sequences at Jamba v0.1 mixer shapes
-// (d_inner 8192, dt_rank 256), which needs about 17 MiB.
+// (d_inner 8192, dt_rank 256), which needs about 14 MiB.
 constexpr size_t kStepScratchBytes = size_t(32) << 20;
 constexpr int kMaxDevices = 64;
 

@@ -4,8 +4,10 @@
 //                   operand; the same launch converts xproj_w and dtproj_w from
 //                   bf16 to fp16 (exact for |w| >= 2^-14; fp16 subnormals below).
 //   k_xproj         p = u . xproj_w^T on tcgen05 (TMA -> SMEM -> MMA -> TMEM),
-//                   split over d_inner; partial tiles added into p (fp32).
-//   k_norms16       dt_n (fp16, the dt_proj operand), B_n and C_n (fp32) = RMSNorm(.) w.
+//                   split over d_inner; each split stores its partial tile.
+//   k_norms16       sums the x_proj partials in a fixed order (so results are
+//                   bitwise reproducible), then dt_n (fp16, the dt_proj operand),
+//                   B_n and C_n (fp32) = RMSNorm(.) w.
 //   k_scan_fused    per (sequence, 128 channels): dt_proj on tcgen05 into TMEM,
 //                   softplus, the conv + SiLU recomputed in fp32 from x, the
 //                   selective scan with fp32 state in registers, the D skip, the
@@ -168,7 +170,7 @@ struct XprojArgs {
   int P, Ntot, N1, N2;
   int kchunks, ksplit;
   uint32_t tmem_cols;
-  float* p;
+  float* part;  // [ksplit, T, P] partial sums
   ErrFlags* err;
 };
 
@@ -260,26 +262,34 @@ __global__ void __launch_bounds__(kXThreads, 1)
       umma_commit(smem_u32(acc_full));
     }
   } else {
-    // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 = tile rows
+    // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 = tile rows, 16
+    // columns at a time, transposes them through shared memory (the stage
+    // buffers are free once the accumulator is complete) and stores two
+    // 64-byte row segments per instruction
     const bool ok = mbar_wait(smem_u32(acc_full), 0, a.err, 13);
     tc_fence_after();
     const int lg = warp & 3;
-    const int64_t g = (int64_t)m_tile * kXM + lg * 32 + lane;
-    const bool row_ok = ok && g < a.T && k_end > k_begin;
+    float* tbuf = reinterpret_cast<float*>(smem) + (warp - 2) * (32 * 17);
+    const int64_t row0 = (int64_t)m_tile * kXM + lg * 32;
+    float* dst = a.part + ((int64_t)split * a.T) * a.P;
+    const bool any = ok && k_end > k_begin;
     for (int c0 = 0; c0 < a.Ntot; c0 += 16) {
       uint32_t r[16];
       tmem_ld16(tmem + ((uint32_t)(lg * 32) << 16) + (uint32_t)c0, r);
       tmem_ld_wait();
-      if (row_ok) {
 #pragma unroll
-        for (int j = 0; j < 16; j += 4) {
-          const int col = c0 + j;
-          if (col < a.P)
-            atomicAdd(reinterpret_cast<float4*>(a.p + g * a.P + col),
-                      make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]),
-                                  __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3])));
+      for (int j = 0; j < 16; ++j) tbuf[lane * 17 + j] = __uint_as_float(r[j]);
+      __syncwarp();
+      if (any) {
+        const int col = c0 + (lane & 15);
+#pragma unroll 4
+        for (int rr = 0; rr < 16; ++rr) {
+          const int row = 2 * rr + (lane >> 4);
+          const int64_t g = row0 + row;
+          if (g < a.T && col < a.P) dst[g * a.P + col] = tbuf[row * 17 + (lane & 15)];
         }
       }
+      __syncwarp();
     }
   }
   tc_fence_before();
@@ -291,32 +301,57 @@ __global__ void __launch_bounds__(kXThreads, 1)
 }
 
 // -------------------------------------------------------------------- norms
-// dt_n is written in fp16, the dt_proj operand type.
+// One block per token: p[j] = sum of the ksplit partial rows in ascending split
+// order (one thread per column), then the norms (warp 0: dt over R, warp 1: B
+// and C over N).  dt_n is written in fp16, the dt_proj operand type.
+constexpr int kMaxP = kMaxRank + 2 * kN;
+constexpr int kNormThreads = 320;  // >= kMaxP
+
 template <typename W>
-__global__ void __launch_bounds__(256) k_norms16(const float* __restrict__ p,
-                                                const W* __restrict__ wdt,
-                                                const W* __restrict__ wb, const W* __restrict__ wc,
-                                                int64_t Tn, int R, float eps,
-                                                __half* __restrict__ dtn,
-                                                float* __restrict__ bc) {
-  const int lane = threadIdx.x & 31;
-  const int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (g >= Tn) return;
+__global__ void __launch_bounds__(kNormThreads) k_norms16(
+    const float* __restrict__ part, int ksplit, const W* __restrict__ wdt,
+    const W* __restrict__ wb, const W* __restrict__ wc, int64_t Tn, int R, float eps,
+    __half* __restrict__ dtn, float* __restrict__ bc) {
+  __shared__ float row[kMaxP];
+  __shared__ float inv_dt;
+  const int64_t g = blockIdx.x;
   const int P = R + 2 * kN;
-  const float* row = p + g * P;
-  float ss = 0.f;
-  for (int j = lane; j < R; j += 32) ss = fmaf(row[j], row[j], ss);
+  const int j = threadIdx.x;
+  if (j < P) {
+    const float* src = part + g * P + j;
+    const int64_t stride = Tn * P;
+    float acc = src[0];
+    int sp = 1;
+    for (; sp + 4 <= ksplit; sp += 4) {
+      const float v0 = src[sp * stride], v1 = src[(sp + 1) * stride];
+      const float v2 = src[(sp + 2) * stride], v3 = src[(sp + 3) * stride];
+      acc += v0;
+      acc += v1;
+      acc += v2;
+      acc += v3;
+    }
+    for (; sp < ksplit; ++sp) acc += src[sp * stride];
+    row[j] = acc;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
+  if (wi == 0) {
+    float ss = 0.f;
+    for (int k = lane; k < R; k += 32) ss = fmaf(row[k], row[k], ss);
 #pragma unroll
-  for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  const float inv = 1.0f / sqrtf(ss / (float)R + eps);
-  for (int j = lane; j < R; j += 32) dtn[g * R + j] = __float2half_rn(row[j] * inv * (float)wdt[j]);
-  const float v = row[R + lane];
-  float s2 = v * v;
+    for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if (lane == 0) inv_dt = 1.0f / sqrtf(ss / (float)R + eps);
+  } else if (wi == 1) {
+    const float v = row[R + lane];
+    float s2 = v * v;
 #pragma unroll
-  for (int o = 8; o; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
-  const float inv2 = 1.0f / sqrtf(s2 / (float)kN + eps);
-  const float wv = lane < 16 ? (float)wb[lane] : (float)wc[lane - 16];
-  bc[g * 2 * kN + lane] = v * inv2 * wv;
+    for (int o = 8; o; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+    const float inv2 = 1.0f / sqrtf(s2 / (float)kN + eps);
+    const float wv = lane < 16 ? (float)wb[lane] : (float)wc[lane - 16];
+    bc[g * 2 * kN + lane] = v * inv2 * wv;
+  }
+  __syncthreads();
+  if (j < R) dtn[g * R + j] = __float2half_rn(row[j] * inv_dt * (float)wdt[j]);
 }
 
 // ------------------------------------------------------- fused dt_proj + scan
@@ -639,6 +674,203 @@ __global__ void __launch_bounds__(kScanThreads, 2)
   }
 }
 
+// ------------------------------------------------------------- decode step
+// One token per sequence.  CTA = 128 channels x kDB sequences: dt_proj for the
+// tile on tcgen05 (A = W_dt tile, B = dt_n of the kDB sequences, D in TMEM with
+// lane = channel, column = sequence); then thread = channel walks the kDB
+// sequences: conv + SiLU from the cached conv state, softplus, the 16-state
+// update in place, the gate, and the conv-state shift.  The SSM state read and
+// write (64 B each per (sequence, channel)) is the HBM traffic that bounds it.
+constexpr int kDB = 16;                                   // sequences per CTA (MMA N)
+constexpr int kDecThreads = 160;
+constexpr int kDecDtn = kMaxSlabs * kDB * 128;            // 8 KB
+constexpr int kDecBC = kDB * 2 * kN * 4;                  // 2 KB
+constexpr int kDecSmem = 1024 + kWdtBytes + kDecDtn + kDecBC + 128;
+
+struct DecArgs {
+  int64_t B, d;
+  int nslab;
+  const bf16* x;
+  const bf16* z;
+  const bf16* conv_w;
+  const bf16* conv_b;
+  const float* dt_bias;
+  const float* A_log;
+  const float* D;
+  bf16* conv_state;   // [B, d, 3] in/out
+  float* ssm_state;   // [B, d, 16] in/out
+  bf16* y;
+  ErrFlags* err;
+};
+
+__global__ void __launch_bounds__(kDecThreads, 2)
+    k_decode_scan(const __grid_constant__ CUtensorMap tm_wdt,
+                  const __grid_constant__ CUtensorMap tm_dtn,
+                  const __grid_constant__ CUtensorMap tm_bc, const DecArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* wdt_s = smem;
+  uint8_t* dtn_s = smem + kWdtBytes;
+  const float4* bcs = reinterpret_cast<const float4*>(dtn_s + kDecDtn);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(dtn_s + kDecDtn + kDecBC);
+  uint64_t* full = bars;
+  uint64_t* mma_done = bars + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t c0 = (int64_t)blockIdx.x * kSC;
+  const int64_t b0 = (int64_t)blockIdx.y * kDB;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(full), 1);
+    mbar_init(smem_u32(mma_done), 1);
+    fence_mbar_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(smem_u32(tmem_slot), 32);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      prefetch_tmap(&tm_wdt);
+      prefetch_tmap(&tm_dtn);
+      prefetch_tmap(&tm_bc);
+      const uint32_t fb = smem_u32(full);
+      mbar_arrive_expect_tx(fb, (uint32_t)(a.nslab * (kSC + kDB) * 128 + kDecBC));
+      for (int j = 0; j < a.nslab; ++j) {
+        tma_load_2d(smem_u32(wdt_s + j * kSC * 128), &tm_wdt, fb, j * 64, (int32_t)c0);
+        tma_load_2d(smem_u32(dtn_s + j * kDB * 128), &tm_dtn, fb, j * 64, (int32_t)b0);
+      }
+      tma_load_2d(smem_u32(bcs), &tm_bc, fb, 0, (int32_t)b0);
+      if (mbar_wait(fb, 0, a.err, 31)) {
+        tc_fence_after();
+        const uint32_t idesc = idesc_f16_f32(kSC, kDB);
+        const uint32_t wbase = smem_u32(wdt_s), db = smem_u32(dtn_s);
+        for (int j = 0; j < a.nslab; ++j)
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_f16(tmem, sw128_kmajor_desc(wbase + j * kSC * 128 + kk * 32),
+                     sw128_kmajor_desc(db + j * kDB * 128 + kk * 32), idesc,
+                     (j > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(smem_u32(mma_done));
+      }
+    }
+  } else {
+    const int cl = warp * 32 + lane;
+    const int64_t c = c0 + cl;
+    const bool cok = c < a.d;
+    const int nb = (int)((a.B - b0) < kDB ? (a.B - b0) : kDB);
+    // per-column inputs, loaded two columns ahead (they do not depend on delta,
+    // so the first loads go out before the dt_proj accumulator is ready)
+    struct Col {
+      float4 h[4];
+      float s[kConv - 1];
+      bf16 xb;
+      float z;
+    };
+    auto load_col = [&](int j, Col& cd) {
+      if (cok && j < nb) {
+        const int64_t bc = (b0 + j) * a.d + c;
+        const float4* st = reinterpret_cast<const float4*>(a.ssm_state + bc * kN);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) cd.h[q] = st[q];
+        const bf16* cs = a.conv_state + bc * (kConv - 1);
+#pragma unroll
+        for (int k = 0; k < kConv - 1; ++k) cd.s[k] = bf(cs[k]);
+        cd.xb = a.x[bc];
+        cd.z = bf(a.z[bc]);
+      }
+    };
+    Col cbuf[2];
+    load_col(0, cbuf[0]);
+    load_col(1, cbuf[1]);
+    float2 A2[kN / 2];
+    float bias = 0.f, Dc = 0.f, cb = 0.f, cw[kConv] = {0.f, 0.f, 0.f, 0.f};
+    if (cok) {
+#pragma unroll
+      for (int q = 0; q < kN / 2; ++q) {
+        A2[q].x = -expf(a.A_log[c * kN + 2 * q]) * kLog2e;
+        A2[q].y = -expf(a.A_log[c * kN + 2 * q + 1]) * kLog2e;
+      }
+      bias = a.dt_bias[c];
+      Dc = a.D[c];
+#pragma unroll
+      for (int k = 0; k < kConv; ++k) cw[k] = bf(a.conv_w[c * kConv + k]);
+      cb = bf(a.conv_b[c]);
+    }
+    const bool ok = mbar_wait(smem_u32(mma_done), 0, a.err, 32) &&
+                    mbar_wait(smem_u32(full), 0, a.err, 33);
+    tc_fence_after();
+    uint32_t r[kDB];
+    tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16), r);
+    tmem_ld_wait();
+    if (ok && cok) {
+#pragma unroll
+      for (int j = 0; j < kDB; ++j) {
+        if (j >= nb) break;
+        Col& cd = cbuf[j & 1];
+        const int64_t bc = (b0 + j) * a.d + c;
+        const float xt = bf(cd.xb);
+        float xc = fmaf(cw[0], cd.s[0], cb);
+        xc = fmaf(cw[1], cd.s[1], xc);
+        xc = fmaf(cw[2], cd.s[2], xc);
+        xc = fmaf(cw[3], xt, xc);
+        const float uv = silu_u(xc);
+        const float dl = softplus_fast(__uint_as_float(r[j]) + bias);
+        const float2 dl2 = make_float2(dl, dl), du2 = make_float2(dl * uv, dl * uv);
+        float2 h[kN / 2];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          h[2 * q] = make_float2(cd.h[q].x, cd.h[q].y);
+          h[2 * q + 1] = make_float2(cd.h[q].z, cd.h[q].w);
+        }
+        float2 acc[4];
+#pragma unroll
+        for (int q4 = 0; q4 < kN / 4; ++q4) {
+          const float4 Bq = bcs[j * 8 + q4];
+          const float4 Cq = bcs[j * 8 + 4 + q4];
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const int q = q4 * 2 + half;
+            const float2 Bp = half ? make_float2(Bq.z, Bq.w) : make_float2(Bq.x, Bq.y);
+            const float2 Cp = half ? make_float2(Cq.z, Cq.w) : make_float2(Cq.x, Cq.y);
+            const float2 xq = __fmul2_rn(dl2, A2[q]);
+            const float2 da = make_float2(ex2_approx(xq.x), ex2_approx(xq.y));
+            h[q] = __ffma2_rn(da, h[q], __fmul2_rn(du2, Bp));
+            acc[q4] = half ? __ffma2_rn(Cp, h[q], acc[q4]) : __fmul2_rn(Cp, h[q]);
+          }
+        }
+        const float2 sa = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+        const float ys = (sa.x + sa.y) + Dc * uv;
+        const bf16 xkeep = cd.xb;
+        const float s1 = cd.s[1], s2 = cd.s[2], zv = cd.z;
+        load_col(j + 2, cd);   // refill this slot two columns ahead
+        a.y[bc] = __float2bfloat16_rn(ys * silu_gate(zv));
+        float4* st = reinterpret_cast<float4*>(a.ssm_state + bc * kN);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          st[q] = make_float4(h[2 * q].x, h[2 * q].y, h[2 * q + 1].x, h[2 * q + 1].y);
+        bf16* cs = a.conv_state + bc * (kConv - 1);
+        cs[0] = __float2bfloat16_rn(s1);
+        cs[1] = __float2bfloat16_rn(s2);
+        cs[2] = xkeep;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 32);
+  }
+}
+
 // ---------------------------------------------------------------- host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -675,15 +907,28 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, size_t esize, const void* 
 
 struct FastWs {
   char* hdr;
-  float* p;
+  float* part;
   __half* u;
   __half* dtn;
   float* bc;
   __half* wx;
   __half* wdt;
   size_t bytes;
-  size_t zero_bytes;  // header + p, cleared each call
+  int ksplit;
 };
+
+// x_proj split over d_inner: about two CTAs per SM of a B200 (2 x 148), at
+// most 64 splits, at least one 64-channel chunk per split.  Depends on the
+// problem only, so the workspace size does too.
+int xproj_ksplit(int64_t T, int64_t d) {
+  if (T <= 0) return 1;
+  const int64_t mtiles = (T + kXM - 1) / kXM;
+  const int64_t kchunks = (d + kXK - 1) / kXK;
+  int64_t ks = (296 + mtiles - 1) / mtiles;
+  if (ks > 64) ks = 64;
+  if (ks > kchunks) ks = kchunks;
+  return ks < 1 ? 1 : (int)ks;
+}
 
 FastWs fast_layout(const Problem& pr, char* base) {
   FastWs w{};
@@ -694,9 +939,9 @@ FastWs fast_layout(const Problem& pr, char* base) {
     return base ? base + o : nullptr;
   };
   const size_t T = (size_t)pr.T, d = (size_t)pr.d, P = (size_t)pr.P, R = (size_t)pr.R;
+  w.ksplit = xproj_ksplit(pr.T, pr.d);
   w.hdr = take(sizeof(ErrFlags));
-  w.p = reinterpret_cast<float*>(take(T * P * 4));
-  w.zero_bytes = off;
+  w.part = reinterpret_cast<float*>(take((size_t)w.ksplit * T * P * 4));
   w.u = reinterpret_cast<__half*>(take(T * d * 2));
   w.dtn = reinterpret_cast<__half*>(take(T * R * 2));
   w.bc = reinterpret_cast<float*>(take(T * 2 * kN * 4));
@@ -706,23 +951,11 @@ FastWs fast_layout(const Problem& pr, char* base) {
   return w;
 }
 
-int g_num_sms = 0;
-
-int num_sms() {
-  if (!g_num_sms) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
-    if (g_num_sms <= 0) g_num_sms = 148;
-  }
-  return g_num_sms;
-}
-
 cudaError_t run_fast_fwd(Problem& p) {
   FastWs w = fast_layout(p, p.ws);
   cudaStream_t s = p.stream;
   ErrFlags* err = reinterpret_cast<ErrFlags*>(w.hdr);
-  cudaError_t e = cudaMemsetAsync(p.ws, 0, w.zero_bytes, s);
+  cudaError_t e = cudaMemsetAsync(p.ws, 0, sizeof(ErrFlags), s);
   if (e != cudaSuccess) return e;
   launches_begin(p);
 
@@ -755,13 +988,10 @@ cudaError_t run_fast_fwd(Problem& p) {
     xa.Ntot = xa.N1 + xa.N2;
     xa.kchunks = (int)((p.d + kXK - 1) / kXK);
     const int64_t mtiles = (p.T + kXM - 1) / kXM;
-    int64_t ks = (2 * num_sms() + mtiles - 1) / mtiles;
-    if (ks < 1) ks = 1;
-    if (ks > xa.kchunks) ks = xa.kchunks;
-    xa.ksplit = (int)ks;
+    xa.ksplit = w.ksplit;
     xa.tmem_cols = xa.Ntot <= 32 ? 32 : xa.Ntot <= 64 ? 64 : xa.Ntot <= 128 ? 128
                    : xa.Ntot <= 256 ? 256 : 512;
-    xa.p = w.p;
+    xa.part = w.part;
     xa.err = err;
     if (!make_map(&tu, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w.u, p.T, p.d, kXK, kXM, true) ||
         !make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w.wx, p.P, p.d, kXK, xa.N1, true))
@@ -772,12 +1002,38 @@ cudaError_t run_fast_fwd(Problem& p) {
     launched(p, "k_xproj");
   }
   // 3. RMSNorms
-  k_norms16<bf16><<<(unsigned)((p.T + 7) / 8), 256, 0, s>>>(
-      w.p, (const bf16*)p.dtn_w, (const bf16*)p.bn_w, (const bf16*)p.cn_w, p.T, (int)p.R, p.eps,
+  k_norms16<bf16><<<(unsigned)p.T, kNormThreads, 0, s>>>(
+      w.part, w.ksplit, (const bf16*)p.dtn_w, (const bf16*)p.bn_w, (const bf16*)p.cn_w, p.T, (int)p.R, p.eps,
       w.dtn, w.bc);
   launched(p, "k_norms16");
   // 4. dt_proj + scan + gate
-  {
+  if (p.decode) {
+    CUtensorMap twdt, tdtn, tbc;
+    if (!make_map(&twdt, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w.wdt, p.d, p.R, 64, kSC, true) ||
+        !make_map(&tdtn, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w.dtn, p.T, p.R, 64, kDB, true) ||
+        !make_map(&tbc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, w.bc, p.T, 2 * kN, 2 * kN, kDB,
+                  false))
+      return cudaErrorInvalidValue;
+    DecArgs da;
+    da.B = p.B;
+    da.d = p.d;
+    da.nslab = (int)((p.R + 63) / 64);
+    da.x = (const bf16*)p.x;
+    da.z = (const bf16*)p.z;
+    da.conv_w = (const bf16*)p.conv_w;
+    da.conv_b = (const bf16*)p.conv_b;
+    da.dt_bias = p.dt_bias;
+    da.A_log = p.A_log;
+    da.D = p.D;
+    da.conv_state = (bf16*)p.final_conv;
+    da.ssm_state = p.final_state;
+    da.y = (bf16*)p.y;
+    da.err = err;
+    cudaFuncSetAttribute(k_decode_scan, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
+    k_decode_scan<<<dim3((unsigned)((p.d + kSC - 1) / kSC), (unsigned)((p.B + kDB - 1) / kDB)),
+                    kDecThreads, kDecSmem, s>>>(twdt, tdtn, tbc, da);
+    launched(p, "k_decode_scan");
+  } else {
     CUtensorMap twdt, tdtn, tbc, tx, tz;
     if (!make_map(&twdt, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w.wdt, p.d, p.R, 64, kSC, true) ||
         !make_map(&tdtn, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w.dtn, p.T, p.R, 64, kSQ, true) ||
@@ -815,13 +1071,8 @@ cudaError_t run_fast_fwd(Problem& p) {
 
 }  // namespace
 
-size_t fast_ws_bytes(const Problem& p) {
-  return p.decode ? simple_ws_bytes(p) : fast_layout(p, nullptr).bytes;
-}
+size_t fast_ws_bytes(const Problem& p) { return fast_layout(p, nullptr).bytes; }
 
-cudaError_t run_fast(Problem& p) {
-  if (p.decode) return run_simple(p);
-  return run_fast_fwd(p);
-}
+cudaError_t run_fast(Problem& p) { return run_fast_fwd(p); }
 
 }  // namespace jmix

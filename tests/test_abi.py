@@ -58,6 +58,13 @@ def fwd(d, ws_bytes=1 << 30, **over):
                              check=False)
 
 
+def test_workspace_size_of_empty_problems(lib):
+    for io in (jmix.JM_BF16, jmix.JM_F32):
+        for B, L in ((0, 5), (2, 0), (0, 0)):
+            assert jmix.jm_mixer_fwd_workspace_size(jmix.dims(B, L, 256, 16, io)) >= 256
+        assert jmix.jm_mixer_step_workspace_size(jmix.dims(0, 1, 256, 16, io)) >= 256
+
+
 def test_workspace_size_rules(lib):
     d = jmix.dims(8, 4096, 8192, 256)
     n = jmix.jm_mixer_fwd_workspace_size(d)
