@@ -71,6 +71,20 @@ __device__ __forceinline__ float silu_u(float v) {
   return v * r;
 }
 
+// v * sigmoid(v) with one MUFU op: 1/(1 + e) by Newton-Raphson on the FMA pipe
+// from a bit-pattern initial guess (3 iterations, relative error < 2e-7 on
+// [1, 8.5e37]); e is clamped so that the guess stays a normal number.
+__device__ __forceinline__ float silu_newton(float v) {
+  float e;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-v * kLog2e));
+  const float den = fminf(1.0f + e, 8.5e37f);
+  float r = __int_as_float(poly::RCP_MAGIC - __float_as_int(den));
+  r = r * fmaf(-den, r, 2.0f);
+  r = r * fmaf(-den, r, 2.0f);
+  r = r * fmaf(-den, r, 2.0f);
+  return v * r;
+}
+
 __global__ void __launch_bounds__(256, 2) k_conv_silu16(
     const bf16* __restrict__ x, const bf16* __restrict__ conv_w, const bf16* __restrict__ conv_b,
     const bf16* __restrict__ hist, int64_t B, int64_t L, int64_t d, __half* __restrict__ u,
@@ -301,25 +315,27 @@ __global__ void __launch_bounds__(kXThreads, 1)
 }
 
 // -------------------------------------------------------------------- norms
-// One block per token: p[j] = sum of the ksplit partial rows in ascending split
-// order (one thread per column), then the norms (warp 0: dt over R, warp 1: B
-// and C over N).  dt_n is written in fp16, the dt_proj operand type.
+// TPB tokens per block: p[j] = sum of the ksplit partial rows in ascending
+// split order (threads over (token, column) pairs), then per token the norms
+// (one warp: dt over R; B and C over N).  dt_n is written in fp16, the dt_proj
+// operand type.  TPB = 8 for many tokens, 1 when few tokens carry many splits.
 constexpr int kMaxP = kMaxRank + 2 * kN;
-constexpr int kNormThreads = 320;  // >= kMaxP
+constexpr int kNormThreads = 256;
 
-template <typename W>
+template <typename W, int TPB>
 __global__ void __launch_bounds__(kNormThreads) k_norms16(
     const float* __restrict__ part, int ksplit, const W* __restrict__ wdt,
     const W* __restrict__ wb, const W* __restrict__ wc, int64_t Tn, int R, float eps,
     __half* __restrict__ dtn, float* __restrict__ bc) {
-  __shared__ float row[kMaxP];
-  __shared__ float inv_dt;
-  const int64_t g = blockIdx.x;
+  __shared__ float rows[TPB][kMaxP];
+  const int64_t g0 = (int64_t)blockIdx.x * TPB;
   const int P = R + 2 * kN;
-  const int j = threadIdx.x;
-  if (j < P) {
+  const int64_t stride = Tn * P;
+  for (int idx = threadIdx.x; idx < TPB * P; idx += kNormThreads) {
+    const int tl = idx / P, j = idx - tl * P;
+    const int64_t g = g0 + tl;
+    if (g >= Tn) continue;
     const float* src = part + g * P + j;
-    const int64_t stride = Tn * P;
     float acc = src[0];
     int sp = 1;
     for (; sp + 4 <= ksplit; sp += 4) {
@@ -331,17 +347,21 @@ __global__ void __launch_bounds__(kNormThreads) k_norms16(
       acc += v3;
     }
     for (; sp < ksplit; ++sp) acc += src[sp * stride];
-    row[j] = acc;
+    rows[tl][j] = acc;
   }
   __syncthreads();
   const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
-  if (wi == 0) {
+  for (int tl = wi; tl < TPB; tl += kNormThreads / 32) {
+    const int64_t g = g0 + tl;
+    if (g >= Tn) break;
+    const float* row = rows[tl];
     float ss = 0.f;
     for (int k = lane; k < R; k += 32) ss = fmaf(row[k], row[k], ss);
 #pragma unroll
     for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if (lane == 0) inv_dt = 1.0f / sqrtf(ss / (float)R + eps);
-  } else if (wi == 1) {
+    const float inv = 1.0f / sqrtf(ss / (float)R + eps);
+    for (int k = lane; k < R; k += 32)
+      dtn[g * R + k] = __float2half_rn(row[k] * inv * (float)wdt[k]);
     const float v = row[R + lane];
     float s2 = v * v;
 #pragma unroll
@@ -350,11 +370,71 @@ __global__ void __launch_bounds__(kNormThreads) k_norms16(
     const float wv = lane < 16 ? (float)wb[lane] : (float)wc[lane - 16];
     bc[g * 2 * kN + lane] = v * inv2 * wv;
   }
-  __syncthreads();
-  if (j < R) dtn[g * R + j] = __float2half_rn(row[j] * inv_dt * (float)wdt[j]);
+}
+
+// One warp per token, for at most 4 splits: every load of the row (9 columns x
+// up to 4 splits per lane) is issued before the sums, which then run in
+// ascending split order; then the norms as in k_norms16.
+template <typename W>
+__global__ void __launch_bounds__(256) k_norms16_warp(
+    const float* __restrict__ part, int ksplit, const W* __restrict__ wdt,
+    const W* __restrict__ wb, const W* __restrict__ wc, int64_t Tn, int R, float eps,
+    __half* __restrict__ dtn, float* __restrict__ bc) {
+  constexpr int kCols = kMaxP / 32;
+  const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
+  const int64_t g = (int64_t)blockIdx.x * 8 + wi;
+  if (g >= Tn) return;
+  const int P = R + 2 * kN;
+  const int64_t stride = Tn * P;
+  float v[kCols][4];
+#pragma unroll
+  for (int jj = 0; jj < kCols; ++jj) {
+    const int j = lane + 32 * jj;
+#pragma unroll
+    for (int sp = 0; sp < 4; ++sp)
+      v[jj][sp] = (j < P && sp < ksplit) ? part[sp * stride + g * P + j] : 0.0f;
+  }
+  float row[kCols];
+#pragma unroll
+  for (int jj = 0; jj < kCols; ++jj) {
+    float acc = v[jj][0];
+#pragma unroll
+    for (int sp = 1; sp < 4; ++sp)
+      if (sp < ksplit) acc += v[jj][sp];
+    row[jj] = acc;
+  }
+  // dt occupies columns [0, R): lanes hold row[jj] for j = lane + 32 jj
+  float ss = 0.f;
+#pragma unroll
+  for (int jj = 0; jj < kCols; ++jj)
+    if (lane + 32 * jj < R) ss = fmaf(row[jj], row[jj], ss);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float inv = 1.0f / sqrtf(ss / (float)R + eps);
+#pragma unroll
+  for (int jj = 0; jj < kCols; ++jj) {
+    const int j = lane + 32 * jj;
+    if (j < R) dtn[g * R + j] = __float2half_rn(row[jj] * inv * (float)wdt[j]);
+  }
+  // B and C occupy columns [R, R + 32): R is a multiple of 8, so pick them up by shuffles
+  float bcv = 0.f;
+#pragma unroll
+  for (int jj = 0; jj < kCols; ++jj) {
+    // column R + lane lives in lane (R + lane) % 32 of slot (R + lane) / 32
+    const int src_j = R + lane;
+    const float t = __shfl_sync(0xffffffffu, row[jj], src_j & 31);
+    if ((src_j >> 5) == jj) bcv = t;
+  }
+  float s2 = bcv * bcv;
+#pragma unroll
+  for (int o = 8; o; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+  const float inv2 = 1.0f / sqrtf(s2 / (float)kN + eps);
+  const float wv = lane < 16 ? (float)wb[lane] : (float)wc[lane - 16];
+  bc[g * 2 * kN + lane] = bcv * inv2 * wv;
 }
 
 // ------------------------------------------------------- fused dt_proj + scan
+
 struct ScanArgs {
   int64_t L, d, T;
   int R, nslab;
@@ -601,7 +681,7 @@ __global__ void __launch_bounds__(kScanThreads, 2)
           xc = fmaf(cw[1], xw[1], xc);
           xc = fmaf(cw[2], xw[2], xc);
           xc = fmaf(cw[3], xt, xc);
-          const float uv = silu_u(xc);
+          const float uv = silu_newton(xc);
           if (g0t + i < nt) {
             xw[0] = xw[1];
             xw[1] = xw[2];
@@ -1002,9 +1082,14 @@ cudaError_t run_fast_fwd(Problem& p) {
     launched(p, "k_xproj");
   }
   // 3. RMSNorms
-  k_norms16<bf16><<<(unsigned)p.T, kNormThreads, 0, s>>>(
-      w.part, w.ksplit, (const bf16*)p.dtn_w, (const bf16*)p.bn_w, (const bf16*)p.cn_w, p.T, (int)p.R, p.eps,
-      w.dtn, w.bc);
+  if (w.ksplit <= 4)
+    k_norms16_warp<bf16><<<(unsigned)((p.T + 7) / 8), 256, 0, s>>>(
+        w.part, w.ksplit, (const bf16*)p.dtn_w, (const bf16*)p.bn_w, (const bf16*)p.cn_w, p.T,
+        (int)p.R, p.eps, w.dtn, w.bc);
+  else
+    k_norms16<bf16, 1><<<(unsigned)p.T, kNormThreads, 0, s>>>(
+        w.part, w.ksplit, (const bf16*)p.dtn_w, (const bf16*)p.bn_w, (const bf16*)p.cn_w, p.T,
+        (int)p.R, p.eps, w.dtn, w.bc);
   launched(p, "k_norms16");
   // 4. dt_proj + scan + gate
   if (p.decode) {

@@ -58,3 +58,21 @@ def test_log1p_polynomial():
     ref = np.log1p(w.astype(np.float64))
     ok = w > 0
     assert (np.abs(val[ok] - ref[ok]) / ref[ok]).max() < 3e-7
+
+
+def test_newton_reciprocal():
+    c = header_consts_int()
+    K = c["RCP_MAGIC"]
+    den = np.concatenate([np.linspace(1, 2, 100001), np.geomspace(1, 8.5e37, 200001)]).astype(
+        np.float32)
+    r = (np.int64(K) - den.view(np.int32).astype(np.int64)).astype(np.int32).view(np.float32)
+    for _ in range(3):   # r * fma(-den, r, 2): the fma is exact to one rounding in float64 here
+        e = (2.0 - den.astype(np.float64) * r.astype(np.float64)).astype(np.float32)
+        r = (r * e).astype(np.float32)
+    rel = np.abs(r.astype(np.float64) * den.astype(np.float64) - 1)
+    assert rel.max() < 2e-7, rel.max()
+
+
+def header_consts_int():
+    src = open(HDR).read()
+    return {k: int(v, 16) for k, v in re.findall(r"constexpr int (\w+) = (0x[0-9a-fA-F]+);", src)}
