@@ -266,19 +266,17 @@ def main():
 
     import torch
     import torch.distributed as dist
-    from mamba_selective_scan_jamba_b200 import devio, jmix
+    from mamba_selective_scan_jamba_b200 import devio, jmix, replicas
 
     torch.cuda.set_device(local)
     if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        replicas.init("nccl", 120.0, torch.device("cuda", local))
     P = peaks()
     # weak scaling: rank r owns sequences r*B .. r*B+B-1 of a world*B batch
     w = base
     wall = base.with_(batch=base.batch * world)
     W = synth.make_weights(w)
-    A = synth.make_activations(wall, rank * w.batch, (rank + 1) * w.batch)
+    A = synth.make_activations(wall, *replicas.shard(w.batch, rank))
     dev = torch.device("cuda", local)
     Wd = devio.weights_to_device(W, dev)
     x = devio.to_device(A["x"], dev)
@@ -321,8 +319,7 @@ def main():
     sampler = ClockSampler(gpu_id)
     time.sleep(0.6)   # let the sampler start
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
+    replicas.barrier()
     torch.cuda.synchronize(dev)
     t_wall0 = time.time()
     launches = 0
@@ -337,8 +334,7 @@ def main():
     stream.synchronize()
     torch.cuda.synchronize(dev)
     t_wall1 = time.time()
-    if world > 1:
-        dist.barrier()
+    replicas.barrier()
     time.sleep(0.3)
     sampler.stop()
     clocks = sampler.summary(t_wall0, t_wall1)
@@ -346,12 +342,9 @@ def main():
     ms = start.elapsed_time(end) / K
     per_kernel = [sum(evs[i][k].elapsed_time(evs[i][k + 1]) for i in range(K)) / K
                   for k in range(nk)]
-    if world > 1:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = replicas.max_over_ranks(ms, dev)
     tokens_rank = w.batch * w.seqlen
-    value = tokens_rank * world / (ms / 1e3)
+    value = replicas.job_rate(tokens_rank, world, ms)
 
     # roofline of the dominant kernel
     kd = max(range(nk), key=lambda k: per_kernel[k])
@@ -376,7 +369,7 @@ def main():
                                 if bound == "alu" else f"{P['src']} MEASURED_PEAKS.json"),
                 "kernel_ms": per_kernel[kd],
                 "kernels_ms": {names[k]: round(per_kernel[k], 4) for k in range(nk)},
-                "north_star": {"roofline_tokens_per_s": roof_tok_s,
+                "step_roofline": {"roofline_tokens_per_s": roof_tok_s,
                                "frac": value / world / roof_tok_s,
                                "definition": "max(tc_flop/bf16 sustained peak, bytes/HBM) "
                                              "per token, bytes = x,z in + y out"}}
@@ -405,8 +398,7 @@ def main():
         with torch.cuda.stream(stream):
             e2e_step()
         stream.synchronize()
-        if world > 1:
-            dist.barrier()
+        replicas.barrier()
         s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
             s2.record(stream)
@@ -414,12 +406,8 @@ def main():
                 e2e_step()
             e2.record(stream)
         stream.synchronize()
-        ems = s2.elapsed_time(e2) / Ke
-        if world > 1:
-            t = torch.tensor([ems], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        line["e2e"] = {"value": tokens_rank * world / (ems / 1e3), "unit": "tokens/s",
+        ems = replicas.max_over_ranks(s2.elapsed_time(e2) / Ke, dev)
+        line["e2e"] = {"value": replicas.job_rate(tokens_rank, world, ems), "unit": "tokens/s",
                        "h2d_bytes_per_step": in_bytes,
                        "d2h_bytes_per_step": y.numel() * y.element_size() + fs.numel() * 4,
                        "ms_per_step": ems, "steps": Ke,
@@ -436,7 +424,7 @@ def main():
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
-        dist.barrier()
+        replicas.barrier()
         dist.destroy_process_group()
 
 

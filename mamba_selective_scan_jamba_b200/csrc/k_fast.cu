@@ -451,7 +451,58 @@ struct ScanArgs {
   const bf16* hist;
   bf16* final_conv;
   ErrFlags* err;
+  // Work schedule (see k_scan_fused).  A pair is one (sequence, 128-channel
+  // tile); each pair's sequence is cut into n_parts time parts of whole chunks.
+  int n_tiles;     // channel tiles per sequence
+  int n_parts;     // time parts per sequence
+  int two_pass;    // 0: parts run in a chain; 1: state pass, then output pass
+  int* counter;    // next unit to claim
+  int* flags;      // [pairs * n_parts]: nonzero once that part's hand-over is written
+  float* carry_h;  // [pairs * n_parts, 128, 16]: a part's end state
+  float* carry_s;  // [pairs * n_parts, 128]: a part's sum of delta (two-pass)
 };
+
+// How the scan kernel cuts the work (host side; also sizes the workspace).
+struct ScanPlan {
+  int n_parts = 1;
+  int two_pass = 0;
+};
+
+// Two CTAs of the scan kernel fit on each of a B200's 148 SMs.
+constexpr int kScanSlots = 296;
+// A time part spans at least this many 16-token chunks.
+constexpr int kMinPartChunks = 16;
+
+ScanPlan scan_plan(int64_t B, int64_t L, int64_t d) {
+  ScanPlan pl;
+  const int64_t pairs = B * ((d + kSC - 1) / kSC);
+  const int64_t nch = (L + kSQ - 1) / kSQ;
+  if (pairs <= 0 || nch <= 0) return pl;
+  if (pairs >= kScanSlots / 2) {
+    // Enough pairs to fill the GPU: parts only even out the last wave.  A part
+    // then starts from the state of the part before it (a chain), which costs
+    // no extra arithmetic.  Waves of part-sized units: ceil(pairs*P/slots)/P.
+    int64_t best_num = (pairs + kScanSlots - 1) / kScanSlots, best_den = 1;
+    for (int P = 2; P <= 8; P *= 2) {
+      if (nch < (int64_t)kMinPartChunks * P) break;
+      const int64_t num = (pairs * P + kScanSlots - 1) / kScanSlots;
+      if (num * best_den < best_num * P) {
+        best_num = num;
+        best_den = P;
+        pl.n_parts = P;
+      }
+    }
+  } else {
+    // Too few pairs for the GPU: a state pass over parts 0..P-2 (from a zero
+    // state) runs side by side, then every part produces its outputs from the
+    // state that the earlier parts' results fold into.
+    int P = 8;
+    while (P > 1 && nch < (int64_t)kMinPartChunks * P) P /= 2;
+    pl.n_parts = P;
+    pl.two_pass = P > 1;
+  }
+  return pl;
+}
 
 constexpr int kScanThreads = 160;  // warps 0..3: one channel per thread; warp 4: TMA + MMA
 constexpr int kWdtBytes = kMaxSlabs * kSC * 128;                  // 64 KB
@@ -477,36 +528,6 @@ __device__ __forceinline__ float softplus_fast(float v) {
   return fmaf(w, q, fmaxf(v, 0.0f));
 }
 
-
-
-// 2^x for a pair of x <= 0 on the FMA pipe: exact base-2 range reduction
-// x = j + f (j = round(x), |f| <= 1/2, via the 1.5*2^23 rounding constant),
-// 2^f by the degree-6 minimax polynomial, and 2^j added into the exponent
-// field.  x is clamped at -126 (results below 2^-126 are flushed anyway).
-__device__ __forceinline__ float2 exp2_pair_fma(float2 x) {
-  const float kRound = 12582912.0f;  // 1.5 * 2^23
-  x.x = fmaxf(x.x, -126.0f);
-  x.y = fmaxf(x.y, -126.0f);
-  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
-  const float2 j = __fadd2_rn(t, make_float2(-kRound, -kRound));
-  const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), x);
-  float2 p = make_float2(poly::E6, poly::E6);
-  p = __ffma2_rn(p, f, make_float2(poly::E5, poly::E5));
-  p = __ffma2_rn(p, f, make_float2(poly::E4, poly::E4));
-  p = __ffma2_rn(p, f, make_float2(poly::E3, poly::E3));
-  p = __ffma2_rn(p, f, make_float2(poly::E2, poly::E2));
-  p = __ffma2_rn(p, f, make_float2(poly::E1, poly::E1));
-  p = __ffma2_rn(p, f, make_float2(poly::E0, poly::E0));
-  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
-}
-
-#ifndef JMIX_SW_PAIRS
-#define JMIX_SW_PAIRS 0
-#endif
-// State pairs (of 8) whose decay is computed on the FMA pipe instead of MUFU;
-// balances the two pipes (16 MUFU ex2 / clk / SM against 128 FMA / clk / SM).
-constexpr int kSwPairs = JMIX_SW_PAIRS;
 #ifndef JMIX_SCAN_G
 #define JMIX_SCAN_G 8
 #endif
@@ -525,6 +546,150 @@ __device__ __forceinline__ float silu_gate(float z) {
   return fmaf(hz, tanh_approx(hz), hz);
 }
 
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Waits (bounded) until *flag is nonzero; one thread calls it.
+__device__ __forceinline__ void wait_flag(const int* flag, ErrFlags* err, unsigned site) {
+  if (ld_acquire_gpu(flag)) return;
+  const uint64_t t0 = globaltimer_ns();
+  while (!ld_acquire_gpu(flag)) {
+    __nanosleep(64);
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (atomicExch(&err->timeout, 1u) == 0u) err->where = site;
+      return;
+    }
+  }
+}
+
+// The compute warps' share of one unit: chunks [kb, kb + nch) of the pair's
+// sequence.  kOut: produce y (else only the state and the sum of delta).
+template <bool kOut>
+__device__ __forceinline__ void scan_chunks(const ScanArgs& a, const uint8_t* stage0,
+                                            uint64_t* full, uint64_t* mma_done, uint64_t* empty,
+                                            uint32_t tmem, int warp, int lane, int kg0, int kb,
+                                            int nch, bool cok, bf16* yrow, float2 (&h)[kN / 2],
+                                            const float2 (&A2)[kN / 2], float (&xw)[kConv - 1],
+                                            const float (&cw)[kConv], float cb, float bias,
+                                            float Dc, float& ssum) {
+  const int cl = warp * 32 + lane;
+  for (int k = 0; k < nch; ++k) {
+    const int kg = kg0 + k;
+    const int s = kg & 1;
+    const uint32_t ph = (uint32_t)(kg >> 1) & 1u;
+    if (!mbar_wait(smem_u32(&mma_done[s]), ph, a.err, 25)) break;
+    if (!mbar_wait(smem_u32(&full[s]), ph, a.err, 26)) break;
+    tc_fence_after();
+    const uint8_t* st = stage0 + s * kStageBytes;
+    const bf16* xs = reinterpret_cast<const bf16*>(st + kDtnStage);
+    const bf16* zs = reinterpret_cast<const bf16*>(st + kDtnStage + kXStage);
+    const float4* bcs = reinterpret_cast<const float4*>(st + kDtnStage + 2 * kXStage);
+    const int64_t tbase = (int64_t)(kb + k) * kSQ;
+    const int nt = (int)((a.L - tbase) < kSQ ? (a.L - tbase) : kSQ);
+    const uint32_t tacc = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(s * kSQ);
+    float csum = 0.0f;
+#pragma unroll 1
+    for (int g0t = 0; g0t < nt; g0t += kG) {
+      uint32_t r[kG];
+      tmem_ld_cols<kG>(tacc + (uint32_t)g0t, r);
+      tmem_ld_wait();
+      // per-token terms: u = SiLU(conv) in float32, delta, delta*u, D*u, SiLU(z)
+      float dl[kG], du[kG], dsk[kG], gz[kG];
+#pragma unroll
+      for (int i = 0; i < kG; ++i) {
+        const float xt = bf(xs[(g0t + i) * kSC + cl]);
+        float xc = fmaf(cw[0], xw[0], cb);
+        xc = fmaf(cw[1], xw[1], xc);
+        xc = fmaf(cw[2], xw[2], xc);
+        xc = fmaf(cw[3], xt, xc);
+        const float uv = silu_newton(xc);
+        const bool live = g0t + i < nt;
+        if (live) {
+          xw[0] = xw[1];
+          xw[1] = xw[2];
+          xw[2] = xt;
+        }
+        dl[i] = softplus_fast(__uint_as_float(r[i]) + bias);
+        du[i] = dl[i] * uv;
+        if constexpr (kOut) {
+          dsk[i] = Dc * uv;
+          gz[i] = silu_gate(bf(zs[(g0t + i) * kSC + cl]));
+        } else {
+          csum += live ? dl[i] : 0.0f;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < kG; ++i) {
+        const int t = g0t + i;
+        if (t >= nt) break;
+        const float2 dl2 = make_float2(dl[i], dl[i]);
+        const float2 du2 = make_float2(du[i], du[i]);
+        float2 acc[4];
+#pragma unroll
+        for (int q4 = 0; q4 < kN / 4; ++q4) {
+          const float4 Bq = bcs[t * 8 + q4];
+          float4 Cq;
+          if constexpr (kOut) Cq = bcs[t * 8 + 4 + q4];
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const int q = q4 * 2 + half;
+            const float2 Bp = half ? make_float2(Bq.z, Bq.w) : make_float2(Bq.x, Bq.y);
+            const float2 x = __fmul2_rn(dl2, A2[q]);
+            float2 da;
+            da.x = ex2_approx(x.x);
+            da.y = ex2_approx(x.y);
+            h[q] = __ffma2_rn(da, h[q], __fmul2_rn(du2, Bp));
+            if constexpr (kOut) {
+              // four independent partial sums of C.h (short dependency chains)
+              const float2 Cp = half ? make_float2(Cq.z, Cq.w) : make_float2(Cq.x, Cq.y);
+              acc[q4] = half ? __ffma2_rn(Cp, h[q], acc[q4]) : __fmul2_rn(Cp, h[q]);
+            }
+          }
+        }
+        if constexpr (kOut) {
+          const float2 s01 = __fadd2_rn(acc[0], acc[1]);
+          const float2 s23 = __fadd2_rn(acc[2], acc[3]);
+          const float2 sa = __fadd2_rn(s01, s23);
+          const float ys = (sa.x + sa.y) + dsk[i];
+          if (cok) yrow[(tbase + t) * a.d] = __float2bfloat16_rn(ys * gz[i]);
+        }
+      }
+    }
+    if constexpr (!kOut) ssum += csum;
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
+  }
+}
+
+// Fused dt_proj (tcgen05, accumulator in TMEM) + softplus + selective scan +
+// D skip + SiLU(z) gate, with the causal conv + SiLU recomputed in fp32 from x.
+//
+// Persistent CTAs (two per SM) claim units from a counter.  A unit is one
+// time part of one pair (sequence, 128-channel tile); warp 4 streams its
+// chunks (dt_n, x, z, B/C rows) by TMA and issues the dt_proj MMAs, warps 0..3
+// run the recurrence with one channel per thread.
+//   chain (two_pass = 0): parts of a pair run in order, each starting from the
+//     end state that the part before it hands over.
+//   two-pass: state units for parts 0..P-2 run the recurrence from a zero
+//     state (part 0: from the initial state) and record the end state and the
+//     sum S of delta; the output unit of part p starts from the fold of parts
+//     0..p-1: h <- exp(A S_q) h + h_end_q, since the state map of a part is
+//     h -> exp(A S) h + h_end(zero start), A being constant over time.
+// Every unit that waits waits only for units that come before it in claim
+// order, and a claimed unit is running or queued behind one with a smaller
+// index on its CTA, so every wait ends; each is still bounded (2 s).
 __global__ void __launch_bounds__(kScanThreads, 2)
     k_scan_fused(const __grid_constant__ CUtensorMap tm_wdt,
                  const __grid_constant__ CUtensorMap tm_dtn,
@@ -541,12 +706,15 @@ __global__ void __launch_bounds__(kScanThreads, 2)
   uint64_t* empty = bars + 4;     // [2] compute warps done with the stage / accumulator
   uint64_t* wfull = bars + 6;     // W_dt tile landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 7);
+  volatile int* unit_slot = reinterpret_cast<volatile int*>(bars + 8);  // [2] claimed units
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t c0 = (int64_t)blockIdx.x * kSC;
-  const int64_t b = blockIdx.y;
-  const int64_t g0 = b * a.L;
-  const int nch = (int)((a.L + kSQ - 1) / kSQ);
+  const int nch_all = (int)((a.L + kSQ - 1) / kSQ);
+  const int64_t B = a.T / a.L;
+  const int pairs = a.n_tiles * (int)B;
+  const int P = a.n_parts;
+  const int n_state = a.two_pass ? pairs * (P - 1) : 0;  // state units come first
+  const int n_units = n_state + pairs * P;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 2; ++s) {
@@ -556,6 +724,7 @@ __global__ void __launch_bounds__(kScanThreads, 2)
     }
     mbar_init(smem_u32(wfull), 1);
     fence_mbar_init();
+    unit_slot[0] = atomicAdd(a.counter, 1);
   }
   if (warp == 4) {
     tmem_alloc(smem_u32(tmem_slot), 2 * kSQ);
@@ -566,185 +735,180 @@ __global__ void __launch_bounds__(kScanThreads, 2)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  auto stage_ptr = [&](int s) { return stage0 + s * kStageBytes; };
+  int kg0 = 0;    // chunks this CTA has run before the current unit (mbarrier phases)
+  int nw = 0;     // W_dt tiles this CTA has loaded (wfull phase)
+  for (int it = 0;; ++it) {
+    const int unit = unit_slot[it & 1];
+    if (unit >= n_units) break;
+    // claim the next unit early, so that its number is ready when this one ends
+    if (threadIdx.x == 128)
+      unit_slot[(it + 1) & 1] = *(volatile unsigned*)&a.err->timeout ? n_units
+                                                                      : atomicAdd(a.counter, 1);
+    const bool out = unit >= n_state;
+    const int uu = out ? unit - n_state : unit;
+    const int part = uu / pairs;
+    const int pair = uu - part * pairs;
+    const int64_t b = pair / a.n_tiles;
+    const int tile = pair - (int)b * a.n_tiles;
+    const int64_t c0 = (int64_t)tile * kSC;
+    const int64_t g0 = b * a.L;
+    const int kb = (int)((int64_t)nch_all * part / P);
+    const int nch = (int)((int64_t)nch_all * (part + 1) / P) - kb;
+    const int64_t hslot = (int64_t)pair * P + part;  // this part's hand-over slot
 
-  if (warp == 4) {
-    if (lane == 0) {
-      prefetch_tmap(&tm_wdt);
-      prefetch_tmap(&tm_dtn);
-      prefetch_tmap(&tm_bc);
-      prefetch_tmap(&tm_x);
-      prefetch_tmap(&tm_z);
-      const uint32_t wb = smem_u32(wfull);
-      mbar_arrive_expect_tx(wb, (uint32_t)(a.nslab * kSC * 128));
-      for (int j = 0; j < a.nslab; ++j)
-        tma_load_2d(smem_u32(wdt_s + j * kSC * 128), &tm_wdt, wb, j * 64, (int32_t)c0);
-      const uint32_t stage_tx = (uint32_t)(a.nslab * kSQ * 128 + 2 * kXStage + kBCStage);
-      auto issue_stage = [&](int k) {
-        const int s = k & 1;
-        uint8_t* st = stage_ptr(s);
-        const uint32_t fb = smem_u32(&full[s]);
-        const int32_t row = (int32_t)(g0 + (int64_t)k * kSQ);
-        mbar_arrive_expect_tx(fb, stage_tx);
+    if (warp == 4) {
+      if (lane == 0 && nch > 0) {
+        const uint32_t wb = smem_u32(wfull);
+        mbar_arrive_expect_tx(wb, (uint32_t)(a.nslab * kSC * 128));
         for (int j = 0; j < a.nslab; ++j)
-          tma_load_2d(smem_u32(st + j * kSQ * 128), &tm_dtn, fb, j * 64, row);
-        tma_load_2d(smem_u32(st + kDtnStage), &tm_x, fb, (int32_t)c0, row);
-        tma_load_2d(smem_u32(st + kDtnStage + kXStage), &tm_z, fb, (int32_t)c0, row);
-        tma_load_2d(smem_u32(st + kDtnStage + 2 * kXStage), &tm_bc, fb, 0, row);
-      };
-      const uint32_t idesc = idesc_f16_f32(kSC, kSQ);
-      auto issue_mma = [&](int k) -> bool {
-        const int s = k & 1;
-        if (!mbar_wait(smem_u32(&full[s]), (uint32_t)(k >> 1) & 1u, a.err, 22)) return false;
-        tc_fence_after();
-        const uint32_t wbase = smem_u32(wdt_s), db = smem_u32(stage_ptr(s));
-        const uint32_t d_tmem = tmem + (uint32_t)(s * kSQ);
-        for (int j = 0; j < a.nslab; ++j)
+          tma_load_2d(smem_u32(wdt_s + j * kSC * 128), &tm_wdt, wb, j * 64, (int32_t)c0);
+        const uint32_t stage_tx =
+            (uint32_t)(a.nslab * kSQ * 128 + (out ? 2 : 1) * kXStage + kBCStage);
+        auto issue_stage = [&](int k) {  // k: chunk of this unit
+          const int s = (kg0 + k) & 1;
+          uint8_t* st = stage0 + s * kStageBytes;
+          const uint32_t fb = smem_u32(&full[s]);
+          const int32_t row = (int32_t)(g0 + (int64_t)(kb + k) * kSQ);
+          mbar_arrive_expect_tx(fb, stage_tx);
+          for (int j = 0; j < a.nslab; ++j)
+            tma_load_2d(smem_u32(st + j * kSQ * 128), &tm_dtn, fb, j * 64, row);
+          tma_load_2d(smem_u32(st + kDtnStage), &tm_x, fb, (int32_t)c0, row);
+          if (out) tma_load_2d(smem_u32(st + kDtnStage + kXStage), &tm_z, fb, (int32_t)c0, row);
+          tma_load_2d(smem_u32(st + kDtnStage + 2 * kXStage), &tm_bc, fb, 0, row);
+        };
+        const uint32_t idesc = idesc_f16_f32(kSC, kSQ);
+        auto issue_mma = [&](int k) -> bool {
+          const int kg = kg0 + k;
+          const int s = kg & 1;
+          if (!mbar_wait(smem_u32(&full[s]), (uint32_t)(kg >> 1) & 1u, a.err, 22)) return false;
+          tc_fence_after();
+          const uint32_t wbase = smem_u32(wdt_s), db = smem_u32(stage0 + s * kStageBytes);
+          const uint32_t d_tmem = tmem + (uint32_t)(s * kSQ);
+          for (int j = 0; j < a.nslab; ++j)
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            umma_f16(d_tmem, sw128_kmajor_desc(wbase + j * kSC * 128 + kk * 32),
-                     sw128_kmajor_desc(db + j * kSQ * 128 + kk * 32), idesc,
-                     (j > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(smem_u32(&mma_done[s]));
-        return true;
-      };
-      bool ok = mbar_wait(wb, 0, a.err, 21);
-      if (ok) {
+            for (int kk = 0; kk < 4; ++kk)
+              umma_f16(d_tmem, sw128_kmajor_desc(wbase + j * kSC * 128 + kk * 32),
+                       sw128_kmajor_desc(db + j * kSQ * 128 + kk * 32), idesc,
+                       (j > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(smem_u32(&mma_done[s]));
+          return true;
+        };
+        // Both stages and accumulators are free here: the previous unit ended
+        // with every compute warp past its last chunk (CTA barrier below).
         issue_stage(0);
         if (nch > 1) issue_stage(1);
-        ok = issue_mma(0);
-      }
-      for (int k = 0; ok && k < nch; ++k) {
-        if (k + 1 < nch) {
-          // accumulator (k+1)&1 was last read by the compute warps for chunk k-1
-          if (k >= 1 && !mbar_wait(smem_u32(&empty[(k + 1) & 1]), (uint32_t)((k - 1) >> 1) & 1u,
-                                   a.err, 23))
-            break;
-          if (!issue_mma(k + 1)) break;
-        }
-        if (k + 2 < nch) {
-          // stage k&1 (dt_n read by MMA k, B/C read by chunk k) is free after chunk k
-          if (!mbar_wait(smem_u32(&empty[k & 1]), (uint32_t)(k >> 1) & 1u, a.err, 24)) break;
-          issue_stage(k + 2);
-        }
-      }
-    }
-  } else {
-    // compute warps: thread = channel c0 + 32*warp + lane = TMEM lane; its 16
-    // states live in registers as 8 float2 pairs, and so does the conv window.
-    // x and z are read straight from global memory one token group ahead.
-    const int cl = warp * 32 + lane;
-    const int64_t c = c0 + cl;
-    const bool cok = c < a.d;
-    float2 A2[kN / 2], h[kN / 2];
-#pragma unroll
-    for (int q = 0; q < kN / 2; ++q) {
-      A2[q].x = cok ? -expf(a.A_log[c * kN + 2 * q]) * kLog2e : 0.0f;
-      A2[q].y = cok ? -expf(a.A_log[c * kN + 2 * q + 1]) * kLog2e : 0.0f;
-      h[q].x = (cok && a.h0) ? a.h0[(b * a.d + c) * kN + 2 * q] : 0.0f;
-      h[q].y = (cok && a.h0) ? a.h0[(b * a.d + c) * kN + 2 * q + 1] : 0.0f;
-    }
-    const float bias = cok ? a.dt_bias[c] : 0.0f;
-    const float Dc = cok ? a.D[c] : 0.0f;
-    float cw[kConv], xw[kConv - 1];
-#pragma unroll
-    for (int k = 0; k < kConv; ++k) cw[k] = cok ? bf(a.conv_w[c * kConv + k]) : 0.0f;
-    const float cb = cok ? bf(a.conv_b[c]) : 0.0f;
-#pragma unroll
-    for (int k = 0; k < kConv - 1; ++k)
-      xw[k] = (cok && a.hist) ? bf(a.hist[(b * a.d + c) * (kConv - 1) + k]) : 0.0f;
-    bf16* yrow = a.y + g0 * a.d + c;
-    for (int k = 0; k < nch; ++k) {
-      const int s = k & 1;
-      const uint32_t ph = (uint32_t)(k >> 1) & 1u;
-      if (!mbar_wait(smem_u32(&mma_done[s]), ph, a.err, 25)) break;
-      if (!mbar_wait(smem_u32(&full[s]), ph, a.err, 26)) break;
-      tc_fence_after();
-      const uint8_t* st = stage_ptr(s);
-      const bf16* xs = reinterpret_cast<const bf16*>(st + kDtnStage);
-      const bf16* zs = reinterpret_cast<const bf16*>(st + kDtnStage + kXStage);
-      const float4* bcs = reinterpret_cast<const float4*>(st + kDtnStage + 2 * kXStage);
-      const int64_t tbase = (int64_t)k * kSQ;
-      const int nt = (int)((a.L - tbase) < kSQ ? (a.L - tbase) : kSQ);
-      const uint32_t tacc = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(s * kSQ);
-#pragma unroll 1
-      for (int g0t = 0; g0t < nt; g0t += kG) {
-        uint32_t r[kG];
-        tmem_ld_cols<kG>(tacc + (uint32_t)g0t, r);
-        tmem_ld_wait();
-        // per-token terms: u = SiLU(conv) in float32, delta, delta*u, D*u, SiLU(z)
-        float dl[kG], du[kG], dsk[kG], gz[kG];
-#pragma unroll
-        for (int i = 0; i < kG; ++i) {
-          const float xt = bf(xs[(g0t + i) * kSC + cl]);
-          float xc = fmaf(cw[0], xw[0], cb);
-          xc = fmaf(cw[1], xw[1], xc);
-          xc = fmaf(cw[2], xw[2], xc);
-          xc = fmaf(cw[3], xt, xc);
-          const float uv = silu_newton(xc);
-          if (g0t + i < nt) {
-            xw[0] = xw[1];
-            xw[1] = xw[2];
-            xw[2] = xt;
+        bool ok = mbar_wait(wb, (uint32_t)nw & 1u, a.err, 21);
+        if (ok) ok = issue_mma(0);
+        for (int k = 0; ok && k < nch; ++k) {
+          const int kg = kg0 + k;
+          if (k + 1 < nch) {
+            if (k >= 1 && !mbar_wait(smem_u32(&empty[(kg + 1) & 1]),
+                                     (uint32_t)((kg - 1) >> 1) & 1u, a.err, 23))
+              break;
+            if (!issue_mma(k + 1)) break;
           }
-          dl[i] = softplus_fast(__uint_as_float(r[i]) + bias);
-          du[i] = dl[i] * uv;
-          dsk[i] = Dc * uv;
-          gz[i] = silu_gate(bf(zs[(g0t + i) * kSC + cl]));
-        }
-#pragma unroll
-        for (int i = 0; i < kG; ++i) {
-          const int t = g0t + i;
-          if (t >= nt) break;
-          const float2 dl2 = make_float2(dl[i], dl[i]);
-          const float2 du2 = make_float2(du[i], du[i]);
-          float2 acc[4];
-#pragma unroll
-          for (int q4 = 0; q4 < kN / 4; ++q4) {
-            const float4 Bq = bcs[t * 8 + q4];
-            const float4 Cq = bcs[t * 8 + 4 + q4];
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-              const int q = q4 * 2 + half;
-              const float2 Bp = half ? make_float2(Bq.z, Bq.w) : make_float2(Bq.x, Bq.y);
-              const float2 Cp = half ? make_float2(Cq.z, Cq.w) : make_float2(Cq.x, Cq.y);
-              const float2 x = __fmul2_rn(dl2, A2[q]);
-              float2 da;
-              if (q >= kN / 2 - kSwPairs) {
-                da = exp2_pair_fma(x);
-              } else {
-                da.x = ex2_approx(x.x);
-                da.y = ex2_approx(x.y);
-              }
-              h[q] = __ffma2_rn(da, h[q], __fmul2_rn(du2, Bp));
-              // four independent partial sums of C.h (short dependency chains)
-              acc[q4] = half ? __ffma2_rn(Cp, h[q], acc[q4]) : __fmul2_rn(Cp, h[q]);
-            }
+          if (k + 2 < nch) {
+            if (!mbar_wait(smem_u32(&empty[kg & 1]), (uint32_t)(kg >> 1) & 1u, a.err, 24)) break;
+            issue_stage(k + 2);
           }
-          const float2 s01 = __fadd2_rn(acc[0], acc[1]);
-          const float2 s23 = __fadd2_rn(acc[2], acc[3]);
-          const float2 sa = __fadd2_rn(s01, s23);
-          const float ys = (sa.x + sa.y) + dsk[i];
-          if (cok) yrow[(tbase + t) * a.d] = __float2bfloat16_rn(ys * gz[i]);
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
-    }
-    if (cok) {
+    } else {
+      // compute warps: thread = channel c0 + 32*warp + lane = TMEM lane
+      const int cl = warp * 32 + lane;
+      const int64_t c = c0 + cl;
+      const bool cok = c < a.d;
+      // a unit that starts from earlier parts waits (bounded) for their hand-over
+      const int n_wait = part == 0 ? 0 : (a.two_pass ? (out ? part : 0) : 1);
+      if (n_wait > 0) {
+        if (threadIdx.x == 0) {
+          for (int q = part - n_wait; q < part; ++q)
+            wait_flag(a.flags + (int64_t)pair * P + q, a.err, 28);
+          __threadfence();
+        }
+        named_bar_sync(1, 128);
+      }
+      float2 A2[kN / 2], h[kN / 2];
 #pragma unroll
       for (int q = 0; q < kN / 2; ++q) {
-        a.hT[(b * a.d + c) * kN + 2 * q] = h[q].x;
-        a.hT[(b * a.d + c) * kN + 2 * q + 1] = h[q].y;
+        A2[q].x = cok ? -expf(a.A_log[c * kN + 2 * q]) * kLog2e : 0.0f;
+        A2[q].y = cok ? -expf(a.A_log[c * kN + 2 * q + 1]) * kLog2e : 0.0f;
+        h[q] = make_float2(0.0f, 0.0f);
+        if (part == 0 && cok && a.h0) {
+          h[q].x = a.h0[(b * a.d + c) * kN + 2 * q];
+          h[q].y = a.h0[(b * a.d + c) * kN + 2 * q + 1];
+        }
       }
-      // the conv window now holds the last d_conv-1 inputs (exact bf16 values)
-      if (a.final_conv) {
+      if (n_wait > 0) {
+        const float* ch = a.carry_h + ((int64_t)pair * P + (part - n_wait)) * kSC * kN + cl * kN;
 #pragma unroll
-        for (int k = 0; k < kConv - 1; ++k)
-          a.final_conv[(b * a.d + c) * (kConv - 1) + k] = __float2bfloat16_rn(xw[k]);
+        for (int q = 0; q < kN / 2; ++q) h[q] = __ldcg(reinterpret_cast<const float2*>(ch) + q);
+        // two-pass: fold in parts 1..p-1 (h <- exp2(A2 S) h + h_end)
+        for (int qp = part - n_wait + 1; qp < part; ++qp) {
+          const int64_t sl = (int64_t)pair * P + qp;
+          const float S = __ldcg(a.carry_s + sl * kSC + cl);
+          const float2* he = reinterpret_cast<const float2*>(a.carry_h + sl * kSC * kN + cl * kN);
+#pragma unroll
+          for (int q = 0; q < kN / 2; ++q) {
+            const float2 e = __ldcg(he + q);
+            h[q].x = fmaf(ex2_approx(A2[q].x * S), h[q].x, e.x);
+            h[q].y = fmaf(ex2_approx(A2[q].y * S), h[q].y, e.y);
+          }
+        }
+      }
+      const float bias = cok ? a.dt_bias[c] : 0.0f;
+      const float Dc = cok ? a.D[c] : 0.0f;
+      float cw[kConv], xw[kConv - 1];
+#pragma unroll
+      for (int k = 0; k < kConv; ++k) cw[k] = cok ? bf(a.conv_w[c * kConv + k]) : 0.0f;
+      const float cb = cok ? bf(a.conv_b[c]) : 0.0f;
+      // conv window: the d_conv-1 inputs before the unit's first token
+      const int64_t t0 = (int64_t)kb * kSQ;
+#pragma unroll
+      for (int k = 0; k < kConv - 1; ++k) {
+        const int64_t t = t0 - (kConv - 1) + k;
+        xw[k] = !cok ? 0.0f
+                : t >= 0 ? bf(a.x[(g0 + t) * a.d + c])
+                : a.hist ? bf(a.hist[(b * a.d + c) * (kConv - 1) + (kConv - 1 + t)])
+                         : 0.0f;
+      }
+      float ssum = 0.0f;
+      if (out)
+        scan_chunks<true>(a, stage0, full, mma_done, empty, tmem, warp, lane, kg0, kb, nch, cok,
+                          a.y + g0 * a.d + c, h, A2, xw, cw, cb, bias, Dc, ssum);
+      else
+        scan_chunks<false>(a, stage0, full, mma_done, empty, tmem, warp, lane, kg0, kb, nch, cok,
+                           nullptr, h, A2, xw, cw, cb, bias, Dc, ssum);
+      if (part + 1 < P && (!out || !a.two_pass)) {
+        // hand the end state (and, two-pass, the sum of delta) to later parts
+        float* ch = a.carry_h + hslot * kSC * kN + cl * kN;
+#pragma unroll
+        for (int q = 0; q < kN / 2; ++q) reinterpret_cast<float2*>(ch)[q] = h[q];
+        if (!out) a.carry_s[hslot * kSC + cl] = ssum;
+        __threadfence();
+        named_bar_sync(1, 128);
+        if (threadIdx.x == 0) st_release_gpu(a.flags + hslot, 1);
+      } else if (out && part + 1 == P && cok) {
+#pragma unroll
+        for (int q = 0; q < kN / 2; ++q) {
+          a.hT[(b * a.d + c) * kN + 2 * q] = h[q].x;
+          a.hT[(b * a.d + c) * kN + 2 * q + 1] = h[q].y;
+        }
+        // the conv window now holds the last d_conv-1 inputs (exact bf16 values)
+        if (a.final_conv) {
+#pragma unroll
+          for (int k = 0; k < kConv - 1; ++k)
+            a.final_conv[(b * a.d + c) * (kConv - 1) + k] = __float2bfloat16_rn(xw[k]);
+        }
       }
     }
+    kg0 += nch;
+    nw += nch > 0 ? 1 : 0;
+    __syncthreads();
+    // stop claiming work once any wait has given up
+    if (threadIdx.x == 128 && *(volatile unsigned*)&a.err->timeout)
+      unit_slot[(it + 1) & 1] = n_units;
+    __syncthreads();
   }
   tc_fence_before();
   __syncthreads();
@@ -993,7 +1157,12 @@ struct FastWs {
   float* bc;
   __half* wx;
   __half* wdt;
+  int* sched;         // [0] unit counter, [1..] hand-over flags of the scan's parts
+  float* carry_h;     // scan hand-over: end state per (pair, part)
+  float* carry_s;     // scan hand-over: sum of delta per (pair, part)
+  ScanPlan plan;
   size_t bytes;
+  size_t zero_bytes;  // error header + scheduler words, cleared each call
   int ksplit;
 };
 
@@ -1020,7 +1189,16 @@ FastWs fast_layout(const Problem& pr, char* base) {
   };
   const size_t T = (size_t)pr.T, d = (size_t)pr.d, P = (size_t)pr.P, R = (size_t)pr.R;
   w.ksplit = xproj_ksplit(pr.T, pr.d);
+  if (!pr.decode) w.plan = scan_plan(pr.B, pr.L, pr.d);
+  // hand-over slots: one per (pair, part) when parts exist
+  const size_t slots = w.plan.n_parts > 1
+                           ? (size_t)pr.B * (size_t)((pr.d + kSC - 1) / kSC) * w.plan.n_parts
+                           : 0;
   w.hdr = take(sizeof(ErrFlags));
+  w.sched = reinterpret_cast<int*>(take((1 + slots) * 4));
+  w.zero_bytes = off;
+  w.carry_h = reinterpret_cast<float*>(take(slots * kSC * kN * 4));
+  w.carry_s = reinterpret_cast<float*>(take(slots * kSC * 4));
   w.part = reinterpret_cast<float*>(take((size_t)w.ksplit * T * P * 4));
   w.u = reinterpret_cast<__half*>(take(T * d * 2));
   w.dtn = reinterpret_cast<__half*>(take(T * R * 2));
@@ -1031,11 +1209,22 @@ FastWs fast_layout(const Problem& pr, char* base) {
   return w;
 }
 
+int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
 cudaError_t run_fast_fwd(Problem& p) {
   FastWs w = fast_layout(p, p.ws);
   cudaStream_t s = p.stream;
   ErrFlags* err = reinterpret_cast<ErrFlags*>(w.hdr);
-  cudaError_t e = cudaMemsetAsync(p.ws, 0, sizeof(ErrFlags), s);
+  cudaError_t e = cudaMemsetAsync(p.ws, 0, w.zero_bytes, s);
   if (e != cudaSuccess) return e;
   launches_begin(p);
 
@@ -1146,9 +1335,19 @@ cudaError_t run_fast_fwd(Problem& p) {
     sa.hist = (const bf16*)p.init_conv;
     sa.final_conv = (bf16*)p.final_conv;
     sa.err = err;
+    sa.n_tiles = (int)((p.d + kSC - 1) / kSC);
+    sa.n_parts = w.plan.n_parts;
+    sa.two_pass = w.plan.two_pass;
+    sa.counter = w.sched;
+    sa.flags = w.sched + 1;
+    sa.carry_h = w.carry_h;
+    sa.carry_s = w.carry_s;
+    const int pairs = sa.n_tiles * (int)p.B;
+    const int units = pairs * sa.n_parts + (sa.two_pass ? pairs * (sa.n_parts - 1) : 0);
+    const int slots = 2 * num_sms();
     cudaFuncSetAttribute(k_scan_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, kScanSmem);
-    k_scan_fused<<<dim3((unsigned)((p.d + kSC - 1) / kSC), (unsigned)p.B), kScanThreads, kScanSmem,
-                   s>>>(twdt, tdtn, tbc, tx, tz, sa);
+    k_scan_fused<<<(unsigned)(units < slots ? units : slots), kScanThreads, kScanSmem, s>>>(
+        twdt, tdtn, tbc, tx, tz, sa);
     launched(p, "k_scan_fused");
   }
   return cudaGetLastError();

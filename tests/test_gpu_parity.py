@@ -42,6 +42,24 @@ def test_bf16_cases(B, L, d, R, extra):
     check_fwd(small(B, L, d, R, extra=extra))
 
 
+@pytest.mark.parametrize("B,L,d,R,use_init", [
+    (1, 1100, 256, 16, True),     # few (sequence, tile) pairs: state pass + output pass, 4 parts
+    (1, 2100, 200, 40, True),     # 8 parts, channel tail, ragged last chunk
+    (2, 700, 384, 64, False),     # 2 parts, zero initial states
+])
+def test_bf16_two_pass_schedule(B, L, d, R, use_init):
+    check_fwd(small(B, L, d, R), use_init=use_init)
+
+
+def test_bf16_chained_parts_schedule():
+    """320 (sequence, tile) pairs on 296 CTA slots: each sequence runs as four
+    parts in a chain, every part starting from the state the previous one left.
+    dt_rank 64: one fp16 rounding flip of dt_n moves delta by about 2^-10/sqrt(R)
+    relative, which at R = 16 over 160 sequences reaches the 1e-4 state gate by
+    itself; the hand-over between parts is an exact copy of the fp32 state."""
+    check_fwd(small(160, 1100, 256, 64, seed=7), channels=[0, 1, 127, 128, 200, 255])
+
+
 def test_bf16_without_initial_states():
     check_fwd(small(2, 150, 256, 32), use_init=False)
 
