@@ -16,13 +16,18 @@ this path) on the host cores, on a bounded sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import glob
+import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
 import time
+
+HERE = os.path.dirname(os.path.abspath(__file__))
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
@@ -81,6 +86,21 @@ def kernel_units(name, w, tokens):
     if "conv" in name:
         return "hbm", tokens * d * es * 2, "GB/s"     # x in, u out
     return "hbm", tokens * (R + 2 * N) * 4 * 2, "GB/s"
+
+
+def measured_traffic(kernel: str, tokens: int):
+    """DRAM bytes of one launch of `kernel` over `tokens` tokens, from the committed
+    ncu summary of that kernel (bytes per token x tokens), if the kernel source is
+    unchanged since the capture; else (None, None)."""
+    src = os.path.join(HERE, "mamba_selective_scan_jamba_b200", "csrc", "k_fast.cu")
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    pat = re.compile(r"<!-- traffic: kernel=(\S+) bytes_per_token=(\d+) source_sha256=(\w+) -->")
+    for path in sorted(glob.glob(os.path.join(HERE, "profiles", f"{kernel}_*.md"))):
+        with open(path) as f:
+            m = pat.search(f.read())
+        if m and m.group(1) == kernel and m.group(3) == sha:
+            return int(m.group(2)) * tokens, os.path.basename(path)
+    return None, None
 
 
 # ------------------------------------------------------------------- clocks
@@ -363,8 +383,12 @@ def main():
     wt = work_per_token(w)
     t_ns = max(wt["tc_flop"] / (P["bf16_sust"] * 1e12), wt["bytes"] / (P["hbm"] * 1e9))
     roof_tok_s = 1.0 / t_ns
+    traffic, traffic_src = measured_traffic(names[kd], tokens_rank)
     roofline = {"kernel": names[kd], "bound": bound, "achieved": achieved, "peak": peak,
-                "unit": unit, "frac": achieved / peak, "traffic": None,
+                "unit": unit, "frac": achieved / peak, "traffic": traffic,
+                "traffic_source": (f"profiles/{traffic_src} (ncu dram__bytes_read.sum + "
+                                   "dram__bytes_write.sum per token, scaled to this launch)"
+                                   if traffic_src else "none for the current kernel source"),
                 "peak_source": (f"MUFU 16/clk/SM x 148 SMs x {P['sm_max']:.0f} MHz (derived)"
                                 if bound == "alu" else f"{P['src']} MEASURED_PEAKS.json"),
                 "kernel_ms": per_kernel[kd],
