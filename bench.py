@@ -212,10 +212,18 @@ def decode_bench(dev, stream, steps: int = 64, warmup: int = 5):
 
 
 # ------------------------------------------------------------- cpu baseline
+def oracle_sample(w, tokens: float):
+    """(sequences, tokens per sequence) of a sample of about `tokens` tokens taken
+    from the start of the workload: a prefix of sequence 0, or whole sequences."""
+    tokens = int(max(16, tokens))
+    if tokens <= w.seqlen:
+        return 1, tokens
+    return max(1, min(w.batch, round(tokens / w.seqlen))), w.seqlen
+
+
 def oracle_rate(w, target_s: float, threads: int = 0):
-    """Time the fp64 oracle on sequence 0 of the workload, with a sample length
-    chosen so that the run takes about target_s seconds.  Returns
-    (tokens/s, cores, sample description)."""
+    """Time the fp64 oracle on a sample of the workload sized so that the run
+    takes about target_s seconds.  Returns (tokens/s, cores, sample description)."""
     import oracle
     from mamba_selective_scan_jamba_b200 import synth
     cores = threads or os.cpu_count() or 1
@@ -225,14 +233,21 @@ def oracle_rate(w, target_s: float, threads: int = 0):
     t = time.perf_counter()
     oracle.mixer_fwd(oracle.dims_of(w, batch=1, seqlen=L0, threads=cores), A["x"], A["z"], W)
     dt0 = time.perf_counter() - t
-    L = int(max(16, min(w.seqlen, L0 * target_s / max(dt0, 1e-3))))
-    A = synth.make_activations(w.with_(batch=1, seqlen=L))
-    t = time.perf_counter()
-    oracle.mixer_fwd(oracle.dims_of(w, batch=1, seqlen=L, threads=cores), A["x"], A["z"], W)
-    dt = time.perf_counter() - t
-    return L / dt, cores, (f"sequence 0 of {w.name}, first {L} tokens (B=1, L={L}, "
-                           f"d_inner={w.d_inner}, dt_rank={w.dt_rank}), fp64 oracle, "
-                           f"{cores} threads, {dt:.1f} s")
+    # the short probe overstates the per-token cost (fixed costs dominate it), so
+    # the sample is resized once more from its own time when it ran short
+    tokens = L0 * target_s / max(dt0, 1e-3)
+    for _ in range(2):
+        nb, L = oracle_sample(w, tokens)
+        A = synth.make_activations(w.with_(seqlen=L), 0, nb)
+        t = time.perf_counter()
+        oracle.mixer_fwd(oracle.dims_of(w, batch=nb, seqlen=L, threads=cores), A["x"], A["z"], W)
+        dt = time.perf_counter() - t
+        if dt >= 0.5 * target_s or nb * L >= w.batch * w.seqlen:
+            break
+        tokens = nb * L * target_s / max(dt, 1e-3)
+    return nb * L / dt, cores, (f"sequences 0..{nb - 1} of {w.name}, first {L} tokens each "
+                                f"(B={nb}, L={L}, d_inner={w.d_inner}, dt_rank={w.dt_rank}), "
+                                f"fp64 oracle, {cores} threads, {dt:.1f} s")
 
 
 def reference_arm(args, w, rank, world):

@@ -176,6 +176,17 @@ int jm_last_launch_count(void);
  * launched ("" when out of range).  The string is static. */
 const char* jm_last_kernel_name(int index);
 
+/* How jm_mixer_fwd will schedule the scan of this problem (bf16 I/O; float32
+ * problems run one part per sequence).  Each sequence is cut into *n_parts time
+ * parts of whole 32-token chunks.  *two_pass = 0: the parts of a sequence run
+ * one after another, each starting from the state the previous one handed over
+ * (used when the (sequence, 128-channel tile) pairs fill the GPU).  *two_pass = 1:
+ * a state pass records each part's end state from a zero start and its sum of
+ * delta, then every part computes its outputs from the fold of the earlier
+ * parts' results (used for few sequences).  Depends only on the dims.  Returns
+ * JM_ERR_INVALID_ARG for invalid dims or NULL outputs. */
+jm_status jm_mixer_fwd_schedule(const jm_dims* dims, int* n_parts, int* two_pass);
+
 /* Per-kernel timing hook for benchmarks.  `events` is an array of n_events
  * cudaEvent_t handles created by the caller.  While set (for calls on this
  * thread), each compute call records events[0] on its stream before its

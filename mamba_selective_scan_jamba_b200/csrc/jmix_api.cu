@@ -168,6 +168,21 @@ JM_API size_t jm_mixer_fwd_workspace_size(const jm_dims* dims) {
   return ws_bytes_for(p);
 }
 
+JM_API jm_status jm_mixer_fwd_schedule(const jm_dims* dims, int* n_parts, int* two_pass) {
+  if (!n_parts || !two_pass) {
+    set_error("jm_mixer_fwd_schedule: NULL output pointer");
+    return JM_ERR_INVALID_ARG;
+  }
+  jm_status st = check_dims(dims, false);
+  if (st != JM_OK) return st;
+  Problem p;
+  fill_problem(p, dims);
+  *n_parts = 1;
+  *two_pass = 0;
+  if (p.io == JM_BF16) fast_scan_schedule(p.B, p.L, p.d, n_parts, two_pass);
+  return JM_OK;
+}
+
 JM_API size_t jm_mixer_step_workspace_size(const jm_dims* dims) {
   if (check_dims(dims, true) != JM_OK) return 0;
   Problem p;

@@ -69,6 +69,8 @@ cudaError_t run_simple(Problem& p);
 
 // The bf16 path on tcgen05 tensor cores.
 size_t fast_ws_bytes(const Problem& p);
+// The scan schedule of the bf16 forward: time parts per sequence, two-pass or chained.
+void fast_scan_schedule(int64_t B, int64_t L, int64_t d, int* n_parts, int* two_pass);
 cudaError_t run_fast(Problem& p);
 
 // Per-thread message for jm_last_error.

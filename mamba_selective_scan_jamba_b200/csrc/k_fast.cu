@@ -41,7 +41,10 @@ constexpr int kConvG = 4;         // tokens per thread in k_conv_silu16
 constexpr int kXM = 128;          // x_proj tile: tokens
 constexpr int kXK = 64;           // x_proj tile: channels per k-chunk (one 128-B swizzle atom)
 constexpr int kXStages = 4;
-constexpr int kSQ = 16;           // scan: tokens per chunk
+#ifndef JMIX_SCAN_CHUNK
+#define JMIX_SCAN_CHUNK 32
+#endif
+constexpr int kSQ = JMIX_SCAN_CHUNK;  // scan: tokens per chunk (the dt_proj MMA's N)
 constexpr int kSC = 128;          // scan: channels per CTA
 constexpr int kMaxSlabs = kMaxRank / 64;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -450,6 +453,7 @@ struct ScanArgs {
   bf16* y;
   const bf16* hist;
   bf16* final_conv;
+  const __half* wdt;  // W_dt in fp16 [d, R]: the compute warps copy its first K slabs to TMEM
   ErrFlags* err;
   // Work schedule (see k_scan_fused).  A pair is one (sequence, 128-channel
   // tile); each pair's sequence is cut into n_parts time parts of whole chunks.
@@ -468,8 +472,12 @@ struct ScanPlan {
   int two_pass = 0;
 };
 
-// Two CTAs of the scan kernel fit on each of a B200's 148 SMs.
-constexpr int kScanSlots = 296;
+#ifndef JMIX_SCAN_CTAS
+#define JMIX_SCAN_CTAS 2
+#endif
+// CTAs of the scan kernel resident on each of a B200's 148 SMs.
+constexpr int kScanCtasPerSm = JMIX_SCAN_CTAS;
+constexpr int kScanSlots = kScanCtasPerSm * 148;
 // A time part spans at least this many 16-token chunks.
 constexpr int kMinPartChunks = 16;
 
@@ -478,10 +486,12 @@ ScanPlan scan_plan(int64_t B, int64_t L, int64_t d) {
   const int64_t pairs = B * ((d + kSC - 1) / kSC);
   const int64_t nch = (L + kSQ - 1) / kSQ;
   if (pairs <= 0 || nch <= 0) return pl;
-  if (pairs >= kScanSlots / 2) {
-    // Enough pairs to fill the GPU: parts only even out the last wave.  A part
-    // then starts from the state of the part before it (a chain), which costs
-    // no extra arithmetic.  Waves of part-sized units: ceil(pairs*P/slots)/P.
+  if (pairs > kScanSlots) {
+    // More pairs than CTA slots: parts only even out the last wave.  A part
+    // starts from the state of the part before it (a chain), which costs no
+    // extra arithmetic; with more pairs than slots a part's predecessor was
+    // claimed at least one wave earlier, so chained parts do not wait.  Waves of
+    // part-sized units: ceil(pairs*P/slots)/P.
     int64_t best_num = (pairs + kScanSlots - 1) / kScanSlots, best_den = 1;
     for (int P = 2; P <= 8; P *= 2) {
       if (nch < (int64_t)kMinPartChunks * P) break;
@@ -492,7 +502,7 @@ ScanPlan scan_plan(int64_t B, int64_t L, int64_t d) {
         pl.n_parts = P;
       }
     }
-  } else {
+  } else if (pairs < kScanSlots / 2) {
     // Too few pairs for the GPU: a state pass over parts 0..P-2 (from a zero
     // state) runs side by side, then every part produces its outputs from the
     // state that the earlier parts' results fold into.
@@ -504,13 +514,40 @@ ScanPlan scan_plan(int64_t B, int64_t L, int64_t d) {
   return pl;
 }
 
-constexpr int kScanThreads = 160;  // warps 0..3: one channel per thread; warp 4: TMA + MMA
-constexpr int kWdtBytes = kMaxSlabs * kSC * 128;                  // 64 KB
+// warps 0..3: one channel per thread (its TMEM lane); warp 4: TMA + MMA
+constexpr int kProdWarp = 4;
+constexpr int kScanThreads = 32 * (kProdWarp + 1);
+constexpr int kAllBar = 1;  // named barrier of the four compute warps
+constexpr int kWdtBytes = kMaxSlabs * kSC * 128;                  // 64 KB (decode kernel)
+// The scan kernel keeps W_dt's first two 64-wide K slabs in TMEM (the MMA's A
+// operand may come from there) and only the rest in shared memory, which lets
+// three CTAs share an SM.  TMEM per CTA: columns [0, 32) hold the two dt_proj
+// accumulators, [64, 128) the W_dt slabs (two fp16 per 32-bit column).
+#ifndef JMIX_SCAN_TMEM_SLABS
+#define JMIX_SCAN_TMEM_SLABS 2
+#endif
+#ifndef JMIX_SCAN_STAGES
+#define JMIX_SCAN_STAGES 2
+#endif
+constexpr int kWdtTmemSlabs = JMIX_SCAN_TMEM_SLABS;
+constexpr int kScanStages = JMIX_SCAN_STAGES;  // ring of {dt_n, x, z, B/C} stages + accumulators
+constexpr int kScanWdtBytes = (kMaxSlabs - kWdtTmemSlabs) * kSC * 128;  // 32 KB
+constexpr uint32_t kTmemWdtCol = kScanStages * kSQ <= 64 ? 64 : 128;
+constexpr uint32_t kScanTmemNeed = kTmemWdtCol + 32 * kWdtTmemSlabs;
+constexpr uint32_t kScanTmemCols = kScanTmemNeed <= 64 ? 64 : kScanTmemNeed <= 128 ? 128
+                                   : kScanTmemNeed <= 256 ? 256 : 512;
+static_assert(kScanStages * kSQ <= (int)kTmemWdtCol, "accumulators overlap the W_dt columns");
+static_assert(kScanCtasPerSm * kScanTmemCols <= 512, "TMEM of the resident CTAs exceeds 512 columns");
 constexpr int kDtnStage = kMaxSlabs * kSQ * 128;                  // 8 KB (SW128 slabs)
 constexpr int kXStage = kSQ * kSC * 2;                            // 4 KB (x or z tile)
 constexpr int kBCStage = kSQ * 2 * kN * 4;                        // 2 KB
 constexpr int kStageBytes = kDtnStage + 2 * kXStage + kBCStage;   // 18 KB
-constexpr int kScanSmem = 1024 + kWdtBytes + 2 * kStageBytes + 256;
+#ifndef JMIX_SCAN_G
+#define JMIX_SCAN_G 8
+#endif
+constexpr int kG = JMIX_SCAN_G;  // tokens per TMEM load / unrolled group in the scan loop
+constexpr int kScanSmem = 1024 + kScanWdtBytes + kScanStages * kStageBytes + 256;
+static_assert(kScanCtasPerSm * (kScanSmem + 1024) <= 228 * 1024, "shared memory per SM exceeded");
 
 // softplus(v) = max(v, 0) + log1p(exp(-|v|)): one MUFU ex2, log1p by a
 // degree-8 minimax polynomial on the FMA pipe (relative error < 3e-7).
@@ -528,10 +565,6 @@ __device__ __forceinline__ float softplus_fast(float v) {
   return fmaf(w, q, fmaxf(v, 0.0f));
 }
 
-#ifndef JMIX_SCAN_G
-#define JMIX_SCAN_G 8
-#endif
-constexpr int kG = JMIX_SCAN_G;  // tokens per TMEM load / unrolled group in the scan loop
 
 __device__ __forceinline__ float tanh_approx(float x) {
   float y;
@@ -586,8 +619,8 @@ __device__ __forceinline__ void scan_chunks(const ScanArgs& a, const uint8_t* st
   const int cl = warp * 32 + lane;
   for (int k = 0; k < nch; ++k) {
     const int kg = kg0 + k;
-    const int s = kg & 1;
-    const uint32_t ph = (uint32_t)(kg >> 1) & 1u;
+    const int s = kg % kScanStages;
+    const uint32_t ph = (uint32_t)(kg / kScanStages) & 1u;
     if (!mbar_wait(smem_u32(&mma_done[s]), ph, a.err, 25)) break;
     if (!mbar_wait(smem_u32(&full[s]), ph, a.err, 26)) break;
     tc_fence_after();
@@ -690,7 +723,7 @@ __device__ __forceinline__ void scan_chunks(const ScanArgs& a, const uint8_t* st
 // Every unit that waits waits only for units that come before it in claim
 // order, and a claimed unit is running or queued behind one with a smaller
 // index on its CTA, so every wait ends; each is still bounded (2 s).
-__global__ void __launch_bounds__(kScanThreads, 2)
+__global__ void __launch_bounds__(kScanThreads, kScanCtasPerSm)
     k_scan_fused(const __grid_constant__ CUtensorMap tm_wdt,
                  const __grid_constant__ CUtensorMap tm_dtn,
                  const __grid_constant__ CUtensorMap tm_bc, const __grid_constant__ CUtensorMap tm_x,
@@ -698,15 +731,17 @@ __global__ void __launch_bounds__(kScanThreads, 2)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* wdt_s = smem;              // W_dt tile: nslab x [128 ch x 64] (SW128)
-  uint8_t* stage0 = smem + kWdtBytes;  // 2 x {dt_n (SW128), x tile, z tile, B/C rows}
-  uint64_t* bars = reinterpret_cast<uint64_t*>(stage0 + 2 * kStageBytes);
-  uint64_t* full = bars;          // [2] stage landed
-  uint64_t* mma_done = bars + 2;  // [2] dt_proj accumulator ready
-  uint64_t* empty = bars + 4;     // [2] compute warps done with the stage / accumulator
-  uint64_t* wfull = bars + 6;     // W_dt tile landed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 7);
-  volatile int* unit_slot = reinterpret_cast<volatile int*>(bars + 8);  // [2] claimed units
+  uint8_t* wdt_s = smem;                  // W_dt K slabs 2.. : [128 ch x 64] each (SW128)
+  uint8_t* stage0 = smem + kScanWdtBytes;  // 2 x {dt_n (SW128), x tile, z tile, B/C rows}
+  uint64_t* bars = reinterpret_cast<uint64_t*>(stage0 + kScanStages * kStageBytes);
+  uint64_t* full = bars;                         // [stages] stage landed
+  uint64_t* mma_done = bars + kScanStages;       // [stages] dt_proj accumulator ready
+  uint64_t* empty = bars + 2 * kScanStages;      // [stages] compute warps done with the slot
+  uint64_t* wfull = bars + 3 * kScanStages;      // W_dt slabs in shared memory landed
+  uint64_t* wready = wfull + 1;  // W_dt slabs in TMEM written (one arrive per compute warp)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wfull + 2);
+  volatile int* unit_slot = reinterpret_cast<volatile int*>(wfull + 3);  // [2] claimed units
+  const int nslab_t = a.nslab < kWdtTmemSlabs ? a.nslab : kWdtTmemSlabs;  // slabs in TMEM
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nch_all = (int)((a.L + kSQ - 1) / kSQ);
@@ -717,23 +752,27 @@ __global__ void __launch_bounds__(kScanThreads, 2)
   const int n_units = n_state + pairs * P;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kScanStages; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
       mbar_init(smem_u32(&mma_done[s]), 1);
-      mbar_init(smem_u32(&empty[s]), 4);
+      mbar_init(smem_u32(&empty[s]), kProdWarp);  // one arrive per compute warp
     }
     mbar_init(smem_u32(wfull), 1);
+    mbar_init(smem_u32(wready), 4);
     fence_mbar_init();
-    unit_slot[0] = atomicAdd(a.counter, 1);
   }
-  if (warp == 4) {
-    tmem_alloc(smem_u32(tmem_slot), 2 * kSQ);
+  if (warp == kProdWarp) {
+    tmem_alloc(smem_u32(tmem_slot), kScanTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // claim the first unit only now: a CTA that waited in tcgen05.alloc (more
+  // CTAs resident than TMEM for) holds no unit that another CTA could wait on
+  if (threadIdx.x == 0) unit_slot[0] = atomicAdd(a.counter, 1);
+  __syncthreads();
 
   int kg0 = 0;    // chunks this CTA has run before the current unit (mbarrier phases)
   int nw = 0;     // W_dt tiles this CTA has loaded (wfull phase)
@@ -741,7 +780,7 @@ __global__ void __launch_bounds__(kScanThreads, 2)
     const int unit = unit_slot[it & 1];
     if (unit >= n_units) break;
     // claim the next unit early, so that its number is ready when this one ends
-    if (threadIdx.x == 128)
+    if (threadIdx.x == 32 * kProdWarp)
       unit_slot[(it + 1) & 1] = *(volatile unsigned*)&a.err->timeout ? n_units
                                                                       : atomicAdd(a.counter, 1);
     const bool out = unit >= n_state;
@@ -756,16 +795,19 @@ __global__ void __launch_bounds__(kScanThreads, 2)
     const int nch = (int)((int64_t)nch_all * (part + 1) / P) - kb;
     const int64_t hslot = (int64_t)pair * P + part;  // this part's hand-over slot
 
-    if (warp == 4) {
+    if (warp == kProdWarp) {
       if (lane == 0 && nch > 0) {
         const uint32_t wb = smem_u32(wfull);
-        mbar_arrive_expect_tx(wb, (uint32_t)(a.nslab * kSC * 128));
-        for (int j = 0; j < a.nslab; ++j)
-          tma_load_2d(smem_u32(wdt_s + j * kSC * 128), &tm_wdt, wb, j * 64, (int32_t)c0);
+        if (a.nslab > nslab_t) {
+          mbar_arrive_expect_tx(wb, (uint32_t)((a.nslab - nslab_t) * kSC * 128));
+          for (int j = nslab_t; j < a.nslab; ++j)
+            tma_load_2d(smem_u32(wdt_s + (j - nslab_t) * kSC * 128), &tm_wdt, wb, j * 64,
+                        (int32_t)c0);
+        }
         const uint32_t stage_tx =
             (uint32_t)(a.nslab * kSQ * 128 + (out ? 2 : 1) * kXStage + kBCStage);
         auto issue_stage = [&](int k) {  // k: chunk of this unit
-          const int s = (kg0 + k) & 1;
+          const int s = (kg0 + k) % kScanStages;
           uint8_t* st = stage0 + s * kStageBytes;
           const uint32_t fb = smem_u32(&full[s]);
           const int32_t row = (int32_t)(g0 + (int64_t)(kb + k) * kSQ);
@@ -779,37 +821,50 @@ __global__ void __launch_bounds__(kScanThreads, 2)
         const uint32_t idesc = idesc_f16_f32(kSC, kSQ);
         auto issue_mma = [&](int k) -> bool {
           const int kg = kg0 + k;
-          const int s = kg & 1;
-          if (!mbar_wait(smem_u32(&full[s]), (uint32_t)(kg >> 1) & 1u, a.err, 22)) return false;
+          const int s = kg % kScanStages;
+          if (!mbar_wait(smem_u32(&full[s]), (uint32_t)(kg / kScanStages) & 1u, a.err, 22))
+            return false;
           tc_fence_after();
           const uint32_t wbase = smem_u32(wdt_s), db = smem_u32(stage0 + s * kStageBytes);
           const uint32_t d_tmem = tmem + (uint32_t)(s * kSQ);
           for (int j = 0; j < a.nslab; ++j)
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              umma_f16(d_tmem, sw128_kmajor_desc(wbase + j * kSC * 128 + kk * 32),
-                       sw128_kmajor_desc(db + j * kSQ * 128 + kk * 32), idesc,
-                       (j > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t bdesc = sw128_kmajor_desc(db + j * kSQ * 128 + kk * 32);
+              const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;
+              if (j < nslab_t)  // A: 16 K values = 8 TMEM columns per step
+                umma_f16_ts(d_tmem, tmem + kTmemWdtCol + (uint32_t)(j * 32 + kk * 8), bdesc, idesc,
+                            acc);
+              else
+                umma_f16(d_tmem, sw128_kmajor_desc(wbase + (j - nslab_t) * kSC * 128 + kk * 32),
+                         bdesc, idesc, acc);
+            }
           umma_commit(smem_u32(&mma_done[s]));
           return true;
         };
-        // Both stages and accumulators are free here: the previous unit ended
+        // Every stage and accumulator is free here: the previous unit ended
         // with every compute warp past its last chunk (CTA barrier below).
-        issue_stage(0);
-        if (nch > 1) issue_stage(1);
-        bool ok = mbar_wait(wb, (uint32_t)nw & 1u, a.err, 21);
+        for (int k = 0; k < kScanStages && k < nch; ++k) issue_stage(k);
+        bool ok = a.nslab <= nslab_t || mbar_wait(wb, (uint32_t)nw & 1u, a.err, 21);
+        if (ok) ok = mbar_wait(smem_u32(wready), (uint32_t)nw & 1u, a.err, 27);
+        if (ok) tc_fence_after();
         if (ok) ok = issue_mma(0);
+        // chunk j's slot (stage + accumulator) is reused by chunk j + stages, once
+        // the compute warps have released chunk j (empty)
         for (int k = 0; ok && k < nch; ++k) {
           const int kg = kg0 + k;
           if (k + 1 < nch) {
-            if (k >= 1 && !mbar_wait(smem_u32(&empty[(kg + 1) & 1]),
-                                     (uint32_t)((kg - 1) >> 1) & 1u, a.err, 23))
+            const int j = kg + 1 - kScanStages;  // last chunk in MMA k+1's accumulator
+            if (j >= kg0 && !mbar_wait(smem_u32(&empty[j % kScanStages]),
+                                       (uint32_t)(j / kScanStages) & 1u, a.err, 23))
               break;
             if (!issue_mma(k + 1)) break;
           }
-          if (k + 2 < nch) {
-            if (!mbar_wait(smem_u32(&empty[kg & 1]), (uint32_t)(kg >> 1) & 1u, a.err, 24)) break;
-            issue_stage(k + 2);
+          if (k + kScanStages < nch) {
+            if (!mbar_wait(smem_u32(&empty[kg % kScanStages]), (uint32_t)(kg / kScanStages) & 1u,
+                           a.err, 24))
+              break;
+            issue_stage(k + kScanStages);
           }
         }
       }
@@ -818,6 +873,31 @@ __global__ void __launch_bounds__(kScanThreads, 2)
       const int cl = warp * 32 + lane;
       const int64_t c = c0 + cl;
       const bool cok = c < a.d;
+      if (nch > 0) {
+        // this channel's W_dt row, K slabs 0..nslab_t-1, into its TMEM lane
+        // (zeros past R and past d, matching the zero fill of the dt_n tiles)
+        const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16) + kTmemWdtCol;
+        // a 64-wide K slab is 32 columns: nslab_t * 2 steps of 16 columns stay
+        // inside [kTmemWdtCol, kTmemWdtCol + 64) of the 128-column allocation
+        for (int q = 0; q < nslab_t * 2; ++q) {  // 16 columns = 32 K values per step
+          uint32_t v[16];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int k = q * 32 + e * 8;
+            uint4 w8 = make_uint4(0u, 0u, 0u, 0u);
+            if (cok && k < a.R) w8 = __ldg(reinterpret_cast<const uint4*>(a.wdt + c * a.R + k));
+            v[4 * e] = w8.x;
+            v[4 * e + 1] = w8.y;
+            v[4 * e + 2] = w8.z;
+            v[4 * e + 3] = w8.w;
+          }
+          tmem_st16(trow + (uint32_t)(q * 16), v);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(wready));
+      }
       // a unit that starts from earlier parts waits (bounded) for their hand-over
       const int n_wait = part == 0 ? 0 : (a.two_pass ? (out ? part : 0) : 1);
       if (n_wait > 0) {
@@ -826,17 +906,18 @@ __global__ void __launch_bounds__(kScanThreads, 2)
             wait_flag(a.flags + (int64_t)pair * P + q, a.err, 28);
           __threadfence();
         }
-        named_bar_sync(1, 128);
+        named_bar_sync(kAllBar, 32 * kProdWarp);
       }
       float2 A2[kN / 2], h[kN / 2];
 #pragma unroll
       for (int q = 0; q < kN / 2; ++q) {
-        A2[q].x = cok ? -expf(a.A_log[c * kN + 2 * q]) * kLog2e : 0.0f;
-        A2[q].y = cok ? -expf(a.A_log[c * kN + 2 * q + 1]) * kLog2e : 0.0f;
+        const int n = 2 * q;
+        A2[q].x = cok ? -expf(a.A_log[c * kN + n]) * kLog2e : 0.0f;
+        A2[q].y = cok ? -expf(a.A_log[c * kN + n + 1]) * kLog2e : 0.0f;
         h[q] = make_float2(0.0f, 0.0f);
         if (part == 0 && cok && a.h0) {
-          h[q].x = a.h0[(b * a.d + c) * kN + 2 * q];
-          h[q].y = a.h0[(b * a.d + c) * kN + 2 * q + 1];
+          h[q].x = a.h0[(b * a.d + c) * kN + n];
+          h[q].y = a.h0[(b * a.d + c) * kN + n + 1];
         }
       }
       if (n_wait > 0) {
@@ -886,7 +967,7 @@ __global__ void __launch_bounds__(kScanThreads, 2)
         for (int q = 0; q < kN / 2; ++q) reinterpret_cast<float2*>(ch)[q] = h[q];
         if (!out) a.carry_s[hslot * kSC + cl] = ssum;
         __threadfence();
-        named_bar_sync(1, 128);
+        named_bar_sync(kAllBar, 32 * kProdWarp);
         if (threadIdx.x == 0) st_release_gpu(a.flags + hslot, 1);
       } else if (out && part + 1 == P && cok) {
 #pragma unroll
@@ -906,15 +987,15 @@ __global__ void __launch_bounds__(kScanThreads, 2)
     nw += nch > 0 ? 1 : 0;
     __syncthreads();
     // stop claiming work once any wait has given up
-    if (threadIdx.x == 128 && *(volatile unsigned*)&a.err->timeout)
+    if (threadIdx.x == 32 * kProdWarp && *(volatile unsigned*)&a.err->timeout)
       unit_slot[(it + 1) & 1] = n_units;
     __syncthreads();
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == kProdWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem, 2 * kSQ);
+    tmem_dealloc(tmem, kScanTmemCols);
   }
 }
 
@@ -1334,6 +1415,7 @@ cudaError_t run_fast_fwd(Problem& p) {
     sa.y = (bf16*)p.y;
     sa.hist = (const bf16*)p.init_conv;
     sa.final_conv = (bf16*)p.final_conv;
+    sa.wdt = w.wdt;
     sa.err = err;
     sa.n_tiles = (int)((p.d + kSC - 1) / kSC);
     sa.n_parts = w.plan.n_parts;
@@ -1344,8 +1426,10 @@ cudaError_t run_fast_fwd(Problem& p) {
     sa.carry_s = w.carry_s;
     const int pairs = sa.n_tiles * (int)p.B;
     const int units = pairs * sa.n_parts + (sa.two_pass ? pairs * (sa.n_parts - 1) : 0);
-    const int slots = 2 * num_sms();
+    const int slots = kScanCtasPerSm * num_sms();
     cudaFuncSetAttribute(k_scan_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, kScanSmem);
+    cudaFuncSetAttribute(k_scan_fused, cudaFuncAttributePreferredSharedMemoryCarveout,
+                         cudaSharedmemCarveoutMaxShared);
     k_scan_fused<<<(unsigned)(units < slots ? units : slots), kScanThreads, kScanSmem, s>>>(
         twdt, tdtn, tbc, tx, tz, sa);
     launched(p, "k_scan_fused");
@@ -1356,6 +1440,12 @@ cudaError_t run_fast_fwd(Problem& p) {
 }  // namespace
 
 size_t fast_ws_bytes(const Problem& p) { return fast_layout(p, nullptr).bytes; }
+
+void fast_scan_schedule(int64_t B, int64_t L, int64_t d, int* n_parts, int* two_pass) {
+  const ScanPlan pl = scan_plan(B, L, d);
+  *n_parts = pl.n_parts;
+  *two_pass = pl.two_pass;
+}
 
 cudaError_t run_fast(Problem& p) { return run_fast_fwd(p); }
 

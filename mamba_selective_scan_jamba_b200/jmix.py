@@ -25,7 +25,7 @@ WEIGHT_NAMES = ("conv_w", "conv_b", "xproj_w", "dt_norm_w", "b_norm_w", "c_norm_
 EXPORTED = ("jm_mixer_fwd_workspace_size", "jm_mixer_step_workspace_size", "jm_mixer_fwd",
             "jm_mixer_step", "jm_mixer_fwd_host", "jm_poll_error", "jm_last_error",
             "jm_last_launch_count", "jm_last_kernel_name", "jm_set_kernel_events",
-            "jm_mixer_step_noalloc")
+            "jm_mixer_step_noalloc", "jm_mixer_fwd_schedule")
 
 
 class jm_dims(ctypes.Structure):
@@ -66,6 +66,9 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.jm_mixer_step_noalloc.argtypes = [ctypes.POINTER(jm_dims)] + [_vp] * 15 + [_vp]
     lib.jm_mixer_fwd_host.restype = ctypes.c_int
     lib.jm_mixer_fwd_host.argtypes = [ctypes.POINTER(jm_dims)] + [_vp] * 19 + [ctypes.c_size_t, _vp]
+    lib.jm_mixer_fwd_schedule.restype = ctypes.c_int
+    lib.jm_mixer_fwd_schedule.argtypes = [ctypes.POINTER(jm_dims), ctypes.POINTER(ctypes.c_int),
+                                          ctypes.POINTER(ctypes.c_int)]
     lib.jm_poll_error.restype = ctypes.c_int
     lib.jm_poll_error.argtypes = [_vp, _vp]
     lib.jm_last_error.restype = ctypes.c_char_p
@@ -110,6 +113,13 @@ def _check(status: int) -> None:
 
 def jm_mixer_fwd_workspace_size(d: jm_dims) -> int:
     return load().jm_mixer_fwd_workspace_size(ctypes.byref(d))
+
+
+def jm_mixer_fwd_schedule(d: jm_dims):
+    """(n_parts, two_pass) of the scan schedule jm_mixer_fwd uses for these dims."""
+    n, t = ctypes.c_int(0), ctypes.c_int(0)
+    _check(load().jm_mixer_fwd_schedule(ctypes.byref(d), ctypes.byref(n), ctypes.byref(t)))
+    return n.value, bool(t.value)
 
 
 def jm_mixer_step_workspace_size(d: jm_dims) -> int:

@@ -123,3 +123,43 @@ def test_binding_raises_on_error(lib):
         jmix.jm_mixer_fwd(jmix.dims(1, 4, 256, 16, d_conv=2), FAKE, FAKE, W, FAKE, FAKE, FAKE,
                           1 << 30, stream=0)
     assert e.value.status == jmix.JM_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("B,L,d,io,want", [
+    (8, 4096, 8192, jmix.JM_BF16, (4, False)),     # 512 pairs on 296 CTA slots: 4 chained parts
+    (1, 4096, 8192, jmix.JM_BF16, (8, True)),      # 64 pairs: state pass + output pass
+    (1, 262144, 8192, jmix.JM_BF16, (8, True)),
+    (3, 4096, 8192, jmix.JM_BF16, (1, False)),     # 192 pairs: one wave already
+    (160, 2100, 256, jmix.JM_BF16, (4, False)),
+    (1, 2200, 256, jmix.JM_BF16, (4, True)),
+    (2, 1100, 384, jmix.JM_BF16, (2, True)),
+    (1, 4200, 200, jmix.JM_BF16, (8, True)),
+    (2, 300, 384, jmix.JM_BF16, (1, False)),       # too short to cut
+    (8, 4096, 8192, jmix.JM_F32, (1, False)),      # float32 path: one part
+])
+def test_scan_schedule(lib, B, L, d, io, want):
+    assert jmix.jm_mixer_fwd_schedule(jmix.dims(B, L, d, 256 if d == 8192 else 16, io=io)) == want
+
+
+def test_scan_schedule_rules(lib):
+    """Parts hold at least 16 chunks of 32 tokens; chained parts are only used with
+    more pairs than CTA slots (two per SM on 148 SMs), where they shorten the last
+    wave; the two-pass schedule only with fewer pairs than half the slots."""
+    slots = 296
+    for B in (1, 2, 5, 8, 16, 64, 160, 300):
+        for L in (1, 31, 512, 1023, 1024, 2048, 4096, 9000):
+            for d in (128, 200, 1024, 8192):
+                n, two = jmix.jm_mixer_fwd_schedule(jmix.dims(B, L, d, 16))
+                assert n in (1, 2, 4, 8)
+                chunks = -(-L // 32)
+                if n > 1:
+                    assert chunks >= 16 * n
+                pairs = B * -(-d // 128)
+                if two:
+                    assert pairs < slots // 2
+                elif n > 1:
+                    assert pairs > slots
+                    waves = lambda P: -(-pairs * P // slots) / P
+                    assert waves(n) < waves(1)
+    with pytest.raises(jmix.JmixError):
+        jmix.jm_mixer_fwd_schedule(jmix.dims(1, 10, 100, 16))   # d % 8 != 0

@@ -42,13 +42,16 @@ def test_bf16_cases(B, L, d, R, extra):
     check_fwd(small(B, L, d, R, extra=extra))
 
 
-@pytest.mark.parametrize("B,L,d,R,use_init", [
-    (1, 1100, 256, 16, True),     # few (sequence, tile) pairs: state pass + output pass, 4 parts
-    (1, 2100, 200, 40, True),     # 8 parts, channel tail, ragged last chunk
-    (2, 700, 384, 64, False),     # 2 parts, zero initial states
+@pytest.mark.parametrize("B,L,d,R,use_init,parts", [
+    (1, 2200, 256, 16, True, 4),    # few (sequence, tile) pairs: state pass + output pass
+    (1, 4200, 200, 40, True, 8),    # channel tail, ragged last chunk
+    (2, 1100, 384, 64, False, 2),   # zero initial states
 ])
-def test_bf16_two_pass_schedule(B, L, d, R, use_init):
-    check_fwd(small(B, L, d, R), use_init=use_init)
+def test_bf16_two_pass_schedule(B, L, d, R, use_init, parts):
+    from mamba_selective_scan_jamba_b200 import devio, jmix
+    w = small(B, L, d, R)
+    assert jmix.jm_mixer_fwd_schedule(devio.dims_of(w)) == (parts, True)
+    check_fwd(w, use_init=use_init)
 
 
 def test_bf16_chained_parts_schedule():
@@ -57,7 +60,10 @@ def test_bf16_chained_parts_schedule():
     dt_rank 64: one fp16 rounding flip of dt_n moves delta by about 2^-10/sqrt(R)
     relative, which at R = 16 over 160 sequences reaches the 1e-4 state gate by
     itself; the hand-over between parts is an exact copy of the fp32 state."""
-    check_fwd(small(160, 1100, 256, 64, seed=7), channels=[0, 1, 127, 128, 200, 255])
+    from mamba_selective_scan_jamba_b200 import devio, jmix
+    w = small(160, 2100, 256, 64, seed=7)
+    assert jmix.jm_mixer_fwd_schedule(devio.dims_of(w)) == (4, False)
+    check_fwd(w, channels=[0, 1, 127, 128, 200, 255])
 
 
 def test_bf16_without_initial_states():
