@@ -37,7 +37,12 @@ namespace {
 using namespace sm100;
 typedef __nv_bfloat16 bf16;
 
-constexpr int kConvG = 4;         // tokens per thread in k_conv_silu16
+#ifndef JMIX_CONV_OCC
+#define JMIX_CONV_OCC 2
+#endif
+// tokens per thread in k_conv_silu16: 8 for sequences (3 history rows shared by
+// 8 tokens), 1 for decode steps (L = 1)
+constexpr int kConvG = 8;
 constexpr int kXM = 128;          // x_proj tile: tokens
 constexpr int kXK = 64;           // x_proj tile: channels per k-chunk (one 128-B swizzle atom)
 constexpr int kXStages = 4;
@@ -55,6 +60,12 @@ __device__ __forceinline__ void unpack8_bf16(const uint4& q, float (&o)[8]) {
   const bf16* h = reinterpret_cast<const bf16*>(&q);
 #pragma unroll
   for (int i = 0; i < 8; ++i) o[i] = __bfloat162float(h[i]);
+}
+
+// Element e (0..7) of 8 packed bf16 values, as float.
+__device__ __forceinline__ float bf16_lane(const uint4& v, int e) {
+  const uint32_t wd = e < 2 ? v.x : e < 4 ? v.y : e < 6 ? v.z : v.w;
+  return __uint_as_float((e & 1) ? (wd & 0xffff0000u) : (wd << 16));
 }
 
 __device__ __forceinline__ __half to_half_sat(float v) {
@@ -88,7 +99,8 @@ __device__ __forceinline__ float silu_newton(float v) {
   return v * r;
 }
 
-__global__ void __launch_bounds__(256, 2) k_conv_silu16(
+template <int kConvG>
+__global__ void __launch_bounds__(256, JMIX_CONV_OCC) k_conv_silu16(
     const bf16* __restrict__ x, const bf16* __restrict__ conv_w, const bf16* __restrict__ conv_b,
     const bf16* __restrict__ hist, int64_t B, int64_t L, int64_t d, __half* __restrict__ u,
     int64_t n_conv, const bf16* __restrict__ wx, int64_t n_wx8, __half* __restrict__ wx16,
@@ -103,7 +115,9 @@ __global__ void __launch_bounds__(256, 2) k_conv_silu16(
     const int64_t c0 = cg * 8, t0 = ck * kConvG;
     const int nt = (int)((L - t0) < kConvG ? (L - t0) : kConvG);
     constexpr int kW = kConv - 1;
-    // rows[0..2] = tokens t0-3..t0-1, rows[3..] = tokens t0..t0+nt-1
+    // rows[0..2] = tokens t0-3..t0-1 (history: x, the cached state or zero),
+    // rows[3..] = tokens t0..t0+nt-1; kept as packed bf16 and unpacked one
+    // channel at a time (fewer live registers than unpacking everything)
     uint4 rows[kW + kConvG];
 #pragma unroll
     for (int i = 0; i < kW + kConvG; ++i) {
@@ -113,51 +127,47 @@ __global__ void __launch_bounds__(256, 2) k_conv_silu16(
       else
         rows[i] = make_uint4(0u, 0u, 0u, 0u);
     }
-    float w[8][kConv], bias[8];
-    {
-      const uint4* wp = reinterpret_cast<const uint4*>(conv_w + c0 * kConv);
+    uint4 wq[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float o[8];
-        unpack8_bf16(__ldg(wp + q), o);
+    for (int q = 0; q < 4; ++q)
+      wq[q] = __ldg(reinterpret_cast<const uint4*>(conv_w + c0 * kConv) + q);
+    const uint4 bq = __ldg(reinterpret_cast<const uint4*>(conv_b + c0));
+    uint32_t outp[kConvG][4];  // [token][channel pair] packed fp16x2
 #pragma unroll
-        for (int i = 0; i < 8; ++i) w[(q * 8 + i) / kConv][(q * 8 + i) % kConv] = o[i];
+    for (int e = 0; e < 8; ++e) {
+      float xe[kW + kConvG];
+#pragma unroll
+      for (int i = 0; i < kW + kConvG; ++i) xe[i] = bf16_lane(rows[i], e);
+      if (t0 < kW) {
+        // taps before the sequence start: the cached conv state, or zero
+#pragma unroll
+        for (int k = 0; k < kW; ++k) {
+          const int64_t tau = t0 - kW + k;
+          if (tau < 0) xe[k] = hist ? bf(hist[(b * d + c0 + e) * kW + kW + tau]) : 0.0f;
+        }
       }
-      unpack8_bf16(__ldg(reinterpret_cast<const uint4*>(conv_b + c0)), bias);
-    }
-    float win[kW][8];
+      float wk[kConv];
 #pragma unroll
-    for (int k = 0; k < kW; ++k) {
-      const int64_t tau = t0 - kW + k;
-      if (tau >= 0) {
-        unpack8_bf16(rows[k], win[k]);
-      } else {
+      for (int k = 0; k < kConv; ++k)
+        wk[k] = bf16_lane(wq[(e * kConv + k) >> 3], (e * kConv + k) & 7);
+      const float be = bf16_lane(bq, e);
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          win[k][j] = hist ? bf(hist[(b * d + c0 + j) * kW + kW + tau]) : 0.0f;
+      for (int i = 0; i < kConvG; ++i) {
+        float acc = be;
+#pragma unroll
+        for (int k = 0; k < kConv; ++k) acc = fmaf(wk[k], xe[i + k], acc);
+        const uint32_t hb = (uint32_t)__half_as_ushort(to_half_sat(silu_u(acc)));
+        if (e & 1)
+          outp[i][e >> 1] |= hb << 16;
+        else
+          outp[i][e >> 1] = hb;
       }
     }
 #pragma unroll
     for (int i = 0; i < kConvG; ++i) {
       if (i >= nt) break;
-      float xt[8];
-      unpack8_bf16(rows[kW + i], xt);
-      __align__(16) __half out[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        float acc = bias[j];
-#pragma unroll
-        for (int k = 0; k < kW; ++k) acc = fmaf(w[j][k], win[k][j], acc);
-        acc = fmaf(w[j][kW], xt[j], acc);
-        out[j] = to_half_sat(silu_u(acc));
-      }
-      *reinterpret_cast<uint4*>(u + (b * L + t0 + i) * d + c0) = *reinterpret_cast<uint4*>(out);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-#pragma unroll
-        for (int k = 0; k < kW - 1; ++k) win[k][j] = win[k + 1][j];
-        win[kW - 1][j] = xt[j];
-      }
+      *reinterpret_cast<uint4*>(u + (b * L + t0 + i) * d + c0) =
+          make_uint4(outp[i][0], outp[i][1], outp[i][2], outp[i][3]);
     }
     return;
   }
@@ -1311,10 +1321,12 @@ cudaError_t run_fast_fwd(Problem& p) {
 
   // 1. conv + SiLU -> u (fp16); weights -> fp16
   {
-    const int64_t n_conv = (p.d / 8) * ((p.L + kConvG - 1) / kConvG) * p.B;
+    const int G = p.L >= kConvG ? kConvG : 1;
+    const int64_t n_conv = (p.d / 8) * ((p.L + G - 1) / G) * p.B;
     const int64_t n_wx8 = (int64_t)p.P * p.d / 8, n_wdt8 = p.d * p.R / 8;
     const int64_t total = n_conv + n_wx8 + n_wdt8;
-    k_conv_silu16<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
+    auto kern = G == kConvG ? k_conv_silu16<kConvG> : k_conv_silu16<1>;
+    kern<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
         (const bf16*)p.x, (const bf16*)p.conv_w, (const bf16*)p.conv_b, (const bf16*)p.init_conv,
         p.B, p.L, p.d, w.u, n_conv, (const bf16*)p.xproj_w, n_wx8, w.wx,
         (const bf16*)p.dtproj_w, n_wdt8, w.wdt);
