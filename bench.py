@@ -27,6 +27,8 @@ import subprocess
 import sys
 import time
 
+import numpy as np
+
 HERE = os.path.dirname(os.path.abspath(__file__))
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -47,6 +49,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--varlen", action="store_true",
+                    help="also time jm_mixer_fwd_varlen on a packed batch of mixed lengths")
     ap.add_argument("--seqlen", type=int, default=0,
                     help="override the workload's sequence length (profiling captures)")
     return ap.parse_args()
@@ -209,6 +213,75 @@ def decode_bench(dev, stream, steps: int = 64, warmup: int = 5):
             "tokens_per_s": B / (ms / 1e3), "algorithmic_bytes_per_step": nbytes,
             "achieved_GBps": nbytes / (ms / 1e3) / 1e9, "kernels_us": per,
             "launches_per_step": nk}
+
+
+VARLEN_SEQS, VARLEN_TOKENS = 16, 32768
+
+
+def varlen_lengths(n: int = VARLEN_SEQS, total: int = VARLEN_TOKENS, seed: int = 11):
+    """Seeded prompt lengths for the packed-batch measurement: log-uniform in
+    [256, 8192] (SplitMix64 uniforms from synth), scaled to `total` tokens."""
+    from mamba_selective_scan_jamba_b200 import synth
+    u = synth.np_uniform(synth.stream_seed(seed, 99), n)
+    raw = np.exp(np.log(256.0) + u * (np.log(8192.0) - np.log(256.0)))
+    lens = np.maximum(1, np.floor(raw * total / raw.sum())).astype(np.int64)
+    lens[-1] += total - int(lens.sum())
+    return [int(v) for v in lens]
+
+
+def varlen_bench(dev, stream, steps: int = 20, warmup: int = 3):
+    """jm_mixer_fwd_varlen on a packed batch of VARLEN_SEQS prompts of mixed lengths
+    (VARLEN_TOKENS tokens in all) at Jamba shapes; returns a dict for the JSON line."""
+    import torch
+    from mamba_selective_scan_jamba_b200 import devio, jmix, synth
+    lens = varlen_lengths()
+    T = sum(lens)
+    base = synth.WORKLOADS["jamba_b8_l4096"]
+    w = base.with_(name="jamba_varlen", batch=1, seqlen=T)
+    W = synth.make_weights(base)
+    A = synth.make_activations(w)
+    Wd = devio.weights_to_device(W, dev)
+    x = devio.to_device(A["x"][0], dev)
+    z = devio.to_device(A["z"][0], dev)
+    y = torch.empty_like(x)
+    B = len(lens)
+    fs = torch.empty((B, w.d_inner, w.d_state), dtype=torch.float32, device=dev)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32, device=dev)
+    d = jmix.dims(B, T, w.d_inner, w.dt_rank, jmix.JM_BF16, w.eps)
+    n = jmix.jm_mixer_fwd_varlen_workspace_size(d)
+    ws = devio.workspace(n, dev)
+
+    def step():
+        jmix.jm_mixer_fwd_varlen(d, cu, x, z, Wd, y, fs, ws, n, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            step()
+    stream.synchronize()
+    nk = jmix.jm_last_launch_count()
+    names = [jmix.jm_last_kernel_name(i) for i in range(nk)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for row in evs:
+            for e in row:
+                e.record(stream)
+    stream.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        for i in range(steps):
+            jmix.jm_set_kernel_events([e.cuda_event for e in evs[i]])
+            step()
+        b.record(stream)
+    jmix.jm_set_kernel_events(None)
+    stream.synchronize()
+    assert jmix.jm_poll_error(ws, stream) == jmix.JM_OK, jmix.jm_last_error()
+    ms = a.elapsed_time(b) / steps
+    per = {names[k]: round(sum(evs[i][k].elapsed_time(evs[i][k + 1]) for i in range(steps))
+                           / steps, 4) for k in range(nk)}
+    return {"workload": "packed prefill at Jamba shapes", "sequences": B, "lengths": lens,
+            "tokens": T, "steps": steps, "ms_per_step": ms, "tokens_per_s": T / (ms / 1e3),
+            "kernels_ms": per, "launches_per_step": nk}
 
 
 # ------------------------------------------------------------- cpu baseline
@@ -452,6 +525,8 @@ def main():
                        "ms_per_step": ems, "steps": Ke,
                        "api": "jm_mixer_fwd_host (pinned host x, z -> y, final_state)"}
 
+    if args.varlen:
+        line["varlen"] = varlen_bench(dev, stream)
     if not args.no_decode:
         dec = decode_bench(dev, stream)
         dec["hbm_frac"] = dec["achieved_GBps"] / P["hbm"]

@@ -162,7 +162,9 @@ jm_status jm_mixer_fwd_host(const jm_dims* dims, const void* x_host, const void*
 /* Synchronises `stream`, then reads the error flags in `workspace`'s first
  * 256 bytes: JM_ERR_TIMEOUT if a bounded device-side wait ran out since the
  * last call that cleared them (every jm_mixer_fwd / jm_mixer_step clears
- * them), JM_ERR_CUDA if the stream reports an error, JM_OK otherwise. */
+ * them), JM_ERR_INVALID_ARG if a device-side input check failed (the
+ * cu_seqlens of jm_mixer_fwd_varlen), JM_ERR_CUDA if the stream reports an
+ * error, JM_OK otherwise. */
 jm_status jm_poll_error(void* workspace, jm_stream_t stream);
 
 /* Message of the last failed call on this thread ("" if none). */
@@ -175,6 +177,30 @@ int jm_last_launch_count(void);
 /* Name of the index-th kernel the last successful compute call on this thread
  * launched ("" when out of range).  The string is static. */
 const char* jm_last_kernel_name(int index);
+
+/* Forward over a packed batch of variable-length sequences (serving prefill).
+ * dims->batch = number of sequences B, dims->seqlen = total tokens T.
+ * x, z, y: [T, d_inner], the sequences one after another.  cu_seqlens: DEVICE
+ * int32 [B + 1] token offsets, cu_seqlens[0] = 0, nondecreasing,
+ * cu_seqlens[B] = T; sequence b is tokens cu_seqlens[b] .. cu_seqlens[b+1]-1
+ * (a sequence may be empty).  final_state, init_ssm_state: [B, d_inner, 16];
+ * init_conv_state, final_conv_state: [B, d_inner, 3], per sequence exactly as
+ * in jm_mixer_fwd (each sequence starts from its own initial states).  bf16 io
+ * only: JM_ERR_UNSUPPORTED for JM_F32.  The offsets live on the device, so
+ * they are checked there: a cu_seqlens that breaks the rules above leaves
+ * y and the states unspecified (no access leaves the buffers) and makes
+ * jm_poll_error return JM_ERR_INVALID_ARG.  Workspace:
+ * jm_mixer_fwd_varlen_workspace_size(dims).  Other arguments, errors and
+ * ownership as jm_mixer_fwd. */
+size_t jm_mixer_fwd_varlen_workspace_size(const jm_dims* dims);
+jm_status jm_mixer_fwd_varlen(const jm_dims* dims, const int32_t* cu_seqlens, const void* x,
+                              const void* z, const void* conv_w, const void* conv_b,
+                              const void* xproj_w, const void* dt_norm_w, const void* b_norm_w,
+                              const void* c_norm_w, const void* dtproj_w, const float* dt_bias,
+                              const float* A_log, const float* D, void* y, float* final_state,
+                              const void* init_conv_state, const float* init_ssm_state,
+                              void* final_conv_state, void* workspace, size_t ws_bytes,
+                              jm_stream_t stream);
 
 /* How jm_mixer_fwd will schedule the scan of this problem (bf16 I/O; float32
  * problems run one part per sequence).  Each sequence is cut into *n_parts time

@@ -197,11 +197,17 @@ static jm_status fwd_impl(const jm_dims* dims, const void* x, const void* z, con
                           const float* dt_bias, const float* A_log, const float* D, void* y,
                           float* final_state, const void* init_conv_state,
                           const float* init_ssm_state, void* final_conv_state, void* workspace,
-                          size_t ws_bytes, jm_stream_t stream, bool step, Problem& p) {
+                          size_t ws_bytes, jm_stream_t stream, bool step, Problem& p,
+                          const int32_t* cu = nullptr) {
   jm_status st = check_dims(dims, step);
   if (st != JM_OK) return st;
   fill_problem(p, dims);
   p.decode = step;
+  if (cu) {  // packed batch: seqlen is the total token count
+    p.T = dims->seqlen;
+    p.L = dims->seqlen;
+    p.cu = cu;
+  }
   const char* const wn[] = {"conv_w", "conv_b", "xproj_w", "dt_norm_w", "b_norm_w", "c_norm_w",
                             "dtproj_w", "dt_bias", "A_log", "D", "final_state"};
   const void* const wp[] = {conv_w, conv_b, xproj_w, dt_norm_w, b_norm_w, c_norm_w,
@@ -250,7 +256,7 @@ static jm_status fwd_impl(const jm_dims* dims, const void* x, const void* z, con
   p.events = g_events;
   p.n_events = g_n_events;
   if (p.B == 0) return finish(p, cudaSuccess);
-  if (p.L == 0) {
+  if (p.T == 0) {
     // nothing to scan: the final states are the initial ones
     const size_t ssz = (size_t)p.B * p.d * kN * 4, csz = (size_t)p.B * p.d * (kConv - 1) * es;
     cudaError_t e = init_ssm_state
@@ -278,6 +284,51 @@ JM_API jm_status jm_mixer_fwd(const jm_dims* dims, const void* x, const void* z,
   return fwd_impl(dims, x, z, conv_w, conv_b, xproj_w, dt_norm_w, b_norm_w, c_norm_w, dtproj_w,
                   dt_bias, A_log, D, y, final_state, init_conv_state, init_ssm_state,
                   final_conv_state, workspace, ws_bytes, stream, false, p);
+}
+
+JM_API size_t jm_mixer_fwd_varlen_workspace_size(const jm_dims* dims) {
+  // the packed batch needs what a batch of one sequence of T tokens needs, plus
+  // nothing per sequence beyond the states the caller passes
+  if (check_dims(dims, false) != JM_OK || dims->io != JM_BF16) return 0;
+  Problem p;
+  fill_problem(p, dims);
+  p.T = dims->seqlen;
+  p.L = dims->seqlen;
+  p.cu = reinterpret_cast<const int*>(uintptr_t(1));  // layout of the packed form
+  return ws_bytes_for(p);
+}
+
+JM_API jm_status jm_mixer_fwd_varlen(const jm_dims* dims, const int32_t* cu_seqlens,
+                                     const void* x, const void* z, const void* conv_w,
+                                     const void* conv_b, const void* xproj_w,
+                                     const void* dt_norm_w, const void* b_norm_w,
+                                     const void* c_norm_w, const void* dtproj_w,
+                                     const float* dt_bias, const float* A_log, const float* D,
+                                     void* y, float* final_state, const void* init_conv_state,
+                                     const float* init_ssm_state, void* final_conv_state,
+                                     void* workspace, size_t ws_bytes, jm_stream_t stream) {
+  jm_status st = check_dims(dims, false);
+  if (st != JM_OK) return st;
+  if (dims->io != JM_BF16) {
+    set_error("jm_mixer_fwd_varlen is built for bf16 io only");
+    return JM_ERR_UNSUPPORTED;
+  }
+  if (!cu_seqlens) {
+    set_error("cu_seqlens is NULL");
+    return JM_ERR_INVALID_ARG;
+  }
+  if (!aligned(cu_seqlens, 4)) {
+    set_error("cu_seqlens is not 4-byte aligned");
+    return JM_ERR_INVALID_ARG;
+  }
+  if (dims->seqlen > 0x7fffffffLL) {
+    set_error("total tokens must fit int32 offsets");
+    return JM_ERR_INVALID_ARG;
+  }
+  Problem p;
+  return fwd_impl(dims, x, z, conv_w, conv_b, xproj_w, dt_norm_w, b_norm_w, c_norm_w, dtproj_w,
+                  dt_bias, A_log, D, y, final_state, init_conv_state, init_ssm_state,
+                  final_conv_state, workspace, ws_bytes, stream, false, p, cu_seqlens);
 }
 
 JM_API jm_status jm_mixer_step(const jm_dims* dims, const void* x_t, const void* z_t,
@@ -370,6 +421,10 @@ JM_API jm_status jm_poll_error(void* workspace, jm_stream_t stream) {
   if (f.timeout) {
     set_error("a bounded device-side wait ran out (site %u)", f.where);
     return JM_ERR_TIMEOUT;
+  }
+  if (f.bad_input) {
+    set_error("cu_seqlens is not 0 = c[0] <= c[1] <= ... <= c[B] = total tokens");
+    return JM_ERR_INVALID_ARG;
   }
   return JM_OK;
 }

@@ -15,9 +15,10 @@ constexpr int kMaxRank = 256;
 
 // The first 256 bytes of every workspace.
 struct ErrFlags {
-  unsigned int timeout;   // a bounded wait ran out
-  unsigned int where;     // kernel-specific code of the first wait that ran out
-  unsigned int pad[62];
+  unsigned int timeout;    // a bounded wait ran out
+  unsigned int where;      // kernel-specific code of the first wait that ran out
+  unsigned int bad_input;  // device-side input check failed (cu_seqlens of a packed batch)
+  unsigned int pad[61];
 };
 static_assert(sizeof(ErrFlags) == 256, "error header is 256 bytes");
 
@@ -47,6 +48,7 @@ struct Problem {
   size_t ws_bytes;
   cudaStream_t stream;
   bool decode;             // jm_mixer_step
+  const int* cu;           // packed batch: [B + 1] token offsets (device); L == T then
   int launches;            // kernels launched so far by this call
   void* const* events;     // optional per-kernel timing events (jm_set_kernel_events)
   int n_events;

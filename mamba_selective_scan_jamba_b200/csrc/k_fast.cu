@@ -99,6 +99,131 @@ __device__ __forceinline__ float silu_newton(float v) {
   return v * r;
 }
 
+// The packed-batch form of k_conv_silu16: thread = 8 channels x 8 consecutive
+// tokens of the packed [T, d] stream, which may span sequence boundaries.  Each
+// token's sequence comes from a binary search in cu (B + 1 offsets); its taps
+// before the sequence's first token come from that sequence's history (or are
+// zero).  Indices are clamped so that a broken cu (reported by the scan kernel)
+// cannot reach outside x or hist.  Threads past the conv range convert weights.
+__global__ void __launch_bounds__(256, JMIX_CONV_OCC) k_conv_silu16_packed(
+    const bf16* __restrict__ x, const bf16* __restrict__ conv_w, const bf16* __restrict__ conv_b,
+    const bf16* __restrict__ hist, const int* __restrict__ cu, int64_t B, int64_t T, int64_t d,
+    __half* __restrict__ u, int64_t n_conv, const bf16* __restrict__ wx, int64_t n_wx8,
+    __half* __restrict__ wx16, const bf16* __restrict__ wdt, int64_t n_wdt8,
+    __half* __restrict__ wdt16) {
+  constexpr int G = 8, kW = kConv - 1;
+  const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (tid < n_conv) {
+    const int64_t ncg = d >> 3;
+    const int64_t cg = tid % ncg, tg = tid / ncg;
+    const int64_t c0 = cg * 8, t0 = tg * G;
+    const int nt = (int)((T - t0) < G ? (T - t0) : G);
+    // rows[i] = packed token t0 - 3 + i (zero outside [0, T))
+    uint4 rows[kW + G];
+#pragma unroll
+    for (int i = 0; i < kW + G; ++i) {
+      const int64_t tau = t0 - kW + i;
+      rows[i] = (tau >= 0 && i < kW + nt)
+                    ? __ldg(reinterpret_cast<const uint4*>(x + tau * d + c0))
+                    : make_uint4(0u, 0u, 0u, 0u);
+    }
+    // sequence of token t0: the last b with cu[b] <= t0
+    int lo = 0, hi = (int)B - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (__ldg(cu + mid) <= t0) lo = mid; else hi = mid - 1;
+    }
+    const int64_t s0 = __ldg(cu + lo);
+    const int64_t s_next = lo + 1 < B ? __ldg(cu + lo + 1) : T;
+    // common case: every tap of the 8 tokens is inside one sequence
+    const bool inner = t0 - kW >= s0 && t0 + G <= s_next;
+    uint4 wq[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      wq[q] = __ldg(reinterpret_cast<const uint4*>(conv_w + c0 * kConv) + q);
+    const uint4 bq = __ldg(reinterpret_cast<const uint4*>(conv_b + c0));
+    uint32_t outp[G][4];
+    if (inner) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        float xe[kW + G];
+#pragma unroll
+        for (int i = 0; i < kW + G; ++i) xe[i] = bf16_lane(rows[i], e);
+        float wk[kConv];
+#pragma unroll
+        for (int k = 0; k < kConv; ++k)
+          wk[k] = bf16_lane(wq[(e * kConv + k) >> 3], (e * kConv + k) & 7);
+        const float be = bf16_lane(bq, e);
+#pragma unroll
+        for (int i = 0; i < G; ++i) {
+          float acc = be;
+#pragma unroll
+          for (int k = 0; k < kConv; ++k) acc = fmaf(wk[k], xe[i + k], acc);
+          const uint32_t hb = (uint32_t)__half_as_ushort(to_half_sat(silu_u(acc)));
+          if (e & 1)
+            outp[i][e >> 1] |= hb << 16;
+          else
+            outp[i][e >> 1] = hb;
+        }
+      }
+    } else {
+      // a sequence starts inside the window: per token, its sequence and start
+#pragma unroll
+      for (int i = 0; i < G; ++i) {
+        int bi = lo;
+        while (bi + 1 < B && __ldg(cu + bi + 1) <= t0 + i) ++bi;
+        const int64_t sti = __ldg(cu + bi);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          float acc = bf16_lane(bq, e);
+#pragma unroll
+          for (int k = 0; k < kConv; ++k) {
+            const int64_t tau = t0 + i - kW + k;
+            float v = bf16_lane(rows[i + k], e);
+            if (tau < sti) {
+              // before the sequence's start: its history (positions -3 .. -1), else zero
+              const int64_t hp = kW + (tau - sti);
+              v = (hist && hp >= 0 && hp < kW) ? bf(hist[((int64_t)bi * d + c0 + e) * kW + hp])
+                                               : 0.0f;
+            }
+            acc = fmaf(bf16_lane(wq[(e * kConv + k) >> 3], (e * kConv + k) & 7), v, acc);
+          }
+          const uint32_t hb = (uint32_t)__half_as_ushort(to_half_sat(silu_u(acc)));
+          if (e & 1)
+            outp[i][e >> 1] |= hb << 16;
+          else
+            outp[i][e >> 1] = hb;
+        }
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < G; ++i) {
+      if (i >= nt) break;
+      *reinterpret_cast<uint4*>(u + (t0 + i) * d + c0) =
+          make_uint4(outp[i][0], outp[i][1], outp[i][2], outp[i][3]);
+    }
+    return;
+  }
+  int64_t i = tid - n_conv;
+  const bf16* src;
+  __half* dst;
+  if (i < n_wx8) {
+    src = wx;
+    dst = wx16;
+  } else if ((i -= n_wx8) < n_wdt8) {
+    src = wdt;
+    dst = wdt16;
+  } else {
+    return;
+  }
+  float o[8];
+  unpack8_bf16(__ldg(reinterpret_cast<const uint4*>(src) + i), o);
+  __align__(16) __half h[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) h[e] = __float2half_rn(o[e]);
+  reinterpret_cast<uint4*>(dst)[i] = *reinterpret_cast<uint4*>(h);
+}
+
 template <int kConvG>
 __global__ void __launch_bounds__(256, JMIX_CONV_OCC) k_conv_silu16(
     const bf16* __restrict__ x, const bf16* __restrict__ conv_w, const bf16* __restrict__ conv_b,
@@ -467,6 +592,9 @@ struct ScanArgs {
   ErrFlags* err;
   // Work schedule (see k_scan_fused).  A pair is one (sequence, 128-channel
   // tile); each pair's sequence is cut into n_parts time parts of whole chunks.
+  int64_t B;       // sequences
+  const int* cu;   // packed batch: [B + 1] token offsets (else sequence b is tokens b*L ..)
+  const int* order;  // packed batch: sequences longest first (claim order), or null
   int n_tiles;     // channel tiles per sequence
   int n_parts;     // time parts per sequence
   int two_pass;    // 0: parts run in a chain; 1: state pass, then output pass
@@ -622,7 +750,8 @@ template <bool kOut>
 __device__ __forceinline__ void scan_chunks(const ScanArgs& a, const uint8_t* stage0,
                                             uint64_t* full, uint64_t* mma_done, uint64_t* empty,
                                             uint32_t tmem, int warp, int lane, int kg0, int kb,
-                                            int nch, bool cok, bf16* yrow, float2 (&h)[kN / 2],
+                                            int nch, int64_t Lb, bool cok, bf16* yrow,
+                                            float2 (&h)[kN / 2],
                                             const float2 (&A2)[kN / 2], float (&xw)[kConv - 1],
                                             const float (&cw)[kConv], float cb, float bias,
                                             float Dc, float& ssum) {
@@ -639,7 +768,7 @@ __device__ __forceinline__ void scan_chunks(const ScanArgs& a, const uint8_t* st
     const bf16* zs = reinterpret_cast<const bf16*>(st + kDtnStage + kXStage);
     const float4* bcs = reinterpret_cast<const float4*>(st + kDtnStage + 2 * kXStage);
     const int64_t tbase = (int64_t)(kb + k) * kSQ;
-    const int nt = (int)((a.L - tbase) < kSQ ? (a.L - tbase) : kSQ);
+    const int nt = (int)((Lb - tbase) < kSQ ? (Lb - tbase) : kSQ);
     const uint32_t tacc = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(s * kSQ);
     float csum = 0.0f;
 #pragma unroll 1
@@ -716,6 +845,27 @@ __device__ __forceinline__ void scan_chunks(const ScanArgs& a, const uint8_t* st
   }
 }
 
+// Claim order of a packed batch's sequences: longest first (ties by index), so
+// that the long sequences, which set the scan's critical path, start first.
+// One CTA; rank of b = number of sequences that come before it.  Lengths of a
+// broken cu are clamped to [0, T] here (the scan kernel reports it).
+__global__ void __launch_bounds__(1024) k_order_by_length(const int* __restrict__ cu, int B,
+                                                         int T, int* __restrict__ order) {
+  for (int b = threadIdx.x; b < B; b += blockDim.x) {
+    auto len = [&](int i) {
+      const int v = __ldg(cu + i + 1) - __ldg(cu + i);
+      return v < 0 ? 0 : (v > T ? T : v);
+    };
+    const int lb = len(b);
+    int rank = 0;
+    for (int i = 0; i < B; ++i) {
+      const int li = len(i);
+      rank += (li > lb) || (li == lb && i < b);
+    }
+    order[rank] = b;  // ranks are a permutation of 0 .. B-1
+  }
+}
+
 // Fused dt_proj (tcgen05, accumulator in TMEM) + softplus + selective scan +
 // D skip + SiLU(z) gate, with the causal conv + SiLU recomputed in fp32 from x.
 //
@@ -754,9 +904,7 @@ __global__ void __launch_bounds__(kScanThreads, kScanCtasPerSm)
   const int nslab_t = a.nslab < kWdtTmemSlabs ? a.nslab : kWdtTmemSlabs;  // slabs in TMEM
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nch_all = (int)((a.L + kSQ - 1) / kSQ);
-  const int64_t B = a.T / a.L;
-  const int pairs = a.n_tiles * (int)B;
+  const int pairs = a.n_tiles * (int)a.B;
   const int P = a.n_parts;
   const int n_state = a.two_pass ? pairs * (P - 1) : 0;  // state units come first
   const int n_units = n_state + pairs * P;
@@ -797,10 +945,25 @@ __global__ void __launch_bounds__(kScanThreads, kScanCtasPerSm)
     const int uu = out ? unit - n_state : unit;
     const int part = uu / pairs;
     const int pair = uu - part * pairs;
-    const int64_t b = pair / a.n_tiles;
-    const int tile = pair - (int)b * a.n_tiles;
+    const int64_t bq = pair / a.n_tiles;
+    const int tile = pair - (int)bq * a.n_tiles;
+    const int64_t b = a.order ? a.order[bq] : bq;  // packed: longest sequences are claimed first
     const int64_t c0 = (int64_t)tile * kSC;
-    const int64_t g0 = b * a.L;
+    // the sequence's first token and length (packed batch: from cu, checked here;
+    // a broken cu is reported and the sequence treated as empty)
+    int64_t g0 = b * a.L, Lb = a.L;
+    if (a.cu) {
+      const int s0 = a.cu[b], s1 = a.cu[b + 1];
+      if (s0 < 0 || s1 < s0 || s1 > a.T || (b == 0 && s0 != 0) || (b == a.B - 1 && s1 != a.T)) {
+        if (threadIdx.x == 0) atomicExch(&a.err->bad_input, 1u);
+        g0 = 0;
+        Lb = 0;
+      } else {
+        g0 = s0;
+        Lb = s1 - s0;
+      }
+    }
+    const int nch_all = (int)((Lb + kSQ - 1) / kSQ);
     const int kb = (int)((int64_t)nch_all * part / P);
     const int nch = (int)((int64_t)nch_all * (part + 1) / P) - kb;
     const int64_t hslot = (int64_t)pair * P + part;  // this part's hand-over slot
@@ -965,11 +1128,11 @@ __global__ void __launch_bounds__(kScanThreads, kScanCtasPerSm)
       }
       float ssum = 0.0f;
       if (out)
-        scan_chunks<true>(a, stage0, full, mma_done, empty, tmem, warp, lane, kg0, kb, nch, cok,
-                          a.y + g0 * a.d + c, h, A2, xw, cw, cb, bias, Dc, ssum);
+        scan_chunks<true>(a, stage0, full, mma_done, empty, tmem, warp, lane, kg0, kb, nch, Lb,
+                          cok, a.y + g0 * a.d + c, h, A2, xw, cw, cb, bias, Dc, ssum);
       else
-        scan_chunks<false>(a, stage0, full, mma_done, empty, tmem, warp, lane, kg0, kb, nch, cok,
-                           nullptr, h, A2, xw, cw, cb, bias, Dc, ssum);
+        scan_chunks<false>(a, stage0, full, mma_done, empty, tmem, warp, lane, kg0, kb, nch, Lb,
+                           cok, nullptr, h, A2, xw, cw, cb, bias, Dc, ssum);
       if (part + 1 < P && (!out || !a.two_pass)) {
         // hand the end state (and, two-pass, the sum of delta) to later parts
         float* ch = a.carry_h + hslot * kSC * kN + cl * kN;
@@ -1251,6 +1414,7 @@ struct FastWs {
   int* sched;         // [0] unit counter, [1..] hand-over flags of the scan's parts
   float* carry_h;     // scan hand-over: end state per (pair, part)
   float* carry_s;     // scan hand-over: sum of delta per (pair, part)
+  int* order;         // packed batch: claim order of the sequences
   ScanPlan plan;
   size_t bytes;
   size_t zero_bytes;  // error header + scheduler words, cleared each call
@@ -1280,7 +1444,7 @@ FastWs fast_layout(const Problem& pr, char* base) {
   };
   const size_t T = (size_t)pr.T, d = (size_t)pr.d, P = (size_t)pr.P, R = (size_t)pr.R;
   w.ksplit = xproj_ksplit(pr.T, pr.d);
-  if (!pr.decode) w.plan = scan_plan(pr.B, pr.L, pr.d);
+  if (!pr.decode && !pr.cu) w.plan = scan_plan(pr.B, pr.L, pr.d);  // packed: one part each
   // hand-over slots: one per (pair, part) when parts exist
   const size_t slots = w.plan.n_parts > 1
                            ? (size_t)pr.B * (size_t)((pr.d + kSC - 1) / kSC) * w.plan.n_parts
@@ -1290,6 +1454,7 @@ FastWs fast_layout(const Problem& pr, char* base) {
   w.zero_bytes = off;
   w.carry_h = reinterpret_cast<float*>(take(slots * kSC * kN * 4));
   w.carry_s = reinterpret_cast<float*>(take(slots * kSC * 4));
+  w.order = pr.cu ? reinterpret_cast<int*>(take((size_t)pr.B * 4)) : nullptr;
   w.part = reinterpret_cast<float*>(take((size_t)w.ksplit * T * P * 4));
   w.u = reinterpret_cast<__half*>(take(T * d * 2));
   w.dtn = reinterpret_cast<__half*>(take(T * R * 2));
@@ -1325,11 +1490,19 @@ cudaError_t run_fast_fwd(Problem& p) {
     const int64_t n_conv = (p.d / 8) * ((p.L + G - 1) / G) * p.B;
     const int64_t n_wx8 = (int64_t)p.P * p.d / 8, n_wdt8 = p.d * p.R / 8;
     const int64_t total = n_conv + n_wx8 + n_wdt8;
-    auto kern = G == kConvG ? k_conv_silu16<kConvG> : k_conv_silu16<1>;
-    kern<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
-        (const bf16*)p.x, (const bf16*)p.conv_w, (const bf16*)p.conv_b, (const bf16*)p.init_conv,
-        p.B, p.L, p.d, w.u, n_conv, (const bf16*)p.xproj_w, n_wx8, w.wx,
-        (const bf16*)p.dtproj_w, n_wdt8, w.wdt);
+    if (p.cu) {
+      const int64_t n_pk = (p.d / 8) * ((p.T + 7) / 8);
+      k_conv_silu16_packed<<<(unsigned)((n_pk + n_wx8 + n_wdt8 + 255) / 256), 256, 0, s>>>(
+          (const bf16*)p.x, (const bf16*)p.conv_w, (const bf16*)p.conv_b,
+          (const bf16*)p.init_conv, p.cu, p.B, p.T, p.d, w.u, n_pk, (const bf16*)p.xproj_w,
+          n_wx8, w.wx, (const bf16*)p.dtproj_w, n_wdt8, w.wdt);
+    } else {
+      auto kern = G == kConvG ? k_conv_silu16<kConvG> : k_conv_silu16<1>;
+      kern<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
+          (const bf16*)p.x, (const bf16*)p.conv_w, (const bf16*)p.conv_b,
+          (const bf16*)p.init_conv, p.B, p.L, p.d, w.u, n_conv, (const bf16*)p.xproj_w, n_wx8,
+          w.wx, (const bf16*)p.dtproj_w, n_wdt8, w.wdt);
+    }
     launched(p, "k_conv_silu16");
   }
   // 2. x_proj on tcgen05
@@ -1411,6 +1584,14 @@ cudaError_t run_fast_fwd(Problem& p) {
       return cudaErrorInvalidValue;
     ScanArgs sa;
     sa.L = p.L;
+    sa.B = p.B;
+    sa.cu = p.cu;
+    sa.order = nullptr;
+    if (p.cu && p.B > 1 && p.B <= 8192) {  // O(B^2) ranking: up to a few thousand prompts
+      k_order_by_length<<<1, 1024, 0, s>>>(p.cu, (int)p.B, (int)p.T, w.order);
+      launched(p, "k_order_by_length");
+      sa.order = w.order;
+    }
     sa.d = p.d;
     sa.T = p.T;
     sa.R = (int)p.R;

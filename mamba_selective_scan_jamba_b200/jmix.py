@@ -25,7 +25,8 @@ WEIGHT_NAMES = ("conv_w", "conv_b", "xproj_w", "dt_norm_w", "b_norm_w", "c_norm_
 EXPORTED = ("jm_mixer_fwd_workspace_size", "jm_mixer_step_workspace_size", "jm_mixer_fwd",
             "jm_mixer_step", "jm_mixer_fwd_host", "jm_poll_error", "jm_last_error",
             "jm_last_launch_count", "jm_last_kernel_name", "jm_set_kernel_events",
-            "jm_mixer_step_noalloc", "jm_mixer_fwd_schedule")
+            "jm_mixer_step_noalloc", "jm_mixer_fwd_schedule",
+            "jm_mixer_fwd_varlen_workspace_size", "jm_mixer_fwd_varlen")
 
 
 class jm_dims(ctypes.Structure):
@@ -66,6 +67,11 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.jm_mixer_step_noalloc.argtypes = [ctypes.POINTER(jm_dims)] + [_vp] * 15 + [_vp]
     lib.jm_mixer_fwd_host.restype = ctypes.c_int
     lib.jm_mixer_fwd_host.argtypes = [ctypes.POINTER(jm_dims)] + [_vp] * 19 + [ctypes.c_size_t, _vp]
+    lib.jm_mixer_fwd_varlen_workspace_size.restype = ctypes.c_size_t
+    lib.jm_mixer_fwd_varlen_workspace_size.argtypes = [ctypes.POINTER(jm_dims)]
+    lib.jm_mixer_fwd_varlen.restype = ctypes.c_int
+    lib.jm_mixer_fwd_varlen.argtypes = ([ctypes.POINTER(jm_dims)] + [_vp] * 19
+                                        + [ctypes.c_size_t, _vp])
     lib.jm_mixer_fwd_schedule.restype = ctypes.c_int
     lib.jm_mixer_fwd_schedule.argtypes = [ctypes.POINTER(jm_dims), ctypes.POINTER(ctypes.c_int),
                                           ctypes.POINTER(ctypes.c_int)]
@@ -136,6 +142,25 @@ def jm_mixer_fwd(d: jm_dims, x, z, w: Mapping, y, final_state, workspace, ws_byt
     st = load().jm_mixer_fwd(ctypes.byref(d), _ptr(x), _ptr(z), *_weights(w), _ptr(y),
                              _ptr(final_state), _ptr(init_conv_state), _ptr(init_ssm_state),
                              _ptr(final_conv_state), _ptr(workspace), ws_bytes, _stream(stream))
+    if check:
+        _check(st)
+    return st
+
+
+def jm_mixer_fwd_varlen_workspace_size(d: jm_dims) -> int:
+    return load().jm_mixer_fwd_varlen_workspace_size(ctypes.byref(d))
+
+
+def jm_mixer_fwd_varlen(d: jm_dims, cu_seqlens, x, z, w: Mapping, y, final_state, workspace,
+                        ws_bytes: int, init_conv_state=None, init_ssm_state=None,
+                        final_conv_state=None, stream=None, check: bool = True) -> int:
+    """Packed batch: d.batch sequences, d.seqlen total tokens; cu_seqlens is a device
+    int32 tensor of d.batch + 1 offsets."""
+    st = load().jm_mixer_fwd_varlen(ctypes.byref(d), _ptr(cu_seqlens), _ptr(x), _ptr(z),
+                                    *_weights(w), _ptr(y), _ptr(final_state),
+                                    _ptr(init_conv_state), _ptr(init_ssm_state),
+                                    _ptr(final_conv_state), _ptr(workspace), ws_bytes,
+                                    _stream(stream))
     if check:
         _check(st)
     return st

@@ -163,3 +163,25 @@ def test_scan_schedule_rules(lib):
                     assert waves(n) < waves(1)
     with pytest.raises(jmix.JmixError):
         jmix.jm_mixer_fwd_schedule(jmix.dims(1, 10, 100, 16))   # d % 8 != 0
+
+
+def test_varlen_host_checks(lib):
+    FAKE = 1 << 40
+    W = {k: FAKE for k in jmix.WEIGHT_NAMES}
+    d = jmix.dims(3, 100, 256, 16)
+    n = jmix.jm_mixer_fwd_varlen_workspace_size(d)
+    assert n > 0
+    assert jmix.jm_mixer_fwd_varlen_workspace_size(jmix.dims(3, 100, 256, 16, io=jmix.JM_F32)) == 0
+    st = jmix.jm_mixer_fwd_varlen(d, None, FAKE, FAKE, W, FAKE + (1 << 30), FAKE, FAKE, n,
+                                  stream=0, check=False)
+    assert st == jmix.JM_ERR_INVALID_ARG and "cu_seqlens" in jmix.jm_last_error()
+    st = jmix.jm_mixer_fwd_varlen(d, FAKE + 2, FAKE, FAKE, W, FAKE + (1 << 30), FAKE, FAKE, n,
+                                  stream=0, check=False)
+    assert st == jmix.JM_ERR_INVALID_ARG and "aligned" in jmix.jm_last_error()
+    f32 = jmix.dims(3, 100, 256, 16, io=jmix.JM_F32)
+    st = jmix.jm_mixer_fwd_varlen(f32, FAKE, FAKE, FAKE, W, FAKE + (1 << 30), FAKE, FAKE, n,
+                                  stream=0, check=False)
+    assert st == jmix.JM_ERR_UNSUPPORTED
+    st = jmix.jm_mixer_fwd_varlen(d, FAKE, FAKE, FAKE, W, FAKE + (1 << 30), FAKE, FAKE, 256,
+                                  stream=0, check=False)
+    assert st == jmix.JM_ERR_WORKSPACE
