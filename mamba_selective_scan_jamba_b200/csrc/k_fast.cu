@@ -1421,15 +1421,18 @@ struct FastWs {
   int ksplit;
 };
 
+#ifndef JMIX_XSPLIT_MAX
+#define JMIX_XSPLIT_MAX 32
+#endif
 // x_proj split over d_inner: about two CTAs per SM of a B200 (2 x 148), at
-// most 64 splits, at least one 64-channel chunk per split.  Depends on the
+// most JMIX_XSPLIT_MAX splits, at least one 64-channel chunk per split.  Depends on the
 // problem only, so the workspace size does too.
 int xproj_ksplit(int64_t T, int64_t d) {
   if (T <= 0) return 1;
   const int64_t mtiles = (T + kXM - 1) / kXM;
   const int64_t kchunks = (d + kXK - 1) / kXK;
   int64_t ks = (296 + mtiles - 1) / mtiles;
-  if (ks > 64) ks = 64;
+  if (ks > JMIX_XSPLIT_MAX) ks = JMIX_XSPLIT_MAX;
   if (ks > kchunks) ks = kchunks;
   return ks < 1 ? 1 : (int)ks;
 }
