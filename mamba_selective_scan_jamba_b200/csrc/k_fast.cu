@@ -1179,7 +1179,11 @@ __global__ void __launch_bounds__(kScanThreads, kScanCtasPerSm)
 // sequences: conv + SiLU from the cached conv state, softplus, the 16-state
 // update in place, the gate, and the conv-state shift.  The SSM state read and
 // write (64 B each per (sequence, channel)) is the HBM traffic that bounds it.
-constexpr int kDB = 16;                                   // sequences per CTA (MMA N)
+#ifndef JMIX_DEC_DB
+#define JMIX_DEC_DB 16
+#endif
+constexpr int kDB = JMIX_DEC_DB;                          // sequences per CTA (MMA N)
+static_assert(kDB % 16 == 0 && kDB <= 32, "16 or 32 sequences per CTA");
 constexpr int kDecThreads = 160;
 constexpr int kDecDtn = kMaxSlabs * kDB * 128;            // 8 KB
 constexpr int kDecBC = kDB * 2 * kN * 4;                  // 2 KB
@@ -1201,7 +1205,15 @@ struct DecArgs {
   ErrFlags* err;
 };
 
-__global__ void __launch_bounds__(kDecThreads, 2)
+#ifndef JMIX_DEC_OCC
+#define JMIX_DEC_OCC 2
+#endif
+#ifndef JMIX_DEC_AHEAD
+#define JMIX_DEC_AHEAD 2
+#endif
+constexpr int kDecAhead = JMIX_DEC_AHEAD;  // sequences whose inputs are in flight per thread
+
+__global__ void __launch_bounds__(kDecThreads, JMIX_DEC_OCC)
     k_decode_scan(const __grid_constant__ CUtensorMap tm_wdt,
                   const __grid_constant__ CUtensorMap tm_dtn,
                   const __grid_constant__ CUtensorMap tm_bc, const DecArgs a) {
@@ -1264,7 +1276,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     const int64_t c = c0 + cl;
     const bool cok = c < a.d;
     const int nb = (int)((a.B - b0) < kDB ? (a.B - b0) : kDB);
-    // per-column inputs, loaded two columns ahead (they do not depend on delta,
+    // per-column inputs, loaded kDecAhead columns ahead (they do not depend on delta,
     // so the first loads go out before the dt_proj accumulator is ready)
     struct Col {
       float4 h[4];
@@ -1285,9 +1297,9 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         cd.z = bf(a.z[bc]);
       }
     };
-    Col cbuf[2];
-    load_col(0, cbuf[0]);
-    load_col(1, cbuf[1]);
+    Col cbuf[kDecAhead];
+#pragma unroll
+    for (int k = 0; k < kDecAhead; ++k) load_col(k, cbuf[k]);
     float2 A2[kN / 2];
     float bias = 0.f, Dc = 0.f, cb = 0.f, cw[kConv] = {0.f, 0.f, 0.f, 0.f};
     if (cok) {
@@ -1306,13 +1318,16 @@ __global__ void __launch_bounds__(kDecThreads, 2)
                     mbar_wait(smem_u32(full), 0, a.err, 33);
     tc_fence_after();
     uint32_t r[kDB];
-    tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16), r);
+#pragma unroll
+    for (int q = 0; q < kDB / 16; ++q)
+      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(16 * q),
+                *reinterpret_cast<uint32_t(*)[16]>(r + 16 * q));
     tmem_ld_wait();
     if (ok && cok) {
 #pragma unroll
       for (int j = 0; j < kDB; ++j) {
         if (j >= nb) break;
-        Col& cd = cbuf[j & 1];
+        Col& cd = cbuf[j % kDecAhead];
         const int64_t bc = (b0 + j) * a.d + c;
         const float xt = bf(cd.xb);
         float xc = fmaf(cw[0], cd.s[0], cb);
@@ -1348,7 +1363,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         const float ys = (sa.x + sa.y) + Dc * uv;
         const bf16 xkeep = cd.xb;
         const float s1 = cd.s[1], s2 = cd.s[2], zv = cd.z;
-        load_col(j + 2, cd);   // refill this slot two columns ahead
+        load_col(j + kDecAhead, cd);   // refill this slot kDecAhead columns ahead
         a.y[bc] = __float2bfloat16_rn(ys * silu_gate(zv));
         float4* st = reinterpret_cast<float4*>(a.ssm_state + bc * kN);
 #pragma unroll
