@@ -36,7 +36,8 @@ class OrcDims(ctypes.Structure):
                 ("d_inner", ctypes.c_int64), ("d_state", ctypes.c_int64),
                 ("d_conv", ctypes.c_int64), ("dt_rank", ctypes.c_int64),
                 ("eps", ctypes.c_double), ("mirror_bf16", ctypes.c_int32),
-                ("threads", ctypes.c_int32)]
+                ("threads", ctypes.c_int32), ("zoh", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
 
 
 def build(force: bool = False) -> str:
@@ -83,14 +84,17 @@ def _p(a: Optional[np.ndarray]):
 
 
 def dims(batch, seqlen, d_inner, dt_rank, d_state=16, d_conv=4, eps=1e-6, mirror=False,
-         threads=0) -> OrcDims:
-    return OrcDims(batch, seqlen, d_inner, d_state, d_conv, dt_rank, eps, int(mirror), threads)
+         threads=0, zoh=False) -> OrcDims:
+    """zoh: discretise B by zero-order hold, (exp(delta A) - 1) / A * B, instead of delta B."""
+    return OrcDims(batch, seqlen, d_inner, d_state, d_conv, dt_rank, eps, int(mirror), threads,
+                   int(zoh), 0)
 
 
-def dims_of(w, mirror=False, threads=0, batch=None, seqlen=None) -> OrcDims:
-    """Oracle dims from a synth.Workload-like object."""
+def dims_of(w, mirror=False, threads=0, batch=None, seqlen=None, zoh=None) -> OrcDims:
+    """Oracle dims from a synth.Workload-like object (zoh defaults to the workload's)."""
     return dims(w.batch if batch is None else batch, w.seqlen if seqlen is None else seqlen,
-                w.d_inner, w.dt_rank, w.d_state, w.d_conv, w.eps, mirror, threads)
+                w.d_inner, w.dt_rank, w.d_state, w.d_conv, w.eps, mirror, threads,
+                getattr(w, "zoh", False) if zoh is None else zoh)
 
 
 _WNAMES = ("conv_w", "conv_b", "xproj_w", "dt_norm_w", "b_norm_w", "c_norm_w", "dtproj_w",
@@ -144,16 +148,17 @@ def rmsnorm(v, w, eps) -> np.ndarray:
     return out
 
 
-def scan(delta, A, Bm, Cm, u, D, h0=None):
+def scan(delta, A, Bm, Cm, u, D, h0=None, zoh=False):
     """Selective scan of one sequence.  delta, u [L,d]; A [d,N] (negative reals);
-    Bm, Cm [L,N]; D [d]; h0 [d,N].  Returns (y_s [L,d], h_T [d,N])."""
+    Bm, Cm [L,N]; D [d]; h0 [d,N].  Returns (y_s [L,d], h_T [d,N]).  zoh: B
+    discretised by zero-order hold instead of delta B."""
     delta, A, Bm, Cm, u, D, h0 = map(_f64, (delta, A, Bm, Cm, u, D, h0))
     L, d = delta.shape
     N = A.shape[1]
     y = np.empty((L, d))
     hT = np.empty((d, N))
     _L().orc_scan(ctypes.c_int64(L), ctypes.c_int64(d), ctypes.c_int64(N), _p(delta), _p(A),
-                  _p(Bm), _p(Cm), _p(u), _p(D), _p(h0), _p(y), _p(hT))
+                  _p(Bm), _p(Cm), _p(u), _p(D), _p(h0), _p(y), _p(hT), ctypes.c_int32(int(zoh)))
     return y, hT
 
 

@@ -30,6 +30,12 @@
 //   6. gate: y = ys * z / (1 + exp(-z)).  Final SSM state = h after the last
 //      token; final conv state = the last K-1 conv inputs, oldest first.
 //
+// Discretisation of B (orc_dims.zoh): 0 = Euler, Bbar = delta B (the guide's
+// "Bbar ~ delta B"); 1 = zero-order hold, Bbar = (exp(delta A) - 1) / A * B,
+// the exact one-step solution of dh/dt = A h + B u for u held over the step
+// (the guide's continuous-time form, "Selective State Space Model (S6) Forward
+// Flow"), taken here as expm1(delta A) / A.
+//
 // Mirror mode (mirror_bf16 = 1) rounds where the bf16-io CUDA path quantises
 // an intermediate: the two tensor-core operands, u as the x_proj operand and
 // dt_n as the dt_proj operand, both stored as IEEE fp16.  The rounding is taken
@@ -107,6 +113,9 @@ struct Stored {
 
 double softplus(double v) { return std::max(v, 0.0) + std::log1p(std::exp(-std::fabs(v))); }
 
+// The factor that multiplies B u in the state update (see zoh above).
+double bbar(double dl, double A, int32_t zoh) { return zoh ? std::expm1(dl * A) / A : dl; }
+
 }  // namespace
 
 extern "C" {
@@ -116,6 +125,8 @@ typedef struct {
   double eps;
   int32_t mirror_bf16;
   int32_t threads;
+  int32_t zoh;      // 0: Bbar = delta B; 1: Bbar = expm1(delta A) / A * B
+  int32_t reserved;
 } orc_dims;
 
 double orc_round_bf16(double v) { return round_bf16(v); }
@@ -161,7 +172,8 @@ void orc_rmsnorm(int64_t rows, int64_t width, int64_t in_stride, const double* i
 // delta, u: [L,d]; A: [d,N] (already -exp(A_log)); Bm, Cm: [L,N]; h0, hT: [d,N].
 void orc_scan_range(int64_t L, int64_t d, int64_t N, const double* delta, const double* A,
                     const double* Bm, const double* Cm, const double* u, const double* D,
-                    const double* h0, double* y, double* hT, int64_t c0, int64_t c1) {
+                    const double* h0, double* y, double* hT, int64_t c0, int64_t c1,
+                    int32_t zoh) {
   std::vector<double> h(N);
   for (int64_t c = c0; c < c1; ++c) {
     for (int64_t n = 0; n < N; ++n) h[n] = h0 ? h0[c * N + n] : 0.0;
@@ -169,7 +181,8 @@ void orc_scan_range(int64_t L, int64_t d, int64_t N, const double* delta, const 
       double dl = delta[t * d + c], uv = u[t * d + c];
       double acc = 0.0;
       for (int64_t n = 0; n < N; ++n) {
-        h[n] = std::exp(dl * A[c * N + n]) * h[n] + dl * Bm[t * N + n] * uv;
+        const double a = A[c * N + n];
+        h[n] = std::exp(dl * a) * h[n] + bbar(dl, a, zoh) * Bm[t * N + n] * uv;
         acc += Cm[t * N + n] * h[n];
       }
       y[t * d + c] = acc + D[c] * uv;
@@ -181,8 +194,8 @@ void orc_scan_range(int64_t L, int64_t d, int64_t N, const double* delta, const 
 
 void orc_scan(int64_t L, int64_t d, int64_t N, const double* delta, const double* A,
               const double* Bm, const double* Cm, const double* u, const double* D,
-              const double* h0, double* y, double* hT) {
-  orc_scan_range(L, d, N, delta, A, Bm, Cm, u, D, h0, y, hT, 0, d);
+              const double* h0, double* y, double* hT, int32_t zoh) {
+  orc_scan_range(L, d, N, delta, A, Bm, Cm, u, D, h0, y, hT, 0, d, zoh);
 }
 
 // Front end of one sequence for tokens [t0, t1): u, p rows (from the
@@ -290,7 +303,7 @@ void orc_mixer_fwd_channels(const orc_dims* m, const void* x_data, int32_t x_kin
         double dl = delta[t * nch + i], uv = usel[t * nch + i];
         double acc = 0.0;
         for (int64_t n = 0; n < N; ++n) {
-          h[n] = std::exp(dl * A[n]) * h[n] + dl * Bn[t * N + n] * uv;
+          h[n] = std::exp(dl * A[n]) * h[n] + bbar(dl, A[n], m->zoh) * Bn[t * N + n] * uv;
           acc += Cn[t * N + n] * h[n];
         }
         double ys = acc + D[c] * uv;

@@ -334,3 +334,88 @@ def test_sampled_channels_match_full():
     np.testing.assert_array_equal(ys, y[:, :, ch])
     np.testing.assert_array_equal(fss, fs[:, ch])
     np.testing.assert_array_equal(fcs, fc[:, ch])
+
+
+# -------------------------------------------------- zero-order-hold variant
+def _rk4_step(a, b, h, dt, steps):
+    """Integrate dh/dt = a h + b from h over dt by classic Runge-Kutta (RK4)."""
+    s = dt / steps
+    for _ in range(steps):
+        k1 = a * h + b
+        k2 = a * (h + 0.5 * s * k1) + b
+        k3 = a * (h + 0.5 * s * k2) + b
+        k4 = a * (h + s * k3) + b
+        h = h + s / 6.0 * (k1 + 2 * k2 + 2 * k3 + k4)
+    return h
+
+
+def test_zoh_step_is_the_exact_ode_step():
+    """Zero-order hold is the exact solution of dh/dt = A h + B u over one step with
+    u held: the oracle's state after each token matches a fine RK4 integration of
+    that ODE (token by token, from the previous state)."""
+    L, d, N = 6, 2, 16
+    delta, A, Bm, Cm, u, D, h0 = rand_scan_inputs(L, d, N, seed=41)
+    h = h0.copy()
+    for t in range(L):
+        _, hT = oracle.scan(delta[: t + 1], A, Bm[: t + 1], Cm[: t + 1], u[: t + 1], D, h0,
+                            zoh=True)
+        b = Bm[t][None, :] * u[t][:, None]
+        h = _rk4_step(A, b, h, delta[t][:, None], 2000)
+        np.testing.assert_allclose(hT, h, rtol=1e-9, atol=1e-11)
+
+
+def test_zoh_constant_inputs_closed_form():
+    """Constant inputs: h_t = a^t h0 + (1 - a^t) h*, with a = exp(delta A) and the
+    fixed point h* = -B u / A of dh/dt = A h + B u (no delta in it)."""
+    L, d, N = 25, 3, 16
+    r = np.random.default_rng(5)
+    dl = np.array([0.02, 0.4, 3.0])
+    A = -np.exp(r.uniform(-1, 2, size=(d, N)))
+    B1, C1 = r.normal(size=N), r.normal(size=N)
+    u1 = np.array([0.5, -2.0, 1.1])
+    D = r.normal(size=d)
+    h0 = r.normal(size=(d, N))
+    y, hT = oracle.scan(np.tile(dl, (L, 1)), A, np.tile(B1, (L, 1)), np.tile(C1, (L, 1)),
+                        np.tile(u1, (L, 1)), D, h0, zoh=True)
+    a = np.exp(dl[:, None] * A)
+    hstar = -B1[None, :] * u1[:, None] / A
+    for t in (1, 3, L):
+        ht = a ** t * h0 + (1 - a ** t) * hstar
+        np.testing.assert_allclose(y[t - 1], ht @ C1 + D * u1, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(hT, a ** L * h0 + (1 - a ** L) * hstar, rtol=1e-12, atol=1e-13)
+
+
+def test_zoh_L1_and_small_delta_limit():
+    """L = 1 from zero: h = (exp(delta A) - 1) / A B u; as delta -> 0 the hold
+    and Euler updates agree to first order (difference O(delta^2))."""
+    delta, A, Bm, Cm, u, D, _ = rand_scan_inputs(1, 4, 16, seed=7)
+    _, hT = oracle.scan(delta, A, Bm, Cm, u, D, None, zoh=True)
+    h = np.expm1(delta[0][:, None] * A) / A * Bm[0][None, :] * u[0][:, None]
+    np.testing.assert_allclose(hT, h, rtol=1e-14, atol=0)
+    for scale in (1e-3, 1e-5):
+        dl = delta * scale
+        _, hz = oracle.scan(dl, A, Bm, Cm, u, D, None, zoh=True)
+        _, he = oracle.scan(dl, A, Bm, Cm, u, D, None)
+        rel = np.abs(hz - he).max() / np.abs(he).max()
+        assert rel <= 5 * scale * np.abs(A).max() * delta.max(), (scale, rel)
+        assert rel > 0
+
+
+def test_zoh_mixer_wiring():
+    """Whole mixer: the flag reaches the scan (results differ at the workloads' delta),
+    and with delta driven to ~1e-6 by dt_bias the hold and Euler mixers agree to
+    O(delta^2) relative, as they must; a wrong hold factor (a dropped 1/A, a sign)
+    fails this at O(1)."""
+    w = synth.Workload("zoh", 1, 9, 32, 8, "f32", seed=13, extra=True)
+    W = synth.make_weights(w)
+    A_ = synth.make_activations(w)
+    args = (A_["x"], A_["z"])
+    kw = dict(init_conv_state=A_["init_conv_state"])
+    ye, _, _ = oracle.mixer_fwd(oracle.dims_of(w), *args, W, **kw)
+    yz, _, _ = oracle.mixer_fwd(oracle.dims_of(w, zoh=True), *args, W, **kw)
+    assert np.abs(yz - ye).max() > 1e-4
+    Wsmall = dict(W, dt_bias=np.full_like(W["dt_bias"], -14.0))   # delta ~ 1e-6 (x O(1))
+    ye, fse, _ = oracle.mixer_fwd(oracle.dims_of(w), *args, Wsmall, **kw)
+    yz, fsz, _ = oracle.mixer_fwd(oracle.dims_of(w, zoh=True), *args, Wsmall, **kw)
+    rel = np.abs(fsz - fse).max() / np.abs(fse).max()
+    assert 0 < rel < 1e-4, rel
