@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--zoh", action="store_true",
+                    help="discretise B by zero-order hold instead of delta B")
     ap.add_argument("--varlen", action="store_true",
                     help="also time jm_mixer_fwd_varlen on a packed batch of mixed lengths")
     ap.add_argument("--seqlen", type=int, default=0,
@@ -163,12 +165,12 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ decode
-def decode_bench(dev, stream, steps: int = 64, warmup: int = 5):
+def decode_bench(dev, stream, steps: int = 64, warmup: int = 5, zoh: bool = False):
     """64 consecutive jm_mixer_step calls on the decode workload (B=256 sequences at
     Jamba shapes, states updated in place); returns a dict for the JSON line."""
     import torch
     from mamba_selective_scan_jamba_b200 import devio, jmix, synth
-    w = synth.WORKLOADS["jamba_decode_b256"]
+    w = synth.WORKLOADS["jamba_decode_b256"].with_(zoh=zoh)
     W = synth.make_weights(w)
     S = synth.make_decode_state(w)
     Wd = devio.weights_to_device(W, dev)
@@ -368,6 +370,8 @@ def main():
     base = synth.WORKLOADS[args.workload]
     if args.seqlen:
         base = base.with_(seqlen=args.seqlen, name=f"{base.name}_L{args.seqlen}")
+    if args.zoh:
+        base = base.with_(zoh=True, name=f"{base.name}_zoh")
     if args.impl == "reference":
         reference_arm(args, base, rank, world)
         return
@@ -528,7 +532,7 @@ def main():
     if args.varlen:
         line["varlen"] = varlen_bench(dev, stream)
     if not args.no_decode:
-        dec = decode_bench(dev, stream)
+        dec = decode_bench(dev, stream, zoh=args.zoh)
         dec["hbm_frac"] = dec["achieved_GBps"] / P["hbm"]
         line["decode"] = dec
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -77,7 +77,15 @@ typedef struct {
   int64_t dt_rank;  /* R, 8..256, multiple of 8 */
   float eps;        /* RMSNorm epsilon, inside the square root, >= 0 */
   jm_dtype io;      /* dtype of x, z, y, conv states and the io-dtype weights */
+  int32_t discretization; /* JM_DISC_EULER (0): Bbar = delta B;
+                             JM_DISC_ZOH (1): Bbar = (exp(delta A) - 1) / A B */
+  int32_t reserved;       /* must be 0 */
 } jm_dims;
+
+/* How B is discretised.  Abar = exp(delta A) in both; Euler takes delta B (the
+ * Jamba guide's "Bbar ~ delta B"), zero-order hold the exact one-step solution
+ * of dh/dt = A h + B u for u held over the step. */
+enum { JM_DISC_EULER = 0, JM_DISC_ZOH = 1 };
 
 /* Bytes of device workspace jm_mixer_fwd needs for these dims (0 if the dims
  * are invalid; see jm_last_error).  The workspace must be 256-byte aligned.

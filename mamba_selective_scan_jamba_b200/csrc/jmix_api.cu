@@ -62,6 +62,14 @@ jm_status check_dims(const jm_dims* dm, bool step) {
     set_error("io dtype must be JM_F32 or JM_BF16");
     return JM_ERR_INVALID_ARG;
   }
+  if (dm->discretization != JM_DISC_EULER && dm->discretization != JM_DISC_ZOH) {
+    set_error("discretization must be JM_DISC_EULER or JM_DISC_ZOH");
+    return JM_ERR_INVALID_ARG;
+  }
+  if (dm->reserved != 0) {
+    set_error("jm_dims.reserved must be 0");
+    return JM_ERR_INVALID_ARG;
+  }
   if (!(dm->eps >= 0.0f) || dm->eps != dm->eps || dm->eps > 1e30f) {
     set_error("eps must be finite and >= 0");
     return JM_ERR_INVALID_ARG;
@@ -99,6 +107,7 @@ void fill_problem(Problem& p, const jm_dims* dm) {
   p.T = dm->batch * dm->seqlen;
   p.eps = dm->eps;
   p.io = dm->io;
+  p.zoh = dm->discretization == JM_DISC_ZOH;
 }
 
 size_t ws_bytes_for(const Problem& p) {

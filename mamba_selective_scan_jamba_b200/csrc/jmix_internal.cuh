@@ -48,6 +48,7 @@ struct Problem {
   size_t ws_bytes;
   cudaStream_t stream;
   bool decode;             // jm_mixer_step
+  bool zoh;                // B discretised by zero-order hold (else delta B)
   const int* cu;           // packed batch: [B + 1] token offsets (device); L == T then
   int launches;            // kernels launched so far by this call
   void* const* events;     // optional per-kernel timing events (jm_set_kernel_events)

@@ -746,13 +746,30 @@ __device__ __forceinline__ void wait_flag(const int* flag, ErrFlags* err, unsign
 
 // The compute warps' share of one unit: chunks [kb, kb + nch) of the pair's
 // sequence.  kOut: produce y (else only the state and the sum of delta).
-template <bool kOut>
+// Zero-order hold: the factor expm1(delta A) / A that multiplies B u, for a pair
+// of states.  x = delta A log2(e) (as passed to ex2), da = 2^x = exp(delta A),
+// inv_a = 1 / A.  For |delta A| >= 1/32: (da - 1) / A (relative error below
+// 1e-5 with ex2.approx); below: delta (1 + y/2 + y^2/6), y = delta A (the
+// series of expm1(y)/y, truncation below 1.3e-6).
+__device__ __forceinline__ float2 zoh_factor(float2 x, float2 da, float2 inv_a, float2 dl2) {
+  const float2 y = __fmul2_rn(x, make_float2(0.69314718f, 0.69314718f));
+  const float2 poly = __ffma2_rn(y, __ffma2_rn(y, make_float2(1.0f / 6.0f, 1.0f / 6.0f),
+                                              make_float2(0.5f, 0.5f)),
+                                 make_float2(1.0f, 1.0f));
+  const float2 small = __fmul2_rn(dl2, poly);
+  const float2 big = __fmul2_rn(__fadd2_rn(da, make_float2(-1.0f, -1.0f)), inv_a);
+  return make_float2(fabsf(y.x) < 0.03125f ? small.x : big.x,
+                     fabsf(y.y) < 0.03125f ? small.y : big.y);
+}
+
+template <bool kOut, bool kZoh>
 __device__ __forceinline__ void scan_chunks(const ScanArgs& a, const uint8_t* stage0,
                                             uint64_t* full, uint64_t* mma_done, uint64_t* empty,
                                             uint32_t tmem, int warp, int lane, int kg0, int kb,
                                             int nch, int64_t Lb, bool cok, bf16* yrow,
                                             float2 (&h)[kN / 2],
-                                            const float2 (&A2)[kN / 2], float (&xw)[kConv - 1],
+                                            const float2 (&A2)[kN / 2],
+                                            const float2 (&invA)[kN / 2], float (&xw)[kConv - 1],
                                             const float (&cw)[kConv], float cb, float bias,
                                             float Dc, float& ssum) {
   const int cl = warp * 32 + lane;
@@ -793,7 +810,7 @@ __device__ __forceinline__ void scan_chunks(const ScanArgs& a, const uint8_t* st
           xw[2] = xt;
         }
         dl[i] = softplus_fast(__uint_as_float(r[i]) + bias);
-        du[i] = dl[i] * uv;
+        du[i] = kZoh ? uv : dl[i] * uv;  // zero-order hold: u (the factor is per state)
         if constexpr (kOut) {
           dsk[i] = Dc * uv;
           gz[i] = silu_gate(bf(zs[(g0t + i) * kSC + cl]));
@@ -821,7 +838,11 @@ __device__ __forceinline__ void scan_chunks(const ScanArgs& a, const uint8_t* st
             float2 da;
             da.x = ex2_approx(x.x);
             da.y = ex2_approx(x.y);
-            h[q] = __ffma2_rn(da, h[q], __fmul2_rn(du2, Bp));
+            if constexpr (kZoh)
+              h[q] = __ffma2_rn(da, h[q],
+                                __fmul2_rn(__fmul2_rn(zoh_factor(x, da, invA[q], dl2), du2), Bp));
+            else
+              h[q] = __ffma2_rn(da, h[q], __fmul2_rn(du2, Bp));
             if constexpr (kOut) {
               // four independent partial sums of C.h (short dependency chains)
               const float2 Cp = half ? make_float2(Cq.z, Cq.w) : make_float2(Cq.x, Cq.y);
@@ -883,6 +904,7 @@ __global__ void __launch_bounds__(1024) k_order_by_length(const int* __restrict_
 // Every unit that waits waits only for units that come before it in claim
 // order, and a claimed unit is running or queued behind one with a smaller
 // index on its CTA, so every wait ends; each is still bounded (2 s).
+template <bool kZoh>  // B by zero-order hold (else delta B)
 __global__ void __launch_bounds__(kScanThreads, kScanCtasPerSm)
     k_scan_fused(const __grid_constant__ CUtensorMap tm_wdt,
                  const __grid_constant__ CUtensorMap tm_dtn,
@@ -1081,12 +1103,15 @@ __global__ void __launch_bounds__(kScanThreads, kScanCtasPerSm)
         }
         named_bar_sync(kAllBar, 32 * kProdWarp);
       }
-      float2 A2[kN / 2], h[kN / 2];
+      float2 A2[kN / 2], h[kN / 2], invA[kN / 2];
 #pragma unroll
       for (int q = 0; q < kN / 2; ++q) {
         const int n = 2 * q;
         A2[q].x = cok ? -expf(a.A_log[c * kN + n]) * kLog2e : 0.0f;
         A2[q].y = cok ? -expf(a.A_log[c * kN + n + 1]) * kLog2e : 0.0f;
+        // 1 / A = -exp(-A_log) (zero-order hold only)
+        invA[q] = cok ? make_float2(-expf(-a.A_log[c * kN + n]), -expf(-a.A_log[c * kN + n + 1]))
+                      : make_float2(0.0f, 0.0f);
         h[q] = make_float2(0.0f, 0.0f);
         if (part == 0 && cok && a.h0) {
           h[q].x = a.h0[(b * a.d + c) * kN + n];
@@ -1128,11 +1153,12 @@ __global__ void __launch_bounds__(kScanThreads, kScanCtasPerSm)
       }
       float ssum = 0.0f;
       if (out)
-        scan_chunks<true>(a, stage0, full, mma_done, empty, tmem, warp, lane, kg0, kb, nch, Lb,
-                          cok, a.y + g0 * a.d + c, h, A2, xw, cw, cb, bias, Dc, ssum);
+        scan_chunks<true, kZoh>(a, stage0, full, mma_done, empty, tmem, warp, lane, kg0, kb, nch,
+                                Lb, cok, a.y + g0 * a.d + c, h, A2, invA, xw, cw, cb, bias, Dc,
+                                ssum);
       else
-        scan_chunks<false>(a, stage0, full, mma_done, empty, tmem, warp, lane, kg0, kb, nch, Lb,
-                           cok, nullptr, h, A2, xw, cw, cb, bias, Dc, ssum);
+        scan_chunks<false, kZoh>(a, stage0, full, mma_done, empty, tmem, warp, lane, kg0, kb, nch,
+                                 Lb, cok, nullptr, h, A2, invA, xw, cw, cb, bias, Dc, ssum);
       if (part + 1 < P && (!out || !a.two_pass)) {
         // hand the end state (and, two-pass, the sum of delta) to later parts
         float* ch = a.carry_h + hslot * kSC * kN + cl * kN;
@@ -1213,6 +1239,7 @@ struct DecArgs {
 #endif
 constexpr int kDecAhead = JMIX_DEC_AHEAD;  // sequences whose inputs are in flight per thread
 
+template <bool kZoh>  // B by zero-order hold (else delta B)
 __global__ void __launch_bounds__(kDecThreads, JMIX_DEC_OCC)
     k_decode_scan(const __grid_constant__ CUtensorMap tm_wdt,
                   const __grid_constant__ CUtensorMap tm_dtn,
@@ -1355,7 +1382,16 @@ __global__ void __launch_bounds__(kDecThreads, JMIX_DEC_OCC)
             const float2 Cp = half ? make_float2(Cq.z, Cq.w) : make_float2(Cq.x, Cq.y);
             const float2 xq = __fmul2_rn(dl2, A2[q]);
             const float2 da = make_float2(ex2_approx(xq.x), ex2_approx(xq.y));
-            h[q] = __ffma2_rn(da, h[q], __fmul2_rn(du2, Bp));
+            if constexpr (kZoh) {
+              // 1 / A = 1 / (A2 ln 2); this path is not the hot one, so it divides
+              const float2 inv_a = make_float2(kLog2e / A2[q].x, kLog2e / A2[q].y);
+              h[q] = __ffma2_rn(da, h[q],
+                                __fmul2_rn(__fmul2_rn(zoh_factor(xq, da, inv_a, dl2),
+                                                      make_float2(uv, uv)),
+                                           Bp));
+            } else {
+              h[q] = __ffma2_rn(da, h[q], __fmul2_rn(du2, Bp));
+            }
             acc[q4] = half ? __ffma2_rn(Cp, h[q], acc[q4]) : __fmul2_rn(Cp, h[q]);
           }
         }
@@ -1587,8 +1623,9 @@ cudaError_t run_fast_fwd(Problem& p) {
     da.ssm_state = p.final_state;
     da.y = (bf16*)p.y;
     da.err = err;
-    cudaFuncSetAttribute(k_decode_scan, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
-    k_decode_scan<<<dim3((unsigned)((p.d + kSC - 1) / kSC), (unsigned)((p.B + kDB - 1) / kDB)),
+    auto dec_kern = p.zoh ? k_decode_scan<true> : k_decode_scan<false>;
+    cudaFuncSetAttribute(dec_kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
+    dec_kern<<<dim3((unsigned)((p.d + kSC - 1) / kSC), (unsigned)((p.B + kDB - 1) / kDB)),
                     kDecThreads, kDecSmem, s>>>(twdt, tdtn, tbc, da);
     launched(p, "k_decode_scan");
   } else {
@@ -1638,10 +1675,11 @@ cudaError_t run_fast_fwd(Problem& p) {
     const int pairs = sa.n_tiles * (int)p.B;
     const int units = pairs * sa.n_parts + (sa.two_pass ? pairs * (sa.n_parts - 1) : 0);
     const int slots = kScanCtasPerSm * num_sms();
-    cudaFuncSetAttribute(k_scan_fused, cudaFuncAttributeMaxDynamicSharedMemorySize, kScanSmem);
-    cudaFuncSetAttribute(k_scan_fused, cudaFuncAttributePreferredSharedMemoryCarveout,
+    auto scan_kern = p.zoh ? k_scan_fused<true> : k_scan_fused<false>;
+    cudaFuncSetAttribute(scan_kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kScanSmem);
+    cudaFuncSetAttribute(scan_kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                          cudaSharedmemCarveoutMaxShared);
-    k_scan_fused<<<(unsigned)(units < slots ? units : slots), kScanThreads, kScanSmem, s>>>(
+    scan_kern<<<(unsigned)(units < slots ? units : slots), kScanThreads, kScanSmem, s>>>(
         twdt, tdtn, tbc, tx, tz, sa);
     launched(p, "k_scan_fused");
   }

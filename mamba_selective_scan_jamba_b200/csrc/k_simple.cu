@@ -136,7 +136,7 @@ __global__ void k_scan_simple(const float* __restrict__ delta, const float* __re
                               const float* __restrict__ Bn, const float* __restrict__ Cn,
                               const T* __restrict__ z, const float* __restrict__ A_log,
                               const float* __restrict__ Dv, const float* h0, float* hT, T* y,
-                              int64_t L, int64_t d) {
+                              int64_t L, int64_t d, bool zoh) {
   const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int64_t b = blockIdx.y;
   if (c >= d) return;
@@ -154,7 +154,9 @@ __global__ void k_scan_simple(const float* __restrict__ delta, const float* __re
     float acc = 0.f;
 #pragma unroll
     for (int n = 0; n < kN; ++n) {
-      h[n] = fmaf(expf(dl * A[n]), h[n], du * __ldg(Bn + g * kN + n));
+      // Euler: delta B u; zero-order hold: expm1(delta A) / A * B u
+      const float bu = zoh ? expm1f(dl * A[n]) / A[n] * uv : du;
+      h[n] = fmaf(expf(dl * A[n]), h[n], bu * __ldg(Bn + g * kN + n));
       acc = fmaf(__ldg(Cn + g * kN + n), h[n], acc);
     }
     const float ys = fmaf(Dc, uv, acc);
@@ -235,7 +237,7 @@ cudaError_t run_simple_t(Problem& p) {
   launched(p, "k_gemm_nt(dt_proj)");
   k_scan_simple<T><<<dim3((unsigned)((p.d + 127) / 128), (unsigned)p.B), 128, 0, s>>>(
       w.delta, w.u, w.Bn, w.Cn, (const T*)p.z, p.A_log, p.D, p.init_ssm, p.final_state, (T*)p.y,
-      p.L, p.d);
+      p.L, p.d, p.zoh);
   launched(p, "k_scan_simple");
   if (p.final_conv) {
     const int64_t bd = p.B * p.d;

@@ -56,4 +56,4 @@ def dims_of(w, batch=None, seqlen=None) -> jmix.jm_dims:
     """jm_dims for a synth.Workload."""
     return jmix.dims(w.batch if batch is None else batch, w.seqlen if seqlen is None else seqlen,
                      w.d_inner, w.dt_rank, jmix.JM_BF16 if w.io == "bf16" else jmix.JM_F32,
-                     w.eps, w.d_state, w.d_conv)
+                     w.eps, w.d_state, w.d_conv, getattr(w, "zoh", False))

@@ -33,7 +33,8 @@ class jm_dims(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64),
                 ("d_inner", ctypes.c_int64), ("d_state", ctypes.c_int64),
                 ("d_conv", ctypes.c_int64), ("dt_rank", ctypes.c_int64),
-                ("eps", ctypes.c_float), ("io", ctypes.c_int)]
+                ("eps", ctypes.c_float), ("io", ctypes.c_int),
+                ("discretization", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 class JmixError(RuntimeError):
@@ -90,9 +91,13 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     return lib
 
 
+JM_DISC_EULER, JM_DISC_ZOH = 0, 1
+
+
 def dims(batch: int, seqlen: int, d_inner: int, dt_rank: int, io: int = JM_BF16,
-         eps: float = 1e-6, d_state: int = 16, d_conv: int = 4) -> jm_dims:
-    return jm_dims(batch, seqlen, d_inner, d_state, d_conv, dt_rank, eps, io)
+         eps: float = 1e-6, d_state: int = 16, d_conv: int = 4, zoh: bool = False) -> jm_dims:
+    return jm_dims(batch, seqlen, d_inner, d_state, d_conv, dt_rank, eps, io,
+                   JM_DISC_ZOH if zoh else JM_DISC_EULER, 0)
 
 
 def _ptr(t) -> Optional[int]:

@@ -174,6 +174,7 @@ class Workload:
     eps: float = 1e-6
     dt_min: float = 1e-3
     dt_max: float = 1e-1
+    zoh: bool = False            # B discretised by zero-order hold (else delta B)
     steps: int = 0               # decode workloads: number of consecutive steps
     extra: bool = False          # random conv_b / norm weights / D / A_log / initial states
 

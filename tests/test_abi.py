@@ -185,3 +185,19 @@ def test_varlen_host_checks(lib):
     st = jmix.jm_mixer_fwd_varlen(d, FAKE, FAKE, FAKE, W, FAKE + (1 << 30), FAKE, FAKE, 256,
                                   stream=0, check=False)
     assert st == jmix.JM_ERR_WORKSPACE
+
+
+def test_discretization_field(lib):
+    FAKE = 1 << 40
+    W = {k: FAKE for k in jmix.WEIGHT_NAMES}
+    d = jmix.dims(2, 10, 256, 16)
+    d.discretization = 2
+    st = jmix.jm_mixer_fwd(d, FAKE, FAKE + (1 << 30), W, FAKE + (2 << 30), FAKE, FAKE, 1 << 30,
+                           stream=0, check=False)
+    assert st == jmix.JM_ERR_INVALID_ARG and "discretization" in jmix.jm_last_error()
+    d = jmix.dims(2, 10, 256, 16, zoh=True)
+    d.reserved = 1
+    assert jmix.jm_mixer_fwd_workspace_size(d) == 0
+    d.reserved = 0
+    assert jmix.jm_mixer_fwd_workspace_size(d) == jmix.jm_mixer_fwd_workspace_size(
+        jmix.dims(2, 10, 256, 16))

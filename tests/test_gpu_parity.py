@@ -239,3 +239,19 @@ def test_full_jamba_b1_l262144():
 @pytest.mark.slow
 def test_full_decode_b256_64_steps():
     run_decode(synth.WORKLOADS["jamba_decode_b256"], 64, channels=FULL_CH)
+
+
+# ------------------------------------------------ zero-order hold of B (variant)
+@pytest.mark.parametrize("B,L,d,R,io", [
+    (2, 300, 384, 64, "bf16"),    # 3 tiles, ragged
+    (1, 2200, 256, 16, "bf16"),   # two-pass schedule (the fold is the same map)
+    (2, 77, 128, 8, "f32"),       # float32 path
+])
+def test_zoh_forward(B, L, d, R, io):
+    check_fwd(small(B, L, d, R, io=io).with_(zoh=True))
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_zoh_decode(io):
+    w = synth.Workload("dec_zoh", 5, 1, 256, 16, io, seed=19, extra=True, steps=6, zoh=True)
+    run_decode(w, 6)
