@@ -94,6 +94,23 @@ def kernel_units(name, w, tokens):
     return "hbm", tokens * (R + 2 * N) * 4 * 2, "GB/s"
 
 
+def nvtx_push(msg: str) -> None:
+    """NVTX range for profilers (a no-op where torch has no NVTX support)."""
+    try:
+        import torch
+        torch.cuda.nvtx.range_push(msg)
+    except Exception:  # noqa: BLE001 - tracing must never stop a measurement
+        pass
+
+
+def nvtx_pop() -> None:
+    try:
+        import torch
+        torch.cuda.nvtx.range_pop()
+    except Exception:  # noqa: BLE001
+        pass
+
+
 def measured_traffic(kernel: str, tokens: int):
     """DRAM bytes of one launch of `kernel` over `tokens` tokens, from the committed
     ncu summary of that kernel (bytes per token x tokens), if the kernel source is
@@ -435,6 +452,7 @@ def main():
     torch.cuda.synchronize(dev)
     t_wall0 = time.time()
     launches = 0
+    nvtx_push(f"jmix timed region: {K} x jm_mixer_fwd ({w.name})")
     with torch.cuda.stream(stream):
         start.record(stream)
         for i in range(K):
@@ -442,6 +460,7 @@ def main():
             step()
             launches += jmix.jm_last_launch_count()
         end.record(stream)
+    nvtx_pop()
     jmix.jm_set_kernel_events(None)
     stream.synchronize()
     torch.cuda.synchronize(dev)

@@ -175,6 +175,15 @@ jm_status jm_mixer_fwd_host(const jm_dims* dims, const void* x_host, const void*
  * error, JM_OK otherwise. */
 jm_status jm_poll_error(void* workspace, jm_stream_t stream);
 
+/* Failure-detection self-test: launches one thread that waits, through the
+ * same bounded wait the pipelines use, on a barrier that nothing completes.
+ * The wait gives up after its limit (2 s), records site 99 in workspace's
+ * error header and returns, so a following jm_poll_error(workspace) returns
+ * JM_ERR_TIMEOUT and the CUDA context stays usable.  workspace: device, at
+ * least 256 bytes (its first 256 bytes are overwritten).  Asynchronous on
+ * `stream`.  JM_ERR_WORKSPACE if workspace is NULL or too small. */
+jm_status jm_selftest_timeout(void* workspace, size_t ws_bytes, jm_stream_t stream);
+
 /* Message of the last failed call on this thread ("" if none). */
 const char* jm_last_error(void);
 

@@ -26,7 +26,7 @@ EXPORTED = ("jm_mixer_fwd_workspace_size", "jm_mixer_step_workspace_size", "jm_m
             "jm_mixer_step", "jm_mixer_fwd_host", "jm_poll_error", "jm_last_error",
             "jm_last_launch_count", "jm_last_kernel_name", "jm_set_kernel_events",
             "jm_mixer_step_noalloc", "jm_mixer_fwd_schedule",
-            "jm_mixer_fwd_varlen_workspace_size", "jm_mixer_fwd_varlen")
+            "jm_mixer_fwd_varlen_workspace_size", "jm_mixer_fwd_varlen", "jm_selftest_timeout")
 
 
 class jm_dims(ctypes.Structure):
@@ -73,6 +73,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.jm_mixer_fwd_varlen.restype = ctypes.c_int
     lib.jm_mixer_fwd_varlen.argtypes = ([ctypes.POINTER(jm_dims)] + [_vp] * 19
                                         + [ctypes.c_size_t, _vp])
+    lib.jm_selftest_timeout.restype = ctypes.c_int
+    lib.jm_selftest_timeout.argtypes = [_vp, ctypes.c_size_t, _vp]
     lib.jm_mixer_fwd_schedule.restype = ctypes.c_int
     lib.jm_mixer_fwd_schedule.argtypes = [ctypes.POINTER(jm_dims), ctypes.POINTER(ctypes.c_int),
                                           ctypes.POINTER(ctypes.c_int)]
@@ -147,6 +149,14 @@ def jm_mixer_fwd(d: jm_dims, x, z, w: Mapping, y, final_state, workspace, ws_byt
     st = load().jm_mixer_fwd(ctypes.byref(d), _ptr(x), _ptr(z), *_weights(w), _ptr(y),
                              _ptr(final_state), _ptr(init_conv_state), _ptr(init_ssm_state),
                              _ptr(final_conv_state), _ptr(workspace), ws_bytes, _stream(stream))
+    if check:
+        _check(st)
+    return st
+
+
+def jm_selftest_timeout(workspace, ws_bytes: int, stream=None, check: bool = True) -> int:
+    """Launch the bounded wait that is never satisfied (see include/jmix.h)."""
+    st = load().jm_selftest_timeout(_ptr(workspace), ws_bytes, _stream(stream))
     if check:
         _check(st)
     return st

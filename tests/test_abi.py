@@ -201,3 +201,8 @@ def test_discretization_field(lib):
     d.reserved = 0
     assert jmix.jm_mixer_fwd_workspace_size(d) == jmix.jm_mixer_fwd_workspace_size(
         jmix.dims(2, 10, 256, 16))
+
+
+def test_selftest_timeout_host_checks(lib):
+    assert jmix.jm_selftest_timeout(None, 0, stream=0, check=False) == jmix.JM_ERR_WORKSPACE
+    assert jmix.jm_selftest_timeout(1 << 40, 128, stream=0, check=False) == jmix.JM_ERR_WORKSPACE
