@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--zoh", action="store_true",
                     help="discretise B by zero-order hold instead of delta B")
+    ap.add_argument("--layer", action="store_true",
+                    help="also time the full layer (in_proj -> mixer -> out_proj, d_model 4096)")
     ap.add_argument("--varlen", action="store_true",
                     help="also time jm_mixer_fwd_varlen on a packed batch of mixed lengths")
     ap.add_argument("--seqlen", type=int, default=0,
@@ -303,6 +305,46 @@ def varlen_bench(dev, stream, steps: int = 20, warmup: int = 3):
             "kernels_ms": per, "launches_per_step": nk}
 
 
+def layer_bench(dev, stream, w, d_model: int = 4096, steps: int = 10, warmup: int = 3):
+    """jm_layer_fwd (in_proj on cuBLASLt -> mixer core -> out_proj on cuBLASLt) on
+    the workload at Jamba's d_model; returns a dict for the JSON line."""
+    import torch
+    from mamba_selective_scan_jamba_b200 import devio, jmix, synth
+    W = synth.make_weights(w)
+    LW = synth.make_layer(w, d_model)
+    Wd = devio.weights_to_device(W, dev)
+    hid = devio.to_device(LW["hidden"], dev)
+    wi, wo = devio.to_device(LW["in_proj_w"], dev), devio.to_device(LW["out_proj_w"], dev)
+    out = torch.empty_like(hid)
+    fs = torch.empty((w.batch, w.d_inner, w.d_state), dtype=torch.float32, device=dev)
+    d = devio.dims_of(w)
+    n = jmix.jm_layer_fwd_workspace_size(d, d_model)
+    ws = devio.workspace(n, dev)
+
+    def step():
+        jmix.jm_layer_fwd(d, d_model, hid, wi, Wd, wo, out, fs, ws, n, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            step()
+    stream.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        for _ in range(steps):
+            step()
+        b.record(stream)
+    stream.synchronize()
+    assert jmix.jm_poll_error(ws, stream) == jmix.JM_OK, jmix.jm_last_error()
+    ms = a.elapsed_time(b) / steps
+    T = w.batch * w.seqlen
+    gemm_flop = 2.0 * T * d_model * 3 * w.d_inner        # in_proj (2 d_inner) + out_proj
+    return {"workload": f"{w.name} + in_proj/out_proj (d_model {d_model})", "tokens": T,
+            "steps": steps, "ms_per_step": ms, "tokens_per_s": T / (ms / 1e3),
+            "projection_tflop_per_step": gemm_flop / 1e12,
+            "projections": "cuBLASLt bf16 GEMMs (fp32 accumulation), not fused"}
+
+
 # ------------------------------------------------------------- cpu baseline
 def oracle_sample(w, tokens: float):
     """(sequences, tokens per sequence) of a sample of about `tokens` tokens taken
@@ -550,6 +592,8 @@ def main():
 
     if args.varlen:
         line["varlen"] = varlen_bench(dev, stream)
+    if args.layer:
+        line["layer"] = layer_bench(dev, stream, w)
     if not args.no_decode:
         dec = decode_bench(dev, stream, zoh=args.zoh)
         dec["hbm_frac"] = dec["achieved_GBps"] / P["hbm"]

@@ -175,6 +175,27 @@ jm_status jm_mixer_fwd_host(const jm_dims* dims, const void* x_host, const void*
  * error, JM_OK otherwise. */
 jm_status jm_poll_error(void* workspace, jm_stream_t stream);
 
+/* The full Mamba layer around the mixer core (bf16 io only):
+ *   [x | z] = hidden . in_proj_w^T,  y = mixer core (as jm_mixer_fwd),
+ *   out = y . out_proj_w^T.
+ * hidden: [B, L, d_model]; in_proj_w: [2 d_inner, d_model] (rows 0 .. d_inner-1
+ * give x, the rest z); out_proj_w: [d_model, d_inner]; out: [B, L, d_model]; all
+ * bf16 device memory, 16-byte aligned; d_model a positive multiple of 8.  The
+ * mixer arguments, states, errors and ownership are those of jm_mixer_fwd.  The
+ * projections run on cuBLASLt (fp32 accumulation, bf16 x, z, y and out) with the
+ * caller's workspace as scratch: jm_layer_fwd_workspace_size(dims, d_model)
+ * bytes, 256-byte aligned; its first 256 bytes are the error header that
+ * jm_poll_error reads.  JM_ERR_UNSUPPORTED for float32 io. */
+size_t jm_layer_fwd_workspace_size(const jm_dims* dims, int64_t d_model);
+jm_status jm_layer_fwd(const jm_dims* dims, int64_t d_model, const void* hidden,
+                       const void* in_proj_w, const void* conv_w, const void* conv_b,
+                       const void* xproj_w, const void* dt_norm_w, const void* b_norm_w,
+                       const void* c_norm_w, const void* dtproj_w, const float* dt_bias,
+                       const float* A_log, const float* D, const void* out_proj_w, void* out,
+                       float* final_state, const void* init_conv_state,
+                       const float* init_ssm_state, void* final_conv_state, void* workspace,
+                       size_t ws_bytes, jm_stream_t stream);
+
 /* Failure-detection self-test: launches one thread that waits, through the
  * same bounded wait the pipelines use, on a barrier that nothing completes.
  * The wait gives up after its limit (2 s), records site 99 in workspace's

@@ -144,11 +144,15 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// 2, 4 or 8 consecutive 32-bit columns of this thread's TMEM lane (warp-wide).
+// 2, 4, 8 or 16 consecutive 32-bit columns of this thread's TMEM lane (warp-wide).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]);
+
 template <int NC>
 __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[NC]) {
-  static_assert(NC == 2 || NC == 4 || NC == 8, "unsupported column count");
-  if constexpr (NC == 2) {
+  static_assert(NC == 2 || NC == 4 || NC == 8 || NC == 16, "unsupported column count");
+  if constexpr (NC == 16) {
+    tmem_ld16(taddr, r);
+  } else if constexpr (NC == 2) {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];"
                  : "=r"(r[0]), "=r"(r[1])
                  : "r"(taddr)

@@ -26,7 +26,8 @@ EXPORTED = ("jm_mixer_fwd_workspace_size", "jm_mixer_step_workspace_size", "jm_m
             "jm_mixer_step", "jm_mixer_fwd_host", "jm_poll_error", "jm_last_error",
             "jm_last_launch_count", "jm_last_kernel_name", "jm_set_kernel_events",
             "jm_mixer_step_noalloc", "jm_mixer_fwd_schedule",
-            "jm_mixer_fwd_varlen_workspace_size", "jm_mixer_fwd_varlen", "jm_selftest_timeout")
+            "jm_mixer_fwd_varlen_workspace_size", "jm_mixer_fwd_varlen", "jm_selftest_timeout",
+            "jm_layer_fwd_workspace_size", "jm_layer_fwd")
 
 
 class jm_dims(ctypes.Structure):
@@ -73,6 +74,11 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.jm_mixer_fwd_varlen.restype = ctypes.c_int
     lib.jm_mixer_fwd_varlen.argtypes = ([ctypes.POINTER(jm_dims)] + [_vp] * 19
                                         + [ctypes.c_size_t, _vp])
+    lib.jm_layer_fwd_workspace_size.restype = ctypes.c_size_t
+    lib.jm_layer_fwd_workspace_size.argtypes = [ctypes.POINTER(jm_dims), ctypes.c_int64]
+    lib.jm_layer_fwd.restype = ctypes.c_int
+    lib.jm_layer_fwd.argtypes = ([ctypes.POINTER(jm_dims), ctypes.c_int64] + [_vp] * 19
+                                 + [ctypes.c_size_t, _vp])
     lib.jm_selftest_timeout.restype = ctypes.c_int
     lib.jm_selftest_timeout.argtypes = [_vp, ctypes.c_size_t, _vp]
     lib.jm_mixer_fwd_schedule.restype = ctypes.c_int
@@ -148,6 +154,24 @@ def jm_mixer_fwd(d: jm_dims, x, z, w: Mapping, y, final_state, workspace, ws_byt
                  stream=None, check: bool = True) -> int:
     st = load().jm_mixer_fwd(ctypes.byref(d), _ptr(x), _ptr(z), *_weights(w), _ptr(y),
                              _ptr(final_state), _ptr(init_conv_state), _ptr(init_ssm_state),
+                             _ptr(final_conv_state), _ptr(workspace), ws_bytes, _stream(stream))
+    if check:
+        _check(st)
+    return st
+
+
+def jm_layer_fwd_workspace_size(d: jm_dims, d_model: int) -> int:
+    return load().jm_layer_fwd_workspace_size(ctypes.byref(d), d_model)
+
+
+def jm_layer_fwd(d: jm_dims, d_model: int, hidden, in_proj_w, w: Mapping, out_proj_w, out,
+                 final_state, workspace, ws_bytes: int, init_conv_state=None,
+                 init_ssm_state=None, final_conv_state=None, stream=None,
+                 check: bool = True) -> int:
+    """The full Mamba layer: in_proj -> mixer core -> out_proj (see include/jmix.h)."""
+    st = load().jm_layer_fwd(ctypes.byref(d), d_model, _ptr(hidden), _ptr(in_proj_w),
+                             *_weights(w), _ptr(out_proj_w), _ptr(out), _ptr(final_state),
+                             _ptr(init_conv_state), _ptr(init_ssm_state),
                              _ptr(final_conv_state), _ptr(workspace), ws_bytes, _stream(stream))
     if check:
         _check(st)

@@ -54,6 +54,7 @@ _CHUNK = 1 << 22
 TID = dict(x=1, z=2, conv_w=3, conv_b=4, xproj_w=5, dtproj_w=6, dt=7,
            dt_norm_w=8, b_norm_w=9, c_norm_w=10, D=11, A_log=12,
            init_conv_state=13, init_ssm_state=14, conv_state=15, ssm_state=16)
+TID_LAYER = dict(hidden=20, in_proj_w=21, out_proj_w=22)  # the full layer's extra tensors
 TID_XT = 1000   # + step index
 TID_ZT = 2000   # + step index
 
@@ -266,6 +267,21 @@ def make_activations(w: Workload, batch_lo: int = 0, batch_hi: Optional[int] = N
                                        math.sqrt(0.1), start=batch_lo * d * N,
                                        out="f32").reshape(nb, d, N)
     return out
+
+
+def make_layer(w: Workload, d_model: int) -> Dict[str, np.ndarray]:
+    """The full Mamba layer's extra tensors around the mixer core: hidden [B, L,
+    d_model] ~ N(0, 1); in_proj_w [2 d_inner, d_model] ~ N(0, 1/d_model) (rows
+    0..d_inner-1 give x, the rest z); out_proj_w [d_model, d_inner] ~ N(0, 1/d_inner).
+    I/O dtype."""
+    d, io = w.d_inner, _io(w)
+    s = lambda name: stream_seed(w.seed, TID_LAYER[name])
+    return {"hidden": normal(s("hidden"), w.batch * w.seqlen * d_model, out=io)
+                      .reshape(w.batch, w.seqlen, d_model),
+            "in_proj_w": normal(s("in_proj_w"), 2 * d * d_model, 1.0 / math.sqrt(d_model),
+                                out=io).reshape(2 * d, d_model),
+            "out_proj_w": normal(s("out_proj_w"), d_model * d, 1.0 / math.sqrt(d),
+                                 out=io).reshape(d_model, d)}
 
 
 def make_decode_state(w: Workload) -> Dict[str, np.ndarray]:

@@ -198,6 +198,32 @@ def mixer_fwd(m: OrcDims, x, z, weights: Dict[str, np.ndarray], init_conv_state=
     return y, fs, fc
 
 
+def _round_bf16_via_f32(a: np.ndarray) -> np.ndarray:
+    """fp64 -> fp32 (nearest even) -> bf16 (nearest even), as a float32-accumulating
+    GEMM that stores bf16 rounds its outputs (finite values)."""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000).astype(np.uint32)
+    return r.view(np.float32).astype(np.float64)
+
+
+def layer_fwd(m: OrcDims, hidden, in_proj_w, out_proj_w, weights: Dict[str, np.ndarray],
+              init_conv_state=None, init_ssm_state=None, round_xz_bf16: bool = False):
+    """The full Mamba layer around the mixer core (TransformerLens "Jamba" adapter
+    page, "Architecture overview": in_proj / conv1d / x_proj / dt_proj / out_proj):
+    [x | z] = hidden . in_proj_w^T, the mixer core, out = y . out_proj_w^T.  fp64
+    matrix products.  round_xz_bf16 rounds x and z to bf16 (nearest even) before the
+    mixer, as a bf16 layer stores them.  Returns (out [B,L,d_model], final_state)."""
+    h = _f64(hidden)
+    wi, wo = _f64(in_proj_w), _f64(out_proj_w)
+    d = m.d_inner
+    xz = h @ wi.T
+    x, z = np.ascontiguousarray(xz[..., :d]), np.ascontiguousarray(xz[..., d:])
+    if round_xz_bf16:
+        x, z = _round_bf16_via_f32(x), _round_bf16_via_f32(z)
+    y, fs, _ = mixer_fwd(m, x, z, weights, init_conv_state, init_ssm_state)
+    return y @ wo.T, fs
+
+
 def mixer_step(m: OrcDims, x_t, z_t, conv_state, ssm_state, weights: Dict[str, np.ndarray]):
     """One decode step for every sequence.  Returns (y_t [B,d], conv_state', ssm_state')
     in float64; the inputs are not modified."""

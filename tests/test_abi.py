@@ -206,3 +206,22 @@ def test_discretization_field(lib):
 def test_selftest_timeout_host_checks(lib):
     assert jmix.jm_selftest_timeout(None, 0, stream=0, check=False) == jmix.JM_ERR_WORKSPACE
     assert jmix.jm_selftest_timeout(1 << 40, 128, stream=0, check=False) == jmix.JM_ERR_WORKSPACE
+
+
+def test_layer_host_checks(lib):
+    FAKE = 1 << 40
+    W = {k: FAKE for k in jmix.WEIGHT_NAMES}
+    d = jmix.dims(2, 10, 256, 16)
+    n = jmix.jm_layer_fwd_workspace_size(d, 128)
+    assert n > jmix.jm_mixer_fwd_workspace_size(d)
+    assert jmix.jm_layer_fwd_workspace_size(d, 100) == 0          # d_model % 8
+    assert jmix.jm_layer_fwd_workspace_size(jmix.dims(2, 10, 256, 16, io=jmix.JM_F32), 128) == 0
+    st = jmix.jm_layer_fwd(d, 100, FAKE, FAKE, W, FAKE, FAKE, FAKE, FAKE, n, stream=0,
+                           check=False)
+    assert st == jmix.JM_ERR_INVALID_ARG and "d_model" in jmix.jm_last_error()
+    st = jmix.jm_layer_fwd(d, 128, FAKE, FAKE, W, FAKE, FAKE, FAKE, FAKE, n - 256, stream=0,
+                           check=False)
+    assert st == jmix.JM_ERR_WORKSPACE
+    st = jmix.jm_layer_fwd(d, 128, None, FAKE, W, FAKE, FAKE, FAKE, FAKE, n, stream=0,
+                           check=False)
+    assert st == jmix.JM_ERR_INVALID_ARG and "hidden" in jmix.jm_last_error()

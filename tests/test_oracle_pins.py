@@ -419,3 +419,18 @@ def test_zoh_mixer_wiring():
     yz, fsz, _ = oracle.mixer_fwd(oracle.dims_of(w, zoh=True), *args, Wsmall, **kw)
     rel = np.abs(fsz - fse).max() / np.abs(fse).max()
     assert 0 < rel < 1e-4, rel
+
+
+def test_layer_oracle_with_identity_projections_is_the_mixer():
+    """The layer's projections: with d_model = d_inner, in_proj_w = [I; s I] and
+    out_proj_w = I, the layer is the mixer on (hidden, s * hidden).  Fixes the x / z
+    split order (x first) and the transposes of both products."""
+    w = synth.Workload("lay", 2, 11, 24, 8, "f32", seed=17, extra=True)
+    W = synth.make_weights(w)
+    hidden = np.random.default_rng(3).normal(size=(2, 11, 24))
+    s = -0.75
+    eye = np.eye(24)
+    out, fs = oracle.layer_fwd(oracle.dims_of(w), hidden, np.vstack([eye, s * eye]), eye, W)
+    y, fsm, _ = oracle.mixer_fwd(oracle.dims_of(w), hidden, s * hidden, W)
+    np.testing.assert_allclose(out, y, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(fs, fsm, rtol=1e-13, atol=1e-14)
