@@ -162,6 +162,26 @@ def scan(delta, A, Bm, Cm, u, D, h0=None, zoh=False):
     return y, hT
 
 
+def scan_bwd(delta, A_log, Bm, Cm, u, D, h0, gy):
+    """Backward of the scan core of one sequence (Euler B), fp64.  delta, u, gy
+    [L,d]; A_log [d,N]; Bm, Cm [L,N]; D [d]; h0 [d,N] or None.  Returns a dict of
+    gradients: delta, u [L,d]; B, C [L,N]; A_log [d,N] (through A = -exp(A_log));
+    D [d]; h0 [d,N]."""
+    delta, A_log, Bm, Cm, u, D, h0, gy = map(_f64, (delta, A_log, Bm, Cm, u, D, h0, gy))
+    L, d = delta.shape
+    N = A_log.shape[1]
+    A = -np.exp(A_log)
+    out = {k: np.zeros(s) for k, s in (("delta", (L, d)), ("u", (L, d)), ("B", (L, N)),
+                                        ("C", (L, N)), ("A", (d, N)), ("D", (d,)),
+                                        ("h0", (d, N)))}
+    _L().orc_scan_bwd(ctypes.c_int64(L), ctypes.c_int64(d), ctypes.c_int64(N), _p(delta), _p(A),
+                      _p(Bm), _p(Cm), _p(u), _p(D), _p(h0), _p(gy), _p(out["delta"]),
+                      _p(out["u"]), _p(out["B"]), _p(out["C"]), _p(out["A"]), _p(out["D"]),
+                      _p(out["h0"]))
+    out["A_log"] = out.pop("A") * A          # dA/dA_log = A
+    return out
+
+
 def mixer_fwd(m: OrcDims, x, z, weights: Dict[str, np.ndarray], init_conv_state=None,
               init_ssm_state=None, channels: Optional[Sequence[int]] = None):
     """Mixer forward.  Returns (y [B,L,d or nch], final_state [B,d or nch,N],

@@ -198,6 +198,48 @@ void orc_scan(int64_t L, int64_t d, int64_t N, const double* delta, const double
   orc_scan_range(L, d, N, delta, A, Bm, Cm, u, D, h0, y, hT, 0, d, zoh);
 }
 
+// Backward of the scan core of one sequence (Euler B): given gy = dLoss/dy_s
+// [L,d], the gradients of delta, u [L,d], B, C [L,N] (summed over channels),
+// A [d,N] and D [d] (accumulated: += into gA, gD) and h0 [d,N].  Reverse mode
+// of h_t = a_t h_{t-1} + delta_t B_t u_t, a_t = exp(delta_t A), y_t = C_t.h_t +
+// D u_t, with every h_t of the forward kept (fp64, small inputs).
+void orc_scan_bwd(int64_t L, int64_t d, int64_t N, const double* delta, const double* A,
+                  const double* Bm, const double* Cm, const double* u, const double* D,
+                  const double* h0, const double* gy, double* gdelta, double* gu, double* gB,
+                  double* gC, double* gA, double* gD, double* gh0) {
+  for (int64_t i = 0; i < L * N; ++i) gB[i] = gC[i] = 0.0;
+  std::vector<double> hs((size_t)(L + 1) * N), g(N);
+  for (int64_t c = 0; c < d; ++c) {
+    for (int64_t n = 0; n < N; ++n) hs[n] = h0 ? h0[c * N + n] : 0.0;
+    for (int64_t t = 0; t < L; ++t) {
+      const double dl = delta[t * d + c], uv = u[t * d + c];
+      for (int64_t n = 0; n < N; ++n)
+        hs[(t + 1) * N + n] = std::exp(dl * A[c * N + n]) * hs[t * N + n] + dl * Bm[t * N + n] * uv;
+    }
+    for (int64_t n = 0; n < N; ++n) g[n] = 0.0;
+    for (int64_t t = L - 1; t >= 0; --t) {
+      const double dl = delta[t * d + c], uv = u[t * d + c], gyt = gy[t * d + c];
+      double gdl = 0.0, gut = D[c] * gyt;
+      gD[c] += gyt * uv;
+      for (int64_t n = 0; n < N; ++n) {
+        const double a = std::exp(dl * A[c * N + n]);
+        const double hp = hs[t * N + n], ht = hs[(t + 1) * N + n];
+        g[n] += Cm[t * N + n] * gyt;             // y_t = C_t . h_t + ...
+        gC[t * N + n] += gyt * ht;
+        gut += g[n] * dl * Bm[t * N + n];
+        gB[t * N + n] += g[n] * dl * uv;
+        gdl += g[n] * (A[c * N + n] * a * hp + Bm[t * N + n] * uv);
+        gA[c * N + n] += g[n] * dl * a * hp;
+        g[n] *= a;                               // to h_{t-1}
+      }
+      gdelta[t * d + c] = gdl;
+      gu[t * d + c] = gut;
+    }
+    if (gh0)
+      for (int64_t n = 0; n < N; ++n) gh0[c * N + n] = g[n];
+  }
+}
+
 // Front end of one sequence for tokens [t0, t1): u, p rows (from the
 // mirror-rounded u in mirror mode), normalised dt_n (mirror-rounded) / Bn / Cn.
 static void front_end_rows(const orc_dims* m, Stored x, const double* conv_w,

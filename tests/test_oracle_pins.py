@@ -434,3 +434,58 @@ def test_layer_oracle_with_identity_projections_is_the_mixer():
     y, fsm, _ = oracle.mixer_fwd(oracle.dims_of(w), hidden, s * hidden, W)
     np.testing.assert_allclose(out, y, rtol=1e-13, atol=1e-14)
     np.testing.assert_allclose(fs, fsm, rtol=1e-13, atol=1e-14)
+
+
+# ------------------------------------------------------ backward of the scan
+def _loss(delta, A_log, Bm, Cm, u, D, h0, gy):
+    """A scalar of the scan core's outputs: <gy, y_s> (its gradient is what
+    scan_bwd returns)."""
+    y, _ = oracle.scan(delta, -np.exp(A_log), Bm, Cm, u, D, h0)
+    return float((gy * y).sum())
+
+
+def _bwd_inputs(seed, L=7, d=3, N=16):
+    r = np.random.default_rng(seed)
+    return dict(delta=np.exp(r.uniform(np.log(0.01), np.log(0.8), size=(L, d))),
+                A_log=r.uniform(np.log(0.3), np.log(4.0), size=(d, N)),
+                Bm=r.normal(size=(L, N)), Cm=r.normal(size=(L, N)), u=r.normal(size=(L, d)),
+                D=r.normal(size=d), h0=r.normal(size=(d, N)), gy=r.normal(size=(L, d)))
+
+
+def test_scan_bwd_matches_central_finite_differences():
+    """Every gradient against (f(x + e) - f(x - e)) / 2e of the forward oracle,
+    entry by entry, for a few entries of each input (fp64, e = 1e-6)."""
+    p = _bwd_inputs(31)
+    g = oracle.scan_bwd(p["delta"], p["A_log"], p["Bm"], p["Cm"], p["u"], p["D"], p["h0"],
+                        p["gy"])
+    names = {"delta": "delta", "A_log": "A_log", "Bm": "B", "Cm": "C", "u": "u", "D": "D",
+             "h0": "h0"}
+    r = np.random.default_rng(0)
+    for key, gname in names.items():
+        for _ in range(4):
+            idx = tuple(int(r.integers(0, s)) for s in p[key].shape)
+            e = 1e-6
+            plus = {k: v.copy() for k, v in p.items()}
+            minus = {k: v.copy() for k, v in p.items()}
+            plus[key][idx] += e
+            minus[key][idx] -= e
+            fd = (_loss(**plus) - _loss(**minus)) / (2 * e)
+            assert abs(g[gname][idx] - fd) <= 1e-6 * max(1.0, abs(fd)), (key, idx, g[gname][idx], fd)
+
+
+def test_scan_bwd_adjoint_dot_product():
+    """Linearity in gy: the gradient of <gy1 + 2 gy2, y> is g(gy1) + 2 g(gy2), and
+    <g_u(gy), du> equals the directional derivative of <gy, y> along du (the
+    forward is linear in h0 and in u for fixed delta, B, C)."""
+    p = _bwd_inputs(32)
+    r = np.random.default_rng(1)
+    gy2 = r.normal(size=p["gy"].shape)
+    g1 = oracle.scan_bwd(**{k: v for k, v in p.items()})
+    g2 = oracle.scan_bwd(**dict(p, gy=gy2))
+    g12 = oracle.scan_bwd(**dict(p, gy=p["gy"] + 2 * gy2))
+    for k in g1:
+        np.testing.assert_allclose(g12[k], g1[k] + 2 * g2[k], rtol=1e-11, atol=1e-12)
+    du, dh0 = r.normal(size=p["u"].shape), r.normal(size=p["h0"].shape)
+    base = _loss(**p)
+    lin = _loss(**dict(p, u=p["u"] + du, h0=p["h0"] + dh0)) - base
+    np.testing.assert_allclose((g1["u"] * du).sum() + (g1["h0"] * dh0).sum(), lin, rtol=1e-11)
