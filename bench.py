@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--zoh", action="store_true",
                     help="discretise B by zero-order hold instead of delta B")
+    ap.add_argument("--bwd", action="store_true",
+                    help="also time the scan-core backward (B=1, L=4096, d_inner 8192)")
     ap.add_argument("--layer", action="store_true",
                     help="also time the full layer (in_proj -> mixer -> out_proj, d_model 4096)")
     ap.add_argument("--varlen", action="store_true",
@@ -345,6 +347,49 @@ def layer_bench(dev, stream, w, d_model: int = 4096, steps: int = 10, warmup: in
             "projections": "cuBLASLt bf16 GEMMs (fp32 accumulation), not fused"}
 
 
+def bwd_bench(dev, stream, B: int = 1, L: int = 4096, d: int = 8192, steps: int = 5,
+              warmup: int = 2):
+    """jm_scan_bwd (backward of the scan core, float32) at Jamba's d_inner; returns a
+    dict for the JSON line."""
+    import torch
+    from mamba_selective_scan_jamba_b200 import devio, jmix
+    g = torch.Generator(device=dev).manual_seed(7)
+    rnd = lambda *s: torch.randn(*s, device=dev, generator=g)
+    delta = torch.exp(torch.empty(B, L, d, device=dev).uniform_(math.log(1e-3), math.log(0.1),
+                                                                generator=g))
+    u, gy = rnd(B, L, d), rnd(B, L, d)
+    Bm, Cm = rnd(B, L, 16), rnd(B, L, 16)
+    A_log = torch.log(torch.arange(1, 17, device=dev, dtype=torch.float32)).repeat(d, 1)
+    D = torch.ones(d, device=dev)
+    outs = [torch.empty(B, L, d, device=dev), torch.empty(B, L, d, device=dev),
+            torch.empty(B, L, 16, device=dev), torch.empty(B, L, 16, device=dev),
+            torch.empty(d, 16, device=dev), torch.empty(d, device=dev),
+            torch.empty(B, d, 16, device=dev)]
+    dm = jmix.dims(B, L, d, 8)
+    n = jmix.jm_scan_bwd_workspace_size(dm)
+    ws = devio.workspace(n, dev)
+
+    def step():
+        jmix.jm_scan_bwd(dm, delta, u, Bm, Cm, A_log, D, None, gy, *outs, ws, n, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            step()
+    stream.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        for _ in range(steps):
+            step()
+        b.record(stream)
+    stream.synchronize()
+    assert jmix.jm_poll_error(ws, stream) == jmix.JM_OK, jmix.jm_last_error()
+    ms = a.elapsed_time(b) / steps
+    return {"workload": f"scan-core backward, B={B}, L={L}, d_inner={d}, float32",
+            "tokens": B * L, "ms_per_step": ms, "tokens_per_s": B * L / (ms / 1e3),
+            "data": "synthetic (torch generator, seed 7)"}
+
+
 # ------------------------------------------------------------- cpu baseline
 def oracle_sample(w, tokens: float):
     """(sequences, tokens per sequence) of a sample of about `tokens` tokens taken
@@ -594,6 +639,8 @@ def main():
         line["varlen"] = varlen_bench(dev, stream)
     if args.layer:
         line["layer"] = layer_bench(dev, stream, w)
+    if args.bwd:
+        line["bwd"] = bwd_bench(dev, stream)
     if not args.no_decode:
         dec = decode_bench(dev, stream, zoh=args.zoh)
         dec["hbm_frac"] = dec["achieved_GBps"] / P["hbm"]

@@ -196,6 +196,26 @@ jm_status jm_layer_fwd(const jm_dims* dims, int64_t d_model, const void* hidden,
                        const float* init_ssm_state, void* final_conv_state, void* workspace,
                        size_t ws_bytes, jm_stream_t stream);
 
+/* Backward of the selective-scan core (training), float32 throughout, Euler B.
+ * Forward: h_t = exp(delta_t A) h_{t-1} + delta_t B_t u_t, A = -exp(A_log),
+ * y_t = C_t . h_t + D u_t (per sequence and channel; the Jamba guide, "Inside
+ * the Mamba State-Space Layers").  Given gy = dLoss/dy it writes every input
+ * gradient: g_delta, g_u [B, L, d]; g_B, g_C [B, L, 16] (summed over channels);
+ * g_A_log [d, 16], g_D [d] (summed over sequences and tokens); g_h0 [B, d, 16]
+ * (may be NULL).  Inputs: delta, u, gy [B, L, d]; B, C [B, L, 16]; A_log [d, 16];
+ * D [d]; h0 [B, d, 16] or NULL (zero).  dims: batch, seqlen, d_inner, d_state
+ * (must be 16) and discretization (JM_DISC_EULER only) are read.  Results are
+ * deterministic (fixed summation order).  Workspace:
+ * jm_scan_bwd_workspace_size(dims) bytes, 256-byte aligned (state checkpoints
+ * every 4 tokens and per-warp partial sums; its first 256 bytes are the error
+ * header jm_poll_error reads).  Asynchronous on `stream`. */
+size_t jm_scan_bwd_workspace_size(const jm_dims* dims);
+jm_status jm_scan_bwd(const jm_dims* dims, const float* delta, const float* u, const float* B,
+                      const float* C, const float* A_log, const float* D, const float* h0,
+                      const float* gy, float* g_delta, float* g_u, float* g_B, float* g_C,
+                      float* g_A_log, float* g_D, float* g_h0, void* workspace, size_t ws_bytes,
+                      jm_stream_t stream);
+
 /* Failure-detection self-test: launches one thread that waits, through the
  * same bounded wait the pipelines use, on a barrier that nothing completes.
  * The wait gives up after its limit (2 s), records site 99 in workspace's

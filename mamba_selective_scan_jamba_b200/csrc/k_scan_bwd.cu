@@ -1,0 +1,318 @@
+// Backward of the selective-scan core (training), float32.
+//
+// Forward (Euler B; Jamba guide, "Inside the Mamba State-Space Layers"):
+//   h_t = a_t h_{t-1} + delta_t B_t u_t,  a_t = exp(delta_t A),  A = -exp(A_log),
+//   y_t = C_t . h_t + D u_t.
+// Given gy = dLoss/dy, reverse mode gives, with g the gradient flowing into h_t:
+//   g   += C_t gy_t;  gC_t += gy_t h_t;  gu_t = D gy_t + sum_n g_n delta_t B_t,n;
+//   gB_t += g delta_t u_t;  gdelta_t = sum_n g_n (A_n a_t,n h_{t-1},n + B_t,n u_t);
+//   gA_n += g_n delta_t a_t,n h_{t-1},n;  gD += gy_t u_t;  g <- a_t g  (to h_{t-1});
+// and g_h0 = g after the first token, gA_log = gA * A.
+//
+// k_scan_bwd: CTA = (128-channel tile, sequence), thread = channel, 16 states in
+// registers.  Pass 1 runs the recurrence forward and stores the state at the
+// start of every kCk-token chunk.  Pass 2 walks the chunks backwards: it
+// recomputes the chunk's states into shared memory ([token][state][channel],
+// conflict-free) and runs the reverse recurrence token by token.  gB and gC are
+// sums over channels: each warp reduces its 32 channels' 32 values (16 gB, 16 gC)
+// by a reduce-scatter of shuffles (lane i ends with index i) into a per-warp
+// partial row; k_scan_bwd_reduce adds the partials in a fixed order, and gA_log,
+// gD over the sequences, so the results are reproducible.
+#include "jmix_internal.cuh"
+
+#define JM_API extern "C" __attribute__((visibility("default")))
+
+namespace jmix {
+namespace {
+
+constexpr int kBwdThreads = 128;
+constexpr int kCk = 4;  // tokens per checkpoint chunk (32 KB of states in shared memory)
+
+struct BwdArgs {
+  int64_t B, L, d;
+  const float* delta;
+  const float* u;
+  const float* Bm;
+  const float* Cm;
+  const float* A_log;
+  const float* D;
+  const float* h0;
+  const float* gy;
+  float* gdelta;
+  float* gu;
+  float* gh0;
+  float* ckpt;      // [B, nck, d, 16]
+  float* part_bc;   // [n_tiles * 4, B * L, 32]: per-warp sums of gB (0..15), gC (16..31)
+  float* part_a;    // [B, d, 16]
+  float* part_d;    // [B, d]
+};
+
+// Sums v over the 32 lanes of the warp, index by index: afterwards lane i holds
+// in v[0] the sum of every lane's v[i].
+__device__ __forceinline__ void warp_reduce_scatter32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    const bool up = lane & off;
+#pragma unroll
+    for (int i = 0; i < off; ++i) {
+      const float send = up ? v[i] : v[i + off];
+      const float keep = up ? v[i + off] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kBwdThreads) k_scan_bwd(const BwdArgs a) {
+  __shared__ float hs[kCk][kN][kBwdThreads];  // states after each token of the chunk
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t b = blockIdx.y;
+  const int64_t c = (int64_t)blockIdx.x * kBwdThreads + threadIdx.x;
+  const bool cok = c < a.d;
+  const int64_t L = a.L, d = a.d;
+  const int64_t nck = (L + kCk - 1) / kCk;
+  float A[kN];
+#pragma unroll
+  for (int n = 0; n < kN; ++n) A[n] = cok ? -expf(a.A_log[c * kN + n]) : 0.0f;
+  const float Dc = cok ? a.D[c] : 0.0f;
+  auto at = [&](const float* p, int64_t t) { return cok ? p[(b * L + t) * d + c] : 0.0f; };
+  // pass 1: forward, checkpoint at every chunk start
+  float h[kN];
+#pragma unroll
+  for (int n = 0; n < kN; ++n) h[n] = (cok && a.h0) ? a.h0[(b * d + c) * kN + n] : 0.0f;
+  for (int64_t t = 0; t < L; ++t) {
+    if (t % kCk == 0 && cok) {
+      float* ck = a.ckpt + ((b * nck + t / kCk) * d + c) * kN;
+#pragma unroll
+      for (int n = 0; n < kN; ++n) ck[n] = h[n];
+    }
+    const float dl = at(a.delta, t), du = dl * at(a.u, t);
+    const float* Bt = a.Bm + (b * L + t) * kN;
+#pragma unroll
+    for (int n = 0; n < kN; ++n) h[n] = fmaf(expf(dl * A[n]), h[n], du * Bt[n]);
+  }
+  // pass 2: reverse
+  float g[kN], gA[kN], gD = 0.0f;
+#pragma unroll
+  for (int n = 0; n < kN; ++n) g[n] = gA[n] = 0.0f;
+  const int64_t tile_warp = (int64_t)blockIdx.x * 4 + warp;
+  for (int64_t j = nck - 1; j >= 0; --j) {
+    const int64_t t0 = j * kCk;
+    const int nt = (int)((L - t0) < kCk ? (L - t0) : kCk);
+    float hstart[kN];
+    if (cok) {
+      const float* ck = a.ckpt + ((b * nck + j) * d + c) * kN;
+#pragma unroll
+      for (int n = 0; n < kN; ++n) hstart[n] = ck[n];
+    } else {
+#pragma unroll
+      for (int n = 0; n < kN; ++n) hstart[n] = 0.0f;
+    }
+#pragma unroll
+    for (int n = 0; n < kN; ++n) h[n] = hstart[n];
+    for (int i = 0; i < nt; ++i) {
+      const int64_t t = t0 + i;
+      const float dl = at(a.delta, t), du = dl * at(a.u, t);
+      const float* Bt = a.Bm + (b * L + t) * kN;
+#pragma unroll
+      for (int n = 0; n < kN; ++n) {
+        h[n] = fmaf(expf(dl * A[n]), h[n], du * Bt[n]);
+        hs[i][n][threadIdx.x] = h[n];
+      }
+    }
+    for (int i = nt - 1; i >= 0; --i) {
+      const int64_t t = t0 + i;
+      const float dl = at(a.delta, t), uv = at(a.u, t), gyt = at(a.gy, t);
+      const float* Bt = a.Bm + (b * L + t) * kN;
+      const float* Ct = a.Cm + (b * L + t) * kN;
+      float v[32];  // this channel's share of gB_t (0..15) and gC_t (16..31)
+      float gdl = 0.0f, gut = Dc * gyt;
+      gD = fmaf(gyt, uv, gD);
+#pragma unroll
+      for (int n = 0; n < kN; ++n) {
+        const float an = expf(dl * A[n]);
+        const float hp = i > 0 ? hs[i - 1][n][threadIdx.x] : hstart[n];
+        const float ht = hs[i][n][threadIdx.x];
+        g[n] = fmaf(Ct[n], gyt, g[n]);
+        v[16 + n] = gyt * ht;
+        gut = fmaf(g[n], dl * Bt[n], gut);
+        v[n] = g[n] * dl * uv;
+        gdl = fmaf(g[n], fmaf(A[n] * an, hp, Bt[n] * uv), gdl);
+        gA[n] = fmaf(g[n] * dl * an, hp, gA[n]);
+        g[n] *= an;
+      }
+      if (!cok) {
+#pragma unroll
+        for (int q = 0; q < 32; ++q) v[q] = 0.0f;
+      }
+      if (cok) {
+        a.gdelta[(b * L + t) * d + c] = gdl;
+        a.gu[(b * L + t) * d + c] = gut;
+      }
+      warp_reduce_scatter32(v, lane);
+      a.part_bc[(tile_warp * (a.B * L) + b * L + t) * 32 + lane] = v[0];
+    }
+  }
+  if (cok) {
+#pragma unroll
+    for (int n = 0; n < kN; ++n) a.part_a[(b * d + c) * kN + n] = gA[n];
+    a.part_d[b * d + c] = gD;
+    if (a.gh0)
+#pragma unroll
+      for (int n = 0; n < kN; ++n) a.gh0[(b * d + c) * kN + n] = g[n];
+  }
+}
+
+// gB, gC: sum over the per-warp partial rows, in order; gA_log, gD: sum over
+// the sequences, in order, then gA_log = gA * A.
+__global__ void k_scan_bwd_reduce(const float* __restrict__ part_bc, int64_t n_rows, int64_t TB,
+                                  const float* __restrict__ part_a, const float* __restrict__ part_d,
+                                  const float* __restrict__ A_log, int64_t B, int64_t d,
+                                  float* __restrict__ gB, float* __restrict__ gC,
+                                  float* __restrict__ gA_log, float* __restrict__ gD) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t n_bc = TB * 32;
+  if (i < n_bc) {
+    float s = 0.0f;
+    for (int64_t r = 0; r < n_rows; ++r) s += part_bc[r * n_bc + i];
+    const int64_t tok = i >> 5;
+    const int k = (int)(i & 31);
+    if (k < kN)
+      gB[tok * kN + k] = s;
+    else
+      gC[tok * kN + k - kN] = s;
+    return;
+  }
+  const int64_t j = i - n_bc;
+  if (j < d * kN) {
+    float s = 0.0f;
+    for (int64_t bb = 0; bb < B; ++bb) s += part_a[bb * d * kN + j];
+    gA_log[j] = s * -expf(A_log[j]);  // dA/dA_log = A
+    return;
+  }
+  const int64_t c = j - d * kN;
+  if (c < d) {
+    float s = 0.0f;
+    for (int64_t bb = 0; bb < B; ++bb) s += part_d[bb * d + c];
+    gD[c] = s;
+  }
+}
+
+struct BwdWs {
+  float* ckpt;
+  float* part_bc;
+  float* part_a;
+  float* part_d;
+  size_t bytes;
+  int64_t n_rows;
+};
+
+BwdWs bwd_layout(int64_t B, int64_t L, int64_t d, char* base) {
+  BwdWs w{};
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    size_t o = off;
+    off = align256(off + n);
+    return base ? reinterpret_cast<float*>(base + o) : nullptr;
+  };
+  const int64_t nck = (L + kCk - 1) / kCk;
+  const int64_t n_tiles = (d + kBwdThreads - 1) / kBwdThreads;
+  w.n_rows = n_tiles * 4;
+  take(sizeof(ErrFlags));  // the error header jm_poll_error reads (cleared each call)
+  w.ckpt = take((size_t)B * nck * d * kN * 4);
+  w.part_bc = take((size_t)w.n_rows * B * L * 32 * 4);
+  w.part_a = take((size_t)B * d * kN * 4);
+  w.part_d = take((size_t)B * d * 4);
+  w.bytes = off;
+  return w;
+}
+
+jm_status check_bwd_dims(const jm_dims* dm) {
+  if (!dm) {
+    set_error("dims is NULL");
+    return JM_ERR_INVALID_ARG;
+  }
+  if (dm->batch < 0 || dm->seqlen < 0 || dm->d_inner <= 0) {
+    set_error("sizes must be positive (batch, seqlen >= 0)");
+    return JM_ERR_INVALID_ARG;
+  }
+  if (dm->d_state != kN) {
+    set_error("only d_state == 16 is built (got %lld)", (long long)dm->d_state);
+    return JM_ERR_UNSUPPORTED;
+  }
+  if (dm->discretization != JM_DISC_EULER) {
+    set_error("the scan backward is built for Euler B (delta B) only");
+    return JM_ERR_UNSUPPORTED;
+  }
+  if ((double)dm->batch * (double)dm->seqlen * (double)dm->d_inner > 1.0e13) {
+    set_error("problem too large");
+    return JM_ERR_INVALID_ARG;
+  }
+  return JM_OK;
+}
+
+}  // namespace
+}  // namespace jmix
+
+using namespace jmix;
+
+JM_API size_t jm_scan_bwd_workspace_size(const jm_dims* dims) {
+  if (check_bwd_dims(dims) != JM_OK) return 0;
+  return bwd_layout(dims->batch, dims->seqlen, dims->d_inner, nullptr).bytes;
+}
+
+JM_API jm_status jm_scan_bwd(const jm_dims* dims, const float* delta, const float* u,
+                             const float* Bm, const float* Cm, const float* A_log, const float* D,
+                             const float* h0, const float* gy, float* g_delta, float* g_u,
+                             float* g_B, float* g_C, float* g_A_log, float* g_D, float* g_h0,
+                             void* workspace, size_t ws_bytes, jm_stream_t stream) {
+  jm_status st = check_bwd_dims(dims);
+  if (st != JM_OK) return st;
+  const int64_t B = dims->batch, L = dims->seqlen, d = dims->d_inner;
+  const bool any = B > 0 && L > 0;
+  const void* const req[] = {A_log, D, g_A_log, g_D};
+  const char* const rn[] = {"A_log", "D", "g_A_log", "g_D"};
+  for (int i = 0; i < 4; ++i)
+    if (!req[i]) {
+      set_error("%s is NULL", rn[i]);
+      return JM_ERR_INVALID_ARG;
+    }
+  if (any) {
+    const void* const act[] = {delta, u, Bm, Cm, gy, g_delta, g_u, g_B, g_C};
+    const char* const an[] = {"delta", "u", "B", "C", "gy", "g_delta", "g_u", "g_B", "g_C"};
+    for (int i = 0; i < 9; ++i)
+      if (!act[i]) {
+        set_error("%s is NULL", an[i]);
+        return JM_ERR_INVALID_ARG;
+      }
+  }
+  const size_t need = jm_scan_bwd_workspace_size(dims);
+  if (!workspace || reinterpret_cast<uintptr_t>(workspace) % 256 || ws_bytes < need) {
+    set_error("workspace must be 256-byte aligned and at least %zu bytes", need);
+    return JM_ERR_WORKSPACE;
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(ErrFlags), s);
+  if (e != cudaSuccess) {
+    // reported below
+  } else if (!any) {
+    // nothing flows back: every gradient is zero
+    e = cudaMemsetAsync(g_A_log, 0, (size_t)d * kN * 4, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(g_D, 0, (size_t)d * 4, s);
+    if (e == cudaSuccess && g_h0 && B > 0) e = cudaMemsetAsync(g_h0, 0, (size_t)B * d * kN * 4, s);
+  } else {
+    BwdWs w = bwd_layout(B, L, d, static_cast<char*>(workspace));
+    BwdArgs a{B, L, d, delta, u, Bm, Cm, A_log, D, h0, gy, g_delta, g_u, g_h0,
+              w.ckpt, w.part_bc, w.part_a, w.part_d};
+    k_scan_bwd<<<dim3((unsigned)((d + kBwdThreads - 1) / kBwdThreads), (unsigned)B), kBwdThreads,
+                 0, s>>>(a);
+    const int64_t total = B * L * 32 + d * kN + d;
+    k_scan_bwd_reduce<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
+        w.part_bc, w.n_rows, B * L, w.part_a, w.part_d, A_log, B, d, g_B, g_C, g_A_log, g_D);
+    e = cudaGetLastError();
+  }
+  if (e != cudaSuccess) {
+    set_error("CUDA error: %s", cudaGetErrorString(e));
+    return JM_ERR_CUDA;
+  }
+  return JM_OK;
+}

@@ -27,7 +27,8 @@ EXPORTED = ("jm_mixer_fwd_workspace_size", "jm_mixer_step_workspace_size", "jm_m
             "jm_last_launch_count", "jm_last_kernel_name", "jm_set_kernel_events",
             "jm_mixer_step_noalloc", "jm_mixer_fwd_schedule",
             "jm_mixer_fwd_varlen_workspace_size", "jm_mixer_fwd_varlen", "jm_selftest_timeout",
-            "jm_layer_fwd_workspace_size", "jm_layer_fwd")
+            "jm_layer_fwd_workspace_size", "jm_layer_fwd", "jm_scan_bwd_workspace_size",
+            "jm_scan_bwd")
 
 
 class jm_dims(ctypes.Structure):
@@ -79,6 +80,10 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.jm_layer_fwd.restype = ctypes.c_int
     lib.jm_layer_fwd.argtypes = ([ctypes.POINTER(jm_dims), ctypes.c_int64] + [_vp] * 19
                                  + [ctypes.c_size_t, _vp])
+    lib.jm_scan_bwd_workspace_size.restype = ctypes.c_size_t
+    lib.jm_scan_bwd_workspace_size.argtypes = [ctypes.POINTER(jm_dims)]
+    lib.jm_scan_bwd.restype = ctypes.c_int
+    lib.jm_scan_bwd.argtypes = [ctypes.POINTER(jm_dims)] + [_vp] * 16 + [ctypes.c_size_t, _vp]
     lib.jm_selftest_timeout.restype = ctypes.c_int
     lib.jm_selftest_timeout.argtypes = [_vp, ctypes.c_size_t, _vp]
     lib.jm_mixer_fwd_schedule.restype = ctypes.c_int
@@ -173,6 +178,22 @@ def jm_layer_fwd(d: jm_dims, d_model: int, hidden, in_proj_w, w: Mapping, out_pr
                              *_weights(w), _ptr(out_proj_w), _ptr(out), _ptr(final_state),
                              _ptr(init_conv_state), _ptr(init_ssm_state),
                              _ptr(final_conv_state), _ptr(workspace), ws_bytes, _stream(stream))
+    if check:
+        _check(st)
+    return st
+
+
+def jm_scan_bwd_workspace_size(d: jm_dims) -> int:
+    return load().jm_scan_bwd_workspace_size(ctypes.byref(d))
+
+
+def jm_scan_bwd(d: jm_dims, delta, u, Bm, Cm, A_log, D, h0, gy, g_delta, g_u, g_B, g_C,
+                g_A_log, g_D, g_h0, workspace, ws_bytes: int, stream=None,
+                check: bool = True) -> int:
+    """Backward of the scan core (see include/jmix.h); float32 device tensors."""
+    st = load().jm_scan_bwd(ctypes.byref(d), *[_ptr(t) for t in (
+        delta, u, Bm, Cm, A_log, D, h0, gy, g_delta, g_u, g_B, g_C, g_A_log, g_D, g_h0,
+        workspace)], ws_bytes, _stream(stream))
     if check:
         _check(st)
     return st
