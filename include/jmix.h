@@ -155,10 +155,18 @@ jm_status jm_mixer_step_noalloc(const jm_dims* dims, const void* x_t, const void
 
 /* End-to-end forward from HOST buffers: copies x_host and z_host (pinned host
  * memory, [B, L, d] io dtype) into the caller's device buffers x_dev / z_dev,
- * runs jm_mixer_fwd, and copies y and the final SSM state back into y_host
- * and final_state_host.  All copies are cudaMemcpyAsync on `stream`; the call
- * returns without waiting (synchronise the stream before reading y_host).
- * Weights and the optional states are device pointers as in jm_mixer_fwd. */
+ * runs the forward, and copies y and the final SSM state back into y_host and
+ * final_state_host.  The batch runs in up to 8 groups of whole sequences so
+ * that copies in both directions overlap the compute: each group's inputs go
+ * up on an internal stream, its forward runs on `stream`, its outputs come down
+ * on a second internal stream (both created once per host thread; no device
+ * memory is allocated).  The call returns without waiting, and `stream` covers
+ * every copy: synchronise it before reading y_host.  A group uses the same
+ * arithmetic as jm_mixer_fwd on its sequences (the x_proj split and the scan
+ * schedule follow the group's size, so bits may differ from one jm_mixer_fwd
+ * call over the whole batch, within the same tolerances).  If a group would
+ * need more than ws_bytes, the batch runs as one group.  Weights are device
+ * pointers as in jm_mixer_fwd; the states start from zero. */
 jm_status jm_mixer_fwd_host(const jm_dims* dims, const void* x_host, const void* z_host,
                             void* y_host, float* final_state_host, void* x_dev, void* z_dev,
                             void* y_dev, float* final_state_dev, const void* conv_w,

@@ -168,6 +168,38 @@ jm_status finish(Problem& p, cudaError_t e) {
 }  // namespace
 }  // namespace jmix
 
+namespace jmix {
+namespace {
+
+// jm_mixer_fwd_host: at most this many sequence groups (pipeline stages).
+constexpr int64_t kHostGroups = 8;
+
+// Copy streams and events of jm_mixer_fwd_host, created once per thread (no
+// device memory is allocated).
+struct HostStreams {
+  bool ok = false;
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t ev_entry = nullptr, ev_exit = nullptr, ev_in[8] = {}, ev_done[8] = {};
+  HostStreams() {
+    const unsigned f = cudaEventDisableTiming;
+    ok = cudaStreamCreateWithFlags(&in, cudaStreamNonBlocking) == cudaSuccess &&
+         cudaStreamCreateWithFlags(&out, cudaStreamNonBlocking) == cudaSuccess &&
+         cudaEventCreateWithFlags(&ev_entry, f) == cudaSuccess &&
+         cudaEventCreateWithFlags(&ev_exit, f) == cudaSuccess;
+    for (int i = 0; ok && i < 8; ++i)
+      ok = cudaEventCreateWithFlags(&ev_in[i], f) == cudaSuccess &&
+           cudaEventCreateWithFlags(&ev_done[i], f) == cudaSuccess;
+  }
+};
+
+HostStreams& host_streams() {
+  static thread_local HostStreams hs;
+  return hs;
+}
+
+}  // namespace
+}  // namespace jmix
+
 using namespace jmix;
 
 JM_API size_t jm_mixer_fwd_workspace_size(const jm_dims* dims) {
@@ -385,27 +417,77 @@ JM_API jm_status jm_mixer_fwd_host(const jm_dims* dims, const void* x_host, cons
     set_error("device staging buffers are required");
     return JM_ERR_INVALID_ARG;
   }
-  cudaError_t e = cudaSuccess;
-  if (act) {
-    e = cudaMemcpyAsync(x_dev, x_host, act, cudaMemcpyHostToDevice, s);
-    if (e == cudaSuccess) e = cudaMemcpyAsync(z_dev, z_host, act, cudaMemcpyHostToDevice, s);
-    if (e != cudaSuccess) {
-      set_error("CUDA error: %s", cudaGetErrorString(e));
-      return JM_ERR_CUDA;
+  // The batch runs in groups of whole sequences so that copies overlap compute:
+  // group g's inputs go up on an inbound stream, its forward runs on `stream`
+  // once they have landed, and its outputs come down on an outbound stream
+  // while later groups compute (PCIe moves both directions at once).  Each group
+  // is independent sequences, and the groups reuse the workspace in stream
+  // order; if a group would need more workspace than given, one group is used.
+  const int64_t B = dims->batch, L = dims->seqlen, d = dims->d_inner;
+  const size_t es = esize(dims->io);
+  int64_t groups = B >= 2 ? (B < kHostGroups ? B : kHostGroups) : 1;
+  int64_t bg = groups > 0 ? (B + groups - 1) / groups : 0;
+  if (groups > 1) {
+    jm_dims gd = *dims;
+    gd.batch = bg;
+    if (jm_mixer_fwd_workspace_size(&gd) > ws_bytes) {
+      groups = 1;
+      bg = B;
+    } else {
+      groups = (B + bg - 1) / bg;
     }
   }
-  Problem p;
-  st = fwd_impl(dims, x_dev, z_dev, conv_w, conv_b, xproj_w, dt_norm_w, b_norm_w, c_norm_w,
-                dtproj_w, dt_bias, A_log, D, y_dev, final_state_dev, nullptr, nullptr, nullptr,
-                workspace, ws_bytes, stream, false, p);
-  if (st != JM_OK) return st;
-  if (act) e = cudaMemcpyAsync(y_host, y_dev, act, cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess)
-    e = cudaMemcpyAsync(final_state_host, final_state_dev, sst, cudaMemcpyDeviceToHost, s);
+  HostStreams& hs = host_streams();
+  if (!hs.ok) {
+    set_error("could not create the copy streams");
+    return JM_ERR_CUDA;
+  }
+  cudaError_t e = cudaEventRecord(hs.ev_entry, s);  // earlier work on `stream` comes first
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(hs.in, hs.ev_entry, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(hs.out, hs.ev_entry, 0);
+  int launches = 0;
+  for (int64_t g = 0; g < groups && e == cudaSuccess; ++g) {
+    const int64_t b0 = g * bg, nb = (B - b0) < bg ? (B - b0) : bg;
+    const size_t a0 = (size_t)b0 * L * d * es, an = (size_t)nb * L * d * es;
+    const size_t s0 = (size_t)b0 * d * kN * 4, sn = (size_t)nb * d * kN * 4;
+    char* xd = static_cast<char*>(x_dev) + a0;
+    char* zd = static_cast<char*>(z_dev) + a0;
+    char* yd = static_cast<char*>(y_dev) + a0;
+    if (an) {
+      e = cudaMemcpyAsync(xd, static_cast<const char*>(x_host) + a0, an, cudaMemcpyHostToDevice,
+                          hs.in);
+      if (e == cudaSuccess)
+        e = cudaMemcpyAsync(zd, static_cast<const char*>(z_host) + a0, an,
+                            cudaMemcpyHostToDevice, hs.in);
+    }
+    if (e == cudaSuccess) e = cudaEventRecord(hs.ev_in[g], hs.in);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, hs.ev_in[g], 0);
+    if (e != cudaSuccess) break;
+    jm_dims gd = *dims;
+    gd.batch = nb;
+    Problem p;
+    st = fwd_impl(&gd, xd, zd, conv_w, conv_b, xproj_w, dt_norm_w, b_norm_w, c_norm_w, dtproj_w,
+                  dt_bias, A_log, D, yd, final_state_dev + s0 / 4, nullptr, nullptr, nullptr,
+                  workspace, ws_bytes, stream, false, p);
+    if (st != JM_OK) return st;
+    launches += p.launches;
+    e = cudaEventRecord(hs.ev_done[g], s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(hs.out, hs.ev_done[g], 0);
+    if (e == cudaSuccess && an)
+      e = cudaMemcpyAsync(static_cast<char*>(y_host) + a0, yd, an, cudaMemcpyDeviceToHost, hs.out);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(reinterpret_cast<char*>(final_state_host) + s0,
+                          reinterpret_cast<char*>(final_state_dev) + s0, sn,
+                          cudaMemcpyDeviceToHost, hs.out);
+  }
+  // the caller's stream covers every copy from here on
+  if (e == cudaSuccess) e = cudaEventRecord(hs.ev_exit, hs.out);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, hs.ev_exit, 0);
   if (e != cudaSuccess) {
     set_error("CUDA error: %s", cudaGetErrorString(e));
     return JM_ERR_CUDA;
   }
+  g_launches = launches;
   return JM_OK;
 }
 

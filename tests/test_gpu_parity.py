@@ -142,6 +142,42 @@ def test_host_entry_point_matches_device_call():
     np.testing.assert_array_equal(fsh.numpy(), fs_ref)
 
 
+@pytest.mark.parametrize("B", [8, 5, 11])
+def test_host_entry_point_runs_sequence_groups(B):
+    """jm_mixer_fwd_host pipelines the batch in groups of ceil(B/8) sequences; each
+    group computes exactly what jm_mixer_fwd computes on that slice."""
+    import torch
+    from mamba_selective_scan_jamba_b200 import devio, jmix
+    w = small(B, 200, 256, 32, extra=False)
+    W = synth.make_weights(w)
+    A = synth.make_activations(w)
+    Wd = devio.weights_to_device(W)
+    bg = -(-B // 8)
+    ys, fss = [], []
+    for b0 in range(0, B, bg):
+        sl = slice(b0, min(B, b0 + bg))
+        wg = w.with_(batch=sl.stop - sl.start)
+        Ag = dict(x=A["x"][sl].copy(), z=A["z"][sl].copy())
+        y, fs, _ = gpu_fwd(wg, W, Ag, use_init=False, want_conv=False)
+        ys.append(y)
+        fss.append(fs)
+    xh, zh = devio.to_pinned(A["x"]), devio.to_pinned(A["z"])
+    yh = torch.empty_like(xh).pin_memory()
+    fsh = torch.empty((B, 256, 16), dtype=torch.float32).pin_memory()
+    xd, zd = torch.empty_like(xh, device="cuda"), torch.empty_like(zh, device="cuda")
+    yd = torch.empty_like(xd)
+    fsd = torch.empty((B, 256, 16), dtype=torch.float32, device="cuda")
+    d = devio.dims_of(w)
+    n = jmix.jm_mixer_fwd_workspace_size(d)
+    ws = devio.workspace(n)
+    s = torch.cuda.Stream()
+    jmix.jm_mixer_fwd_host(d, xh, zh, yh, fsh, xd, zd, yd, fsd, Wd, ws, n, stream=s)
+    s.synchronize()
+    assert jmix.jm_poll_error(ws, s) == jmix.JM_OK
+    np.testing.assert_array_equal(devio.to_host(yh), np.concatenate(ys))
+    np.testing.assert_array_equal(fsh.numpy(), np.concatenate(fss))
+
+
 def run_decode(w: synth.Workload, steps: int, channels=None, threads=0):
     """GPU decode steps vs the oracle; returns errors."""
     import torch
