@@ -429,6 +429,16 @@ def oracle_rate(w, target_s: float, threads: int = 0):
                                 f"fp64 oracle, {cores} threads, {dt:.1f} s")
 
 
+def bench_config(w, world: int) -> dict:
+    """The `config` object of both arms' JSON lines."""
+    in_bytes = w.batch * w.seqlen * w.d_inner * (2 if w.io == "bf16" else 4) * 2
+    return {"workload": w.name, "batch_per_gpu": w.batch, "seqlen": w.seqlen,
+            "d_inner": w.d_inner, "d_state": w.d_state, "dt_rank": w.dt_rank,
+            "discretization": "zoh" if w.zoh else "euler",
+            "parallelism": f"replicas x{world} (independent sequences)",
+            "l2": f"no flush: x+z = {in_bytes / 1e9:.2f} GB per step > 126 MB L2"}
+
+
 def reference_arm(args, w, rank, world):
     if rank != 0:
         return
@@ -455,8 +465,7 @@ def reference_arm(args, w, rank, world):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "batch": w.batch, "seqlen": w.seqlen,
-                       "d_inner": w.d_inner, "d_state": w.d_state, "dt_rank": w.dt_rank},
+            "config": bench_config(w, world),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -600,10 +609,7 @@ def main():
             "warmup": Wm, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16" if w.io == "bf16" else "f32",
             "data": "synthetic",
-            "config": {"workload": w.name, "batch_per_gpu": w.batch, "seqlen": w.seqlen,
-                       "d_inner": w.d_inner, "d_state": w.d_state, "dt_rank": w.dt_rank,
-                       "parallelism": f"replicas x{world} (independent sequences)",
-                       "l2": f"no flush: x+z = {in_bytes / 1e9:.2f} GB per step > 126 MB L2"},
+            "config": bench_config(w, world),
             "roofline": roofline, "gpu_launches": launches, "clocks": clocks}
 
     # end to end through the host-buffer entry point
