@@ -52,7 +52,7 @@ def parse():
     ap.add_argument("--zoh", action="store_true",
                     help="discretise B by zero-order hold instead of delta B")
     ap.add_argument("--bwd", action="store_true",
-                    help="also time the scan-core backward (B=1, L=4096, d_inner 8192)")
+                    help="also time the scan-core backward (B=1 and B=8, L=4096, d_inner 8192)")
     ap.add_argument("--layer", action="store_true",
                     help="also time the full layer (in_proj -> mixer -> out_proj, d_model 4096)")
     ap.add_argument("--varlen", action="store_true",
@@ -646,7 +646,7 @@ def main():
     if args.layer:
         line["layer"] = layer_bench(dev, stream, w)
     if args.bwd:
-        line["bwd"] = bwd_bench(dev, stream)
+        line["bwd"] = [bwd_bench(dev, stream, B=1), bwd_bench(dev, stream, B=8)]
     if not args.no_decode:
         dec = decode_bench(dev, stream, zoh=args.zoh)
         dec["hbm_frac"] = dec["achieved_GBps"] / P["hbm"]

@@ -9,15 +9,27 @@
 //   gA_n += g_n delta_t a_t,n h_{t-1},n;  gD += gy_t u_t;  g <- a_t g  (to h_{t-1});
 // and g_h0 = g after the first token, gA_log = gA * A.
 //
-// k_scan_bwd: CTA = (128-channel tile, sequence), thread = channel, 16 states in
-// registers.  Pass 1 runs the recurrence forward and stores the state at the
-// start of every kCk-token chunk.  Pass 2 walks the chunks backwards: it
-// recomputes the chunk's states into shared memory ([token][state][channel],
-// conflict-free) and runs the reverse recurrence token by token.  gB and gC are
-// sums over channels: each warp reduces its 32 channels' 32 values (16 gB, 16 gC)
-// by a reduce-scatter of shuffles (lane i ends with index i) into a per-warp
-// partial row; k_scan_bwd_reduce adds the partials in a fixed order, and gA_log,
-// gD over the sequences, so the results are reproducible.
+// Time parts.  Each sequence is cut into P parts of whole chunks that run side by
+// side.  Both recurrences are linear with the same decays, so a part acts on
+// what enters it through one factor, exp(A S), S = sum of delta over the part:
+//   forward:  h_end = exp(A S) h_start + f_p   (f_p: the part's end state from 0)
+//   adjoint:  g_out = exp(A S) g_in + r_p      (r_p: the gradient the part sends
+//             to h before it when nothing enters from its right; g_in is what
+//             the part after it sends)
+// k_scan_bwd_parts computes f_p, r_p and S for every part; each part of
+// k_scan_bwd then folds them (forward over the parts before it, from h0;
+// adjoint over the parts after it, from zero) into its own h_start and g_in.
+//
+// k_scan_bwd: CTA = (128-channel tile, sequence, part), thread = channel, 16
+// states in registers.  Pass 1 runs the recurrence forward over the part and
+// stores the state at the start of every kCk-token chunk.  Pass 2 walks the
+// part's chunks backwards: it recomputes the chunk's states into shared memory
+// ([token][state][channel], conflict-free) and runs the reverse recurrence
+// token by token.  gB and gC are sums over channels: each warp reduces its 32
+// channels' 32 values (16 gB, 16 gC) by a reduce-scatter of shuffles (lane i
+// ends with index i) into a per-warp partial row; k_scan_bwd_reduce adds the
+// partials in a fixed order, and gA_log, gD over the (sequence, part) rows, so
+// the results are reproducible.
 #include "jmix_internal.cuh"
 
 #define JM_API extern "C" __attribute__((visibility("default")))
@@ -27,6 +39,36 @@ namespace {
 
 constexpr int kBwdThreads = 128;
 constexpr int kCk = 4;  // tokens per checkpoint chunk (32 KB of states in shared memory)
+constexpr int kBwdMaxParts = 16;
+constexpr int kBwdMinPartChunks = 2;
+// Resident k_scan_bwd CTAs on a B200: 3 per SM (154 registers x 128 threads).
+constexpr int kBwdSlots = 3 * 148;
+
+// Time parts per sequence.  Parts cost an extra kernel (two passes over the
+// tokens), so a batch that already fills the GPU's CTA slots well runs as one
+// part; otherwise P (at most kBwdMaxParts, parts of at least kBwdMinPartChunks
+// chunks) maximises the filled fraction of the waves of (tile, sequence, part)
+// CTAs, less 1% per part for the folds.
+int bwd_parts(int64_t B, int64_t L, int64_t d) {
+  const int64_t n_tiles = (d + kBwdThreads - 1) / kBwdThreads;
+  const int64_t nck = (L + kCk - 1) / kCk;
+  if (B <= 0 || nck <= 0) return 1;
+  auto fill = [&](int64_t P) {
+    const int64_t ctas = n_tiles * B * P;
+    return (double)ctas / (double)(((ctas + kBwdSlots - 1) / kBwdSlots) * kBwdSlots);
+  };
+  if (fill(1) >= 0.9) return 1;
+  int best = 1;
+  double best_score = fill(1);
+  for (int P = 2; P <= kBwdMaxParts && P * kBwdMinPartChunks <= nck; ++P) {
+    const double score = fill(P) - 0.01 * (P - 1);
+    if (score > best_score) {
+      best_score = score;
+      best = P;
+    }
+  }
+  return best;
+}
 
 struct BwdArgs {
   int64_t B, L, d;
@@ -43,9 +85,60 @@ struct BwdArgs {
   float* gh0;
   float* ckpt;      // [B, nck, d, 16]
   float* part_bc;   // [n_tiles * 4, B * L, 32]: per-warp sums of gB (0..15), gC (16..31)
-  float* part_a;    // [B, d, 16]
-  float* part_d;    // [B, d]
+  float* part_a;    // [P * B, d, 16]
+  float* part_d;    // [P * B, d]
+  int P;            // time parts per sequence
+  float* f_end;     // [P * B, d, 16]: a part's end state from a zero start
+  float* r_out;     // [P * B, d, 16]: a part's outgoing gradient with nothing entering
+  float* s_sum;     // [P * B, d]: a part's sum of delta
 };
+
+// Chunks [k0, k1) of the sequence form part p.
+__device__ __forceinline__ void part_chunks(int64_t nck, int P, int p, int64_t& k0, int64_t& k1) {
+  k0 = nck * p / P;
+  k1 = nck * (p + 1) / P;
+}
+
+// For each part: f_p (forward from a zero state), S (sum of delta) and r_p (the
+// adjoint run backwards from a zero incoming gradient: g += C_t gy_t, g <- a_t g).
+__global__ void __launch_bounds__(kBwdThreads) k_scan_bwd_parts(const BwdArgs a) {
+  const int64_t b = blockIdx.y;
+  const int p = blockIdx.z;
+  const int64_t c = (int64_t)blockIdx.x * kBwdThreads + threadIdx.x;
+  if (c >= a.d) return;
+  const int64_t L = a.L, d = a.d;
+  const int64_t nck = (L + kCk - 1) / kCk;
+  int64_t k0, k1;
+  part_chunks(nck, a.P, p, k0, k1);
+  const int64_t t0 = k0 * kCk, t1 = k1 * kCk < L ? k1 * kCk : L;
+  float A[kN];
+#pragma unroll
+  for (int n = 0; n < kN; ++n) A[n] = -expf(a.A_log[c * kN + n]);
+  float h[kN], g[kN];
+#pragma unroll
+  for (int n = 0; n < kN; ++n) h[n] = g[n] = 0.0f;
+  float S = 0.0f;
+  for (int64_t t = t0; t < t1; ++t) {
+    const float dl = a.delta[(b * L + t) * d + c], du = dl * a.u[(b * L + t) * d + c];
+    const float* Bt = a.Bm + (b * L + t) * kN;
+    S += dl;
+#pragma unroll
+    for (int n = 0; n < kN; ++n) h[n] = fmaf(expf(dl * A[n]), h[n], du * Bt[n]);
+  }
+  for (int64_t t = t1 - 1; t >= t0; --t) {
+    const float dl = a.delta[(b * L + t) * d + c], gyt = a.gy[(b * L + t) * d + c];
+    const float* Ct = a.Cm + (b * L + t) * kN;
+#pragma unroll
+    for (int n = 0; n < kN; ++n) g[n] = expf(dl * A[n]) * fmaf(Ct[n], gyt, g[n]);
+  }
+  const int64_t row = ((int64_t)p * a.B + b) * d + c;
+#pragma unroll
+  for (int n = 0; n < kN; ++n) {
+    a.f_end[row * kN + n] = h[n];
+    a.r_out[row * kN + n] = g[n];
+  }
+  a.s_sum[row] = S;
+}
 
 // Sums v over the 32 lanes of the warp, index by index: afterwards lane i holds
 // in v[0] the sum of every lane's v[i].
@@ -66,20 +159,31 @@ __global__ void __launch_bounds__(kBwdThreads) k_scan_bwd(const BwdArgs a) {
   __shared__ float hs[kCk][kN][kBwdThreads];  // states after each token of the chunk
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t b = blockIdx.y;
+  const int p = blockIdx.z, P = a.P;
   const int64_t c = (int64_t)blockIdx.x * kBwdThreads + threadIdx.x;
   const bool cok = c < a.d;
   const int64_t L = a.L, d = a.d;
   const int64_t nck = (L + kCk - 1) / kCk;
+  int64_t k0, k1;
+  part_chunks(nck, P, p, k0, k1);
+  const int64_t t_begin = k0 * kCk, t_end = k1 * kCk < L ? k1 * kCk : L;
   float A[kN];
 #pragma unroll
   for (int n = 0; n < kN; ++n) A[n] = cok ? -expf(a.A_log[c * kN + n]) : 0.0f;
   const float Dc = cok ? a.D[c] : 0.0f;
-  auto at = [&](const float* p, int64_t t) { return cok ? p[(b * L + t) * d + c] : 0.0f; };
-  // pass 1: forward, checkpoint at every chunk start
+  auto at = [&](const float* q, int64_t t) { return cok ? q[(b * L + t) * d + c] : 0.0f; };
+  // the part's start state: h0 folded through the parts before it
   float h[kN];
 #pragma unroll
   for (int n = 0; n < kN; ++n) h[n] = (cok && a.h0) ? a.h0[(b * d + c) * kN + n] : 0.0f;
-  for (int64_t t = 0; t < L; ++t) {
+  for (int q = 0; q < p && cok; ++q) {
+    const int64_t row = ((int64_t)q * a.B + b) * d + c;
+    const float S = a.s_sum[row];
+#pragma unroll
+    for (int n = 0; n < kN; ++n) h[n] = fmaf(expf(A[n] * S), h[n], a.f_end[row * kN + n]);
+  }
+  // pass 1: forward, checkpoint at every chunk start
+  for (int64_t t = t_begin; t < t_end; ++t) {
     if (t % kCk == 0 && cok) {
       float* ck = a.ckpt + ((b * nck + t / kCk) * d + c) * kN;
 #pragma unroll
@@ -90,12 +194,18 @@ __global__ void __launch_bounds__(kBwdThreads) k_scan_bwd(const BwdArgs a) {
 #pragma unroll
     for (int n = 0; n < kN; ++n) h[n] = fmaf(expf(dl * A[n]), h[n], du * Bt[n]);
   }
-  // pass 2: reverse
+  // pass 2: reverse, from the gradient the parts after this one send into it
   float g[kN], gA[kN], gD = 0.0f;
 #pragma unroll
   for (int n = 0; n < kN; ++n) g[n] = gA[n] = 0.0f;
+  for (int q = P - 1; q > p && cok; --q) {
+    const int64_t row = ((int64_t)q * a.B + b) * d + c;
+    const float S = a.s_sum[row];
+#pragma unroll
+    for (int n = 0; n < kN; ++n) g[n] = fmaf(expf(A[n] * S), g[n], a.r_out[row * kN + n]);
+  }
   const int64_t tile_warp = (int64_t)blockIdx.x * 4 + warp;
-  for (int64_t j = nck - 1; j >= 0; --j) {
+  for (int64_t j = k1 - 1; j >= k0; --j) {
     const int64_t t0 = j * kCk;
     const int nt = (int)((L - t0) < kCk ? (L - t0) : kCk);
     float hstart[kN];
@@ -153,20 +263,21 @@ __global__ void __launch_bounds__(kBwdThreads) k_scan_bwd(const BwdArgs a) {
     }
   }
   if (cok) {
+    const int64_t row = ((int64_t)p * a.B + b) * d + c;
 #pragma unroll
-    for (int n = 0; n < kN; ++n) a.part_a[(b * d + c) * kN + n] = gA[n];
-    a.part_d[b * d + c] = gD;
-    if (a.gh0)
+    for (int n = 0; n < kN; ++n) a.part_a[row * kN + n] = gA[n];
+    a.part_d[row] = gD;
+    if (a.gh0 && p == 0)
 #pragma unroll
       for (int n = 0; n < kN; ++n) a.gh0[(b * d + c) * kN + n] = g[n];
   }
 }
 
 // gB, gC: sum over the per-warp partial rows, in order; gA_log, gD: sum over
-// the sequences, in order, then gA_log = gA * A.
+// the (part, sequence) rows, in order, then gA_log = gA * A.
 __global__ void k_scan_bwd_reduce(const float* __restrict__ part_bc, int64_t n_rows, int64_t TB,
                                   const float* __restrict__ part_a, const float* __restrict__ part_d,
-                                  const float* __restrict__ A_log, int64_t B, int64_t d,
+                                  const float* __restrict__ A_log, int64_t n_ad, int64_t d,
                                   float* __restrict__ gB, float* __restrict__ gC,
                                   float* __restrict__ gA_log, float* __restrict__ gD) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -185,14 +296,14 @@ __global__ void k_scan_bwd_reduce(const float* __restrict__ part_bc, int64_t n_r
   const int64_t j = i - n_bc;
   if (j < d * kN) {
     float s = 0.0f;
-    for (int64_t bb = 0; bb < B; ++bb) s += part_a[bb * d * kN + j];
+    for (int64_t bb = 0; bb < n_ad; ++bb) s += part_a[bb * d * kN + j];
     gA_log[j] = s * -expf(A_log[j]);  // dA/dA_log = A
     return;
   }
   const int64_t c = j - d * kN;
   if (c < d) {
     float s = 0.0f;
-    for (int64_t bb = 0; bb < B; ++bb) s += part_d[bb * d + c];
+    for (int64_t bb = 0; bb < n_ad; ++bb) s += part_d[bb * d + c];
     gD[c] = s;
   }
 }
@@ -202,8 +313,12 @@ struct BwdWs {
   float* part_bc;
   float* part_a;
   float* part_d;
+  float* f_end;
+  float* r_out;
+  float* s_sum;
   size_t bytes;
   int64_t n_rows;
+  int P;
 };
 
 BwdWs bwd_layout(int64_t B, int64_t L, int64_t d, char* base) {
@@ -217,11 +332,16 @@ BwdWs bwd_layout(int64_t B, int64_t L, int64_t d, char* base) {
   const int64_t nck = (L + kCk - 1) / kCk;
   const int64_t n_tiles = (d + kBwdThreads - 1) / kBwdThreads;
   w.n_rows = n_tiles * 4;
+  w.P = bwd_parts(B, L, d);
+  const size_t rows = (size_t)w.P * B * d;
   take(sizeof(ErrFlags));  // the error header jm_poll_error reads (cleared each call)
   w.ckpt = take((size_t)B * nck * d * kN * 4);
   w.part_bc = take((size_t)w.n_rows * B * L * 32 * 4);
-  w.part_a = take((size_t)B * d * kN * 4);
-  w.part_d = take((size_t)B * d * 4);
+  w.part_a = take(rows * kN * 4);
+  w.part_d = take(rows * 4);
+  w.f_end = take(rows * kN * 4);
+  w.r_out = take(rows * kN * 4);
+  w.s_sum = take(rows * 4);
   w.bytes = off;
   return w;
 }
@@ -242,6 +362,10 @@ jm_status check_bwd_dims(const jm_dims* dm) {
   if (dm->discretization != JM_DISC_EULER) {
     set_error("the scan backward is built for Euler B (delta B) only");
     return JM_ERR_UNSUPPORTED;
+  }
+  if (dm->batch > 65535) {
+    set_error("batch above 65535 is not supported by the scan backward's launch grid");
+    return JM_ERR_INVALID_ARG;
   }
   if ((double)dm->batch * (double)dm->seqlen * (double)dm->d_inner > 1.0e13) {
     set_error("problem too large");
@@ -301,13 +425,17 @@ JM_API jm_status jm_scan_bwd(const jm_dims* dims, const float* delta, const floa
     if (e == cudaSuccess && g_h0 && B > 0) e = cudaMemsetAsync(g_h0, 0, (size_t)B * d * kN * 4, s);
   } else {
     BwdWs w = bwd_layout(B, L, d, static_cast<char*>(workspace));
-    BwdArgs a{B, L, d, delta, u, Bm, Cm, A_log, D, h0, gy, g_delta, g_u, g_h0,
-              w.ckpt, w.part_bc, w.part_a, w.part_d};
-    k_scan_bwd<<<dim3((unsigned)((d + kBwdThreads - 1) / kBwdThreads), (unsigned)B), kBwdThreads,
-                 0, s>>>(a);
+    BwdArgs a{B,          L,          d,       delta,   u,       Bm,      Cm,
+              A_log,      D,          h0,      gy,      g_delta, g_u,     g_h0,
+              w.ckpt,     w.part_bc,  w.part_a, w.part_d, w.P,    w.f_end, w.r_out,
+              w.s_sum};
+    const dim3 grid((unsigned)((d + kBwdThreads - 1) / kBwdThreads), (unsigned)B, (unsigned)w.P);
+    if (w.P > 1) k_scan_bwd_parts<<<grid, kBwdThreads, 0, s>>>(a);
+    k_scan_bwd<<<grid, kBwdThreads, 0, s>>>(a);
     const int64_t total = B * L * 32 + d * kN + d;
     k_scan_bwd_reduce<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
-        w.part_bc, w.n_rows, B * L, w.part_a, w.part_d, A_log, B, d, g_B, g_C, g_A_log, g_D);
+        w.part_bc, w.n_rows, B * L, w.part_a, w.part_d, A_log, (int64_t)w.P * B, d, g_B, g_C,
+        g_A_log, g_D);
     e = cudaGetLastError();
   }
   if (e != cudaSuccess) {

@@ -61,8 +61,11 @@ def _oracle_bwd(p):
                 h0=np.stack([g["h0"] for g in per]))
 
 
+# (2, 301, 384) and (1, 1000, 1024) run as 16 time parts (ragged parts and a
+# ragged last chunk); (2, 37, 200) and (3, 4, 128) as one part.
 @pytest.mark.parametrize("B,L,d,h0", [(2, 37, 200, True), (1, 1000, 1024, False),
-                                      (3, 4, 128, True)])
+                                      (3, 4, 128, True), (2, 301, 384, True),
+                                      (1, 2048, 2048, True)])
 def test_scan_bwd_matches_oracle(B, L, d, h0):
     p = _inputs(B, L, d, seed=B * 1000 + L, with_h0=h0)
     got = _gpu_bwd(p)
