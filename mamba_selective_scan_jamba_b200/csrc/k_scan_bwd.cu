@@ -40,6 +40,7 @@ namespace {
 constexpr int kBwdThreads = 128;
 constexpr int kCk = 4;  // tokens per checkpoint chunk (32 KB of states in shared memory)
 constexpr int kBwdMaxParts = 16;
+constexpr int kPg = 8;  // tokens per load group in k_scan_bwd_parts
 constexpr int kBwdMinPartChunks = 2;
 // Resident k_scan_bwd CTAs on a B200: 3 per SM (154 registers x 128 threads).
 constexpr int kBwdSlots = 3 * 148;
@@ -118,18 +119,41 @@ __global__ void __launch_bounds__(kBwdThreads) k_scan_bwd_parts(const BwdArgs a)
 #pragma unroll
   for (int n = 0; n < kN; ++n) h[n] = g[n] = 0.0f;
   float S = 0.0f;
-  for (int64_t t = t0; t < t1; ++t) {
-    const float dl = a.delta[(b * L + t) * d + c], du = dl * a.u[(b * L + t) * d + c];
-    const float* Bt = a.Bm + (b * L + t) * kN;
-    S += dl;
+  // groups of kPg tokens: the group's per-channel loads go out before its
+  // arithmetic, so their latency is paid once per group, not once per token
+  for (int64_t tg = t0; tg < t1; tg += kPg) {
+    float dl[kPg], uv[kPg];
 #pragma unroll
-    for (int n = 0; n < kN; ++n) h[n] = fmaf(expf(dl * A[n]), h[n], du * Bt[n]);
+    for (int i = 0; i < kPg; ++i) {
+      const int64_t t = tg + i < t1 ? tg + i : t1 - 1;
+      dl[i] = a.delta[(b * L + t) * d + c];
+      uv[i] = a.u[(b * L + t) * d + c];
+    }
+#pragma unroll
+    for (int i = 0; i < kPg; ++i) {
+      if (tg + i >= t1) break;
+      const float du = dl[i] * uv[i];
+      const float* Bt = a.Bm + (b * L + tg + i) * kN;
+      S += dl[i];
+#pragma unroll
+      for (int n = 0; n < kN; ++n) h[n] = fmaf(expf(dl[i] * A[n]), h[n], du * Bt[n]);
+    }
   }
-  for (int64_t t = t1 - 1; t >= t0; --t) {
-    const float dl = a.delta[(b * L + t) * d + c], gyt = a.gy[(b * L + t) * d + c];
-    const float* Ct = a.Cm + (b * L + t) * kN;
+  for (int64_t tg = t1 - 1; tg >= t0; tg -= kPg) {  // tokens tg, tg-1, .. (at least t0)
+    float dl[kPg], gyt[kPg];
 #pragma unroll
-    for (int n = 0; n < kN; ++n) g[n] = expf(dl * A[n]) * fmaf(Ct[n], gyt, g[n]);
+    for (int i = 0; i < kPg; ++i) {
+      const int64_t t = tg - i >= t0 ? tg - i : t0;
+      dl[i] = a.delta[(b * L + t) * d + c];
+      gyt[i] = a.gy[(b * L + t) * d + c];
+    }
+#pragma unroll
+    for (int i = 0; i < kPg; ++i) {
+      if (tg - i < t0) break;
+      const float* Ct = a.Cm + (b * L + tg - i) * kN;
+#pragma unroll
+      for (int n = 0; n < kN; ++n) g[n] = expf(dl[i] * A[n]) * fmaf(Ct[n], gyt[i], g[n]);
+    }
   }
   const int64_t row = ((int64_t)p * a.B + b) * d + c;
 #pragma unroll
@@ -182,17 +206,30 @@ __global__ void __launch_bounds__(kBwdThreads) k_scan_bwd(const BwdArgs a) {
 #pragma unroll
     for (int n = 0; n < kN; ++n) h[n] = fmaf(expf(A[n] * S), h[n], a.f_end[row * kN + n]);
   }
-  // pass 1: forward, checkpoint at every chunk start
-  for (int64_t t = t_begin; t < t_end; ++t) {
-    if (t % kCk == 0 && cok) {
-      float* ck = a.ckpt + ((b * nck + t / kCk) * d + c) * kN;
+  // pass 1: forward, checkpoint at every chunk start; a chunk's loads go out
+  // before its arithmetic
+  for (int64_t j = k0; j < k1; ++j) {
+    const int64_t t0 = j * kCk;
+    const int nt = (int)((L - t0) < kCk ? (L - t0) : kCk);
+    if (cok) {
+      float* ck = a.ckpt + ((b * nck + j) * d + c) * kN;
 #pragma unroll
       for (int n = 0; n < kN; ++n) ck[n] = h[n];
     }
-    const float dl = at(a.delta, t), du = dl * at(a.u, t);
-    const float* Bt = a.Bm + (b * L + t) * kN;
+    float dl[kCk], uv[kCk];
 #pragma unroll
-    for (int n = 0; n < kN; ++n) h[n] = fmaf(expf(dl * A[n]), h[n], du * Bt[n]);
+    for (int i = 0; i < kCk; ++i) {
+      dl[i] = i < nt ? at(a.delta, t0 + i) : 0.0f;
+      uv[i] = i < nt ? at(a.u, t0 + i) : 0.0f;
+    }
+#pragma unroll
+    for (int i = 0; i < kCk; ++i) {
+      if (i >= nt) break;
+      const float du = dl[i] * uv[i];
+      const float* Bt = a.Bm + (b * L + t0 + i) * kN;
+#pragma unroll
+      for (int n = 0; n < kN; ++n) h[n] = fmaf(expf(dl[i] * A[n]), h[n], du * Bt[n]);
+    }
   }
   // pass 2: reverse, from the gradient the parts after this one send into it
   float g[kN], gA[kN], gD = 0.0f;
@@ -217,21 +254,31 @@ __global__ void __launch_bounds__(kBwdThreads) k_scan_bwd(const BwdArgs a) {
 #pragma unroll
       for (int n = 0; n < kN; ++n) hstart[n] = 0.0f;
     }
+    float dlc[kCk], uvc[kCk], gyc[kCk];  // the chunk's per-channel inputs
+#pragma unroll
+    for (int i = 0; i < kCk; ++i) {
+      dlc[i] = i < nt ? at(a.delta, t0 + i) : 0.0f;
+      uvc[i] = i < nt ? at(a.u, t0 + i) : 0.0f;
+      gyc[i] = i < nt ? at(a.gy, t0 + i) : 0.0f;
+    }
 #pragma unroll
     for (int n = 0; n < kN; ++n) h[n] = hstart[n];
-    for (int i = 0; i < nt; ++i) {
-      const int64_t t = t0 + i;
-      const float dl = at(a.delta, t), du = dl * at(a.u, t);
-      const float* Bt = a.Bm + (b * L + t) * kN;
+#pragma unroll
+    for (int i = 0; i < kCk; ++i) {
+      if (i >= nt) break;
+      const float du = dlc[i] * uvc[i];
+      const float* Bt = a.Bm + (b * L + t0 + i) * kN;
 #pragma unroll
       for (int n = 0; n < kN; ++n) {
-        h[n] = fmaf(expf(dl * A[n]), h[n], du * Bt[n]);
+        h[n] = fmaf(expf(dlc[i] * A[n]), h[n], du * Bt[n]);
         hs[i][n][threadIdx.x] = h[n];
       }
     }
-    for (int i = nt - 1; i >= 0; --i) {
+#pragma unroll
+    for (int i = kCk - 1; i >= 0; --i) {
+      if (i >= nt) continue;
       const int64_t t = t0 + i;
-      const float dl = at(a.delta, t), uv = at(a.u, t), gyt = at(a.gy, t);
+      const float dl = dlc[i], uv = uvc[i], gyt = gyc[i];
       const float* Bt = a.Bm + (b * L + t) * kN;
       const float* Ct = a.Cm + (b * L + t) * kN;
       float v[32];  // this channel's share of gB_t (0..15) and gC_t (16..31)
