@@ -38,6 +38,17 @@ namespace jmix {
 namespace {
 
 constexpr int kBwdThreads = 128;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// exp(y) as MUFU ex2 of y log2(e), with y = delta A already scaled: the argument
+// is A2 delta, A2 = A log2(e) (relative error ~2 ulp of ex2 plus the rounding of
+// the product; far inside the 1e-4 gradient tolerance).
+__device__ __forceinline__ float ex2f(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 constexpr int kCk = 4;  // tokens per checkpoint chunk (32 KB of states in shared memory)
 constexpr int kBwdMaxParts = 16;
 constexpr int kPg = 8;  // tokens per load group in k_scan_bwd_parts
@@ -106,55 +117,66 @@ __global__ void __launch_bounds__(kBwdThreads) k_scan_bwd_parts(const BwdArgs a)
   const int64_t b = blockIdx.y;
   const int p = blockIdx.z;
   const int64_t c = (int64_t)blockIdx.x * kBwdThreads + threadIdx.x;
-  if (c >= a.d) return;
+  // a group's kPg rows of B (forward) or C (adjoint): kPg * 16 = 128 floats, one
+  // per thread, double-buffered (one barrier per group)
+  __shared__ float rows[2][kPg * kN];
+  static_assert(kPg * kN == kBwdThreads, "one row element per thread");
+  const bool cok = c < a.d;
   const int64_t L = a.L, d = a.d;
   const int64_t nck = (L + kCk - 1) / kCk;
   int64_t k0, k1;
   part_chunks(nck, a.P, p, k0, k1);
   const int64_t t0 = k0 * kCk, t1 = k1 * kCk < L ? k1 * kCk : L;
-  float A[kN];
+  const int ri = threadIdx.x / kN, rn = threadIdx.x % kN;  // this thread's row element
+  float A2[kN];  // A log2(e)
 #pragma unroll
-  for (int n = 0; n < kN; ++n) A[n] = -expf(a.A_log[c * kN + n]);
+  for (int n = 0; n < kN; ++n) A2[n] = cok ? -expf(a.A_log[c * kN + n]) * kLog2e : 0.0f;
   float h[kN], g[kN];
 #pragma unroll
   for (int n = 0; n < kN; ++n) h[n] = g[n] = 0.0f;
   float S = 0.0f;
   // groups of kPg tokens: the group's per-channel loads go out before its
   // arithmetic, so their latency is paid once per group, not once per token
-  for (int64_t tg = t0; tg < t1; tg += kPg) {
+  int buf = 0;
+  for (int64_t tg = t0; tg < t1; tg += kPg, buf ^= 1) {
     float dl[kPg], uv[kPg];
 #pragma unroll
     for (int i = 0; i < kPg; ++i) {
       const int64_t t = tg + i < t1 ? tg + i : t1 - 1;
-      dl[i] = a.delta[(b * L + t) * d + c];
-      uv[i] = a.u[(b * L + t) * d + c];
+      dl[i] = cok ? a.delta[(b * L + t) * d + c] : 0.0f;
+      uv[i] = cok ? a.u[(b * L + t) * d + c] : 0.0f;
     }
+    rows[buf][threadIdx.x] = tg + ri < t1 ? a.Bm[(b * L + tg + ri) * kN + rn] : 0.0f;
+    __syncthreads();
 #pragma unroll
     for (int i = 0; i < kPg; ++i) {
       if (tg + i >= t1) break;
       const float du = dl[i] * uv[i];
-      const float* Bt = a.Bm + (b * L + tg + i) * kN;
+      const float* Bt = rows[buf] + i * kN;
       S += dl[i];
 #pragma unroll
-      for (int n = 0; n < kN; ++n) h[n] = fmaf(expf(dl[i] * A[n]), h[n], du * Bt[n]);
+      for (int n = 0; n < kN; ++n) h[n] = fmaf(ex2f(dl[i] * A2[n]), h[n], du * Bt[n]);
     }
   }
-  for (int64_t tg = t1 - 1; tg >= t0; tg -= kPg) {  // tokens tg, tg-1, .. (at least t0)
+  for (int64_t tg = t1 - 1; tg >= t0; tg -= kPg, buf ^= 1) {  // tokens tg, tg-1, .. (>= t0)
     float dl[kPg], gyt[kPg];
 #pragma unroll
     for (int i = 0; i < kPg; ++i) {
       const int64_t t = tg - i >= t0 ? tg - i : t0;
-      dl[i] = a.delta[(b * L + t) * d + c];
-      gyt[i] = a.gy[(b * L + t) * d + c];
+      dl[i] = cok ? a.delta[(b * L + t) * d + c] : 0.0f;
+      gyt[i] = cok ? a.gy[(b * L + t) * d + c] : 0.0f;
     }
+    rows[buf][threadIdx.x] = tg - ri >= t0 ? a.Cm[(b * L + tg - ri) * kN + rn] : 0.0f;
+    __syncthreads();
 #pragma unroll
     for (int i = 0; i < kPg; ++i) {
       if (tg - i < t0) break;
-      const float* Ct = a.Cm + (b * L + tg - i) * kN;
+      const float* Ct = rows[buf] + i * kN;
 #pragma unroll
-      for (int n = 0; n < kN; ++n) g[n] = expf(dl[i] * A[n]) * fmaf(Ct[n], gyt[i], g[n]);
+      for (int n = 0; n < kN; ++n) g[n] = ex2f(dl[i] * A2[n]) * fmaf(Ct[n], gyt[i], g[n]);
     }
   }
+  if (!cok) return;
   const int64_t row = ((int64_t)p * a.B + b) * d + c;
 #pragma unroll
   for (int n = 0; n < kN; ++n) {
@@ -179,8 +201,12 @@ __device__ __forceinline__ void warp_reduce_scatter32(float (&v)[32], int lane) 
   }
 }
 
-__global__ void __launch_bounds__(kBwdThreads) k_scan_bwd(const BwdArgs a) {
+__global__ void __launch_bounds__(kBwdThreads, 3) k_scan_bwd(const BwdArgs a) {
   __shared__ float hs[kCk][kN][kBwdThreads];  // states after each token of the chunk
+  // the chunk's rows of B (0..15) and C (16..31): kCk * 32 = 128 floats, one per
+  // thread, double-buffered (one barrier per chunk)
+  __shared__ float bcrow[2][kCk * 2 * kN];
+  static_assert(kCk * 2 * kN == kBwdThreads, "one row element per thread");
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t b = blockIdx.y;
   const int p = blockIdx.z, P = a.P;
@@ -191,11 +217,20 @@ __global__ void __launch_bounds__(kBwdThreads) k_scan_bwd(const BwdArgs a) {
   int64_t k0, k1;
   part_chunks(nck, P, p, k0, k1);
   const int64_t t_begin = k0 * kCk, t_end = k1 * kCk < L ? k1 * kCk : L;
-  float A[kN];
+  float A2[kN];  // A log2(e)
 #pragma unroll
-  for (int n = 0; n < kN; ++n) A[n] = cok ? -expf(a.A_log[c * kN + n]) : 0.0f;
+  for (int n = 0; n < kN; ++n) A2[n] = cok ? -expf(a.A_log[c * kN + n]) * kLog2e : 0.0f;
   const float Dc = cok ? a.D[c] : 0.0f;
   auto at = [&](const float* q, int64_t t) { return cok ? q[(b * L + t) * d + c] : 0.0f; };
+  // this thread's element of chunk j's B/C rows
+  const int ri = threadIdx.x / (2 * kN), rk = threadIdx.x % (2 * kN);
+  auto stage_rows = [&](int64_t j, int buf) {
+    const int64_t t = j * kCk + ri;
+    bcrow[buf][threadIdx.x] =
+        t < L ? (rk < kN ? a.Bm[(b * L + t) * kN + rk] : a.Cm[(b * L + t) * kN + rk - kN]) : 0.0f;
+    __syncthreads();
+  };
+  int buf = 0;
   // the part's start state: h0 folded through the parts before it
   float h[kN];
 #pragma unroll
@@ -204,7 +239,7 @@ __global__ void __launch_bounds__(kBwdThreads) k_scan_bwd(const BwdArgs a) {
     const int64_t row = ((int64_t)q * a.B + b) * d + c;
     const float S = a.s_sum[row];
 #pragma unroll
-    for (int n = 0; n < kN; ++n) h[n] = fmaf(expf(A[n] * S), h[n], a.f_end[row * kN + n]);
+    for (int n = 0; n < kN; ++n) h[n] = fmaf(ex2f(A2[n] * S), h[n], a.f_end[row * kN + n]);
   }
   // pass 1: forward, checkpoint at every chunk start; a chunk's loads go out
   // before its arithmetic
@@ -222,14 +257,16 @@ __global__ void __launch_bounds__(kBwdThreads) k_scan_bwd(const BwdArgs a) {
       dl[i] = i < nt ? at(a.delta, t0 + i) : 0.0f;
       uv[i] = i < nt ? at(a.u, t0 + i) : 0.0f;
     }
+    stage_rows(j, buf);
 #pragma unroll
     for (int i = 0; i < kCk; ++i) {
       if (i >= nt) break;
       const float du = dl[i] * uv[i];
-      const float* Bt = a.Bm + (b * L + t0 + i) * kN;
+      const float* Bt = bcrow[buf] + i * 2 * kN;
 #pragma unroll
-      for (int n = 0; n < kN; ++n) h[n] = fmaf(expf(dl[i] * A[n]), h[n], du * Bt[n]);
+      for (int n = 0; n < kN; ++n) h[n] = fmaf(ex2f(dl[i] * A2[n]), h[n], du * Bt[n]);
     }
+    buf ^= 1;
   }
   // pass 2: reverse, from the gradient the parts after this one send into it
   float g[kN], gA[kN], gD = 0.0f;
@@ -239,7 +276,7 @@ __global__ void __launch_bounds__(kBwdThreads) k_scan_bwd(const BwdArgs a) {
     const int64_t row = ((int64_t)q * a.B + b) * d + c;
     const float S = a.s_sum[row];
 #pragma unroll
-    for (int n = 0; n < kN; ++n) g[n] = fmaf(expf(A[n] * S), g[n], a.r_out[row * kN + n]);
+    for (int n = 0; n < kN; ++n) g[n] = fmaf(ex2f(A2[n] * S), g[n], a.r_out[row * kN + n]);
   }
   const int64_t tile_warp = (int64_t)blockIdx.x * 4 + warp;
   for (int64_t j = k1 - 1; j >= k0; --j) {
@@ -261,16 +298,17 @@ __global__ void __launch_bounds__(kBwdThreads) k_scan_bwd(const BwdArgs a) {
       uvc[i] = i < nt ? at(a.u, t0 + i) : 0.0f;
       gyc[i] = i < nt ? at(a.gy, t0 + i) : 0.0f;
     }
+    stage_rows(j, buf);
 #pragma unroll
     for (int n = 0; n < kN; ++n) h[n] = hstart[n];
 #pragma unroll
     for (int i = 0; i < kCk; ++i) {
       if (i >= nt) break;
       const float du = dlc[i] * uvc[i];
-      const float* Bt = a.Bm + (b * L + t0 + i) * kN;
+      const float* Bt = bcrow[buf] + i * 2 * kN;
 #pragma unroll
       for (int n = 0; n < kN; ++n) {
-        h[n] = fmaf(expf(dlc[i] * A[n]), h[n], du * Bt[n]);
+        h[n] = fmaf(ex2f(dlc[i] * A2[n]), h[n], du * Bt[n]);
         hs[i][n][threadIdx.x] = h[n];
       }
     }
@@ -279,24 +317,28 @@ __global__ void __launch_bounds__(kBwdThreads) k_scan_bwd(const BwdArgs a) {
       if (i >= nt) continue;
       const int64_t t = t0 + i;
       const float dl = dlc[i], uv = uvc[i], gyt = gyc[i];
-      const float* Bt = a.Bm + (b * L + t) * kN;
-      const float* Ct = a.Cm + (b * L + t) * kN;
+      const float* Bt = bcrow[buf] + i * 2 * kN;
+      const float* Ct = Bt + kN;
       float v[32];  // this channel's share of gB_t (0..15) and gC_t (16..31)
-      float gdl = 0.0f, gut = Dc * gyt;
+      // gdelta = sum_n g_n (A_n a_n h_{t-1},n + B_n u) = ln2 s_a + u s_b and
+      // gu = D gy + delta s_b, with s_a = sum_n g_n A2_n a_n h_{t-1},n, s_b = sum_n g_n B_n
+      float s_a = 0.0f, s_b = 0.0f;
       gD = fmaf(gyt, uv, gD);
 #pragma unroll
       for (int n = 0; n < kN; ++n) {
-        const float an = expf(dl * A[n]);
+        const float an = ex2f(dl * A2[n]);
         const float hp = i > 0 ? hs[i - 1][n][threadIdx.x] : hstart[n];
         const float ht = hs[i][n][threadIdx.x];
         g[n] = fmaf(Ct[n], gyt, g[n]);
         v[16 + n] = gyt * ht;
-        gut = fmaf(g[n], dl * Bt[n], gut);
+        s_b = fmaf(g[n], Bt[n], s_b);
         v[n] = g[n] * dl * uv;
-        gdl = fmaf(g[n], fmaf(A[n] * an, hp, Bt[n] * uv), gdl);
+        s_a = fmaf(g[n] * A2[n] * an, hp, s_a);
         gA[n] = fmaf(g[n] * dl * an, hp, gA[n]);
         g[n] *= an;
       }
+      const float gdl = fmaf(kLn2, s_a, uv * s_b);
+      const float gut = fmaf(dl, s_b, Dc * gyt);
       if (!cok) {
 #pragma unroll
         for (int q = 0; q < 32; ++q) v[q] = 0.0f;
@@ -308,6 +350,7 @@ __global__ void __launch_bounds__(kBwdThreads) k_scan_bwd(const BwdArgs a) {
       warp_reduce_scatter32(v, lane);
       a.part_bc[(tile_warp * (a.B * L) + b * L + t) * 32 + lane] = v[0];
     }
+    buf ^= 1;
   }
   if (cok) {
     const int64_t row = ((int64_t)p * a.B + b) * d + c;
