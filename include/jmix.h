@@ -224,6 +224,16 @@ jm_status jm_scan_bwd(const jm_dims* dims, const float* delta, const float* u, c
                       float* g_A_log, float* g_D, float* g_h0, void* workspace, size_t ws_bytes,
                       jm_stream_t stream);
 
+/* How jm_scan_bwd will cut each sequence into time parts for these dims:
+ * *n_parts parts (1..16) of whole 4-token chunks, at least 2 chunks each, that
+ * run side by side; each part folds the others' results in through exp(A S), S
+ * the part's sum of delta (both the state recurrence and its adjoint are linear
+ * with the same decays).  One part when the (128-channel tile, sequence) CTAs
+ * already fill at least 90% of their waves on a B200.  Depends only on the
+ * dims, like the workspace size.  Returns JM_ERR_INVALID_ARG for invalid dims or
+ * a NULL output, JM_ERR_UNSUPPORTED as jm_scan_bwd does. */
+jm_status jm_scan_bwd_schedule(const jm_dims* dims, int* n_parts);
+
 /* Failure-detection self-test: launches one thread that waits, through the
  * same bounded wait the pipelines use, on a barrier that nothing completes.
  * The wait gives up after its limit (2 s), records site 99 in workspace's

@@ -469,6 +469,17 @@ jm_status check_bwd_dims(const jm_dims* dm) {
 
 using namespace jmix;
 
+JM_API jm_status jm_scan_bwd_schedule(const jm_dims* dims, int* n_parts) {
+  if (!n_parts) {
+    set_error("jm_scan_bwd_schedule: NULL output pointer");
+    return JM_ERR_INVALID_ARG;
+  }
+  const jm_status st = check_bwd_dims(dims);
+  if (st != JM_OK) return st;
+  *n_parts = bwd_parts(dims->batch, dims->seqlen, dims->d_inner);
+  return JM_OK;
+}
+
 JM_API size_t jm_scan_bwd_workspace_size(const jm_dims* dims) {
   if (check_bwd_dims(dims) != JM_OK) return 0;
   return bwd_layout(dims->batch, dims->seqlen, dims->d_inner, nullptr).bytes;

@@ -28,7 +28,7 @@ EXPORTED = ("jm_mixer_fwd_workspace_size", "jm_mixer_step_workspace_size", "jm_m
             "jm_mixer_step_noalloc", "jm_mixer_fwd_schedule",
             "jm_mixer_fwd_varlen_workspace_size", "jm_mixer_fwd_varlen", "jm_selftest_timeout",
             "jm_layer_fwd_workspace_size", "jm_layer_fwd", "jm_scan_bwd_workspace_size",
-            "jm_scan_bwd")
+            "jm_scan_bwd", "jm_scan_bwd_schedule")
 
 
 class jm_dims(ctypes.Structure):
@@ -86,6 +86,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.jm_scan_bwd.argtypes = [ctypes.POINTER(jm_dims)] + [_vp] * 16 + [ctypes.c_size_t, _vp]
     lib.jm_selftest_timeout.restype = ctypes.c_int
     lib.jm_selftest_timeout.argtypes = [_vp, ctypes.c_size_t, _vp]
+    lib.jm_scan_bwd_schedule.restype = ctypes.c_int
+    lib.jm_scan_bwd_schedule.argtypes = [ctypes.POINTER(jm_dims), ctypes.POINTER(ctypes.c_int)]
     lib.jm_mixer_fwd_schedule.restype = ctypes.c_int
     lib.jm_mixer_fwd_schedule.argtypes = [ctypes.POINTER(jm_dims), ctypes.POINTER(ctypes.c_int),
                                           ctypes.POINTER(ctypes.c_int)]
@@ -144,6 +146,13 @@ def jm_mixer_fwd_schedule(d: jm_dims):
     n, t = ctypes.c_int(0), ctypes.c_int(0)
     _check(load().jm_mixer_fwd_schedule(ctypes.byref(d), ctypes.byref(n), ctypes.byref(t)))
     return n.value, bool(t.value)
+
+
+def jm_scan_bwd_schedule(d: jm_dims) -> int:
+    """Time parts per sequence that jm_scan_bwd uses for these dims."""
+    n = ctypes.c_int(0)
+    _check(load().jm_scan_bwd_schedule(ctypes.byref(d), ctypes.byref(n)))
+    return n.value
 
 
 def jm_mixer_step_workspace_size(d: jm_dims) -> int:

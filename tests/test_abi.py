@@ -165,6 +165,41 @@ def test_scan_schedule_rules(lib):
         jmix.jm_mixer_fwd_schedule(jmix.dims(1, 10, 100, 16))   # d % 8 != 0
 
 
+@pytest.mark.parametrize("B,L,d,want", [
+    (1, 4096, 8192, 13),   # 64 CTAs per part: 13 parts fill two waves of 444 slots to 94%
+    (8, 4096, 8192, 6),    # 512 CTAs per part: 6 parts, 3072 CTAs in 7 waves (99%)
+    (4, 4096, 8192, 5),
+    (1, 1000, 1024, 16),
+    (2, 301, 384, 16),     # 76 chunks: 16 ragged parts of 4-5 chunks
+    (2, 37, 200, 1),       # tiny: the folds cost more than the parallelism saves
+    (3, 4, 128, 1),        # one chunk
+    (1, 0, 8192, 1),       # empty sequences
+])
+def test_scan_bwd_schedule(lib, B, L, d, want):
+    assert jmix.jm_scan_bwd_schedule(jmix.dims(B, L, d, 8)) == want
+
+
+def test_scan_bwd_schedule_rules(lib):
+    """At most 16 parts of at least 2 four-token chunks; one part when the
+    (tile, sequence) CTAs already fill 90% of their waves (3 CTAs per SM on 148
+    SMs); with parts, the waves are at least as full as with one part."""
+    slots = 3 * 148
+    fill = lambda ctas: ctas / (-(-ctas // slots) * slots)
+    for B in (1, 2, 3, 8, 32, 300):
+        for L in (1, 4, 8, 9, 100, 1024, 4096):
+            for d in (64, 200, 1024, 8192):
+                n = jmix.jm_scan_bwd_schedule(jmix.dims(B, L, d, 8))
+                assert 1 <= n <= 16
+                chunks = -(-L // 4)
+                tiles = -(-d // 128)
+                if n > 1:
+                    assert chunks >= 2 * n
+                    assert fill(tiles * B) < 0.9
+                    assert fill(tiles * B * n) >= fill(tiles * B)
+    with pytest.raises(jmix.JmixError):
+        jmix.jm_scan_bwd_schedule(jmix.dims(1, 10, 128, 8, d_state=8))
+
+
 def test_varlen_host_checks(lib):
     FAKE = 1 << 40
     W = {k: FAKE for k in jmix.WEIGHT_NAMES}
