@@ -68,8 +68,13 @@ __device__ __forceinline__ float bf16_lane(const uint4& v, int e) {
   return __uint_as_float((e & 1) ? (wd & 0xffff0000u) : (wd << 16));
 }
 
-__device__ __forceinline__ __half to_half_sat(float v) {
-  return __float2half_rn(fminf(fmaxf(v, -65504.0f), 65504.0f));
+__device__ __forceinline__ float clamp_half(float v) { return fminf(fmaxf(v, -65504.0f), 65504.0f); }
+
+// Two floats to a packed fp16 pair (lo in the low 16 bits), each rounded to
+// nearest even: one paired conversion instead of two single ones.
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
 }
 
 // ------------------------------------------------------------------ conv + SiLU
@@ -144,6 +149,7 @@ __global__ void __launch_bounds__(256, JMIX_CONV_OCC) k_conv_silu16_packed(
     const uint4 bq = __ldg(reinterpret_cast<const uint4*>(conv_b + c0));
     uint32_t outp[G][4];
     if (inner) {
+      float sv_even[G];  // SiLU of the pair's even channel, per token
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         float xe[kW + G];
@@ -159,11 +165,11 @@ __global__ void __launch_bounds__(256, JMIX_CONV_OCC) k_conv_silu16_packed(
           float acc = be;
 #pragma unroll
           for (int k = 0; k < kConv; ++k) acc = fmaf(wk[k], xe[i + k], acc);
-          const uint32_t hb = (uint32_t)__half_as_ushort(to_half_sat(silu_u(acc)));
+          const float sv = clamp_half(silu_u(acc));
           if (e & 1)
-            outp[i][e >> 1] |= hb << 16;
+            outp[i][e >> 1] = pack_half2(sv_even[i], sv);
           else
-            outp[i][e >> 1] = hb;
+            sv_even[i] = sv;
         }
       }
     } else {
@@ -173,6 +179,7 @@ __global__ void __launch_bounds__(256, JMIX_CONV_OCC) k_conv_silu16_packed(
         int bi = lo;
         while (bi + 1 < B && __ldg(cu + bi + 1) <= t0 + i) ++bi;
         const int64_t sti = __ldg(cu + bi);
+        float sv_even = 0.0f;  // SiLU of the pair's even channel
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           float acc = bf16_lane(bq, e);
@@ -188,11 +195,11 @@ __global__ void __launch_bounds__(256, JMIX_CONV_OCC) k_conv_silu16_packed(
             }
             acc = fmaf(bf16_lane(wq[(e * kConv + k) >> 3], (e * kConv + k) & 7), v, acc);
           }
-          const uint32_t hb = (uint32_t)__half_as_ushort(to_half_sat(silu_u(acc)));
+          const float sv = clamp_half(silu_u(acc));
           if (e & 1)
-            outp[i][e >> 1] |= hb << 16;
+            outp[i][e >> 1] = pack_half2(sv_even, sv);
           else
-            outp[i][e >> 1] = hb;
+            sv_even = sv;
         }
       }
     }
@@ -218,10 +225,8 @@ __global__ void __launch_bounds__(256, JMIX_CONV_OCC) k_conv_silu16_packed(
   }
   float o[8];
   unpack8_bf16(__ldg(reinterpret_cast<const uint4*>(src) + i), o);
-  __align__(16) __half h[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) h[e] = __float2half_rn(o[e]);
-  reinterpret_cast<uint4*>(dst)[i] = *reinterpret_cast<uint4*>(h);
+  reinterpret_cast<uint4*>(dst)[i] = make_uint4(pack_half2(o[0], o[1]), pack_half2(o[2], o[3]),
+                                                pack_half2(o[4], o[5]), pack_half2(o[6], o[7]));
 }
 
 template <int kConvG>
@@ -258,6 +263,7 @@ __global__ void __launch_bounds__(256, JMIX_CONV_OCC) k_conv_silu16(
       wq[q] = __ldg(reinterpret_cast<const uint4*>(conv_w + c0 * kConv) + q);
     const uint4 bq = __ldg(reinterpret_cast<const uint4*>(conv_b + c0));
     uint32_t outp[kConvG][4];  // [token][channel pair] packed fp16x2
+    float sv_even[kConvG];     // SiLU of the pair's even channel, per token
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       float xe[kW + kConvG];
@@ -281,11 +287,11 @@ __global__ void __launch_bounds__(256, JMIX_CONV_OCC) k_conv_silu16(
         float acc = be;
 #pragma unroll
         for (int k = 0; k < kConv; ++k) acc = fmaf(wk[k], xe[i + k], acc);
-        const uint32_t hb = (uint32_t)__half_as_ushort(to_half_sat(silu_u(acc)));
+        const float sv = clamp_half(silu_u(acc));
         if (e & 1)
-          outp[i][e >> 1] |= hb << 16;
+          outp[i][e >> 1] = pack_half2(sv_even[i], sv);
         else
-          outp[i][e >> 1] = hb;
+          sv_even[i] = sv;
       }
     }
 #pragma unroll
@@ -310,10 +316,8 @@ __global__ void __launch_bounds__(256, JMIX_CONV_OCC) k_conv_silu16(
   }
   float o[8];
   unpack8_bf16(__ldg(reinterpret_cast<const uint4*>(src) + i), o);
-  __align__(16) __half h[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) h[j] = __float2half_rn(o[j]);
-  reinterpret_cast<uint4*>(dst)[i] = *reinterpret_cast<uint4*>(h);
+  reinterpret_cast<uint4*>(dst)[i] = make_uint4(pack_half2(o[0], o[1]), pack_half2(o[2], o[3]),
+                                                pack_half2(o[4], o[5]), pack_half2(o[6], o[7]));
 }
 
 // ------------------------------------------------------------------- x_proj
