@@ -399,7 +399,6 @@ JM_API jm_status jm_mixer_fwd_host(const jm_dims* dims, const void* x_host, cons
   jm_status st = check_dims(dims, false);
   if (st != JM_OK) return st;
   const size_t act = (size_t)dims->batch * dims->seqlen * dims->d_inner * esize(dims->io);
-  const size_t sst = (size_t)dims->batch * dims->d_inner * kN * 4;
   if (act && (!x_host || !z_host || !y_host)) {
     set_error("host buffers are required");
     return JM_ERR_INVALID_ARG;

@@ -216,7 +216,6 @@ __global__ void __launch_bounds__(kBwdThreads, 3) k_scan_bwd(const BwdArgs a) {
   const int64_t nck = (L + kCk - 1) / kCk;
   int64_t k0, k1;
   part_chunks(nck, P, p, k0, k1);
-  const int64_t t_begin = k0 * kCk, t_end = k1 * kCk < L ? k1 * kCk : L;
   float A2[kN];  // A log2(e)
 #pragma unroll
   for (int n = 0; n < kN; ++n) A2[n] = cok ? -expf(a.A_log[c * kN + n]) * kLog2e : 0.0f;
