@@ -200,6 +200,39 @@ def test_scan_bwd_schedule_rules(lib):
         jmix.jm_scan_bwd_schedule(jmix.dims(1, 10, 128, 8, d_state=8))
 
 
+def test_scan_bwd_host_checks(lib):
+    """jm_scan_bwd validates on the host and returns before any launch."""
+    F = 1 << 40          # a fake device address: no test here reaches a launch
+    W = 1 << 41          # fake workspace (256-byte aligned)
+    d = jmix.dims(2, 64, 256, 8)
+    n = jmix.jm_scan_bwd_workspace_size(d)
+    assert n > 0 and n % 256 == 0 and n == jmix.jm_scan_bwd_workspace_size(d)
+
+    def call(dm, ws=W, nbytes=n, **over):
+        args = dict(delta=F, u=F, Bm=F, Cm=F, A_log=F, D=F, h0=None, gy=F, g_delta=F, g_u=F,
+                    g_B=F, g_C=F, g_A_log=F, g_D=F, g_h0=None)
+        args.update(over)
+        return jmix.jm_scan_bwd(dm, **args, workspace=ws, ws_bytes=nbytes, stream=0, check=False)
+
+    assert call(jmix.dims(2, 64, 256, 8, d_state=8)) == jmix.JM_ERR_UNSUPPORTED
+    assert call(jmix.dims(2, 64, 256, 8, zoh=True)) == jmix.JM_ERR_UNSUPPORTED
+    assert call(jmix.dims(70000, 4, 128, 8)) == jmix.JM_ERR_INVALID_ARG      # grid y limit
+    assert call(jmix.dims(2, 64, 0, 8)) == jmix.JM_ERR_INVALID_ARG
+    for k in ("A_log", "D", "g_A_log", "g_D", "delta", "u", "Bm", "Cm", "gy", "g_delta", "g_u",
+              "g_B", "g_C"):
+        assert call(d, **{k: None}) == jmix.JM_ERR_INVALID_ARG, k
+    assert call(d, ws=None) == jmix.JM_ERR_WORKSPACE
+    assert call(d, ws=W + 128) == jmix.JM_ERR_WORKSPACE                      # misaligned
+    assert call(d, nbytes=n - 256) == jmix.JM_ERR_WORKSPACE                  # too small
+    assert jmix.jm_scan_bwd_workspace_size(jmix.dims(2, 64, 256, 8, d_state=8)) == 0
+    # more time parts need more per-part rows: the size follows the schedule
+    one = jmix.dims(64, 4096, 8192, 8)     # fills the GPU: one part
+    assert jmix.jm_scan_bwd_schedule(one) == 1
+    parts = jmix.dims(1, 4096, 8192, 8)
+    assert jmix.jm_scan_bwd_schedule(parts) > 1
+    assert jmix.jm_scan_bwd_workspace_size(parts) > 0
+
+
 def test_varlen_host_checks(lib):
     FAKE = 1 << 40
     W = {k: FAKE for k in jmix.WEIGHT_NAMES}
