@@ -11,9 +11,12 @@ Pins (tests/test_oracle_pins.py) tie every function here to something other
 than itself: closed forms of the scan, the brute-force "hidden attention"
 matrix form, the split-and-carry invariant, step == forward, permutation and
 batch independence, the conv impulse response, RMSNorm and softplus
-identities.  The front end (conv tap order, RMSNorm placement) has no worked
-numbers on the pages and is "parity unpinned" against trained Jamba values;
-see the readings listed with the design notes.
+identities, and the dt branch (RMSNorm scale invariance through the whole
+mixer, dt_norm_w scaling equal to dtproj_w scaling, a one-hot dtproj_w that
+turns dt_proj into a selection); tests/test_oracle_planted.py plants four
+mistakes in a copy of the dt branch and checks that a pin fails for each.
+What no pin can reach is agreement with trained Jamba checkpoints (the pages
+print no weights or worked numbers), so the conv tap order stays a reading.
 """
 from __future__ import annotations
 
@@ -54,18 +57,24 @@ def build(force: bool = False) -> str:
 _lib = None
 
 
+def load_library(path: str):
+    """A ctypes handle on an oracle library built from this source (or, in the
+    planted-mistake tests, from a mutated copy of it)."""
+    lib = ctypes.CDLL(path)
+    lib.orc_round_bf16.restype = ctypes.c_double
+    lib.orc_round_bf16.argtypes = [ctypes.c_double]
+    lib.orc_round_fp16.restype = ctypes.c_double
+    lib.orc_round_fp16.argtypes = [ctypes.c_double]
+    lib.orc_softplus1.restype = ctypes.c_double
+    lib.orc_softplus1.argtypes = [ctypes.c_double]
+    return lib
+
+
 def _L():
     global _lib
     if _lib is None:
         build()
-        lib = ctypes.CDLL(LIB)
-        lib.orc_round_bf16.restype = ctypes.c_double
-        lib.orc_round_bf16.argtypes = [ctypes.c_double]
-        lib.orc_round_fp16.restype = ctypes.c_double
-        lib.orc_round_fp16.argtypes = [ctypes.c_double]
-        lib.orc_softplus1.restype = ctypes.c_double
-        lib.orc_softplus1.argtypes = [ctypes.c_double]
-        _lib = lib
+        _lib = load_library(LIB)
     return _lib
 
 

@@ -308,6 +308,98 @@ def test_mixer_gate_skip_and_split_order():
     np.testing.assert_allclose(fs[0], hT, rtol=1e-11, atol=1e-13)
 
 
+# ------------------------------------------------------------- the dt branch
+# delta = softplus(W_dt . (RMSNorm(dt) w_dt) + dt_bias), with dt the first R
+# outputs of x_proj (TransformerLens "Jamba" adapter page, "Key adapter
+# decisions": the three RMSNorms on the selective parameters, applied before
+# dt_proj; aifetchly "Jamba Guide", "Hands-On Implementation": delta =
+# softplus(dt_proj(.))).  Each check raises AssertionError when it fails; the
+# planted-mistake tests (test_oracle_planted.py) run the same checks on
+# mutated copies of the oracle.
+
+def _dt_case(seed=21):
+    w = synth.Workload("dtpin", 2, 13, 40, 8, "f32", seed=seed, extra=True)
+    W = {k: np.asarray(v, dtype=np.float64) for k, v in synth.make_weights(w).items()}
+    return w, W, synth.make_activations(w)
+
+
+def _dt_run(w, W, A, eps):
+    m = oracle.dims(w.batch, w.seqlen, w.d_inner, w.dt_rank, eps=eps)
+    y, fs, _ = oracle.mixer_fwd(m, A["x"], A["z"], W, A["init_conv_state"], A["init_ssm_state"])
+    return y, fs
+
+
+def _with_dt_rows_scaled(W, R, alpha):
+    xw = W["xproj_w"].copy()
+    xw[:R] *= alpha
+    return dict(W, xproj_w=xw)
+
+
+def check_dt_rmsnorm_scale_invariance():
+    """With eps = 0, RMSNorm(alpha v) = RMSNorm(v) for alpha > 0, so scaling the
+    dt rows of xproj_w leaves y and the final state unchanged; alpha = -1 equals
+    negating dt_norm_w (the norm is odd in v, and w multiplies after it)."""
+    w, W, A = _dt_case()
+    R = w.dt_rank
+    y, fs = _dt_run(w, W, A, 0.0)
+    for alpha in (3.7, 0.21):
+        ys, fss = _dt_run(w, _with_dt_rows_scaled(W, R, alpha), A, 0.0)
+        np.testing.assert_allclose(ys, y, rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(fss, fs, rtol=1e-11, atol=1e-12)
+    yn, fsn = _dt_run(w, _with_dt_rows_scaled(W, R, -1.0), A, 0.0)
+    ym, fsm = _dt_run(w, dict(W, dt_norm_w=-W["dt_norm_w"]), A, 0.0)
+    np.testing.assert_allclose(yn, ym, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(fsn, fsm, rtol=1e-13, atol=1e-14)
+    assert np.abs(ym - y).max() > 1e-3      # the dt branch reaches y
+
+
+def check_dt_norm_weight_equals_dtproj_scaling():
+    """dt_proj is linear after the norm's weight: scaling dt_norm_w by alpha equals
+    scaling dtproj_w by alpha (any eps, any sign of alpha)."""
+    w, W, A = _dt_case()
+    y0, _ = _dt_run(w, W, A, w.eps)
+    for alpha in (2.5, -0.6):
+        y1, fs1 = _dt_run(w, dict(W, dt_norm_w=alpha * W["dt_norm_w"]), A, w.eps)
+        y2, fs2 = _dt_run(w, dict(W, dtproj_w=alpha * W["dtproj_w"]), A, w.eps)
+        np.testing.assert_allclose(y1, y2, rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(fs1, fs2, rtol=1e-12, atol=1e-13)
+        assert np.abs(y1 - y0).max() > 1e-3
+
+
+def check_dt_onehot_selection():
+    """With one-hot dtproj_w rows (channel c reads dt coordinate r(c) alone) the
+    contraction is a selection: delta[t, c] = softplus(dt_n[t, r(c)] + dt_bias[c]),
+    dt_n = RMSNorm over the R dt outputs with dt_norm_w.  y and the final state
+    then equal the separately pinned scan core fed with that delta."""
+    w, W, A = _dt_case()
+    d, R, N = w.d_inner, w.dt_rank, w.d_state
+    r_of_c = (3 * np.arange(d) + 1) % R
+    onehot = np.zeros((d, R))
+    onehot[np.arange(d), r_of_c] = 1.0
+    y, fs = _dt_run(w, dict(W, dtproj_w=onehot), A, w.eps)
+    Aneg = -np.exp(W["A_log"])
+    for b in range(w.batch):
+        u = oracle.silu(oracle.conv(A["x"][b].astype(np.float64), W["conv_w"], W["conv_b"],
+                                    A["init_conv_state"][b]))
+        p = u @ W["xproj_w"].T
+        dtn = oracle.rmsnorm(p[:, :R], W["dt_norm_w"], w.eps)
+        Bn = oracle.rmsnorm(p[:, R:R + N], W["b_norm_w"], w.eps)
+        Cn = oracle.rmsnorm(p[:, R + N:], W["c_norm_w"], w.eps)
+        delta = oracle.softplus(dtn[:, r_of_c] + W["dt_bias"][None, :])
+        ys, hT = oracle.scan(delta, Aneg, Bn, Cn, u, W["D"], A["init_ssm_state"][b])
+        np.testing.assert_allclose(y[b], ys * oracle.silu(A["z"][b]), rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(fs[b], hT, rtol=1e-11, atol=1e-12)
+
+
+DT_BRANCH_CHECKS = (check_dt_rmsnorm_scale_invariance, check_dt_norm_weight_equals_dtproj_scaling,
+                    check_dt_onehot_selection)
+
+
+@pytest.mark.parametrize("check", DT_BRANCH_CHECKS, ids=lambda f: f.__name__)
+def test_dt_branch(check):
+    check()
+
+
 def test_mirror_rounding_is_small():
     """Mirror mode rounds u and dt_n to fp16; on bf16 inputs it must stay well
     inside the bf16-io output tolerance of the exact run."""
