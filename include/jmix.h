@@ -144,14 +144,28 @@ jm_status jm_mixer_step(const jm_dims* dims, const void* x_t, const void* z_t, v
  * cleared, so the previous call's contents never leak into a result; but two
  * calls whose kernels overlap on the GPU (different streams, or different
  * host threads on one device) race on the array and must be serialised by the
- * caller.  jm_poll_error does not apply (there is no caller workspace); launch
- * errors are returned as JM_ERR_CUDA. */
+ * caller.  Launch errors are returned as JM_ERR_CUDA; device-side flags (a
+ * bounded wait that ran out) are read with jm_noalloc_poll_error, since
+ * jm_poll_error needs a caller workspace. */
 jm_status jm_mixer_step_noalloc(const jm_dims* dims, const void* x_t, const void* z_t,
                                 void* conv_state, float* ssm_state, const void* conv_w,
                                 const void* conv_b, const void* xproj_w, const void* dt_norm_w,
                                 const void* b_norm_w, const void* c_norm_w,
                                 const void* dtproj_w, const float* dt_bias, const float* A_log,
                                 const float* D, void* y_t, jm_stream_t stream);
+
+/* jm_poll_error for jm_mixer_step_noalloc: synchronises `stream`, then reads
+ * the error flags that the steps write into the header of the static array on
+ * the current device.  JM_ERR_TIMEOUT if a bounded device-side wait ran out
+ * since the last jm_mixer_step_noalloc on this device (each step clears the
+ * flags), JM_ERR_CUDA if the stream reports an error, JM_OK otherwise.
+ * Allocates nothing. */
+jm_status jm_noalloc_poll_error(jm_stream_t stream);
+
+/* The failure-detection self-test (see jm_selftest_timeout) aimed at the static
+ * array's error header: a following jm_noalloc_poll_error returns
+ * JM_ERR_TIMEOUT.  The same sharing rules as jm_mixer_step_noalloc apply. */
+jm_status jm_noalloc_selftest_timeout(jm_stream_t stream);
 
 /* End-to-end forward from HOST buffers: copies x_host and z_host (pinned host
  * memory, [B, L, d] io dtype) into the caller's device buffers x_dev / z_dev,

@@ -154,6 +154,22 @@ jm_status check_ws(const Problem& p, void* ws, size_t ws_bytes) {
   return JM_OK;
 }
 
+}  // namespace
+
+jm_status status_of_flags(const ErrFlags& f) {
+  if (f.timeout) {
+    set_error("a bounded device-side wait ran out (site %u)", f.where);
+    return JM_ERR_TIMEOUT;
+  }
+  if (f.bad_input) {
+    set_error("cu_seqlens is not 0 = c[0] <= c[1] <= ... <= c[B] = total tokens");
+    return JM_ERR_INVALID_ARG;
+  }
+  return JM_OK;
+}
+
+namespace {
+
 jm_status finish(Problem& p, cudaError_t e) {
   if (e != cudaSuccess) {
     set_error("CUDA error: %s", cudaGetErrorString(e));
@@ -508,15 +524,7 @@ JM_API jm_status jm_poll_error(void* workspace, jm_stream_t stream) {
     set_error("CUDA error: %s", cudaGetErrorString(e));
     return JM_ERR_CUDA;
   }
-  if (f.timeout) {
-    set_error("a bounded device-side wait ran out (site %u)", f.where);
-    return JM_ERR_TIMEOUT;
-  }
-  if (f.bad_input) {
-    set_error("cu_seqlens is not 0 = c[0] <= c[1] <= ... <= c[B] = total tokens");
-    return JM_ERR_INVALID_ARG;
-  }
-  return JM_OK;
+  return status_of_flags(f);
 }
 
 JM_API const char* jm_last_error(void) { return g_msg; }

@@ -66,7 +66,7 @@ constexpr int kMaxLaunches = 16;
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
-// The portable SIMT path (any io dtype; the only path for float32 io).
+// The SIMT path of float32 io.
 size_t simple_ws_bytes(const Problem& p);
 cudaError_t run_simple(Problem& p);
 
@@ -78,5 +78,14 @@ cudaError_t run_fast(Problem& p);
 
 // Per-thread message for jm_last_error.
 void set_error(const char* fmt, ...);
+
+// Status of an error header read back to the host (JM_OK when no flag is set;
+// sets the message otherwise).
+jm_status status_of_flags(const ErrFlags& f);
+
+// Launches the failure-detection self-test on `err` (cleared first): one
+// thread waits, bounded, on a barrier that nothing completes, then records its
+// site in *err and returns.
+cudaError_t launch_wait_never(ErrFlags* err, cudaStream_t s);
 
 }  // namespace jmix

@@ -87,3 +87,41 @@ JM_API jm_status jm_mixer_step_noalloc(const jm_dims* dims, const void* x_t, con
                        b_norm_w, c_norm_w, dtproj_w, dt_bias, A_log, D, y_t, scratch,
                        kStepScratchBytes, stream);
 }
+
+// The device-side error flags of jm_mixer_step_noalloc live in the first 256
+// bytes of the static array, where a caller cannot reach them; this reads them
+// back (one device-to-host copy into a host struct, no allocation).
+JM_API jm_status jm_noalloc_poll_error(jm_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    set_error("CUDA error: %s", cudaGetErrorString(e));
+    return JM_ERR_CUDA;
+  }
+  void* scratch = nullptr;
+  jm_status st = scratch_for_current_device(&scratch);
+  if (st != JM_OK) return st;
+  ErrFlags f;
+  e = cudaMemcpyAsync(&f, scratch, sizeof(f), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    set_error("CUDA error: %s", cudaGetErrorString(e));
+    return JM_ERR_CUDA;
+  }
+  return status_of_flags(f);
+}
+
+// The failure-detection self-test aimed at the static array's error header, so
+// that the report path of jm_noalloc_poll_error can be checked without a fault.
+JM_API jm_status jm_noalloc_selftest_timeout(jm_stream_t stream) {
+  void* scratch = nullptr;
+  jm_status st = scratch_for_current_device(&scratch);
+  if (st != JM_OK) return st;
+  const cudaError_t e =
+      launch_wait_never(static_cast<ErrFlags*>(scratch), reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    set_error("CUDA error: %s", cudaGetErrorString(e));
+    return JM_ERR_CUDA;
+  }
+  return JM_OK;
+}

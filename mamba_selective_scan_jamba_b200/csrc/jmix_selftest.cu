@@ -26,6 +26,14 @@ __global__ void k_wait_never(ErrFlags* err) {
 }
 
 }  // namespace
+
+cudaError_t launch_wait_never(ErrFlags* err, cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(err, 0, sizeof(ErrFlags), s);
+  if (e != cudaSuccess) return e;
+  k_wait_never<<<1, 32, 0, s>>>(err);
+  return cudaGetLastError();
+}
+
 }  // namespace jmix
 
 using namespace jmix;
@@ -35,12 +43,8 @@ JM_API jm_status jm_selftest_timeout(void* workspace, size_t ws_bytes, jm_stream
     set_error("jm_selftest_timeout: needs a workspace of at least %zu bytes", sizeof(ErrFlags));
     return JM_ERR_WORKSPACE;
   }
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = cudaMemsetAsync(workspace, 0, sizeof(ErrFlags), s);
-  if (e == cudaSuccess) {
-    k_wait_never<<<1, 32, 0, s>>>(static_cast<ErrFlags*>(workspace));
-    e = cudaGetLastError();
-  }
+  const cudaError_t e = launch_wait_never(static_cast<ErrFlags*>(workspace),
+                                          reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {
     set_error("CUDA error: %s", cudaGetErrorString(e));
     return JM_ERR_CUDA;

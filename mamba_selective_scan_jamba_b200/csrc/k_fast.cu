@@ -27,6 +27,8 @@
 #include <cuda.h>
 #include <cuda_fp16.h>
 
+#include <atomic>
+
 #include "jmix_internal.cuh"
 #include "poly_consts.cuh"
 #include "sm100.cuh"
@@ -1523,13 +1525,18 @@ FastWs fast_layout(const Problem& pr, char* base) {
   return w;
 }
 
+// SM count of the current device, cached per device (threads that race on a
+// slot store the same value).
 int num_sms() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
+  constexpr int kMaxDev = 64;
+  static std::atomic<int> cache[kMaxDev];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) dev = 0;
+  int n = dev < kMaxDev ? cache[dev].load(std::memory_order_relaxed) : 0;
+  if (n <= 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    if (dev < kMaxDev) cache[dev].store(n, std::memory_order_relaxed);
   }
   return n;
 }

@@ -1,10 +1,7 @@
-// The portable SIMT path of the mixer core: one kernel per step, float32
-// arithmetic throughout, intermediates in the workspace as float32.
-//
-// It is the only path for float32 io (TF32 tensor cores cannot meet a 1e-4
-// tolerance) and serves any io dtype.  In bf16 mode it rounds where the
-// tensor-core path quantises: u to fp16 as the x_proj operand and dt_n to fp16
-// as the dt_proj operand (the scan keeps the float32 u).
+// The float32-io path of the mixer core: SIMT kernels, one per step, float32
+// arithmetic throughout, intermediates in the workspace as float32.  TF32
+// tensor cores cannot meet the 1e-4 float32 tolerance, so both contractions run
+// as FFMA GEMMs here.  (bf16 io always takes the tensor-core path.)
 //
 // Steps (TransformerLens "Jamba" adapter page for the pipeline; aifetchly
 // "Jamba Guide", "Inside the Mamba State-Space Layers", for the scan):
@@ -14,18 +11,13 @@
 //   k_gemm_nt       delta = softplus(dt_n . dtproj_w^T + dt_bias)   (dt_proj)
 //   k_scan_simple   h, y (one thread per (sequence, channel), 16 states)
 //   k_final_conv    final conv state
-#include <cuda_fp16.h>
-
 #include "jmix_internal.cuh"
 
 namespace jmix {
 namespace {
 
 __device__ __forceinline__ float ld(const float* p) { return *p; }
-__device__ __forceinline__ float ld(const __nv_bfloat16* p) { return __bfloat162float(*p); }
 __device__ __forceinline__ void st(float* p, float v) { *p = v; }
-__device__ __forceinline__ void st(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
-__device__ __forceinline__ float to_fp16_value(float v) { return __half2float(__float2half_rn(v)); }
 
 __device__ __forceinline__ float silu_precise(float v) { return v / (1.0f + expf(-v)); }
 
@@ -60,7 +52,7 @@ __global__ void k_conv_silu(const T* __restrict__ x, const T* __restrict__ conv_
 // Tile 32 (m) x 32 (n), k-step 32, 256 threads, 4 outputs per thread.
 template <typename T, int EPI>
 __global__ void k_gemm_nt(const float* __restrict__ A, const T* __restrict__ W, int64_t M,
-                          int64_t N, int64_t K, const float* __restrict__ bias, int round_a,
+                          int64_t N, int64_t K, const float* __restrict__ bias,
                           float* __restrict__ out) {
   __shared__ float As[32][33];
   __shared__ float Ws[32][33];
@@ -72,8 +64,7 @@ __global__ void k_gemm_nt(const float* __restrict__ A, const T* __restrict__ W, 
     for (int i = 0; i < 4; ++i) {
       int r = ty + 8 * i;
       int64_t m = m0 + r, n = n0 + r, k = k0 + tx;
-      const float av = (m < M && k < K) ? A[m * K + k] : 0.0f;
-      As[r][tx] = round_a ? to_fp16_value(av) : av;
+      As[r][tx] = (m < M && k < K) ? A[m * K + k] : 0.0f;
       Ws[r][tx] = (n < N && k < K) ? ld(W + n * K + k) : 0.0f;
     }
     __syncthreads();
@@ -217,7 +208,6 @@ template <typename T>
 cudaError_t run_simple_t(Problem& p) {
   SimpleWs w = simple_layout(p, p.ws);
   cudaStream_t s = p.stream;
-  const int round = p.io == JM_BF16 ? 1 : 0;
   const int64_t td = p.T * p.d;
   cudaMemsetAsync(p.ws, 0, sizeof(ErrFlags), s);
   launches_begin(p);
@@ -226,14 +216,14 @@ cudaError_t run_simple_t(Problem& p) {
       w.u);
   launched(p, "k_conv_silu");
   k_gemm_nt<T, 0><<<dim3((unsigned)((p.P + 31) / 32), (unsigned)((p.T + 31) / 32)), 256, 0, s>>>(
-      w.u, (const T*)p.xproj_w, p.T, p.P, p.d, nullptr, round, w.p);
+      w.u, (const T*)p.xproj_w, p.T, p.P, p.d, nullptr, w.p);
   launched(p, "k_gemm_nt(x_proj)");
   k_norms<T><<<(unsigned)((p.T + 7) / 8), 256, 0, s>>>(w.p, (const T*)p.dtn_w, (const T*)p.bn_w,
                                                         (const T*)p.cn_w, p.T, (int)p.R, p.eps,
                                                         w.dtn, w.Bn, w.Cn);
   launched(p, "k_norms");
   k_gemm_nt<T, 1><<<dim3((unsigned)((p.d + 31) / 32), (unsigned)((p.T + 31) / 32)), 256, 0, s>>>(
-      w.dtn, (const T*)p.dtproj_w, p.T, p.d, p.R, p.dt_bias, round, w.delta);
+      w.dtn, (const T*)p.dtproj_w, p.T, p.d, p.R, p.dt_bias, w.delta);
   launched(p, "k_gemm_nt(dt_proj)");
   k_scan_simple<T><<<dim3((unsigned)((p.d + 127) / 128), (unsigned)p.B), 128, 0, s>>>(
       w.delta, w.u, w.Bn, w.Cn, (const T*)p.z, p.A_log, p.D, p.init_ssm, p.final_state, (T*)p.y,
@@ -252,8 +242,6 @@ cudaError_t run_simple_t(Problem& p) {
 
 size_t simple_ws_bytes(const Problem& p) { return simple_layout(p, nullptr).bytes; }
 
-cudaError_t run_simple(Problem& p) {
-  return p.io == JM_BF16 ? run_simple_t<__nv_bfloat16>(p) : run_simple_t<float>(p);
-}
+cudaError_t run_simple(Problem& p) { return run_simple_t<float>(p); }
 
 }  // namespace jmix

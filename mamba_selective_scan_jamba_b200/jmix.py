@@ -28,7 +28,8 @@ EXPORTED = ("jm_mixer_fwd_workspace_size", "jm_mixer_step_workspace_size", "jm_m
             "jm_mixer_step_noalloc", "jm_mixer_fwd_schedule",
             "jm_mixer_fwd_varlen_workspace_size", "jm_mixer_fwd_varlen", "jm_selftest_timeout",
             "jm_layer_fwd_workspace_size", "jm_layer_fwd", "jm_scan_bwd_workspace_size",
-            "jm_scan_bwd", "jm_scan_bwd_schedule")
+            "jm_scan_bwd", "jm_scan_bwd_schedule", "jm_noalloc_poll_error",
+            "jm_noalloc_selftest_timeout")
 
 
 class jm_dims(ctypes.Structure):
@@ -93,6 +94,10 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
                                           ctypes.POINTER(ctypes.c_int)]
     lib.jm_poll_error.restype = ctypes.c_int
     lib.jm_poll_error.argtypes = [_vp, _vp]
+    lib.jm_noalloc_poll_error.restype = ctypes.c_int
+    lib.jm_noalloc_poll_error.argtypes = [_vp]
+    lib.jm_noalloc_selftest_timeout.restype = ctypes.c_int
+    lib.jm_noalloc_selftest_timeout.argtypes = [_vp]
     lib.jm_last_error.restype = ctypes.c_char_p
     lib.jm_last_error.argtypes = []
     lib.jm_last_launch_count.restype = ctypes.c_int
@@ -269,6 +274,17 @@ def jm_mixer_fwd_host(d: jm_dims, x_host, z_host, y_host, final_state_host, x_de
 
 def jm_poll_error(workspace, stream=None) -> int:
     return load().jm_poll_error(_ptr(workspace), _stream(stream))
+
+
+def jm_noalloc_poll_error(stream=None) -> int:
+    return load().jm_noalloc_poll_error(_stream(stream))
+
+
+def jm_noalloc_selftest_timeout(stream=None, check: bool = True) -> int:
+    st = load().jm_noalloc_selftest_timeout(_stream(stream))
+    if check:
+        _check(st)
+    return st
 
 
 def jm_last_error() -> str:

@@ -255,26 +255,47 @@ def test_decode_step_matches_forward():
 
 # ------------------------------------------------------------- full sizes
 FULL_CH = [0, 1, 127, 128, 1000, 4095, 4096, 5555, 8064, 8191]
+# lanes at both ends and both sides of the middle of a warp
+LANES = (0, 1, 15, 16, 30, 31)
+
+
+def tile_channels(tiles, lanes=LANES, warps=(0, 1, 2, 3)):
+    """Channels of the given 128-channel tiles that sit at the given lanes of the
+    given warps (a thread of the scan and decode kernels owns one channel: warp w,
+    lane l of tile k is channel 128 k + 32 w + l)."""
+    return sorted(128 * k + 32 * w + l for k in tiles for w in warps for l in lanes)
+
+
+def test_tile_channels_cover_every_warp_and_lane_class():
+    ch = tile_channels((0, 17, 40, 63))
+    assert len(ch) == 96 and ch[0] == 0 and ch[-1] == 8191
+    assert {(c % 128) // 32 for c in ch} == {0, 1, 2, 3}
+    assert {c % 32 for c in ch} == set(LANES)
+    assert len({c // 128 for c in ch}) == 4
 
 
 @pytest.mark.slow
 def test_full_jamba_b1_l4096():
-    check_fwd(synth.WORKLOADS["jamba_b1_l4096"], channels=FULL_CH)
+    check_fwd(synth.WORKLOADS["jamba_b1_l4096"], channels=tile_channels((0, 21, 42, 63)))
 
 
 @pytest.mark.slow
 def test_full_jamba_b8_l4096():
-    check_fwd(synth.WORKLOADS["jamba_b8_l4096"], channels=FULL_CH[::3])
+    """All 8 sequences, 96 channels: every compute warp of the scan CTA and lanes
+    0, 1, 15, 16, 30, 31 in four channel tiles, under the chained 4-part schedule."""
+    check_fwd(synth.WORKLOADS["jamba_b8_l4096"], channels=tile_channels((0, 17, 40, 63)))
 
 
 @pytest.mark.slow
 def test_full_jamba_b1_l262144():
-    check_fwd(synth.WORKLOADS["jamba_b1_l262144"], channels=[0, 3333, 8191])
+    check_fwd(synth.WORKLOADS["jamba_b1_l262144"],
+              channels=tile_channels((0, 63), lanes=(0, 31)))
 
 
 @pytest.mark.slow
 def test_full_decode_b256_64_steps():
-    run_decode(synth.WORKLOADS["jamba_decode_b256"], 64, channels=FULL_CH)
+    run_decode(synth.WORKLOADS["jamba_decode_b256"], 64,
+               channels=tile_channels((0, 31, 63), lanes=(0, 15, 16, 31)))
 
 
 # ------------------------------------------------ zero-order hold of B (variant)
