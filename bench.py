@@ -35,6 +35,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
+from mamba_selective_scan_jamba_b200.clocks import ClockSampler, gpu_id_of  # noqa: E402
+
 METRIC = "Mamba-mixer tokens/sec at Jamba shapes (d_inner 8192, N 16) and % of roofline"
 L2_BYTES = 126 * 1024 * 1024
 
@@ -115,74 +117,45 @@ def nvtx_pop() -> None:
         pass
 
 
-def measured_traffic(kernel: str, tokens: int):
-    """DRAM bytes of one launch of `kernel` over `tokens` tokens, from the committed
-    ncu summary of that kernel (bytes per token x tokens), if the kernel source is
-    unchanged since the capture; else (None, None)."""
+TRAFFIC_JSON = os.path.join(HERE, "profiles", "traffic.json")
+PIPES_JSON = os.path.join(HERE, "profiles", "pipe_rates_b200.json")
+
+
+def kernel_source_sha() -> str:
     src = os.path.join(HERE, "mamba_selective_scan_jamba_b200", "csrc", "k_fast.cu")
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
-    pat = re.compile(r"<!-- traffic: kernel=(\S+) bytes_per_token=(\d+) source_sha256=(\w+) -->")
-    for path in sorted(glob.glob(os.path.join(HERE, "profiles", f"{kernel}_*.md"))):
+    with open(src, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def measured_traffic(kernel: str, tokens: int, path: str = TRAFFIC_JSON):
+    """DRAM bytes of one launch of `kernel` over `tokens` tokens from the committed
+    ncu record (profiles/traffic.json: bytes per token of a capture, scaled by the
+    tokens of this launch), if the kernel source is unchanged since the capture;
+    else (None, None)."""
+    try:
         with open(path) as f:
-            m = pat.search(f.read())
-        if m and m.group(1) == kernel and m.group(3) == sha:
-            return int(m.group(2)) * tokens, os.path.basename(path)
-    return None, None
+            rec = json.load(f).get(kernel)
+    except (OSError, ValueError):
+        return None, None
+    if not rec or rec.get("source_sha256") != kernel_source_sha():
+        return None, None
+    return int(round(rec["bytes_per_token"] * tokens)), rec
 
 
-# ------------------------------------------------------------------- clocks
-class ClockSampler:
-    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
-
-    def __init__(self, gpu_id: str):
-        self.proc = None
-        self.lines = []
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100", "-i", gpu_id], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
-                text=True)
-        except Exception:
-            self.proc = None
-
-    def stop(self):
-        if self.proc is None:
-            return
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=5)
-        except Exception:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
-        self.lines = [l for l in out.splitlines() if l.strip()]
-
-    def summary(self, t0: float, t1: float):
-        import datetime
-        rows = []
-        for l in self.lines:
-            f = [x.strip() for x in l.split(",")]
-            if len(f) < 10:
-                continue
-            try:
-                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
-                rows.append((ts, float(f[2]), float(f[3]), f[4], f[5:]))
-            except Exception:
-                continue
-        inside = [r for r in rows if t0 - 0.05 <= r[0] <= t1 + 0.05] or rows
-        if not inside:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
-        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
-                 "sw_power_cap"]
-        reasons = set()
-        for r in inside:
-            for n, v in zip(names[1:], r[4][1:]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(r[1] for r in inside),
-                "sm_max_mhz": max(r[2] for r in inside), "reasons": sorted(reasons),
-                "samples": len(inside)}
+def alu_peak(P):
+    """(ex2 per second, where it comes from): the measured MUFU ex2 rate of the
+    committed pipe-rate record, else the nominal 16 per clock per SM at the
+    maximum clock (said so in the source string)."""
+    try:
+        with open(PIPES_JSON) as f:
+            rec = json.load(f)
+        rate = float(rec["rates"]["ex2"]["ops_per_s"])
+        mhz = rec.get("clocks", {}).get("sm_mhz")
+        return rate, (f"measured: profiles/pipe_rates_b200.json (ex2.approx on all SMs, "
+                      f"SM clock {mhz} MHz)")
+    except (OSError, ValueError, KeyError, TypeError):
+        return 16 * 148 * P["sm_max"] * 1e6, (f"nominal: 16 ex2/clk/SM x 148 SMs x "
+                                              f"{P['sm_max']:.0f} MHz (no measured record)")
 
 
 # ------------------------------------------------------------------ decode
@@ -229,11 +202,14 @@ def decode_bench(dev, stream, steps: int = 64, warmup: int = 5, zoh: bool = Fals
     ms = a.elapsed_time(b) / steps
     per = {names[k]: round(sum(evs[i][k].elapsed_time(evs[i][k + 1]) for i in range(steps))
                            / steps * 1e3, 2) for k in range(nk)}
-    # algorithmic bytes per step: ssm state r+w, conv state r+w, x_t, z_t, y_t
+    # algorithmic bytes per step: ssm state r+w, conv state r+w, x_t, z_t, y_t, and
+    # every weight read once
     B, dd, N = w.batch, w.d_inner, w.d_state
-    nbytes = B * dd * (N * 4 * 2 + 3 * 2 * 2 + 2 * 3)
+    wbytes = sum(int(v.nbytes) for v in W.values())
+    nbytes = B * dd * (N * 4 * 2 + 3 * 2 * 2 + 2 * 3) + wbytes
     return {"workload": w.name, "batch": B, "steps": steps, "us_per_step": ms * 1e3,
             "tokens_per_s": B / (ms / 1e3), "algorithmic_bytes_per_step": nbytes,
+            "weight_bytes_per_step": wbytes,
             "achieved_GBps": nbytes / (ms / 1e3) / 1e9, "kernels_us": per,
             "launches_per_step": nk}
 
@@ -390,6 +366,63 @@ def bwd_bench(dev, stream, B: int = 1, L: int = 4096, d: int = 8192, steps: int 
             "data": "synthetic (torch generator, seed 7)"}
 
 
+def roofline_block(P, w, names, per_kernel_ms, tok_s, tokens):
+    """The roofline object of the JSON line.  Top level: the whole step against
+    the stated roofline, max(projection FLOPs / bf16 peak, x,z,y bytes / HBM) per
+    token; at Jamba shapes the HBM term is the larger, so `achieved` is the
+    step's algorithmic bytes per second and `frac` the stated fraction.  The
+    dominant kernel follows with its own HBM and ALU (MUFU ex2) fractions."""
+    wt = work_per_token(w)
+    t_hbm = wt["bytes"] / (P["hbm"] * 1e9)
+    t_tc = wt["tc_flop"] / (P["bf16_sust"] * 1e12)
+    hbm_bound = t_hbm >= t_tc
+    roof_tok_s = 1.0 / max(t_hbm, t_tc)
+    kd = max(range(len(names)), key=lambda k: per_kernel_ms[k])
+    t_k = per_kernel_ms[kd] / 1e3
+    kname = names[kd]
+    traffic, trec = measured_traffic(kname, tokens)
+    dom = {"kernel": kname, "ms": per_kernel_ms[kd], "share_of_step":
+           per_kernel_ms[kd] / max(sum(per_kernel_ms), 1e-12)}
+    if "scan" in kname:
+        # algorithmic bytes of the scan kernel: x, z in, y out, dt_n (fp16) and B/C in
+        kb = tokens * (wt["bytes"] + 2 * w.dt_rank + 4 * 2 * w.d_state)
+        dom["hbm"] = {"achieved": kb / t_k / 1e9, "peak": P["hbm"], "unit": "GB/s",
+                      "frac": kb / t_k / 1e9 / P["hbm"],
+                      "algorithmic_bytes_per_token": kb / tokens}
+        rate, src = alu_peak(P)
+        exps = tokens * wt["exp"]
+        dom["alu"] = {"achieved": exps / t_k / 1e9, "peak": rate / 1e9, "unit": "Gexp/s",
+                      "frac": exps / t_k / rate, "peak_source": src,
+                      "counted": "16 ex2 per (token, channel): the state decays"}
+    else:
+        bound, amount, unit = kernel_units(kname, w, tokens)
+        peak = P["bf16_sust"] if bound == "tensor" else P["hbm"]
+        ach = amount / t_k / (1e12 if bound == "tensor" else 1e9)
+        dom[bound] = {"achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak}
+    dom["traffic"] = traffic
+    dom["traffic_source"] = ("profiles/traffic.json: %s (%s), ncu dram__bytes_read.sum + "
+                             "dram__bytes_write.sum per token x this launch's tokens"
+                             % (trec.get("workload"), trec.get("capture"))
+                             if trec else "none for the current kernel source")
+    if hbm_bound:
+        ach, peak, unit, bound = tok_s * wt["bytes"] / 1e9, P["hbm"], "GB/s", "hbm"
+    else:
+        ach, peak, unit, bound = tok_s * wt["tc_flop"] / 1e12, P["bf16_sust"], "TFLOP/s", "tensor"
+    step_traffic = None
+    recs = [measured_traffic(n, tokens)[0] for n in names]
+    if all(r is not None for r in recs):
+        step_traffic = sum(recs)
+    return {"bound": bound, "achieved": ach, "peak": peak, "unit": unit, "frac": ach / peak,
+            "traffic": step_traffic,
+            "scope": "whole step (every kernel of one jm_mixer_fwd), stated roofline",
+            "definition": "max(x_proj + dt_proj FLOPs / bf16 sustained peak, x,z in + y out "
+                          "bytes / HBM) per token",
+            "roofline_tokens_per_s": roof_tok_s,
+            "peak_source": f"{P['src']} MEASURED_PEAKS.json",
+            "kernels_ms": {names[k]: round(per_kernel_ms[k], 4) for k in range(len(names))},
+            "dominant_kernel": dom}
+
+
 # ------------------------------------------------------------- cpu baseline
 def oracle_sample(w, tokens: float):
     """(sequences, tokens per sequence) of a sample of about `tokens` tokens taken
@@ -538,10 +571,7 @@ def main():
         for _ in range(Wm):
             step()
     stream.synchronize()
-    props = torch.cuda.get_device_properties(dev)
-    uuid = str(getattr(props, "uuid", ""))
-    gpu_id = (uuid if uuid.startswith("GPU-") else "GPU-" + uuid) if uuid else str(local)
-    sampler = ClockSampler(gpu_id)
+    sampler = ClockSampler(gpu_id_of(dev))
     time.sleep(0.6)   # let the sampler start
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     replicas.barrier()
@@ -573,37 +603,7 @@ def main():
     tokens_rank = w.batch * w.seqlen
     value = replicas.job_rate(tokens_rank, world, ms)
 
-    # roofline of the dominant kernel
-    kd = max(range(nk), key=lambda k: per_kernel[k])
-    bound, amount, unit = kernel_units(names[kd], w, tokens_rank)
-    t_k = per_kernel[kd] / 1e3
-    if bound == "alu":
-        clk = P["sm_max"] * 1e6
-        peak = 16 * 148 * clk / 1e9        # MUFU ex2: 16 per clock per SM, 148 SMs
-        achieved = amount / t_k / 1e9
-    elif bound == "tensor":
-        peak = P["bf16_sust"]
-        achieved = amount / t_k / 1e12
-    else:
-        peak = P["hbm"]
-        achieved = amount / t_k / 1e9
-    wt = work_per_token(w)
-    t_ns = max(wt["tc_flop"] / (P["bf16_sust"] * 1e12), wt["bytes"] / (P["hbm"] * 1e9))
-    roof_tok_s = 1.0 / t_ns
-    traffic, traffic_src = measured_traffic(names[kd], tokens_rank)
-    roofline = {"kernel": names[kd], "bound": bound, "achieved": achieved, "peak": peak,
-                "unit": unit, "frac": achieved / peak, "traffic": traffic,
-                "traffic_source": (f"profiles/{traffic_src} (ncu dram__bytes_read.sum + "
-                                   "dram__bytes_write.sum per token, scaled to this launch)"
-                                   if traffic_src else "none for the current kernel source"),
-                "peak_source": (f"MUFU 16/clk/SM x 148 SMs x {P['sm_max']:.0f} MHz (derived)"
-                                if bound == "alu" else f"{P['src']} MEASURED_PEAKS.json"),
-                "kernel_ms": per_kernel[kd],
-                "kernels_ms": {names[k]: round(per_kernel[k], 4) for k in range(nk)},
-                "step_roofline": {"roofline_tokens_per_s": roof_tok_s,
-                               "frac": value / world / roof_tok_s,
-                               "definition": "max(tc_flop/bf16 sustained peak, bytes/HBM) "
-                                             "per token, bytes = x,z in + y out"}}
+    roofline = roofline_block(P, w, names, per_kernel, value / world, tokens_rank)
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
             "warmup": Wm, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",

@@ -2,6 +2,8 @@
 
 * ``libjmix.so``: the CUDA kernels and the C ABI, compiled for sm_100a only.
 * ``libjmix_synth.so``: the seeded input generator (host C).
+* ``libjmix_pipes.so``: the pipe-rate microbenchmarks (``pipe_rates.py``), kept
+  out of libjmix.
 
 Both are built in-tree under ``_build/`` so that they travel with the source.
 """
@@ -18,6 +20,8 @@ BUILD = os.path.join(HERE, "_build")
 INCLUDE = os.path.join(ROOT, "include")
 LIBJMIX = os.path.join(BUILD, "libjmix.so")
 LIBSYNTH = os.path.join(BUILD, "libjmix_synth.so")
+LIBPIPES = os.path.join(BUILD, "libjmix_pipes.so")
+PIPES_SRC = os.path.join(CSRC, "pipe_rates.cu")
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
               "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden"]
@@ -48,7 +52,7 @@ def build_synth(force: bool = False) -> str:
 
 
 def jmix_sources():
-    return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    return sorted(p for p in glob.glob(os.path.join(CSRC, "*.cu")) if p != PIPES_SRC)
 
 
 def jmix_deps():
@@ -90,9 +94,20 @@ def build_libjmix(force: bool = False, verbose: bool = False) -> str:
     return LIBJMIX
 
 
+def build_pipes(force: bool = False) -> str:
+    """nvcc ... -shared pipe_rates.cu -> _build/libjmix_pipes.so (sm_100a)."""
+    if force or _stale(LIBPIPES, [PIPES_SRC]):
+        os.makedirs(BUILD, exist_ok=True)
+        tmp = LIBPIPES + ".tmp%d" % os.getpid()
+        subprocess.check_call([_nvcc(), *NVCC_FLAGS, "-shared", PIPES_SRC, "-o", tmp])
+        os.replace(tmp, LIBPIPES)
+    return LIBPIPES
+
+
 def build_all(force: bool = False) -> None:
     build_synth(force)
     build_libjmix(force)
+    build_pipes(force)
 
 
 if __name__ == "__main__":

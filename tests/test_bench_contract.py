@@ -75,3 +75,41 @@ def test_reference_arm_json_line():
     e2e = line["e2e"]
     assert e2e["value"] == line["value"] and e2e["unit"] == line["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_roofline_block_leads_with_the_stated_fraction(tmp_path, monkeypatch):
+    """frac is the step against max(projection FLOPs / bf16 peak, bytes / HBM); the
+    dominant kernel's HBM and ALU fractions follow, labelled, with the ALU peak
+    from the committed pipe-rate record when there is one."""
+    w = synth.WORKLOADS["jamba_b8_l4096"]
+    P = dict(hbm=6531.3, bf16=1632.8, bf16_sust=1361.8, sm_max=1965.0, src="measured")
+    names = ["k_conv_silu16", "k_xproj", "k_norms16", "k_scan_fused"]
+    ms = [0.27, 0.18, 0.02, 2.12]
+    tokens = 8 * 4096
+    tok_s = tokens / (sum(ms) / 1e3)
+    r = bench.roofline_block(P, w, names, ms, tok_s, tokens)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["peak"] == P["hbm"]
+    assert abs(r["achieved"] - tok_s * 49152 / 1e9) < 1e-6
+    assert abs(r["frac"] - tok_s / r["roofline_tokens_per_s"]) < 1e-12
+    dom = r["dominant_kernel"]
+    assert dom["kernel"] == "k_scan_fused"
+    assert abs(dom["hbm"]["frac"] - dom["hbm"]["achieved"] / P["hbm"]) < 1e-12
+    exps = tokens * 8192 * 16
+    assert abs(dom["alu"]["achieved"] - exps / 2.12e-3 / 1e9) < 1e-6
+    # without a pipe-rate record the nominal rate is used, and said so
+    monkeypatch.setattr(bench, "PIPES_JSON", str(tmp_path / "none.json"))
+    r2 = bench.roofline_block(P, w, names, ms, tok_s, tokens)
+    assert r2["dominant_kernel"]["alu"]["peak_source"].startswith("nominal")
+    assert abs(r2["dominant_kernel"]["alu"]["peak"] - 16 * 148 * 1.965) < 1e-9
+
+
+def test_traffic_record_is_keyed_to_the_kernel_source(tmp_path):
+    p = tmp_path / "traffic.json"
+    sha = bench.kernel_source_sha()
+    p.write_text(json.dumps({"k_scan_fused": {"bytes_per_token": 51000.5, "source_sha256": sha,
+                                              "workload": "w", "capture": "c"},
+                             "k_xproj": {"bytes_per_token": 10, "source_sha256": "0" * 64}}))
+    got, rec = bench.measured_traffic("k_scan_fused", 1000, str(p))
+    assert got == 51000500 and rec["workload"] == "w"
+    assert bench.measured_traffic("k_xproj", 1000, str(p)) == (None, None)   # stale source
+    assert bench.measured_traffic("k_conv_silu16", 1000, str(p)) == (None, None)
