@@ -61,6 +61,10 @@ def parse():
                     help="also time jm_mixer_fwd_varlen on a packed batch of mixed lengths")
     ap.add_argument("--seqlen", type=int, default=0,
                     help="override the workload's sequence length (profiling captures)")
+    ap.add_argument("--record-traffic", default="",
+                    help="ncu CSV (dram__bytes_read.sum, dram__bytes_write.sum per launch) of "
+                         "one jm_mixer_fwd of this workload: write profiles/traffic.json and exit")
+    ap.add_argument("--capture", default="", help="the ncu command that made --record-traffic")
     return ap.parse_args()
 
 
@@ -134,12 +138,47 @@ def measured_traffic(kernel: str, tokens: int, path: str = TRAFFIC_JSON):
     else (None, None)."""
     try:
         with open(path) as f:
-            rec = json.load(f).get(kernel)
+            recs = json.load(f)
     except (OSError, ValueError):
         return None, None
+    # a launch name may be the family of the recorded kernel (k_norms16 -> k_norms16_warp)
+    rec = recs.get(kernel) or next((v for k, v in sorted(recs.items())
+                                    if k.startswith(kernel + "_")), None)
     if not rec or rec.get("source_sha256") != kernel_source_sha():
         return None, None
     return int(round(rec["bytes_per_token"] * tokens)), rec
+
+
+def record_traffic(csv_path: str, w, capture: str, path: str = TRAFFIC_JSON) -> dict:
+    """profiles/traffic.json from an ncu CSV of one forward call: DRAM bytes per
+    token of each kernel (read + write, summed over its launches in the CSV and
+    divided by their tokens), keyed to the current kernel source."""
+    import csv
+    tokens = w.batch * w.seqlen
+    per = {}
+    with open(csv_path) as f:
+        rows = [r for r in csv.reader(l for l in f if l.startswith('"'))]
+    head = rows[0]
+    ki, mi, vi, ii = (head.index("Kernel Name"), head.index("Metric Name"),
+                      head.index("Metric Value"), head.index("ID"))
+    launches = {}
+    for r in rows[1:]:
+        if r[mi] in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+            name = re.sub(r"^(void )?(unnamed>::)?", "", r[ki]).split("(")[0].split("<")[0]
+            name = name.replace("jmix::", "").strip()
+            per[name] = per.get(name, 0.0) + float(r[vi].replace(",", ""))
+            launches.setdefault(name, set()).add(r[ii])
+    sha = kernel_source_sha()
+    out = {}
+    for name, b in per.items():
+        out[name] = {"bytes_per_token": b / len(launches[name]) / tokens, "source_sha256": sha,
+                     "workload": f"{w.name} (B={w.batch}, L={w.seqlen}, {tokens} tokens)",
+                     "capture": capture, "launches": len(launches[name]),
+                     "metric": "dram__bytes_read.sum + dram__bytes_write.sum"}
+    with open(path, "w") as f:
+        json.dump(out, f, indent=1, sort_keys=True)
+        f.write("\n")
+    return out
 
 
 def alu_peak(P):
@@ -159,14 +198,18 @@ def alu_peak(P):
 
 
 # ------------------------------------------------------------------ decode
-def decode_bench(dev, stream, steps: int = 64, warmup: int = 5, zoh: bool = False):
-    """64 consecutive jm_mixer_step calls on the decode workload (B=256 sequences at
-    Jamba shapes, states updated in place); returns a dict for the JSON line."""
+def decode_bench(dev, stream, steps: int = 64, warmup: int = 5, zoh: bool = False,
+                 pool_slots: int = 0):
+    """64 consecutive decode steps on the decode workload (B=256 sequences at Jamba
+    shapes, states updated in place); returns a dict for the JSON line.  With
+    pool_slots > 0 the steps are jm_mixer_step_indexed calls whose 256 rows use
+    distinct, permuted slots of a pool of that many slots (a fresh set every
+    step), with the weights prepared once; else jm_mixer_step calls."""
     import torch
     from mamba_selective_scan_jamba_b200 import devio, jmix, synth
     w = synth.WORKLOADS["jamba_decode_b256"].with_(zoh=zoh)
     W = synth.make_weights(w)
-    S = synth.make_decode_state(w)
+    S = synth.make_decode_state(w.with_(batch=pool_slots) if pool_slots else w)
     Wd = devio.weights_to_device(W, dev)
     cs = devio.to_device(S["conv_state"], dev)
     ss = devio.to_device(S["ssm_state"], dev)
@@ -177,9 +220,23 @@ def decode_bench(dev, stream, steps: int = 64, warmup: int = 5, zoh: bool = Fals
     d = devio.dims_of(w)
     n = jmix.jm_mixer_step_workspace_size(d)
     ws = devio.workspace(n, dev)
+    if pool_slots:
+        rng = np.random.default_rng(3)
+        idxs = [torch.from_numpy(rng.permutation(pool_slots)[:w.batch].astype(np.int32)).to(dev)
+                for _ in range(4)]
+        npw = jmix.jm_prepared_weights_size(d)
+        prep = devio.workspace(npw, dev)
+        jmix.jm_prepare_weights(d, Wd["xproj_w"], Wd["dtproj_w"], prep, npw, stream=stream)
+
+        def one(i):
+            jmix.jm_mixer_step_indexed(d, idxs[i % 4], pool_slots, xs[i % 4], zs[i % 4], cs, ss,
+                                       Wd, prep, y, ws, n, stream=stream)
+    else:
+        def one(i):
+            jmix.jm_mixer_step(d, xs[i % 4], zs[i % 4], cs, ss, Wd, y, ws, n, stream=stream)
     with torch.cuda.stream(stream):
         for i in range(warmup):
-            jmix.jm_mixer_step(d, xs[i % 4], zs[i % 4], cs, ss, Wd, y, ws, n, stream=stream)
+            one(i)
     stream.synchronize()
     nk = jmix.jm_last_launch_count()
     names = [jmix.jm_last_kernel_name(i) for i in range(nk)]
@@ -194,7 +251,7 @@ def decode_bench(dev, stream, steps: int = 64, warmup: int = 5, zoh: bool = Fals
         a.record(stream)
         for i in range(steps):
             jmix.jm_set_kernel_events([e.cuda_event for e in evs[i]])
-            jmix.jm_mixer_step(d, xs[i % 4], zs[i % 4], cs, ss, Wd, y, ws, n, stream=stream)
+            one(i)
         b.record(stream)
     jmix.jm_set_kernel_events(None)
     stream.synchronize()
@@ -207,7 +264,9 @@ def decode_bench(dev, stream, steps: int = 64, warmup: int = 5, zoh: bool = Fals
     B, dd, N = w.batch, w.d_inner, w.d_state
     wbytes = sum(int(v.nbytes) for v in W.values())
     nbytes = B * dd * (N * 4 * 2 + 3 * 2 * 2 + 2 * 3) + wbytes
-    return {"workload": w.name, "batch": B, "steps": steps, "us_per_step": ms * 1e3,
+    api = (f"jm_mixer_step_indexed: {B} rows in a {pool_slots}-slot pool, permuted slots, "
+           "weights prepared once" if pool_slots else "jm_mixer_step")
+    return {"workload": w.name, "api": api, "batch": B, "steps": steps, "us_per_step": ms * 1e3,
             "tokens_per_s": B / (ms / 1e3), "algorithmic_bytes_per_step": nbytes,
             "weight_bytes_per_step": wbytes,
             "achieved_GBps": nbytes / (ms / 1e3) / 1e9, "kernels_us": per,
@@ -283,9 +342,12 @@ def varlen_bench(dev, stream, steps: int = 20, warmup: int = 3):
             "kernels_ms": per, "launches_per_step": nk}
 
 
-def layer_bench(dev, stream, w, d_model: int = 4096, steps: int = 10, warmup: int = 3):
-    """jm_layer_fwd (in_proj on cuBLASLt -> mixer core -> out_proj on cuBLASLt) on
-    the workload at Jamba's d_model; returns a dict for the JSON line."""
+def layer_bench(dev, stream, w, d_model: int = 4096, steps: int = 10, warmup: int = 3,
+                mixer_ms: float = 0.0):
+    """jm_layer_fwd (in_proj -> mixer core -> out_proj, both projections on libjmix's
+    tcgen05 GEMM) on the workload at Jamba's d_model; returns a dict for the JSON
+    line.  mixer_ms (the mixer core alone, timed by the caller on the same
+    workload) splits the layer's time into mixer and projections."""
     import torch
     from mamba_selective_scan_jamba_b200 import devio, jmix, synth
     W = synth.make_weights(w)
@@ -317,10 +379,16 @@ def layer_bench(dev, stream, w, d_model: int = 4096, steps: int = 10, warmup: in
     ms = a.elapsed_time(b) / steps
     T = w.batch * w.seqlen
     gemm_flop = 2.0 * T * d_model * 3 * w.d_inner        # in_proj (2 d_inner) + out_proj
-    return {"workload": f"{w.name} + in_proj/out_proj (d_model {d_model})", "tokens": T,
-            "steps": steps, "ms_per_step": ms, "tokens_per_s": T / (ms / 1e3),
-            "projection_tflop_per_step": gemm_flop / 1e12,
-            "projections": "cuBLASLt bf16 GEMMs (fp32 accumulation), not fused"}
+    out = {"workload": f"{w.name} + in_proj/out_proj (d_model {d_model})", "tokens": T,
+           "steps": steps, "ms_per_step": ms, "tokens_per_s": T / (ms / 1e3),
+           "projection_tflop_per_step": gemm_flop / 1e12,
+           "projections": "k_gemm_bf16: tcgen05 bf16 GEMM, fp32 accumulation in TMEM; in_proj "
+                          "writes x and z in the mixer's layout"}
+    if mixer_ms > 0:
+        proj_ms = ms - mixer_ms
+        out.update({"mixer_ms": mixer_ms, "projections_ms": proj_ms,
+                    "projection_tflops": gemm_flop / (proj_ms / 1e3) / 1e12})
+    return out
 
 
 def bwd_bench(dev, stream, B: int = 1, L: int = 4096, d: int = 8192, steps: int = 5,
@@ -521,6 +589,9 @@ def main():
     if args.impl == "reference":
         reference_arm(args, base, rank, world)
         return
+    if args.record_traffic:
+        print(json.dumps(record_traffic(args.record_traffic, base, args.capture), indent=1))
+        return
 
     import torch
     import torch.distributed as dist
@@ -644,13 +715,16 @@ def main():
     if args.varlen:
         line["varlen"] = varlen_bench(dev, stream)
     if args.layer:
-        line["layer"] = layer_bench(dev, stream, w)
+        line["layer"] = layer_bench(dev, stream, w, mixer_ms=ms)
     if args.bwd:
         line["bwd"] = [bwd_bench(dev, stream, B=1), bwd_bench(dev, stream, B=8)]
     if not args.no_decode:
         dec = decode_bench(dev, stream, zoh=args.zoh)
         dec["hbm_frac"] = dec["achieved_GBps"] / P["hbm"]
         line["decode"] = dec
+        ind = decode_bench(dev, stream, zoh=args.zoh, pool_slots=1024)
+        ind["hbm_frac"] = ind["achieved_GBps"] / P["hbm"]
+        line["decode_indexed"] = ind
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, cores, sample = oracle_rate(w, 12.0)
         line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": cores,

@@ -125,6 +125,48 @@ jm_status jm_mixer_step(const jm_dims* dims, const void* x_t, const void* z_t, v
                         const float* A_log, const float* D, void* y_t, void* workspace,
                         size_t ws_bytes, jm_stream_t stream);
 
+/* Bytes of the fp16 weight copies jm_prepare_weights writes (0 for invalid
+ * dims or float32 io). */
+size_t jm_prepared_weights_size(const jm_dims* dims);
+
+/* Converts xproj_w [R + 2N, d] and dtproj_w [d, R] (bf16, device) once into the
+ * fp16 operands the tensor-core path feeds its two contractions (exact for
+ * |w| >= 2^-14; fp16 subnormals below), into `prepared` (device, 256-byte
+ * aligned, at least jm_prepared_weights_size bytes, owned by the caller).  A
+ * decode loop passes it to jm_mixer_step_indexed so that no step re-converts
+ * the weights; it stays valid until the weights change.  bf16 io only
+ * (JM_ERR_UNSUPPORTED otherwise).  Asynchronous on `stream`. */
+jm_status jm_prepare_weights(const jm_dims* dims, const void* xproj_w, const void* dtproj_w,
+                             void* prepared, size_t bytes, jm_stream_t stream);
+
+/* One decode step for a batch of rows whose states live in slots of a state
+ * pool, as a continuously batching server keeps them: the set of active
+ * sequences changes from step to step, their cached states stay in place.
+ * (TransformerLens "Jamba" adapter page: generation threads the cache of conv
+ * and recurrent states through the mixer.)
+ *   dims->batch  B rows this step; dims->seqlen must be 1; bf16 io only
+ *   state_idx    DEVICE int32 [B]: row b of x_t, z_t, y_t uses slot state_idx[b];
+ *                the B slots must be distinct (duplicates leave those slots and
+ *                rows unspecified; no access leaves the buffers)
+ *   n_slots      slots S in the pools, B <= S < 2^31
+ *   conv_pool    in/out [S, d, d_conv-1] bf16;  ssm_pool in/out [S, d, N] float32
+ *   prepared     fp16 weights from jm_prepare_weights, or NULL (then the step
+ *                converts xproj_w and dtproj_w itself, as jm_mixer_step does)
+ * Slot state_idx[b] is updated in place exactly as jm_mixer_step updates row b;
+ * no other slot is read or written.  A slot outside [0, S) is checked on the
+ * device: that row's y_t is left unwritten, its slot untouched, and
+ * jm_poll_error returns JM_ERR_INVALID_ARG.  Workspace: at least
+ * jm_mixer_step_workspace_size(dims) bytes.  Other arguments, errors and
+ * ownership as jm_mixer_step. */
+jm_status jm_mixer_step_indexed(const jm_dims* dims, const int32_t* state_idx, int64_t n_slots,
+                                const void* x_t, const void* z_t, void* conv_pool,
+                                float* ssm_pool, const void* conv_w, const void* conv_b,
+                                const void* xproj_w, const void* dt_norm_w,
+                                const void* b_norm_w, const void* c_norm_w,
+                                const void* dtproj_w, const float* dt_bias, const float* A_log,
+                                const float* D, const void* prepared, void* y_t,
+                                void* workspace, size_t ws_bytes, jm_stream_t stream);
+
 /* jm_mixer_step without a caller workspace, for callers that cannot allocate
  * device memory: code inside CUDA stream capture (where cudaMalloc is not
  * allowed), serving engines that hand all device memory to their own caches
@@ -193,8 +235,8 @@ jm_status jm_mixer_fwd_host(const jm_dims* dims, const void* x_host, const void*
  * 256 bytes: JM_ERR_TIMEOUT if a bounded device-side wait ran out since the
  * last call that cleared them (every jm_mixer_fwd / jm_mixer_step clears
  * them), JM_ERR_INVALID_ARG if a device-side input check failed (the
- * cu_seqlens of jm_mixer_fwd_varlen), JM_ERR_CUDA if the stream reports an
- * error, JM_OK otherwise. */
+ * cu_seqlens of jm_mixer_fwd_varlen, the state_idx of jm_mixer_step_indexed),
+ * JM_ERR_CUDA if the stream reports an error, JM_OK otherwise. */
 jm_status jm_poll_error(void* workspace, jm_stream_t stream);
 
 /* The full Mamba layer around the mixer core (bf16 io only):
@@ -204,10 +246,12 @@ jm_status jm_poll_error(void* workspace, jm_stream_t stream);
  * give x, the rest z); out_proj_w: [d_model, d_inner]; out: [B, L, d_model]; all
  * bf16 device memory, 16-byte aligned; d_model a positive multiple of 8.  The
  * mixer arguments, states, errors and ownership are those of jm_mixer_fwd.  The
- * projections run on cuBLASLt (fp32 accumulation, bf16 x, z, y and out) with the
+ * projections run on libjmix's tcgen05 GEMM (fp32 accumulation, bf16 x, z, y
+ * and out; in_proj writes x and z straight into the mixer's layout) with the
  * caller's workspace as scratch: jm_layer_fwd_workspace_size(dims, d_model)
  * bytes, 256-byte aligned; its first 256 bytes are the error header that
- * jm_poll_error reads.  JM_ERR_UNSUPPORTED for float32 io. */
+ * jm_poll_error reads (the projections' flags and the mixer's).  JM_ERR_UNSUPPORTED
+ * for float32 io. */
 size_t jm_layer_fwd_workspace_size(const jm_dims* dims, int64_t d_model);
 jm_status jm_layer_fwd(const jm_dims* dims, int64_t d_model, const void* hidden,
                        const void* in_proj_w, const void* conv_w, const void* conv_b,

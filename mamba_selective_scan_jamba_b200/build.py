@@ -88,7 +88,7 @@ def build_libjmix(force: bool = False, verbose: bool = False) -> str:
     tmp = LIBJMIX + ".tmp%d" % os.getpid()
     cuda_lib = os.path.join(os.path.dirname(os.path.dirname(nvcc)), "lib64")
     subprocess.check_call([nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-shared",
-                           "-Xcompiler", "-fPIC", *objs, "-o", tmp, "-lcublasLt",
+                           "-Xcompiler", "-fPIC", *objs, "-o", tmp,
                            "-Xlinker", "-rpath=" + cuda_lib])
     os.replace(tmp, LIBJMIX)
     return LIBJMIX

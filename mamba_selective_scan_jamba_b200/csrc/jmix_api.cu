@@ -162,7 +162,10 @@ jm_status status_of_flags(const ErrFlags& f) {
     return JM_ERR_TIMEOUT;
   }
   if (f.bad_input) {
-    set_error("cu_seqlens is not 0 = c[0] <= c[1] <= ... <= c[B] = total tokens");
+    if (f.where == kSiteBadSlot)
+      set_error("a state_idx entry is outside [0, n_slots): that row was skipped");
+    else
+      set_error("cu_seqlens is not 0 = c[0] <= c[1] <= ... <= c[B] = total tokens");
     return JM_ERR_INVALID_ARG;
   }
   return JM_OK;
@@ -255,7 +258,8 @@ static jm_status fwd_impl(const jm_dims* dims, const void* x, const void* z, con
                           float* final_state, const void* init_conv_state,
                           const float* init_ssm_state, void* final_conv_state, void* workspace,
                           size_t ws_bytes, jm_stream_t stream, bool step, Problem& p,
-                          const int32_t* cu = nullptr) {
+                          const int32_t* cu = nullptr, const int32_t* sidx = nullptr,
+                          int64_t n_slots = 0, const void* prepared = nullptr) {
   jm_status st = check_dims(dims, step);
   if (st != JM_OK) return st;
   fill_problem(p, dims);
@@ -306,6 +310,9 @@ static jm_status fwd_impl(const jm_dims* dims, const void* x, const void* z, con
   p.init_conv = init_conv_state;
   p.init_ssm = init_ssm_state;
   p.final_conv = final_conv_state;
+  p.sidx = sidx;
+  p.n_slots = n_slots;
+  p.prepared = prepared;
   p.ws = static_cast<char*>(workspace);
   p.ws_bytes = ws_bytes;
   p.stream = reinterpret_cast<cudaStream_t>(stream);
@@ -402,6 +409,80 @@ JM_API jm_status jm_mixer_step(const jm_dims* dims, const void* x_t, const void*
   return fwd_impl(dims, x_t, z_t, conv_w, conv_b, xproj_w, dt_norm_w, b_norm_w, c_norm_w,
                   dtproj_w, dt_bias, A_log, D, y_t, ssm_state, conv_state, ssm_state, conv_state,
                   workspace, ws_bytes, stream, true, p);
+}
+
+JM_API size_t jm_prepared_weights_size(const jm_dims* dims) {
+  if (check_dims(dims, false) != JM_OK || dims->io != JM_BF16) return 0;
+  return prepared_weights_bytes(dims->d_inner, dims->dt_rank);
+}
+
+JM_API jm_status jm_prepare_weights(const jm_dims* dims, const void* xproj_w,
+                                    const void* dtproj_w, void* prepared, size_t bytes,
+                                    jm_stream_t stream) {
+  jm_status st = check_dims(dims, false);
+  if (st != JM_OK) return st;
+  if (dims->io != JM_BF16) {
+    set_error("jm_prepare_weights: only bf16 weights are converted (float32 io uses them as is)");
+    return JM_ERR_UNSUPPORTED;
+  }
+  if (!xproj_w || !dtproj_w || !prepared) {
+    set_error("jm_prepare_weights: NULL pointer");
+    return JM_ERR_INVALID_ARG;
+  }
+  if (!aligned(xproj_w, 16) || !aligned(dtproj_w, 16) || !aligned(prepared, 256)) {
+    set_error("jm_prepare_weights: weights must be 16-byte aligned, prepared 256-byte aligned");
+    return JM_ERR_INVALID_ARG;
+  }
+  const size_t need = prepared_weights_bytes(dims->d_inner, dims->dt_rank);
+  if (bytes < need) {
+    set_error("jm_prepare_weights: %zu bytes given, %zu needed", bytes, need);
+    return JM_ERR_WORKSPACE;
+  }
+  const cudaError_t e = run_prepare_weights(dims->d_inner, dims->dt_rank, xproj_w, dtproj_w,
+                                            prepared, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) {
+    set_error("CUDA error: %s", cudaGetErrorString(e));
+    return JM_ERR_CUDA;
+  }
+  return JM_OK;
+}
+
+JM_API jm_status jm_mixer_step_indexed(const jm_dims* dims, const int32_t* state_idx,
+                                       int64_t n_slots, const void* x_t, const void* z_t,
+                                       void* conv_pool, float* ssm_pool, const void* conv_w,
+                                       const void* conv_b, const void* xproj_w,
+                                       const void* dt_norm_w, const void* b_norm_w,
+                                       const void* c_norm_w, const void* dtproj_w,
+                                       const float* dt_bias, const float* A_log, const float* D,
+                                       const void* prepared, void* y_t, void* workspace,
+                                       size_t ws_bytes, jm_stream_t stream) {
+  jm_status st = check_dims(dims, true);
+  if (st != JM_OK) return st;
+  if (dims->io != JM_BF16) {
+    set_error("jm_mixer_step_indexed is built for bf16 io only");
+    return JM_ERR_UNSUPPORTED;
+  }
+  if (!conv_pool || !ssm_pool) {
+    set_error("conv_pool and ssm_pool are required");
+    return JM_ERR_INVALID_ARG;
+  }
+  if (dims->batch > 0 && (!state_idx || !aligned(state_idx, 4))) {
+    set_error("state_idx must be a 4-byte aligned device array of batch entries");
+    return JM_ERR_INVALID_ARG;
+  }
+  if (n_slots < dims->batch || n_slots > 0x7fffffffLL || (dims->batch > 0 && n_slots < 1)) {
+    set_error("n_slots must be in [batch, 2^31) (the batch's slots are distinct), got %lld",
+              (long long)n_slots);
+    return JM_ERR_INVALID_ARG;
+  }
+  if (prepared && !aligned(prepared, 256)) {
+    set_error("prepared weights must be 256-byte aligned");
+    return JM_ERR_INVALID_ARG;
+  }
+  Problem p;
+  return fwd_impl(dims, x_t, z_t, conv_w, conv_b, xproj_w, dt_norm_w, b_norm_w, c_norm_w,
+                  dtproj_w, dt_bias, A_log, D, y_t, ssm_pool, conv_pool, ssm_pool, conv_pool,
+                  workspace, ws_bytes, stream, true, p, nullptr, state_idx, n_slots, prepared);
 }
 
 JM_API jm_status jm_mixer_fwd_host(const jm_dims* dims, const void* x_host, const void* z_host,

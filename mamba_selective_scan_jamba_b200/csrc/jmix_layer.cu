@@ -1,11 +1,10 @@
 // jm_layer_fwd: the full Mamba layer around the mixer core,
 //   [x | z] = hidden . in_proj_w^T,  y = mixer(x, z),  out = y . out_proj_w^T
 // (TransformerLens "Jamba" adapter page, "Architecture overview": in_proj /
-// conv1d / x_proj / dt_proj / out_proj).  The two projections are plain dense
-// GEMMs and go to cuBLASLt (bf16 in, fp32 accumulate, bf16 out), with the
-// caller's workspace as its scratch: x and z are written as two separate
-// [T, d_inner] matrices, the layout the mixer reads, and y feeds out_proj.
-#include <cublasLt.h>
+// conv1d / x_proj / dt_proj / out_proj).  The two projections run on the
+// tcgen05 GEMM of k_gemm.cu (bf16 in, fp32 accumulation, bf16 out): in_proj is
+// one GEMM over N = 2 d_inner whose epilogue writes x and z as the two
+// [T, d_inner] matrices the mixer reads; out_proj reads y.
 #include <string.h>
 
 #include "jmix_internal.cuh"
@@ -15,13 +14,14 @@
 namespace jmix {
 namespace {
 
-constexpr size_t kLtWorkspace = size_t(32) << 20;
-
+// Layer workspace: [error header][mixer workspace][x][z][y].  The projections
+// record into the layer's header; out_proj carries the mixer's flags into it,
+// so jm_poll_error on the layer workspace reports all three.
 struct LayerWs {
+  ErrFlags* hdr;
   char* x;
   char* z;
   char* y;
-  char* lt;
   char* mixer;
   size_t mixer_bytes;
   size_t bytes;
@@ -36,66 +36,14 @@ LayerWs layer_layout(int64_t T, int64_t d, size_t mixer_bytes, char* base) {
     return base ? base + o : nullptr;
   };
   const size_t act = (size_t)T * (size_t)d * 2;
-  // the mixer's workspace comes first: its error header is the layer's
+  w.hdr = reinterpret_cast<ErrFlags*>(take(sizeof(ErrFlags)));
   w.mixer = take(mixer_bytes);
   w.mixer_bytes = mixer_bytes;
   w.x = take(act);
   w.z = take(act);
   w.y = take(act);
-  w.lt = take(kLtWorkspace);
   w.bytes = off;
   return w;
-}
-
-cublasLtHandle_t lt_handle() {
-  static thread_local cublasLtHandle_t h = nullptr;
-  if (!h && cublasLtCreate(&h) != CUBLAS_STATUS_SUCCESS) h = nullptr;
-  return h;
-}
-
-// Out [M, N] = X [M, K] . W[N, K]^T, all row-major bf16, fp32 accumulation.
-// In cuBLAS's column-major terms: Out^T [N, M] = op_T(W as K x N) . X^T (K x M).
-jm_status lt_gemm(int64_t M, int64_t N, int64_t K, const void* X, const void* W, void* Out,
-                  void* ws, size_t ws_bytes, cudaStream_t s) {
-  cublasLtHandle_t h = lt_handle();
-  if (!h) {
-    set_error("cublasLtCreate failed");
-    return JM_ERR_CUDA;
-  }
-  cublasLtMatmulDesc_t op = nullptr;
-  cublasLtMatrixLayout_t la = nullptr, lb = nullptr, lc = nullptr;
-  cublasLtMatmulPreference_t pref = nullptr;
-  jm_status st = JM_ERR_CUDA;
-  const cublasOperation_t ta = CUBLAS_OP_T, tb = CUBLAS_OP_N;
-  const float alpha = 1.0f, beta = 0.0f;
-  cublasLtMatmulHeuristicResult_t heur;
-  int found = 0;
-  if (cublasLtMatmulDescCreate(&op, CUBLAS_COMPUTE_32F, CUDA_R_32F) != CUBLAS_STATUS_SUCCESS ||
-      cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSA, &ta, sizeof(ta)) ||
-      cublasLtMatmulDescSetAttribute(op, CUBLASLT_MATMUL_DESC_TRANSB, &tb, sizeof(tb)) ||
-      cublasLtMatrixLayoutCreate(&la, CUDA_R_16BF, (uint64_t)K, (uint64_t)N, K) ||
-      cublasLtMatrixLayoutCreate(&lb, CUDA_R_16BF, (uint64_t)K, (uint64_t)M, K) ||
-      cublasLtMatrixLayoutCreate(&lc, CUDA_R_16BF, (uint64_t)N, (uint64_t)M, N) ||
-      cublasLtMatmulPreferenceCreate(&pref) ||
-      cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES,
-                                           &ws_bytes, sizeof(ws_bytes)) ||
-      cublasLtMatmulAlgoGetHeuristic(h, op, la, lb, lc, lc, pref, 1, &heur, &found) ||
-      found < 1) {
-    set_error("cuBLASLt has no bf16 GEMM for %lld x %lld x %lld", (long long)M, (long long)N,
-              (long long)K);
-  } else if (cublasLtMatmul(h, op, &alpha, W, la, X, lb, &beta, Out, lc, Out, lc, &heur.algo, ws,
-                            ws_bytes, s) != CUBLAS_STATUS_SUCCESS) {
-    set_error("cublasLtMatmul failed (%lld x %lld x %lld)", (long long)M, (long long)N,
-              (long long)K);
-  } else {
-    st = JM_OK;
-  }
-  if (pref) cublasLtMatmulPreferenceDestroy(pref);
-  if (lc) cublasLtMatrixLayoutDestroy(lc);
-  if (lb) cublasLtMatrixLayoutDestroy(lb);
-  if (la) cublasLtMatrixLayoutDestroy(la);
-  if (op) cublasLtMatmulDescDestroy(op);
-  return st;
 }
 
 jm_status check_layer(const jm_dims* dims, int64_t d_model) {
@@ -162,18 +110,24 @@ JM_API jm_status jm_layer_fwd(const jm_dims* dims, int64_t d_model, const void* 
   }
   LayerWs w = layer_layout(T, d, jm_mixer_fwd_workspace_size(dims), static_cast<char*>(workspace));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const char* wi = static_cast<const char*>(in_proj_w);
-  if (T > 0) {
-    if ((st = lt_gemm(T, d, d_model, hidden, wi, w.x, w.lt, kLtWorkspace, s)) != JM_OK) return st;
-    if ((st = lt_gemm(T, d, d_model, hidden, wi + (size_t)d * d_model * 2, w.z, w.lt, kLtWorkspace,
-                      s)) != JM_OK)
-      return st;
+  cudaError_t e = cudaMemsetAsync(w.hdr, 0, sizeof(ErrFlags), s);
+  if (e == cudaSuccess && T > 0)  // in_proj: N = 2 d_inner, x = columns [0, d), z = [d, 2d)
+    e = gemm_bf16_tn(T, 2 * d, d_model, hidden, in_proj_w, w.x, w.z, d, w.hdr, nullptr, s, false);
+  if (e != cudaSuccess) {
+    set_error("in_proj: CUDA error: %s", cudaGetErrorString(e));
+    return JM_ERR_CUDA;
   }
   st = jm_mixer_fwd(dims, w.x, w.z, conv_w, conv_b, xproj_w, dt_norm_w, b_norm_w, c_norm_w,
                     dtproj_w, dt_bias, A_log, D, w.y, final_state, init_conv_state, init_ssm_state,
                     final_conv_state, w.mixer, w.mixer_bytes, stream);
   if (st != JM_OK) return st;
-  if (T > 0 && (st = lt_gemm(T, d_model, d, w.y, out_proj_w, out, w.lt, kLtWorkspace, s)) != JM_OK)
-    return st;
+  if (T > 0) {  // (with no tokens nothing ran that could set a flag)
+    e = gemm_bf16_tn(T, d_model, d, w.y, out_proj_w, out, nullptr, d_model, w.hdr,
+                     reinterpret_cast<const ErrFlags*>(w.mixer), s, true);
+    if (e != cudaSuccess) {
+      set_error("out_proj: CUDA error: %s", cudaGetErrorString(e));
+      return JM_ERR_CUDA;
+    }
+  }
   return JM_OK;
 }

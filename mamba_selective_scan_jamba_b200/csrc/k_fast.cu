@@ -234,9 +234,10 @@ __global__ void __launch_bounds__(256, JMIX_CONV_OCC) k_conv_silu16_packed(
 template <int kConvG>
 __global__ void __launch_bounds__(256, JMIX_CONV_OCC) k_conv_silu16(
     const bf16* __restrict__ x, const bf16* __restrict__ conv_w, const bf16* __restrict__ conv_b,
-    const bf16* __restrict__ hist, int64_t B, int64_t L, int64_t d, __half* __restrict__ u,
-    int64_t n_conv, const bf16* __restrict__ wx, int64_t n_wx8, __half* __restrict__ wx16,
-    const bf16* __restrict__ wdt, int64_t n_wdt8, __half* __restrict__ wdt16) {
+    const bf16* __restrict__ hist, const int* __restrict__ sidx, int64_t n_slots, int64_t B,
+    int64_t L, int64_t d, __half* __restrict__ u, int64_t n_conv, const bf16* __restrict__ wx,
+    int64_t n_wx8, __half* __restrict__ wx16, const bf16* __restrict__ wdt, int64_t n_wdt8,
+    __half* __restrict__ wdt16) {
   const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (tid < n_conv) {
     const int64_t ncg = d >> 3;
@@ -244,6 +245,13 @@ __global__ void __launch_bounds__(256, JMIX_CONV_OCC) k_conv_silu16(
     const int64_t rest = tid / ncg;
     const int64_t nck = (L + kConvG - 1) / kConvG;
     const int64_t ck = rest % nck, b = rest / nck;
+    // history row: the sequence's own, or (indexed decode step) its pool slot,
+    // clamped into the pool (a bad slot is reported by the decode kernel)
+    int64_t hb = b;
+    if (sidx) {
+      hb = __ldg(sidx + b);
+      hb = hb < 0 ? 0 : (hb >= n_slots ? n_slots - 1 : hb);
+    }
     const int64_t c0 = cg * 8, t0 = ck * kConvG;
     const int nt = (int)((L - t0) < kConvG ? (L - t0) : kConvG);
     constexpr int kW = kConv - 1;
@@ -276,7 +284,7 @@ __global__ void __launch_bounds__(256, JMIX_CONV_OCC) k_conv_silu16(
 #pragma unroll
         for (int k = 0; k < kW; ++k) {
           const int64_t tau = t0 - kW + k;
-          if (tau < 0) xe[k] = hist ? bf(hist[(b * d + c0 + e) * kW + kW + tau]) : 0.0f;
+          if (tau < 0) xe[k] = hist ? bf(hist[(hb * d + c0 + e) * kW + kW + tau]) : 0.0f;
         }
       }
       float wk[kConv];
@@ -380,6 +388,8 @@ __global__ void __launch_bounds__(kXThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  grid_dep_wait();    // u and the fp16 W_x come from the conv kernel
+  grid_dep_launch();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -472,6 +482,8 @@ __global__ void __launch_bounds__(kNormThreads) k_norms16(
     const W* __restrict__ wb, const W* __restrict__ wc, int64_t Tn, int R, float eps,
     __half* __restrict__ dtn, float* __restrict__ bc) {
   __shared__ float rows[TPB][kMaxP];
+  grid_dep_wait();    // the partial sums come from x_proj
+  grid_dep_launch();
   const int64_t g0 = (int64_t)blockIdx.x * TPB;
   const int P = R + 2 * kN;
   const int64_t stride = Tn * P;
@@ -525,6 +537,8 @@ __global__ void __launch_bounds__(256) k_norms16_warp(
     const W* __restrict__ wb, const W* __restrict__ wc, int64_t Tn, int R, float eps,
     __half* __restrict__ dtn, float* __restrict__ bc) {
   constexpr int kCols = kMaxP / 32;
+  grid_dep_wait();    // the partial sums come from x_proj
+  grid_dep_launch();
   const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
   const int64_t g = (int64_t)blockIdx.x * 8 + wi;
   if (g >= Tn) return;
@@ -662,7 +676,6 @@ ScanPlan scan_plan(int64_t B, int64_t L, int64_t d) {
 constexpr int kProdWarp = 4;
 constexpr int kScanThreads = 32 * (kProdWarp + 1);
 constexpr int kAllBar = 1;  // named barrier of the four compute warps
-constexpr int kWdtBytes = kMaxSlabs * kSC * 128;                  // 64 KB (decode kernel)
 // The scan kernel keeps W_dt's first two 64-wide K slabs in TMEM (the MMA's A
 // operand may come from there) and only the rest in shared memory, which lets
 // three CTAs share an SM.  TMEM per CTA: columns [0, 32) hold the two dt_proj
@@ -955,6 +968,7 @@ __global__ void __launch_bounds__(kScanThreads, kScanCtasPerSm)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  grid_dep_wait();    // dt_n, B/C and the fp16 W_dt come from the kernels before it
   // claim the first unit only now: a CTA that waited in tcgen05.alloc (more
   // CTAs resident than TMEM for) holds no unit that another CTA could wait on
   if (threadIdx.x == 0) unit_slot[0] = atomicAdd(a.counter, 1);
@@ -1205,25 +1219,44 @@ __global__ void __launch_bounds__(kScanThreads, kScanCtasPerSm)
 }
 
 // ------------------------------------------------------------- decode step
-// One token per sequence.  CTA = 128 channels x kDB sequences: dt_proj for the
-// tile on tcgen05 (A = W_dt tile, B = dt_n of the kDB sequences, D in TMEM with
-// lane = channel, column = sequence); then thread = channel walks the kDB
-// sequences: conv + SiLU from the cached conv state, softplus, the 16-state
-// update in place, the gate, and the conv-state shift.  The SSM state read and
-// write (64 B each per (sequence, channel)) is the HBM traffic that bounds it.
-#ifndef JMIX_DEC_DB
-#define JMIX_DEC_DB 16
-#endif
-constexpr int kDB = JMIX_DEC_DB;                          // sequences per CTA (MMA N)
-static_assert(kDB % 16 == 0 && kDB <= 32, "16 or 32 sequences per CTA");
-constexpr int kDecThreads = 160;
-constexpr int kDecDtn = kMaxSlabs * kDB * 128;            // 8 KB
+// One token per row.  The work is B x (d / 128) pairs (row, 128-channel tile);
+// each of the persistent CTAs (two per SM) takes a contiguous, equal share of
+// them in tile-major order, so it changes channel tile at most a few times and
+// keeps that tile's W_dt in TMEM (the dt_proj MMA's A operand).
+//   warp 5: per group of kDB = 16 rows of a tile, TMA-loads the rows' dt_n
+//     (SW128, the MMA's B operand) and B/C rows into one of two buffers and
+//     issues dt_proj into one of two TMEM accumulators (lane = channel,
+//     column = row).
+//   warp 4: per row, loads the row's SSM-state tile ([128 channels x 16] fp32,
+//     8 KB, by a 2-D TMA with 64-byte swizzle), conv-state tile (768 B), x and
+//     z (256 B each) into a ring of kDecStages stages, kDecStages rows ahead.
+//   warps 0..3 (thread = channel): per row, read the stage into registers and
+//     release it, then conv + SiLU, softplus, the 16-state update, the gate,
+//     and store y, the state and the shifted conv state straight to global.
+// The state read and write (64 B each per row and channel) is the HBM traffic
+// that bounds the step.  Rows whose state slot is outside the pool (indexed
+// step) are reported and skipped: nothing is loaded from or stored to a slot
+// outside the pool.
+constexpr int kDB = 16;                                   // rows per dt_proj MMA (N)
+constexpr int kDecThreads = 192;
+constexpr int kDecStages = 8;
+constexpr int kDecState = kSC * kN * 4;                   // 8 KB state tile
+constexpr int kDecConv = kSC * (kConv - 1) * 2;           // 768 B conv-state tile
+constexpr int kDecRow = kSC * 2;                          // 256 B of x or z
+constexpr int kDecStage = 10240;                          // state | conv | x | z, 1 KB aligned
+static_assert(kDecState + kDecConv + 2 * kDecRow <= kDecStage, "decode stage overflow");
+constexpr int kDecDtn = kMaxSlabs * kDB * 128;            // 8 KB (SW128 slabs)
 constexpr int kDecBC = kDB * 2 * kN * 4;                  // 2 KB
-constexpr int kDecSmem = 1024 + kWdtBytes + kDecDtn + kDecBC + 128;
+constexpr int kDecSmem = 1024 + kDecStages * kDecStage + 2 * kDecDtn + 2 * kDecBC + 256;
+static_assert(2 * (kDecSmem + 1024) <= 228 * 1024, "two decode CTAs per SM");
+constexpr uint32_t kDecTmemCols = 256;                    // W_dt [0, 128) | acc 128 + 16 b
+constexpr uint32_t kDecAccCol = 128;
 
 struct DecArgs {
   int64_t B, d;
-  int nslab;
+  int nslab, R;
+  int64_t pairs;       // B * tiles
+  int n_tiles;
   const bf16* x;
   const bf16* z;
   const bf16* conv_w;
@@ -1231,47 +1264,67 @@ struct DecArgs {
   const float* dt_bias;
   const float* A_log;
   const float* D;
-  bf16* conv_state;   // [B, d, 3] in/out
-  float* ssm_state;   // [B, d, 16] in/out
+  const __half* wdt;   // W_dt in fp16 [d, R]
+  bf16* conv_state;    // [B, d, 3] in/out (indexed: [n_slots, d, 3])
+  float* ssm_state;    // [B, d, 16] in/out (indexed: [n_slots, d, 16])
   bf16* y;
   ErrFlags* err;
+  const int* sidx;     // indexed step: state slot of each row, or null (slot = row)
+  int64_t n_slots;
 };
 
-#ifndef JMIX_DEC_OCC
-#define JMIX_DEC_OCC 2
-#endif
-#ifndef JMIX_DEC_AHEAD
-#define JMIX_DEC_AHEAD 2
-#endif
-constexpr int kDecAhead = JMIX_DEC_AHEAD;  // sequences whose inputs are in flight per thread
+// State slot of row b, or -1 when it is outside the pool.
+__device__ __forceinline__ int64_t dec_slot(const DecArgs& a, int64_t b) {
+  if (!a.sidx) return b;
+  const int64_t sl = __ldg(a.sidx + b);
+  return (sl >= 0 && sl < a.n_slots) ? sl : -1;
+}
 
 template <bool kZoh>  // B by zero-order hold (else delta B)
-__global__ void __launch_bounds__(kDecThreads, JMIX_DEC_OCC)
-    k_decode_scan(const __grid_constant__ CUtensorMap tm_wdt,
+__global__ void __launch_bounds__(kDecThreads, 2)
+    k_decode_scan(const __grid_constant__ CUtensorMap tm_state,
                   const __grid_constant__ CUtensorMap tm_dtn,
                   const __grid_constant__ CUtensorMap tm_bc, const DecArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint8_t* wdt_s = smem;
-  uint8_t* dtn_s = smem + kWdtBytes;
-  const float4* bcs = reinterpret_cast<const float4*>(dtn_s + kDecDtn);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(dtn_s + kDecDtn + kDecBC);
-  uint64_t* full = bars;
-  uint64_t* mma_done = bars + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2);
+  uint8_t* stages = smem;                                  // kDecStages x kDecStage
+  uint8_t* dtn_s = stages + kDecStages * kDecStage;        // 2 x kDecDtn
+  uint8_t* bc_s = dtn_s + 2 * kDecDtn;                     // 2 x kDecBC
+  uint64_t* bars = reinterpret_cast<uint64_t*>(bc_s + 2 * kDecBC);
+  uint64_t* full = bars;                                   // [stages] row landed
+  uint64_t* empty = bars + kDecStages;                     // [stages] row read (4 warps)
+  uint64_t* gfull = bars + 2 * kDecStages;                 // [2] dt_n + B/C landed
+  uint64_t* mma_done = gfull + 2;                          // [2] accumulator ready
+  uint64_t* acc_free = mma_done + 2;                       // [2] group done (4 warps)
+  uint64_t* wready = acc_free + 2;                         // W_dt of a new tile in TMEM
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wready + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t c0 = (int64_t)blockIdx.x * kSC;
-  const int64_t b0 = (int64_t)blockIdx.y * kDB;
+  // this CTA's pairs [p0, p1), tile-major: pair p = (tile p / B, row p % B)
+  const int64_t p0 = a.pairs * blockIdx.x / gridDim.x;
+  const int64_t p1 = a.pairs * (blockIdx.x + 1) / gridDim.x;
+  const int64_t ngrp = (a.B + kDB - 1) / kDB;  // row groups per tile
+  // groups this CTA touches: g = tile * ngrp + row / kDB
+  auto grp_of = [&](int64_t p) { return (p / a.B) * ngrp + (p % a.B) / kDB; };
+  const int64_t g0 = p0 < p1 ? grp_of(p0) : 0;
+  const int64_t g1 = p0 < p1 ? grp_of(p1 - 1) + 1 : 0;
 
   if (threadIdx.x == 0) {
-    mbar_init(smem_u32(full), 1);
-    mbar_init(smem_u32(mma_done), 1);
+    for (int s = 0; s < kDecStages; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 4);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&gfull[b]), 1);
+      mbar_init(smem_u32(&mma_done[b]), 1);
+      mbar_init(smem_u32(&acc_free[b]), 4);
+    }
+    mbar_init(smem_u32(wready), 4);
     fence_mbar_init();
   }
-  if (warp == 4) {
-    tmem_alloc(smem_u32(tmem_slot), 32);
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_slot), kDecTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -1280,102 +1333,183 @@ __global__ void __launch_bounds__(kDecThreads, JMIX_DEC_OCC)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 4) {
+    // ---- row streamer: the inputs do not depend on earlier kernels of the
+    // step (the conv kernel only reads the conv states), so it starts at once
     if (lane == 0) {
-      prefetch_tmap(&tm_wdt);
+      prefetch_tmap(&tm_state);
+      for (int64_t p = p0, i = 0; p < p1; ++p, ++i) {
+        const int s = (int)(i % kDecStages);
+        if (i >= kDecStages &&
+            !mbar_wait(smem_u32(&empty[s]), (uint32_t)((i / kDecStages) - 1) & 1u, a.err, 41))
+          break;
+        const int64_t tile = p / a.B, b = p % a.B, c0 = tile * kSC;
+        const int64_t sl = dec_slot(a, b);
+        // channels of this tile that exist (a multiple of 8): the 1-D copies
+        // stop there, so none reads past the end of its buffer
+        const int64_t nc = (a.d - c0) < kSC ? (a.d - c0) : kSC;
+        const uint32_t conv_bytes = (uint32_t)(nc * (kConv - 1) * 2), row_bytes = (uint32_t)(nc * 2);
+        uint8_t* st = stages + s * kDecStage;
+        const uint32_t fb = smem_u32(&full[s]);
+        if (sl >= 0) {
+          mbar_arrive_expect_tx(fb, (uint32_t)kDecState + conv_bytes + 2 * row_bytes);
+          tma_load_2d(smem_u32(st), &tm_state, fb, 0, (int32_t)(sl * a.d + c0));
+          bulk_load(smem_u32(st + kDecState), a.conv_state + (sl * a.d + c0) * (kConv - 1),
+                    conv_bytes, fb);
+        } else {
+          mbar_arrive_expect_tx(fb, 2 * row_bytes);
+        }
+        bulk_load(smem_u32(st + kDecState + kDecConv), a.x + b * a.d + c0, row_bytes, fb);
+        bulk_load(smem_u32(st + kDecState + kDecConv + kDecRow), a.z + b * a.d + c0, row_bytes,
+                  fb);
+      }
+    }
+  } else if (warp == 5) {
+    // ---- dt_proj issuer: dt_n and B/C come from the norms kernel
+    if (lane == 0) {
       prefetch_tmap(&tm_dtn);
       prefetch_tmap(&tm_bc);
-      const uint32_t fb = smem_u32(full);
-      mbar_arrive_expect_tx(fb, (uint32_t)(a.nslab * (kSC + kDB) * 128 + kDecBC));
-      for (int j = 0; j < a.nslab; ++j) {
-        tma_load_2d(smem_u32(wdt_s + j * kSC * 128), &tm_wdt, fb, j * 64, (int32_t)c0);
-        tma_load_2d(smem_u32(dtn_s + j * kDB * 128), &tm_dtn, fb, j * 64, (int32_t)b0);
-      }
-      tma_load_2d(smem_u32(bcs), &tm_bc, fb, 0, (int32_t)b0);
-      if (mbar_wait(fb, 0, a.err, 31)) {
+      grid_dep_wait();
+      const uint32_t idesc = idesc_f16_f32(kSC, kDB);
+      int64_t cur_tile = -1;
+      int ntile = 0;
+      for (int64_t g = g0, k = 0; g < g1; ++g, ++k) {
+        const int bsel = (int)(k & 1);
+        if (k >= 2 &&
+            !mbar_wait(smem_u32(&acc_free[bsel]), (uint32_t)((k >> 1) - 1) & 1u, a.err, 42))
+          break;
+        const int64_t tile = g / ngrp, r0 = (g % ngrp) * kDB;
+        const uint32_t gb = smem_u32(&gfull[bsel]);
+        uint8_t* dtb = dtn_s + bsel * kDecDtn;
+        mbar_arrive_expect_tx(gb, (uint32_t)(a.nslab * kDB * 128 + kDecBC));
+        for (int j = 0; j < a.nslab; ++j)
+          tma_load_2d(smem_u32(dtb + j * kDB * 128), &tm_dtn, gb, j * 64, (int32_t)r0);
+        tma_load_2d(smem_u32(bc_s + bsel * kDecBC), &tm_bc, gb, 0, (int32_t)r0);
+        if (!mbar_wait(gb, (uint32_t)(k >> 1) & 1u, a.err, 43)) break;
+        if (tile != cur_tile) {  // the compute warps put this tile's W_dt into TMEM
+          if (!mbar_wait(smem_u32(wready), (uint32_t)ntile & 1u, a.err, 44)) break;
+          cur_tile = tile;
+          ++ntile;
+        }
         tc_fence_after();
-        const uint32_t idesc = idesc_f16_f32(kSC, kDB);
-        const uint32_t wbase = smem_u32(wdt_s), db = smem_u32(dtn_s);
+        const uint32_t db = smem_u32(dtb);
+        const uint32_t d_tmem = tmem + kDecAccCol + (uint32_t)(bsel * kDB);
         for (int j = 0; j < a.nslab; ++j)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            umma_f16(tmem, sw128_kmajor_desc(wbase + j * kSC * 128 + kk * 32),
-                     sw128_kmajor_desc(db + j * kDB * 128 + kk * 32), idesc,
-                     (j > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(smem_u32(mma_done));
+            umma_f16_ts(d_tmem, tmem + (uint32_t)(j * 32 + kk * 8),
+                        sw128_kmajor_desc(db + j * kDB * 128 + kk * 32), idesc,
+                        (j > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(smem_u32(&mma_done[bsel]));
       }
     }
   } else {
+    // ---- compute warps: thread = channel c0 + cl of the current tile
     const int cl = warp * 32 + lane;
-    const int64_t c = c0 + cl;
-    const bool cok = c < a.d;
-    const int nb = (int)((a.B - b0) < kDB ? (a.B - b0) : kDB);
-    // per-column inputs, loaded kDecAhead columns ahead (they do not depend on delta,
-    // so the first loads go out before the dt_proj accumulator is ready)
-    struct Col {
-      float4 h[4];
-      float s[kConv - 1];
-      bf16 xb;
-      float z;
-    };
-    auto load_col = [&](int j, Col& cd) {
-      if (cok && j < nb) {
-        const int64_t bc = (b0 + j) * a.d + c;
-        const float4* st = reinterpret_cast<const float4*>(a.ssm_state + bc * kN);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) cd.h[q] = st[q];
-        const bf16* cs = a.conv_state + bc * (kConv - 1);
-#pragma unroll
-        for (int k = 0; k < kConv - 1; ++k) cd.s[k] = bf(cs[k]);
-        cd.xb = a.x[bc];
-        cd.z = bf(a.z[bc]);
-      }
-    };
-    Col cbuf[kDecAhead];
-#pragma unroll
-    for (int k = 0; k < kDecAhead; ++k) load_col(k, cbuf[k]);
+    grid_dep_wait();  // W_dt's fp16 copy may come from this step's conv kernel
+    int64_t cur_tile = -1;
+    bool cok = false;
+    int64_t c = 0;
     float2 A2[kN / 2];
     float bias = 0.f, Dc = 0.f, cb = 0.f, cw[kConv] = {0.f, 0.f, 0.f, 0.f};
-    if (cok) {
+    int64_t p = p0, i = 0;
+    bool ok = true;
+    for (int64_t g = g0, k = 0; ok && g < g1; ++g, ++k) {
+      const int bsel = (int)(k & 1);
+      const int64_t tile = g / ngrp, r0 = (g % ngrp) * kDB;
+      if (tile != cur_tile) {
+        // new channel tile: W_dt rows into TMEM (zeros past R and past d), per-channel params
+        cur_tile = tile;
+        c = tile * kSC + cl;
+        cok = c < a.d;
+        const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+        for (int q = 0; q < a.nslab * 2; ++q) {  // 16 columns = 32 K values per step
+          uint32_t v[16];
 #pragma unroll
-      for (int q = 0; q < kN / 2; ++q) {
-        A2[q].x = -expf(a.A_log[c * kN + 2 * q]) * kLog2e;
-        A2[q].y = -expf(a.A_log[c * kN + 2 * q + 1]) * kLog2e;
+          for (int e = 0; e < 4; ++e) {
+            const int kx = q * 32 + e * 8;
+            uint4 w8 = make_uint4(0u, 0u, 0u, 0u);
+            if (cok && kx < a.R) w8 = __ldg(reinterpret_cast<const uint4*>(a.wdt + c * a.R + kx));
+            v[4 * e] = w8.x;
+            v[4 * e + 1] = w8.y;
+            v[4 * e + 2] = w8.z;
+            v[4 * e + 3] = w8.w;
+          }
+          tmem_st16(trow + (uint32_t)(q * 16), v);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(wready));
+#pragma unroll
+        for (int q = 0; q < kN / 2; ++q) {
+          A2[q].x = cok ? -expf(a.A_log[c * kN + 2 * q]) * kLog2e : 0.0f;
+          A2[q].y = cok ? -expf(a.A_log[c * kN + 2 * q + 1]) * kLog2e : 0.0f;
+        }
+        bias = cok ? a.dt_bias[c] : 0.f;
+        Dc = cok ? a.D[c] : 0.f;
+#pragma unroll
+        for (int kx = 0; kx < kConv; ++kx) cw[kx] = cok ? bf(a.conv_w[c * kConv + kx]) : 0.f;
+        cb = cok ? bf(a.conv_b[c]) : 0.f;
       }
-      bias = a.dt_bias[c];
-      Dc = a.D[c];
+      if (!mbar_wait(smem_u32(&mma_done[bsel]), (uint32_t)(k >> 1) & 1u, a.err, 45)) break;
+      tc_fence_after();
+      const uint32_t tacc =
+          tmem + ((uint32_t)(warp * 32) << 16) + kDecAccCol + (uint32_t)(bsel * kDB);
+      const float4* bcs = reinterpret_cast<const float4*>(bc_s + bsel * kDecBC);
+      // the rows of this group that fall in [p0, p1)
+      for (; p < p1 && (p / a.B) == tile && (p % a.B) < r0 + kDB; ++p, ++i) {
+        const int s = (int)(i % kDecStages);
+        const int j = (int)((p % a.B) - r0);
+        if (!mbar_wait(smem_u32(&full[s]), (uint32_t)(i / kDecStages) & 1u, a.err, 46)) {
+          ok = false;
+          break;
+        }
+        const int64_t b = p % a.B;
+        const int64_t sl = dec_slot(a, b);
+        const uint8_t* st = stages + s * kDecStage;
+        uint32_t racc[1];  // this row's dt_proj accumulator (column j of the group)
+        tmem_ld_cols<1>(tacc + (uint32_t)j, racc);
+        tmem_ld_wait();
+        // read the stage (state rows are 64-byte swizzled: 16-byte chunk q of
+        // row cl sits at chunk q ^ ((cl >> 1) & 3)), then release it
+        float2 h[kN / 2];
+        float sv[kConv - 1];
+        float xt, zv;
+        const uint32_t xraw = reinterpret_cast<const uint16_t*>(st + kDecState + kDecConv)[cl];
+        const uint32_t zraw =
+            reinterpret_cast<const uint16_t*>(st + kDecState + kDecConv + kDecRow)[cl];
+        xt = __uint_as_float(xraw << 16);
+        zv = __uint_as_float(zraw << 16);
+        if (sl >= 0) {
 #pragma unroll
-      for (int k = 0; k < kConv; ++k) cw[k] = bf(a.conv_w[c * kConv + k]);
-      cb = bf(a.conv_b[c]);
-    }
-    const bool ok = mbar_wait(smem_u32(mma_done), 0, a.err, 32) &&
-                    mbar_wait(smem_u32(full), 0, a.err, 33);
-    tc_fence_after();
-    uint32_t r[kDB];
+          for (int q = 0; q < 4; ++q) {
+            const float4 v = *reinterpret_cast<const float4*>(
+                st + cl * 64 + 16 * (q ^ ((cl >> 1) & 3)));
+            h[2 * q] = make_float2(v.x, v.y);
+            h[2 * q + 1] = make_float2(v.z, v.w);
+          }
+          const uint16_t* cs = reinterpret_cast<const uint16_t*>(st + kDecState) + cl * 3;
 #pragma unroll
-    for (int q = 0; q < kDB / 16; ++q)
-      tmem_ld16(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(16 * q),
-                *reinterpret_cast<uint32_t(*)[16]>(r + 16 * q));
-    tmem_ld_wait();
-    if (ok && cok) {
+          for (int kx = 0; kx < kConv - 1; ++kx) sv[kx] = __uint_as_float((uint32_t)cs[kx] << 16);
+        } else {
 #pragma unroll
-      for (int j = 0; j < kDB; ++j) {
-        if (j >= nb) break;
-        Col& cd = cbuf[j % kDecAhead];
-        const int64_t bc = (b0 + j) * a.d + c;
-        const float xt = bf(cd.xb);
-        float xc = fmaf(cw[0], cd.s[0], cb);
-        xc = fmaf(cw[1], cd.s[1], xc);
-        xc = fmaf(cw[2], cd.s[2], xc);
+          for (int q = 0; q < kN / 2; ++q) h[q] = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int kx = 0; kx < kConv - 1; ++kx) sv[kx] = 0.f;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
+        if (sl < 0) {
+          if (cl == 0 && atomicExch(&a.err->bad_input, 1u) == 0u) a.err->where = kSiteBadSlot;
+          continue;
+        }
+        float xc = fmaf(cw[0], sv[0], cb);
+        xc = fmaf(cw[1], sv[1], xc);
+        xc = fmaf(cw[2], sv[2], xc);
         xc = fmaf(cw[3], xt, xc);
         const float uv = silu_u(xc);
-        const float dl = softplus_fast(__uint_as_float(r[j]) + bias);
+        const float dl = softplus_fast(__uint_as_float(racc[0]) + bias);
         const float2 dl2 = make_float2(dl, dl), du2 = make_float2(dl * uv, dl * uv);
-        float2 h[kN / 2];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          h[2 * q] = make_float2(cd.h[q].x, cd.h[q].y);
-          h[2 * q + 1] = make_float2(cd.h[q].z, cd.h[q].w);
-        }
         float2 acc[4];
 #pragma unroll
         for (int q4 = 0; q4 < kN / 4; ++q4) {
@@ -1401,28 +1535,31 @@ __global__ void __launch_bounds__(kDecThreads, JMIX_DEC_OCC)
             acc[q4] = half ? __ffma2_rn(Cp, h[q], acc[q4]) : __fmul2_rn(Cp, h[q]);
           }
         }
-        const float2 sa = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
-        const float ys = (sa.x + sa.y) + Dc * uv;
-        const bf16 xkeep = cd.xb;
-        const float s1 = cd.s[1], s2 = cd.s[2], zv = cd.z;
-        load_col(j + kDecAhead, cd);   // refill this slot kDecAhead columns ahead
-        a.y[bc] = __float2bfloat16_rn(ys * silu_gate(zv));
-        float4* st = reinterpret_cast<float4*>(a.ssm_state + bc * kN);
+        if (cok) {  // (no divergent exit: the next row starts with a warp-wide TMEM load)
+          const float2 sa = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
+          const float ys = (sa.x + sa.y) + Dc * uv;
+          a.y[b * a.d + c] = __float2bfloat16_rn(ys * silu_gate(zv));
+          float4* hs = reinterpret_cast<float4*>(a.ssm_state + (sl * a.d + c) * kN);
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          st[q] = make_float4(h[2 * q].x, h[2 * q].y, h[2 * q + 1].x, h[2 * q + 1].y);
-        bf16* cs = a.conv_state + bc * (kConv - 1);
-        cs[0] = __float2bfloat16_rn(s1);
-        cs[1] = __float2bfloat16_rn(s2);
-        cs[2] = xkeep;
+          for (int q = 0; q < 4; ++q)
+            hs[q] = make_float4(h[2 * q].x, h[2 * q].y, h[2 * q + 1].x, h[2 * q + 1].y);
+          uint16_t* cs =
+              reinterpret_cast<uint16_t*>(a.conv_state + (sl * a.d + c) * (kConv - 1));
+          cs[0] = (uint16_t)(__float_as_uint(sv[1]) >> 16);
+          cs[1] = (uint16_t)(__float_as_uint(sv[2]) >> 16);
+          cs[2] = (uint16_t)xraw;
+        }
       }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&acc_free[bsel]));
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 5) {
     tc_fence_after();
-    tmem_dealloc(tmem, 32);
+    tmem_dealloc(tmem, kDecTmemCols);
   }
 }
 
@@ -1445,9 +1582,11 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D tensor map of a row-major [rows, cols] matrix, box [box_rows, box_cols].
-bool make_map(CUtensorMap* m, CUtensorMapDataType dt, size_t esize, const void* base,
-              uint64_t rows, uint64_t cols, uint32_t box_cols, uint32_t box_rows, bool swz) {
+// 2-D tensor map of a row-major [rows, cols] matrix, box [box_rows, box_cols],
+// with the given shared-memory swizzle.
+bool make_map_swz(CUtensorMap* m, CUtensorMapDataType dt, size_t esize, const void* base,
+                  uint64_t rows, uint64_t cols, uint32_t box_cols, uint32_t box_rows,
+                  CUtensorMapSwizzle swz) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {cols, rows};
@@ -1455,9 +1594,15 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, size_t esize, const void* 
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE,
-            swz ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// As make_map_swz with the 128-byte swizzle (swz) or none.
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, size_t esize, const void* base,
+              uint64_t rows, uint64_t cols, uint32_t box_cols, uint32_t box_rows, bool swz) {
+  return make_map_swz(m, dt, esize, base, rows, cols, box_cols, box_rows,
+                      swz ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 struct FastWs {
@@ -1522,7 +1667,32 @@ FastWs fast_layout(const Problem& pr, char* base) {
   w.wx = reinterpret_cast<__half*>(take(P * d * 2));
   w.wdt = reinterpret_cast<__half*>(take(d * R * 2));
   w.bytes = off;
+  if (pr.prepared) {  // fp16 copies made once by jm_prepare_weights: W_x, then W_dt
+    char* pw = static_cast<char*>(const_cast<void*>(pr.prepared));
+    w.wx = reinterpret_cast<__half*>(pw);
+    w.wdt = reinterpret_cast<__half*>(pw + align256(P * d * 2));
+  }
   return w;
+}
+
+// Launch with programmatic stream serialisation: the kernel may start its
+// prologue while the previous kernel on the stream finishes (once every CTA of
+// that kernel has executed griddepcontrol.launch_dependents); it reads the
+// previous kernels' results only after griddepcontrol.wait.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, unsigned block, size_t smem,
+                       cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
 // SM count of the current device, cached per device (threads that race on a
@@ -1549,11 +1719,12 @@ cudaError_t run_fast_fwd(Problem& p) {
   if (e != cudaSuccess) return e;
   launches_begin(p);
 
-  // 1. conv + SiLU -> u (fp16); weights -> fp16
+  // 1. conv + SiLU -> u (fp16); weights -> fp16 (unless prepared once beforehand)
   {
     const int G = p.L >= kConvG ? kConvG : 1;
     const int64_t n_conv = (p.d / 8) * ((p.L + G - 1) / G) * p.B;
-    const int64_t n_wx8 = (int64_t)p.P * p.d / 8, n_wdt8 = p.d * p.R / 8;
+    const int64_t n_wx8 = p.prepared ? 0 : (int64_t)p.P * p.d / 8;
+    const int64_t n_wdt8 = p.prepared ? 0 : p.d * p.R / 8;
     const int64_t total = n_conv + n_wx8 + n_wdt8;
     if (p.cu) {
       const int64_t n_pk = (p.d / 8) * ((p.T + 7) / 8);
@@ -1565,8 +1736,8 @@ cudaError_t run_fast_fwd(Problem& p) {
       auto kern = G == kConvG ? k_conv_silu16<kConvG> : k_conv_silu16<1>;
       kern<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
           (const bf16*)p.x, (const bf16*)p.conv_w, (const bf16*)p.conv_b,
-          (const bf16*)p.init_conv, p.B, p.L, p.d, w.u, n_conv, (const bf16*)p.xproj_w, n_wx8,
-          w.wx, (const bf16*)p.dtproj_w, n_wdt8, w.wdt);
+          (const bf16*)p.init_conv, p.sidx, p.n_slots, p.B, p.L, p.d, w.u, n_conv,
+          (const bf16*)p.xproj_w, n_wx8, w.wx, (const bf16*)p.dtproj_w, n_wdt8, w.wdt);
     }
     launched(p, "k_conv_silu16");
   }
@@ -1598,23 +1769,28 @@ cudaError_t run_fast_fwd(Problem& p) {
       return cudaErrorInvalidValue;
     const int smem = 1024 + kXStages * (kXM * 128 + xa.Ntot * 128) + 256;
     cudaFuncSetAttribute(k_xproj, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    k_xproj<<<dim3((unsigned)mtiles, (unsigned)xa.ksplit), kXThreads, smem, s>>>(tu, tw, xa);
+    e = launch_pdl(k_xproj, dim3((unsigned)mtiles, (unsigned)xa.ksplit), kXThreads, (size_t)smem,
+                   s, tu, tw, xa);
+    if (e != cudaSuccess) return e;
     launched(p, "k_xproj");
   }
   // 3. RMSNorms
   if (w.ksplit <= 4)
-    k_norms16_warp<bf16><<<(unsigned)((p.T + 7) / 8), 256, 0, s>>>(
-        w.part, w.ksplit, (const bf16*)p.dtn_w, (const bf16*)p.bn_w, (const bf16*)p.cn_w, p.T,
-        (int)p.R, p.eps, w.dtn, w.bc);
+    e = launch_pdl(k_norms16_warp<bf16>, dim3((unsigned)((p.T + 7) / 8)), 256, 0, s, w.part,
+                   w.ksplit, (const bf16*)p.dtn_w, (const bf16*)p.bn_w, (const bf16*)p.cn_w, p.T,
+                   (int)p.R, p.eps, w.dtn, w.bc);
   else
-    k_norms16<bf16, 1><<<(unsigned)p.T, kNormThreads, 0, s>>>(
-        w.part, w.ksplit, (const bf16*)p.dtn_w, (const bf16*)p.bn_w, (const bf16*)p.cn_w, p.T,
-        (int)p.R, p.eps, w.dtn, w.bc);
+    e = launch_pdl(k_norms16<bf16, 1>, dim3((unsigned)p.T), kNormThreads, 0, s, w.part, w.ksplit,
+                   (const bf16*)p.dtn_w, (const bf16*)p.bn_w, (const bf16*)p.cn_w, p.T, (int)p.R,
+                   p.eps, w.dtn, w.bc);
+  if (e != cudaSuccess) return e;
   launched(p, "k_norms16");
   // 4. dt_proj + scan + gate
   if (p.decode) {
-    CUtensorMap twdt, tdtn, tbc;
-    if (!make_map(&twdt, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w.wdt, p.d, p.R, 64, kSC, true) ||
+    CUtensorMap tstate, tdtn, tbc;
+    const int64_t slots = p.sidx ? p.n_slots : p.B;
+    if (!make_map_swz(&tstate, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.final_state,
+                      (uint64_t)(slots * p.d), kN, kN, kSC, CU_TENSOR_MAP_SWIZZLE_64B) ||
         !make_map(&tdtn, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w.dtn, p.T, p.R, 64, kDB, true) ||
         !make_map(&tbc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, w.bc, p.T, 2 * kN, 2 * kN, kDB,
                   false))
@@ -1622,7 +1798,10 @@ cudaError_t run_fast_fwd(Problem& p) {
     DecArgs da;
     da.B = p.B;
     da.d = p.d;
+    da.R = (int)p.R;
     da.nslab = (int)((p.R + 63) / 64);
+    da.n_tiles = (int)((p.d + kSC - 1) / kSC);
+    da.pairs = p.B * da.n_tiles;
     da.x = (const bf16*)p.x;
     da.z = (const bf16*)p.z;
     da.conv_w = (const bf16*)p.conv_w;
@@ -1630,14 +1809,18 @@ cudaError_t run_fast_fwd(Problem& p) {
     da.dt_bias = p.dt_bias;
     da.A_log = p.A_log;
     da.D = p.D;
+    da.wdt = w.wdt;
     da.conv_state = (bf16*)p.final_conv;
     da.ssm_state = p.final_state;
     da.y = (bf16*)p.y;
     da.err = err;
+    da.sidx = p.sidx;
+    da.n_slots = slots;
     auto dec_kern = p.zoh ? k_decode_scan<true> : k_decode_scan<false>;
     cudaFuncSetAttribute(dec_kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
-    dec_kern<<<dim3((unsigned)((p.d + kSC - 1) / kSC), (unsigned)((p.B + kDB - 1) / kDB)),
-                    kDecThreads, kDecSmem, s>>>(twdt, tdtn, tbc, da);
+    const int64_t ctas = std::min<int64_t>(2 * num_sms(), da.pairs);
+    e = launch_pdl(dec_kern, (unsigned)ctas, kDecThreads, kDecSmem, s, tstate, tdtn, tbc, da);
+    if (e != cudaSuccess) return e;
     launched(p, "k_decode_scan");
   } else {
     CUtensorMap twdt, tdtn, tbc, tx, tz;
@@ -1690,8 +1873,9 @@ cudaError_t run_fast_fwd(Problem& p) {
     cudaFuncSetAttribute(scan_kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kScanSmem);
     cudaFuncSetAttribute(scan_kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                          cudaSharedmemCarveoutMaxShared);
-    scan_kern<<<(unsigned)(units < slots ? units : slots), kScanThreads, kScanSmem, s>>>(
-        twdt, tdtn, tbc, tx, tz, sa);
+    e = launch_pdl(scan_kern, dim3((unsigned)(units < slots ? units : slots)), kScanThreads,
+                   (size_t)kScanSmem, s, twdt, tdtn, tbc, tx, tz, sa);
+    if (e != cudaSuccess) return e;
     launched(p, "k_scan_fused");
   }
   return cudaGetLastError();
@@ -1700,6 +1884,23 @@ cudaError_t run_fast_fwd(Problem& p) {
 }  // namespace
 
 size_t fast_ws_bytes(const Problem& p) { return fast_layout(p, nullptr).bytes; }
+
+size_t prepared_weights_bytes(int64_t d, int64_t R) {
+  return align256((size_t)(R + 2 * kN) * d * 2) + align256((size_t)d * R * 2);
+}
+
+// The weight-conversion threads of the conv kernel alone (no conv work).
+cudaError_t run_prepare_weights(int64_t d, int64_t R, const void* xproj_w, const void* dtproj_w,
+                                void* out, cudaStream_t s) {
+  const int64_t P = R + 2 * kN;
+  const int64_t n_wx8 = P * d / 8, n_wdt8 = d * R / 8;
+  __half* wx16 = static_cast<__half*>(out);
+  __half* wdt16 = reinterpret_cast<__half*>(static_cast<char*>(out) + align256((size_t)P * d * 2));
+  k_conv_silu16<1><<<(unsigned)((n_wx8 + n_wdt8 + 255) / 256), 256, 0, s>>>(
+      nullptr, nullptr, nullptr, nullptr, nullptr, 0, 0, 1, d, nullptr, 0,
+      (const bf16*)xproj_w, n_wx8, wx16, (const bf16*)dtproj_w, n_wdt8, wdt16);
+  return cudaGetLastError();
+}
 
 void fast_scan_schedule(int64_t B, int64_t L, int64_t d, int* n_parts, int* two_pass) {
   const ScanPlan pl = scan_plan(B, L, d);

@@ -85,6 +85,28 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// 1-D bulk copy of `bytes` (a multiple of 16; both addresses 16-byte aligned)
+// from global memory into this CTA's shared memory; completion counted on `bar`.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// ------------------------------------------------ programmatic dependent launch
+// Waits until the grids this one depends on (launched before it on the stream
+// with programmatic stream serialisation) have completed and their writes are
+// visible; a no-op when the launch had no such dependency.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Lets the next grid on the stream (launched with programmatic stream
+// serialisation) start its prologue once every CTA of this grid got here.
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
@@ -144,14 +166,19 @@ __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// 2, 4, 8 or 16 consecutive 32-bit columns of this thread's TMEM lane (warp-wide).
+// 1, 2, 4, 8 or 16 consecutive 32-bit columns of this thread's TMEM lane (warp-wide).
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]);
 
 template <int NC>
 __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[NC]) {
-  static_assert(NC == 2 || NC == 4 || NC == 8 || NC == 16, "unsupported column count");
+  static_assert(NC == 1 || NC == 2 || NC == 4 || NC == 8 || NC == 16, "unsupported column count");
   if constexpr (NC == 16) {
     tmem_ld16(taddr, r);
+  } else if constexpr (NC == 1) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];"
+                 : "=r"(r[0])
+                 : "r"(taddr)
+                 : "memory");
   } else if constexpr (NC == 2) {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];"
                  : "=r"(r[0]), "=r"(r[1])

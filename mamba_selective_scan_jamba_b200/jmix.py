@@ -29,7 +29,8 @@ EXPORTED = ("jm_mixer_fwd_workspace_size", "jm_mixer_step_workspace_size", "jm_m
             "jm_mixer_fwd_varlen_workspace_size", "jm_mixer_fwd_varlen", "jm_selftest_timeout",
             "jm_layer_fwd_workspace_size", "jm_layer_fwd", "jm_scan_bwd_workspace_size",
             "jm_scan_bwd", "jm_scan_bwd_schedule", "jm_noalloc_poll_error",
-            "jm_noalloc_selftest_timeout")
+            "jm_noalloc_selftest_timeout", "jm_prepared_weights_size", "jm_prepare_weights",
+            "jm_mixer_step_indexed")
 
 
 class jm_dims(ctypes.Structure):
@@ -94,6 +95,14 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
                                           ctypes.POINTER(ctypes.c_int)]
     lib.jm_poll_error.restype = ctypes.c_int
     lib.jm_poll_error.argtypes = [_vp, _vp]
+    lib.jm_prepared_weights_size.restype = ctypes.c_size_t
+    lib.jm_prepared_weights_size.argtypes = [ctypes.POINTER(jm_dims)]
+    lib.jm_prepare_weights.restype = ctypes.c_int
+    lib.jm_prepare_weights.argtypes = [ctypes.POINTER(jm_dims), _vp, _vp, _vp, ctypes.c_size_t,
+                                       _vp]
+    lib.jm_mixer_step_indexed.restype = ctypes.c_int
+    lib.jm_mixer_step_indexed.argtypes = ([ctypes.POINTER(jm_dims), _vp, ctypes.c_int64]
+                                          + [_vp] * 14 + [_vp, _vp, _vp, ctypes.c_size_t, _vp])
     lib.jm_noalloc_poll_error.restype = ctypes.c_int
     lib.jm_noalloc_poll_error.argtypes = [_vp]
     lib.jm_noalloc_selftest_timeout.restype = ctypes.c_int
@@ -245,6 +254,32 @@ def jm_mixer_step(d: jm_dims, x_t, z_t, conv_state, ssm_state, w: Mapping, y_t, 
     st = load().jm_mixer_step(ctypes.byref(d), _ptr(x_t), _ptr(z_t), _ptr(conv_state),
                               _ptr(ssm_state), *_weights(w), _ptr(y_t), _ptr(workspace), ws_bytes,
                               _stream(stream))
+    if check:
+        _check(st)
+    return st
+
+
+def jm_prepared_weights_size(d: jm_dims) -> int:
+    return load().jm_prepared_weights_size(ctypes.byref(d))
+
+
+def jm_prepare_weights(d: jm_dims, xproj_w, dtproj_w, prepared, nbytes: int, stream=None,
+                       check: bool = True) -> int:
+    st = load().jm_prepare_weights(ctypes.byref(d), _ptr(xproj_w), _ptr(dtproj_w), _ptr(prepared),
+                                   nbytes, _stream(stream))
+    if check:
+        _check(st)
+    return st
+
+
+def jm_mixer_step_indexed(d: jm_dims, state_idx, n_slots: int, x_t, z_t, conv_pool, ssm_pool,
+                          w: Mapping, prepared, y_t, workspace, ws_bytes: int, stream=None,
+                          check: bool = True) -> int:
+    """One decode step whose rows use slots state_idx[b] of the state pools."""
+    st = load().jm_mixer_step_indexed(ctypes.byref(d), _ptr(state_idx), n_slots, _ptr(x_t),
+                                      _ptr(z_t), _ptr(conv_pool), _ptr(ssm_pool), *_weights(w),
+                                      _ptr(prepared), _ptr(y_t), _ptr(workspace), ws_bytes,
+                                      _stream(stream))
     if check:
         _check(st)
     return st

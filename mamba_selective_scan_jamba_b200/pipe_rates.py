@@ -25,9 +25,12 @@ DEFAULT_OUT = os.path.join(ROOT, "profiles", "pipe_rates_b200.json")
 
 # op code -> (name, operations per lane per instruction, what is counted)
 OPS = {0: ("ex2", 1, "ex2.approx.ftz.f32"), 1: ("tanh", 1, "tanh.approx.f32 (+1 add)"),
-       2: ("rcp", 1, "rcp.approx.ftz.f32"), 3: ("ffma", 1, "fma.rn.f32"),
+       2: ("rcp", 1, "rcp.approx.ftz.f32 (+1 add)"), 3: ("ffma", 1, "fma.rn.f32"),
        4: ("ffma2", 2, "fma.rn.f32x2, 2 FMAs per lane"),
        5: ("ex2_with_2ffma2", 1, "ex2 counted; 2 fma.rn.f32x2 issued beside each")}
+# the scan's recurrence alone: 16 ex2 per token and thread (counted per ex2)
+RECURRENCE = {6: ("recurrence_bc_smem", 16, "16-state update, B/C rows from shared memory"),
+              7: ("recurrence_bc_regs", 16, "16-state update, B/C in registers")}
 
 
 def source_sha256() -> str:
@@ -72,10 +75,16 @@ def measure(target_ms: float = 60.0, reps: int = 5) -> dict:
              in OPS.items()]
     cases += [(op, OPS[op][0] + "_2warps_per_smsp", OPS[op][1], OPS[op][2], sms * 2, 128)
               for op in (0, 5)]
+    # the recurrence at the scan kernel's occupancy (2 compute warps per
+    # scheduler) and at 4 warps per scheduler
+    for op, (name, per_lane, what) in RECURRENCE.items():
+        cases.append((op, name + "_2warps_per_smsp", per_lane / chains, what, sms * 2, 128))
+        cases.append((op, name + "_4warps_per_smsp", per_lane / chains, what, sms * 4, 128))
     for op, name, per_lane, what, nb, nt in cases:
-        iters = 256
+        iters = 4096
+        run(op, iters, nb, nt)              # first launch of this kernel: module load
         ms = run(op, iters, nb, nt)
-        iters = max(256, int(iters * target_ms / max(ms, 1e-3)))
+        iters = max(4096, int(iters * target_ms / max(ms, 1e-3)))
         times = [run(op, iters, nb, nt) for _ in range(reps)]
         ms = statistics.median(times)
         ops = float(nb) * nt * iters * chains * per_lane
@@ -86,8 +95,10 @@ def measure(target_ms: float = 60.0, reps: int = 5) -> dict:
     sampler.stop()
     clocks = sampler.summary(t0, t1)
     mhz = clocks.get("sm_mhz") or 0.0
-    for r in rates.values():
+    for name, r in rates.items():
         r["per_clk_per_sm"] = r["ops_per_s"] / (mhz * 1e6 * sms) if mhz else None
+        # a launch that took far less than intended did not do the work it counts
+        assert r["ms_median"] > 0.25 * target_ms, (name, r)
     return {"gpu": props.name, "sms": sms, "chains_per_thread": chains, "clocks": clocks, "rates": rates,
             "source": "mamba_selective_scan_jamba_b200/csrc/pipe_rates.cu",
             "source_sha256": source_sha256(),

@@ -293,3 +293,44 @@ def test_layer_host_checks(lib):
     st = jmix.jm_layer_fwd(d, 128, None, FAKE, W, FAKE, FAKE, FAKE, FAKE, n, stream=0,
                            check=False)
     assert st == jmix.JM_ERR_INVALID_ARG and "hidden" in jmix.jm_last_error()
+
+
+def test_prepare_weights_host_checks(lib):
+    d = jmix.dims(2, 1, 8192, 256)
+    n = jmix.jm_prepared_weights_size(d)
+    assert n == 288 * 8192 * 2 + 8192 * 256 * 2           # both multiples of 256 here
+    assert jmix.jm_prepared_weights_size(jmix.dims(2, 1, 8192, 256, jmix.JM_F32)) == 0
+    ok = dict(xproj_w=FAKE, dtproj_w=FAKE, prepared=FAKE, nbytes=n)
+
+    def call(dm=d, **over):
+        a = dict(ok, **over)
+        return jmix.jm_prepare_weights(dm, a["xproj_w"], a["dtproj_w"], a["prepared"],
+                                       a["nbytes"], stream=0, check=False)
+    assert call(xproj_w=None) == jmix.JM_ERR_INVALID_ARG
+    assert call(prepared=FAKE + 16) == jmix.JM_ERR_INVALID_ARG     # not 256-byte aligned
+    assert call(nbytes=n - 1) == jmix.JM_ERR_WORKSPACE
+    assert call(dm=jmix.dims(2, 1, 8192, 256, jmix.JM_F32)) == jmix.JM_ERR_UNSUPPORTED
+
+
+def test_indexed_step_host_checks(lib):
+    d = jmix.dims(4, 1, 256, 16)
+    n = jmix.jm_mixer_step_workspace_size(d)
+    W = {k: FAKE for k in jmix.WEIGHT_NAMES}
+    ok = dict(idx=FAKE, slots=16, x=FAKE, z=FAKE + (1 << 36), cp=FAKE, sp=FAKE, prep=None,
+              y=FAKE + (2 << 36), ws=FAKE, n=n)
+
+    def call(dm=d, **over):
+        a = dict(ok, **over)
+        return jmix.jm_mixer_step_indexed(dm, a["idx"], a["slots"], a["x"], a["z"], a["cp"],
+                                          a["sp"], W, a["prep"], a["y"], a["ws"], a["n"], stream=0,
+                                          check=False)
+    assert call(idx=None) == jmix.JM_ERR_INVALID_ARG
+    assert call(idx=FAKE + 2) == jmix.JM_ERR_INVALID_ARG              # not 4-byte aligned
+    assert call(slots=3) == jmix.JM_ERR_INVALID_ARG                   # fewer slots than rows
+    assert "n_slots" in jmix.jm_last_error()
+    assert call(slots=1 << 31) == jmix.JM_ERR_INVALID_ARG
+    assert call(cp=None) == jmix.JM_ERR_INVALID_ARG
+    assert call(prep=FAKE + 16) == jmix.JM_ERR_INVALID_ARG           # not 256-byte aligned
+    assert call(n=n - 1) == jmix.JM_ERR_WORKSPACE
+    assert call(dm=jmix.dims(4, 2, 256, 16)) == jmix.JM_ERR_INVALID_ARG   # seqlen must be 1
+    assert call(dm=jmix.dims(4, 1, 256, 16, jmix.JM_F32)) == jmix.JM_ERR_UNSUPPORTED

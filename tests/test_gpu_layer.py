@@ -1,5 +1,8 @@
 """jm_layer_fwd: in_proj -> mixer core -> out_proj on cuda:0, against the fp64
-layer oracle (matrix products in fp64 around the mixer oracle).
+layer oracle (matrix products in fp64 around the mixer oracle).  The cases
+cover the tcgen05 GEMM's edges: ragged row tiles, one partial row tile, and
+enough tiles that every persistent CTA runs many, alternating its two TMEM
+accumulators and wrapping its stage ring.
 
 Gates: out within 2e-2 max(1, |ref|) of the exact oracle (as y); the final
 SSM state within 2e-3 max(1, |ref|) of the mirror oracle fed with x, z rounded
@@ -19,7 +22,11 @@ from tests.helpers import f64, max_scaled_err
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("B,L,d,R,d_model", [(2, 130, 512, 32, 256), (1, 64, 8192, 256, 4096)])
+@pytest.mark.parametrize("B,L,d,R,d_model", [
+    (2, 130, 512, 32, 256),       # ragged row tiles; in_proj N = 1024, out_proj N = 256
+    (1, 64, 8192, 256, 4096),     # Jamba's d_model / d_inner, a single partial row tile
+    (2, 4096, 4096, 128, 2048),   # many tiles per CTA: 2048 in_proj and 512 out_proj tiles
+])
 def test_layer_matches_oracle(B, L, d, R, d_model):
     import torch
     from mamba_selective_scan_jamba_b200 import devio, jmix
