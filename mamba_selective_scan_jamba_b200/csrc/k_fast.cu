@@ -274,17 +274,31 @@ __global__ void __launch_bounds__(256, JMIX_CONV_OCC) k_conv_silu16(
     const uint4 bq = __ldg(reinterpret_cast<const uint4*>(conv_b + c0));
     uint32_t outp[kConvG][4];  // [token][channel pair] packed fp16x2
     float sv_even[kConvG];     // SiLU of the pair's even channel, per token
+    // the 8 channels' cached conv states (3 taps each, oldest first): 48
+    // contiguous bytes, 16-byte aligned since c0 is a multiple of 8
+    uint4 hq[3] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u),
+                   make_uint4(0u, 0u, 0u, 0u)};
+    if (t0 < kW && hist) {
+      const uint4* hp = reinterpret_cast<const uint4*>(hist + (hb * d + c0) * kW);
+#pragma unroll
+      for (int q = 0; q < 3; ++q) hq[q] = __ldg(hp + q);
+    }
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       float xe[kW + kConvG];
 #pragma unroll
       for (int i = 0; i < kW + kConvG; ++i) xe[i] = bf16_lane(rows[i], e);
       if (t0 < kW) {
-        // taps before the sequence start: the cached conv state, or zero
+        // taps before the sequence start: the cached conv state (zero without one);
+        // history slot kW + tau of channel e is element 3 e + kW + tau of the 24
+        static_assert(kConv - 1 == 3, "three history taps");
+        float hv[kW];
+#pragma unroll
+        for (int k = 0; k < kW; ++k) hv[k] = bf16_lane(hq[(e * kW + k) >> 3], (e * kW + k) & 7);
 #pragma unroll
         for (int k = 0; k < kW; ++k) {
-          const int64_t tau = t0 - kW + k;
-          if (tau < 0) xe[k] = hist ? bf(hist[(hb * d + c0 + e) * kW + kW + tau]) : 0.0f;
+          const int64_t slot = t0 + k;  // = kW + tau
+          if (slot < kW) xe[k] = slot == 0 ? hv[0] : (slot == 1 ? hv[1] : hv[2]);
         }
       }
       float wk[kConv];
@@ -352,8 +366,9 @@ __global__ void __launch_bounds__(kXThreads, 1)
     k_xproj(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_w,
             const XprojArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  // (offset arithmetic on the shared array keeps its address space known, so
+  // accesses through these pointers compile to shared-memory loads)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int a_bytes = kXM * 128;
   const int b_bytes = a.Ntot * 128;
   const int stage_bytes = a_bytes + b_bytes;
@@ -630,8 +645,11 @@ struct ScanPlan {
   int two_pass = 0;
 };
 
+#ifndef JMIX_SCAN_LEAD
+#define JMIX_SCAN_LEAD 0    // 4-warp CTAs whose thread 0 also feeds the ring: 3 CTAs per SM
+#endif
 #ifndef JMIX_SCAN_CTAS
-#define JMIX_SCAN_CTAS 2
+#define JMIX_SCAN_CTAS (JMIX_SCAN_LEAD ? 3 : 2)
 #endif
 // CTAs of the scan kernel resident on each of a B200's 148 SMs.
 constexpr int kScanCtasPerSm = JMIX_SCAN_CTAS;
@@ -695,10 +713,10 @@ constexpr uint32_t kScanTmemCols = kScanTmemNeed <= 64 ? 64 : kScanTmemNeed <= 1
                                    : kScanTmemNeed <= 256 ? 256 : 512;
 static_assert(kScanStages * kSQ <= (int)kTmemWdtCol, "accumulators overlap the W_dt columns");
 static_assert(kScanCtasPerSm * kScanTmemCols <= 512, "TMEM of the resident CTAs exceeds 512 columns");
-constexpr int kDtnStage = kMaxSlabs * kSQ * 128;                  // 8 KB (SW128 slabs)
-constexpr int kXStage = kSQ * kSC * 2;                            // 4 KB (x or z tile)
-constexpr int kBCStage = kSQ * 2 * kN * 4;                        // 2 KB
-constexpr int kStageBytes = kDtnStage + 2 * kXStage + kBCStage;   // 18 KB
+constexpr int kDtnStage = kMaxSlabs * kSQ * 128;                  // 16 KB at kSQ = 32 (SW128)
+constexpr int kXStage = kSQ * kSC * 2;                            // 8 KB (x or z tile)
+constexpr int kBCStage = kSQ * 2 * kN * 4;                        // 4 KB
+constexpr int kStageBytes = kDtnStage + 2 * kXStage + kBCStage;   // 36 KB
 #ifndef JMIX_SCAN_G
 #define JMIX_SCAN_G 8
 #endif
@@ -781,8 +799,144 @@ __device__ __forceinline__ float2 zoh_factor(float2 x, float2 da, float2 inv_a, 
                      fabsf(y.y) < 0.03125f ? small.y : big.y);
 }
 
-template <bool kOut, bool kZoh>
-__device__ __forceinline__ void scan_chunks(const ScanArgs& a, const uint8_t* stage0,
+
+#ifndef JMIX_SCAN_SLEEP
+#define JMIX_SCAN_SLEEP 256  // ns the scan's producer sleeps between barrier tries (0: spin)
+#endif
+#ifndef JMIX_SCAN_FULL
+#define JMIX_SCAN_FULL 1     // chunks of a full kSQ tokens take a path without per-token checks
+#endif
+
+// The per-token terms of one group of kG tokens: delta, the factor of B in the
+// update (delta u, or u under zero-order hold), D u and SiLU(z).
+struct TokTerms {
+  float dl[kG], du[kG], dsk[kG], gz[kG];
+};
+
+// Per-token terms of tokens g0t .. g0t + kG - 1 of the current chunk: u =
+// SiLU(conv) recomputed in float32 from x (the conv window xw slides over the
+// live tokens), delta = softplus(dt_proj accumulator r + bias), and for kOut
+// D u and SiLU(z).  Without kOut the live deltas are summed into csum.
+template <bool kOut, bool kZoh, bool kFull>
+__device__ __forceinline__ void scan_terms(const uint32_t (&r)[kG], const bf16* xs, const bf16* zs,
+                                           int g0t, int nt, int cl, float (&xw)[kConv - 1],
+                                           const float (&cw)[kConv], float cb, float bias,
+                                           float Dc, TokTerms& T, float& csum) {
+#pragma unroll
+  for (int i = 0; i < kG; ++i) {
+    const float xt = bf(xs[(g0t + i) * kSC + cl]);
+    float xc = fmaf(cw[0], xw[0], cb);
+    xc = fmaf(cw[1], xw[1], xc);
+    xc = fmaf(cw[2], xw[2], xc);
+    xc = fmaf(cw[3], xt, xc);
+    const float uv = silu_newton(xc);
+    const bool live = kFull || g0t + i < nt;
+    if (live) {
+      xw[0] = xw[1];
+      xw[1] = xw[2];
+      xw[2] = xt;
+    }
+    T.dl[i] = softplus_fast(__uint_as_float(r[i]) + bias);
+    T.du[i] = kZoh ? uv : T.dl[i] * uv;  // zero-order hold: u (the factor is per state)
+    if constexpr (kOut) {
+      T.dsk[i] = Dc * uv;
+      T.gz[i] = silu_gate(bf(zs[(g0t + i) * kSC + cl]));
+    } else {
+      csum += live ? T.dl[i] : 0.0f;
+    }
+  }
+}
+
+// The 16-state recurrence over tokens g0t .. g0t + kG - 1 (those below nt) of
+// the current chunk, with B and C rows from the stage; for kOut, y = (C.h + D u)
+// SiLU(z) is stored to yrow (row stride d) when the channel exists.
+template <bool kOut, bool kZoh, bool kFull, bool kYS>
+__device__ __forceinline__ void scan_recur(const TokTerms& T, const float4* bcs, int g0t, int nt,
+                                           float2 (&h)[kN / 2], const float2 (&A2)[kN / 2],
+                                           const float2 (&invA)[kN / 2], bf16* yrow,
+                                           int64_t tbase, int64_t d, bool cok, bf16* ys_smem,
+                                           int cl) {
+#pragma unroll
+  for (int i = 0; i < kG; ++i) {
+    const int t = g0t + i;
+    if (!kFull && t >= nt) break;
+    const float2 dl2 = make_float2(T.dl[i], T.dl[i]);
+    const float2 du2 = make_float2(T.du[i], T.du[i]);
+    float2 acc[4];
+#pragma unroll
+    for (int q4 = 0; q4 < kN / 4; ++q4) {
+      const float4 Bq = bcs[t * 8 + q4];
+      float4 Cq;
+      if constexpr (kOut) Cq = bcs[t * 8 + 4 + q4];
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int q = q4 * 2 + half;
+        const float2 Bp = half ? make_float2(Bq.z, Bq.w) : make_float2(Bq.x, Bq.y);
+        const float2 x = __fmul2_rn(dl2, A2[q]);
+        float2 da;
+        da.x = ex2_approx(x.x);
+        da.y = ex2_approx(x.y);
+        if constexpr (kZoh)
+          h[q] = __ffma2_rn(da, h[q],
+                            __fmul2_rn(__fmul2_rn(zoh_factor(x, da, invA[q], dl2), du2), Bp));
+        else
+          h[q] = __ffma2_rn(da, h[q], __fmul2_rn(du2, Bp));
+        if constexpr (kOut) {
+          // four independent partial sums of C.h (short dependency chains)
+          const float2 Cp = half ? make_float2(Cq.z, Cq.w) : make_float2(Cq.x, Cq.y);
+          acc[q4] = half ? __ffma2_rn(Cp, h[q], acc[q4]) : __fmul2_rn(Cp, h[q]);
+        }
+      }
+    }
+    if constexpr (kOut) {
+      const float2 s01 = __fadd2_rn(acc[0], acc[1]);
+      const float2 s23 = __fadd2_rn(acc[2], acc[3]);
+      const float2 sa = __fadd2_rn(s01, s23);
+      const float ys = (sa.x + sa.y) + T.dsk[i];
+      if constexpr (kYS)  // into the stage's x tile (token t's x is already read)
+        ys_smem[t * kSC + cl] = __float2bfloat16_rn(ys * T.gz[i]);
+      else if (cok)
+        yrow[(tbase + t) * d] = __float2bfloat16_rn(ys * T.gz[i]);
+    }
+  }
+}
+
+// The groups of one chunk: tokens 0 .. nt - 1 (kFull: nt == kSQ, so no
+// per-token live checks are needed).
+template <bool kOut, bool kZoh, bool kFull, bool kYS, class GroupHook>
+__device__ __forceinline__ void scan_chunk_body(uint32_t tacc, const bf16* xs, const bf16* zs,
+                                                const float4* bcs, int nt, int cl,
+                                                float (&xw)[kConv - 1], const float (&cw)[kConv],
+                                                float cb, float bias, float Dc,
+                                                float2 (&h)[kN / 2], const float2 (&A2)[kN / 2],
+                                                const float2 (&invA)[kN / 2], bf16* yrow,
+                                                int64_t tbase, int64_t d, bool cok, float& csum,
+                                                const GroupHook& ghook) {
+#pragma unroll 1
+    for (int g0t = 0; g0t < nt; g0t += kG) {
+      uint32_t r[kG];
+      tmem_ld_cols<kG>(tacc + (uint32_t)g0t, r);
+      tmem_ld_wait();
+      TokTerms T;
+      scan_terms<kOut, kZoh, kFull>(r, xs, zs, g0t, nt, cl, xw, cw, cb, bias, Dc, T, csum);
+      scan_recur<kOut, kZoh, kFull, kYS>(T, bcs, g0t, nt, h, A2, invA, yrow, tbase, d, cok,
+                                         const_cast<bf16*>(xs), cl);
+      ghook();
+    }
+}
+
+#ifndef JMIX_SCAN_YTMA
+#define JMIX_SCAN_YTMA 1    // y of whole chunks leaves through the stage by TMA
+#endif
+// Whether a chunk of nt tokens of an output unit stores its y tile by TMA from
+// the stage (whole chunks of fixed-length sequences), else thread by thread.
+__device__ __forceinline__ bool y_by_tma(const ScanArgs& a, bool out, int nt) {
+  return JMIX_SCAN_YTMA && out && !a.cu && nt == kSQ;
+}
+
+template <bool kOut, bool kZoh, bool kLead, class Hook>
+__device__ __forceinline__ void scan_chunks(const Hook& hook, const ScanArgs& a,
+                                            const uint8_t* stage0,
                                             uint64_t* full, uint64_t* mma_done, uint64_t* empty,
                                             uint32_t tmem, int warp, int lane, int kg0, int kb,
                                             int nch, int64_t Lb, bool cok, bf16* yrow,
@@ -807,81 +961,25 @@ __device__ __forceinline__ void scan_chunks(const ScanArgs& a, const uint8_t* st
     const int nt = (int)((Lb - tbase) < kSQ ? (Lb - tbase) : kSQ);
     const uint32_t tacc = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(s * kSQ);
     float csum = 0.0f;
-#pragma unroll 1
-    for (int g0t = 0; g0t < nt; g0t += kG) {
-      uint32_t r[kG];
-      tmem_ld_cols<kG>(tacc + (uint32_t)g0t, r);
-      tmem_ld_wait();
-      // per-token terms: u = SiLU(conv) in float32, delta, delta*u, D*u, SiLU(z)
-      float dl[kG], du[kG], dsk[kG], gz[kG];
-#pragma unroll
-      for (int i = 0; i < kG; ++i) {
-        const float xt = bf(xs[(g0t + i) * kSC + cl]);
-        float xc = fmaf(cw[0], xw[0], cb);
-        xc = fmaf(cw[1], xw[1], xc);
-        xc = fmaf(cw[2], xw[2], xc);
-        xc = fmaf(cw[3], xt, xc);
-        const float uv = silu_newton(xc);
-        const bool live = g0t + i < nt;
-        if (live) {
-          xw[0] = xw[1];
-          xw[1] = xw[2];
-          xw[2] = xt;
-        }
-        dl[i] = softplus_fast(__uint_as_float(r[i]) + bias);
-        du[i] = kZoh ? uv : dl[i] * uv;  // zero-order hold: u (the factor is per state)
-        if constexpr (kOut) {
-          dsk[i] = Dc * uv;
-          gz[i] = silu_gate(bf(zs[(g0t + i) * kSC + cl]));
-        } else {
-          csum += live ? dl[i] : 0.0f;
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < kG; ++i) {
-        const int t = g0t + i;
-        if (t >= nt) break;
-        const float2 dl2 = make_float2(dl[i], dl[i]);
-        const float2 du2 = make_float2(du[i], du[i]);
-        float2 acc[4];
-#pragma unroll
-        for (int q4 = 0; q4 < kN / 4; ++q4) {
-          const float4 Bq = bcs[t * 8 + q4];
-          float4 Cq;
-          if constexpr (kOut) Cq = bcs[t * 8 + 4 + q4];
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            const int q = q4 * 2 + half;
-            const float2 Bp = half ? make_float2(Bq.z, Bq.w) : make_float2(Bq.x, Bq.y);
-            const float2 x = __fmul2_rn(dl2, A2[q]);
-            float2 da;
-            da.x = ex2_approx(x.x);
-            da.y = ex2_approx(x.y);
-            if constexpr (kZoh)
-              h[q] = __ffma2_rn(da, h[q],
-                                __fmul2_rn(__fmul2_rn(zoh_factor(x, da, invA[q], dl2), du2), Bp));
-            else
-              h[q] = __ffma2_rn(da, h[q], __fmul2_rn(du2, Bp));
-            if constexpr (kOut) {
-              // four independent partial sums of C.h (short dependency chains)
-              const float2 Cp = half ? make_float2(Cq.z, Cq.w) : make_float2(Cq.x, Cq.y);
-              acc[q4] = half ? __ffma2_rn(Cp, h[q], acc[q4]) : __fmul2_rn(Cp, h[q]);
-            }
-          }
-        }
-        if constexpr (kOut) {
-          const float2 s01 = __fadd2_rn(acc[0], acc[1]);
-          const float2 s23 = __fadd2_rn(acc[2], acc[3]);
-          const float2 sa = __fadd2_rn(s01, s23);
-          const float ys = (sa.x + sa.y) + dsk[i];
-          if (cok) yrow[(tbase + t) * a.d] = __float2bfloat16_rn(ys * gz[i]);
-        }
-      }
-    }
+    // whole chunks of fixed-length sequences leave y in the stage; the producer
+    // stores the [32 x 128] y tile by TMA (partial chunks store y directly)
+    const bool ytile = y_by_tma(a, kOut && !kLead, nt);
+    auto ghook = [&]() { hook(k, false); };
+    if (ytile)
+      scan_chunk_body<kOut, kZoh, true, true>(tacc, xs, zs, bcs, nt, cl, xw, cw, cb, bias, Dc, h,
+                                              A2, invA, yrow, tbase, a.d, cok, csum, ghook);
+    else if (JMIX_SCAN_FULL && nt == kSQ)
+      scan_chunk_body<kOut, kZoh, true, false>(tacc, xs, zs, bcs, nt, cl, xw, cw, cb, bias, Dc, h,
+                                               A2, invA, yrow, tbase, a.d, cok, csum, ghook);
+    else
+      scan_chunk_body<kOut, kZoh, false, false>(tacc, xs, zs, bcs, nt, cl, xw, cw, cb, bias, Dc, h,
+                                                A2, invA, yrow, tbase, a.d, cok, csum, ghook);
     if constexpr (!kOut) ssum += csum;
+    if (ytile) fence_proxy_async_smem();  // y in the stage, before the TMA store reads it
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
+    hook(k, true);
   }
 }
 
@@ -923,15 +1021,19 @@ __global__ void __launch_bounds__(1024) k_order_by_length(const int* __restrict_
 // Every unit that waits waits only for units that come before it in claim
 // order, and a claimed unit is running or queued behind one with a smaller
 // index on its CTA, so every wait ends; each is still bounded (2 s).
-template <bool kZoh>  // B by zero-order hold (else delta B)
-__global__ void __launch_bounds__(kScanThreads, kScanCtasPerSm)
+// kLead: no producer warp; thread 0 issues the ring's TMA loads and the dt_proj
+// MMAs between its own groups of tokens (4 warps per CTA, 3 CTAs per SM).
+template <bool kZoh, bool kLead>  // B by zero-order hold (else delta B)
+__global__ void __launch_bounds__(kLead ? 128 : kScanThreads, kScanCtasPerSm)
     k_scan_fused(const __grid_constant__ CUtensorMap tm_wdt,
                  const __grid_constant__ CUtensorMap tm_dtn,
                  const __grid_constant__ CUtensorMap tm_bc, const __grid_constant__ CUtensorMap tm_x,
-                 const __grid_constant__ CUtensorMap tm_z, const ScanArgs a) {
+                 const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_y,
+                 const ScanArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  // (offset arithmetic on the shared array keeps its address space known, so
+  // accesses through these pointers compile to shared-memory loads)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* wdt_s = smem;                  // W_dt K slabs 2.. : [128 ch x 64] each (SW128)
   uint8_t* stage0 = smem + kScanWdtBytes;  // 2 x {dt_n (SW128), x tile, z tile, B/C rows}
   uint64_t* bars = reinterpret_cast<uint64_t*>(stage0 + kScanStages * kStageBytes);
@@ -960,7 +1062,9 @@ __global__ void __launch_bounds__(kScanThreads, kScanCtasPerSm)
     mbar_init(smem_u32(wready), 4);
     fence_mbar_init();
   }
-  if (warp == kProdWarp) {
+  constexpr int kAllocWarp = kLead ? 0 : kProdWarp;
+  constexpr int kFeedThread = kLead ? 0 : 32 * kProdWarp;  // claims units, feeds the ring
+  if (warp == kAllocWarp) {
     tmem_alloc(smem_u32(tmem_slot), kScanTmemCols);
     tmem_relinquish();
   }
@@ -980,7 +1084,7 @@ __global__ void __launch_bounds__(kScanThreads, kScanCtasPerSm)
     const int unit = unit_slot[it & 1];
     if (unit >= n_units) break;
     // claim the next unit early, so that its number is ready when this one ends
-    if (threadIdx.x == 32 * kProdWarp)
+    if (threadIdx.x == kFeedThread)
       unit_slot[(it + 1) & 1] = *(volatile unsigned*)&a.err->timeout ? n_units
                                                                       : atomicAdd(a.counter, 1);
     const bool out = unit >= n_state;
@@ -1010,15 +1114,23 @@ __global__ void __launch_bounds__(kScanThreads, kScanCtasPerSm)
     const int nch = (int)((int64_t)nch_all * (part + 1) / P) - kb;
     const int64_t hslot = (int64_t)pair * P + part;  // this part's hand-over slot
 
-    if (warp == kProdWarp) {
-      if (lane == 0 && nch > 0) {
+    // ---- feeding the ring (the producer warp's lane 0, or thread 0 with kLead):
+    // its waits last about a chunk of the compute warps' work, so the producer
+    // sleeps between tries and its scheduler's slots go to the compute warps
+        auto kWait = [](uint32_t bar, uint32_t par, ErrFlags* e, unsigned site) {
+          return JMIX_SCAN_SLEEP > 0 && !kLead
+                     ? mbar_wait_sleep(bar, par, e, site, JMIX_SCAN_SLEEP)
+                     : mbar_wait(bar, par, e, site);
+        };
         const uint32_t wb = smem_u32(wfull);
-        if (a.nslab > nslab_t) {
-          mbar_arrive_expect_tx(wb, (uint32_t)((a.nslab - nslab_t) * kSC * 128));
-          for (int j = nslab_t; j < a.nslab; ++j)
-            tma_load_2d(smem_u32(wdt_s + (j - nslab_t) * kSC * 128), &tm_wdt, wb, j * 64,
-                        (int32_t)c0);
-        }
+        auto issue_wdt = [&]() {  // W_dt K slabs past the TMEM ones, into shared memory
+          if (a.nslab > nslab_t) {
+            mbar_arrive_expect_tx(wb, (uint32_t)((a.nslab - nslab_t) * kSC * 128));
+            for (int j = nslab_t; j < a.nslab; ++j)
+              tma_load_2d(smem_u32(wdt_s + (j - nslab_t) * kSC * 128), &tm_wdt, wb, j * 64,
+                          (int32_t)c0);
+          }
+        };
         const uint32_t stage_tx =
             (uint32_t)(a.nslab * kSQ * 128 + (out ? 2 : 1) * kXStage + kBCStage);
         auto issue_stage = [&](int k) {  // k: chunk of this unit
@@ -1033,11 +1145,23 @@ __global__ void __launch_bounds__(kScanThreads, kScanCtasPerSm)
           if (out) tma_load_2d(smem_u32(st + kDtnStage + kXStage), &tm_z, fb, (int32_t)c0, row);
           tma_load_2d(smem_u32(st + kDtnStage + 2 * kXStage), &tm_bc, fb, 0, row);
         };
+        // y tile of chunk k (whole chunks of fixed-length sequences): the compute
+        // warps left it in the stage's x tile; one TMA store per chunk
+        auto store_y = [&](int k) -> bool {
+          if (!y_by_tma(a, out, (int)((Lb - (int64_t)(kb + k) * kSQ) < kSQ
+                                          ? (Lb - (int64_t)(kb + k) * kSQ) : kSQ)))
+            return false;
+          const int s = (kg0 + k) % kScanStages;
+          tma_store_3d(&tm_y, smem_u32(stage0 + s * kStageBytes + kDtnStage), (int32_t)c0,
+                       (int32_t)((kb + k) * kSQ), (int32_t)b);
+          bulk_commit();
+          return true;
+        };
         const uint32_t idesc = idesc_f16_f32(kSC, kSQ);
         auto issue_mma = [&](int k) -> bool {
           const int kg = kg0 + k;
           const int s = kg % kScanStages;
-          if (!mbar_wait(smem_u32(&full[s]), (uint32_t)(kg / kScanStages) & 1u, a.err, 22))
+          if (!kWait(smem_u32(&full[s]), (uint32_t)(kg / kScanStages) & 1u, a.err, 22))
             return false;
           tc_fence_after();
           const uint32_t wbase = smem_u32(wdt_s), db = smem_u32(stage0 + s * kStageBytes);
@@ -1057,11 +1181,14 @@ __global__ void __launch_bounds__(kScanThreads, kScanCtasPerSm)
           umma_commit(smem_u32(&mma_done[s]));
           return true;
         };
+    if (!kLead && warp == kProdWarp) {
+      if (lane == 0 && nch > 0) {
+        issue_wdt();
         // Every stage and accumulator is free here: the previous unit ended
         // with every compute warp past its last chunk (CTA barrier below).
         for (int k = 0; k < kScanStages && k < nch; ++k) issue_stage(k);
-        bool ok = a.nslab <= nslab_t || mbar_wait(wb, (uint32_t)nw & 1u, a.err, 21);
-        if (ok) ok = mbar_wait(smem_u32(wready), (uint32_t)nw & 1u, a.err, 27);
+        bool ok = a.nslab <= nslab_t || kWait(wb, (uint32_t)nw & 1u, a.err, 21);
+        if (ok) ok = kWait(smem_u32(wready), (uint32_t)nw & 1u, a.err, 27);
         if (ok) tc_fence_after();
         if (ok) ok = issue_mma(0);
         // chunk j's slot (stage + accumulator) is reused by chunk j + stages, once
@@ -1070,24 +1197,40 @@ __global__ void __launch_bounds__(kScanThreads, kScanCtasPerSm)
           const int kg = kg0 + k;
           if (k + 1 < nch) {
             const int j = kg + 1 - kScanStages;  // last chunk in MMA k+1's accumulator
-            if (j >= kg0 && !mbar_wait(smem_u32(&empty[j % kScanStages]),
-                                       (uint32_t)(j / kScanStages) & 1u, a.err, 23))
+            if (j >= kg0 && !kWait(smem_u32(&empty[j % kScanStages]),
+                                   (uint32_t)(j / kScanStages) & 1u, a.err, 23))
               break;
             if (!issue_mma(k + 1)) break;
           }
           if (k + kScanStages < nch) {
-            if (!mbar_wait(smem_u32(&empty[kg % kScanStages]), (uint32_t)(kg / kScanStages) & 1u,
+            if (!kWait(smem_u32(&empty[kg % kScanStages]), (uint32_t)(kg / kScanStages) & 1u,
                            a.err, 24))
               break;
+            if (store_y(k)) bulk_wait_read<0>();  // the stage is reloaded right after
             issue_stage(k + kScanStages);
           }
         }
+        // the y tiles of the last chunks (no reload follows them)
+        for (int k = nch > kScanStages ? nch - kScanStages : 0; ok && k < nch; ++k) {
+          const int kg = kg0 + k;
+          if (!kWait(smem_u32(&empty[kg % kScanStages]), (uint32_t)(kg / kScanStages) & 1u,
+                     a.err, 29))
+            break;
+          store_y(k);
+        }
+        bulk_wait_read<0>();  // the next unit reuses every stage
       }
     } else {
       // compute warps: thread = channel c0 + 32*warp + lane = TMEM lane
       const int cl = warp * 32 + lane;
       const int64_t c = c0 + cl;
       const bool cok = c < a.d;
+      bool lead_ok = true;  // kLead, thread 0: no bounded wait has given up
+      if (kLead && threadIdx.x == 0 && nch > 0) {
+        // every stage and accumulator is free at a unit's start (CTA barrier below)
+        issue_wdt();
+        for (int k = 0; k < kScanStages && k < nch; ++k) issue_stage(k);
+      }
       if (nch > 0) {
         // this channel's W_dt row, K slabs 0..nslab_t-1, into its TMEM lane
         // (zeros past R and past d, matching the zero fill of the dt_n tiles)
@@ -1113,6 +1256,37 @@ __global__ void __launch_bounds__(kScanThreads, kScanCtasPerSm)
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(wready));
       }
+      if (kLead && threadIdx.x == 0 && nch > 0) {  // the first chunk's dt_proj
+        lead_ok = a.nslab <= nslab_t || kWait(wb, (uint32_t)nw & 1u, a.err, 21);
+        if (lead_ok) lead_ok = kWait(smem_u32(wready), (uint32_t)nw & 1u, a.err, 27);
+        if (lead_ok) tc_fence_after();
+        if (lead_ok) lead_ok = issue_mma(0);
+      }
+      // kLead, thread 0: feeds chunk k + 1 while the warps run chunk k.  Its stage
+      // and accumulator were chunk k - 1's, so the TMA goes out once every warp
+      // is done with chunk k - 1 and the MMA once the TMA has landed; between
+      // groups of tokens only non-blocking tests, at the chunk's end waits.
+      bool tma_next = true, mma_next = false;  // for chunk 1: its TMA went out above
+      auto hook = [&](int k, bool block) {
+        if (!kLead || threadIdx.x != 0 || !lead_ok || k + 1 >= nch) return;
+        const int kg = kg0 + k;
+        if (!tma_next) {
+          const int j = kg - 1;
+          const uint32_t eb = smem_u32(&empty[j % kScanStages]);
+          const uint32_t ep = (uint32_t)(j / kScanStages) & 1u;
+          if (!(block ? (lead_ok = kWait(eb, ep, a.err, 23)) : mbar_test_wait(eb, ep))) return;
+          issue_stage(k + 1);
+          tma_next = true;
+        }
+        if (!mma_next) {
+          const int kn = kg + 1;
+          const uint32_t fb = smem_u32(&full[kn % kScanStages]);
+          if (!block && !mbar_test_wait(fb, (uint32_t)(kn / kScanStages) & 1u)) return;
+          if (!(lead_ok = issue_mma(k + 1))) return;
+          mma_next = true;
+        }
+        if (block) tma_next = mma_next = false;  // chunk k + 2 is next
+      };
       // a unit that starts from earlier parts waits (bounded) for their hand-over
       const int n_wait = part == 0 ? 0 : (a.two_pass ? (out ? part : 0) : 1);
       if (n_wait > 0) {
@@ -1173,11 +1347,13 @@ __global__ void __launch_bounds__(kScanThreads, kScanCtasPerSm)
       }
       float ssum = 0.0f;
       if (out)
-        scan_chunks<true, kZoh>(a, stage0, full, mma_done, empty, tmem, warp, lane, kg0, kb, nch,
+        scan_chunks<true, kZoh, kLead>(hook, a, stage0, full, mma_done, empty, tmem, warp, lane,
+                                       kg0, kb, nch,
                                 Lb, cok, a.y + g0 * a.d + c, h, A2, invA, xw, cw, cb, bias, Dc,
                                 ssum);
       else
-        scan_chunks<false, kZoh>(a, stage0, full, mma_done, empty, tmem, warp, lane, kg0, kb, nch,
+        scan_chunks<false, kZoh, kLead>(hook, a, stage0, full, mma_done, empty, tmem, warp, lane,
+                                        kg0, kb, nch,
                                  Lb, cok, nullptr, h, A2, invA, xw, cw, cb, bias, Dc, ssum);
       if (part + 1 < P && (!out || !a.two_pass)) {
         // hand the end state (and, two-pass, the sum of delta) to later parts
@@ -1206,13 +1382,14 @@ __global__ void __launch_bounds__(kScanThreads, kScanCtasPerSm)
     nw += nch > 0 ? 1 : 0;
     __syncthreads();
     // stop claiming work once any wait has given up
-    if (threadIdx.x == 32 * kProdWarp && *(volatile unsigned*)&a.err->timeout)
+    if (threadIdx.x == kFeedThread && *(volatile unsigned*)&a.err->timeout)
       unit_slot[(it + 1) & 1] = n_units;
     __syncthreads();
   }
+  if (!kLead && threadIdx.x == kFeedThread) bulk_wait_all();  // the y tile stores completed
   tc_fence_before();
   __syncthreads();
-  if (warp == kProdWarp) {
+  if (warp == kAllocWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kScanTmemCols);
   }
@@ -1286,8 +1463,9 @@ __global__ void __launch_bounds__(kDecThreads, 2)
                   const __grid_constant__ CUtensorMap tm_dtn,
                   const __grid_constant__ CUtensorMap tm_bc, const DecArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  // (offset arithmetic on the shared array keeps its address space known, so
+  // accesses through these pointers compile to shared-memory loads)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* stages = smem;                                  // kDecStages x kDecStage
   uint8_t* dtn_s = stages + kDecStages * kDecStage;        // 2 x kDecDtn
   uint8_t* bc_s = dtn_s + 2 * kDecDtn;                     // 2 x kDecBC
@@ -1313,7 +1491,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kDecStages; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
-      mbar_init(smem_u32(&empty[s]), 4);
+      mbar_init(smem_u32(&empty[s]), 4);  // one arrive per compute warp, once it read the stage
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&gfull[b]), 1);
@@ -1352,7 +1530,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         const uint32_t fb = smem_u32(&full[s]);
         if (sl >= 0) {
           mbar_arrive_expect_tx(fb, (uint32_t)kDecState + conv_bytes + 2 * row_bytes);
-          tma_load_2d(smem_u32(st), &tm_state, fb, 0, (int32_t)(sl * a.d + c0));
+          tma_load_3d(smem_u32(st), &tm_state, fb, 0, (int32_t)c0, (int32_t)sl);
           bulk_load(smem_u32(st + kDecState), a.conv_state + (sl * a.d + c0) * (kConv - 1),
                     conv_bytes, fb);
         } else {
@@ -1598,6 +1776,35 @@ bool make_map_swz(CUtensorMap* m, CUtensorMapDataType dt, size_t esize, const vo
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D tensor map of an SSM-state pool [slots, d, 16] fp32 with box [1, 128, 16]
+// and 64-byte swizzle: a box never reaches past its slot's channels, so a tile
+// store at the last channel tile writes only channels that exist.
+bool make_state_map(CUtensorMap* m, const float* base, uint64_t slots, uint64_t d) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)kN, d, slots};
+  cuuint64_t strides[2] = {(cuuint64_t)kN * 4, d * kN * 4};
+  cuuint32_t box[3] = {(cuuint32_t)kN, (cuuint32_t)kSC, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3-D tensor map of y [B, L, d] bf16 with box [1, 32 tokens, 128 channels]: a
+// tile store never reaches past its sequence's tokens or past d.
+bool make_y_map(CUtensorMap* m, const void* y, uint64_t B, uint64_t L, uint64_t d) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d, L, B};
+  cuuint64_t strides[2] = {d * 2, L * d * 2};
+  cuuint32_t box[3] = {(cuuint32_t)kSC, (cuuint32_t)kSQ, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(y), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // As make_map_swz with the 128-byte swizzle (swz) or none.
 bool make_map(CUtensorMap* m, CUtensorMapDataType dt, size_t esize, const void* base,
               uint64_t rows, uint64_t cols, uint32_t box_cols, uint32_t box_rows, bool swz) {
@@ -1789,8 +1996,7 @@ cudaError_t run_fast_fwd(Problem& p) {
   if (p.decode) {
     CUtensorMap tstate, tdtn, tbc;
     const int64_t slots = p.sidx ? p.n_slots : p.B;
-    if (!make_map_swz(&tstate, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p.final_state,
-                      (uint64_t)(slots * p.d), kN, kN, kSC, CU_TENSOR_MAP_SWIZZLE_64B) ||
+    if (!make_state_map(&tstate, p.final_state, (uint64_t)slots, (uint64_t)p.d) ||
         !make_map(&tdtn, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w.dtn, p.T, p.R, 64, kDB, true) ||
         !make_map(&tbc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, w.bc, p.T, 2 * kN, 2 * kN, kDB,
                   false))
@@ -1869,12 +2075,18 @@ cudaError_t run_fast_fwd(Problem& p) {
     const int pairs = sa.n_tiles * (int)p.B;
     const int units = pairs * sa.n_parts + (sa.two_pass ? pairs * (sa.n_parts - 1) : 0);
     const int slots = kScanCtasPerSm * num_sms();
-    auto scan_kern = p.zoh ? k_scan_fused<true> : k_scan_fused<false>;
+    auto scan_kern = p.zoh ? k_scan_fused<true, JMIX_SCAN_LEAD != 0>
+                           : k_scan_fused<false, JMIX_SCAN_LEAD != 0>;
     cudaFuncSetAttribute(scan_kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kScanSmem);
     cudaFuncSetAttribute(scan_kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                          cudaSharedmemCarveoutMaxShared);
-    e = launch_pdl(scan_kern, dim3((unsigned)(units < slots ? units : slots)), kScanThreads,
-                   (size_t)kScanSmem, s, twdt, tdtn, tbc, tx, tz, sa);
+    CUtensorMap ty;  // y as [B, L, d] (a packed batch stores y thread by thread)
+    if (!make_y_map(&ty, p.y, p.cu ? 1 : (uint64_t)p.B, p.cu ? (uint64_t)p.T : (uint64_t)p.L,
+                    (uint64_t)p.d))
+      return cudaErrorInvalidValue;
+    e = launch_pdl(scan_kern, dim3((unsigned)(units < slots ? units : slots)),
+                   JMIX_SCAN_LEAD ? 128u : (unsigned)kScanThreads, (size_t)kScanSmem, s, twdt,
+                   tdtn, tbc, tx, tz, ty, sa);
     if (e != cudaSuccess) return e;
     launched(p, "k_scan_fused");
   }

@@ -70,8 +70,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     k_gemm_bf16(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                 const GemmArgs g) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kGStages * kGStageBytes);
   uint64_t* full = bars;                       // [stages] A and B tiles landed
   uint64_t* empty = bars + kGStages;           // [stages] MMAs done reading the stage
@@ -212,6 +211,172 @@ __global__ void __launch_bounds__(kGThreads, 1)
   }
 }
 
+// ------------------------------------------------------------ CTA-pair form
+// The same GEMM with a 256 x 256 tile per CTA pair (cluster of 2): each CTA
+// loads half of the tile's A rows and half of its B rows (32 KB per K chunk
+// instead of 48 KB for a 128 x 256 tile), the leader issues
+// tcgen05.mma.cta_group::2 (M 256, N 256, K 16) over both CTAs' stages, and each
+// CTA's TMEM receives its 128 rows.  Barriers: the leader's full[s] counts both
+// CTAs' TMA bytes; the leader's commits arrive on empty[s] and acc_full[b] in
+// both CTAs; both CTAs' epilogue warps arrive on the leader's acc_empty[b].
+constexpr int kPStages = 6;
+constexpr int kPHalf = 128;                              // rows of A and of B per CTA
+constexpr int kPStageBytes = 2 * kPHalf * kGK * 2;      // 32 KB: A half + B half
+constexpr int kPSmem = 1024 + kPStages * kPStageBytes + 256;
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
+    k_gemm_bf16_pair(const __grid_constant__ CUtensorMap tm_a,
+                     const __grid_constant__ CUtensorMap tm_b, const GemmArgs g) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kPStages * kPStageBytes);
+  uint64_t* full = bars;                       // [stages] (leader) both halves landed
+  uint64_t* empty = bars + kPStages;           // [stages] the pair MMAs read the stage
+  uint64_t* acc_full = bars + 2 * kPStages;    // [2] accumulator complete
+  uint64_t* acc_empty = acc_full + 2;          // [2] (leader) both epilogues done (8 warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int64_t pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  // tiles of 256 rows x 256 columns; g.m_tiles counts 256-row tiles here
+  const int64_t n_tiles_total = g.m_tiles * g.n_tiles;
+  const int kchunks = (int)((g.K + kGK - 1) / kGK);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPStages; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&acc_full[b]), 1);
+      mbar_init(smem_u32(&acc_empty[b]), 8);
+    }
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(tmem_slot), kGTmemCols);
+    tmem_relinquish_pair();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_a);
+    prefetch_tmap(&tm_b);
+  }
+  tc_fence_before();
+  cluster_sync();   // both CTAs' barriers exist before either signals the other's
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  grid_dep_wait();
+  if (g.fold && blockIdx.x == 0 && threadIdx.x == 0) {
+    if (g.fold->timeout && atomicExch(&g.err->timeout, 1u) == 0u) g.err->where = g.fold->where;
+    if (g.fold->bad_input) atomicExch(&g.err->bad_input, 1u);
+  }
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int64_t it = 0;
+      bool ok = true;
+      for (int64_t t = pair; ok && t < n_tiles_total; t += npairs) {
+        int64_t mt, nt;
+        tile_coords(g, t, mt, nt);
+        for (int kc = 0; kc < kchunks; ++kc, ++it) {
+          const int s = (int)(it % kPStages);
+          if (it >= kPStages &&
+              !mbar_wait(smem_u32(&empty[s]), (uint32_t)((it / kPStages) - 1) & 1u, g.err, 71)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + s * kPStageBytes;
+          const uint32_t fb = leader_addr(smem_u32(&full[s]));
+          // the leader expects both CTAs' bytes on its barrier
+          if (leader) mbar_arrive_expect_tx(smem_u32(&full[s]), (uint32_t)(2 * kPStageBytes));
+          tma_load_2d_pair(smem_u32(st), &tm_a, fb, kc * kGK,
+                           (int32_t)(mt * (2 * kPHalf) + rank * kPHalf));
+          tma_load_2d_pair(smem_u32(st + kPHalf * kGK * 2), &tm_b, fb, kc * kGK,
+                           (int32_t)(nt * kGN + rank * kPHalf));
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      const uint32_t idesc = idesc_bf16_f32(2 * kPHalf, kGN);
+      int64_t it = 0, j = 0;
+      bool ok = true;
+      for (int64_t t = pair; ok && t < n_tiles_total; t += npairs, ++j) {
+        const int b = (int)(j & 1);
+        if (j >= 2 &&
+            !mbar_wait(smem_u32(&acc_empty[b]), (uint32_t)((j >> 1) - 1) & 1u, g.err, 72))
+          break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + (uint32_t)(b * kGN);
+        for (int kc = 0; kc < kchunks; ++kc, ++it) {
+          const int s = (int)(it % kPStages);
+          if (!mbar_wait(smem_u32(&full[s]), (uint32_t)(it / kPStages) & 1u, g.err, 73)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t ab = smem_u32(smem + s * kPStageBytes), bb = ab + kPHalf * kGK * 2;
+#pragma unroll
+          for (int kk = 0; kk < kGK / 16; ++kk)
+            umma_f16_pair(d_tmem, sw128_kmajor_desc(ab + kk * 32), sw128_kmajor_desc(bb + kk * 32),
+                          idesc, (kc > 0 || kk > 0) ? 1u : 0u);
+          umma_commit_pair(smem_u32(&empty[s]), 0x3);
+        }
+        if (ok) umma_commit_pair(smem_u32(&acc_full[b]), 0x3);
+      }
+    }
+  } else {
+    // epilogue: this CTA's 128 rows of the pair's 256-row tile
+    const int lg = warp & 3;
+    const uint32_t acc_empty_leader = leader_addr(smem_u32(&acc_empty[0]));
+    int64_t j = 0;
+    for (int64_t t = pair; t < n_tiles_total; t += npairs, ++j) {
+      int64_t mt, nt;
+      tile_coords(g, t, mt, nt);
+      const int b = (int)(j & 1);
+      if (!mbar_wait(smem_u32(&acc_full[b]), (uint32_t)(j >> 1) & 1u, g.err, 74)) break;
+      tc_fence_after();
+      const int64_t row = mt * (2 * kPHalf) + rank * kPHalf + lg * 32 + lane;
+      const int64_t n0 = nt * kGN;
+      const uint32_t tbase = tmem + ((uint32_t)(lg * 32) << 16) + (uint32_t)(b * kGN);
+#pragma unroll 1
+      for (int c = 0; c < kGN; c += 32) {
+        uint32_t r[32];
+        tmem_ld16(tbase + (uint32_t)c, *reinterpret_cast<uint32_t(*)[16]>(r));
+        tmem_ld16(tbase + (uint32_t)(c + 16), *reinterpret_cast<uint32_t(*)[16]>(r + 16));
+        tmem_ld_wait();
+        if (row < g.M) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int64_t col = n0 + c + 8 * q;
+            if (col + 8 > g.N) break;
+            const uint4 v = make_uint4(
+                pack_bf16x2(__uint_as_float(r[8 * q]), __uint_as_float(r[8 * q + 1])),
+                pack_bf16x2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3])),
+                pack_bf16x2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5])),
+                pack_bf16x2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7])));
+            __nv_bfloat16* dst = col < g.n_split
+                                     ? g.C0 + row * g.n_split + col
+                                     : g.C1 + row * (g.N - g.n_split) + (col - g.n_split);
+            *reinterpret_cast<uint4*>(dst) = v;
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acc_empty_leader + (uint32_t)(b * 8));
+    }
+  }
+  tc_fence_before();
+  cluster_sync();   // no CTA leaves while its pair may still signal it
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kGTmemCols);
+  }
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
@@ -249,10 +414,54 @@ int sm_count() {
 
 }  // namespace
 
+#ifndef JMIX_GEMM_PAIR
+#define JMIX_GEMM_PAIR 1
+#endif
+
 cudaError_t gemm_bf16_tn(int64_t M, int64_t N, int64_t K, const void* A, const void* B,
                          void* C0, void* C1, int64_t n_split, ErrFlags* err,
                          const ErrFlags* fold, cudaStream_t s, bool pdl) {
   if (M <= 0 || N <= 0) return cudaSuccess;
+  if (JMIX_GEMM_PAIR) {
+    // CTA pairs: A and B tiles of 128 rows per CTA
+    CUtensorMap ta, tb;
+    if (!bf16_kmajor_map(&ta, A, (uint64_t)M, (uint64_t)K, kPHalf) ||
+        !bf16_kmajor_map(&tb, B, (uint64_t)N, (uint64_t)K, kPHalf))
+      return cudaErrorInvalidValue;
+    GemmArgs g;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.n_split = n_split;
+    g.C0 = static_cast<__nv_bfloat16*>(C0);
+    g.C1 = static_cast<__nv_bfloat16*>(C1);
+    g.m_tiles = (M + 2 * kPHalf - 1) / (2 * kPHalf);
+    g.n_tiles = (N + kGN - 1) / kGN;
+    g.err = err;
+    g.fold = fold;
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_bf16_pair,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem);
+    if (e != cudaSuccess) return e;
+    const int64_t tiles = g.m_tiles * g.n_tiles;
+    // as many pairs as can be resident at once (a pair needs two SMs of one GPC)
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(sm_count() & ~1));
+    cfg.blockDim = dim3(kGThreads);
+    cfg.dynamicSmemBytes = kPSmem;
+    int max_pairs = 0;
+    if (cudaOccupancyMaxActiveClusters(&max_pairs, k_gemm_bf16_pair, &cfg) != cudaSuccess ||
+        max_pairs <= 0)
+      max_pairs = sm_count() / 2;
+    const int64_t pairs = tiles < max_pairs ? tiles : max_pairs;
+    cfg.gridDim = dim3((unsigned)(2 * pairs));
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, k_gemm_bf16_pair, ta, tb, g);
+  }
   CUtensorMap ta, tb;
   if (!bf16_kmajor_map(&ta, A, (uint64_t)M, (uint64_t)K, kGM) ||
       !bf16_kmajor_map(&tb, B, (uint64_t)N, (uint64_t)K, kGN))

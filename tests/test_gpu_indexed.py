@@ -91,7 +91,9 @@ def run_indexed(w, S, steps, prepared, channels=None, seed=5):
 
 @pytest.mark.parametrize("prepared", [False, True])
 def test_indexed_small(prepared):
-    w = synth.Workload("idx", 12, 1, 256, 16, "bf16", seed=41, extra=True, steps=4)
+    # dt_rank 64: one fp16 rounding flip of dt_n moves delta by about 2^-10/sqrt(R)
+    # relative; at R = 16 over 12 rows x 4 steps that alone nears the 1e-4 state gate
+    w = synth.Workload("idx", 12, 1, 256, 64, "bf16", seed=41, extra=True, steps=4)
     run_indexed(w, 40, 4, prepared)
 
 
