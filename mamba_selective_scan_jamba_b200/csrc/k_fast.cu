@@ -48,6 +48,10 @@ constexpr int kConvG = 8;
 constexpr int kXM = 128;          // x_proj tile: tokens
 constexpr int kXK = 64;           // x_proj tile: channels per k-chunk (one 128-B swizzle atom)
 constexpr int kXStages = 4;
+#ifndef JMIX_XSPLIT_MAX
+#define JMIX_XSPLIT_MAX 32
+#endif
+constexpr int kMaxSplit = JMIX_XSPLIT_MAX;  // x_proj splits over d_inner, at most
 #ifndef JMIX_SCAN_CHUNK
 #define JMIX_SCAN_CHUNK 32
 #endif
@@ -507,17 +511,15 @@ __global__ void __launch_bounds__(kNormThreads) k_norms16(
     const int64_t g = g0 + tl;
     if (g >= Tn) continue;
     const float* src = part + g * P + j;
-    float acc = src[0];
-    int sp = 1;
-    for (; sp + 4 <= ksplit; sp += 4) {
-      const float v0 = src[sp * stride], v1 = src[(sp + 1) * stride];
-      const float v2 = src[(sp + 2) * stride], v3 = src[(sp + 3) * stride];
-      acc += v0;
-      acc += v1;
-      acc += v2;
-      acc += v3;
-    }
-    for (; sp < ksplit; ++sp) acc += src[sp * stride];
+    // every split's value is loaded before the sum (one memory round trip);
+    // the sum still runs in ascending split order
+    float v[kMaxSplit];
+#pragma unroll
+    for (int sp = 0; sp < kMaxSplit; ++sp) v[sp] = sp < ksplit ? src[sp * stride] : 0.0f;
+    float acc = v[0];
+#pragma unroll
+    for (int sp = 1; sp < kMaxSplit; ++sp)
+      if (sp < ksplit) acc += v[sp];
     rows[tl][j] = acc;
   }
   __syncthreads();
@@ -1634,6 +1636,15 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       const uint32_t tacc =
           tmem + ((uint32_t)(warp * 32) << 16) + kDecAccCol + (uint32_t)(bsel * kDB);
       const float4* bcs = reinterpret_cast<const float4*>(bc_s + bsel * kDecBC);
+      // the group's 16 accumulators in one TMEM load; the rows are taken in
+      // order, so the current row's value is kept in racc[0] by shifting
+      uint32_t racc[kDB];
+      tmem_ld16(tacc, racc);
+      tmem_ld_wait();
+      for (int q = (int)((p % a.B) - r0); q > 0; --q) {
+#pragma unroll
+        for (int e = 0; e < kDB - 1; ++e) racc[e] = racc[e + 1];
+      }
       // the rows of this group that fall in [p0, p1)
       for (; p < p1 && (p / a.B) == tile && (p % a.B) < r0 + kDB; ++p, ++i) {
         const int s = (int)(i % kDecStages);
@@ -1645,9 +1656,6 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         const int64_t b = p % a.B;
         const int64_t sl = dec_slot(a, b);
         const uint8_t* st = stages + s * kDecStage;
-        uint32_t racc[1];  // this row's dt_proj accumulator (column j of the group)
-        tmem_ld_cols<1>(tacc + (uint32_t)j, racc);
-        tmem_ld_wait();
         // read the stage (state rows are 64-byte swizzled: 16-byte chunk q of
         // row cl sits at chunk q ^ ((cl >> 1) & 3)), then release it
         float2 h[kN / 2];
@@ -1687,6 +1695,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         xc = fmaf(cw[3], xt, xc);
         const float uv = silu_u(xc);
         const float dl = softplus_fast(__uint_as_float(racc[0]) + bias);
+#pragma unroll
+        for (int e = 0; e < kDB - 1; ++e) racc[e] = racc[e + 1];  // the next row's first
         const float2 dl2 = make_float2(dl, dl), du2 = make_float2(dl * uv, dl * uv);
         float2 acc[4];
 #pragma unroll
@@ -1830,9 +1840,7 @@ struct FastWs {
   int ksplit;
 };
 
-#ifndef JMIX_XSPLIT_MAX
-#define JMIX_XSPLIT_MAX 32
-#endif
+
 // x_proj split over d_inner: about two CTAs per SM of a B200 (2 x 148), at
 // most JMIX_XSPLIT_MAX splits, at least one 64-channel chunk per split.  Depends on the
 // problem only, so the workspace size does too.
