@@ -47,7 +47,10 @@ typedef __nv_bfloat16 bf16;
 constexpr int kConvG = 8;
 constexpr int kXM = 128;          // x_proj tile: tokens
 constexpr int kXK = 64;           // x_proj tile: channels per k-chunk (one 128-B swizzle atom)
-constexpr int kXStages = 4;
+constexpr int kXStages = 3;
+#ifndef JMIX_XPROJ_CTAS  // x_proj grid target: two resident CTAs per SM
+#define JMIX_XPROJ_CTAS 296
+#endif
 #ifndef JMIX_XSPLIT_MAX
 #define JMIX_XSPLIT_MAX 32
 #endif
@@ -366,7 +369,12 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
          | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-__global__ void __launch_bounds__(kXThreads, 1)
+// Grid (2 x token tiles, d_inner splits): the R + 2N columns are cut in two
+// parts of N1 (each one MMA of N <= 256, a TMEM allocation of at most 256
+// columns and a 3-stage ring), so two CTAs share an SM and one's epilogue
+// overlaps the other's loads.  The part is the fastest grid index: the two
+// CTAs of a token tile run together and the second read of its u tile hits L2.
+__global__ void __launch_bounds__(kXThreads, 2)
     k_xproj(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_w,
             const XprojArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -374,7 +382,8 @@ __global__ void __launch_bounds__(kXThreads, 1)
   // accesses through these pointers compile to shared-memory loads)
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int a_bytes = kXM * 128;
-  const int b_bytes = a.Ntot * 128;
+  const int b_bytes = a.N1 * 128;
+  const int col0 = (int)(blockIdx.x & 1u) * a.N1;  // this CTA's first column of p
   const int stage_bytes = a_bytes + b_bytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kXStages * stage_bytes);
   uint64_t* full = bars;
@@ -383,7 +392,7 @@ __global__ void __launch_bounds__(kXThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * kXStages + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m_tile = blockIdx.x, split = blockIdx.y;
+  const int m_tile = (int)(blockIdx.x >> 1), split = blockIdx.y;
   const int k_begin = (int)((int64_t)split * a.kchunks / a.ksplit);
   const int k_end = (int)((int64_t)(split + 1) * a.kchunks / a.ksplit);
 
@@ -421,14 +430,12 @@ __global__ void __launch_bounds__(kXThreads, 1)
         const uint32_t fb = smem_u32(&full[s]);
         mbar_arrive_expect_tx(fb, (uint32_t)stage_bytes);
         tma_load_2d(smem_u32(As), &tm_u, fb, kc * kXK, m_tile * kXM);
-        tma_load_2d(smem_u32(Bs), &tm_w, fb, kc * kXK, 0);
-        if (a.N2) tma_load_2d(smem_u32(Bs + a.N1 * 128), &tm_w, fb, kc * kXK, a.N1);
+        tma_load_2d(smem_u32(Bs), &tm_w, fb, kc * kXK, col0);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t id1 = idesc_f16_f32(kXM, a.N1);
-      const uint32_t id2 = idesc_f16_f32(kXM, a.N2 ? a.N2 : 16);
       for (int kc = k_begin, i = 0; kc < k_end; ++kc, ++i) {
         const int s = i % kXStages;
         const uint32_t ph = (uint32_t)(i / kXStages) & 1u;
@@ -441,8 +448,6 @@ __global__ void __launch_bounds__(kXThreads, 1)
           const uint64_t ad = sw128_kmajor_desc(ab + kk * 32);
           const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
           umma_f16(tmem, ad, sw128_kmajor_desc(bb + kk * 32), id1, acc);
-          if (a.N2)
-            umma_f16(tmem + a.N1, ad, sw128_kmajor_desc(bb + a.N1 * 128 + kk * 32), id2, acc);
         }
         umma_commit(smem_u32(&empty[s]));
       }
@@ -460,7 +465,7 @@ __global__ void __launch_bounds__(kXThreads, 1)
     const int64_t row0 = (int64_t)m_tile * kXM + lg * 32;
     float* dst = a.part + ((int64_t)split * a.T) * a.P;
     const bool any = ok && k_end > k_begin;
-    for (int c0 = 0; c0 < a.Ntot; c0 += 16) {
+    for (int c0 = 0; c0 < a.N1; c0 += 16) {
       uint32_t r[16];
       tmem_ld16(tmem + ((uint32_t)(lg * 32) << 16) + (uint32_t)c0, r);
       tmem_ld_wait();
@@ -468,7 +473,7 @@ __global__ void __launch_bounds__(kXThreads, 1)
       for (int j = 0; j < 16; ++j) tbuf[lane * 17 + j] = __uint_as_float(r[j]);
       __syncwarp();
       if (any) {
-        const int col = c0 + (lane & 15);
+        const int col = col0 + c0 + (lane & 15);
 #pragma unroll 4
         for (int rr = 0; rr < 16; ++rr) {
           const int row = 2 * rr + (lane >> 4);
@@ -1848,7 +1853,7 @@ int xproj_ksplit(int64_t T, int64_t d) {
   if (T <= 0) return 1;
   const int64_t mtiles = (T + kXM - 1) / kXM;
   const int64_t kchunks = (d + kXK - 1) / kXK;
-  int64_t ks = (296 + mtiles - 1) / mtiles;
+  int64_t ks = (JMIX_XPROJ_CTAS + 2 * mtiles - 1) / (2 * mtiles);  // 2 column parts
   if (ks > JMIX_XSPLIT_MAX) ks = JMIX_XSPLIT_MAX;
   if (ks > kchunks) ks = kchunks;
   return ks < 1 ? 1 : (int)ks;
@@ -1962,30 +1967,23 @@ cudaError_t run_fast_fwd(Problem& p) {
     XprojArgs xa;
     xa.T = p.T;
     xa.P = (int)p.P;
-    // one MMA of N <= 256, or two equal halves (the second W box then has the
-    // same row count as the first, so both fill exactly their part of the stage)
-    if (p.P <= 256) {
-      xa.N1 = (int)((p.P + 15) / 16 * 16);
-      xa.N2 = 0;
-    } else {
-      xa.N1 = (int)(((p.P + 1) / 2 + 15) / 16 * 16);
-      xa.N2 = xa.N1;
-    }
+    // two column parts of N1 (a multiple of 16), one per CTA of the grid's z
+    xa.N1 = (int)(((p.P + 1) / 2 + 15) / 16 * 16);
+    xa.N2 = xa.N1;
     xa.Ntot = xa.N1 + xa.N2;
     xa.kchunks = (int)((p.d + kXK - 1) / kXK);
     const int64_t mtiles = (p.T + kXM - 1) / kXM;
     xa.ksplit = w.ksplit;
-    xa.tmem_cols = xa.Ntot <= 32 ? 32 : xa.Ntot <= 64 ? 64 : xa.Ntot <= 128 ? 128
-                   : xa.Ntot <= 256 ? 256 : 512;
+    xa.tmem_cols = xa.N1 <= 32 ? 32 : xa.N1 <= 64 ? 64 : xa.N1 <= 128 ? 128 : 256;
     xa.part = w.part;
     xa.err = err;
     if (!make_map(&tu, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w.u, p.T, p.d, kXK, kXM, true) ||
         !make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w.wx, p.P, p.d, kXK, xa.N1, true))
       return cudaErrorInvalidValue;
-    const int smem = 1024 + kXStages * (kXM * 128 + xa.Ntot * 128) + 256;
+    const int smem = 1024 + kXStages * (kXM * 128 + xa.N1 * 128) + 256;
     cudaFuncSetAttribute(k_xproj, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    e = launch_pdl(k_xproj, dim3((unsigned)mtiles, (unsigned)xa.ksplit), kXThreads, (size_t)smem,
-                   s, tu, tw, xa);
+    e = launch_pdl(k_xproj, dim3((unsigned)(2 * mtiles), (unsigned)xa.ksplit), kXThreads,
+                   (size_t)smem, s, tu, tw, xa);
     if (e != cudaSuccess) return e;
     launched(p, "k_xproj");
   }
