@@ -613,6 +613,503 @@ __global__ void __launch_bounds__(256) k_norms16_warp(
   bc[g * 2 * kN + lane] = bcv * inv2 * wv;
 }
 
+// ------------------------------------------------ conv + SiLU inside x_proj
+// The prefill form of steps 1-3 for sequences of one length (T = B L tokens):
+// x_proj's A operand u = SiLU(conv(x)) is computed in shared memory from TMA
+// tiles of x, so u never goes through global memory (the scan recomputes its
+// own u in float32).  Grid (token tiles of 128, splits of d_inner); each CTA
+// computes all R + 2N columns of its tiles as two MMAs of N1 columns.
+//   warp 0      TMA: per 64-channel chunk the x rows m0 - 3 .. m0 + 127 (one
+//               box of 131 rows; rows before token 0 and past T read as zero),
+//               the chunk's conv weights and biases (bulk copies) and its two
+//               W_x boxes;
+//   warp 1      TMEM owner and MMA issuer (2 x 4 tcgen05.mma per chunk);
+//   warps 2-    conv (JMIX_XCONV_WARPS of them): thread = 8 channels x kFG
+//               tokens (4 with 8 warps).  The kFG + 3 x rows come from
+//               the stage, taps before a sequence's first token from its
+//               history (or zero); u in fp16 goes into the 128-byte-swizzled A
+//               stage, rounded exactly as k_conv_silu16 rounds it.  Then the
+//               epilogue.
+// With one split the epilogue applies the RMSNorms itself (thread = token row
+// of TMEM, the sums of squares taken in the order of k_norms16_warp's
+// reductions) and writes dt_n and B, C; with several it writes the fp32
+// partial sums that k_norms16 adds up.
+#ifndef JMIX_XCONV_WARPS
+#define JMIX_XCONV_WARPS 8  // conv warps (8: 4 tokens per thread, 16: 2)
+#endif
+constexpr int kFConvWarps = JMIX_XCONV_WARPS;
+constexpr int kFG = kXM * (kXK / 8) / (kFConvWarps * 32);  // tokens per conv thread
+constexpr int kFThreads = 64 + 32 * kFConvWarps;
+constexpr int kFStages = 3;
+constexpr int kFXRows = kXM + kConv - 1;                    // 131 x rows per chunk
+constexpr int kFXBytes = kFXRows * kXK * 2;                 // 16768 B
+constexpr int kFCwBytes = kXK * kConv * 2;                  // 512 B: the chunk's conv weights
+constexpr int kFCbBytes = kXK * 2;                          // 128 B: its conv biases
+constexpr int kFXStride = (kFXBytes + kFCwBytes + kFCbBytes + 1023) / 1024 * 1024;  // 17 KB
+constexpr int kFABytes = kXM * kXK * 2;                     // 16 KB u tile
+constexpr int kFMaxN1 = (kMaxRank + 2 * kN) / 2;            // 144
+constexpr int kFBMax = 2 * kFMaxN1 * kXK * 2;               // 36 KB of W_x rows
+constexpr int kFSmem = 1024 + kFStages * (kFABytes + kFBMax + kFXStride) + 256;
+static_assert(kFSmem <= 227 * 1024, "fused x_proj stage ring exceeds shared memory");
+static_assert(kFConvWarps * 32 * kFG == kXM * (kXK / 8), "conv threads = kFG-token x 8-channel cells");
+
+struct XconvArgs {
+  int64_t T, L, d;
+  int P, N1, R;
+  int kchunks, ksplit;
+  uint32_t tmem_cols;
+  const bf16* conv_w;  // [d, 4]
+  const bf16* conv_b;  // [d]
+  const bf16* hist;    // [B, d, 3] conv history of each sequence, or null (zeros)
+  const int* sidx;     // decode step (L == 1): history slot of each row, or null (slot = row)
+  int64_t n_slots;     // decode step: slots of the history pool
+  float* part;         // [ksplit, T, P] partial sums (ksplit > 1)
+  const bf16* dtn_w;   // [R]
+  const bf16* bn_w;    // [N]
+  const bf16* cn_w;    // [N]
+  float eps;
+  __half* dtn;         // [T, R] (ksplit == 1)
+  float* bc;           // [T, 2N] (ksplit == 1)
+  ErrFlags* err;
+};
+
+// Channels (2q, 2q + 1) of 8 packed bf16 values as a float pair.
+__device__ __forceinline__ float2 bf16_pair(const uint4& v, int q) {
+  const uint32_t w = q == 0 ? v.x : q == 1 ? v.y : q == 2 ? v.z : v.w;
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+#ifndef JMIX_XCONV_SILU1
+#define JMIX_XCONV_SILU1 0  // 1: the reciprocal by Newton steps on the FMA pipe (one MUFU op)
+#endif
+// SiLU of a pair, clamped to the fp16 range and packed as fp16x2: the same
+// operations, in the same order, as clamp_half(silu_u(v)) on each element
+// (with JMIX_XCONV_SILU1, as silu_newton).
+__device__ __forceinline__ uint32_t silu_u_half2(float2 v) {
+  const float2 t = __fmul2_rn(v, make_float2(-kLog2e, -kLog2e));
+  float2 e, r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e.x) : "f"(t.x));
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e.y) : "f"(t.y));
+  float2 den = __fadd2_rn(make_float2(1.0f, 1.0f), e);
+#if JMIX_XCONV_SILU1
+  den = make_float2(fminf(den.x, 8.5e37f), fminf(den.y, 8.5e37f));
+  r = make_float2(__int_as_float(poly::RCP_MAGIC - __float_as_int(den.x)),
+                  __int_as_float(poly::RCP_MAGIC - __float_as_int(den.y)));
+  const float2 nd = make_float2(-den.x, -den.y), two = make_float2(2.0f, 2.0f);
+  r = __fmul2_rn(r, __ffma2_rn(nd, r, two));
+  r = __fmul2_rn(r, __ffma2_rn(nd, r, two));
+  r = __fmul2_rn(r, __ffma2_rn(nd, r, two));
+#else
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r.x) : "f"(den.x));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r.y) : "f"(den.y));
+#endif
+  const float2 s = __fmul2_rn(v, r);
+  return pack_half2(clamp_half(s.x), clamp_half(s.y));
+}
+
+__global__ void __launch_bounds__(kFThreads, 1)
+    k_xproj_conv(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                 const XconvArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* As = smem;                          // [stages] u tiles (128-byte swizzle)
+  uint8_t* Bs = As + kFStages * kFABytes;      // [stages] W_x boxes (128-byte swizzle)
+  uint8_t* Xs = Bs + kFStages * kFBMax;        // [stages] x rows (plain)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(Xs + kFStages * kFXStride);
+  uint64_t* full = bars;                       // [stages] x rows and W_x landed
+  uint64_t* afull = bars + kFStages;           // [stages] u tile written (conv warps)
+  uint64_t* mdone = bars + 2 * kFStages;       // [stages] the MMAs have read the stage
+  uint64_t* acc_full = bars + 3 * kFStages;    // accumulator complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t m0 = (int64_t)blockIdx.x * kXM;
+  const int split = blockIdx.y;
+  const int k_begin = (int)((int64_t)split * a.kchunks / a.ksplit);
+  const int k_end = (int)((int64_t)(split + 1) * a.kchunks / a.ksplit);
+  const uint32_t half_b = (uint32_t)(a.N1 * kXK * 2);  // bytes of one W_x box
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kFStages; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&afull[s]), kFConvWarps);
+      mbar_init(smem_u32(&mdone[s]), 1);
+    }
+    mbar_init(smem_u32(acc_full), 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), a.tmem_cols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_x);
+    prefetch_tmap(&tm_w);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  grid_dep_wait();    // the fp16 W_x may come from the kernel before this one
+  grid_dep_launch();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int kc = k_begin, i = 0; kc < k_end; ++kc, ++i) {
+        const int s = i % kFStages;
+        if (i >= kFStages &&
+            !mbar_wait(smem_u32(&mdone[s]), (uint32_t)((i / kFStages) - 1) & 1u, a.err, 85))
+          break;
+        const uint32_t fb = smem_u32(&full[s]);
+        // conv weights and biases of the chunk's channels that exist (a multiple of 8)
+        const int64_t c0 = (int64_t)kc * kXK;
+        const uint32_t nch = (uint32_t)((a.d - c0) < kXK ? (a.d - c0) : kXK);
+        mbar_arrive_expect_tx(fb, (uint32_t)kFXBytes + nch * (kConv * 2 + 2) + 2 * half_b);
+        uint8_t* xst = Xs + s * kFXStride;
+        tma_load_2d(smem_u32(xst), &tm_x, fb, kc * kXK, (int32_t)(m0 - (kConv - 1)));
+        bulk_load(smem_u32(xst + kFXBytes), a.conv_w + c0 * kConv, nch * kConv * 2, fb);
+        bulk_load(smem_u32(xst + kFXBytes + kFCwBytes), a.conv_b + c0, nch * 2, fb);
+        const uint32_t bs = smem_u32(Bs + s * kFBMax);
+        tma_load_2d(bs, &tm_w, fb, kc * kXK, 0);
+        tma_load_2d(bs + half_b, &tm_w, fb, kc * kXK, a.N1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id = idesc_f16_f32(kXM, a.N1);
+      for (int kc = k_begin, i = 0; kc < k_end; ++kc, ++i) {
+        const int s = i % kFStages;
+        const uint32_t ph = (uint32_t)(i / kFStages) & 1u;
+        if (!mbar_wait(smem_u32(&afull[s]), ph, a.err, 86)) break;
+        if (!mbar_wait(smem_u32(&full[s]), ph, a.err, 87)) break;
+        tc_fence_after();
+        const uint32_t ab = smem_u32(As + s * kFABytes), bb = smem_u32(Bs + s * kFBMax);
+#pragma unroll
+        for (int kk = 0; kk < kXK / 16; ++kk) {
+          const uint64_t ad = sw128_kmajor_desc(ab + kk * 32);
+          const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+          umma_f16(tmem, ad, sw128_kmajor_desc(bb + kk * 32), id, acc);
+          umma_f16(tmem + (uint32_t)a.N1, ad, sw128_kmajor_desc(bb + half_b + kk * 32), id, acc);
+        }
+        umma_commit(smem_u32(&mdone[s]));
+      }
+      umma_commit(smem_u32(acc_full));
+    }
+  } else {
+    // ---- conv: thread = channels cg*8 .. +7 of the chunk, tile rows kFG tg .. + kFG - 1
+    const int ct = threadIdx.x - 64;
+    const int cg = ct & 7, tg = ct >> 3;
+    constexpr int kW = kConv - 1;
+    // sequence and position of the thread's 4 tokens (the same for every
+    // chunk); a token at position < 3 takes taps from its sequence's history
+    int64_t tseq[kFG];
+    int tpos[kFG];
+    bool tedge[kFG], edge = false;
+#pragma unroll
+    for (int ti = 0; ti < kFG; ++ti) {
+      const int64_t g = m0 + kFG * tg + ti;
+      tseq[ti] = g / a.L;
+      tpos[ti] = (int)(g - tseq[ti] * a.L);
+      tedge[ti] = g < a.T && tpos[ti] < kW;
+      edge |= tedge[ti];
+    }
+    // When the thread's first token is at position < 3 and all its tokens lie
+    // in that sequence (every sequence start when kFG divides L), the x rows
+    // before the sequence are needed by this thread alone: they are replaced by
+    // the history rows once per chunk, and the common path computes the rest.
+    // Other layouts of sequence starts recompute their edge tokens (slow).
+    const bool sub = tedge[0] && tpos[0] + kFG <= a.L;
+    const bool slow = edge && !sub;
+    // decode step (L == 1): every tap but the last is history; a row's history
+    // sits in its pool slot, clamped into the pool (a bad slot is reported and
+    // skipped by the decode kernel), -1 for rows past T
+    const bool step = a.L == 1;
+    int64_t hrow[kFG];
+#pragma unroll
+    for (int ti = 0; ti < kFG; ++ti) {
+      const int64_t g = m0 + kFG * tg + ti;
+      int64_t sl = g;
+      if (step && a.sidx && g < a.T) {
+        sl = __ldg(a.sidx + g);
+        sl = sl < 0 ? 0 : (sl >= a.n_slots ? a.n_slots - 1 : sl);
+      }
+      hrow[ti] = (g < a.T && a.hist) ? sl : -1;
+    }
+    for (int kc = k_begin, i = 0; kc < k_end; ++kc, ++i) {
+      const int s = i % kFStages;
+      const uint32_t ph = (uint32_t)(i / kFStages) & 1u;
+      const int64_t c0 = (int64_t)kc * kXK + cg * 8;
+      const bool cin = c0 < a.d;  // d is a multiple of 8: all 8 channels exist, or none
+      if (!mbar_wait(smem_u32(&full[s]), ph, a.err, 88)) break;
+      // this thread's 8 channels' conv weights (64 B) and biases (16 B) from the
+      // stage (stale past d: those outputs are zeroed below)
+      const uint8_t* xst = Xs + s * kFXStride;
+      uint4 wq[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        wq[q] = *reinterpret_cast<const uint4*>(xst + kFXBytes + cg * 64 + 16 * q);
+      const uint4 bq = *reinterpret_cast<const uint4*>(xst + kFXBytes + kFCwBytes + cg * 16);
+      const uint8_t* xs = xst + (kFG * tg) * (kXK * 2) + cg * 16;
+      uint4 xr[kFG + kW];
+#pragma unroll
+      for (int j = 0; j < kFG + kW; ++j) xr[j] = *reinterpret_cast<const uint4*>(xs + j * (kXK * 2));
+      // weights and bias of the 4 channel pairs
+      float2 w2[4][kConv], b2[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+#pragma unroll
+        for (int k = 0; k < kConv; ++k) {
+          const int e0 = (2 * q) * kConv + k, e1 = (2 * q + 1) * kConv + k;
+          w2[q][k] = make_float2(bf16_lane(wq[e0 >> 3], e0 & 7), bf16_lane(wq[e1 >> 3], e1 & 7));
+        }
+        b2[q] = make_float2(bf16_lane(bq, 2 * q), bf16_lane(bq, 2 * q + 1));
+      }
+      uint32_t outw[kFG][4];  // [token][channel pair] fp16x2
+      if (!step) {
+        if (sub) {
+          // raw row j < 3 - tpos[0] holds position tpos[0] - 3 + j < 0 of the
+          // sequence: history slot tpos[0] + j (channel e's slots sit at 3 e ..)
+          uint4 hq[3] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u),
+                         make_uint4(0u, 0u, 0u, 0u)};
+          if (cin && a.hist) {
+            const uint4* hp = reinterpret_cast<const uint4*>(a.hist + (tseq[0] * a.d + c0) * kW);
+#pragma unroll
+            for (int q = 0; q < 3; ++q) hq[q] = __ldg(hp + q);
+          }
+          const uint32_t* hw = reinterpret_cast<const uint32_t*>(hq);
+          uint4 hrows[kW];  // [slot]: the 8 channels' values at that history slot
+#pragma unroll
+          for (int sl = 0; sl < kW; ++sl) {
+            uint32_t wv[4];
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              const int i0 = 3 * (2 * w) + sl, i1 = 3 * (2 * w + 1) + sl;  // 16-bit elements
+              const uint32_t lo = (hw[i0 >> 1] >> (16 * (i0 & 1))) & 0xffffu;
+              const uint32_t hi = (hw[i1 >> 1] >> (16 * (i1 & 1))) & 0xffffu;
+              wv[w] = lo | (hi << 16);
+            }
+            hrows[sl] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+          }
+#pragma unroll
+          for (int j = 0; j < kW; ++j) {
+            if (j < kW - tpos[0]) {
+              const int sl = tpos[0] + j;
+              xr[j] = sl == 0 ? hrows[0] : (sl == 1 ? hrows[1] : hrows[2]);
+            }
+          }
+        }
+        // every token from the kFG + 3 x rows (one basic block: the chains interleave)
+#pragma unroll
+        for (int ti = 0; ti < kFG; ++ti) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float2 acc = b2[q];
+#pragma unroll
+            for (int k = 0; k < kConv; ++k) acc = __ffma2_rn(w2[q][k], bf16_pair(xr[ti + k], q), acc);
+            outw[ti][q] = silu_u_half2(acc);
+          }
+        }
+        if (slow) {
+          // rare: tokens at positions 0-2 of their sequence in a thread that
+          // also holds tokens of the sequence before, again with the taps before
+          // the sequence's first token from its history (or zero)
+#pragma unroll
+          for (int ti = 0; ti < kFG; ++ti) {
+            if (!tedge[ti]) continue;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              float2 acc = b2[q];
+#pragma unroll
+              for (int k = 0; k < kConv; ++k) {
+                float2 xv = bf16_pair(xr[ti + k], q);
+                if (k < kW && tpos[ti] + k < kW) {
+                  xv = make_float2(0.f, 0.f);
+                  if (a.hist) {
+                    const bf16* hp =
+                        a.hist + (tseq[ti] * a.d + c0 + 2 * q) * kW + tpos[ti] + k;
+                    xv = make_float2(bf(hp[0]), bf(hp[kW]));
+                  }
+                }
+                acc = __ffma2_rn(w2[q][k], xv, acc);
+              }
+              outw[ti][q] = silu_u_half2(acc);
+            }
+          }
+        }
+      } else {
+        // decode step: the 8 channels' 3 history taps per row (48 contiguous bytes)
+        uint4 hq[kFG][3];
+#pragma unroll
+        for (int ti = 0; ti < kFG; ++ti) {
+#pragma unroll
+          for (int q = 0; q < 3; ++q) hq[ti][q] = make_uint4(0u, 0u, 0u, 0u);
+          if (cin && hrow[ti] >= 0) {
+            const uint4* hp = reinterpret_cast<const uint4*>(a.hist + (hrow[ti] * a.d + c0) * kW);
+#pragma unroll
+            for (int q = 0; q < 3; ++q) hq[ti][q] = __ldg(hp + q);
+          }
+        }
+#pragma unroll
+        for (int ti = 0; ti < kFG; ++ti) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float2 acc = b2[q];
+#pragma unroll
+            for (int k = 0; k < kW; ++k) {
+              const int e0 = (2 * q) * kW + k, e1 = (2 * q + 1) * kW + k;
+              acc = __ffma2_rn(w2[q][k],
+                               make_float2(bf16_lane(hq[ti][e0 >> 3], e0 & 7),
+                                           bf16_lane(hq[ti][e1 >> 3], e1 & 7)),
+                               acc);
+            }
+            acc = __ffma2_rn(w2[q][kW], bf16_pair(xr[ti + kW], q), acc);
+            outw[ti][q] = silu_u_half2(acc);
+          }
+        }
+      }
+      if (!cin) {
+#pragma unroll
+        for (int ti = 0; ti < kFG; ++ti)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) outw[ti][q] = 0u;
+      }
+      // into the A stage: row r, 16-byte chunk cg at cg ^ (r % 8) (128-byte swizzle)
+      uint8_t* at = As + s * kFABytes;
+#pragma unroll
+      for (int ti = 0; ti < kFG; ++ti) {
+        const int r = kFG * tg + ti;
+        *reinterpret_cast<uint4*>(at + r * (kXK * 2) + ((cg ^ (r & 7)) << 4)) =
+            make_uint4(outw[ti][0], outw[ti][1], outw[ti][2], outw[ti][3]);
+      }
+      fence_proxy_async_smem();  // u in the stage, before the tensor cores read it
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&afull[s]));
+    }
+
+    // ---- epilogue (warps 2-9): warp w reads TMEM lanes 32 (w % 4) .. + 31 = tile rows
+    if (warp < 10) {
+      const bool ok = mbar_wait(smem_u32(acc_full), 0, a.err, 89);
+      tc_fence_after();
+      const int lg = warp & 3;
+      const bool lower = warp < 6;  // warps 2-5, else 6-9: two warps per lane group
+      const int64_t g = m0 + lg * 32 + lane;  // this thread's token
+      const uint32_t trow = tmem + ((uint32_t)(lg * 32) << 16);
+      if (a.ksplit == 1) {
+        if (lower) {
+          // dt: sum of squares as k_norms16_warp takes it (lane l: columns l + 32 j
+          // in order, then the xor-butterfly over the lanes)
+          float ps[32];
+#pragma unroll
+          for (int l = 0; l < 32; ++l) ps[l] = 0.0f;
+#pragma unroll 1
+          for (int c = 0; c < a.R; c += 32) {
+            uint32_t r0[16], r1[16];
+            const bool two = c + 16 < a.R;  // R is a multiple of 16
+            tmem_ld16(trow + (uint32_t)c, r0);
+            if (two) tmem_ld16(trow + (uint32_t)(c + 16), r1);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float v = __uint_as_float(r0[e]);
+              ps[e] = fmaf(v, v, ps[e]);
+            }
+            if (two) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                const float v = __uint_as_float(r1[e]);
+                ps[16 + e] = fmaf(v, v, ps[16 + e]);
+              }
+            }
+          }
+#pragma unroll
+          for (int o = 16; o; o >>= 1)
+#pragma unroll
+            for (int l = 0; l < o; ++l) ps[l] = ps[l] + ps[l + o];
+          const float inv = 1.0f / sqrtf(ps[0] / (float)a.R + a.eps);
+#pragma unroll 1
+          for (int c = 0; c < a.R; c += 16) {
+            uint32_t r[16];
+            tmem_ld16(trow + (uint32_t)c, r);
+            tmem_ld_wait();
+            if (ok && g < a.T) {
+              uint32_t hw[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                hw[e] = pack_half2(__uint_as_float(r[2 * e]) * inv * bf(a.dtn_w[c + 2 * e]),
+                                   __uint_as_float(r[2 * e + 1]) * inv * bf(a.dtn_w[c + 2 * e + 1]));
+              uint4* dst = reinterpret_cast<uint4*>(a.dtn + g * a.R + c);
+              dst[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+              dst[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+            }
+          }
+        } else {
+          // B (columns R .. R + 15) and C (R + 16 .. R + 31): 16-lane butterflies
+          uint32_t rv[2][16];
+          tmem_ld16(trow + (uint32_t)a.R, rv[0]);
+          tmem_ld16(trow + (uint32_t)(a.R + 16), rv[1]);
+          tmem_ld_wait();
+          if (ok && g < a.T) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              float sq[16];
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                const float v = __uint_as_float(rv[h][e]);
+                sq[e] = v * v;
+              }
+#pragma unroll
+              for (int o = 8; o; o >>= 1)
+#pragma unroll
+                for (int l = 0; l < o; ++l) sq[l] = sq[l] + sq[l + o];
+              const float inv2 = 1.0f / sqrtf(sq[0] / (float)kN + a.eps);
+              const bf16* wn = h ? a.cn_w : a.bn_w;
+              float4* dst = reinterpret_cast<float4*>(a.bc + g * 2 * kN + h * kN);
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                dst[e] = make_float4(__uint_as_float(rv[h][4 * e]) * inv2 * bf(wn[4 * e]),
+                                     __uint_as_float(rv[h][4 * e + 1]) * inv2 * bf(wn[4 * e + 1]),
+                                     __uint_as_float(rv[h][4 * e + 2]) * inv2 * bf(wn[4 * e + 2]),
+                                     __uint_as_float(rv[h][4 * e + 3]) * inv2 * bf(wn[4 * e + 3]));
+            }
+          }
+        }
+      } else {
+        // partial sums: columns [0, N1) by warps 2-5, [N1, 2 N1) by warps 6-9,
+        // transposed through shared memory (the stages are free once the
+        // accumulator is complete) into 64-byte row segments
+        float* tbuf = reinterpret_cast<float*>(smem) + (warp - 2) * (32 * 17);
+        const int64_t row0 = m0 + lg * 32;
+        float* dst = a.part + ((int64_t)split * a.T) * a.P;
+        const int cbeg = lower ? 0 : a.N1;
+        for (int c0 = cbeg; c0 < cbeg + a.N1; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld16(trow + (uint32_t)c0, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) tbuf[lane * 17 + j] = __uint_as_float(r[j]);
+          __syncwarp();
+          if (ok) {
+            const int col = c0 + (lane & 15);
+#pragma unroll 4
+            for (int rr = 0; rr < 16; ++rr) {
+              const int row = 2 * rr + (lane >> 4);
+              const int64_t gg = row0 + row;
+              if (gg < a.T && col < a.P) dst[gg * a.P + col] = tbuf[row * 17 + (lane & 15)];
+            }
+          }
+          __syncwarp();
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, a.tmem_cols);
+  }
+}
+
 // ------------------------------------------------------- fused dt_proj + scan
 
 struct ScanArgs {
@@ -1522,12 +2019,18 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     // step (the conv kernel only reads the conv states), so it starts at once
     if (lane == 0) {
       prefetch_tmap(&tm_state);
-      for (int64_t p = p0, i = 0; p < p1; ++p, ++i) {
+      // (tile, row) of pair p, advanced by one row per pair (no divisions in the loop)
+      int64_t tile = p0 / a.B, b = p0 - tile * a.B;
+      for (int64_t p = p0, i = 0; p < p1; ++p, ++i, ++b) {
+        if (b == a.B) {
+          b = 0;
+          ++tile;
+        }
         const int s = (int)(i % kDecStages);
         if (i >= kDecStages &&
             !mbar_wait(smem_u32(&empty[s]), (uint32_t)((i / kDecStages) - 1) & 1u, a.err, 41))
           break;
-        const int64_t tile = p / a.B, b = p % a.B, c0 = tile * kSC;
+        const int64_t c0 = tile * kSC;
         const int64_t sl = dec_slot(a, b);
         // channels of this tile that exist (a multiple of 8): the 1-D copies
         // stop there, so none reads past the end of its buffer
@@ -1590,75 +2093,99 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   } else {
     // ---- compute warps: thread = channel c0 + cl of the current tile
     const int cl = warp * 32 + lane;
-    grid_dep_wait();  // W_dt's fp16 copy may come from this step's conv kernel
     int64_t cur_tile = -1;
     bool cok = false;
     int64_t c = 0;
     float2 A2[kN / 2];
     float bias = 0.f, Dc = 0.f, cb = 0.f, cw[kConv] = {0.f, 0.f, 0.f, 0.f};
+    // a new channel tile: its W_dt rows into TMEM (zeros past R and past d),
+    // 16 loads in flight per thread at a time, then the per-channel parameters
+    auto load_tile = [&](int64_t tile) {
+      cur_tile = tile;
+      c = tile * kSC + cl;
+      cok = c < a.d;
+      const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+      const int nq = a.nslab * 2;  // steps of 16 columns = 32 K values
+      for (int q0 = 0; q0 < nq; q0 += 4) {
+        uint4 w8[4][4];
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int kx = (q0 + qq) * 32 + e * 8;
+            w8[qq][e] = (cok && q0 + qq < nq && kx < a.R)
+                            ? __ldg(reinterpret_cast<const uint4*>(a.wdt + c * a.R + kx))
+                            : make_uint4(0u, 0u, 0u, 0u);
+          }
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+          if (q0 + qq >= nq) break;
+          uint32_t v[16];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            v[4 * e] = w8[qq][e].x;
+            v[4 * e + 1] = w8[qq][e].y;
+            v[4 * e + 2] = w8[qq][e].z;
+            v[4 * e + 3] = w8[qq][e].w;
+          }
+          tmem_st16(trow + (uint32_t)((q0 + qq) * 16), v);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(wready));
+#pragma unroll
+      for (int q = 0; q < kN / 2; ++q) {
+        A2[q].x = cok ? -expf(a.A_log[c * kN + 2 * q]) * kLog2e : 0.0f;
+        A2[q].y = cok ? -expf(a.A_log[c * kN + 2 * q + 1]) * kLog2e : 0.0f;
+      }
+      bias = cok ? a.dt_bias[c] : 0.f;
+      Dc = cok ? a.D[c] : 0.f;
+#pragma unroll
+      for (int kx = 0; kx < kConv; ++kx) cw[kx] = cok ? bf(a.conv_w[c * kConv + kx]) : 0.f;
+      cb = cok ? bf(a.conv_b[c]) : 0.f;
+    };
+    // The first tile's W_dt is read before griddepcontrol.wait: when it is this
+    // step's fp16 copy, the kernel that wrote it ran three launches back and has
+    // completed by now (this kernel starts only once every CTA of the norms
+    // kernel passed its own wait, which returned after x_proj completed, and
+    // x_proj waited for the conversion); the weights are inputs otherwise.
+    if (g0 < g1) load_tile(g0 / ngrp);
+    grid_dep_wait();  // dt_n and B/C come from the norms kernel
     int64_t p = p0, i = 0;
     bool ok = true;
     for (int64_t g = g0, k = 0; ok && g < g1; ++g, ++k) {
       const int bsel = (int)(k & 1);
       const int64_t tile = g / ngrp, r0 = (g % ngrp) * kDB;
-      if (tile != cur_tile) {
-        // new channel tile: W_dt rows into TMEM (zeros past R and past d), per-channel params
-        cur_tile = tile;
-        c = tile * kSC + cl;
-        cok = c < a.d;
-        const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-        for (int q = 0; q < a.nslab * 2; ++q) {  // 16 columns = 32 K values per step
-          uint32_t v[16];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int kx = q * 32 + e * 8;
-            uint4 w8 = make_uint4(0u, 0u, 0u, 0u);
-            if (cok && kx < a.R) w8 = __ldg(reinterpret_cast<const uint4*>(a.wdt + c * a.R + kx));
-            v[4 * e] = w8.x;
-            v[4 * e + 1] = w8.y;
-            v[4 * e + 2] = w8.z;
-            v[4 * e + 3] = w8.w;
-          }
-          tmem_st16(trow + (uint32_t)(q * 16), v);
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(wready));
-#pragma unroll
-        for (int q = 0; q < kN / 2; ++q) {
-          A2[q].x = cok ? -expf(a.A_log[c * kN + 2 * q]) * kLog2e : 0.0f;
-          A2[q].y = cok ? -expf(a.A_log[c * kN + 2 * q + 1]) * kLog2e : 0.0f;
-        }
-        bias = cok ? a.dt_bias[c] : 0.f;
-        Dc = cok ? a.D[c] : 0.f;
-#pragma unroll
-        for (int kx = 0; kx < kConv; ++kx) cw[kx] = cok ? bf(a.conv_w[c * kConv + kx]) : 0.f;
-        cb = cok ? bf(a.conv_b[c]) : 0.f;
-      }
+      if (tile != cur_tile) load_tile(tile);
       if (!mbar_wait(smem_u32(&mma_done[bsel]), (uint32_t)(k >> 1) & 1u, a.err, 45)) break;
       tc_fence_after();
       const uint32_t tacc =
           tmem + ((uint32_t)(warp * 32) << 16) + kDecAccCol + (uint32_t)(bsel * kDB);
       const float4* bcs = reinterpret_cast<const float4*>(bc_s + bsel * kDecBC);
+      // the group's rows that fall in [p0, p1): pairs [lo, hi)
+      const int64_t gp0 = tile * a.B + r0;  // pair of the group's first row
+      const int64_t lo = p0 > gp0 ? p0 : gp0;
+      const int64_t gend = gp0 + ((a.B - r0) < kDB ? (a.B - r0) : kDB);
+      const int64_t hi = p1 < gend ? p1 : gend;
       // the group's 16 accumulators in one TMEM load; the rows are taken in
       // order, so the current row's value is kept in racc[0] by shifting
       uint32_t racc[kDB];
       tmem_ld16(tacc, racc);
       tmem_ld_wait();
-      for (int q = (int)((p % a.B) - r0); q > 0; --q) {
+      for (int q = (int)(lo - gp0); q > 0; --q) {
 #pragma unroll
         for (int e = 0; e < kDB - 1; ++e) racc[e] = racc[e + 1];
       }
-      // the rows of this group that fall in [p0, p1)
-      for (; p < p1 && (p / a.B) == tile && (p % a.B) < r0 + kDB; ++p, ++i) {
+      for (p = lo; p < hi; ++p, ++i) {
         const int s = (int)(i % kDecStages);
-        const int j = (int)((p % a.B) - r0);
+        const int j = (int)(p - gp0);
         if (!mbar_wait(smem_u32(&full[s]), (uint32_t)(i / kDecStages) & 1u, a.err, 46)) {
           ok = false;
           break;
         }
-        const int64_t b = p % a.B;
+        const int64_t b = r0 + j;
         const int64_t sl = dec_slot(a, b);
         const uint8_t* st = stages + s * kDecStage;
         // read the stage (state rows are 64-byte swizzled: 16-byte chunk q of
@@ -1859,6 +2386,32 @@ int xproj_ksplit(int64_t T, int64_t d) {
   return ks < 1 ? 1 : (int)ks;
 }
 
+#ifndef JMIX_XCONV
+#define JMIX_XCONV 1  // prefill of sequences of one length: conv inside x_proj (k_xproj_conv)
+#endif
+// Whether steps 1-3 run as k_xproj_conv (plus k_norms16 when split): sequences
+// of one length, dt_rank a multiple of 16.  Depends on the problem's shape only.
+#ifndef JMIX_XCONV_DECODE
+#define JMIX_XCONV_DECODE 1  // decode steps too
+#endif
+bool use_xconv(const Problem& pr) {
+  return JMIX_XCONV && (JMIX_XCONV_DECODE || !pr.decode) && !pr.cu && pr.R % 16 == 0 &&
+         pr.T > 0;
+}
+
+// k_xproj_conv's split over d_inner: one split once the token tiles fill the
+// GPU's 148 SMs (the norms then run in its epilogue), else enough splits for
+// about one CTA per SM.
+int xconv_ksplit(int64_t T, int64_t d) {
+  const int64_t mtiles = (T + kXM - 1) / kXM;
+  const int64_t kchunks = (d + kXK - 1) / kXK;
+  if (mtiles >= 148) return 1;
+  int64_t ks = (148 + mtiles - 1) / mtiles;
+  if (ks > JMIX_XSPLIT_MAX) ks = JMIX_XSPLIT_MAX;
+  if (ks > kchunks) ks = kchunks;
+  return ks < 1 ? 1 : (int)ks;
+}
+
 FastWs fast_layout(const Problem& pr, char* base) {
   FastWs w{};
   size_t off = 0;
@@ -1868,7 +2421,8 @@ FastWs fast_layout(const Problem& pr, char* base) {
     return base ? base + o : nullptr;
   };
   const size_t T = (size_t)pr.T, d = (size_t)pr.d, P = (size_t)pr.P, R = (size_t)pr.R;
-  w.ksplit = xproj_ksplit(pr.T, pr.d);
+  const bool xconv = use_xconv(pr);
+  w.ksplit = xconv ? xconv_ksplit(pr.T, pr.d) : xproj_ksplit(pr.T, pr.d);
   if (!pr.decode && !pr.cu) w.plan = scan_plan(pr.B, pr.L, pr.d);  // packed: one part each
   // hand-over slots: one per (pair, part) when parts exist
   const size_t slots = w.plan.n_parts > 1
@@ -1880,8 +2434,9 @@ FastWs fast_layout(const Problem& pr, char* base) {
   w.carry_h = reinterpret_cast<float*>(take(slots * kSC * kN * 4));
   w.carry_s = reinterpret_cast<float*>(take(slots * kSC * 4));
   w.order = pr.cu ? reinterpret_cast<int*>(take((size_t)pr.B * 4)) : nullptr;
-  w.part = reinterpret_cast<float*>(take((size_t)w.ksplit * T * P * 4));
-  w.u = reinterpret_cast<__half*>(take(T * d * 2));
+  // (k_xproj_conv with one split writes no partial sums, and never u)
+  w.part = reinterpret_cast<float*>(take(xconv && w.ksplit == 1 ? 0 : (size_t)w.ksplit * T * P * 4));
+  w.u = reinterpret_cast<__half*>(take(xconv ? 0 : T * d * 2));
   w.dtn = reinterpret_cast<__half*>(take(T * R * 2));
   w.bc = reinterpret_cast<float*>(take(T * 2 * kN * 4));
   w.wx = reinterpret_cast<__half*>(take(P * d * 2));
@@ -1939,65 +2494,129 @@ cudaError_t run_fast_fwd(Problem& p) {
   if (e != cudaSuccess) return e;
   launches_begin(p);
 
-  // 1. conv + SiLU -> u (fp16); weights -> fp16 (unless prepared once beforehand)
-  {
-    const int G = p.L >= kConvG ? kConvG : 1;
-    const int64_t n_conv = (p.d / 8) * ((p.L + G - 1) / G) * p.B;
-    const int64_t n_wx8 = p.prepared ? 0 : (int64_t)p.P * p.d / 8;
-    const int64_t n_wdt8 = p.prepared ? 0 : p.d * p.R / 8;
-    const int64_t total = n_conv + n_wx8 + n_wdt8;
-    if (p.cu) {
-      const int64_t n_pk = (p.d / 8) * ((p.T + 7) / 8);
-      k_conv_silu16_packed<<<(unsigned)((n_pk + n_wx8 + n_wdt8 + 255) / 256), 256, 0, s>>>(
-          (const bf16*)p.x, (const bf16*)p.conv_w, (const bf16*)p.conv_b,
-          (const bf16*)p.init_conv, p.cu, p.B, p.T, p.d, w.u, n_pk, (const bf16*)p.xproj_w,
-          n_wx8, w.wx, (const bf16*)p.dtproj_w, n_wdt8, w.wdt);
-    } else {
-      auto kern = G == kConvG ? k_conv_silu16<kConvG> : k_conv_silu16<1>;
-      kern<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
-          (const bf16*)p.x, (const bf16*)p.conv_w, (const bf16*)p.conv_b,
-          (const bf16*)p.init_conv, p.sidx, p.n_slots, p.B, p.L, p.d, w.u, n_conv,
-          (const bf16*)p.xproj_w, n_wx8, w.wx, (const bf16*)p.dtproj_w, n_wdt8, w.wdt);
+  if (use_xconv(p)) {
+    // 1-3. W_x, W_dt -> fp16 (unless prepared once beforehand); conv + SiLU
+    // inside x_proj; the norms in its epilogue (one split) or after it
+    const bool convert = !p.prepared;
+    if (convert) {
+      const int64_t n_wx8 = (int64_t)p.P * p.d / 8, n_wdt8 = p.d * p.R / 8;
+      k_conv_silu16<1><<<(unsigned)((n_wx8 + n_wdt8 + 255) / 256), 256, 0, s>>>(
+          (const bf16*)p.x, (const bf16*)p.conv_w, (const bf16*)p.conv_b, nullptr, nullptr, 0,
+          p.B, p.L, p.d, nullptr, 0, (const bf16*)p.xproj_w, n_wx8, w.wx,
+          (const bf16*)p.dtproj_w, n_wdt8, w.wdt);
+      launched(p, "k_convert_weights");
     }
-    launched(p, "k_conv_silu16");
-  }
-  // 2. x_proj on tcgen05
-  {
-    CUtensorMap tu, tw;
-    XprojArgs xa;
+    CUtensorMap tx, tw;
+    XconvArgs xa;
     xa.T = p.T;
+    xa.L = p.L;
+    xa.d = p.d;
     xa.P = (int)p.P;
-    // two column parts of N1 (a multiple of 16), one per CTA of the grid's z
-    xa.N1 = (int)(((p.P + 1) / 2 + 15) / 16 * 16);
-    xa.N2 = xa.N1;
-    xa.Ntot = xa.N1 + xa.N2;
+    xa.R = (int)p.R;
+    xa.N1 = (int)(((p.P + 1) / 2 + 15) / 16 * 16);  // two MMAs of N1 columns
     xa.kchunks = (int)((p.d + kXK - 1) / kXK);
-    const int64_t mtiles = (p.T + kXM - 1) / kXM;
     xa.ksplit = w.ksplit;
-    xa.tmem_cols = xa.N1 <= 32 ? 32 : xa.N1 <= 64 ? 64 : xa.N1 <= 128 ? 128 : 256;
+    xa.tmem_cols = 2 * xa.N1 <= 64 ? 64 : 2 * xa.N1 <= 128 ? 128 : 2 * xa.N1 <= 256 ? 256 : 512;
+    xa.conv_w = (const bf16*)p.conv_w;
+    xa.conv_b = (const bf16*)p.conv_b;
+    xa.hist = (const bf16*)p.init_conv;
+    xa.sidx = p.sidx;
+    xa.n_slots = p.sidx ? p.n_slots : p.B;
     xa.part = w.part;
+    xa.dtn_w = (const bf16*)p.dtn_w;
+    xa.bn_w = (const bf16*)p.bn_w;
+    xa.cn_w = (const bf16*)p.cn_w;
+    xa.eps = p.eps;
+    xa.dtn = w.dtn;
+    xa.bc = w.bc;
     xa.err = err;
-    if (!make_map(&tu, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w.u, p.T, p.d, kXK, kXM, true) ||
+    if (!make_map_swz(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p.x, p.T, p.d, kXK, kFXRows,
+                      CU_TENSOR_MAP_SWIZZLE_NONE) ||
         !make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w.wx, p.P, p.d, kXK, xa.N1, true))
       return cudaErrorInvalidValue;
-    const int smem = 1024 + kXStages * (kXM * 128 + xa.N1 * 128) + 256;
-    cudaFuncSetAttribute(k_xproj, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    e = launch_pdl(k_xproj, dim3((unsigned)(2 * mtiles), (unsigned)xa.ksplit), kXThreads,
-                   (size_t)smem, s, tu, tw, xa);
+    cudaFuncSetAttribute(k_xproj_conv, cudaFuncAttributeMaxDynamicSharedMemorySize, kFSmem);
+    const dim3 grid((unsigned)((p.T + kXM - 1) / kXM), (unsigned)xa.ksplit);
+    if (convert)
+      e = launch_pdl(k_xproj_conv, grid, kFThreads, (size_t)kFSmem, s, tx, tw, xa);
+    else {
+      k_xproj_conv<<<grid, kFThreads, kFSmem, s>>>(tx, tw, xa);
+      e = cudaGetLastError();
+    }
     if (e != cudaSuccess) return e;
-    launched(p, "k_xproj");
+    launched(p, "k_xproj_conv");
+    if (w.ksplit > 1) {
+      if (w.ksplit <= 4)
+        e = launch_pdl(k_norms16_warp<bf16>, dim3((unsigned)((p.T + 7) / 8)), 256, 0, s, w.part,
+                       w.ksplit, (const bf16*)p.dtn_w, (const bf16*)p.bn_w,
+                       (const bf16*)p.cn_w, p.T, (int)p.R, p.eps, w.dtn, w.bc);
+      else
+        e = launch_pdl(k_norms16<bf16, 1>, dim3((unsigned)p.T), kNormThreads, 0, s, w.part,
+                       w.ksplit, (const bf16*)p.dtn_w, (const bf16*)p.bn_w,
+                       (const bf16*)p.cn_w, p.T, (int)p.R, p.eps, w.dtn, w.bc);
+      if (e != cudaSuccess) return e;
+      launched(p, "k_norms16");
+    }
+  } else {
+    // 1. conv + SiLU -> u (fp16); weights -> fp16 (unless prepared once beforehand)
+    {
+      const int G = p.L >= kConvG ? kConvG : 1;
+      const int64_t n_conv = (p.d / 8) * ((p.L + G - 1) / G) * p.B;
+      const int64_t n_wx8 = p.prepared ? 0 : (int64_t)p.P * p.d / 8;
+      const int64_t n_wdt8 = p.prepared ? 0 : p.d * p.R / 8;
+      const int64_t total = n_conv + n_wx8 + n_wdt8;
+      if (p.cu) {
+        const int64_t n_pk = (p.d / 8) * ((p.T + 7) / 8);
+        k_conv_silu16_packed<<<(unsigned)((n_pk + n_wx8 + n_wdt8 + 255) / 256), 256, 0, s>>>(
+            (const bf16*)p.x, (const bf16*)p.conv_w, (const bf16*)p.conv_b,
+            (const bf16*)p.init_conv, p.cu, p.B, p.T, p.d, w.u, n_pk, (const bf16*)p.xproj_w,
+            n_wx8, w.wx, (const bf16*)p.dtproj_w, n_wdt8, w.wdt);
+      } else {
+        auto kern = G == kConvG ? k_conv_silu16<kConvG> : k_conv_silu16<1>;
+        kern<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(
+            (const bf16*)p.x, (const bf16*)p.conv_w, (const bf16*)p.conv_b,
+            (const bf16*)p.init_conv, p.sidx, p.n_slots, p.B, p.L, p.d, w.u, n_conv,
+            (const bf16*)p.xproj_w, n_wx8, w.wx, (const bf16*)p.dtproj_w, n_wdt8, w.wdt);
+      }
+      launched(p, "k_conv_silu16");
+    }
+    // 2. x_proj on tcgen05
+    {
+      CUtensorMap tu, tw;
+      XprojArgs xa;
+      xa.T = p.T;
+      xa.P = (int)p.P;
+      // two column parts of N1 (a multiple of 16), one per CTA of the grid's z
+      xa.N1 = (int)(((p.P + 1) / 2 + 15) / 16 * 16);
+      xa.N2 = xa.N1;
+      xa.Ntot = xa.N1 + xa.N2;
+      xa.kchunks = (int)((p.d + kXK - 1) / kXK);
+      const int64_t mtiles = (p.T + kXM - 1) / kXM;
+      xa.ksplit = w.ksplit;
+      xa.tmem_cols = xa.N1 <= 32 ? 32 : xa.N1 <= 64 ? 64 : xa.N1 <= 128 ? 128 : 256;
+      xa.part = w.part;
+      xa.err = err;
+      if (!make_map(&tu, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w.u, p.T, p.d, kXK, kXM, true) ||
+          !make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w.wx, p.P, p.d, kXK, xa.N1, true))
+        return cudaErrorInvalidValue;
+      const int smem = 1024 + kXStages * (kXM * 128 + xa.N1 * 128) + 256;
+      cudaFuncSetAttribute(k_xproj, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      e = launch_pdl(k_xproj, dim3((unsigned)(2 * mtiles), (unsigned)xa.ksplit), kXThreads,
+                     (size_t)smem, s, tu, tw, xa);
+      if (e != cudaSuccess) return e;
+      launched(p, "k_xproj");
+    }
+    // 3. RMSNorms
+    if (w.ksplit <= 4)
+      e = launch_pdl(k_norms16_warp<bf16>, dim3((unsigned)((p.T + 7) / 8)), 256, 0, s, w.part,
+                     w.ksplit, (const bf16*)p.dtn_w, (const bf16*)p.bn_w, (const bf16*)p.cn_w, p.T,
+                     (int)p.R, p.eps, w.dtn, w.bc);
+    else
+      e = launch_pdl(k_norms16<bf16, 1>, dim3((unsigned)p.T), kNormThreads, 0, s, w.part, w.ksplit,
+                     (const bf16*)p.dtn_w, (const bf16*)p.bn_w, (const bf16*)p.cn_w, p.T, (int)p.R,
+                     p.eps, w.dtn, w.bc);
+    if (e != cudaSuccess) return e;
+    launched(p, "k_norms16");
   }
-  // 3. RMSNorms
-  if (w.ksplit <= 4)
-    e = launch_pdl(k_norms16_warp<bf16>, dim3((unsigned)((p.T + 7) / 8)), 256, 0, s, w.part,
-                   w.ksplit, (const bf16*)p.dtn_w, (const bf16*)p.bn_w, (const bf16*)p.cn_w, p.T,
-                   (int)p.R, p.eps, w.dtn, w.bc);
-  else
-    e = launch_pdl(k_norms16<bf16, 1>, dim3((unsigned)p.T), kNormThreads, 0, s, w.part, w.ksplit,
-                   (const bf16*)p.dtn_w, (const bf16*)p.bn_w, (const bf16*)p.cn_w, p.T, (int)p.R,
-                   p.eps, w.dtn, w.bc);
-  if (e != cudaSuccess) return e;
-  launched(p, "k_norms16");
   // 4. dt_proj + scan + gate
   if (p.decode) {
     CUtensorMap tstate, tdtn, tbc;

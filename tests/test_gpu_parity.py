@@ -37,6 +37,8 @@ def test_fp32_extra_terms_and_ragged(B, L, d, R):
     (2, 3, 256, 16, True),
     (2, 515, 1024, 256, True),    # Jamba rank, ragged L
     (1, 130, 8192, 256, False),   # Jamba shapes, short sequence, the workloads' constants
+    (2, 77, 200, 48, True),       # conv inside x_proj: channel tail in the last 64-channel chunk
+    (2, 9500, 256, 32, True),     # one x_proj split (norms in its epilogue), tiles across sequences
 ])
 def test_bf16_cases(B, L, d, R, extra):
     check_fwd(small(B, L, d, R, extra=extra))
