@@ -684,7 +684,8 @@ __device__ __forceinline__ float2 bf16_pair(const uint4& v, int q) {
 #endif
 // SiLU of a pair, clamped to the fp16 range and packed as fp16x2: the same
 // operations, in the same order, as clamp_half(silu_u(v)) on each element
-// (with JMIX_XCONV_SILU1, as silu_newton).
+// (with JMIX_XCONV_SILU1, as silu_newton), one saturating conversion for the
+// clamp and the rounding.
 __device__ __forceinline__ uint32_t silu_u_half2(float2 v) {
   const float2 t = __fmul2_rn(v, make_float2(-kLog2e, -kLog2e));
   float2 e, r;
@@ -704,7 +705,11 @@ __device__ __forceinline__ uint32_t silu_u_half2(float2 v) {
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r.y) : "f"(den.y));
 #endif
   const float2 s = __fmul2_rn(v, r);
-  return pack_half2(clamp_half(s.x), clamp_half(s.y));
+  // round to fp16, saturating to +-65504: the same bits as clamp_half then
+  // rounding for every number (a NaN stays NaN here)
+  uint32_t h;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(s.y), "f"(s.x));
+  return h;
 }
 
 __global__ void __launch_bounds__(kFThreads, 1)
@@ -1928,7 +1933,12 @@ constexpr int kDecStage = 10240;                          // state | conv | x | 
 static_assert(kDecState + kDecConv + 2 * kDecRow <= kDecStage, "decode stage overflow");
 constexpr int kDecDtn = kMaxSlabs * kDB * 128;            // 8 KB (SW128 slabs)
 constexpr int kDecBC = kDB * 2 * kN * 4;                  // 2 KB
-constexpr int kDecSmem = 1024 + kDecStages * kDecStage + 2 * kDecDtn + 2 * kDecBC + 256;
+// A warp's write-back scratch: 32 state rows (2 KB, 64-byte swizzle) and their
+// conv states (192 B), 512-byte aligned (the swizzle pattern's period).
+constexpr int kDecWb = 2560;
+static_assert(kDecWb >= 32 * kN * 4 + 32 * (kConv - 1) * 2 && kDecWb % 512 == 0, "scratch");
+constexpr int kDecSmem =
+    1024 + kDecStages * kDecStage + 2 * kDecDtn + 2 * kDecBC + 4 * kDecWb + 256;
 static_assert(2 * (kDecSmem + 1024) <= 228 * 1024, "two decode CTAs per SM");
 constexpr uint32_t kDecTmemCols = 256;                    // W_dt [0, 128) | acc 128 + 16 b
 constexpr uint32_t kDecAccCol = 128;
@@ -1964,6 +1974,7 @@ __device__ __forceinline__ int64_t dec_slot(const DecArgs& a, int64_t b) {
 template <bool kZoh>  // B by zero-order hold (else delta B)
 __global__ void __launch_bounds__(kDecThreads, 2)
     k_decode_scan(const __grid_constant__ CUtensorMap tm_state,
+                  const __grid_constant__ CUtensorMap tm_state_wb,
                   const __grid_constant__ CUtensorMap tm_dtn,
                   const __grid_constant__ CUtensorMap tm_bc, const DecArgs a) {
   extern __shared__ uint8_t smem_raw[];
@@ -1973,7 +1984,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   uint8_t* stages = smem;                                  // kDecStages x kDecStage
   uint8_t* dtn_s = stages + kDecStages * kDecStage;        // 2 x kDecDtn
   uint8_t* bc_s = dtn_s + 2 * kDecDtn;                     // 2 x kDecBC
-  uint64_t* bars = reinterpret_cast<uint64_t*>(bc_s + 2 * kDecBC);
+  uint8_t* wb_s = bc_s + 2 * kDecBC;                       // 4 x kDecWb
+  uint64_t* bars = reinterpret_cast<uint64_t*>(wb_s + 4 * kDecWb);
   uint64_t* full = bars;                                   // [stages] row landed
   uint64_t* empty = bars + kDecStages;                     // [stages] row read (4 warps)
   uint64_t* gfull = bars + 2 * kDecStages;                 // [2] dt_n + B/C landed
@@ -2153,6 +2165,19 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     // x_proj waited for the conversion); the weights are inputs otherwise.
     if (g0 < g1) load_tile(g0 / ngrp);
     grid_dep_wait();  // dt_n and B/C come from the norms kernel
+    // A row's new SSM and conv state go to global memory through the warp's
+    // scratch rows (64-byte swizzled like the stage): one tensor store and one
+    // bulk store issued by lane 0, whose reads of the scratch are waited for
+    // only one row later, so the stores leave the row's dependency chain.
+    uint8_t* wb = wb_s + warp * kDecWb;
+    bool pend = false;
+    auto wb_flush = [&]() {
+      // the tensor store of one row ago has read the scratch (lane 0 issued it)
+      if (!pend) return;
+      if (lane == 0) bulk_wait_read<0>();
+      __syncwarp();
+      pend = false;
+    };
     int64_t p = p0, i = 0;
     bool ok = true;
     for (int64_t g = g0, k = 0; ok && g < g1; ++g, ++k) {
@@ -2187,9 +2212,9 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         }
         const int64_t b = r0 + j;
         const int64_t sl = dec_slot(a, b);
-        const uint8_t* st = stages + s * kDecStage;
         // read the stage (state rows are 64-byte swizzled: 16-byte chunk q of
         // row cl sits at chunk q ^ ((cl >> 1) & 3)), then release it
+        const uint8_t* st = stages + s * kDecStage;
         float2 h[kN / 2];
         float sv[kConv - 1];
         float xt, zv;
@@ -2219,6 +2244,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         if (lane == 0) mbar_arrive(smem_u32(&empty[s]));
         if (sl < 0) {
           if (cl == 0 && atomicExch(&a.err->bad_input, 1u) == 0u) a.err->where = kSiteBadSlot;
+#pragma unroll
+          for (int e = 0; e < kDB - 1; ++e) racc[e] = racc[e + 1];  // the next row's first
           continue;
         }
         float xc = fmaf(cw[0], sv[0], cb);
@@ -2259,21 +2286,38 @@ __global__ void __launch_bounds__(kDecThreads, 2)
           const float2 sa = __fadd2_rn(__fadd2_rn(acc[0], acc[1]), __fadd2_rn(acc[2], acc[3]));
           const float ys = (sa.x + sa.y) + Dc * uv;
           a.y[b * a.d + c] = __float2bfloat16_rn(ys * silu_gate(zv));
-          float4* hs = reinterpret_cast<float4*>(a.ssm_state + (sl * a.d + c) * kN);
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            hs[q] = make_float4(h[2 * q].x, h[2 * q].y, h[2 * q + 1].x, h[2 * q + 1].y);
-          uint16_t* cs =
-              reinterpret_cast<uint16_t*>(a.conv_state + (sl * a.d + c) * (kConv - 1));
-          cs[0] = (uint16_t)(__float_as_uint(sv[1]) >> 16);
-          cs[1] = (uint16_t)(__float_as_uint(sv[2]) >> 16);
-          cs[2] = (uint16_t)xraw;
         }
+        // the previous row's stores have read the scratch; this row's state goes into it
+        wb_flush();
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          *reinterpret_cast<float4*>(wb + lane * 64 + 16 * (q ^ ((lane >> 1) & 3))) =
+              make_float4(h[2 * q].x, h[2 * q].y, h[2 * q + 1].x, h[2 * q + 1].y);
+        uint16_t* csw = reinterpret_cast<uint16_t*>(wb + 32 * 64) + lane * 3;
+        csw[0] = (uint16_t)(__float_as_uint(sv[1]) >> 16);
+        csw[1] = (uint16_t)(__float_as_uint(sv[2]) >> 16);
+        csw[2] = (uint16_t)xraw;
+        // one tensor store of the warp's [32 channels x 16] rows (channels past d
+        // are outside the map and not written) and one bulk store of their conv
+        // states, both reading the scratch
+        const int64_t wc0 = c - lane;  // the warp's first channel
+        const int64_t nv64 = a.d - wc0;
+        const int nvalid = nv64 < 32 ? (int)nv64 : 32;  // of its channels that exist (may be <= 0)
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && nvalid > 0) {
+          tma_store_3d(&tm_state_wb, smem_u32(wb), 0, (int32_t)wc0, (int32_t)sl);
+          bulk_store(a.conv_state + (sl * a.d + wc0) * (kConv - 1), smem_u32(wb + 32 * 64),
+                     (uint32_t)(nvalid * 6));
+          bulk_commit();
+        }
+        pend = true;
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&acc_free[bsel]));
     }
+    if (lane == 0) bulk_wait_all();
   }
   tc_fence_before();
   __syncthreads();
@@ -2318,15 +2362,16 @@ bool make_map_swz(CUtensorMap* m, CUtensorMapDataType dt, size_t esize, const vo
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 3-D tensor map of an SSM-state pool [slots, d, 16] fp32 with box [1, 128, 16]
-// and 64-byte swizzle: a box never reaches past its slot's channels, so a tile
-// store at the last channel tile writes only channels that exist.
-bool make_state_map(CUtensorMap* m, const float* base, uint64_t slots, uint64_t d) {
+// 3-D tensor map of an SSM-state pool [slots, d, 16] fp32 with box [1, box_rows,
+// 16] and 64-byte swizzle: a box never reaches past its slot's channels, so a
+// tile store at the last channel tile writes only channels that exist.
+bool make_state_map(CUtensorMap* m, const float* base, uint64_t slots, uint64_t d,
+                    uint32_t box_rows = kSC) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {(cuuint64_t)kN, d, slots};
   cuuint64_t strides[2] = {(cuuint64_t)kN * 4, d * kN * 4};
-  cuuint32_t box[3] = {(cuuint32_t)kN, (cuuint32_t)kSC, 1};
+  cuuint32_t box[3] = {(cuuint32_t)kN, box_rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box,
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
@@ -2389,10 +2434,13 @@ int xproj_ksplit(int64_t T, int64_t d) {
 #ifndef JMIX_XCONV
 #define JMIX_XCONV 1  // prefill of sequences of one length: conv inside x_proj (k_xproj_conv)
 #endif
-// Whether steps 1-3 run as k_xproj_conv (plus k_norms16 when split): sequences
-// of one length, dt_rank a multiple of 16.  Depends on the problem's shape only.
+// Whether steps 1-3 run as k_xproj_conv (plus k_norms16 when split): prefill
+// of sequences of one length, dt_rank a multiple of 16.  Depends on the
+// problem's shape only.
 #ifndef JMIX_XCONV_DECODE
-#define JMIX_XCONV_DECODE 1  // decode steps too
+// decode steps too (measured slower at 256 rows: the separate weight
+// conversion launch costs more than the fused conv saves)
+#define JMIX_XCONV_DECODE 0
 #endif
 bool use_xconv(const Problem& pr) {
   return JMIX_XCONV && (JMIX_XCONV_DECODE || !pr.decode) && !pr.cu && pr.R % 16 == 0 &&
@@ -2619,9 +2667,10 @@ cudaError_t run_fast_fwd(Problem& p) {
   }
   // 4. dt_proj + scan + gate
   if (p.decode) {
-    CUtensorMap tstate, tdtn, tbc;
+    CUtensorMap tstate, tstate_wb, tdtn, tbc;
     const int64_t slots = p.sidx ? p.n_slots : p.B;
     if (!make_state_map(&tstate, p.final_state, (uint64_t)slots, (uint64_t)p.d) ||
+        !make_state_map(&tstate_wb, p.final_state, (uint64_t)slots, (uint64_t)p.d, 32) ||
         !make_map(&tdtn, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w.dtn, p.T, p.R, 64, kDB, true) ||
         !make_map(&tbc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, w.bc, p.T, 2 * kN, 2 * kN, kDB,
                   false))
@@ -2650,7 +2699,8 @@ cudaError_t run_fast_fwd(Problem& p) {
     auto dec_kern = p.zoh ? k_decode_scan<true> : k_decode_scan<false>;
     cudaFuncSetAttribute(dec_kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
     const int64_t ctas = std::min<int64_t>(2 * num_sms(), da.pairs);
-    e = launch_pdl(dec_kern, (unsigned)ctas, kDecThreads, kDecSmem, s, tstate, tdtn, tbc, da);
+    e = launch_pdl(dec_kern, (unsigned)ctas, kDecThreads, kDecSmem, s, tstate, tstate_wb, tdtn,
+                   tbc, da);
     if (e != cudaSuccess) return e;
     launched(p, "k_decode_scan");
   } else {

@@ -160,3 +160,13 @@ def test_slot_outside_the_pool_is_reported_and_skipped():
     for s in (1, 2, 4, 5):                                                  # slots no row used
         assert torch.equal(cp[s], c0[s]) and torch.equal(sp[s], s0[s])
     assert not torch.equal(sp[3], s0[3]) and not torch.equal(sp[0], s0[0])
+    # the rows after a skipped one are computed exactly as when every slot is valid
+    cp2, sp2 = devio.to_device(c_h), devio.to_device(s_h)
+    yt2 = torch.full_like(xt, 7.0)
+    idx2 = torch.tensor([3, 1, 0, 2], dtype=torch.int32, device="cuda")
+    jmix.jm_mixer_step_indexed(d, idx2, 6, xt, zt, cp2, sp2, Wd, None, yt2, ws, n)
+    assert jmix.jm_poll_error(ws) == jmix.JM_OK, jmix.jm_last_error()
+    torch.cuda.synchronize()
+    assert torch.equal(yt[0], yt2[0]) and torch.equal(yt[2], yt2[2])
+    for s in (3, 0):
+        assert torch.equal(cp[s], cp2[s]) and torch.equal(sp[s], sp2[s])
