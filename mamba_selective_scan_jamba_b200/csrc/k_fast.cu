@@ -52,7 +52,7 @@ constexpr int kXStages = 3;
 #define JMIX_XPROJ_CTAS 296
 #endif
 #ifndef JMIX_XSPLIT_MAX
-#define JMIX_XSPLIT_MAX 32
+#define JMIX_XSPLIT_MAX 16  // (32 measured ~1 us slower on a 256-row decode step)
 #endif
 constexpr int kMaxSplit = JMIX_XSPLIT_MAX;  // x_proj splits over d_inner, at most
 #ifndef JMIX_SCAN_CHUNK
