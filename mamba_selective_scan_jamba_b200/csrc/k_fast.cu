@@ -1365,6 +1365,8 @@ __device__ __forceinline__ void scan_recur(const TokTerms& T, const float4* bcs,
                                            const float2 (&invA)[kN / 2], bf16* yrow,
                                            int64_t tbase, int64_t d, bool cok, bf16* ys_smem,
                                            int cl) {
+  static_assert(!kYS || (kFull && kG % 2 == 0), "y through the stage: whole groups of token pairs");
+  float yprev = 0.0f;  // (kYS) the even token's y, rounded with the odd one's
 #pragma unroll
   for (int i = 0; i < kG; ++i) {
     const int t = g0t + i;
@@ -1402,9 +1404,17 @@ __device__ __forceinline__ void scan_recur(const TokTerms& T, const float4* bcs,
       const float2 s23 = __fadd2_rn(acc[2], acc[3]);
       const float2 sa = __fadd2_rn(s01, s23);
       const float ys = (sa.x + sa.y) + T.dsk[i];
-      if constexpr (kYS)  // into the stage's x tile (token t's x is already read)
-        ys_smem[t * kSC + cl] = __float2bfloat16_rn(ys * T.gz[i]);
-      else if (cok)
+      if constexpr (kYS) {
+        // into the stage's x tile (tokens t - 1 and t's x are already read); two
+        // tokens' y are rounded to bf16 by one paired conversion (same bits)
+        if (i & 1) {
+          const __nv_bfloat162 y2 = __floats2bfloat162_rn(yprev, ys * T.gz[i]);
+          ys_smem[(t - 1) * kSC + cl] = y2.x;
+          ys_smem[t * kSC + cl] = y2.y;
+        } else {
+          yprev = ys * T.gz[i];
+        }
+      } else if (cok)
         yrow[(tbase + t) * d] = __float2bfloat16_rn(ys * T.gz[i]);
     }
   }
