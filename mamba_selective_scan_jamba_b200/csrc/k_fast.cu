@@ -1965,7 +1965,8 @@ struct DecArgs {
   const float* dt_bias;
   const float* A_log;
   const float* D;
-  const __half* wdt;   // W_dt in fp16 [d, R]
+  const uint16_t* wdt;  // W_dt [d, R]: the prepared fp16 copy, or (wdt_bf16) the bf16 input,
+  int wdt_bf16;         // which is rounded to fp16 on its way into TMEM
   bf16* conv_state;    // [B, d, 3] in/out (indexed: [n_slots, d, 3])
   float* ssm_state;    // [B, d, 16] in/out (indexed: [n_slots, d, 16])
   bf16* y;
@@ -2145,10 +2146,19 @@ __global__ void __launch_bounds__(kDecThreads, 2)
           uint32_t v[16];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            v[4 * e] = w8[qq][e].x;
-            v[4 * e + 1] = w8[qq][e].y;
-            v[4 * e + 2] = w8[qq][e].z;
-            v[4 * e + 3] = w8[qq][e].w;
+            if (a.wdt_bf16) {  // 8 bf16 -> 8 fp16, rounded as the weight conversion rounds
+              float o[8];
+              unpack8_bf16(w8[qq][e], o);
+              v[4 * e] = pack_half2(o[0], o[1]);
+              v[4 * e + 1] = pack_half2(o[2], o[3]);
+              v[4 * e + 2] = pack_half2(o[4], o[5]);
+              v[4 * e + 3] = pack_half2(o[6], o[7]);
+            } else {
+              v[4 * e] = w8[qq][e].x;
+              v[4 * e + 1] = w8[qq][e].y;
+              v[4 * e + 2] = w8[qq][e].z;
+              v[4 * e + 3] = w8[qq][e].w;
+            }
           }
           tmem_st16(trow + (uint32_t)((q0 + qq) * 16), v);
         }
@@ -2168,11 +2178,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       for (int kx = 0; kx < kConv; ++kx) cw[kx] = cok ? bf(a.conv_w[c * kConv + kx]) : 0.f;
       cb = cok ? bf(a.conv_b[c]) : 0.f;
     };
-    // The first tile's W_dt is read before griddepcontrol.wait: when it is this
-    // step's fp16 copy, the kernel that wrote it ran three launches back and has
-    // completed by now (this kernel starts only once every CTA of the norms
-    // kernel passed its own wait, which returned after x_proj completed, and
-    // x_proj waited for the conversion); the weights are inputs otherwise.
+    // The first tile's W_dt (an input, or its copy prepared before the call) is
+    // read before griddepcontrol.wait.
     if (g0 < g1) load_tile(g0 / ngrp);
     grid_dep_wait();  // dt_n and B/C come from the norms kernel
     // A row's new SSM and conv state go to global memory through the warp's
@@ -2620,7 +2627,8 @@ cudaError_t run_fast_fwd(Problem& p) {
       const int G = p.L >= kConvG ? kConvG : 1;
       const int64_t n_conv = (p.d / 8) * ((p.L + G - 1) / G) * p.B;
       const int64_t n_wx8 = p.prepared ? 0 : (int64_t)p.P * p.d / 8;
-      const int64_t n_wdt8 = p.prepared ? 0 : p.d * p.R / 8;
+      // (a decode step rounds W_dt to fp16 as it loads it into TMEM)
+      const int64_t n_wdt8 = (p.prepared || p.decode) ? 0 : p.d * p.R / 8;
       const int64_t total = n_conv + n_wx8 + n_wdt8;
       if (p.cu) {
         const int64_t n_pk = (p.d / 8) * ((p.T + 7) / 8);
@@ -2699,7 +2707,10 @@ cudaError_t run_fast_fwd(Problem& p) {
     da.dt_bias = p.dt_bias;
     da.A_log = p.A_log;
     da.D = p.D;
-    da.wdt = w.wdt;
+    // the prepared fp16 W_dt when there is one, else the bf16 input
+    da.wdt = p.prepared ? reinterpret_cast<const uint16_t*>(w.wdt)
+                        : reinterpret_cast<const uint16_t*>(p.dtproj_w);
+    da.wdt_bf16 = p.prepared ? 0 : 1;
     da.conv_state = (bf16*)p.final_conv;
     da.ssm_state = p.final_state;
     da.y = (bf16*)p.y;
