@@ -614,7 +614,8 @@ __global__ void __launch_bounds__(256) k_norms16_warp(
 }
 
 // ------------------------------------------------ conv + SiLU inside x_proj
-// The prefill form of steps 1-3 for sequences of one length (T = B L tokens):
+// The prefill form of steps 1-3 (sequences of one length, T = B L tokens, or a
+// packed batch whose tokens find their sequence in cu):
 // x_proj's A operand u = SiLU(conv(x)) is computed in shared memory from TMA
 // tiles of x, so u never goes through global memory (the scan recomputes its
 // own u in float32).  Grid (token tiles of 128, splits of d_inner); each CTA
@@ -661,6 +662,8 @@ struct XconvArgs {
   const bf16* conv_w;  // [d, 4]
   const bf16* conv_b;  // [d]
   const bf16* hist;    // [B, d, 3] conv history of each sequence, or null (zeros)
+  const int* cu;       // packed batch: [B + 1] token offsets of the sequences, or null
+  int64_t nseq;        // packed batch: sequences B
   const int* sidx;     // decode step (L == 1): history slot of each row, or null (slot = row)
   int64_t n_slots;     // decode step: slots of the history pool
   float* part;         // [ksplit, T, P] partial sums (ksplit > 1)
@@ -813,9 +816,21 @@ __global__ void __launch_bounds__(kFThreads, 1)
 #pragma unroll
     for (int ti = 0; ti < kFG; ++ti) {
       const int64_t g = m0 + kFG * tg + ti;
-      tseq[ti] = g / a.L;
-      tpos[ti] = (int)(g - tseq[ti] * a.L);
-      tedge[ti] = g < a.T && tpos[ti] < kW;
+      if (a.cu) {
+        // packed batch: the last sequence whose first token is at or before g
+        // (clamped to [0, B); a broken cu is reported by the scan kernel)
+        int lo = 0, hi = (int)a.nseq - 1;
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (__ldg(a.cu + mid) <= g) lo = mid; else hi = mid - 1;
+        }
+        tseq[ti] = lo;
+        tpos[ti] = (int)(g - __ldg(a.cu + lo));
+      } else {
+        tseq[ti] = g / a.L;
+        tpos[ti] = (int)(g - tseq[ti] * a.L);
+      }
+      tedge[ti] = g < a.T && tpos[ti] >= 0 && tpos[ti] < kW;
       edge |= tedge[ti];
     }
     // When the thread's first token is at position < 3 and all its tokens lie
@@ -823,12 +838,12 @@ __global__ void __launch_bounds__(kFThreads, 1)
     // before the sequence are needed by this thread alone: they are replaced by
     // the history rows once per chunk, and the common path computes the rest.
     // Other layouts of sequence starts recompute their edge tokens (slow).
-    const bool sub = tedge[0] && tpos[0] + kFG <= a.L;
+    const bool sub = tedge[0] && tseq[kFG - 1] == tseq[0];
     const bool slow = edge && !sub;
     // decode step (L == 1): every tap but the last is history; a row's history
     // sits in its pool slot, clamped into the pool (a bad slot is reported and
     // skipped by the decode kernel), -1 for rows past T
-    const bool step = a.L == 1;
+    const bool step = a.L == 1 && !a.cu;
     int64_t hrow[kFG];
 #pragma unroll
     for (int ti = 0; ti < kFG; ++ti) {
@@ -2452,16 +2467,15 @@ int xproj_ksplit(int64_t T, int64_t d) {
 #define JMIX_XCONV 1  // prefill of sequences of one length: conv inside x_proj (k_xproj_conv)
 #endif
 // Whether steps 1-3 run as k_xproj_conv (plus k_norms16 when split): prefill
-// of sequences of one length, dt_rank a multiple of 16.  Depends on the
-// problem's shape only.
+// (sequences of one length or a packed batch), dt_rank a multiple of 16.
+// Depends on the problem's shape only.
 #ifndef JMIX_XCONV_DECODE
 // decode steps too (measured slower at 256 rows: the separate weight
 // conversion launch costs more than the fused conv saves)
 #define JMIX_XCONV_DECODE 0
 #endif
 bool use_xconv(const Problem& pr) {
-  return JMIX_XCONV && (JMIX_XCONV_DECODE || !pr.decode) && !pr.cu && pr.R % 16 == 0 &&
-         pr.T > 0;
+  return JMIX_XCONV && (JMIX_XCONV_DECODE || !pr.decode) && pr.R % 16 == 0 && pr.T > 0;
 }
 
 // k_xproj_conv's split over d_inner: one split once the token tiles fill the
@@ -2585,6 +2599,8 @@ cudaError_t run_fast_fwd(Problem& p) {
     xa.conv_w = (const bf16*)p.conv_w;
     xa.conv_b = (const bf16*)p.conv_b;
     xa.hist = (const bf16*)p.init_conv;
+    xa.cu = p.cu;
+    xa.nseq = p.B;
     xa.sidx = p.sidx;
     xa.n_slots = p.sidx ? p.n_slots : p.B;
     xa.part = w.part;
