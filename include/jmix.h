@@ -168,9 +168,8 @@ jm_status jm_mixer_step_indexed(const jm_dims* dims, const int32_t* state_idx, i
                                 void* workspace, size_t ws_bytes, jm_stream_t stream);
 
 /* jm_mixer_step without a caller workspace, for callers that cannot allocate
- * device memory: code inside CUDA stream capture (where cudaMalloc is not
- * allowed), serving engines that hand all device memory to their own caches
- * and give plug-ins no allocator, or host code that must stay off the
+ * device memory: serving engines that hand all device memory to their own
+ * caches and give plug-ins no allocator, or host code that must stay off the
  * allocator.  The paper has no counterpart to this entry point.
  *
  * Arguments and results are those of jm_mixer_step without workspace and
@@ -181,8 +180,7 @@ jm_status jm_mixer_step_indexed(const jm_dims* dims, const int32_t* state_idx, i
  * message and launches nothing.  The function itself allocates nothing.
  *
  * The first call on a device looks up the array's device address (once per
- * device, with that device current); make that first call before any stream
- * capture.  All calls share the one array, and each call clears what it needs
+ * device, with that device current).  All calls share the one array, and each call clears what it needs
  * cleared, so the previous call's contents never leak into a result; but two
  * calls whose kernels overlap on the GPU (different streams, or different
  * host threads on one device) race on the array and must be serialised by the

@@ -1,10 +1,9 @@
 // jm_mixer_step_noalloc: the decode step with its scratch in a static device
 // array, for callers that cannot allocate device memory themselves.
 //
-// Some callers have no way to get scratch memory for a step: code running
-// inside CUDA stream capture (cudaMalloc is not allowed there), serving
-// engines that reserve all device memory up front for their caches and expose
-// no allocator to plug-ins, and host code that must not touch the allocator at
+// Some callers have no way to get scratch memory for a step: serving engines
+// that reserve all device memory up front for their caches and expose no
+// allocator to plug-ins, and host code that must not touch the allocator at
 // all.  This entry point needs nothing from them beyond the step's own inputs
 // and outputs: its scratch is the file-scope array below, which every GPU that
 // loads libjmix holds until the process exits.

@@ -1,6 +1,5 @@
 """jm_mixer_step_noalloc: the decode step for callers that cannot allocate
-device memory (code inside stream capture, engines that give plug-ins no
-allocator).  Its scratch is a static device array inside libjmix; these tests
+device memory (engines that give plug-ins no allocator).  Its scratch is a static device array inside libjmix; these tests
 check it against jm_mixer_step with a caller workspace, on two steps in a row.
 
 This file is collected last on purpose, so that a run stopping at the first
