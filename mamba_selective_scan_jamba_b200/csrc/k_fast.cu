@@ -2057,6 +2057,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     // step (the conv kernel only reads the conv states), so it starts at once
     if (lane == 0) {
       prefetch_tmap(&tm_state);
+      const uint64_t evict_first = l2_evict_first_policy();
       // (tile, row) of pair p, advanced by one row per pair (no divisions in the loop)
       int64_t tile = p0 / a.B, b = p0 - tile * a.B;
       for (int64_t p = p0, i = 0; p < p1; ++p, ++i, ++b) {
@@ -2078,7 +2079,9 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         const uint32_t fb = smem_u32(&full[s]);
         if (sl >= 0) {
           mbar_arrive_expect_tx(fb, (uint32_t)kDecState + conv_bytes + 2 * row_bytes);
-          tma_load_3d(smem_u32(st), &tm_state, fb, 0, (int32_t)c0, (int32_t)sl);
+          // (the state is streamed through once a step: evict-first in L2, for
+          // the load and for the tensor store that writes it back)
+          tma_load_3d(smem_u32(st), &tm_state, fb, 0, (int32_t)c0, (int32_t)sl, evict_first);
           bulk_load(smem_u32(st + kDecState), a.conv_state + (sl * a.d + c0) * (kConv - 1),
                     conv_bytes, fb);
         } else {
@@ -2338,7 +2341,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0 && nvalid > 0) {
-          tma_store_3d(&tm_state_wb, smem_u32(wb), 0, (int32_t)wc0, (int32_t)sl);
+          tma_store_3d(&tm_state_wb, smem_u32(wb), 0, (int32_t)wc0, (int32_t)sl,
+                       l2_evict_first_policy());
           bulk_store(a.conv_state + (sl * a.d + wc0) * (kConv - 1), smem_u32(wb + 32 * 64),
                      (uint32_t)(nvalid * 6));
           bulk_commit();
