@@ -1,17 +1,27 @@
 // The bf16-io path of the mixer core on sm_100a.
 //
-//   k_conv_silu16   u = SiLU(conv1d(x) + conv_b) rounded to fp16, the x_proj
-//                   operand; the same launch converts xproj_w and dtproj_w from
-//                   bf16 to fp16 (exact for |w| >= 2^-14; fp16 subnormals below).
-//   k_xproj         p = u . xproj_w^T on tcgen05 (TMA -> SMEM -> MMA -> TMEM),
-//                   split over d_inner; each split stores its partial tile.
-//   k_norms16       sums the x_proj partials in a fixed order (so results are
-//                   bitwise reproducible), then dt_n (fp16, the dt_proj operand),
-//                   B_n and C_n (fp32) = RMSNorm(.) w.
-//   k_scan_fused    per (sequence, 128 channels): dt_proj on tcgen05 into TMEM,
-//                   softplus, the conv + SiLU recomputed in fp32 from x, the
-//                   selective scan with fp32 state in registers, the D skip, the
-//                   SiLU(z) gate, the final SSM and conv states.
+// Prefill (a batch of sequences of one length, or a packed batch):
+//   k_conv_silu16<1>  (no conv work: "k_convert_weights") xproj_w and dtproj_w
+//                     from bf16 to fp16 (exact for |w| >= 2^-14; fp16
+//                     subnormals below), unless prepared once beforehand.
+//   k_xproj_conv      u = SiLU(conv1d(x) + conv_b) in fp16, computed into the A
+//                     operand of p = u . xproj_w^T on tcgen05 (TMA -> SMEM ->
+//                     MMA -> TMEM); with one split over d_inner the RMSNorms in
+//                     its epilogue give dt_n (fp16, the dt_proj operand) and
+//                     B_n, C_n (fp32); with several each split stores its
+//                     partial tile for k_norms16.
+//   k_scan_fused      per (sequence, 128 channels): dt_proj on tcgen05 into
+//                     TMEM, softplus, the conv + SiLU recomputed in fp32 from x,
+//                     the selective scan with fp32 state in registers, the D
+//                     skip, the SiLU(z) gate, the final SSM and conv states.
+// Decode step (one token per row, states updated in place):
+//   k_conv_step       u from x_t and each row's cached conv history; W_x to fp16.
+//   k_xproj           p = u . xproj_w^T on tcgen05, split over d_inner.
+//   k_norms16         sums the x_proj partials in a fixed order (so results are
+//                     bitwise reproducible), then the three RMSNorms.
+//   k_decode_scan     dt_proj on tcgen05 + the one-token update of the states.
+// (A dt_rank that is not a multiple of 16 runs k_conv_silu16 / _packed,
+// k_xproj and k_norms16 in place of k_xproj_conv.)
 //
 // Precision: the quantised intermediates are the two tensor-core operands, u
 // for x_proj and dt_n for dt_proj, in fp16 (10 mantissa bits; their rounding
@@ -506,6 +516,15 @@ __global__ void __launch_bounds__(kNormThreads) k_norms16(
     const W* __restrict__ wb, const W* __restrict__ wc, int64_t Tn, int R, float eps,
     __half* __restrict__ dtn, float* __restrict__ bc) {
   __shared__ float rows[TPB][kMaxP];
+  const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
+  // the norm weights this lane applies (inputs: loaded before the wait)
+  float wk[kMaxRank / 32];
+#pragma unroll
+  for (int j = 0; j < kMaxRank / 32; ++j) {
+    const int k = lane + 32 * j;
+    wk[j] = k < R ? (float)__ldg(wdt + k) : 0.0f;
+  }
+  const float wv = lane < kN ? (float)__ldg(wb + lane) : (float)__ldg(wc + lane - kN);
   grid_dep_wait();    // the partial sums come from x_proj
   grid_dep_launch();
   const int64_t g0 = (int64_t)blockIdx.x * TPB;
@@ -528,7 +547,6 @@ __global__ void __launch_bounds__(kNormThreads) k_norms16(
     rows[tl][j] = acc;
   }
   __syncthreads();
-  const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
   for (int tl = wi; tl < TPB; tl += kNormThreads / 32) {
     const int64_t g = g0 + tl;
     if (g >= Tn) break;
@@ -538,14 +556,16 @@ __global__ void __launch_bounds__(kNormThreads) k_norms16(
 #pragma unroll
     for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     const float inv = 1.0f / sqrtf(ss / (float)R + eps);
-    for (int k = lane; k < R; k += 32)
-      dtn[g * R + k] = __float2half_rn(row[k] * inv * (float)wdt[k]);
+#pragma unroll
+    for (int j = 0; j < kMaxRank / 32; ++j) {
+      const int k = lane + 32 * j;
+      if (k < R) dtn[g * R + k] = __float2half_rn(row[k] * inv * wk[j]);
+    }
     const float v = row[R + lane];
     float s2 = v * v;
 #pragma unroll
     for (int o = 8; o; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
     const float inv2 = 1.0f / sqrtf(s2 / (float)kN + eps);
-    const float wv = lane < 16 ? (float)wb[lane] : (float)wc[lane - 16];
     bc[g * 2 * kN + lane] = v * inv2 * wv;
   }
 }
@@ -559,9 +579,17 @@ __global__ void __launch_bounds__(256) k_norms16_warp(
     const W* __restrict__ wb, const W* __restrict__ wc, int64_t Tn, int R, float eps,
     __half* __restrict__ dtn, float* __restrict__ bc) {
   constexpr int kCols = kMaxP / 32;
+  const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
+  // the norm weights this lane applies (inputs: loaded before the wait)
+  float wk[kCols];
+#pragma unroll
+  for (int jj = 0; jj < kCols; ++jj) {
+    const int j = lane + 32 * jj;
+    wk[jj] = j < R ? (float)__ldg(wdt + j) : 0.0f;
+  }
+  const float wv = lane < kN ? (float)__ldg(wb + lane) : (float)__ldg(wc + lane - kN);
   grid_dep_wait();    // the partial sums come from x_proj
   grid_dep_launch();
-  const int lane = threadIdx.x & 31, wi = threadIdx.x >> 5;
   const int64_t g = (int64_t)blockIdx.x * 8 + wi;
   if (g >= Tn) return;
   const int P = R + 2 * kN;
@@ -594,7 +622,7 @@ __global__ void __launch_bounds__(256) k_norms16_warp(
 #pragma unroll
   for (int jj = 0; jj < kCols; ++jj) {
     const int j = lane + 32 * jj;
-    if (j < R) dtn[g * R + j] = __float2half_rn(row[jj] * inv * (float)wdt[j]);
+    if (j < R) dtn[g * R + j] = __float2half_rn(row[jj] * inv * wk[jj]);
   }
   // B and C occupy columns [R, R + 32): R is a multiple of 8, so pick them up by shuffles
   float bcv = 0.f;
@@ -609,7 +637,6 @@ __global__ void __launch_bounds__(256) k_norms16_warp(
 #pragma unroll
   for (int o = 8; o; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
   const float inv2 = 1.0f / sqrtf(s2 / (float)kN + eps);
-  const float wv = lane < 16 ? (float)wb[lane] : (float)wc[lane - 16];
   bc[g * 2 * kN + lane] = bcv * inv2 * wv;
 }
 
@@ -713,6 +740,114 @@ __device__ __forceinline__ uint32_t silu_u_half2(float2 v) {
   uint32_t h;
   asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(s.y), "f"(s.x));
   return h;
+}
+
+// ------------------------------------------------- conv + SiLU of a decode step
+// One token per row (L = 1): every tap but the last comes from the row's cached
+// history (its pool slot for an indexed step, clamped into the pool; a bad slot
+// is reported and skipped by the decode kernel).  Thread = 8 channels of
+// kStepRows rows, so the channels' conv weights are unpacked once for all of
+// them; all of its loads are issued before any arithmetic, and the index
+// arithmetic is 32-bit (the host checks the sizes).  u is rounded to fp16 with
+// the same operations, in the same order, as k_conv_silu16 (pairs of channels).
+// Threads past the conv range convert 8 W_x weights each to fp16.
+#ifndef JMIX_STEP_ROWS
+#define JMIX_STEP_ROWS 4
+#endif
+#ifndef JMIX_STEP_CVT
+#define JMIX_STEP_CVT 4  // 16-byte groups of W_x converted per thread
+#endif
+#ifndef JMIX_STEP_OCC
+#define JMIX_STEP_OCC 2
+#endif
+constexpr int kStepRows = JMIX_STEP_ROWS;
+constexpr int kStepCvt = JMIX_STEP_CVT;
+
+__global__ void __launch_bounds__(256, JMIX_STEP_OCC) k_conv_step(
+    const bf16* __restrict__ x, const bf16* __restrict__ conv_w, const bf16* __restrict__ conv_b,
+    const bf16* __restrict__ hist, const int* __restrict__ sidx, int n_slots, int B, int d,
+    __half* __restrict__ u, int n_conv, const bf16* __restrict__ wx, int n_wx8,
+    __half* __restrict__ wx16) {
+  const int tid = (int)(blockIdx.x * blockDim.x + threadIdx.x);
+  if (tid < n_conv) {
+    constexpr int kW = kConv - 1;
+    const int ncg = d >> 3;
+    const int rg = tid / ncg, cg = tid - rg * ncg;
+    const int c0 = cg * 8, b0 = rg * kStepRows;
+    uint4 xq[kStepRows], hq[kStepRows][kW];
+#pragma unroll
+    for (int r = 0; r < kStepRows; ++r) {
+      const int b = b0 + r;
+      xq[r] = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int q = 0; q < kW; ++q) hq[r][q] = make_uint4(0u, 0u, 0u, 0u);
+      if (b < B) {
+        xq[r] = __ldg(reinterpret_cast<const uint4*>(x + (int64_t)b * d + c0));
+        if (hist) {
+          int hb = b;
+          if (sidx) {
+            hb = __ldg(sidx + b);
+            hb = hb < 0 ? 0 : (hb >= n_slots ? n_slots - 1 : hb);
+          }
+          // the 8 channels' 3 taps each, oldest first: 48 contiguous bytes
+          const uint4* hp = reinterpret_cast<const uint4*>(hist + ((int64_t)hb * d + c0) * kW);
+#pragma unroll
+          for (int q = 0; q < kW; ++q) hq[r][q] = __ldg(hp + q);
+        }
+      }
+    }
+    uint4 wq[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) wq[q] = __ldg(reinterpret_cast<const uint4*>(conv_w + c0 * kConv) + q);
+    const uint4 bq = __ldg(reinterpret_cast<const uint4*>(conv_b + c0));
+    float2 w2[4][kConv], b2[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+#pragma unroll
+      for (int k = 0; k < kConv; ++k) {
+        const int e0 = (2 * q) * kConv + k, e1 = (2 * q + 1) * kConv + k;
+        w2[q][k] = make_float2(bf16_lane(wq[e0 >> 3], e0 & 7), bf16_lane(wq[e1 >> 3], e1 & 7));
+      }
+      b2[q] = make_float2(bf16_lane(bq, 2 * q), bf16_lane(bq, 2 * q + 1));
+    }
+#pragma unroll
+    for (int r = 0; r < kStepRows; ++r) {
+      uint32_t out[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        float2 acc = b2[q];
+#pragma unroll
+        for (int k = 0; k < kW; ++k) {
+          const int e0 = (2 * q) * kW + k, e1 = (2 * q + 1) * kW + k;
+          acc = __ffma2_rn(w2[q][k],
+                           make_float2(bf16_lane(hq[r][e0 >> 3], e0 & 7),
+                                       bf16_lane(hq[r][e1 >> 3], e1 & 7)),
+                           acc);
+        }
+        acc = __ffma2_rn(w2[q][kW], bf16_pair(xq[r], q), acc);
+        out[q] = silu_u_half2(acc);
+      }
+      const int b = b0 + r;
+      if (b < B)
+        *reinterpret_cast<uint4*>(u + (int64_t)b * d + c0) = make_uint4(out[0], out[1], out[2], out[3]);
+    }
+    return;
+  }
+  // kStepCvt groups of 8 weights per thread, every load before the stores
+  const int i0 = (tid - n_conv) * kStepCvt;
+  uint4 wv[kStepCvt];
+#pragma unroll
+  for (int j = 0; j < kStepCvt; ++j)
+    if (i0 + j < n_wx8) wv[j] = __ldg(reinterpret_cast<const uint4*>(wx) + i0 + j);
+#pragma unroll
+  for (int j = 0; j < kStepCvt; ++j) {
+    if (i0 + j >= n_wx8) break;
+    float o[8];
+    unpack8_bf16(wv[j], o);
+    reinterpret_cast<uint4*>(wx16)[i0 + j] =
+        make_uint4(pack_half2(o[0], o[1]), pack_half2(o[2], o[3]), pack_half2(o[4], o[5]),
+                   pack_half2(o[6], o[7]));
+  }
 }
 
 __global__ void __launch_bounds__(kFThreads, 1)
@@ -2650,7 +2785,17 @@ cudaError_t run_fast_fwd(Problem& p) {
       // (a decode step rounds W_dt to fp16 as it loads it into TMEM)
       const int64_t n_wdt8 = (p.prepared || p.decode) ? 0 : p.d * p.R / 8;
       const int64_t total = n_conv + n_wx8 + n_wdt8;
-      if (p.cu) {
+      const int64_t n_step = (p.d / 8) * ((p.B + kStepRows - 1) / kStepRows);
+      const int64_t n_cvt = (n_wx8 + kStepCvt - 1) / kStepCvt;
+      const bool step = p.decode && n_step + n_wx8 + 2048 < (int64_t)INT32_MAX &&
+                        p.B < (int64_t)INT32_MAX && p.n_slots < (int64_t)INT32_MAX &&
+                        p.d < (int64_t)INT32_MAX;
+      if (step) {
+        k_conv_step<<<(unsigned)((n_step + n_cvt + 255) / 256), 256, 0, s>>>(
+            (const bf16*)p.x, (const bf16*)p.conv_w, (const bf16*)p.conv_b,
+            (const bf16*)p.init_conv, p.sidx, (int)p.n_slots, (int)p.B, (int)p.d, w.u,
+            (int)n_step, (const bf16*)p.xproj_w, (int)n_wx8, w.wx);
+      } else if (p.cu) {
         const int64_t n_pk = (p.d / 8) * ((p.T + 7) / 8);
         k_conv_silu16_packed<<<(unsigned)((n_pk + n_wx8 + n_wdt8 + 255) / 256), 256, 0, s>>>(
             (const bf16*)p.x, (const bf16*)p.conv_w, (const bf16*)p.conv_b,
@@ -2663,7 +2808,7 @@ cudaError_t run_fast_fwd(Problem& p) {
             (const bf16*)p.init_conv, p.sidx, p.n_slots, p.B, p.L, p.d, w.u, n_conv,
             (const bf16*)p.xproj_w, n_wx8, w.wx, (const bf16*)p.dtproj_w, n_wdt8, w.wdt);
       }
-      launched(p, "k_conv_silu16");
+      launched(p, step ? "k_conv_step" : "k_conv_silu16");
     }
     // 2. x_proj on tcgen05
     {
