@@ -2066,8 +2066,9 @@ __global__ void __launch_bounds__(kLead ? 128 : kScanThreads, kScanCtasPerSm)
 
 // ------------------------------------------------------------- decode step
 // One token per row.  The work is B x (d / 128) pairs (row, 128-channel tile);
-// each of the persistent CTAs (two per SM) takes a contiguous, equal share of
-// them in tile-major order, so it changes channel tile at most a few times and
+// each of the persistent CTAs (two per SM) takes a contiguous share of them in
+// tile-major order (equal once each change of tile is counted as
+// kDecSwitchRows rows), so it changes channel tile at most a few times and
 // keeps that tile's W_dt in TMEM (the dt_proj MMA's A operand).
 //   warp 5: per group of kDB = 16 rows of a tile, TMA-loads the rows' dt_n
 //     (SW128, the MMA's B operand) and B/C rows into one of two buffers and
@@ -2083,6 +2084,10 @@ __global__ void __launch_bounds__(kLead ? 128 : kScanThreads, kScanCtasPerSm)
 // that bounds the step.  Rows whose state slot is outside the pool (indexed
 // step) are reported and skipped: nothing is loaded from or stored to a slot
 // outside the pool.
+#ifndef JMIX_DEC_SWITCH_ROWS
+#define JMIX_DEC_SWITCH_ROWS 12
+#endif
+constexpr int kDecSwitchRows = JMIX_DEC_SWITCH_ROWS;      // a W_dt reload, in rows of work
 constexpr int kDB = 16;                                   // rows per dt_proj MMA (N)
 constexpr int kDecThreads = 192;
 constexpr int kDecStages = 8;
@@ -2156,9 +2161,20 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wready + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // this CTA's pairs [p0, p1), tile-major: pair p = (tile p / B, row p % B)
-  const int64_t p0 = a.pairs * blockIdx.x / gridDim.x;
-  const int64_t p1 = a.pairs * (blockIdx.x + 1) / gridDim.x;
+  // this CTA's pairs [p0, p1), tile-major: pair p = (tile p / B, row p % B).
+  // A CTA whose range crosses into another tile reloads W_dt on the way (its
+  // first tile's load overlaps the wait for the norms), which costs about
+  // kDecSwitchRows rows of work: the ranges are equal shares of a virtual
+  // sequence in which each tile starts with that many units of no rows.
+  constexpr int64_t P = kDecSwitchRows;
+  const int64_t Bv = a.B + P;
+  const int64_t V = (int64_t)a.n_tiles * Bv;
+  auto pair_at = [&](int64_t v) {
+    const int64_t t = v / Bv, r = v - t * Bv - P;
+    return t * a.B + (r < 0 ? 0 : r);
+  };
+  const int64_t p0 = pair_at(V * blockIdx.x / gridDim.x);
+  const int64_t p1 = pair_at(V * (blockIdx.x + 1) / gridDim.x);
   const int64_t ngrp = (a.B + kDB - 1) / kDB;  // row groups per tile
   // groups this CTA touches: g = tile * ngrp + row / kDB
   auto grp_of = [&](int64_t p) { return (p / a.B) * ngrp + (p % a.B) / kDB; };
