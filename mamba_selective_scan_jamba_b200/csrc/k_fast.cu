@@ -671,9 +671,11 @@ constexpr int kFThreads = 64 + 32 * kFConvWarps;
 constexpr int kFStages = 3;
 constexpr int kFXRows = kXM + kConv - 1;                    // 131 x rows per chunk
 constexpr int kFXBytes = kFXRows * kXK * 2;                 // 16768 B
-constexpr int kFCwBytes = kXK * kConv * 2;                  // 512 B: the chunk's conv weights
-constexpr int kFCbBytes = kXK * 2;                          // 128 B: its conv biases
-constexpr int kFXStride = (kFXBytes + kFCwBytes + kFCbBytes + 1023) / 1024 * 1024;  // 17 KB
+// the chunk's conv weights and biases in float32, laid out for the conv threads
+// (see k_conv_table): 8 weight units and 2 bias units of 16 B per 8 channels
+constexpr int kFTabUnits = (kXK / 8) * 10;                  // 80
+constexpr int kFTabBytes = kFTabUnits * 16;                 // 1280 B
+constexpr int kFXStride = (kFXBytes + kFTabBytes + 1023) / 1024 * 1024;  // 18 KB
 constexpr int kFABytes = kXM * kXK * 2;                     // 16 KB u tile
 constexpr int kFMaxN1 = (kMaxRank + 2 * kN) / 2;            // 144
 constexpr int kFBMax = 2 * kFMaxN1 * kXK * 2;               // 36 KB of W_x rows
@@ -681,13 +683,60 @@ constexpr int kFSmem = 1024 + kFStages * (kFABytes + kFBMax + kFXStride) + 256;
 static_assert(kFSmem <= 227 * 1024, "fused x_proj stage ring exceeds shared memory");
 static_assert(kFConvWarps * 32 * kFG == kXM * (kXK / 8), "conv threads = kFG-token x 8-channel cells");
 
+// The weight preparation of a prefill: W_x and W_dt to fp16 (unless prepared
+// once beforehand), 8 weights per thread, and the conv weights and biases as
+// k_xproj_conv's float32 table: per 64-channel chunk kFTabUnits 16-byte units,
+// unit u * 8 + g (u < 8) = the taps 2 (u % 2), 2 (u % 2) + 1 of the channel pair
+// 2 (u / 2), 2 (u / 2) + 1 of the chunk's channel group g (8 channels), as
+// (w[c][k], w[c + 1][k], w[c][k + 1], w[c + 1][k + 1]); unit 64 + v * 8 + g =
+// the biases of channels 4 v .. 4 v + 3 of group g.  Zeros past d.
+__global__ void __launch_bounds__(256) k_convert_weights(
+    const bf16* __restrict__ wx, int64_t n_wx8, __half* __restrict__ wx16,
+    const bf16* __restrict__ wdt, int64_t n_wdt8, __half* __restrict__ wdt16,
+    const bf16* __restrict__ conv_w, const bf16* __restrict__ conv_b, int64_t d,
+    float4* __restrict__ ctab, int64_t n_tab) {
+  int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const bf16* src = nullptr;
+  __half* dst = nullptr;
+  if (i < n_wx8) {
+    src = wx;
+    dst = wx16;
+  } else if ((i -= n_wx8) < n_wdt8) {
+    src = wdt;
+    dst = wdt16;
+  } else if ((i -= n_wdt8) < n_tab) {
+    const int64_t kc = i / kFTabUnits;
+    const int r = (int)(i - kc * kFTabUnits);
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (r < 64) {
+      const int u = r >> 3, g = r & 7, k = 2 * (u & 1);
+      const int64_t c = kc * kXK + g * 8 + 2 * (u >> 1);
+      if (c < d)  // d is a multiple of 8: both channels of the pair exist, or neither
+        v = make_float4(bf(conv_w[c * kConv + k]), bf(conv_w[(c + 1) * kConv + k]),
+                        bf(conv_w[c * kConv + k + 1]), bf(conv_w[(c + 1) * kConv + k + 1]));
+    } else {
+      const int hv = (r - 64) >> 3, g = (r - 64) & 7;
+      const int64_t c = kc * kXK + g * 8 + 4 * hv;
+      if (c < d)
+        v = make_float4(bf(conv_b[c]), bf(conv_b[c + 1]), bf(conv_b[c + 2]), bf(conv_b[c + 3]));
+    }
+    ctab[i] = v;
+    return;
+  } else {
+    return;
+  }
+  float o[8];
+  unpack8_bf16(__ldg(reinterpret_cast<const uint4*>(src) + i), o);
+  reinterpret_cast<uint4*>(dst)[i] = make_uint4(pack_half2(o[0], o[1]), pack_half2(o[2], o[3]),
+                                                pack_half2(o[4], o[5]), pack_half2(o[6], o[7]));
+}
+
 struct XconvArgs {
   int64_t T, L, d;
   int P, N1, R;
   int kchunks, ksplit;
   uint32_t tmem_cols;
-  const bf16* conv_w;  // [d, 4]
-  const bf16* conv_b;  // [d]
+  const float4* ctab;  // [kchunks * kFTabUnits] the conv weights and biases (k_conv_table)
   const bf16* hist;    // [B, d, 3] conv history of each sequence, or null (zeros)
   const int* cu;       // packed batch: [B + 1] token offsets of the sequences, or null
   int64_t nseq;        // packed batch: sequences B
@@ -904,14 +953,11 @@ __global__ void __launch_bounds__(kFThreads, 1)
             !mbar_wait(smem_u32(&mdone[s]), (uint32_t)((i / kFStages) - 1) & 1u, a.err, 85))
           break;
         const uint32_t fb = smem_u32(&full[s]);
-        // conv weights and biases of the chunk's channels that exist (a multiple of 8)
-        const int64_t c0 = (int64_t)kc * kXK;
-        const uint32_t nch = (uint32_t)((a.d - c0) < kXK ? (a.d - c0) : kXK);
-        mbar_arrive_expect_tx(fb, (uint32_t)kFXBytes + nch * (kConv * 2 + 2) + 2 * half_b);
+        mbar_arrive_expect_tx(fb, (uint32_t)(kFXBytes + kFTabBytes) + 2 * half_b);
         uint8_t* xst = Xs + s * kFXStride;
         tma_load_2d(smem_u32(xst), &tm_x, fb, kc * kXK, (int32_t)(m0 - (kConv - 1)));
-        bulk_load(smem_u32(xst + kFXBytes), a.conv_w + c0 * kConv, nch * kConv * 2, fb);
-        bulk_load(smem_u32(xst + kFXBytes + kFCwBytes), a.conv_b + c0, nch * 2, fb);
+        // the chunk's conv weights and biases (zeros for channels past d)
+        bulk_load(smem_u32(xst + kFXBytes), a.ctab + (int64_t)kc * kFTabUnits, kFTabBytes, fb);
         const uint32_t bs = smem_u32(Bs + s * kFBMax);
         tma_load_2d(bs, &tm_w, fb, kc * kXK, 0);
         tma_load_2d(bs + half_b, &tm_w, fb, kc * kXK, a.N1);
@@ -996,29 +1042,31 @@ __global__ void __launch_bounds__(kFThreads, 1)
       const int64_t c0 = (int64_t)kc * kXK + cg * 8;
       const bool cin = c0 < a.d;  // d is a multiple of 8: all 8 channels exist, or none
       if (!mbar_wait(smem_u32(&full[s]), ph, a.err, 88)) break;
-      // this thread's 8 channels' conv weights (64 B) and biases (16 B) from the
-      // stage (stale past d: those outputs are zeroed below)
+      // this thread's 8 channels' conv weights and biases in float32, as pairs
+      // of channels: unit u * 8 + cg of the stage's table, so that the 8 threads
+      // of a quarter warp read 128 consecutive bytes
       const uint8_t* xst = Xs + s * kFXStride;
-      uint4 wq[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        wq[q] = *reinterpret_cast<const uint4*>(xst + kFXBytes + cg * 64 + 16 * q);
-      const uint4 bq = *reinterpret_cast<const uint4*>(xst + kFXBytes + kFCwBytes + cg * 16);
-      const uint8_t* xs = xst + (kFG * tg) * (kXK * 2) + cg * 16;
-      uint4 xr[kFG + kW];
-#pragma unroll
-      for (int j = 0; j < kFG + kW; ++j) xr[j] = *reinterpret_cast<const uint4*>(xs + j * (kXK * 2));
-      // weights and bias of the 4 channel pairs
+      const float4* tab = reinterpret_cast<const float4*>(xst + kFXBytes);
       float2 w2[4][kConv], b2[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
 #pragma unroll
-        for (int k = 0; k < kConv; ++k) {
-          const int e0 = (2 * q) * kConv + k, e1 = (2 * q + 1) * kConv + k;
-          w2[q][k] = make_float2(bf16_lane(wq[e0 >> 3], e0 & 7), bf16_lane(wq[e1 >> 3], e1 & 7));
+        for (int kh = 0; kh < kConv / 2; ++kh) {
+          const float4 v = tab[(q * 2 + kh) * 8 + cg];
+          w2[q][2 * kh] = make_float2(v.x, v.y);
+          w2[q][2 * kh + 1] = make_float2(v.z, v.w);
         }
-        b2[q] = make_float2(bf16_lane(bq, 2 * q), bf16_lane(bq, 2 * q + 1));
       }
+#pragma unroll
+      for (int hv = 0; hv < 2; ++hv) {
+        const float4 v = tab[64 + hv * 8 + cg];
+        b2[2 * hv] = make_float2(v.x, v.y);
+        b2[2 * hv + 1] = make_float2(v.z, v.w);
+      }
+      const uint8_t* xs = xst + (kFG * tg) * (kXK * 2) + cg * 16;
+      uint4 xr[kFG + kW];
+#pragma unroll
+      for (int j = 0; j < kFG + kW; ++j) xr[j] = *reinterpret_cast<const uint4*>(xs + j * (kXK * 2));
       uint32_t outw[kFG][4];  // [token][channel pair] fp16x2
       if (!step) {
         if (sub) {
@@ -2594,6 +2642,7 @@ struct FastWs {
   float* bc;
   __half* wx;
   __half* wdt;
+  float4* ctab;       // k_xproj_conv: the conv weights and biases as its float32 table
   int* sched;         // [0] unit counter, [1..] hand-over flags of the scan's parts
   float* carry_h;     // scan hand-over: end state per (pair, part)
   float* carry_s;     // scan hand-over: sum of delta per (pair, part)
@@ -2675,6 +2724,7 @@ FastWs fast_layout(const Problem& pr, char* base) {
   w.bc = reinterpret_cast<float*>(take(T * 2 * kN * 4));
   w.wx = reinterpret_cast<__half*>(take(P * d * 2));
   w.wdt = reinterpret_cast<__half*>(take(d * R * 2));
+  w.ctab = reinterpret_cast<float4*>(take(xconv ? (d + kXK - 1) / kXK * kFTabBytes : 0));
   w.bytes = off;
   if (pr.prepared) {  // fp16 copies made once by jm_prepare_weights: W_x, then W_dt
     char* pw = static_cast<char*>(const_cast<void*>(pr.prepared));
@@ -2729,15 +2779,16 @@ cudaError_t run_fast_fwd(Problem& p) {
   launches_begin(p);
 
   if (use_xconv(p)) {
-    // 1-3. W_x, W_dt -> fp16 (unless prepared once beforehand); conv + SiLU
-    // inside x_proj; the norms in its epilogue (one split) or after it
-    const bool convert = !p.prepared;
-    if (convert) {
-      const int64_t n_wx8 = (int64_t)p.P * p.d / 8, n_wdt8 = p.d * p.R / 8;
-      k_conv_silu16<1><<<(unsigned)((n_wx8 + n_wdt8 + 255) / 256), 256, 0, s>>>(
-          (const bf16*)p.x, (const bf16*)p.conv_w, (const bf16*)p.conv_b, nullptr, nullptr, 0,
-          p.B, p.L, p.d, nullptr, 0, (const bf16*)p.xproj_w, n_wx8, w.wx,
-          (const bf16*)p.dtproj_w, n_wdt8, w.wdt);
+    // 1-3. W_x, W_dt -> fp16 (unless prepared once beforehand) and the conv
+    // weight table; conv + SiLU inside x_proj; the norms in its epilogue (one
+    // split) or after it
+    {
+      const int64_t n_wx8 = p.prepared ? 0 : (int64_t)p.P * p.d / 8;
+      const int64_t n_wdt8 = p.prepared ? 0 : p.d * p.R / 8;
+      const int64_t n_tab = (p.d + kXK - 1) / kXK * kFTabUnits;
+      k_convert_weights<<<(unsigned)((n_wx8 + n_wdt8 + n_tab + 255) / 256), 256, 0, s>>>(
+          (const bf16*)p.xproj_w, n_wx8, w.wx, (const bf16*)p.dtproj_w, n_wdt8, w.wdt,
+          (const bf16*)p.conv_w, (const bf16*)p.conv_b, p.d, w.ctab, n_tab);
       launched(p, "k_convert_weights");
     }
     CUtensorMap tx, tw;
@@ -2751,8 +2802,7 @@ cudaError_t run_fast_fwd(Problem& p) {
     xa.kchunks = (int)((p.d + kXK - 1) / kXK);
     xa.ksplit = w.ksplit;
     xa.tmem_cols = 2 * xa.N1 <= 64 ? 64 : 2 * xa.N1 <= 128 ? 128 : 2 * xa.N1 <= 256 ? 256 : 512;
-    xa.conv_w = (const bf16*)p.conv_w;
-    xa.conv_b = (const bf16*)p.conv_b;
+    xa.ctab = w.ctab;
     xa.hist = (const bf16*)p.init_conv;
     xa.cu = p.cu;
     xa.nseq = p.B;
@@ -2772,12 +2822,7 @@ cudaError_t run_fast_fwd(Problem& p) {
       return cudaErrorInvalidValue;
     cudaFuncSetAttribute(k_xproj_conv, cudaFuncAttributeMaxDynamicSharedMemorySize, kFSmem);
     const dim3 grid((unsigned)((p.T + kXM - 1) / kXM), (unsigned)xa.ksplit);
-    if (convert)
-      e = launch_pdl(k_xproj_conv, grid, kFThreads, (size_t)kFSmem, s, tx, tw, xa);
-    else {
-      k_xproj_conv<<<grid, kFThreads, kFSmem, s>>>(tx, tw, xa);
-      e = cudaGetLastError();
-    }
+    e = launch_pdl(k_xproj_conv, grid, kFThreads, (size_t)kFSmem, s, tx, tw, xa);
     if (e != cudaSuccess) return e;
     launched(p, "k_xproj_conv");
     if (w.ksplit > 1) {
