@@ -2190,7 +2190,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     k_decode_scan(const __grid_constant__ CUtensorMap tm_state,
                   const __grid_constant__ CUtensorMap tm_state_wb,
                   const __grid_constant__ CUtensorMap tm_dtn,
-                  const __grid_constant__ CUtensorMap tm_bc, const DecArgs a) {
+                  const __grid_constant__ CUtensorMap tm_bc,
+                  const __grid_constant__ CUtensorMap tm_wdt, const DecArgs a) {
   extern __shared__ uint8_t smem_raw[];
   // (offset arithmetic on the shared array keeps its address space known, so
   // accesses through these pointers compile to shared-memory loads)
@@ -2206,7 +2207,9 @@ __global__ void __launch_bounds__(kDecThreads, 2)
   uint64_t* mma_done = gfull + 2;                          // [2] accumulator ready
   uint64_t* acc_free = mma_done + 2;                       // [2] group done (4 warps)
   uint64_t* wready = acc_free + 2;                         // W_dt of a new tile in TMEM
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wready + 1);
+  uint64_t* wfull = wready + 1;                            // the first tile's W_dt in the ring
+  uint64_t* wcopied = wready + 2;                          // ... and out of it (4 warps)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(wready + 3);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // this CTA's pairs [p0, p1), tile-major: pair p = (tile p / B, row p % B).
@@ -2240,6 +2243,8 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       mbar_init(smem_u32(&acc_free[b]), 4);
     }
     mbar_init(smem_u32(wready), 4);
+    mbar_init(smem_u32(wfull), 1);
+    mbar_init(smem_u32(wcopied), 4);
     fence_mbar_init();
   }
   if (warp == 5) {
@@ -2257,9 +2262,23 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     if (lane == 0) {
       prefetch_tmap(&tm_state);
       const uint64_t evict_first = l2_evict_first_policy();
+      int64_t pend_s = p1;  // the rows this streamer loads: [p0, pend_s)
+      if (p0 < p1) {
+        // the first tile's W_dt rows come through the ring (one 16 KB box per 64
+        // K values, 128-byte swizzle: the compute threads' row reads are free of
+        // bank conflicts); the state rows follow once the compute warps have
+        // moved them into TMEM
+        prefetch_tmap(&tm_wdt);
+        const uint32_t wf = smem_u32(wfull);
+        mbar_arrive_expect_tx(wf, (uint32_t)(a.nslab * kSC * 128));
+        for (int j = 0; j < a.nslab; ++j)
+          tma_load_2d(smem_u32(stages + j * kSC * 128), &tm_wdt, wf, j * 64,
+                      (int32_t)((p0 / a.B) * kSC));
+        if (!mbar_wait(smem_u32(wcopied), 0u, a.err, 47)) pend_s = p0;  // (reported; no rows)
+      }
       // (tile, row) of pair p, advanced by one row per pair (no divisions in the loop)
       int64_t tile = p0 / a.B, b = p0 - tile * a.B;
-      for (int64_t p = p0, i = 0; p < p1; ++p, ++i, ++b) {
+      for (int64_t p = p0, i = 0; p < pend_s; ++p, ++i, ++b) {
         if (b == a.B) {
           b = 0;
           ++tile;
@@ -2338,7 +2357,63 @@ __global__ void __launch_bounds__(kDecThreads, 2)
     int64_t c = 0;
     float2 A2[kN / 2];
     float bias = 0.f, Dc = 0.f, cb = 0.f, cw[kConv] = {0.f, 0.f, 0.f, 0.f};
-    // a new channel tile: its W_dt rows into TMEM (zeros past R and past d),
+    // 8 W_dt values (bf16, or the prepared fp16) as fp16 pairs
+    auto to_half8 = [&](const uint4& w, uint32_t* v) {
+      if (a.wdt_bf16) {  // rounded as the weight conversion rounds
+        float o[8];
+        unpack8_bf16(w, o);
+        v[0] = pack_half2(o[0], o[1]);
+        v[1] = pack_half2(o[2], o[3]);
+        v[2] = pack_half2(o[4], o[5]);
+        v[3] = pack_half2(o[6], o[7]);
+      } else {
+        v[0] = w.x;
+        v[1] = w.y;
+        v[2] = w.z;
+        v[3] = w.w;
+      }
+    };
+    // the per-channel parameters of the current tile
+    auto load_params = [&]() {
+#pragma unroll
+      for (int q = 0; q < kN / 2; ++q) {
+        A2[q].x = cok ? -expf(a.A_log[c * kN + 2 * q]) * kLog2e : 0.0f;
+        A2[q].y = cok ? -expf(a.A_log[c * kN + 2 * q + 1]) * kLog2e : 0.0f;
+      }
+      bias = cok ? a.dt_bias[c] : 0.f;
+      Dc = cok ? a.D[c] : 0.f;
+#pragma unroll
+      for (int kx = 0; kx < kConv; ++kx) cw[kx] = cok ? bf(a.conv_w[c * kConv + kx]) : 0.f;
+      cb = cok ? bf(a.conv_b[c]) : 0.f;
+    };
+    // the CTA's first tile: its W_dt rows from the ring, where the streamer put
+    // them by TMA (zeros past R and past d), into TMEM
+    auto load_first_tile = [&](int64_t tile) {
+      cur_tile = tile;
+      c = tile * kSC + cl;
+      cok = c < a.d;
+      const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+      mbar_wait(smem_u32(wfull), 0u, a.err, 48);
+      for (int qs = 0; qs < a.nslab * 2; ++qs) {  // 16 columns = 32 K values of box qs / 2
+        const uint8_t* rowp = stages + (qs >> 1) * (kSC * 128) + cl * 128;
+        uint32_t v[16];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int q = (qs & 1) * 4 + e;  // 16-byte chunk of the row, stored at q ^ (row % 8)
+          to_half8(*reinterpret_cast<const uint4*>(rowp + ((q ^ (cl & 7)) << 4)), v + 4 * e);
+        }
+        tmem_st16(trow + (uint32_t)(qs * 16), v);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(smem_u32(wready));
+        mbar_arrive(smem_u32(wcopied));
+      }
+      load_params();
+    };
+    // a later channel tile: its W_dt rows into TMEM (zeros past R and past d),
     // 16 loads in flight per thread at a time, then the per-channel parameters
     auto load_tile = [&](int64_t tile) {
       cur_tile = tile;
@@ -2362,21 +2437,7 @@ __global__ void __launch_bounds__(kDecThreads, 2)
           if (q0 + qq >= nq) break;
           uint32_t v[16];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            if (a.wdt_bf16) {  // 8 bf16 -> 8 fp16, rounded as the weight conversion rounds
-              float o[8];
-              unpack8_bf16(w8[qq][e], o);
-              v[4 * e] = pack_half2(o[0], o[1]);
-              v[4 * e + 1] = pack_half2(o[2], o[3]);
-              v[4 * e + 2] = pack_half2(o[4], o[5]);
-              v[4 * e + 3] = pack_half2(o[6], o[7]);
-            } else {
-              v[4 * e] = w8[qq][e].x;
-              v[4 * e + 1] = w8[qq][e].y;
-              v[4 * e + 2] = w8[qq][e].z;
-              v[4 * e + 3] = w8[qq][e].w;
-            }
-          }
+          for (int e = 0; e < 4; ++e) to_half8(w8[qq][e], v + 4 * e);
           tmem_st16(trow + (uint32_t)((q0 + qq) * 16), v);
         }
       }
@@ -2384,20 +2445,11 @@ __global__ void __launch_bounds__(kDecThreads, 2)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(wready));
-#pragma unroll
-      for (int q = 0; q < kN / 2; ++q) {
-        A2[q].x = cok ? -expf(a.A_log[c * kN + 2 * q]) * kLog2e : 0.0f;
-        A2[q].y = cok ? -expf(a.A_log[c * kN + 2 * q + 1]) * kLog2e : 0.0f;
-      }
-      bias = cok ? a.dt_bias[c] : 0.f;
-      Dc = cok ? a.D[c] : 0.f;
-#pragma unroll
-      for (int kx = 0; kx < kConv; ++kx) cw[kx] = cok ? bf(a.conv_w[c * kConv + kx]) : 0.f;
-      cb = cok ? bf(a.conv_b[c]) : 0.f;
+      load_params();
     };
     // The first tile's W_dt (an input, or its copy prepared before the call) is
     // read before griddepcontrol.wait.
-    if (g0 < g1) load_tile(g0 / ngrp);
+    if (g0 < g1) load_first_tile(g0 / ngrp);
     grid_dep_wait();  // dt_n and B/C come from the norms kernel
     // A row's new SSM and conv state go to global memory through the warp's
     // scratch rows (64-byte swizzled like the stage): one tensor store and one
@@ -2911,7 +2963,7 @@ cudaError_t run_fast_fwd(Problem& p) {
   }
   // 4. dt_proj + scan + gate
   if (p.decode) {
-    CUtensorMap tstate, tstate_wb, tdtn, tbc;
+    CUtensorMap tstate, tstate_wb, tdtn, tbc, twdt;
     const int64_t slots = p.sidx ? p.n_slots : p.B;
     if (!make_state_map(&tstate, p.final_state, (uint64_t)slots, (uint64_t)p.d) ||
         !make_state_map(&tstate_wb, p.final_state, (uint64_t)slots, (uint64_t)p.d, 32) ||
@@ -2937,6 +2989,11 @@ cudaError_t run_fast_fwd(Problem& p) {
     da.wdt = p.prepared ? reinterpret_cast<const uint16_t*>(w.wdt)
                         : reinterpret_cast<const uint16_t*>(p.dtproj_w);
     da.wdt_bf16 = p.prepared ? 0 : 1;
+    // W_dt [d, R] in boxes of 64 K values x 128 channels (a CTA's first tile)
+    if (!make_map(&twdt,
+                  p.prepared ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  da.wdt, p.d, p.R, 64, kSC, true))
+      return cudaErrorInvalidValue;
     da.conv_state = (bf16*)p.final_conv;
     da.ssm_state = p.final_state;
     da.y = (bf16*)p.y;
@@ -2947,7 +3004,7 @@ cudaError_t run_fast_fwd(Problem& p) {
     cudaFuncSetAttribute(dec_kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kDecSmem);
     const int64_t ctas = std::min<int64_t>(2 * num_sms(), da.pairs);
     e = launch_pdl(dec_kern, (unsigned)ctas, kDecThreads, kDecSmem, s, tstate, tstate_wb, tdtn,
-                   tbc, da);
+                   tbc, twdt, da);
     if (e != cudaSuccess) return e;
     launched(p, "k_decode_scan");
   } else {
