@@ -372,6 +372,7 @@ struct XprojArgs {
 };
 
 constexpr int kXThreads = 192;  // warp 0 TMA, warp 1 MMA + TMEM, warps 2..5 epilogue
+constexpr int kXMaxBoxes = 9;   // the epilogue's [32 x 16] fp32 boxes per warp (N1 <= 144)
 
 __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
   return (1u << 4)                                  // D format: f32
@@ -386,7 +387,7 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
 // CTAs of a token tile run together and the second read of its u tile hits L2.
 __global__ void __launch_bounds__(kXThreads, 2)
     k_xproj(const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_w,
-            const XprojArgs a) {
+            const __grid_constant__ CUtensorMap tm_part, const XprojArgs a) {
   extern __shared__ uint8_t smem_raw[];
   // (offset arithmetic on the shared array keeps its address space known, so
   // accesses through these pointers compile to shared-memory loads)
@@ -465,34 +466,38 @@ __global__ void __launch_bounds__(kXThreads, 2)
     }
   } else {
     // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 = tile rows, 16
-    // columns at a time, transposes them through shared memory (the stage
-    // buffers are free once the accumulator is complete) and stores two
-    // 64-byte row segments per instruction
+    // columns at a time, into [32 rows x 16 columns] boxes of shared memory
+    // (64-byte swizzle: 16-byte chunk q of row r at chunk q ^ ((r >> 1) & 3),
+    // free of bank conflicts; the stage buffers are free once the accumulator is
+    // complete), which one tensor store per box writes to the split's partial
+    // tile (rows past T and columns past P are not written)
     const bool ok = mbar_wait(smem_u32(acc_full), 0, a.err, 13);
     tc_fence_after();
     const int lg = warp & 3;
-    float* tbuf = reinterpret_cast<float*>(smem) + (warp - 2) * (32 * 17);
-    const int64_t row0 = (int64_t)m_tile * kXM + lg * 32;
-    float* dst = a.part + ((int64_t)split * a.T) * a.P;
     const bool any = ok && k_end > k_begin;
-    for (int c0 = 0; c0 < a.N1; c0 += 16) {
+    uint8_t* boxes = smem + lg * (kXMaxBoxes * 2048);
+    const int nbox = a.N1 / 16;
+    for (int j = 0; j < nbox; ++j) {
       uint32_t r[16];
-      tmem_ld16(tmem + ((uint32_t)(lg * 32) << 16) + (uint32_t)c0, r);
+      tmem_ld16(tmem + ((uint32_t)(lg * 32) << 16) + (uint32_t)(j * 16), r);
       tmem_ld_wait();
+      uint8_t* row = boxes + j * 2048 + lane * 64;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) tbuf[lane * 17 + j] = __uint_as_float(r[j]);
-      __syncwarp();
-      if (any) {
-        const int col = col0 + c0 + (lane & 15);
-#pragma unroll 4
-        for (int rr = 0; rr < 16; ++rr) {
-          const int row = 2 * rr + (lane >> 4);
-          const int64_t g = row0 + row;
-          if (g < a.T && col < a.P) dst[g * a.P + col] = tbuf[row * 17 + (lane & 15)];
-        }
-      }
-      __syncwarp();
+      for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4*>(row + ((q ^ ((lane >> 1) & 3)) << 4)) =
+            any ? make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3])
+                : make_uint4(0u, 0u, 0u, 0u);
     }
+    fence_proxy_async_smem();  // the boxes, before the tensor stores read them
+    __syncwarp();
+    if (lane == 0) {
+      for (int j = 0; j < nbox; ++j)
+        tma_store_3d(&tm_part, smem_u32(boxes + j * 2048), col0 + j * 16,
+                     m_tile * kXM + lg * 32, split);
+      bulk_commit();
+      bulk_wait_all();  // the partial tile written (and the boxes read) before the CTA ends
+    }
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
@@ -2665,6 +2670,20 @@ bool make_state_map(CUtensorMap* m, const float* base, uint64_t slots, uint64_t 
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D tensor map of x_proj's partial sums [S, T, P] fp32 with box [1, 32 rows,
+// 16 columns] and the 64-byte swizzle: a box store never reaches past T or P.
+bool make_part_map(CUtensorMap* m, const float* base, uint64_t S, uint64_t T, uint64_t P) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {P, T, S};
+  cuuint64_t strides[2] = {P * 4, T * P * 4};
+  cuuint32_t box[3] = {16, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 3-D tensor map of y [B, L, d] bf16 with box [1, 32 tokens, 128 channels]: a
 // tile store never reaches past its sequence's tokens or past d.
 bool make_y_map(CUtensorMap* m, const void* y, uint64_t B, uint64_t L, uint64_t d) {
@@ -2942,10 +2961,13 @@ cudaError_t run_fast_fwd(Problem& p) {
       if (!make_map(&tu, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w.u, p.T, p.d, kXK, kXM, true) ||
           !make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w.wx, p.P, p.d, kXK, xa.N1, true))
         return cudaErrorInvalidValue;
+      CUtensorMap tp;  // the partial sums [ksplit, T, P], boxes of 16 columns x 32 rows
+      if (!make_part_map(&tp, w.part, (uint64_t)xa.ksplit, (uint64_t)p.T, (uint64_t)p.P))
+        return cudaErrorInvalidValue;
       const int smem = 1024 + kXStages * (kXM * 128 + xa.N1 * 128) + 256;
       cudaFuncSetAttribute(k_xproj, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
       e = launch_pdl(k_xproj, dim3((unsigned)(2 * mtiles), (unsigned)xa.ksplit), kXThreads,
-                     (size_t)smem, s, tu, tw, xa);
+                     (size_t)smem, s, tu, tw, tp, xa);
       if (e != cudaSuccess) return e;
       launched(p, "k_xproj");
     }
