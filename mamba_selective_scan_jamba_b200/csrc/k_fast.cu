@@ -821,7 +821,13 @@ __global__ void __launch_bounds__(256, JMIX_STEP_OCC) k_conv_step(
     const bf16* __restrict__ x, const bf16* __restrict__ conv_w, const bf16* __restrict__ conv_b,
     const bf16* __restrict__ hist, const int* __restrict__ sidx, int n_slots, int B, int d,
     __half* __restrict__ u, int n_conv, const bf16* __restrict__ wx, int n_wx8,
-    __half* __restrict__ wx16) {
+    __half* __restrict__ wx16, unsigned* __restrict__ zero_w, int n_zero_w) {
+  // x_t and the conv states may come from the kernels before this one; the
+  // step's error header is cleared here (the later kernels of the step start
+  // after this one has completed)
+  grid_dep_wait();
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < n_zero_w; i += blockDim.x) zero_w[i] = 0u;
   const int tid = (int)(blockIdx.x * blockDim.x + threadIdx.x);
   if (tid < n_conv) {
     constexpr int kW = kConv - 1;
@@ -2841,12 +2847,28 @@ int num_sms() {
   return n;
 }
 
+// Whether a decode step's conv runs as k_conv_step (32-bit index arithmetic).
+bool conv_step_fits(const Problem& p) {
+  if (!p.decode) return false;
+  const int64_t n_step = (p.d / 8) * ((p.B + kStepRows - 1) / kStepRows);
+  const int64_t n_wx8 = p.prepared ? 0 : (int64_t)p.P * p.d / 8;
+  return n_step + n_wx8 + 2048 < (int64_t)INT32_MAX && p.B < (int64_t)INT32_MAX &&
+         p.n_slots < (int64_t)INT32_MAX && p.d < (int64_t)INT32_MAX;
+}
+
 cudaError_t run_fast_fwd(Problem& p) {
   FastWs w = fast_layout(p, p.ws);
   cudaStream_t s = p.stream;
   ErrFlags* err = reinterpret_cast<ErrFlags*>(w.hdr);
-  cudaError_t e = cudaMemsetAsync(p.ws, 0, w.zero_bytes, s);
-  if (e != cudaSuccess) return e;
+  // a decode step's conv kernel clears the error header and scheduler words
+  // itself (so it can follow the kernel before it with programmatic dependent
+  // launch); every other call clears them with a memset first
+  const bool step_conv = !use_xconv(p) && conv_step_fits(p);
+  cudaError_t e = cudaSuccess;
+  if (!step_conv) {
+    e = cudaMemsetAsync(p.ws, 0, w.zero_bytes, s);
+    if (e != cudaSuccess) return e;
+  }
   launches_begin(p);
 
   if (use_xconv(p)) {
@@ -2919,14 +2941,14 @@ cudaError_t run_fast_fwd(Problem& p) {
       const int64_t total = n_conv + n_wx8 + n_wdt8;
       const int64_t n_step = (p.d / 8) * ((p.B + kStepRows - 1) / kStepRows);
       const int64_t n_cvt = (n_wx8 + kStepCvt - 1) / kStepCvt;
-      const bool step = p.decode && n_step + n_wx8 + 2048 < (int64_t)INT32_MAX &&
-                        p.B < (int64_t)INT32_MAX && p.n_slots < (int64_t)INT32_MAX &&
-                        p.d < (int64_t)INT32_MAX;
+      const bool step = step_conv;
       if (step) {
-        k_conv_step<<<(unsigned)((n_step + n_cvt + 255) / 256), 256, 0, s>>>(
-            (const bf16*)p.x, (const bf16*)p.conv_w, (const bf16*)p.conv_b,
-            (const bf16*)p.init_conv, p.sidx, (int)p.n_slots, (int)p.B, (int)p.d, w.u,
-            (int)n_step, (const bf16*)p.xproj_w, (int)n_wx8, w.wx);
+        e = launch_pdl(k_conv_step, dim3((unsigned)((n_step + n_cvt + 255) / 256)), 256, 0, s,
+                       (const bf16*)p.x, (const bf16*)p.conv_w, (const bf16*)p.conv_b,
+                       (const bf16*)p.init_conv, p.sidx, (int)p.n_slots, (int)p.B, (int)p.d, w.u,
+                       (int)n_step, (const bf16*)p.xproj_w, (int)n_wx8, w.wx,
+                       reinterpret_cast<unsigned*>(p.ws), (int)(w.zero_bytes / 4));
+        if (e != cudaSuccess) return e;
       } else if (p.cu) {
         const int64_t n_pk = (p.d / 8) * ((p.T + 7) / 8);
         k_conv_silu16_packed<<<(unsigned)((n_pk + n_wx8 + n_wdt8 + 255) / 256), 256, 0, s>>>(
