@@ -699,7 +699,13 @@ __global__ void __launch_bounds__(256) k_convert_weights(
     const bf16* __restrict__ wx, int64_t n_wx8, __half* __restrict__ wx16,
     const bf16* __restrict__ wdt, int64_t n_wdt8, __half* __restrict__ wdt16,
     const bf16* __restrict__ conv_w, const bf16* __restrict__ conv_b, int64_t d,
-    float4* __restrict__ ctab, int64_t n_tab) {
+    float4* __restrict__ ctab, int64_t n_tab, unsigned* __restrict__ zero_w, int n_zero_w) {
+  // the kernels before this one may still read the workspace; the call's error
+  // header and scheduler words are cleared here (the later kernels of the call
+  // start after this one has completed)
+  grid_dep_wait();
+  if (blockIdx.x == 0)
+    for (int z = threadIdx.x; z < n_zero_w; z += blockDim.x) zero_w[z] = 0u;
   int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const bf16* src = nullptr;
   __half* dst = nullptr;
@@ -2860,18 +2866,20 @@ cudaError_t run_fast_fwd(Problem& p) {
   FastWs w = fast_layout(p, p.ws);
   cudaStream_t s = p.stream;
   ErrFlags* err = reinterpret_cast<ErrFlags*>(w.hdr);
-  // a decode step's conv kernel clears the error header and scheduler words
-  // itself (so it can follow the kernel before it with programmatic dependent
-  // launch); every other call clears them with a memset first
-  const bool step_conv = !use_xconv(p) && conv_step_fits(p);
+  // a prefill's weight preparation and a decode step's conv kernel clear the
+  // error header and scheduler words themselves (so they can follow the kernel
+  // before them with programmatic dependent launch); other calls clear them
+  // with a memset first
+  const bool xconv = use_xconv(p);
+  const bool step_conv = !xconv && conv_step_fits(p);
   cudaError_t e = cudaSuccess;
-  if (!step_conv) {
+  if (!xconv && !step_conv) {
     e = cudaMemsetAsync(p.ws, 0, w.zero_bytes, s);
     if (e != cudaSuccess) return e;
   }
   launches_begin(p);
 
-  if (use_xconv(p)) {
+  if (xconv) {
     // 1-3. W_x, W_dt -> fp16 (unless prepared once beforehand) and the conv
     // weight table; conv + SiLU inside x_proj; the norms in its epilogue (one
     // split) or after it
@@ -2879,9 +2887,11 @@ cudaError_t run_fast_fwd(Problem& p) {
       const int64_t n_wx8 = p.prepared ? 0 : (int64_t)p.P * p.d / 8;
       const int64_t n_wdt8 = p.prepared ? 0 : p.d * p.R / 8;
       const int64_t n_tab = (p.d + kXK - 1) / kXK * kFTabUnits;
-      k_convert_weights<<<(unsigned)((n_wx8 + n_wdt8 + n_tab + 255) / 256), 256, 0, s>>>(
-          (const bf16*)p.xproj_w, n_wx8, w.wx, (const bf16*)p.dtproj_w, n_wdt8, w.wdt,
-          (const bf16*)p.conv_w, (const bf16*)p.conv_b, p.d, w.ctab, n_tab);
+      e = launch_pdl(k_convert_weights, dim3((unsigned)((n_wx8 + n_wdt8 + n_tab + 255) / 256)),
+                     256, 0, s, (const bf16*)p.xproj_w, n_wx8, w.wx, (const bf16*)p.dtproj_w,
+                     n_wdt8, w.wdt, (const bf16*)p.conv_w, (const bf16*)p.conv_b, p.d, w.ctab,
+                     n_tab, reinterpret_cast<unsigned*>(p.ws), (int)(w.zero_bytes / 4));
+      if (e != cudaSuccess) return e;
       launched(p, "k_convert_weights");
     }
     CUtensorMap tx, tw;
