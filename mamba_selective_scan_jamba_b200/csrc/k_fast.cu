@@ -1662,10 +1662,14 @@ __device__ __forceinline__ void scan_chunk_body(uint32_t tacc, const bf16* xs, c
 #ifndef JMIX_SCAN_YTMA
 #define JMIX_SCAN_YTMA 1    // y of whole chunks leaves through the stage by TMA
 #endif
+#ifndef JMIX_SCAN_YTMA_PACKED
+#define JMIX_SCAN_YTMA_PACKED 1  // ... in packed batches too
+#endif
 // Whether a chunk of nt tokens of an output unit stores its y tile by TMA from
-// the stage (whole chunks of fixed-length sequences), else thread by thread.
+// the stage (whole chunks: the tile stays inside its sequence), else thread by
+// thread.
 __device__ __forceinline__ bool y_by_tma(const ScanArgs& a, bool out, int nt) {
-  return JMIX_SCAN_YTMA && out && !a.cu && nt == kSQ;
+  return JMIX_SCAN_YTMA && out && (JMIX_SCAN_YTMA_PACKED || !a.cu) && nt == kSQ;
 }
 
 template <bool kOut, bool kZoh, bool kLead, class Hook>
@@ -1879,15 +1883,17 @@ __global__ void __launch_bounds__(kLead ? 128 : kScanThreads, kScanCtasPerSm)
           if (out) tma_load_2d(smem_u32(st + kDtnStage + kXStage), &tm_z, fb, (int32_t)c0, row);
           tma_load_2d(smem_u32(st + kDtnStage + 2 * kXStage), &tm_bc, fb, 0, row);
         };
-        // y tile of chunk k (whole chunks of fixed-length sequences): the compute
-        // warps left it in the stage's x tile; one TMA store per chunk
+        // y tile of chunk k (whole chunks): the compute warps left it in the
+        // stage's x tile; one TMA store per chunk (y is [B, L, d], or [1, T, d]
+        // for a packed batch, whose sequence starts at token g0)
         auto store_y = [&](int k) -> bool {
           if (!y_by_tma(a, out, (int)((Lb - (int64_t)(kb + k) * kSQ) < kSQ
                                           ? (Lb - (int64_t)(kb + k) * kSQ) : kSQ)))
             return false;
           const int s = (kg0 + k) % kScanStages;
           tma_store_3d(&tm_y, smem_u32(stage0 + s * kStageBytes + kDtnStage), (int32_t)c0,
-                       (int32_t)((kb + k) * kSQ), (int32_t)b);
+                       (int32_t)((a.cu ? g0 : 0) + (int64_t)(kb + k) * kSQ),
+                       (int32_t)(a.cu ? 0 : b));
           bulk_commit();
           return true;
         };
