@@ -686,6 +686,8 @@ constexpr int kFMaxN1 = (kMaxRank + 2 * kN) / 2;            // 144
 constexpr int kFBMax = 2 * kFMaxN1 * kXK * 2;               // 36 KB of W_x rows
 constexpr int kFSmem = 1024 + kFStages * (kFABytes + kFBMax + kFXStride) + 256;
 static_assert(kFSmem <= 227 * 1024, "fused x_proj stage ring exceeds shared memory");
+static_assert(8 * kXMaxBoxes * 2048 <= kFStages * (kFABytes + kFBMax),
+              "the epilogue's partial-sum boxes exceed the A and B stages");
 static_assert(kFConvWarps * 32 * kFG == kXM * (kXK / 8), "conv threads = kFG-token x 8-channel cells");
 
 // The weight preparation of a prefill: W_x and W_dt to fp16 (unless prepared
@@ -918,7 +920,7 @@ __global__ void __launch_bounds__(256, JMIX_STEP_OCC) k_conv_step(
 
 __global__ void __launch_bounds__(kFThreads, 1)
     k_xproj_conv(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
-                 const XconvArgs a) {
+                 const __grid_constant__ CUtensorMap tm_part, const XconvArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* As = smem;                          // [stages] u tiles (128-byte swizzle)
@@ -1295,30 +1297,34 @@ __global__ void __launch_bounds__(kFThreads, 1)
         }
       } else {
         // partial sums: columns [0, N1) by warps 2-5, [N1, 2 N1) by warps 6-9,
-        // transposed through shared memory (the stages are free once the
-        // accumulator is complete) into 64-byte row segments
-        float* tbuf = reinterpret_cast<float*>(smem) + (warp - 2) * (32 * 17);
-        const int64_t row0 = m0 + lg * 32;
-        float* dst = a.part + ((int64_t)split * a.T) * a.P;
+        // 16 at a time into [32 rows x 16 columns] boxes of shared memory
+        // (64-byte swizzle: 16-byte chunk q of row r at chunk q ^ ((r >> 1) & 3);
+        // the A and B stages are free once the accumulator is complete), which
+        // one tensor store per box writes (rows past T, columns past P are not)
         const int cbeg = lower ? 0 : a.N1;
-        for (int c0 = cbeg; c0 < cbeg + a.N1; c0 += 16) {
+        uint8_t* boxes = smem + (warp - 2) * (kXMaxBoxes * 2048);
+        const int nbox = a.N1 / 16;
+        for (int j = 0; j < nbox; ++j) {
           uint32_t r[16];
-          tmem_ld16(trow + (uint32_t)c0, r);
+          tmem_ld16(trow + (uint32_t)(cbeg + j * 16), r);
           tmem_ld_wait();
+          uint8_t* rowp = boxes + j * 2048 + lane * 64;
 #pragma unroll
-          for (int j = 0; j < 16; ++j) tbuf[lane * 17 + j] = __uint_as_float(r[j]);
-          __syncwarp();
-          if (ok) {
-            const int col = c0 + (lane & 15);
-#pragma unroll 4
-            for (int rr = 0; rr < 16; ++rr) {
-              const int row = 2 * rr + (lane >> 4);
-              const int64_t gg = row0 + row;
-              if (gg < a.T && col < a.P) dst[gg * a.P + col] = tbuf[row * 17 + (lane & 15)];
-            }
-          }
-          __syncwarp();
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4*>(rowp + ((q ^ ((lane >> 1) & 3)) << 4)) =
+                ok ? make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3])
+                   : make_uint4(0u, 0u, 0u, 0u);
         }
+        fence_proxy_async_smem();  // the boxes, before the tensor stores read them
+        __syncwarp();
+        if (lane == 0) {
+          for (int j = 0; j < nbox; ++j)
+            tma_store_3d(&tm_part, smem_u32(boxes + j * 2048), cbeg + j * 16,
+                         (int32_t)(m0 + lg * 32), split);
+          bulk_commit();
+          bulk_wait_all();  // the partial tile written (and the boxes read) before the CTA ends
+        }
+        __syncwarp();
       }
     }
   }
@@ -2929,9 +2935,14 @@ cudaError_t run_fast_fwd(Problem& p) {
                       CU_TENSOR_MAP_SWIZZLE_NONE) ||
         !make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, w.wx, p.P, p.d, kXK, xa.N1, true))
       return cudaErrorInvalidValue;
+    CUtensorMap tp;  // the partial sums [ksplit, T, P] (several splits), boxes of 16 x 32
+    if (xa.ksplit > 1 && !make_part_map(&tp, w.part, (uint64_t)xa.ksplit, (uint64_t)p.T,
+                                        (uint64_t)p.P))
+      return cudaErrorInvalidValue;
+    if (xa.ksplit == 1) tp = tw;  // (not read with one split)
     cudaFuncSetAttribute(k_xproj_conv, cudaFuncAttributeMaxDynamicSharedMemorySize, kFSmem);
     const dim3 grid((unsigned)((p.T + kXM - 1) / kXM), (unsigned)xa.ksplit);
-    e = launch_pdl(k_xproj_conv, grid, kFThreads, (size_t)kFSmem, s, tx, tw, xa);
+    e = launch_pdl(k_xproj_conv, grid, kFThreads, (size_t)kFSmem, s, tx, tw, tp, xa);
     if (e != cudaSuccess) return e;
     launched(p, "k_xproj_conv");
     if (w.ksplit > 1) {
