@@ -1,9 +1,9 @@
 // The bf16-io path of the mixer core on sm_100a.
 //
 // Prefill (a batch of sequences of one length, or a packed batch):
-//   k_conv_silu16<1>  (no conv work: "k_convert_weights") xproj_w and dtproj_w
-//                     from bf16 to fp16 (exact for |w| >= 2^-14; fp16
-//                     subnormals below), unless prepared once beforehand.
+//   k_convert_weights xproj_w and dtproj_w from bf16 to fp16 (exact for |w| >=
+//                     2^-14; fp16 subnormals below), unless prepared once
+//                     beforehand; the conv weights as k_xproj_conv's table.
 //   k_xproj_conv      u = SiLU(conv1d(x) + conv_b) in fp16, computed into the A
 //                     operand of p = u . xproj_w^T on tcgen05 (TMA -> SMEM ->
 //                     MMA -> TMEM); with one split over d_inner the RMSNorms in
@@ -53,7 +53,7 @@ typedef __nv_bfloat16 bf16;
 #define JMIX_CONV_OCC 2
 #endif
 // tokens per thread in k_conv_silu16: 8 for sequences (3 history rows shared by
-// 8 tokens), 1 for decode steps (L = 1)
+// 8 tokens), 1 for shorter ones
 constexpr int kConvG = 8;
 constexpr int kXM = 128;          // x_proj tile: tokens
 constexpr int kXK = 64;           // x_proj tile: channels per k-chunk (one 128-B swizzle atom)
@@ -3151,16 +3151,17 @@ size_t prepared_weights_bytes(int64_t d, int64_t R) {
   return align256((size_t)(R + 2 * kN) * d * 2) + align256((size_t)d * R * 2);
 }
 
-// The weight-conversion threads of the conv kernel alone (no conv work).
+// The fp16 copies of W_x and W_dt, rounded as a call's weight preparation
+// rounds them (k_convert_weights with no conv table and no header to clear).
 cudaError_t run_prepare_weights(int64_t d, int64_t R, const void* xproj_w, const void* dtproj_w,
                                 void* out, cudaStream_t s) {
   const int64_t P = R + 2 * kN;
   const int64_t n_wx8 = P * d / 8, n_wdt8 = d * R / 8;
   __half* wx16 = static_cast<__half*>(out);
   __half* wdt16 = reinterpret_cast<__half*>(static_cast<char*>(out) + align256((size_t)P * d * 2));
-  k_conv_silu16<1><<<(unsigned)((n_wx8 + n_wdt8 + 255) / 256), 256, 0, s>>>(
-      nullptr, nullptr, nullptr, nullptr, nullptr, 0, 0, 1, d, nullptr, 0,
-      (const bf16*)xproj_w, n_wx8, wx16, (const bf16*)dtproj_w, n_wdt8, wdt16);
+  k_convert_weights<<<(unsigned)((n_wx8 + n_wdt8 + 255) / 256), 256, 0, s>>>(
+      (const bf16*)xproj_w, n_wx8, wx16, (const bf16*)dtproj_w, n_wdt8, wdt16, nullptr, nullptr,
+      d, nullptr, 0, nullptr, 0);
   return cudaGetLastError();
 }
 
