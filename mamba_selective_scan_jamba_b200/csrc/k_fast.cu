@@ -657,12 +657,14 @@ __global__ void __launch_bounds__(256) k_norms16_warp(
 //               the chunk's conv weights and biases (bulk copies) and its two
 //               W_x boxes;
 //   warp 1      TMEM owner and MMA issuer (2 x 4 tcgen05.mma per chunk);
-//   warps 2-    conv (JMIX_XCONV_WARPS of them): thread = 8 channels x kFG
-//               tokens (4 with 8 warps).  The kFG + 3 x rows come from
-//               the stage, taps before a sequence's first token from its
-//               history (or zero); u in fp16 goes into the 128-byte-swizzled A
-//               stage, rounded exactly as k_conv_silu16 rounds it.  Then the
-//               epilogue.
+//   warps 2-    conv (JMIX_XCONV_WARPS of them; with JMIX_XCONV_GROUPS > 1 in
+//               groups that take alternate chunks): thread = 8 channels x kFG
+//               tokens (4 with 8 warps in one group), each token's u stored as
+//               soon as it is computed.
+//               The kFG + 3 x rows come from the stage, taps before a
+//               sequence's first token from its history (or zero); u in fp16
+//               goes into the 128-byte-swizzled A stage, rounded exactly as
+//               k_conv_silu16 rounds it.  Then the epilogue.
 // With one split the epilogue applies the RMSNorms itself (thread = token row
 // of TMEM, the sums of squares taken in the order of k_norms16_warp's
 // reductions) and writes dt_n and B, C; with several it writes the fp32
@@ -670,8 +672,13 @@ __global__ void __launch_bounds__(256) k_norms16_warp(
 #ifndef JMIX_XCONV_WARPS
 #define JMIX_XCONV_WARPS 8  // conv warps (8: 4 tokens per thread, 16: 2)
 #endif
+#ifndef JMIX_XCONV_GROUPS
+#define JMIX_XCONV_GROUPS 1  // conv warp groups taking alternate chunks (2 measured slower)
+#endif
 constexpr int kFConvWarps = JMIX_XCONV_WARPS;
-constexpr int kFG = kXM * (kXK / 8) / (kFConvWarps * 32);  // tokens per conv thread
+constexpr int kFGroups = JMIX_XCONV_GROUPS;
+constexpr int kFGroupWarps = kFConvWarps / kFGroups;
+constexpr int kFG = kXM * (kXK / 8) / (kFGroupWarps * 32);  // tokens per conv thread
 constexpr int kFThreads = 64 + 32 * kFConvWarps;
 constexpr int kFStages = 3;
 constexpr int kFXRows = kXM + kConv - 1;                    // 131 x rows per chunk
@@ -688,7 +695,9 @@ constexpr int kFSmem = 1024 + kFStages * (kFABytes + kFBMax + kFXStride) + 256;
 static_assert(kFSmem <= 227 * 1024, "fused x_proj stage ring exceeds shared memory");
 static_assert(8 * kXMaxBoxes * 2048 <= kFStages * (kFABytes + kFBMax),
               "the epilogue's partial-sum boxes exceed the A and B stages");
-static_assert(kFConvWarps * 32 * kFG == kXM * (kXK / 8), "conv threads = kFG-token x 8-channel cells");
+static_assert(kFGroupWarps * kFGroups == kFConvWarps &&
+                  kFGroupWarps * 32 * kFG == kXM * (kXK / 8),
+              "a group's conv threads = kFG-token x 8-channel cells of a chunk");
 
 // The weight preparation of a prefill: W_x and W_dt to fp16 (unless prepared
 // once beforehand), 8 weights per thread, and the conv weights and biases as
@@ -753,8 +762,6 @@ struct XconvArgs {
   const bf16* hist;    // [B, d, 3] conv history of each sequence, or null (zeros)
   const int* cu;       // packed batch: [B + 1] token offsets of the sequences, or null
   int64_t nseq;        // packed batch: sequences B
-  const int* sidx;     // decode step (L == 1): history slot of each row, or null (slot = row)
-  int64_t n_slots;     // decode step: slots of the history pool
   float* part;         // [ksplit, T, P] partial sums (ksplit > 1)
   const bf16* dtn_w;   // [R]
   const bf16* bn_w;    // [N]
@@ -943,7 +950,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kFStages; ++s) {
       mbar_init(smem_u32(&full[s]), 1);
-      mbar_init(smem_u32(&afull[s]), kFConvWarps);
+      mbar_init(smem_u32(&afull[s]), kFGroupWarps);
       mbar_init(smem_u32(&mdone[s]), 1);
     }
     mbar_init(smem_u32(acc_full), 1);
@@ -1004,13 +1011,15 @@ __global__ void __launch_bounds__(kFThreads, 1)
       umma_commit(smem_u32(acc_full));
     }
   } else {
-    // ---- conv: thread = channels cg*8 .. +7 of the chunk, tile rows kFG tg .. + kFG - 1
-    const int ct = threadIdx.x - 64;
+    // ---- conv: group grp takes chunks grp, grp + kFGroups, ...; thread =
+    // channels cg*8 .. +7 of the chunk, tile rows kFG tg .. + kFG - 1
+    const int grp = (warp - 2) / kFGroupWarps;
+    const int ct = threadIdx.x - 64 - grp * kFGroupWarps * 32;
     const int cg = ct & 7, tg = ct >> 3;
     constexpr int kW = kConv - 1;
-    // sequence and position of the thread's 4 tokens (the same for every
+    // sequence and position of the thread's kFG tokens (the same for every
     // chunk); a token at position < 3 takes taps from its sequence's history
-    int64_t tseq[kFG];
+    int tseq[kFG];  // (a sequence index)
     int tpos[kFG];
     bool tedge[kFG], edge = false;
 #pragma unroll
@@ -1027,8 +1036,8 @@ __global__ void __launch_bounds__(kFThreads, 1)
         tseq[ti] = lo;
         tpos[ti] = (int)(g - __ldg(a.cu + lo));
       } else {
-        tseq[ti] = g / a.L;
-        tpos[ti] = (int)(g - tseq[ti] * a.L);
+        tseq[ti] = (int)(g / a.L);
+        tpos[ti] = (int)(g - (int64_t)tseq[ti] * a.L);
       }
       tedge[ti] = g < a.T && tpos[ti] >= 0 && tpos[ti] < kW;
       edge |= tedge[ti];
@@ -1040,22 +1049,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
     // Other layouts of sequence starts recompute their edge tokens (slow).
     const bool sub = tedge[0] && tseq[kFG - 1] == tseq[0];
     const bool slow = edge && !sub;
-    // decode step (L == 1): every tap but the last is history; a row's history
-    // sits in its pool slot, clamped into the pool (a bad slot is reported and
-    // skipped by the decode kernel), -1 for rows past T
-    const bool step = a.L == 1 && !a.cu;
-    int64_t hrow[kFG];
-#pragma unroll
-    for (int ti = 0; ti < kFG; ++ti) {
-      const int64_t g = m0 + kFG * tg + ti;
-      int64_t sl = g;
-      if (step && a.sidx && g < a.T) {
-        sl = __ldg(a.sidx + g);
-        sl = sl < 0 ? 0 : (sl >= a.n_slots ? a.n_slots - 1 : sl);
-      }
-      hrow[ti] = (g < a.T && a.hist) ? sl : -1;
-    }
-    for (int kc = k_begin, i = 0; kc < k_end; ++kc, ++i) {
+    for (int kc = k_begin + grp, i = grp; kc < k_end; kc += kFGroups, i += kFGroups) {
       const int s = i % kFStages;
       const uint32_t ph = (uint32_t)(i / kFStages) & 1u;
       const int64_t c0 = (int64_t)kc * kXK + cg * 8;
@@ -1086,122 +1080,88 @@ __global__ void __launch_bounds__(kFThreads, 1)
       uint4 xr[kFG + kW];
 #pragma unroll
       for (int j = 0; j < kFG + kW; ++j) xr[j] = *reinterpret_cast<const uint4*>(xs + j * (kXK * 2));
-      uint32_t outw[kFG][4];  // [token][channel pair] fp16x2
-      if (!step) {
-        if (sub) {
-          // raw row j < 3 - tpos[0] holds position tpos[0] - 3 + j < 0 of the
-          // sequence: history slot tpos[0] + j (channel e's slots sit at 3 e ..)
-          uint4 hq[3] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u),
-                         make_uint4(0u, 0u, 0u, 0u)};
-          if (cin && a.hist) {
-            const uint4* hp = reinterpret_cast<const uint4*>(a.hist + (tseq[0] * a.d + c0) * kW);
-#pragma unroll
-            for (int q = 0; q < 3; ++q) hq[q] = __ldg(hp + q);
-          }
-          const uint32_t* hw = reinterpret_cast<const uint32_t*>(hq);
-          uint4 hrows[kW];  // [slot]: the 8 channels' values at that history slot
-#pragma unroll
-          for (int sl = 0; sl < kW; ++sl) {
-            uint32_t wv[4];
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-              const int i0 = 3 * (2 * w) + sl, i1 = 3 * (2 * w + 1) + sl;  // 16-bit elements
-              const uint32_t lo = (hw[i0 >> 1] >> (16 * (i0 & 1))) & 0xffffu;
-              const uint32_t hi = (hw[i1 >> 1] >> (16 * (i1 & 1))) & 0xffffu;
-              wv[w] = lo | (hi << 16);
-            }
-            hrows[sl] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-          }
-#pragma unroll
-          for (int j = 0; j < kW; ++j) {
-            if (j < kW - tpos[0]) {
-              const int sl = tpos[0] + j;
-              xr[j] = sl == 0 ? hrows[0] : (sl == 1 ? hrows[1] : hrows[2]);
-            }
-          }
-        }
-        // every token from the kFG + 3 x rows (one basic block: the chains interleave)
-#pragma unroll
-        for (int ti = 0; ti < kFG; ++ti) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            float2 acc = b2[q];
-#pragma unroll
-            for (int k = 0; k < kConv; ++k) acc = __ffma2_rn(w2[q][k], bf16_pair(xr[ti + k], q), acc);
-            outw[ti][q] = silu_u_half2(acc);
-          }
-        }
-        if (slow) {
-          // rare: tokens at positions 0-2 of their sequence in a thread that
-          // also holds tokens of the sequence before, again with the taps before
-          // the sequence's first token from its history (or zero)
-#pragma unroll
-          for (int ti = 0; ti < kFG; ++ti) {
-            if (!tedge[ti]) continue;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              float2 acc = b2[q];
-#pragma unroll
-              for (int k = 0; k < kConv; ++k) {
-                float2 xv = bf16_pair(xr[ti + k], q);
-                if (k < kW && tpos[ti] + k < kW) {
-                  xv = make_float2(0.f, 0.f);
-                  if (a.hist) {
-                    const bf16* hp =
-                        a.hist + (tseq[ti] * a.d + c0 + 2 * q) * kW + tpos[ti] + k;
-                    xv = make_float2(bf(hp[0]), bf(hp[kW]));
-                  }
-                }
-                acc = __ffma2_rn(w2[q][k], xv, acc);
-              }
-              outw[ti][q] = silu_u_half2(acc);
-            }
-          }
-        }
-      } else {
-        // decode step: the 8 channels' 3 history taps per row (48 contiguous bytes)
-        uint4 hq[kFG][3];
-#pragma unroll
-        for (int ti = 0; ti < kFG; ++ti) {
-#pragma unroll
-          for (int q = 0; q < 3; ++q) hq[ti][q] = make_uint4(0u, 0u, 0u, 0u);
-          if (cin && hrow[ti] >= 0) {
-            const uint4* hp = reinterpret_cast<const uint4*>(a.hist + (hrow[ti] * a.d + c0) * kW);
-#pragma unroll
-            for (int q = 0; q < 3; ++q) hq[ti][q] = __ldg(hp + q);
-          }
-        }
-#pragma unroll
-        for (int ti = 0; ti < kFG; ++ti) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            float2 acc = b2[q];
-#pragma unroll
-            for (int k = 0; k < kW; ++k) {
-              const int e0 = (2 * q) * kW + k, e1 = (2 * q + 1) * kW + k;
-              acc = __ffma2_rn(w2[q][k],
-                               make_float2(bf16_lane(hq[ti][e0 >> 3], e0 & 7),
-                                           bf16_lane(hq[ti][e1 >> 3], e1 & 7)),
-                               acc);
-            }
-            acc = __ffma2_rn(w2[q][kW], bf16_pair(xr[ti + kW], q), acc);
-            outw[ti][q] = silu_u_half2(acc);
-          }
-        }
-      }
-      if (!cin) {
-#pragma unroll
-        for (int ti = 0; ti < kFG; ++ti)
-#pragma unroll
-          for (int q = 0; q < 4; ++q) outw[ti][q] = 0u;
-      }
-      // into the A stage: row r, 16-byte chunk cg at cg ^ (r % 8) (128-byte swizzle)
+      // token ti's u into the A stage: row r, 16-byte chunk cg at cg ^ (r % 8)
+      // (128-byte swizzle); zeros for channels past d
       uint8_t* at = As + s * kFABytes;
-#pragma unroll
-      for (int ti = 0; ti < kFG; ++ti) {
+      auto store_u = [&](int ti, const uint32_t (&o)[4]) {
         const int r = kFG * tg + ti;
         *reinterpret_cast<uint4*>(at + r * (kXK * 2) + ((cg ^ (r & 7)) << 4)) =
-            make_uint4(outw[ti][0], outw[ti][1], outw[ti][2], outw[ti][3]);
+            cin ? make_uint4(o[0], o[1], o[2], o[3]) : make_uint4(0u, 0u, 0u, 0u);
+      };
+      if (sub) {
+        // raw row j < 3 - tpos[0] holds position tpos[0] - 3 + j < 0 of the
+        // sequence: history slot tpos[0] + j (channel e's slots sit at 3 e ..)
+        uint4 hq[3] = {make_uint4(0u, 0u, 0u, 0u), make_uint4(0u, 0u, 0u, 0u),
+                       make_uint4(0u, 0u, 0u, 0u)};
+        if (cin && a.hist) {
+          const uint4* hp =
+              reinterpret_cast<const uint4*>(a.hist + ((int64_t)tseq[0] * a.d + c0) * kW);
+#pragma unroll
+          for (int q = 0; q < 3; ++q) hq[q] = __ldg(hp + q);
+        }
+        const uint32_t* hw = reinterpret_cast<const uint32_t*>(hq);
+        uint4 hrows[kW];  // [slot]: the 8 channels' values at that history slot
+#pragma unroll
+        for (int sl = 0; sl < kW; ++sl) {
+          uint32_t wv[4];
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const int i0 = 3 * (2 * w) + sl, i1 = 3 * (2 * w + 1) + sl;  // 16-bit elements
+            const uint32_t lo = (hw[i0 >> 1] >> (16 * (i0 & 1))) & 0xffffu;
+            const uint32_t hi = (hw[i1 >> 1] >> (16 * (i1 & 1))) & 0xffffu;
+            wv[w] = lo | (hi << 16);
+          }
+          hrows[sl] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        }
+#pragma unroll
+        for (int j = 0; j < kW; ++j) {
+          if (j < kW - tpos[0]) {
+            const int sl = tpos[0] + j;
+            xr[j] = sl == 0 ? hrows[0] : (sl == 1 ? hrows[1] : hrows[2]);
+          }
+        }
+      }
+      // every token from the kFG + 3 x rows (one basic block: the chains interleave)
+#pragma unroll
+      for (int ti = 0; ti < kFG; ++ti) {
+        uint32_t o[4];  // channel pairs as fp16x2
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float2 acc = b2[q];
+#pragma unroll
+          for (int k = 0; k < kConv; ++k) acc = __ffma2_rn(w2[q][k], bf16_pair(xr[ti + k], q), acc);
+          o[q] = silu_u_half2(acc);
+        }
+        store_u(ti, o);
+      }
+      if (slow) {
+        // rare: tokens at positions 0-2 of their sequence in a thread that
+        // also holds tokens of the sequence before, again with the taps before
+        // the sequence's first token from its history (or zero)
+#pragma unroll
+        for (int ti = 0; ti < kFG; ++ti) {
+          if (!tedge[ti]) continue;
+          uint32_t o[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float2 acc = b2[q];
+#pragma unroll
+            for (int k = 0; k < kConv; ++k) {
+              float2 xv = bf16_pair(xr[ti + k], q);
+              if (k < kW && tpos[ti] + k < kW) {
+                xv = make_float2(0.f, 0.f);
+                if (a.hist) {
+                  const bf16* hp =
+                      a.hist + ((int64_t)tseq[ti] * a.d + c0 + 2 * q) * kW + tpos[ti] + k;
+                  xv = make_float2(bf(hp[0]), bf(hp[kW]));
+                }
+              }
+              acc = __ffma2_rn(w2[q][k], xv, acc);
+            }
+            o[q] = silu_u_half2(acc);
+          }
+          store_u(ti, o);  // (over the first pass's value)
+        }
       }
       fence_proxy_async_smem();  // u in the stage, before the tensor cores read it
       __syncwarp();
@@ -2766,15 +2726,12 @@ int xproj_ksplit(int64_t T, int64_t d) {
 #define JMIX_XCONV 1  // prefill of sequences of one length: conv inside x_proj (k_xproj_conv)
 #endif
 // Whether steps 1-3 run as k_xproj_conv (plus k_norms16 when split): prefill
-// (sequences of one length or a packed batch), dt_rank a multiple of 16.
-// Depends on the problem's shape only.
-#ifndef JMIX_XCONV_DECODE
-// decode steps too (measured slower at 256 rows: the separate weight
-// conversion launch costs more than the fused conv saves)
-#define JMIX_XCONV_DECODE 0
-#endif
+// (sequences of one length or a packed batch), dt_rank a multiple of 16; a
+// decode step runs k_conv_step, k_xproj and k_norms16 (the conv spread over
+// every SM: inside x_proj it measured slower at 256 rows).  Depends on the
+// problem's shape only.
 bool use_xconv(const Problem& pr) {
-  return JMIX_XCONV && (JMIX_XCONV_DECODE || !pr.decode) && pr.R % 16 == 0 && pr.T > 0;
+  return JMIX_XCONV && !pr.decode && pr.R % 16 == 0 && pr.T > 0;
 }
 
 // k_xproj_conv's split over d_inner: one split once the token tiles fill the
@@ -2921,8 +2878,6 @@ cudaError_t run_fast_fwd(Problem& p) {
     xa.hist = (const bf16*)p.init_conv;
     xa.cu = p.cu;
     xa.nseq = p.B;
-    xa.sidx = p.sidx;
-    xa.n_slots = p.sidx ? p.n_slots : p.B;
     xa.part = w.part;
     xa.dtn_w = (const bf16*)p.dtn_w;
     xa.bn_w = (const bf16*)p.bn_w;
