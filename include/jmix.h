@@ -35,7 +35,11 @@
  * All pointers given to the compute entry points are DEVICE pointers (the
  * _host variant below is the one exception), owned by the caller.  libjmix
  * never allocates, frees or synchronises, except jm_poll_error (which
- * synchronises the given stream).  Calls are asynchronous on `stream`.
+ * synchronises the given stream).  Calls are asynchronous on `stream`.  A
+ * call's kernels follow one another (and the kernel before the call) with
+ * programmatic dependent launch: a kernel may be scheduled while the one before
+ * it finishes, and waits for it to complete before it reads what that kernel
+ * (or any earlier work on the stream) wrote; to the caller, stream order holds.
  *
  * Errors: host-side validation runs before any launch and returns
  * JM_ERR_INVALID_ARG (NULL required pointer, negative size, pointer not
