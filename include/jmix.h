@@ -38,8 +38,8 @@
  * synchronises the given stream).  Calls are asynchronous on `stream`.  A
  * call's kernels follow one another (and the kernel before the call) with
  * programmatic dependent launch: a kernel may be scheduled while the one before
- * it finishes, and waits for it to complete before it reads what that kernel
- * (or any earlier work on the stream) wrote; to the caller, stream order holds.
+ * it finishes, but none reads what earlier work on the stream writes before
+ * that work has completed; to the caller, stream order holds.
  *
  * Errors: host-side validation runs before any launch and returns
  * JM_ERR_INVALID_ARG (NULL required pointer, negative size, pointer not
